@@ -1,0 +1,285 @@
+"""CPU oracle for the NVFP4 W4A4 linear layer and NVFP4 KV-cache store.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline / reference leg may import this package.  The product
+path (``bit_video_dit_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``nvfp4_oracle.c`` (plain C, binary32 steps with
+``-ffp-contract=off``, binary64 GEMM accumulation); this module only builds
+that file with gcc and marshals numpy arrays through ctypes.  Format source:
+"LongLive-2.0：用 NVFP4 并行底座做长视频生成" (yingwang.github.io reading note),
+section 二 方法 / "NVFP4 量化格式" (E2M1 codes, per-16 E4M3 block scale, FP32
+tensor scale, the Dequant equation) and "推理底座" (per-chunk KV quantization).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+MODE_COMPUTE = 0
+MODE_GIVEN = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile nvfp4_oracle.c into liboracle.so (gcc, OpenMP, no FP contraction)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+           "-fPIC", "-shared", "-fvisibility=hidden", _SRC, "-o", tmp, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class _Epilogue(ctypes.Structure):
+    _fields_ = [("bias", ctypes.c_void_p), ("mod_scale", ctypes.c_void_p),
+                ("mod_shift", ctypes.c_void_p), ("gate", ctypes.c_void_p),
+                ("residual", ctypes.c_void_p), ("ld_res", ctypes.c_int64),
+                ("act", ctypes.c_int)]
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            i64, f32, vp, u16 = ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_uint16
+            L.orc_set_threads.argtypes = [ctypes.c_int]
+            L.orc_get_threads.restype = ctypes.c_int
+            L.orc_bf16_to_f32.argtypes = [u16]
+            L.orc_bf16_to_f32.restype = f32
+            L.orc_f64_to_bf16.argtypes = [ctypes.c_double]
+            L.orc_f64_to_bf16.restype = u16
+            L.orc_f32_to_bf16.argtypes = [f32]
+            L.orc_f32_to_bf16.restype = u16
+            L.orc_e2m1_value.argtypes = [ctypes.c_uint]
+            L.orc_e2m1_value.restype = ctypes.c_double
+            L.orc_e4m3_value.argtypes = [ctypes.c_uint]
+            L.orc_e4m3_value.restype = ctypes.c_double
+            L.orc_e2m1_encode.argtypes = [f32]
+            L.orc_e2m1_encode.restype = ctypes.c_uint
+            L.orc_e4m3_encode.argtypes = [f32]
+            L.orc_e4m3_encode.restype = ctypes.c_uint
+            for name in ("orc_quantize_f32", "orc_quantize_bf16"):
+                fn = getattr(L, name)
+                fn.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp, vp]
+                fn.restype = ctypes.c_int
+            L.orc_swizzled_bytes.argtypes = [i64, i64]
+            L.orc_swizzled_bytes.restype = i64
+            L.orc_swizzle_offset.argtypes = [i64, i64, i64]
+            L.orc_swizzle_offset.restype = i64
+            L.orc_swizzle_scales.argtypes = [vp, i64, i64, vp]
+            L.orc_unswizzle_scales.argtypes = [vp, i64, i64, vp]
+            L.orc_dequant_f32.argtypes = [vp, vp, f32, i64, i64, vp]
+            L.orc_dequant_bf16.argtypes = [vp, vp, f32, i64, i64, vp]
+            L.orc_gemm.argtypes = [vp, vp, f32, vp, vp, f32, i64, i64, i64,
+                                   ctypes.POINTER(_Epilogue), vp, i64, vp, vp]
+            L.orc_gemm.restype = ctypes.c_int
+            L.orc_gemm_exact_bf16.argtypes = [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp]
+            L.orc_gemm_exact_bf16.restype = ctypes.c_int
+            L.orc_kv_slot_bytes.argtypes = [i64, i64, i64]
+            L.orc_kv_slot_bytes.restype = i64
+            L.orc_kv_append.argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
+            L.orc_kv_append.restype = ctypes.c_int
+            L.orc_kv_dequant.argtypes = [vp, vp, f32, i64, i64, i64, vp]
+            _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def set_threads(n: int) -> None:
+    lib().orc_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().orc_get_threads())
+
+
+# ---- scalar format helpers ---------------------------------------------------
+
+def e2m1_value(code: int) -> float:
+    return float(lib().orc_e2m1_value(int(code)))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().orc_e4m3_value(int(code)))
+
+
+def e2m1_encode(y: float) -> int:
+    return int(lib().orc_e2m1_encode(float(np.float32(y))))
+
+
+def e4m3_encode(r: float) -> int:
+    return int(lib().orc_e4m3_encode(float(np.float32(r))))
+
+
+def f64_to_bf16(x: float) -> int:
+    return int(lib().orc_f64_to_bf16(float(x)))
+
+
+def bf16_to_f32(h: int) -> float:
+    return float(lib().orc_bf16_to_f32(int(h)))
+
+
+# ---- array API ---------------------------------------------------------------
+
+def quantize(x: np.ndarray, alpha: float | None = None):
+    """Quantize a 2-D array (uint16 bf16 bits or float32).
+
+    Returns (codes uint8 [R, C/2], scales uint8 logical [R, C/16], alpha float32).
+    alpha=None computes the tensor scale (R1); otherwise it is used as given.
+    """
+    assert x.ndim == 2
+    x = np.ascontiguousarray(x)
+    R, C = x.shape
+    codes = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    a = np.zeros(1, np.float32)
+    mode = MODE_COMPUTE
+    if alpha is not None:
+        a[0] = np.float32(alpha)
+        mode = MODE_GIVEN
+    if x.dtype == np.uint16:
+        fn = lib().orc_quantize_bf16
+    elif x.dtype == np.float32:
+        fn = lib().orc_quantize_f32
+    else:
+        raise TypeError("oracle.quantize takes bf16 bits (uint16) or float32")
+    rc = fn(_p(x), R, C, C, mode, _p(a), _p(codes), _p(scales))
+    if rc != 0:
+        raise ValueError(f"orc_quantize failed ({rc})")
+    return codes, scales, np.float32(a[0])
+
+
+def swizzled_bytes(rows: int, sc: int) -> int:
+    return int(lib().orc_swizzled_bytes(rows, sc))
+
+
+def swizzle_offset(r: int, c: int, sc: int) -> int:
+    return int(lib().orc_swizzle_offset(r, c, sc))
+
+
+def swizzle(scales: np.ndarray) -> np.ndarray:
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    R, S = scales.shape
+    out = np.zeros(swizzled_bytes(R, S), np.uint8)
+    lib().orc_swizzle_scales(_p(scales), R, S, _p(out))
+    return out
+
+
+def unswizzle(swz: np.ndarray, rows: int, sc: int) -> np.ndarray:
+    swz = np.ascontiguousarray(swz, dtype=np.uint8).reshape(-1)
+    assert swz.size >= swizzled_bytes(rows, sc)
+    out = np.zeros((rows, sc), np.uint8)
+    lib().orc_unswizzle_scales(_p(swz), rows, sc, _p(out))
+    return out
+
+
+def dequant_f32(codes, scales, alpha) -> np.ndarray:
+    R = codes.shape[0]
+    C = codes.shape[1] * 2
+    out = np.zeros((R, C), np.float32)
+    lib().orc_dequant_f32(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)),
+                          float(alpha), R, C, _p(out))
+    return out
+
+
+def dequant_bf16(codes, scales, alpha) -> np.ndarray:
+    R = codes.shape[0]
+    C = codes.shape[1] * 2
+    out = np.zeros((R, C), np.uint16)
+    lib().orc_dequant_bf16(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)),
+                           float(alpha), R, C, _p(out))
+    return out
+
+
+def gemm(a, b, *, bias=None, mod_scale=None, mod_shift=None, gate=None, residual=None,
+         act: int = 0, rows=None, want_bf16: bool = True):
+    """fp64 reference GEMM.  a, b = (codes, logical scales, alpha) triples with
+    A [M x K] and B [N x K].  Epilogue vectors are bf16 bits (uint16).
+    Returns (y fp64 [R x N], out bf16 bits [R x N] or None)."""
+    ac, asc, aa = a
+    bc, bsc, ba = b
+    M, K = ac.shape[0], ac.shape[1] * 2
+    N = bc.shape[0]
+    assert bc.shape[1] * 2 == K
+    keep = []
+
+    def cp(v):
+        if v is None:
+            return None
+        v = np.ascontiguousarray(v)
+        keep.append(v)
+        return v.ctypes.data
+
+    ep = _Epilogue(cp(bias), cp(mod_scale), cp(mod_shift), cp(gate), cp(residual),
+                   N if residual is None else residual.shape[1], int(act))
+    rl = None
+    R = M
+    if rows is not None:
+        rl = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        R = rl.size
+    y = np.zeros((R, N), np.float64)
+    out = np.zeros((R, N), np.uint16) if want_bf16 else None
+    rc = lib().orc_gemm(_p(np.ascontiguousarray(ac)), _p(np.ascontiguousarray(asc)), float(aa),
+                        _p(np.ascontiguousarray(bc)), _p(np.ascontiguousarray(bsc)), float(ba),
+                        M, N, K, ctypes.byref(ep), _p(rl), R, _p(y), _p(out))
+    if rc != 0:
+        raise ValueError(f"orc_gemm failed ({rc})")
+    return y, out
+
+
+def gemm_exact_bf16(a, b) -> np.ndarray:
+    ac, asc, aa = a
+    bc, bsc, ba = b
+    M, K = ac.shape[0], ac.shape[1] * 2
+    N = bc.shape[0]
+    out = np.zeros((M, N), np.uint16)
+    rc = lib().orc_gemm_exact_bf16(_p(np.ascontiguousarray(ac)), _p(np.ascontiguousarray(asc)), float(aa),
+                                   _p(np.ascontiguousarray(bc)), _p(np.ascontiguousarray(bsc)), float(ba),
+                                   M, N, K, _p(out))
+    if rc != 0:
+        raise ValueError(f"orc_gemm_exact_bf16 failed ({rc})")
+    return out
+
+
+def kv_slot_bytes(T: int, H: int, d: int) -> int:
+    return int(lib().orc_kv_slot_bytes(T, H, d))
+
+
+def kv_append(x: np.ndarray):
+    """x: bf16 bits [T, H, d].  Returns (codes [T*H, d/2], scales [T*H, d/16], alpha)."""
+    T, H, d = x.shape
+    x = np.ascontiguousarray(x)
+    codes = np.zeros((T * H, d // 2), np.uint8)
+    scales = np.zeros((T * H, d // 16), np.uint8)
+    a = np.zeros(1, np.float32)
+    rc = lib().orc_kv_append(_p(x), T, H, d, d, _p(codes), _p(scales), _p(a))
+    if rc != 0:
+        raise ValueError(f"orc_kv_append failed ({rc})")
+    return codes, scales, np.float32(a[0])
+
+
+def kv_dequant(codes, scales, alpha, T: int, H: int, d: int) -> np.ndarray:
+    out = np.zeros((T, H, d), np.uint16)
+    lib().orc_kv_dequant(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)), float(alpha),
+                         T, H, d, _p(out))
+    return out
