@@ -1,0 +1,406 @@
+"""Throughput of the NVFP4 hot path on B200.
+
+One step = one pass of the whole path on seeded synthetic DiT-shaped inputs:
+  1. nvfp4_quantize  of the activation A [4096 x 3072] bf16 (tensor amax,
+     block scales, E2M1 codes, swizzled scale tiles)
+  2. nvfp4_gemm      QKV projection 4096 x 9216 x 3072, W pre-quantized once,
+     bias epilogue, bf16 out
+  3. nvfp4_kv_append of one frame-chunk's K and V [2640 x 24 x 128] into ring
+     slot step % 21
+  4. nvfp4_kv_dequant of all 21 slots (ring order) back to bf16
+`value` is the W4A4 linear-layer throughput (2*M*N*K of step 2 per second of
+steps 1+2, device-timed with CUDA events); the KV rows are reported under
+"kv".  The 681 MB bf16 output of step 4 overwrites L2 (126 MB) every step, so
+each step's GEMM and quantize read their inputs from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the same per-GPU workload on its own GPU (weak
+scaling; the path has no exchange step); rank 0 prints one JSON line with the
+max-over-ranks time.  --impl reference times the CPU oracle instead (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from bit_video_dit_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "W4A4 GEMM TFLOPS (% B200 FP4 peak); quantize/KV-append GB/s (% HBM peak)"
+WORKLOAD = "dit_qkv_4096x9216x3072_bias+kv_append_dequant_21x2640x24x128"
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput (9 / 2.25 PFLOP/s)
+NOMINAL_FP4_TFLOPS = 9000.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_video_dit_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "gemm_qkv_traffic.json")
+    try:
+        with open(path) as f:
+            r = json.load(f)
+        if r.get("kernel_hash") == kernel_hash():
+            return r
+    except Exception:
+        pass
+    return None
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------- ours
+def run_ours(args, rank: int, world: int) -> dict | None:
+    from bit_video_dit_b200 import build as nvbuild
+    from bit_video_dit_b200 import nvfp4 as nv
+
+    nvbuild.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
+    S, T, H, D = syn.KV_SLOTS, syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+
+    a_host = syn.activations_bf16(M, K, seed=2 + 1000 * rank)
+    w_host = syn.normal_bf16((N, K), seed=3, std=0.02)
+    bias_host = syn.normal_bf16((N,), seed=4, std=0.02)
+    a = dev_bf16(a_host)
+    w = dev_bf16(w_host)
+    bias = dev_bf16(bias_host)
+    qw = nv.quantize(w)  # weights quantized once
+    del w
+    qa = nv.empty_nvfp4(M, K, dev)
+    ws_q = nv.workspace(nv.OP_QUANTIZE, M, 0, K, dev)
+    ws_g = nv.workspace(nv.OP_GEMM, M, N, K, dev)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    cache = nv.KVCache(S, T, H, D, dev)
+    n_chunks = 4  # distinct K/V chunks cycled through the ring
+    chunks = [tuple(dev_bf16(x) for x in syn.kv_chunk_bf16(T, H, D, seed=50 + i + 1000 * rank))
+              for i in range(n_chunks)]
+    for s in range(S):
+        cache.append(s, *chunks[s % n_chunks])
+    ring = torch.arange(S, dtype=torch.int32, device=dev)
+    k_out = torch.empty((S, T, H, D), dtype=torch.bfloat16, device=dev)
+    v_out = torch.empty_like(k_out)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        if ev:
+            ev[0].record(stream)
+        nv.quantize(a, out=qa, ws=ws_q)
+        if ev:
+            ev[1].record(stream)
+        nv.gemm(qa, qw, out=c, bias=bias, ws=ws_g)
+        if ev:
+            ev[2].record(stream)
+        slot = i % S
+        cache.append(slot, *chunks[i % n_chunks])
+        if ev:
+            ev[3].record(stream)
+        cache.dequant(ring, k_out, v_out)
+        if ev:
+            ev[4].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    code, _ = nv.read_device_error(ws_g)
+    if code != nv.OK:
+        raise RuntimeError(f"device error {code} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+
+    total_ms = t_start.elapsed_time(t_end)
+    comp = np.zeros(4)
+    for e in evs:
+        comp += [e[j].elapsed_time(e[j + 1]) for j in range(4)]
+    comp /= args.steps  # ms per step per component: quantize, gemm, append, dequant
+
+    # --- e2e through the public API with host buffers (linear layer) -------
+    a_pin = torch.from_numpy(a_host.view(np.int16)).pin_memory()
+    c_pin = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    a_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        a_dev.view(torch.int16).copy_(a_pin, non_blocking=True)
+        nv.quantize(a_dev, out=qa, ws=ws_q)
+        nv.gemm(qa, qw, out=c, bias=bias, ws=ws_g)
+        c_pin.copy_(c.view(torch.int16), non_blocking=True)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        a_dev.view(torch.int16).copy_(a_pin, non_blocking=True)
+        nv.quantize(a_dev, out=qa, ws=ws_q)
+        nv.gemm(qa, qw, out=c, bias=bias, ws=ws_g)
+        c_pin.copy_(c.view(torch.int16), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    times = torch.tensor([total_ms, *comp.tolist(), e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    total_ms, q_ms, g_ms, ap_ms, dq_ms, e2e_ms = times.tolist()
+    if rank != 0:
+        return None
+
+    pk = peaks()
+    flops = 2.0 * M * N * K
+    lin_ms = q_ms + g_ms
+    value = world * flops / (lin_ms * 1e-3) / 1e12
+    gemm_tflops = flops / (g_ms * 1e-3) / 1e12
+    fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
+    quant_bytes = M * K * 2.5625
+    kv_elems = T * H * D
+    append_bytes = 2 * kv_elems * 2.5625
+    dequant_bytes = 2 * S * kv_elems * (0.5625 + 2.0)
+    tr = recorded_traffic()
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate); bf16 in/out",
+        "data": "synthetic (seeded N(0,1) activations with 0.1% x20 outlier channels, N(0,0.02) weights)",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "kv_slots": S, "kv_tokens": T, "kv_heads": H,
+                   "kv_head_dim": D, "parallelism": f"dp{world} (independent replicas, no collective)",
+                   "l2": "inputs larger than L2: each step's 681 MB KV dequant output overwrites the 126 MB L2"},
+        "roofline": {"kernel": "nvfp4 gemm (tcgen05 mxf4nvf4)", "bound": "tensor",
+                     "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / fp4_peak, 4),
+                     "peak_source": f"{pk['source']} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16)",
+                     "frac_of_nominal_9pf": round(gemm_tflops / NOMINAL_FP4_TFLOPS, 4),
+                     "traffic": None if tr is None else tr["dram_bytes_per_launch"],
+                     "algorithmic_bytes": M * K // 2 + N * K // 2 + (M + N) * K // 16 + M * N * 2},
+        "components_ms": {"quantize": round(q_ms, 4), "gemm": round(g_ms, 4), "kv_append": round(ap_ms, 4),
+                          "kv_dequant": round(dq_ms, 4)},
+        "quantize": {"GB/s": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                     "bytes_per_call": quant_bytes},
+        "kv": {"append_GB/s": round(append_bytes / (ap_ms * 1e-3) / 1e9, 1),
+               "append_frac_hbm": round(append_bytes / (ap_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+               "dequant_GB/s": round(dequant_bytes / (dq_ms * 1e-3) / 1e9, 1),
+               "dequant_frac_hbm": round(dequant_bytes / (dq_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+               "hbm_peak_GB/s": pk["hbm_gbs"], "cache_bytes": cache.nbytes()},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                "what": "pinned host A -> device, quantize, gemm+bias, C -> pinned host"},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk,
+    }
+    return out
+
+
+# --------------------------------------------------------------------------- oracle
+def oracle_linear_rows(rows: int, w_codes, a_host, bias_host, seed_rows: int):
+    """Time the CPU oracle on `rows` rows of the QKV layer: quantize those rows
+    of A (with the full tensor scale), then their GEMM rows with bias."""
+    import oracle
+
+    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
+    sub = np.ascontiguousarray(a_host[:rows])
+    t0 = time.perf_counter()
+    codes, scales, a32 = oracle.quantize(sub)
+    oracle.gemm((codes, scales, a32), w_codes, bias=bias_host, want_bf16=True)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(steps: int = 1, rows: int = 8) -> dict:
+    import oracle
+
+    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
+    a_host = syn.activations_bf16(M, K, seed=2)
+    w_host = syn.normal_bf16((N, K), seed=3, std=0.02)
+    bias_host = syn.normal_bf16((N,), seed=4, std=0.02)
+    wq = oracle.quantize(w_host)
+    ts = [oracle_linear_rows(rows, wq, a_host, bias_host, i) for i in range(steps)]
+    t = min(ts)
+    return {"value": round(2.0 * rows * N * K / t / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
+            "kind": "oracle", "host_cores": os.cpu_count(),
+            "sample": f"{rows} of {M} token rows of the QKV layer per step (quantize rows + fp64 GEMM rows + bias)",
+            "seconds_per_step": round(t, 3)}
+
+
+def run_reference(args) -> dict:
+    import oracle
+
+    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
+    rows = 8
+    a_host = syn.activations_bf16(M, K, seed=2)
+    w_host = syn.normal_bf16((N, K), seed=3, std=0.02)
+    bias_host = syn.normal_bf16((N,), seed=4, std=0.02)
+    wq = oracle.quantize(w_host)
+    for i in range(args.warmup):
+        oracle_linear_rows(rows, wq, a_host, bias_host, i)
+    t = 0.0
+    for i in range(args.steps):
+        t += oracle_linear_rows(rows, wq, a_host, bias_host, i)
+    value = args.steps * 2.0 * rows * N * K / t / 1e12
+    cb = {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(), "kind": "oracle",
+          "sample": f"{rows} of {M} token rows of the QKV layer per step (quantize rows + fp64 GEMM rows + bias)"}
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 GEMM over NVFP4 operands; f32 quantize",
+            "data": "synthetic (seeded, same generators as the GPU arm)", "impl": "reference",
+            "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "parallelism": "cpu oracle, rank 0"},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        out = run_ours(args, rank, world)
+        if rank == 0 and out is not None:
+            if not args.no_cpu_baseline and world == 1:
+                out["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

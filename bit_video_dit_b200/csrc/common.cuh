@@ -1,0 +1,329 @@
+// common.cuh -- device helpers shared by the NVFP4 kernels: the element and
+// block-scale encoders, the device error record, and thin inline-PTX wrappers
+// for mbarrier, TMA and tcgen05 (sm_100a only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nvfp4.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libnvfp4 is written for sm_100a (B200) only"
+#endif
+
+namespace nvfp4 {
+
+// ---------------------------------------------------------------------------
+// Device error record: the first 16 bytes of every call's workspace.
+//   word 0: status code (0 = none), word 1: call-specific info.
+// The first error wins (compare-and-swap on word 0).
+// ---------------------------------------------------------------------------
+struct DevError {
+    uint32_t code;
+    uint32_t info;
+    uint32_t pad[2];
+};
+
+__device__ __forceinline__ void record_error(DevError* e, uint32_t code, uint32_t info) {
+    if (e == nullptr) return;
+    if (atomicCAS(&e->code, 0u, code) == 0u) atomicExch(&e->info, info);
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 encoders.  The quantize rule (readings of the reading note's
+// three-level scaling; every step one binary32 op, nearest-even):
+//   d6 = 6 * a32;  r = amax_b / d6;  s = E4M3_rne_satfinite(r)
+//   s == 0 -> codes +0;  else inv = 1 / (s * a32),  y = x * inv,
+//   code = E2M1_rne_satfinite(y) with the sign of y.
+// The hardware conversions below implement exactly these roundings; the
+// test suite checks them exhaustively (all 2^32 inputs) against the oracle.
+// ---------------------------------------------------------------------------
+
+// Two binary32 -> two E2M1 codes in one byte: lo -> bits 3:0, hi -> bits 7:4.
+// Eight values -> 32 bits, element i in bits 4i+3:4i.
+__device__ __forceinline__ uint32_t e2m1x8(const float* y) {
+    uint32_t out;
+    asm("{\n\t"
+        ".reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+        "}"
+        : "=r"(out)
+        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+    return out;
+}
+
+// One non-negative binary32 -> E4M3 code (nearest-even, saturating at 448).
+__device__ __forceinline__ uint32_t e4m3_code(float r) {
+    uint16_t two;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(two) : "f"(0.0f), "f"(r));
+    return two & 0xFFu;
+}
+
+// E4M3 code -> its exact value (every E4M3 value is exact in binary16).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Two E4M3 codes (byte 0, byte 1 of `two`) -> half2 {value0, value1}.
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t two) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(two));
+    return *reinterpret_cast<__half2*>(&h2);
+}
+
+// Two E2M1 codes (bits 3:0 = first, 7:4 = second) -> half2 {first, second}.
+__device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n\t"
+        ".reg .b8 b;\n\t"
+        "cvt.u8.u32 b, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b;\n\t"
+        "}"
+        : "=r"(h2)
+        : "r"(byte));
+    return *reinterpret_cast<__half2*>(&h2);
+}
+
+// Per-block scale: returns the E4M3 code and the reciprocal 1 / (s * a32)
+// (0 when the block is flushed, i.e. s == 0 or a32 == 0).
+struct BlockScale {
+    uint32_t code;
+    float inv;
+};
+
+__device__ __forceinline__ BlockScale block_scale(float amax_b, float a32) {
+    BlockScale b;
+    if (a32 == 0.0f) {
+        b.code = 0u;
+        b.inv = 0.0f;
+        return b;
+    }
+    const float d6 = __fmul_rn(6.0f, a32);
+    const float r = __fdiv_rn(amax_b, d6);
+    b.code = e4m3_code(r);
+    const float s = e4m3_value(b.code);
+    b.inv = (s == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(s, a32));
+    return b;
+}
+
+// Eight elements of one block (binary32) -> 32 bits of codes.  A flushed
+// block (inv == 0) encodes to +0 codes.
+__device__ __forceinline__ uint32_t encode8(const float* x, float inv) {
+    if (inv == 0.0f) return 0u;
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) y[i] = __fmul_rn(x[i], inv);
+    return e2m1x8(y);
+}
+
+// bf16x8 (one uint4) -> 8 binary32
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ float absmax8(const float* f) {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) m = fmaxf(m, fabsf(f[i]));
+    return m;
+}
+
+// Streaming 16-byte load (read once, do not keep in L1).
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Byte offset of scale (r, c) in the swizzled 128x4 tile layout.
+__device__ __forceinline__ int64_t swz_offset(int64_t r, int64_t c, int64_t tiles_c) {
+    return ((r >> 7) * tiles_c + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+// ---------------------------------------------------------------------------
+// Time for bounded waits (%globaltimer, nanoseconds).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on phase `parity` of `bar`.  Gives up (returns false) when
+// *abort becomes non-zero or after limit_ns nanoseconds.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                  uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA (no multicast anywhere in this library)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Plain bulk copy global -> shared (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 (TMEM allocation, MMA, copies, loads)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Arrive on `bar` once every tcgen05 op issued so far by this thread is done.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// Block-scaled FP4 MMA: D[tmem] (+)= (A . SFA)(B . SFB)^T, M=128, K=64 per op.
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Shared memory (32 rows x 16 bytes, no swizzle) -> TMEM lanes 0..31, 4
+// columns, replicated into all four 32-lane sub-partitions.
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// TMEM -> registers: this warp's 32 lanes x 32 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (sm_100 format, version 1).
+//   bits 0-13 start >> 4, 16-29 leading byte offset >> 4, 32-45 stride byte
+//   offset >> 4, 46-47 version = 1, 49-51 base offset, 61-63 layout type.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)(layout & 7u) << 61;
+    return d;
+}
+
+constexpr uint32_t kLayoutNone = 0;
+constexpr uint32_t kLayoutSw128 = 2;
+
+}  // namespace nvfp4

@@ -1,0 +1,548 @@
+// gemm.cu -- W4A4 NVFP4 GEMM for sm_100a with a fused epilogue.
+//
+//   C[M x N] = a32_A * a32_B * (A_q . S_A)(B_q . S_B)^T  -> epilogue -> bf16
+//              and/or NVFP4 re-quantization for the next layer.
+//
+// Method: the W4A4 linear layers of "LongLive-2.0：用 NVFP4 并行底座做长视频生成"
+// (yingwang.github.io reading note), sections "NVFP4 训练的工程细节" (weights and
+// activations in NVFP4, 1D block scaling along K, self-written CUDA kernels)
+// and "推理底座" (4-bit weights and activations at inference); the Dequant
+// equation of section "NVFP4 量化格式" is what the block-scaled MMA applies
+// per 16-element block.  The adaLN modulate/gate epilogue stands in for the
+// fused adaLN kernels of the anzhuoshouzhuan.com article ("NVFP4 量化").
+//
+// Kernel design (B200):
+//  * persistent grid, one CTA per SM, static round-robin tile schedule over
+//    128 x 256 output tiles;
+//  * warp 0: TMA producer (A/B code tiles with 128B swizzle, scale tiles as
+//    plain bulk copies of the 512-byte scale-factor tiles); a 4-stage ring of
+//    K-slices of 256 elements (54 KB per stage);
+//  * warp 1: owns TMEM (512 columns: accumulator 0..255, scales 256..303) and
+//    issues, from one thread, tcgen05.cp of the scale tiles into TMEM and
+//    tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=256, K=64), releasing
+//    each stage with tcgen05.commit;
+//  * warps 2..5: epilogue, tcgen05.ld of 32 columns at a time, binary32 math,
+//    16-byte stores (and the NVFP4 requant with the same encoder as the
+//    quantize kernel);
+//  * every mbarrier wait is bounded (globaltimer); on expiry the kernel
+//    records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
+//    drains what it issued and frees TMEM before returning.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 256;        // K elements per stage
+constexpr int BKB = BK / 2;    // bytes per row per stage (128: one swizzle atom row)
+constexpr int KB_PER_STAGE = BK / 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BKB;            // 16 KB
+constexpr int B_BYTES = BN * BKB;            // 32 KB
+constexpr int SFA_BYTES = KB_PER_STAGE * 512;      // 2 KB
+constexpr int SFB_BYTES = 2 * KB_PER_STAGE * 512;  // 4 KB (two 128-row halves)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t SFA_COL = 256;
+constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;
+
+static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment for 128B swizzle");
+static_assert(SFB_COL + 8 * KB_PER_STAGE <= TMEM_COLS, "TMEM budget");
+
+// instruction descriptor: E2M1 x E2M1, UE4M3 scales, f32 accumulate, K-major
+// A and B, M = 128, N = BN, K = 64 (dense).
+constexpr uint32_t make_idesc(int m, int n) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+constexpr uint32_t IDESC = make_idesc(BM, BN);
+
+struct Params {
+    int M, N, K;
+    int tiles_m, tiles_n, num_tiles;
+    int kt_count;      // ceil(K / BK)
+    int kb_total;      // K / 64
+    int64_t sf_tiles_k;  // scale tiles per 128-row block along K (= K / 64)
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* ga;
+    const float* gb;
+    __nv_bfloat16* c;
+    int64_t ldc;
+    const __nv_bfloat16* bias;
+    const __nv_bfloat16* mod_scale;
+    const __nv_bfloat16* mod_shift;
+    const __nv_bfloat16* gate;
+    const __nv_bfloat16* residual;
+    int64_t ld_res;
+    int act;
+    uint8_t* out_codes;
+    uint8_t* out_scales;
+    const float* out_gscale;
+    float* out_amax;
+    float* debug_y;
+    DevError* err;
+    uint64_t limit_ns;
+    uint32_t dbg;
+};
+
+struct Smem {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tmem_full;
+    uint64_t tmem_empty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ void tile_coords(const Params& p, int tile, int& mb, int& nb) {
+    mb = tile % p.tiles_m;
+    nb = tile / p.tiles_m;
+}
+
+__device__ __forceinline__ void raise_abort(Smem* s, const Params& p, uint32_t where) {
+    record_error(p.err, NVFP4_ERR_TIMEOUT, where);
+    *(volatile int*)&s->abort_flag = 1;
+}
+
+// ---------------------------------------------------------------- producer --
+__device__ void producer(const Params& p, Smem* s, uint8_t* ring, const CUtensorMap* tma_a,
+                         const CUtensorMap* tma_b) {
+    prefetch_tmap(tma_a);
+    prefetch_tmap(tma_b);
+    volatile int* abort = &s->abort_flag;
+    int last_parity[STAGES];
+    for (int i = 0; i < STAGES; i++) last_parity[i] = -1;
+    if (p.dbg & NVFP4_DBG_SKIP_LOADS) return;
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(p, tile, mb, nb);
+        const int halves = ((int64_t)nb * BN + 128 < p.N) ? 2 : 1;
+        for (int kt = 0; kt < p.kt_count; kt++, it++) {
+            const int st = it % STAGES;
+            const uint32_t round = it / STAGES;
+            if (!mbar_wait_bounded(&s->empty[st], (round & 1) ^ 1, abort, p.limit_ns)) {
+                if (!*abort) raise_abort(s, p, 1);
+                goto drain;
+            }
+            {
+                uint8_t* a_s = ring + st * STAGE_BYTES;
+                uint8_t* b_s = a_s + A_BYTES;
+                uint8_t* sfa_s = b_s + B_BYTES;
+                uint8_t* sfb_s = sfa_s + SFA_BYTES;
+                const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
+                const uint32_t bytes = A_BYTES + B_BYTES + (uint32_t)nkb * 512u * (1u + halves);
+                mbar_expect_tx(&s->full[st], bytes);
+                tma_load_2d(a_s, tma_a, &s->full[st], kt * BKB, mb * BM);
+                tma_load_2d(b_s, tma_b, &s->full[st], kt * BKB, nb * BN);
+                const int64_t kt4 = (int64_t)kt * KB_PER_STAGE;
+                bulk_load(sfa_s, p.sfa + ((int64_t)mb * p.sf_tiles_k + kt4) * 512, nkb * 512, &s->full[st]);
+                for (int h = 0; h < halves; h++)
+                    bulk_load(sfb_s + h * (KB_PER_STAGE * 512),
+                              p.sfb + ((int64_t)(nb * 2 + h) * p.sf_tiles_k + kt4) * 512, nkb * 512, &s->full[st]);
+                last_parity[st] = (int)(round & 1);
+            }
+        }
+    }
+    return;
+drain:
+    // the only loads that can still be in flight are the last one per stage
+    for (int i = 0; i < STAGES; i++)
+        if (last_parity[i] >= 0) {
+            volatile int never = 0;
+            mbar_wait_bounded(&s->full[i], (uint32_t)last_parity[i], &never, p.limit_ns);
+        }
+}
+
+// ---------------------------------------------------------------- MMA -------
+__device__ void mma_issuer(const Params& p, Smem* s, uint8_t* ring, uint32_t tmem) {
+    volatile int* abort = &s->abort_flag;
+    uint32_t it = 0;
+    uint32_t tcount = 0;
+    bool issued = false;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, tcount++) {
+        int mb, nb;
+        tile_coords(p, tile, mb, nb);
+        const int halves = ((int64_t)nb * BN + 128 < p.N) ? 2 : 1;
+        if (!mbar_wait_bounded(&s->tmem_empty, (tcount & 1) ^ 1, abort, p.limit_ns)) {
+            if (!*abort) raise_abort(s, p, 2);
+            goto drain;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < p.kt_count; kt++, it++) {
+            const int st = it % STAGES;
+            const uint32_t round = it / STAGES;
+            if (!mbar_wait_bounded(&s->full[st], round & 1, abort, p.limit_ns)) {
+                if (!*abort) raise_abort(s, p, 3);
+                goto drain;
+            }
+            tc_fence_after();
+            const uint32_t a_s = smem_u32(ring + st * STAGE_BYTES);
+            const uint32_t b_s = a_s + A_BYTES;
+            const uint32_t sfa_s = b_s + B_BYTES;
+            const uint32_t sfb_s = sfa_s + SFA_BYTES;
+            const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
+            for (int kb = 0; kb < nkb; kb++) {
+                tc_cp_32x128b_x4(tmem + SFA_COL + 4 * kb, smem_desc(sfa_s + kb * 512, 0, 128, kLayoutNone));
+                for (int h = 0; h < halves; h++)
+                    tc_cp_32x128b_x4(tmem + SFB_COL + 8 * kb + 4 * h,
+                                     smem_desc(sfb_s + h * (KB_PER_STAGE * 512) + kb * 512, 0, 128, kLayoutNone));
+            }
+            for (int kb = 0; kb < nkb; kb++) {
+                const uint64_t ad = smem_desc(a_s + kb * 32, 16, 1024, kLayoutSw128);
+                const uint64_t bd = smem_desc(b_s + kb * 32, 16, 1024, kLayoutSw128);
+                tc_mma_nvf4(tmem + ACC_COL, ad, bd, IDESC, tmem + SFA_COL + 4 * kb, tmem + SFB_COL + 8 * kb,
+                            (kt > 0 || kb > 0) ? 1u : 0u);
+            }
+            issued = true;
+            tc_commit(&s->empty[st]);
+        }
+        tc_commit(&s->tmem_full);
+    }
+    return;
+drain:
+    if (issued) {
+        // wait until every tcgen05 op issued so far has finished
+        tc_commit(&s->drain);
+        volatile int never = 0;
+        mbar_wait_bounded(&s->drain, 0, &never, p.limit_ns);
+    }
+}
+
+// ---------------------------------------------------------------- epilogue --
+__device__ __forceinline__ float gelu_tanh(float y) {
+    const float k = 0.7978845608028654f;  // sqrt(2 / pi)
+    return 0.5f * y * (1.0f + tanhf(k * (y + 0.044715f * y * y * y)));
+}
+
+// 32 consecutive bf16 (as binary32), columns n0.. with `valid` of them in range
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* p, int valid, float* out) {
+    if (valid >= 32) {
+        const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+        for (int i = 0; i < 4; i++) bf16x8_to_f32(__ldg(q + i), out + 8 * i);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) out[i] = (i < valid) ? __bfloat162float(p[i]) : 0.0f;
+    }
+}
+
+__device__ void epilogue(const Params& p, Smem* s, uint32_t tmem, int warp, int lane) {
+    volatile int* abort = &s->abort_flag;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
+    const bool requant = p.out_codes != nullptr;
+    const float oa32 = requant ? __ldg(p.out_gscale) : 0.0f;
+    const int64_t tiles_on = (p.N + 63) / 64;  // scale tiles along N of the output
+    float amax_run = 0.0f;
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, tcount++) {
+        int mb, nb;
+        tile_coords(p, tile, mb, nb);
+        if (!mbar_wait_bounded(&s->tmem_full, tcount & 1, abort, p.limit_ns)) {
+            if (!*abort) raise_abort(s, p, 4);
+            return;
+        }
+        tc_fence_after();
+        const int64_t m = (int64_t)mb * BM + q * 32 + lane;
+        const bool row_ok = m < p.M;
+        const int ncols = min(BN, p.N - nb * BN);
+        const int nchunks = (ncols + 31) / 32;
+        for (int j = 0; j < nchunks; j++) {
+            uint32_t r[32];
+            tmem_ld_32cols(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + j * 32, r);
+            tmem_ld_wait();
+            if (j == nchunks - 1) {
+                // accumulator fully read: let the MMA warp start the next tile
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s->tmem_empty);
+            }
+            const int64_t n0 = (int64_t)nb * BN + j * 32;
+            const int valid = (int)min((int64_t)32, p.N - n0);
+            float y[32];
+#pragma unroll
+            for (int i = 0; i < 32; i++) y[i] = __uint_as_float(r[i]) * alpha;
+            float v[32];
+            if (p.bias) {
+                load_row32(p.bias + n0, valid, v);
+#pragma unroll
+                for (int i = 0; i < 32; i++) y[i] += v[i];
+            }
+            if (p.act == NVFP4_ACT_GELU_TANH) {
+#pragma unroll
+                for (int i = 0; i < 32; i++) y[i] = gelu_tanh(y[i]);
+            }
+            if (p.mod_scale || p.mod_shift) {
+                float w[32];
+                if (p.mod_scale) load_row32(p.mod_scale + n0, valid, v);
+                else
+#pragma unroll
+                    for (int i = 0; i < 32; i++) v[i] = 0.0f;
+                if (p.mod_shift) load_row32(p.mod_shift + n0, valid, w);
+                else
+#pragma unroll
+                    for (int i = 0; i < 32; i++) w[i] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 32; i++) y[i] = y[i] * (1.0f + v[i]) + w[i];
+            }
+            if (p.gate) {
+                load_row32(p.gate + n0, valid, v);
+#pragma unroll
+                for (int i = 0; i < 32; i++) y[i] = v[i] * y[i];
+            }
+            if (p.residual && row_ok) {
+                load_row32(p.residual + m * p.ld_res + n0, valid, v);
+#pragma unroll
+                for (int i = 0; i < 32; i++) y[i] = v[i] + y[i];
+            }
+            if (row_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; i++)
+                    if (i < valid) amax_run = fmaxf(amax_run, fabsf(y[i]));
+            }
+            if (p.debug_y && row_ok) {
+                float* d = p.debug_y + m * p.N + n0;
+                for (int i = 0; i < valid; i++) d[i] = y[i];
+            }
+            if (p.c && row_ok) {
+                __nv_bfloat16* cp = p.c + m * p.ldc + n0;
+                if (valid == 32) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+                        w[i] = *reinterpret_cast<uint32_t*>(&b);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(cp);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                } else {
+                    for (int i = 0; i < valid; i++) cp[i] = __float2bfloat16_rn(y[i]);
+                }
+            }
+            if (requant) {
+                // N % 64 == 0 for requant, so a 32-column chunk is whole
+                const int64_t bj = n0 / 16;
+                uint16_t sc2 = 0;
+                if (row_ok) {
+                    float am0 = 0.0f, am1 = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        am0 = fmaxf(am0, fabsf(y[i]));
+                        am1 = fmaxf(am1, fabsf(y[16 + i]));
+                    }
+                    const BlockScale b0 = block_scale(am0, oa32);
+                    const BlockScale b1 = block_scale(am1, oa32);
+                    const uint4 w = make_uint4(encode8(y, b0.inv), encode8(y + 8, b0.inv), encode8(y + 16, b1.inv),
+                                               encode8(y + 24, b1.inv));
+                    *reinterpret_cast<uint4*>(p.out_codes + m * (p.N / 2) + n0 / 2) = w;
+                    sc2 = (uint16_t)(b0.code | (b1.code << 8));
+                }
+                // rows past M inside the last 128-row tile are scale padding: zero
+                *reinterpret_cast<uint16_t*>(p.out_scales + swz_offset(m, bj, tiles_on)) = sc2;
+            }
+        }
+        if (nchunks == 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s->tmem_empty);
+        }
+    }
+    if (p.out_amax) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax_run = fmaxf(amax_run, __shfl_xor_sync(0xFFFFFFFFu, amax_run, o));
+        if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(p.out_amax), __float_as_uint(amax_run));
+    }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                const __grid_constant__ Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem* s = reinterpret_cast<Smem*>(ring + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; i++) {
+            mbar_init(&s->full[i], 1);
+            mbar_init(&s->empty[i], 1);
+        }
+        mbar_init(&s->tmem_full, 1);
+        mbar_init(&s->tmem_empty, 4);
+        mbar_init(&s->drain, 1);
+        s->abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(&s->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) producer(p, s, ring, &tma_a, &tma_b);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) mma_issuer(p, s, ring, tmem);
+        __syncwarp();
+    } else {
+        epilogue(p, s, tmem, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace gemm
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn g_encode_tiled = nullptr;
+static int g_gemm_sms = 0;
+static int g_gemm_attr_dev = -1;
+
+static nvfp4_status gemm_setup(int& sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (g_encode_tiled == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return NVFP4_ERR_CUDA;
+        g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    if (g_gemm_attr_dev != dev) {
+        int major = 0, minor = 0, n = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (major != 10 || minor != 0) return NVFP4_ERR_UNSUPPORTED;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+        if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        g_gemm_sms = n;
+        g_gemm_attr_dev = dev;
+    }
+    sms = g_gemm_sms;
+    return NVFP4_OK;
+}
+
+static bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t K, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {(cuuint32_t)gemm::BKB, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* c_bf16, int64_t ldc,
+                                   const nvfp4_epilogue* ep, void* workspace, size_t ws_bytes,
+                                   nvfp4_stream_t stream) {
+    if (!A || !B || !workspace) return NVFP4_ERR_INVALID_ARG;
+    if (!A->codes || !A->scales || !A->global_scale || !B->codes || !B->scales || !B->global_scale)
+        return NVFP4_ERR_INVALID_ARG;
+    const int64_t M = A->rows, N = B->rows, K = A->cols;
+    if (M <= 0 || N <= 0 || K <= 0 || B->cols != K) return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
+    if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return NVFP4_ERR_UNSUPPORTED;
+    if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_GEMM, M, N, K)) return NVFP4_ERR_INVALID_ARG;
+    const bool requant = ep && ep->out_codes;
+    if (!c_bf16 && !requant) return NVFP4_ERR_INVALID_ARG;
+    if (requant && (!ep->out_scales || !ep->out_global_scale)) return NVFP4_ERR_INVALID_ARG;
+    if (requant && N % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
+    if (ep && ep->act != NVFP4_ACT_NONE && ep->act != NVFP4_ACT_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
+    if (ep && (ep->debug_flags & ~NVFP4_DBG_SKIP_LOADS)) return NVFP4_ERR_INVALID_ARG;
+    if (ep && ep->residual && ep->ld_residual < N) return NVFP4_ERR_INVALID_ARG;
+    if (c_bf16 && ldc < N) return NVFP4_ERR_INVALID_ARG;
+    if (!al16(A->codes) || !al16(A->scales) || !al16(B->codes) || !al16(B->scales) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return NVFP4_ERR_MISALIGNED;
+    if (c_bf16 && (!al16(c_bf16) || ldc % 8 != 0)) return NVFP4_ERR_MISALIGNED;
+    if (ep) {
+        const void* vecs[4] = {ep->bias, ep->mod_scale, ep->mod_shift, ep->gate};
+        for (const void* v : vecs)
+            if (v && !al16(v)) return NVFP4_ERR_MISALIGNED;
+        if (ep->residual && (!al16(ep->residual) || ep->ld_residual % 8 != 0)) return NVFP4_ERR_MISALIGNED;
+        if (requant && (!al16(ep->out_codes) || !al16(ep->out_scales))) return NVFP4_ERR_MISALIGNED;
+        if (ep->out_amax && (reinterpret_cast<uintptr_t>(ep->out_amax) & 3u)) return NVFP4_ERR_MISALIGNED;
+        if (ep->debug_y && (reinterpret_cast<uintptr_t>(ep->debug_y) & 3u)) return NVFP4_ERR_MISALIGNED;
+    }
+    int sms = 0;
+    nvfp4_status st = gemm_setup(sms);
+    if (st != NVFP4_OK) return st;
+
+    CUtensorMap ma, mb;
+    if (!make_code_map(&ma, A->codes, M, K, gemm::BM) || !make_code_map(&mb, B->codes, N, K, gemm::BN))
+        return NVFP4_ERR_CUDA;
+
+    gemm::Params p{};
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.tiles_m = (int)((M + gemm::BM - 1) / gemm::BM);
+    p.tiles_n = (int)((N + gemm::BN - 1) / gemm::BN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.kt_count = (int)((K + gemm::BK - 1) / gemm::BK);
+    p.kb_total = (int)(K / 64);
+    p.sf_tiles_k = K / 64;
+    p.sfa = static_cast<const uint8_t*>(A->scales);
+    p.sfb = static_cast<const uint8_t*>(B->scales);
+    p.ga = A->global_scale;
+    p.gb = B->global_scale;
+    p.c = static_cast<__nv_bfloat16*>(c_bf16);
+    p.ldc = ldc;
+    if (ep) {
+        p.bias = static_cast<const __nv_bfloat16*>(ep->bias);
+        p.mod_scale = static_cast<const __nv_bfloat16*>(ep->mod_scale);
+        p.mod_shift = static_cast<const __nv_bfloat16*>(ep->mod_shift);
+        p.gate = static_cast<const __nv_bfloat16*>(ep->gate);
+        p.residual = static_cast<const __nv_bfloat16*>(ep->residual);
+        p.ld_res = ep->ld_residual;
+        p.act = ep->act;
+        p.out_codes = static_cast<uint8_t*>(ep->out_codes);
+        p.out_scales = static_cast<uint8_t*>(ep->out_scales);
+        p.out_gscale = ep->out_global_scale;
+        p.out_amax = ep->out_amax;
+        p.debug_y = ep->debug_y;
+        p.dbg = ep->debug_flags;
+        p.limit_ns = (uint64_t)(ep->wait_limit_us ? ep->wait_limit_us : 2000000u) * 1000ull;
+    } else {
+        p.limit_ns = 2000000000ull;
+    }
+    p.err = static_cast<DevError*>(workspace);
+    const int grid = std::min(p.num_tiles, sms);
+    gemm::gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, (cudaStream_t)stream>>>(ma, mb, p);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}

@@ -1,0 +1,233 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: the NVFP4 W4A4 linear layer and the NVFP4
+ * KV-cache store, hand-written for NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title + section):
+ *  [RN]   "LongLive-2.0：用 NVFP4 并行底座做长视频生成" (yingwang.github.io
+ *         reading note), section 二 方法 / "NVFP4 量化格式": E2M1 element codes,
+ *         three-level scaling (FP32 tensor factor, FP8 E4M3 factor per
+ *         16-element block, FP4 element) and the Dequant equation
+ *         Dequant(X) = X^FP4 * a^FP8 * a^FP32.
+ *  [RN-T] same note, "NVFP4 训练的工程细节": weights and activations both 4-bit
+ *         (W4A4) through self-written CUDA kernels; 1D block scaling along K.
+ *  [RN-I] same note, "推理底座": 4-bit weights and activations at inference;
+ *         per-frame-chunk KV quantization, K and V separately, storage
+ *         9/8 * T_c * H * d bytes, dequant in a self-written CUDA kernel.
+ *  [NEWS] anzhuoshouzhuan.com LongLive 2.0 article, "NVFP4 量化" section:
+ *         fused RoPE/adaLN kernels and an in-place quantized KV-cache update.
+ *
+ * Data formats (all buffers are device memory owned by the caller):
+ *  - codes: packed E2M1, two per byte, element 2i in bits 3:0 and element
+ *    2i+1 in bits 7:4; a [rows x cols] tensor takes rows*cols/2 bytes,
+ *    row-major with rows of cols/2 bytes.
+ *  - block scales: one E4M3 byte per 16 consecutive elements of a row.
+ *    GEMM operands use the tensor-core scale-factor tile layout ("swizzled"):
+ *    rows padded to a multiple of 128 and scale columns to a multiple of 4;
+ *    tile (i, j) (rows 128i.., scale columns 4j..) is 512 contiguous bytes at
+ *    (i * ceil(cols/64) + j) * 512; inside it element (r, c) is at byte
+ *    (r % 32) * 16 + (r / 32) * 4 + c.  Padding bytes are zero.  KV slots use
+ *    plain row-major scales [rows x cols/16].
+ *  - tensor scale a32: one binary32 in device memory.
+ *  Quantization of x with tensor scale a32 (readings of [RN]; the pages give
+ *  no rounding rule):  a32 = amax|x| / 2688 (2688 = 6 * 448) when computed;
+ *  per block  s = E4M3_rne_satfinite(amax_b / (6 * a32));  if s == 0 the
+ *  block's codes are +0, else  code = E2M1_rne_satfinite(x * (1 / (s * a32)))
+ *  with the sign of the product kept (negative values that round to zero give
+ *  code 0x8).  Every step is one binary32 operation rounded to nearest-even.
+ *
+ * Conventions:
+ *  - The library never allocates, frees or synchronizes (except
+ *    nvfp4_read_device_error).  All work is enqueued on `stream`.
+ *  - Host-side argument checks run before any launch and return a status;
+ *    nothing is launched when a check fails.  Launch failures return
+ *    NVFP4_ERR_CUDA.  Errors found on the device (a bounded wait that ran out,
+ *    a page-table entry out of range) are recorded in the first 16 bytes of
+ *    the workspace and read back with nvfp4_read_device_error.
+ *  - Device pointers must be 16-byte aligned.  Inputs must be finite.
+ *  - Thread safety: calls may be issued from several host threads on
+ *    different streams as long as each call has its own workspace.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream (NULL = the legacy default stream). */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad flag */
+    NVFP4_ERR_UNSUPPORTED = 2, /* shape the kernels do not handle, or no sm_100 device */
+    NVFP4_ERR_MISALIGNED = 3,  /* pointer or leading dimension not 16-byte aligned */
+    NVFP4_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+    NVFP4_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (device error) */
+    NVFP4_ERR_DEVICE = 6       /* other device-detected error, e.g. slot out of range */
+} nvfp4_status;
+
+/* Static text for a status; never NULL. */
+const char* nvfp4_status_string(nvfp4_status s);
+
+/* Library version, (major << 16) | minor. */
+int nvfp4_version(void);
+
+/* Bytes of packed E2M1 codes for a [rows x cols] tensor: rows * cols / 2.
+ * Returns 0 for negative sizes or odd cols. */
+size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of block scales for a [rows x cols] tensor (cols % 16 == 0):
+ * swizzled != 0 -> ceil(rows/128)*128 * ceil(cols/64)*4 (GEMM operand layout);
+ * swizzled == 0 -> rows * cols / 16 (row-major, KV slots).  0 on bad sizes. */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int swizzled);
+
+enum {
+    NVFP4_OP_QUANTIZE = 0,  /* nvfp4_quantize: m = rows, k = cols, n unused */
+    NVFP4_OP_GEMM = 1,      /* nvfp4_gemm */
+    NVFP4_OP_KV_APPEND = 2, /* nvfp4_kv_append */
+    NVFP4_OP_KV_DEQUANT = 3 /* nvfp4_kv_dequant */
+};
+
+/* Workspace bytes the caller must pass to the call `op` (device memory,
+ * 256-byte aligned).  Never 0: every call keeps its device error record in
+ * the first 16 bytes, which must be zero before a workspace is first used
+ * (nvfp4_read_device_error zeroes them again); the rest needs no
+ * initialization.  A workspace may be shared by calls on one stream. */
+size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k);
+
+/* Synchronizes `stream`, then reads and clears the device error record of
+ * `workspace` (written by the calls that used it).  *code receives
+ * NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_DEVICE; *info (may be NULL) a
+ * call-specific detail (which wait ran out, the offending page-table index).
+ * Returns NVFP4_ERR_CUDA if the synchronization or the copy fails. */
+nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int* code, uint32_t* info);
+
+/* ------------------------------------------------------------------------ */
+/* Quantize  [RN] three-level scaling, [RN-T] 1D blocks of 16 along a row     */
+/* ------------------------------------------------------------------------ */
+#define NVFP4_Q_COMPUTE_GLOBAL 0u /* compute a32 = amax / 2688 and write *global_scale */
+#define NVFP4_Q_GIVEN_GLOBAL 1u   /* read a32 from *global_scale (delayed scaling) */
+#define NVFP4_Q_ROWMAJOR_SCALES 2u /* write row-major scales instead of the swizzled tiles */
+
+/* x_bf16: bf16 [rows x cols], row stride ld elements (ld >= cols, ld % 8 == 0).
+ * cols % 64 == 0, rows >= 0.
+ * codes: nvfp4_codes_bytes(rows, cols) bytes, rows of cols/2 bytes.
+ * scales: nvfp4_scales_bytes(rows, cols, swizzled) bytes (padding zeroed).
+ * global_scale: device binary32, written (COMPUTE) or read (GIVEN).
+ * workspace: nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols) bytes.
+ * Two launches for COMPUTE (amax partials, then encode), one for GIVEN. */
+nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
+                            void* scales, float* global_scale, unsigned flags, void* workspace,
+                            size_t ws_bytes, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* W4A4 GEMM  [RN-T] / [RN-I] W4A4 linears; [NEWS] fused adaLN epilogue        */
+/* ------------------------------------------------------------------------ */
+/* One NVFP4 operand: codes [rows x cols/2], swizzled scales, device a32. */
+typedef struct {
+    const void* codes;
+    const void* scales;
+    const float* global_scale;
+    int64_t rows, cols;
+} nvfp4_tensor;
+
+#define NVFP4_ACT_NONE 0
+#define NVFP4_ACT_GELU_TANH 1 /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) */
+
+/* Debug / test flags of nvfp4_epilogue.debug_flags (0 in production). */
+#define NVFP4_DBG_SKIP_LOADS 1u /* producer issues no loads: the consumer's bounded wait
+                                   must run out and record NVFP4_ERR_TIMEOUT (tests only) */
+
+/* Epilogue, applied in binary32 to y = a32_A * a32_B * acc, in this order:
+ *   y += bias[n];  y = act(y);  y = y * (1 + mod_scale[n]) + mod_shift[n];
+ *   y = gate[n] * y;  y = residual[m, n] + y
+ * (each step skipped when its pointer is NULL / act is NONE).  Then y is
+ * stored as bf16 to c (if non-NULL) and/or re-quantized to NVFP4 with the
+ * given output tensor scale (if out_codes is non-NULL): blocks of 16 along N,
+ * swizzled scales for an [M x N] operand, exactly the quantize rule above.
+ * out_amax (optional) receives atomically max(|y|) over the output, for
+ * calibrating out_global_scale; the caller initializes it.
+ * debug_y (optional, tests) receives y as binary32 [M x N] before the store. */
+typedef struct {
+    const void* bias;      /* bf16 [N] or NULL */
+    const void* mod_scale; /* bf16 [N] or NULL (adaLN scale) */
+    const void* mod_shift; /* bf16 [N] or NULL (adaLN shift) */
+    const void* gate;      /* bf16 [N] or NULL (adaLN gate) */
+    const void* residual;  /* bf16 [M x N], row stride ld_residual, or NULL */
+    int64_t ld_residual;
+    int act;               /* NVFP4_ACT_* */
+    void* out_codes;       /* NVFP4 requant: codes [M x N/2] or NULL */
+    void* out_scales;      /* swizzled scales for [M x N] */
+    const float* out_global_scale; /* device binary32 a32 of the output */
+    float* out_amax;       /* device binary32 or NULL */
+    float* debug_y;        /* device binary32 [M x N] or NULL */
+    unsigned debug_flags;  /* NVFP4_DBG_*, 0 in production */
+    uint32_t wait_limit_us; /* bound of every device-side wait; 0 = default (2 s) */
+} nvfp4_epilogue;
+
+/* C[M x N] = a32_A * a32_B * (A_q . S_A)(B_q . S_B)^T, then the epilogue.
+ * A: [M x K] activations, B: [N x K] weights (both K-major, K = A->cols =
+ * B->cols, K % 64 == 0).  M, N >= 1, arbitrary (tails handled).
+ * c_bf16: [M x N] with row stride ldc (ldc >= N, ldc % 8 == 0) or NULL when
+ * ep->out_codes is set.  ep may be NULL (plain bf16 output).
+ * Requant needs N % 16 == 0.
+ * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM, M, N, K) bytes.
+ * One persistent launch (tcgen05 block-scaled MMA, TMEM accumulators, TMA). */
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* c_bf16, int64_t ldc,
+                        const nvfp4_epilogue* ep, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 KV cache  [RN-I] per-chunk K/V quantization; [NEWS] in-place update  */
+/* ------------------------------------------------------------------------ */
+/* n_slots slots (frame-chunks), each tokens_per_slot x heads x head_dim.
+ * Slot s of K: k_codes + s * T*H*d/2 (T*H*d/2 bytes), k_scales + s * T*H*d/16
+ * (row-major scales over rows of head_dim), k_global[s]; same for V.
+ * head_dim % 16 == 0; T*H*d % 64 == 0. */
+typedef struct {
+    void* k_codes;
+    void* k_scales;
+    void* v_codes;
+    void* v_scales;
+    float* k_global; /* [n_slots] device binary32 */
+    float* v_global; /* [n_slots] device binary32 */
+    int32_t n_slots, tokens_per_slot, heads, head_dim;
+} nvfp4_kv_cache;
+
+/* Quantizes one chunk's K and V (bf16, token-major [T][H][d], contiguous)
+ * in place into slot `slot`: one tensor scale per (slot, K|V) = amax / 2688
+ * over the whole chunk, then the quantize rule above with row-major scales.
+ * workspace: nvfp4_workspace_bytes(NVFP4_OP_KV_APPEND, T*H, 0, d) bytes.
+ * Two launches (amax partials of K and V, then encode of both). */
+nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
+                             const void* v_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* Gathers the n slots listed in slots_dev (device int32 [n], values in
+ * [0, n_slots)) back to bf16: output i covers rows i*T*H .. of k_out / v_out
+ * (bf16 [n][T][H][d]).  Each value is bf16_rne(fl32(fl32(e2m1 * s) * a32)).
+ * An out-of-range slot index records NVFP4_ERR_DEVICE (info = list position)
+ * in the workspace and leaves that output chunk unwritten.
+ * workspace: nvfp4_workspace_bytes(NVFP4_OP_KV_DEQUANT, 0, 0, 0) bytes. */
+nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n, void* k_out_bf16,
+                              void* v_out_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+
+/* ------------------------------------------------------------------------ */
+/* Test support                                                              */
+/* ------------------------------------------------------------------------ */
+/* Runs the device encoders used by every kernel above on n arbitrary
+ * binary32 inputs: e2m1_out[i] = E2M1 code of x[i] (nearest-even, saturating
+ * at 6, sign kept), e4m3_out[i] = E4M3 code of x[i] (nearest-even, saturating
+ * at 448; meant for x >= 0).  Either output may be NULL.  Lets a test sweep
+ * all 2^32 inputs against the CPU definition.  One launch. */
+nvfp4_status nvfp4_test_encode(const float* x, int64_t n, uint8_t* e2m1_out, uint8_t* e4m3_out,
+                               nvfp4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

@@ -1,0 +1,100 @@
+"""CPU checks of the C-ABI boundary: libnvfp4.so loads without a GPU, exports
+every function include/nvfp4.h declares, answers the size queries, and rejects
+bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_video_dit_b200 import build as nvbuild
+from bit_video_dit_b200 import nvfp4 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nvbuild.build()
+    return nv.lib()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_function_is_exported(L):
+    names = _declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(nv.EXPORTS)
+
+
+def test_size_queries(L):
+    assert nv.codes_bytes(4096, 3072) == 4096 * 1536
+    assert nv.scales_bytes(4096, 3072, True) == 4096 * 192
+    assert nv.scales_bytes(4096, 3072, False) == 4096 * 192
+    assert nv.scales_bytes(200, 320, True) == 256 * 20
+    assert nv.scales_bytes(1, 64, True) == 128 * 4
+    assert nv.codes_bytes(3, 5) == 0 and nv.scales_bytes(3, 8, True) == 0
+    for op in range(4):
+        assert nv.workspace_bytes(op, 4096, 9216, 3072) >= 16
+    assert nv.status_string(nv.OK) == "ok"
+    assert "wait" in nv.status_string(nv.ERR_TIMEOUT)
+    assert L.nvfp4_version() >> 16 == 1
+
+
+def test_kv_bytes_are_nine_eighths(L):
+    # K + V per chunk: 2 * (codes + row-major scales) = 9/8 * T * H * d
+    T, H, d = 2640, 24, 128
+    per = nv.codes_bytes(T * H, d) + nv.scales_bytes(T * H, d, False)
+    assert 2 * per == 9 * T * H * d // 8
+
+
+def test_host_side_argument_checks(L):
+    st = L.nvfp4_quantize(None, 16, 64, 64, None, None, None, 0, None, 0, None)
+    assert st == nv.ERR_INVALID_ARG
+    fake = 1 << 20  # never dereferenced: the checks below fail first
+    st = L.nvfp4_quantize(fake, 16, 48, 48, fake, fake, fake, 0, fake, 1 << 16, None)
+    assert st == nv.ERR_UNSUPPORTED  # cols % 64 != 0
+    st = L.nvfp4_quantize(fake, 16, 64, 64, fake, fake, fake, 8, fake, 1 << 16, None)
+    assert st == nv.ERR_INVALID_ARG  # unknown flag
+    st = L.nvfp4_quantize(fake + 8, 16, 64, 64, fake, fake, fake, 0, fake, 1 << 16, None)
+    assert st == nv.ERR_MISALIGNED
+    st = L.nvfp4_quantize(fake, 16, 64, 64, fake, fake, fake, 0, fake, 16, None)
+    assert st == nv.ERR_INVALID_ARG  # workspace too small
+    a = nv.CTensor(fake, fake, fake, 64, 256)
+    b = nv.CTensor(fake, fake, fake, 128, 192)
+    st = L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), fake, 128, None, fake, 4096, None)
+    assert st == nv.ERR_INVALID_ARG  # K mismatch
+    b = nv.CTensor(fake, fake, fake, 128, 96)
+    a = nv.CTensor(fake, fake, fake, 64, 96)
+    st = L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), fake, 128, None, fake, 4096, None)
+    assert st == nv.ERR_UNSUPPORTED  # K % 64
+    a = nv.CTensor(fake, fake, fake, 64, 256)
+    b = nv.CTensor(fake, fake, fake, 128, 256)
+    st = L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), None, 128, None, fake, 4096, None)
+    assert st == nv.ERR_INVALID_ARG  # no output at all
+    st = L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), fake + 16, 100, None, fake, 4096, None)
+    assert st == nv.ERR_INVALID_ARG  # ldc < N
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 24)
+    st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 16, None)
+    assert st == nv.ERR_UNSUPPORTED  # head_dim % 16
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32)
+    st = L.nvfp4_kv_append(ctypes.byref(kv), 4, fake, fake, fake, 1 << 16, None)
+    assert st == nv.ERR_INVALID_ARG  # slot out of range
+    st = L.nvfp4_kv_dequant(ctypes.byref(kv), fake, -1, fake, fake, fake, 1 << 16, None)
+    assert st == nv.ERR_INVALID_ARG
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "bit_video_dit_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
+                assert "nvfp4_oracle" not in src and "liboracle" not in src, f

@@ -1,0 +1,194 @@
+"""GPU parity of nvfp4_gemm against the oracle's fp64 GEMM.
+
+Metric (reading R12): max_ij |C - ref| / max_ij |ref| <= 2e-3, where ref is the
+oracle's fp64 result on the same NVFP4 operands (the operands themselves are
+checked bit-exact by the quantize tests, and re-checked here).  The fused
+requant is checked bit-exact against the oracle's quantize applied to the
+kernel's own binary32 pre-quant values (reading R13).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_video_dit_b200 import nvfp4 as nv
+from bit_video_dit_b200 import synthetic as syn
+
+from .gpu_util import GEMM_TOL, bf16_to_f64, dev_bf16, f32_bits, host_bits, host_u8, normwise_err, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _qboth(bits, alpha=None):
+    """Quantize on the GPU and with the oracle; assert they agree; return both."""
+    xd = dev_bf16(bits)
+    gs = None if alpha is None else torch.tensor([alpha], dtype=torch.float32, device="cuda")
+    q = nv.quantize(xd, global_scale=gs)
+    oc, osc, oa = oracle.quantize(bits, alpha)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_u8(q.codes), oc)
+    assert np.array_equal(host_u8(q.scales), oracle.swizzle(osc))
+    assert f32_bits(q.global_scale.cpu().numpy()) == f32_bits(oa)
+    return q, (oc, osc, oa)
+
+
+def _gemm_case(M, N, K, seed, **ep):
+    a = syn.activations_bf16(M, K, seed=seed)
+    b = syn.normal_bf16((N, K), seed=seed + 1, std=0.02)
+    qa, oa = _qboth(a)
+    qb, ob = _qboth(b)
+    return qa, oa, qb, ob
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 128, 256)])
+def test_tiny_workload(M, N, K):
+    require_gpu()
+    a = syn.tiny_a_bf16(M, K, seed=0)
+    b = syn.normal_bf16((N, K), seed=1)
+    qa, oa = _qboth(a)
+    qb, ob = _qboth(b)
+    c = nv.gemm(qa, qb)
+    y, _ = oracle.gemm(oa, ob, want_bf16=False)
+    got = bf16_to_f64(host_bits(c))
+    assert normwise_err(got, y) <= GEMM_TOL
+    exact = bf16_to_f64(oracle.gemm_exact_bf16(oa, ob))
+    assert normwise_err(got, exact) <= GEMM_TOL
+
+
+def _lossless(rows, cols, seed):
+    g = np.random.default_rng(seed)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    v = grid[g.integers(0, 8, size=(rows, cols))] * g.choice([-1.0, 1.0], size=(rows, cols))
+    v[:, ::16] = 6.0 * g.choice([-1.0, 1.0], size=(rows, cols // 16))
+    e = g.integers(-3, 1, size=(rows, cols // 16)).astype(np.float64)
+    return v * np.repeat(2.0 ** e, 16, axis=1)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 136, 320), (64, 512, 1024)])
+def test_lossless_operands_give_textbook_matmul(M, N, K):
+    # Exact operands: any error in code nibble order, scale-tile layout,
+    # operand transposition or K stepping shows up as an O(1) error.
+    require_gpu()
+    a = _lossless(M, K, 1000 + M)
+    b = _lossless(N, K, 2000 + N)
+    alpha = np.float32(2.0 ** -8)
+    qa, _ = _qboth(syn.f32_to_bf16_bits(a.astype(np.float32)), alpha)
+    qb, _ = _qboth(syn.f32_to_bf16_bits(b.astype(np.float32)), alpha)
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.gemm(qa, qb, debug_y=y)
+    ref = (a @ b.T) * float(alpha) * float(alpha)
+    got = y.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got - ref)) <= 1e-6 * np.max(np.abs(ref))
+
+
+def test_qkv_full_size_sampled_rows():
+    require_gpu()
+    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
+    qa, oa, qb, ob = _gemm_case(M, N, K, seed=2)
+    bias = syn.normal_bf16((N,), seed=4, std=0.02)
+    c = nv.gemm(qa, qb, bias=dev_bf16(bias))
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1],
+                                     np.random.default_rng(5).integers(0, M, 59)]))
+    y, _ = oracle.gemm(oa, ob, bias=bias, rows=rows, want_bf16=False)
+    got = bf16_to_f64(host_bits(c)[rows])
+    assert np.isfinite(got).all()
+    assert normwise_err(got, y) <= GEMM_TOL
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 64), (100, 136, 320), (130, 264, 512), (300, 520, 192),
+                                   (257, 256, 1024), (129, 1000, 64)])
+def test_ragged_shapes(M, N, K):
+    require_gpu()
+    qa, oa, qb, ob = _gemm_case(M, N, K, seed=M + N + K)
+    ldc = (N + 7) // 8 * 8 + 8
+    buf = torch.full((M, ldc), float("nan"), dtype=torch.bfloat16, device="cuda")
+    c = nv.gemm(qa, qb, out=buf[:, :N])
+    y, _ = oracle.gemm(oa, ob, want_bf16=False)
+    got = bf16_to_f64(host_bits(buf[:, :N]))
+    assert normwise_err(got, y) <= GEMM_TOL
+    assert torch.isnan(buf[:, N:]).all()  # nothing written past N
+
+
+def test_epilogue_bias_gelu_modulate_gate_residual():
+    require_gpu()
+    M, N, K = 256, 512, 512
+    qa, oa, qb, ob = _gemm_case(M, N, K, seed=11)
+    bias = syn.normal_bf16((N,), seed=12, std=0.1)
+    ms = syn.normal_bf16((N,), seed=13, std=0.1)
+    sh = syn.normal_bf16((N,), seed=14, std=0.1)
+    gt = syn.normal_bf16((N,), seed=15, std=0.5)
+    res = syn.normal_bf16((M, N), seed=16)
+    for kw in (dict(bias=bias, act=nv.ACT_GELU_TANH), dict(mod_scale=ms, mod_shift=sh),
+               dict(bias=bias, gate=gt, residual=res), dict(bias=bias, act=1, mod_scale=ms, mod_shift=sh,
+                                                             gate=gt, residual=res)):
+        dk = {k: (dev_bf16(v) if isinstance(v, np.ndarray) else v) for k, v in kw.items()}
+        c = nv.gemm(qa, qb, **dk)
+        y, _ = oracle.gemm(oa, ob, want_bf16=False, **kw)
+        assert normwise_err(bf16_to_f64(host_bits(c)), y) <= GEMM_TOL, list(kw)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 320, 512)])
+def test_requant_epilogue_bit_exact_given_prequant_values(M, N, K):
+    require_gpu()
+    qa, oa, qb, ob = _gemm_case(M, N, K, seed=21)
+    bias = syn.normal_bf16((N,), seed=22, std=0.1)
+    y_ref, _ = oracle.gemm(oa, ob, bias=bias, act=1, want_bf16=False)
+    out_a32 = np.float32(np.max(np.abs(y_ref)) / 2688.0)
+    rq = nv.empty_nvfp4(M, N)
+    rq.global_scale.fill_(float(out_a32))
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    dy = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    c = nv.gemm(qa, qb, bias=dev_bf16(bias), act=nv.ACT_GELU_TANH, requant=rq, out_amax=amax, debug_y=dy)
+    torch.cuda.synchronize()
+    y = dy.cpu().numpy()
+    assert normwise_err(y.astype(np.float64), y_ref) <= GEMM_TOL
+    assert normwise_err(bf16_to_f64(host_bits(c)), y_ref) <= GEMM_TOL
+    codes, scales, _ = oracle.quantize(np.ascontiguousarray(y), out_a32)
+    assert np.array_equal(host_u8(rq.codes), codes)
+    assert np.array_equal(host_u8(rq.scales), oracle.swizzle(scales))
+    assert float(amax.item()) == float(np.max(np.abs(y)))
+    # requant alone (no bf16 output) gives the same codes
+    rq2 = nv.empty_nvfp4(M, N)
+    rq2.global_scale.fill_(float(out_a32))
+    nv.gemm(qa, qb, bias=dev_bf16(bias), act=nv.ACT_GELU_TANH, requant=rq2, bf16_out=False)
+    torch.cuda.synchronize()
+    assert torch.equal(rq2.codes, rq.codes) and torch.equal(rq2.scales, rq.scales)
+
+
+def test_ffn_pair_up_requant_feeds_down():
+    require_gpu()
+    M, D, F = 512, 768, 1536
+    a = syn.activations_bf16(M, D, seed=31)
+    wu = syn.normal_bf16((F, D), seed=32, std=0.02)
+    wd = syn.normal_bf16((D, F), seed=33, std=0.02)
+    qa, oa = _qboth(a)
+    qu, ou = _qboth(wu)
+    qd, od = _qboth(wd)
+    # calibration pass: out_amax of the up-projection gives its output scale
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, out_amax=amax)
+    h = nv.empty_nvfp4(M, F)
+    h.global_scale.copy_(amax / 2688.0)
+    nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, requant=h, bf16_out=False)
+    out = nv.gemm(h, qd)
+    torch.cuda.synchronize()
+    oh = (host_u8(h.codes), oracle.unswizzle(host_u8(h.scales), M, F // 16), np.float32(h.global_scale.item()))
+    y, _ = oracle.gemm(oh, od, want_bf16=False)
+    assert normwise_err(bf16_to_f64(host_bits(out)), y) <= GEMM_TOL
+    # and the whole chain stays close to the fp64 chain of the oracle
+    yu, _ = oracle.gemm(oa, ou, act=1, want_bf16=False)
+    assert abs(float(amax.item()) - np.max(np.abs(yu))) <= 2e-3 * np.max(np.abs(yu))
+
+
+def test_bounded_wait_records_timeout_and_context_survives():
+    require_gpu()
+    qa, oa, qb, ob = _gemm_case(128, 256, 256, seed=41)
+    ws = nv.workspace(nv.OP_GEMM)
+    nv.gemm(qa, qb, debug_flags=nv.DBG_SKIP_LOADS, wait_limit_us=50000, ws=ws)
+    code, info = nv.read_device_error(ws)
+    assert code == nv.ERR_TIMEOUT and info in (2, 3, 4)
+    c = nv.gemm(qa, qb, ws=ws)
+    code, _ = nv.read_device_error(ws)
+    assert code == nv.OK
+    y, _ = oracle.gemm(oa, ob, want_bf16=False)
+    assert normwise_err(bf16_to_f64(host_bits(c)), y) <= GEMM_TOL

@@ -1,0 +1,80 @@
+"""GPU parity of nvfp4_quantize against the CPU oracle: codes, scales (swizzled
+bytes including the zero padding) and the tensor scale, bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_video_dit_b200 import nvfp4 as nv
+from bit_video_dit_b200 import synthetic as syn
+
+from .gpu_util import dev_bf16, f32_bits, host_u8, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(x_bits, *, ld=None, alpha=None, rowmajor=False):
+    require_gpu()
+    rows, cols = x_bits.shape
+    if ld is None:
+        xd = dev_bf16(x_bits)
+    else:  # embed in a wider buffer: row stride ld elements
+        buf = np.zeros((rows, ld), np.uint16)
+        buf[:, :cols] = x_bits
+        xd = dev_bf16(buf)[:, :cols]
+    gs = None if alpha is None else torch.tensor([alpha], dtype=torch.float32, device="cuda")
+    q = nv.quantize(xd, global_scale=gs, rowmajor_scales=rowmajor)
+    torch.cuda.synchronize()
+    codes, scales, a32 = oracle.quantize(x_bits, alpha)
+    assert f32_bits(q.global_scale.cpu().numpy()) == f32_bits(a32)
+    gc = host_u8(q.codes)
+    bad = np.argwhere(gc != codes)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:4].tolist()}"
+    gsc = host_u8(q.scales)
+    want = scales.reshape(-1) if rowmajor else oracle.swizzle(scales)
+    assert gsc.shape == want.shape
+    bad = np.nonzero(gsc != want)[0]
+    assert bad.size == 0, f"{bad.size} scale bytes differ, first at {bad[:4].tolist()}"
+    return q
+
+
+def test_tiny_operands():
+    _check(syn.tiny_a_bf16(64, 256, seed=0))
+    _check(syn.normal_bf16((128, 256), seed=1))
+
+
+def test_qkv_activation_full_size():
+    _check(syn.activations_bf16(4096, 3072, seed=2))
+
+
+def test_qkv_weight_full_size():
+    _check(syn.normal_bf16((9216, 3072), seed=3, std=0.02))
+
+
+@pytest.mark.parametrize("rows,cols,ld", [(1, 64, None), (200, 320, None), (129, 576, 640), (3, 1024, None),
+                                          (130, 64, 72), (257, 128, None)])
+def test_ragged_shapes_and_strides(rows, cols, ld):
+    _check(syn.activations_bf16(rows, cols, seed=rows + cols), ld=ld)
+
+
+def test_all_zero_tensor():
+    q = _check(np.zeros((64, 128), np.uint16))
+    assert float(q.global_scale.item()) == 0.0
+
+
+def test_given_scale_saturates_and_flushes():
+    x = syn.activations_bf16(128, 512, seed=7)
+    _, _, a32 = oracle.quantize(x)
+    _check(x, alpha=np.float32(a32 / 8))    # block scales saturate at 448
+    _check(x, alpha=np.float32(a32 * 1e5))  # most block scales flush to zero
+
+
+def test_rowmajor_scales():
+    _check(syn.activations_bf16(96, 256, seed=8), rowmajor=True)
+
+
+def test_zero_rows_is_a_noop():
+    require_gpu()
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    q = nv.quantize(x)
+    assert q.codes.numel() == 0
