@@ -3,8 +3,10 @@
 #include "common.cuh"
 
 namespace {
-constexpr size_t kWsError = 256;                            // DevError, padded
-constexpr size_t kWsAmax = 256 + 2 * 1024 * sizeof(float);  // error + 2 x 1024 amax partials
+// Every call's workspace starts with a 256-byte control block: the device
+// error record (bytes 0..15) and, for quantize / KV append, the grid-barrier
+// words and tensor maxima of the fused kernel.
+constexpr size_t kWsControl = 256;
 }
 
 extern "C" const char* nvfp4_status_string(nvfp4_status s) {
@@ -41,11 +43,11 @@ extern "C" size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
     (void)k;
     switch (op) {
         case NVFP4_OP_QUANTIZE:
-        case NVFP4_OP_KV_APPEND: return kWsAmax;
+        case NVFP4_OP_KV_APPEND:
         case NVFP4_OP_GEMM:
-        case NVFP4_OP_KV_DEQUANT: return kWsError;
+        case NVFP4_OP_KV_DEQUANT: return kWsControl;
     }
-    return kWsAmax;
+    return kWsControl;
 }
 
 extern "C" nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int* code, uint32_t* info) {
@@ -53,8 +55,10 @@ extern "C" nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t 
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     nvfp4::DevError e;
     if (cudaMemcpy(&e, workspace, sizeof e, cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4_ERR_CUDA;
-    const nvfp4::DevError zero{};
-    if (cudaMemcpy(workspace, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return NVFP4_ERR_CUDA;
+    // after an error the whole control block is reset (a wait that ran out
+    // may have left the grid-barrier words of the fused quantize mid-way)
+    const size_t n = e.code ? kWsControl : sizeof e;
+    if (cudaMemset(workspace, 0, n) != cudaSuccess) return NVFP4_ERR_CUDA;
     *code = (int)e.code;
     if (info) *info = e.info;
     return NVFP4_OK;

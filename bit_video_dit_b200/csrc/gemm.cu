@@ -17,13 +17,14 @@
 //  * warp 0: TMA producer (A/B code tiles with 128B swizzle, scale tiles as
 //    plain bulk copies of the 512-byte scale-factor tiles); a 4-stage ring of
 //    K-slices of 256 elements (54 KB per stage);
-//  * warp 1: owns TMEM (512 columns: accumulator 0..255, scales 256..303) and
-//    issues, from one thread, tcgen05.cp of the scale tiles into TMEM and
-//    tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=256, K=64), releasing
-//    each stage with tcgen05.commit;
+//  * warp 1: owns TMEM (512 columns: two overlapping 256-column accumulators
+//    and 48 scale columns) and issues, from one thread, tcgen05.cp of the
+//    scale tiles into TMEM and tcgen05.mma.kind::mxf4nvf4.block_scale (M=128,
+//    N=256, K=64), releasing each stage with tcgen05.commit;
 //  * warps 2..5: epilogue, tcgen05.ld of 32 columns at a time, binary32 math,
 //    16-byte stores (and the NVFP4 requant with the same encoder as the
-//    quantize kernel);
+//    quantize kernel); it drains the columns both accumulators share first,
+//    so the next tile's MMAs run while the rest of the epilogue proceeds;
 //  * every mbarrier wait is bounded (globaltimer); on expiry the kernel
 //    records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
 //    drains what it issued and frees TMEM before returning.
@@ -48,12 +49,20 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SFA_COL = 256;
-constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;
+// Two accumulators of BN columns share TMEM with the 48 scale columns:
+// acc0 = [0, 256), acc1 = [192, 448), scales = [448, 496).  They overlap in
+// columns [192, 256); the epilogue drains those first (acc0: its chunks 6, 7;
+// acc1: its chunks 0, 1) and then lets the next tile's MMAs start, so the
+// rest of the epilogue overlaps the next mainloop.
+constexpr uint32_t SF_COLS = 4 * KB_PER_STAGE + 8 * KB_PER_STAGE;  // 48
+constexpr uint32_t ACC1_COL = 192;
+constexpr uint32_t SFA_COL = ACC1_COL + BN;                        // 448
+constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;           // 464
+constexpr int OVERLAP_CHUNKS = (BN - (int)ACC1_COL) / 32;          // 2
 
 static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment for 128B swizzle");
-static_assert(SFB_COL + 8 * KB_PER_STAGE <= TMEM_COLS, "TMEM budget");
+static_assert(SFA_COL + SF_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(ACC1_COL % 32 == 0 && OVERLAP_CHUNKS == 2, "overlap must be whole 32-column chunks");
 
 // instruction descriptor: E2M1 x E2M1, UE4M3 scales, f32 accumulate, K-major
 // A and B, M = 128, N = BN, K = 64 (dense).
@@ -117,8 +126,7 @@ __device__ void producer(const Params& p, Smem* s, uint8_t* ring, const CUtensor
     prefetch_tmap(tma_a);
     prefetch_tmap(tma_b);
     volatile int* abort = &s->abort_flag;
-    int last_parity[STAGES];
-    for (int i = 0; i < STAGES; i++) last_parity[i] = -1;
+    uint32_t issued_mask = 0, parity_mask = 0;  // per stage: a load was issued / its phase parity
     if (p.dbg & NVFP4_DBG_SKIP_LOADS) return;
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -147,7 +155,8 @@ __device__ void producer(const Params& p, Smem* s, uint8_t* ring, const CUtensor
                 for (int h = 0; h < halves; h++)
                     bulk_load(sfb_s + h * (KB_PER_STAGE * 512),
                               p.sfb + ((int64_t)(nb * 2 + h) * p.sf_tiles_k + kt4) * 512, nkb * 512, &s->full[st]);
-                last_parity[st] = (int)(round & 1);
+                issued_mask |= 1u << st;
+                parity_mask = (parity_mask & ~(1u << st)) | ((round & 1u) << st);
             }
         }
     }
@@ -155,9 +164,9 @@ __device__ void producer(const Params& p, Smem* s, uint8_t* ring, const CUtensor
 drain:
     // the only loads that can still be in flight are the last one per stage
     for (int i = 0; i < STAGES; i++)
-        if (last_parity[i] >= 0) {
+        if (issued_mask & (1u << i)) {
             volatile int never = 0;
-            mbar_wait_bounded(&s->full[i], (uint32_t)last_parity[i], &never, p.limit_ns);
+            mbar_wait_bounded(&s->full[i], (parity_mask >> i) & 1u, &never, p.limit_ns);
         }
 }
 
@@ -195,10 +204,11 @@ __device__ void mma_issuer(const Params& p, Smem* s, uint8_t* ring, uint32_t tme
                     tc_cp_32x128b_x4(tmem + SFB_COL + 8 * kb + 4 * h,
                                      smem_desc(sfb_s + h * (KB_PER_STAGE * 512) + kb * 512, 0, 128, kLayoutNone));
             }
+            const uint32_t acc = tmem + ((tcount & 1) ? ACC1_COL : 0u);
             for (int kb = 0; kb < nkb; kb++) {
                 const uint64_t ad = smem_desc(a_s + kb * 32, 16, 1024, kLayoutSw128);
                 const uint64_t bd = smem_desc(b_s + kb * 32, 16, 1024, kLayoutSw128);
-                tc_mma_nvf4(tmem + ACC_COL, ad, bd, IDESC, tmem + SFA_COL + 4 * kb, tmem + SFB_COL + 8 * kb,
+                tc_mma_nvf4(acc, ad, bd, IDESC, tmem + SFA_COL + 4 * kb, tmem + SFB_COL + 8 * kb,
                             (kt > 0 || kb > 0) ? 1u : 0u);
             }
             issued = true;
@@ -222,7 +232,8 @@ __device__ __forceinline__ float gelu_tanh(float y) {
     return 0.5f * y * (1.0f + tanhf(k * (y + 0.044715f * y * y * y)));
 }
 
-// 32 consecutive bf16 (as binary32), columns n0.. with `valid` of them in range
+// 32 consecutive bf16 (as binary32), columns n0.. with `valid` of them in
+// range (fully unrolled: the values stay in registers)
 __device__ __forceinline__ void load_row32(const __nv_bfloat16* p, int valid, float* out) {
     if (valid >= 32) {
         const uint4* q = reinterpret_cast<const uint4*>(p);
@@ -234,13 +245,102 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* p, int valid, fl
     }
 }
 
+// One 32-column chunk of one output row: epilogue math and stores.
+__device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* r, float alpha, int64_t m, bool row_ok,
+                                               int64_t n0, int valid, float oa32, int64_t tiles_on,
+                                               float& amax_run) {
+    float y[32];
+#pragma unroll
+    for (int i = 0; i < 32; i++) y[i] = __uint_as_float(r[i]) * alpha;
+    float v[32];
+    if (p.bias) {
+        load_row32(p.bias + n0, valid, v);
+#pragma unroll
+        for (int i = 0; i < 32; i++) y[i] += v[i];
+    }
+    if (p.act == NVFP4_ACT_GELU_TANH) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) y[i] = gelu_tanh(y[i]);
+    }
+    if (p.mod_scale) {
+        load_row32(p.mod_scale + n0, valid, v);
+#pragma unroll
+        for (int i = 0; i < 32; i++) y[i] = y[i] * (1.0f + v[i]);
+    }
+    if (p.mod_shift) {
+        load_row32(p.mod_shift + n0, valid, v);
+#pragma unroll
+        for (int i = 0; i < 32; i++) y[i] += v[i];
+    }
+    if (p.gate) {
+        load_row32(p.gate + n0, valid, v);
+#pragma unroll
+        for (int i = 0; i < 32; i++) y[i] = v[i] * y[i];
+    }
+    if (p.residual && row_ok) {
+        load_row32(p.residual + m * p.ld_res + n0, valid, v);
+#pragma unroll
+        for (int i = 0; i < 32; i++) y[i] = v[i] + y[i];
+    }
+    if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; i++)
+            if (i < valid) amax_run = fmaxf(amax_run, fabsf(y[i]));
+    }
+    if (p.debug_y && row_ok) {
+        float* d = p.debug_y + m * p.N + n0;
+#pragma unroll
+        for (int i = 0; i < 32; i++)
+            if (i < valid) d[i] = y[i];
+    }
+    if (p.c && row_ok) {
+        __nv_bfloat16* cp = p.c + m * p.ldc + n0;
+        if (valid == 32) {
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+                w[i] = *reinterpret_cast<uint32_t*>(&b);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(cp);
+#pragma unroll
+            for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; i++)
+                if (i < valid) cp[i] = __float2bfloat16_rn(y[i]);
+        }
+    }
+    if (p.out_codes) {
+        // N % 64 == 0 for requant, so a 32-column chunk is whole
+        const int64_t bj = n0 / 16;
+        uint16_t sc2 = 0;
+        if (row_ok) {
+            float am0 = 0.0f, am1 = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                am0 = fmaxf(am0, fabsf(y[i]));
+                am1 = fmaxf(am1, fabsf(y[16 + i]));
+            }
+            const BlockScale b0 = block_scale(am0, oa32);
+            const BlockScale b1 = block_scale(am1, oa32);
+            const uint4 w = make_uint4(encode8(y, b0.inv), encode8(y + 8, b0.inv), encode8(y + 16, b1.inv),
+                                       encode8(y + 24, b1.inv));
+            *reinterpret_cast<uint4*>(p.out_codes + m * (p.N / 2) + n0 / 2) = w;
+            sc2 = (uint16_t)(b0.code | (b1.code << 8));
+        }
+        // rows past M inside the last 128-row tile are scale padding: zero
+        *reinterpret_cast<uint16_t*>(p.out_scales + swz_offset(m, bj, tiles_on)) = sc2;
+    }
+}
+
 __device__ void epilogue(const Params& p, Smem* s, uint32_t tmem, int warp, int lane) {
     volatile int* abort = &s->abort_flag;
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
-    const bool requant = p.out_codes != nullptr;
-    const float oa32 = requant ? __ldg(p.out_gscale) : 0.0f;
+    const float oa32 = p.out_codes ? __ldg(p.out_gscale) : 0.0f;
     const int64_t tiles_on = (p.N + 63) / 64;  // scale tiles along N of the output
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     float amax_run = 0.0f;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, tcount++) {
@@ -255,105 +355,31 @@ __device__ void epilogue(const Params& p, Smem* s, uint32_t tmem, int warp, int 
         const bool row_ok = m < p.M;
         const int ncols = min(BN, p.N - nb * BN);
         const int nchunks = (ncols + 31) / 32;
-        for (int j = 0; j < nchunks; j++) {
+        const bool buf1 = tcount & 1;
+        const uint32_t acc = lane_base + (buf1 ? ACC1_COL : 0u);
+        // chunks of this buffer that the other buffer overlaps come first
+        const int first = buf1 ? 0 : (BN / 32 - OVERLAP_CHUNKS);
+        int n_overlap = buf1 ? min(nchunks, OVERLAP_CHUNKS) : max(0, nchunks - first);
+        if (n_overlap == 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s->tmem_empty);
+        }
+        for (int i = 0; i < nchunks; i++) {
+            // buffer 0 visits chunks 6, 7, 0, 1, ..., 5; buffer 1 visits 0..7
+            const int j = buf1 ? i : ((i < n_overlap) ? first + i : i - n_overlap);
             uint32_t r[32];
-            tmem_ld_32cols(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + j * 32, r);
+            tmem_ld_32cols(acc + j * 32, r);
             tmem_ld_wait();
-            if (j == nchunks - 1) {
-                // accumulator fully read: let the MMA warp start the next tile
+            if (i == n_overlap - 1) {
+                // the overlapped columns are in registers: next tile may start
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s->tmem_empty);
             }
             const int64_t n0 = (int64_t)nb * BN + j * 32;
             const int valid = (int)min((int64_t)32, p.N - n0);
-            float y[32];
-#pragma unroll
-            for (int i = 0; i < 32; i++) y[i] = __uint_as_float(r[i]) * alpha;
-            float v[32];
-            if (p.bias) {
-                load_row32(p.bias + n0, valid, v);
-#pragma unroll
-                for (int i = 0; i < 32; i++) y[i] += v[i];
-            }
-            if (p.act == NVFP4_ACT_GELU_TANH) {
-#pragma unroll
-                for (int i = 0; i < 32; i++) y[i] = gelu_tanh(y[i]);
-            }
-            if (p.mod_scale || p.mod_shift) {
-                float w[32];
-                if (p.mod_scale) load_row32(p.mod_scale + n0, valid, v);
-                else
-#pragma unroll
-                    for (int i = 0; i < 32; i++) v[i] = 0.0f;
-                if (p.mod_shift) load_row32(p.mod_shift + n0, valid, w);
-                else
-#pragma unroll
-                    for (int i = 0; i < 32; i++) w[i] = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 32; i++) y[i] = y[i] * (1.0f + v[i]) + w[i];
-            }
-            if (p.gate) {
-                load_row32(p.gate + n0, valid, v);
-#pragma unroll
-                for (int i = 0; i < 32; i++) y[i] = v[i] * y[i];
-            }
-            if (p.residual && row_ok) {
-                load_row32(p.residual + m * p.ld_res + n0, valid, v);
-#pragma unroll
-                for (int i = 0; i < 32; i++) y[i] = v[i] + y[i];
-            }
-            if (row_ok) {
-#pragma unroll
-                for (int i = 0; i < 32; i++)
-                    if (i < valid) amax_run = fmaxf(amax_run, fabsf(y[i]));
-            }
-            if (p.debug_y && row_ok) {
-                float* d = p.debug_y + m * p.N + n0;
-                for (int i = 0; i < valid; i++) d[i] = y[i];
-            }
-            if (p.c && row_ok) {
-                __nv_bfloat16* cp = p.c + m * p.ldc + n0;
-                if (valid == 32) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int i = 0; i < 16; i++) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
-                        w[i] = *reinterpret_cast<uint32_t*>(&b);
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(cp);
-#pragma unroll
-                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-                } else {
-                    for (int i = 0; i < valid; i++) cp[i] = __float2bfloat16_rn(y[i]);
-                }
-            }
-            if (requant) {
-                // N % 64 == 0 for requant, so a 32-column chunk is whole
-                const int64_t bj = n0 / 16;
-                uint16_t sc2 = 0;
-                if (row_ok) {
-                    float am0 = 0.0f, am1 = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 16; i++) {
-                        am0 = fmaxf(am0, fabsf(y[i]));
-                        am1 = fmaxf(am1, fabsf(y[16 + i]));
-                    }
-                    const BlockScale b0 = block_scale(am0, oa32);
-                    const BlockScale b1 = block_scale(am1, oa32);
-                    const uint4 w = make_uint4(encode8(y, b0.inv), encode8(y + 8, b0.inv), encode8(y + 16, b1.inv),
-                                               encode8(y + 24, b1.inv));
-                    *reinterpret_cast<uint4*>(p.out_codes + m * (p.N / 2) + n0 / 2) = w;
-                    sc2 = (uint16_t)(b0.code | (b1.code << 8));
-                }
-                // rows past M inside the last 128-row tile are scale padding: zero
-                *reinterpret_cast<uint16_t*>(p.out_scales + swz_offset(m, bj, tiles_on)) = sc2;
-            }
-        }
-        if (nchunks == 0) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s->tmem_empty);
+            epilogue_chunk(p, r, alpha, m, row_ok, n0, valid, oa32, tiles_on, amax_run);
         }
     }
     if (p.out_amax) {

@@ -8,132 +8,237 @@
 // anzhuoshouzhuan.com article's in-place quantized KV-cache update.
 //
 // All kernels here are HBM-bandwidth bound.  Layout of the work:
-//  * amax pass: 16-byte streaming loads, |x| max on the bf16 bit patterns
-//    (two 16-bit lanes per 32-bit SIMD max), one partial per CTA -- no atomics
-//    and no memset launch.
-//  * encode pass: a warp owns a 512-element run of one row; lane i loads the
-//    16-byte chunks i and i+32 (each warp-wide load is 512 contiguous bytes),
+//  * quantize / KV append: one cooperative launch (see quantize_fused_kernel):
+//    bulk copies into shared memory, |x| max on the bf16 bit patterns (two
+//    16-bit lanes per 32-bit SIMD max), a bounded grid barrier for the tensor
+//    scale, then the encode from shared memory.  In the encode a warp owns a
+//    512-element run of one row; lane i holds the 16-byte chunks i and i+32,
 //    a block of 16 elements is a lane pair (one shuffle for the block amax),
-//    and the 4-byte code stores of a warp are 128 contiguous bytes.
-//  * dequant-gather: a warp owns 256 elements of a slot: 4-byte code loads,
-//    16-byte bf16 stores (512 contiguous bytes per warp store).
+//    and a warp's 4-byte code stores are 128 contiguous bytes.
+//  * dequant-gather: a warp owns 512-element runs of a slot; lane i decodes
+//    elements 8i..8i+7 and 256+8i..256+8i+7 (4-byte code loads, 16-byte bf16
+//    stores, each warp-wide access contiguous), two runs in flight per lane.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace nvfp4 {
 
-constexpr int kThreads = 256;
-constexpr int kMaxPartials = 1024;  // amax partials per tensor (one per CTA)
+constexpr int kThreads = 256;  // dequant / probe kernels
 
-// Workspace layout shared by quantize and kv_append:
-//   [0, 16)        DevError
-//   [256, 256+4K)  amax partials of tensor 0
-//   [256+4K, ..)   amax partials of tensor 1
-constexpr size_t kWsPartials = 256;
-constexpr size_t kWsQuantize = kWsPartials + 2 * kMaxPartials * sizeof(float);
+// ---------------------------------------------------------------------------
+// Fused quantize: one cooperative launch, one CTA per SM.
+//   phase 1  every CTA bulk-copies (cp.async.bulk, no registers involved) its
+//            contiguous share of 512-element row runs into shared memory and
+//            takes the |x| max of it;
+//   barrier  the CTA maxima meet in one atomicMax word per tensor; the last
+//            CTA to arrive turns it into a32 = amax / 2688 and releases the
+//            grid (bounded wait everywhere else);
+//   phase 2  every CTA encodes its runs straight from shared memory.
+// HBM is read once and written once.  Runs that do not fit in shared memory
+// (tensors larger than ~#SMs x 200 KB) are read from global memory in both
+// phases instead.
+// ---------------------------------------------------------------------------
+constexpr int kQThreads = 512;
+constexpr int kQWarps = kQThreads / 32;
+constexpr int kRunBytes = 1024;  // one 512-element bf16 run
 
-struct AmaxArgs {
-    const uint8_t* x[2];
-    int64_t rows, cols, ld;  // elements
-    float* partials;         // [2][kMaxPartials]
-};
+// Control block in the first 256 bytes of the workspace (zero before first use).
+constexpr int kCtlCount = 8;   // uint32 index: CTAs arrived at the grid barrier
+constexpr int kCtlGen = 9;     // barrier generation
+constexpr int kCtlAmax = 10;   // [2] bf16 magnitude bit patterns, reset by the releasing CTA
+constexpr int kCtlAlpha = 12;  // [2] a32 bits
 
-// max of |bf16| over 8 values, on the bit patterns (exact for finite values)
-__device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
-    const uint32_t m = 0x7FFF7FFFu;
-    uint32_t a = __vmaxu2(v.x & m, v.y & m);
-    uint32_t b = __vmaxu2(v.z & m, v.w & m);
-    return __vmaxu2(a, b);
-}
-
-__global__ void __launch_bounds__(kThreads) amax_kernel(AmaxArgs a) {
-    const uint8_t* base = a.x[blockIdx.y];
-    const int64_t cpr = a.cols / 8;  // 16-byte chunks per row
-    const int64_t total = a.rows * cpr;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    uint32_t m2 = 0;
-    if (a.ld == a.cols) {
-        for (; i + 3 * stride < total; i += 4 * stride) {
-            uint4 v0 = ld_stream16(base + i * 16);
-            uint4 v1 = ld_stream16(base + (i + stride) * 16);
-            uint4 v2 = ld_stream16(base + (i + 2 * stride) * 16);
-            uint4 v3 = ld_stream16(base + (i + 3 * stride) * 16);
-            m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(absmax_bits8(v0), absmax_bits8(v1)),
-                                       __vmaxu2(absmax_bits8(v2), absmax_bits8(v3))));
-        }
-        for (; i < total; i += stride) m2 = __vmaxu2(m2, absmax_bits8(ld_stream16(base + i * 16)));
-    } else {
-        for (; i < total; i += stride) {
-            const int64_t r = i / cpr, c = i - r * cpr;
-            m2 = __vmaxu2(m2, absmax_bits8(ld_stream16(base + (r * a.ld + c * 8) * 2)));
-        }
-    }
-    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __shared__ uint32_t red[kThreads / 32];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t r = 0;
-        for (int w = 0; w < kThreads / 32; w++) r = max(r, red[w]);
-        a.partials[blockIdx.y * kMaxPartials + blockIdx.x] = __uint_as_float(r << 16);
-    }
-}
-
-struct EncodeArgs {
+struct QuantArgs {
     const uint8_t* x[2];
     uint8_t* codes[2];
     uint8_t* scales[2];
-    float* gscale[2];        // a32: written (computed) or read (given)
-    int64_t rows, cols, ld;  // elements
-    const float* partials;   // [2][kMaxPartials] when computed
-    int nparts;
+    float* gscale[2];
+    int64_t rows, cols, ld;   // per tensor, elements
+    int64_t upr;              // 512-element runs per row
+    int64_t runs_per_tensor;
+    int64_t total_runs;       // ntensors * runs_per_tensor
     int given;
     int swizzled;
-    int64_t tiles_c;         // ceil(cols / 64)
+    int64_t tiles_c;          // ceil(cols / 64)
+    int cap;                  // runs cached in shared memory per CTA
+    uint32_t* ctl;
+    DevError* err;
+    uint64_t limit_ns;
 };
 
-__global__ void __launch_bounds__(kThreads) encode_kernel(EncodeArgs a) {
-    const int t = blockIdx.y;
-    __shared__ float s_a32;
-    if (threadIdx.x < 32) {
-        float a32;
-        if (a.given) {
-            a32 = *a.gscale[t];
-        } else {
-            float m = 0.0f;
-            for (int i = threadIdx.x; i < a.nparts; i += 32) m = fmaxf(m, a.partials[t * kMaxPartials + i]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-            a32 = __fdiv_rn(m, 2688.0f);  // a32 = amax / (6 * 448)
-            if (blockIdx.x == 0 && threadIdx.x == 0) *a.gscale[t] = a32;
-        }
-        if (threadIdx.x == 0) s_a32 = a32;
+// max of |bf16| over 8 values, on the bit patterns (two 16-bit lanes per
+// 32-bit SIMD max; exact for finite values)
+__device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
+    const uint32_t m = 0x7FFF7FFFu;
+    const uint32_t a = __vmaxu2(v.x & m, v.y & m);
+    const uint32_t b = __vmaxu2(v.z & m, v.w & m);
+    return __vmaxu2(a, b);
+}
+
+struct Run {
+    int t;            // tensor
+    int64_t r, c0;    // row, first column
+    int nchunks;      // valid 16-byte chunks (L / 8)
+};
+
+__device__ __forceinline__ Run run_of(const QuantArgs& a, int64_t g) {
+    Run u;
+    u.t = g >= a.runs_per_tensor ? 1 : 0;
+    const int64_t gl = g - (u.t ? a.runs_per_tensor : 0);
+    u.r = gl / a.upr;
+    u.c0 = (gl - u.r * a.upr) * 512;
+    u.nchunks = (int)(min((int64_t)512, a.cols - u.c0) / 8);
+    return u;
+}
+
+__device__ __forceinline__ const uint8_t* run_src(const QuantArgs& a, const Run& u) {
+    return (u.t ? a.x[1] : a.x[0]) + (u.r * a.ld + u.c0) * 2;
+}
+
+__global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
+    extern __shared__ __align__(128) uint8_t qsmem[];
+    uint4* cache = reinterpret_cast<uint4*>(qsmem);  // [cap][64]
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ uint32_t s_red[2][kQWarps];
+    __shared__ float s_alpha[2];
+    __shared__ int s_ok;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t G = gridDim.x;
+    const int64_t begin = a.total_runs * (int64_t)blockIdx.x / G;
+    const int64_t end = a.total_runs * ((int64_t)blockIdx.x + 1) / G;
+    const int64_t ncached = min(end - begin, (int64_t)a.cap);
+
+    // ---- phase 1: bulk-copy this CTA's runs into shared memory
+    if (threadIdx.x == 0) {
+        mbar_init(&s_bar, 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        s_ok = 1;
     }
     __syncthreads();
-    const float a32 = s_a32;
+    {
+        // every thread announces its own bytes, then issues its copies; the
+        // single arrival comes after all announcements (the __syncthreads)
+        uint32_t mine = 0;
+        for (int64_t l = threadIdx.x; l < ncached; l += kQThreads) mine += (uint32_t)run_of(a, begin + l).nchunks * 16u;
+        if (mine) mbar_expect_tx_only(&s_bar, mine);
+        for (int64_t l = threadIdx.x; l < ncached; l += kQThreads) {
+            const Run u = run_of(a, begin + l);
+            bulk_load(cache + l * 64, run_src(a, u), (uint32_t)u.nchunks * 16u, &s_bar);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_arrive(&s_bar);
+    if (ncached > 0) {
+        volatile int never = 0;
+        if (!mbar_wait_bounded(&s_bar, 0, &never, a.limit_ns)) {
+            record_error(a.err, NVFP4_ERR_TIMEOUT, 1);
+            s_ok = 0;  // the copies may still land: wait for them once more below
+        }
+    }
+    __syncthreads();
+    if (!s_ok) {
+        if (threadIdx.x == 0) {
+            volatile int never = 0;
+            mbar_wait_bounded(&s_bar, 0, &never, a.limit_ns);
+        }
+        return;
+    }
 
-    const int lane = threadIdx.x & 31;
-    const int64_t upr = (a.cols + 511) / 512;  // 512-element runs per row
-    const int64_t units = a.rows * upr;
-    const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
-    const uint8_t* xb = a.x[t];
-    uint8_t* cb = a.codes[t];
-    uint8_t* sb = a.scales[t];
+    if (!a.given) {
+        uint32_t m0 = 0, m1 = 0;
+        for (int64_t g = begin + warp; g < end; g += kQWarps) {
+            const Run u = run_of(a, g);
+            const int64_t l = g - begin;
+            const bool v0 = lane < u.nchunks, v1 = lane + 32 < u.nchunks;
+            uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
+            if (l < ncached) {
+                if (v0) q0 = cache[l * 64 + lane];
+                if (v1) q1 = cache[l * 64 + 32 + lane];
+            } else {
+                const uint8_t* src = run_src(a, u);
+                if (v0) q0 = ld_stream16(src + lane * 16);
+                if (v1) q1 = ld_stream16(src + (lane + 32) * 16);
+            }
+            const uint32_t mm = __vmaxu2(absmax_bits8(q0), absmax_bits8(q1));
+            if (u.t) m1 = __vmaxu2(m1, mm);
+            else m0 = __vmaxu2(m0, mm);
+        }
+        m0 = max(m0 & 0xFFFFu, m0 >> 16);
+        m1 = max(m1 & 0xFFFFu, m1 >> 16);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            m0 = max(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
+            m1 = max(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
+        }
+        if (lane == 0) {
+            s_red[0][warp] = m0;
+            s_red[1][warp] = m1;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t c0 = 0, c1 = 0;
+            for (int w = 0; w < kQWarps; w++) {
+                c0 = max(c0, s_red[0][w]);
+                c1 = max(c1, s_red[1][w]);
+            }
+            volatile uint32_t* vctl = a.ctl;
+            const uint32_t gen = vctl[kCtlGen];
+            atomicMax(&a.ctl[kCtlAmax + 0], c0);
+            atomicMax(&a.ctl[kCtlAmax + 1], c1);
+            __threadfence();
+            const uint32_t arrived = atomicAdd(&a.ctl[kCtlCount], 1u);
+            if (arrived == (uint32_t)G - 1) {
+                // last CTA: finish the tensor maxima and release the grid
+                __threadfence();
+                for (int t = 0; t < 2; t++) {
+                    const uint32_t bits = atomicExch(&a.ctl[kCtlAmax + t], 0u);
+                    const float a32 = __fdiv_rn(__uint_as_float(bits << 16), 2688.0f);  // amax / (6 * 448)
+                    vctl[kCtlAlpha + t] = __float_as_uint(a32);
+                    if (t < (a.total_runs > a.runs_per_tensor ? 2 : 1)) *(t ? a.gscale[1] : a.gscale[0]) = a32;
+                }
+                vctl[kCtlCount] = 0;
+                __threadfence();
+                atomicAdd(&a.ctl[kCtlGen], 1u);
+            } else {
+                const uint64_t t0 = global_ns();
+                uint32_t it = 0;
+                while (vctl[kCtlGen] == gen) {
+                    if ((++it & 255u) == 0 && global_ns() - t0 > a.limit_ns) {
+                        record_error(a.err, NVFP4_ERR_TIMEOUT, 2);
+                        s_ok = 0;
+                        break;
+                    }
+                }
+                __threadfence();
+            }
+            s_alpha[0] = __uint_as_float(vctl[kCtlAlpha + 0]);
+            s_alpha[1] = __uint_as_float(vctl[kCtlAlpha + 1]);
+        }
+        __syncthreads();
+        if (!s_ok) return;
+    } else {
+        if (threadIdx.x < 2) s_alpha[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
+        __syncthreads();
+    }
+
+    // ---- phase 2: encode
     const int64_t sc_row = a.cols / 16;
-
-    for (int64_t unit = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); unit < units;
-         unit += nwarps) {
-        const int64_t r = unit / upr;
-        const int64_t c0 = (unit - r * upr) * 512;
-        const int64_t L = min((int64_t)512, a.cols - c0);
-        const int nchunks = (int)(L / 8);
-        const bool v0 = lane < nchunks, v1 = lane + 32 < nchunks;
-        const uint8_t* row = xb + (r * a.ld + c0) * 2;
+    for (int64_t g = begin + warp; g < end; g += kQWarps) {
+        const Run u = run_of(a, g);
+        const int64_t l = g - begin;
+        const bool v0 = lane < u.nchunks, v1 = lane + 32 < u.nchunks;
         uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-        if (v0) q0 = ld_stream16(row + lane * 16);
-        if (v1) q1 = ld_stream16(row + (lane + 32) * 16);
+        if (l < ncached) {
+            if (v0) q0 = cache[l * 64 + lane];
+            if (v1) q1 = cache[l * 64 + 32 + lane];
+        } else {
+            const uint8_t* src = run_src(a, u);
+            if (v0) q0 = ld_stream16(src + lane * 16);
+            if (v1) q1 = ld_stream16(src + (lane + 32) * 16);
+        }
+        const float a32 = s_alpha[u.t];
         float f0[8], f1[8];
         bf16x8_to_f32(q0, f0);
         bf16x8_to_f32(q1, f1);
@@ -144,32 +249,36 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeArgs a) {
         const BlockScale b1 = block_scale(am1, a32);
         const uint32_t w0 = encode8(f0, b0.inv);
         const uint32_t w1 = encode8(f1, b1.inv);
-        uint8_t* crow = cb + r * (a.cols / 2) + c0 / 2;
+        uint8_t* crow = (u.t ? a.codes[1] : a.codes[0]) + u.r * (a.cols / 2) + u.c0 / 2;
         if (v0) *reinterpret_cast<uint32_t*>(crow + 4 * lane) = w0;
         if (v1) *reinterpret_cast<uint32_t*>(crow + 128 + 4 * lane) = w1;
-        // even lanes store the scale of their first-half block, odd lanes the
-        // scale of their second-half block
+        // even lanes store the scale of their first-half block, odd lanes
+        // the scale of their second-half block
         const bool odd = lane & 1;
-        const bool vs = odd ? v1 : v0;
-        if (vs) {
-            const int64_t bj = c0 / 16 + (odd ? 16 : 0) + (lane >> 1);
+        if (odd ? v1 : v0) {
+            const int64_t bj = u.c0 / 16 + (odd ? 16 : 0) + (lane >> 1);
             const uint8_t code = (uint8_t)(odd ? b1.code : b0.code);
+            uint8_t* sb = u.t ? a.scales[1] : a.scales[0];
             if (a.swizzled)
-                sb[swz_offset(r, bj, a.tiles_c)] = code;
+                sb[swz_offset(u.r, bj, a.tiles_c)] = code;
             else
-                sb[r * sc_row + bj] = code;
+                sb[u.r * sc_row + bj] = code;
         }
     }
 
     // zero the padding rows of the swizzled scale tiles (cols % 64 == 0, so
-    // only rows past `rows` up to the next multiple of 128 are padding)
+    // only the rows past `rows` up to the next multiple of 128 are padding)
     if (a.swizzled) {
         const int64_t rows_pad = (a.rows + 127) / 128 * 128;
         const int64_t sc_pad = a.tiles_c * 4;
         const int64_t npad = (rows_pad - a.rows) * sc_pad;
-        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < npad; i += (int64_t)gridDim.x * kThreads) {
-            const int64_t r = a.rows + i / sc_pad, c = i % sc_pad;
-            sb[swz_offset(r, c, a.tiles_c)] = 0;
+        const int nt = a.total_runs > a.runs_per_tensor ? 2 : 1;
+        for (int t = 0; t < nt; t++) {
+            uint8_t* sb = t ? a.scales[1] : a.scales[0];
+            for (int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x; i < npad; i += G * kQThreads) {
+                const int64_t r = a.rows + i / sc_pad, c = i % sc_pad;
+                sb[swz_offset(r, c, a.tiles_c)] = 0;
+            }
         }
     }
 }
@@ -186,40 +295,76 @@ struct DequantArgs {
     DevError* err;
 };
 
+// 8 E2M1 codes (32 bits) with one block scale and the slot's a32 -> 8 bf16
+// (16 bytes): bf16_rne(fl32(fl32(e2m1 * s) * a32)); e2m1 * s is exact in
+// binary16, so the only roundings are the two the definition has.
+__device__ __forceinline__ uint4 dequant8(uint32_t q, uint8_t sc, float a32) {
+    const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const __half2 v = __hmul2(e2m1x2_to_half2((q >> (8 * j)) & 0xFFu), s2);  // exact
+        const float2 f = __half22float2(v);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(f.x, a32), __fmul_rn(f.y, a32));
+        o[j] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(DequantArgs a) {
     const int t = blockIdx.y;
     const int lane = threadIdx.x & 31;
-    const int64_t ups = (a.slot_elems + 255) / 256;  // 256-element runs per slot
+    const int64_t ups = (a.slot_elems + 511) / 512;  // 512-element runs per slot
     const int64_t units = (int64_t)a.n * ups;
     const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
-    const uint8_t* cb = a.codes[t];
-    const uint8_t* sb = a.scales[t];
-    uint8_t* ob = a.out[t];
-    for (int64_t unit = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); unit < units;
-         unit += nwarps) {
-        const int64_t i = unit / ups;
-        const int64_t u = unit - i * ups;
-        const int32_t s = __ldg(a.slots + i);
-        if (s < 0 || s >= a.n_slots) {
-            if (lane == 0 && u == 0 && t == 0) record_error(a.err, NVFP4_ERR_DEVICE, (uint32_t)i);
-            continue;
-        }
-        const int64_t e0 = u * 256 + 8 * lane;
-        if (e0 >= a.slot_elems) continue;
-        const int64_t sbase = (int64_t)s * a.slot_elems;
-        const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(cb + (sbase + e0) / 2));
-        const uint8_t sc = __ldg(sb + (sbase + e0) / 16);
-        const float a32 = __ldg(a.gscale[t] + s);
-        const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
-        uint32_t o[4];
+    const uint8_t* cb = t ? a.codes[1] : a.codes[0];
+    const uint8_t* sb = t ? a.scales[1] : a.scales[0];
+    const float* gb = t ? a.gscale[1] : a.gscale[0];
+    uint8_t* ob = t ? a.out[1] : a.out[0];
+    const int64_t w0 = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    for (int64_t base = w0; base < units; base += 2 * nwarps) {
+        // two runs per iteration: all loads first, then decode and store
+        uint32_t q[2][2];
+        uint8_t sc[2][2];
+        float a32[2];
+        bool ok[2][2];
+        int64_t obase[2], e0[2];
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const __half2 v = __hmul2(e2m1x2_to_half2((q >> (8 * j)) & 0xFFu), s2);  // exact
-            const float2 f = __half22float2(v);
-            const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(f.x, a32), __fmul_rn(f.y, a32));
-            o[j] = *reinterpret_cast<const uint32_t*>(&b);
+        for (int k = 0; k < 2; k++) {
+            const int64_t unit = base + k * nwarps;
+            ok[k][0] = ok[k][1] = false;
+            a32[k] = 0.0f;
+            obase[k] = e0[k] = 0;
+            q[k][0] = q[k][1] = 0;
+            sc[k][0] = sc[k][1] = 0;
+            if (unit >= units) continue;
+            const int64_t i = unit / ups;
+            const int64_t u = unit - i * ups;
+            const int32_t s = __ldg(a.slots + i);
+            if (s < 0 || s >= a.n_slots) {
+                if (lane == 0 && u == 0 && t == 0) record_error(a.err, NVFP4_ERR_DEVICE, (uint32_t)i);
+                continue;
+            }
+            const int64_t sbase = (int64_t)s * a.slot_elems;
+            e0[k] = u * 512 + 8 * lane;
+            obase[k] = (int64_t)i * a.slot_elems;
+            a32[k] = __ldg(gb + s);
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int64_t e = e0[k] + 256 * h;
+                ok[k][h] = e < a.slot_elems;
+                if (ok[k][h]) {
+                    q[k][h] = __ldg(reinterpret_cast<const uint32_t*>(cb + (sbase + e) / 2));
+                    sc[k][h] = __ldg(sb + (sbase + e) / 16);
+                }
+            }
         }
-        *reinterpret_cast<uint4*>(ob + ((int64_t)i * a.slot_elems + e0) * 2) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+        for (int k = 0; k < 2; k++)
+#pragma unroll
+            for (int h = 0; h < 2; h++)
+                if (ok[k][h])
+                    *reinterpret_cast<uint4*>(ob + (obase[k] + e0[k] + 256 * h) * 2) = dequant8(q[k][h], sc[k][h], a32[k]);
     }
 }
 
@@ -264,45 +409,64 @@ static nvfp4_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-// amax + encode over one or two tensors of the same shape
+static int g_q_dev = -1;
+static int g_q_smem = 0;
+
+// one fused, cooperative launch over one or two tensors of the same shape
 static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t rows, int64_t cols, int64_t ld,
                                   void* const* codes, void* const* scales, float* const* gscale, bool given,
                                   bool swizzled, void* workspace, cudaStream_t stream) {
-    const int sms = num_sms();
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    float* partials = reinterpret_cast<float*>(ws + kWsPartials);
-    int nparts = 0;
-    const int64_t chunks = rows * (cols / 8);
-    if (!given) {
-        AmaxArgs aa{};
-        for (int t = 0; t < ntensors; t++) aa.x[t] = static_cast<const uint8_t*>(x[t]);
-        aa.rows = rows;
-        aa.cols = cols;
-        aa.ld = ld;
-        aa.partials = partials;
-        nparts = grid_for(chunks, kThreads * 8, std::min(kMaxPartials, sms * 4));
-        amax_kernel<<<dim3(nparts, ntensors), kThreads, 0, stream>>>(aa);
-        if (launch_status() != NVFP4_OK) return NVFP4_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (g_q_dev != dev) {
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        // leave room for the kernel's static shared memory
+        const int smem = (optin - 2048) / kRunBytes * kRunBytes;
+        if (cudaFuncSetAttribute(quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        g_q_smem = smem;
+        g_q_dev = dev;
     }
-    EncodeArgs ea{};
+    QuantArgs a{};
     for (int t = 0; t < ntensors; t++) {
-        ea.x[t] = static_cast<const uint8_t*>(x[t]);
-        ea.codes[t] = static_cast<uint8_t*>(codes[t]);
-        ea.scales[t] = static_cast<uint8_t*>(scales[t]);
-        ea.gscale[t] = gscale[t];
+        a.x[t] = static_cast<const uint8_t*>(x[t]);
+        a.codes[t] = static_cast<uint8_t*>(codes[t]);
+        a.scales[t] = static_cast<uint8_t*>(scales[t]);
+        a.gscale[t] = gscale[t];
     }
-    ea.rows = rows;
-    ea.cols = cols;
-    ea.ld = ld;
-    ea.partials = partials;
-    ea.nparts = nparts;
-    ea.given = given ? 1 : 0;
-    ea.swizzled = swizzled ? 1 : 0;
-    ea.tiles_c = (cols + 63) / 64;
-    const int64_t units = rows * ((cols + 511) / 512);
-    const int g = grid_for(units, kThreads / 32, sms * 8);
-    encode_kernel<<<dim3(g, ntensors), kThreads, 0, stream>>>(ea);
-    return launch_status();
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.upr = (cols + 511) / 512;
+    a.runs_per_tensor = rows * a.upr;
+    a.total_runs = a.runs_per_tensor * ntensors;
+    a.given = given ? 1 : 0;
+    a.swizzled = swizzled ? 1 : 0;
+    a.tiles_c = (cols + 63) / 64;
+    a.ctl = static_cast<uint32_t*>(workspace);
+    a.err = static_cast<DevError*>(workspace);
+    a.limit_ns = 2000000000ull;
+    const int G = (int)std::min<int64_t>(num_sms(), a.total_runs);
+    const int64_t per_cta = (a.total_runs + G - 1) / G;
+    a.cap = (int)std::min<int64_t>(per_cta, g_q_smem / kRunBytes);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kQThreads);
+    cfg.dynamicSmemBytes = (size_t)a.cap * kRunBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, quantize_fused_kernel, a) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+    }
+    return NVFP4_OK;
 }
 
 }  // namespace nvfp4
@@ -393,8 +557,8 @@ extern "C" nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int3
     a.n_slots = cache->n_slots;
     a.slot_elems = (int64_t)cache->tokens_per_slot * cache->heads * cache->head_dim;
     a.err = static_cast<DevError*>(workspace);
-    const int64_t units = (int64_t)n * ((a.slot_elems + 255) / 256);
-    const int g = grid_for(units, kThreads / 32, num_sms() * 8);
+    const int64_t units = (int64_t)n * ((a.slot_elems + 511) / 512);
+    const int g = grid_for(units, 2 * (kThreads / 32), num_sms() * 8);
     kv_dequant_kernel<<<dim3(g, 2), kThreads, 0, (cudaStream_t)stream>>>(a);
     return launch_status();
 }

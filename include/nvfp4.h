@@ -93,14 +93,17 @@ enum {
 };
 
 /* Workspace bytes the caller must pass to the call `op` (device memory,
- * 256-byte aligned).  Never 0: every call keeps its device error record in
- * the first 16 bytes, which must be zero before a workspace is first used
- * (nvfp4_read_device_error zeroes them again); the rest needs no
- * initialization.  A workspace may be shared by calls on one stream. */
+ * 256-byte aligned).  Never 0.  Its first 256 bytes are a control block (the
+ * device error record in bytes 0..15; for quantize and KV append also the
+ * grid-barrier words and tensor maxima of the fused kernel): they must be
+ * zero before a workspace is first used, and the calls leave them ready for
+ * the next call.  A workspace may be reused by calls that are ordered on one
+ * stream; calls that can run concurrently need their own workspaces. */
 size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k);
 
 /* Synchronizes `stream`, then reads and clears the device error record of
- * `workspace` (written by the calls that used it).  *code receives
+ * `workspace` (written by the calls that used it); after an error the whole
+ * 256-byte control block is reset.  *code receives
  * NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_DEVICE; *info (may be NULL) a
  * call-specific detail (which wait ran out, the offending page-table index).
  * Returns NVFP4_ERR_CUDA if the synchronization or the copy fails. */
@@ -119,7 +122,10 @@ nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int
  * scales: nvfp4_scales_bytes(rows, cols, swizzled) bytes (padding zeroed).
  * global_scale: device binary32, written (COMPUTE) or read (GIVEN).
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols) bytes.
- * Two launches for COMPUTE (amax partials, then encode), one for GIVEN. */
+ * One cooperative launch (one CTA per SM): the input is read from HBM once
+ * (held in shared memory across a bounded grid barrier that turns the
+ * per-CTA maxima into a32) unless it exceeds ~#SMs x 200 KB, in which case
+ * the excess is read twice. */
 nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
                             void* scales, float* global_scale, unsigned flags, void* workspace,
                             size_t ws_bytes, nvfp4_stream_t stream);
@@ -201,7 +207,7 @@ typedef struct {
  * in place into slot `slot`: one tensor scale per (slot, K|V) = amax / 2688
  * over the whole chunk, then the quantize rule above with row-major scales.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_KV_APPEND, T*H, 0, d) bytes.
- * Two launches (amax partials of K and V, then encode of both). */
+ * One cooperative launch covering K and V (as nvfp4_quantize). */
 nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
                              const void* v_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 

@@ -1,10 +1,13 @@
 """GPU parity of nvfp4_gemm against the oracle's fp64 GEMM.
 
-Metric (reading R12): max_ij |C - ref| / max_ij |ref| <= 2e-3, where ref is the
-oracle's fp64 result on the same NVFP4 operands (the operands themselves are
-checked bit-exact by the quantize tests, and re-checked here).  The fused
-requant is checked bit-exact against the oracle's quantize applied to the
-kernel's own binary32 pre-quant values (reading R13).
+Metric (reading R12): max_ij |y - ref| / max_ij |ref| <= 2e-3, where y is the
+kernel's binary32 result (accumulation and epilogue, before the output store;
+written to the debug output) and ref the oracle's fp64 result on the same
+NVFP4 operands (the operands are checked bit-exact here too).  The bf16
+output is then checked bit for bit as the nearest-even bf16 of y, and the
+fused requant bit for bit as the oracle's quantize of y (reading R13).  The
+bf16 store alone can move a value by 2^-8 relative, so the 2e-3 bound is not
+applied to it.
 """
 import numpy as np
 import pytest
@@ -40,6 +43,26 @@ def _gemm_case(M, N, K, seed, **ep):
     return qa, oa, qb, ob
 
 
+def _run_checked(qa, qb, oa, ob, rows=None, out=None, **ep):
+    """Run nvfp4_gemm with the debug output, check y against the oracle at
+    GEMM_TOL and the bf16 output against bf16(y) exactly; return (c, y)."""
+    M, N = qa.rows, qb.rows
+    dy = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    dk = {k: (dev_bf16(v) if isinstance(v, np.ndarray) else v) for k, v in ep.items()}
+    c = nv.gemm(qa, qb, out=out, debug_y=dy, **dk)
+    torch.cuda.synchronize()
+    ref, _ = oracle.gemm(oa, ob, rows=rows, want_bf16=False, **ep)
+    y = dy.cpu().numpy()
+    ys = y if rows is None else y[rows]
+    err = normwise_err(ys.astype(np.float64), ref)
+    assert np.isfinite(ys).all()
+    assert err <= GEMM_TOL, err
+    cb = host_bits(c if out is None else out)
+    want = host_bits(dy.to(torch.bfloat16))
+    assert np.array_equal(cb, want), "bf16 output is not the nearest-even bf16 of y"
+    return c, y, err
+
+
 @pytest.mark.parametrize("M,N,K", [(64, 128, 256)])
 def test_tiny_workload(M, N, K):
     require_gpu()
@@ -47,12 +70,9 @@ def test_tiny_workload(M, N, K):
     b = syn.normal_bf16((N, K), seed=1)
     qa, oa = _qboth(a)
     qb, ob = _qboth(b)
-    c = nv.gemm(qa, qb)
-    y, _ = oracle.gemm(oa, ob, want_bf16=False)
-    got = bf16_to_f64(host_bits(c))
-    assert normwise_err(got, y) <= GEMM_TOL
+    c, y, _ = _run_checked(qa, qb, oa, ob)
     exact = bf16_to_f64(oracle.gemm_exact_bf16(oa, ob))
-    assert normwise_err(got, exact) <= GEMM_TOL
+    assert normwise_err(y.astype(np.float64), exact) <= GEMM_TOL
 
 
 def _lossless(rows, cols, seed):
@@ -76,7 +96,8 @@ def test_lossless_operands_give_textbook_matmul(M, N, K):
     qb, _ = _qboth(syn.f32_to_bf16_bits(b.astype(np.float32)), alpha)
     y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     nv.gemm(qa, qb, debug_y=y)
-    ref = (a @ b.T) * float(alpha) * float(alpha)
+    # s * a32 = 2^e exactly, so a32_A a32_B (A_q S_A)(B_q S_B)^T = A B^T
+    ref = a @ b.T
     got = y.cpu().numpy().astype(np.float64)
     assert np.max(np.abs(got - ref)) <= 1e-6 * np.max(np.abs(ref))
 
@@ -86,13 +107,9 @@ def test_qkv_full_size_sampled_rows():
     M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
     qa, oa, qb, ob = _gemm_case(M, N, K, seed=2)
     bias = syn.normal_bf16((N,), seed=4, std=0.02)
-    c = nv.gemm(qa, qb, bias=dev_bf16(bias))
     rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1],
                                      np.random.default_rng(5).integers(0, M, 59)]))
-    y, _ = oracle.gemm(oa, ob, bias=bias, rows=rows, want_bf16=False)
-    got = bf16_to_f64(host_bits(c)[rows])
-    assert np.isfinite(got).all()
-    assert normwise_err(got, y) <= GEMM_TOL
+    _run_checked(qa, qb, oa, ob, rows=rows, bias=bias)
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 8, 64), (100, 136, 320), (130, 264, 512), (300, 520, 192),
@@ -102,10 +119,7 @@ def test_ragged_shapes(M, N, K):
     qa, oa, qb, ob = _gemm_case(M, N, K, seed=M + N + K)
     ldc = (N + 7) // 8 * 8 + 8
     buf = torch.full((M, ldc), float("nan"), dtype=torch.bfloat16, device="cuda")
-    c = nv.gemm(qa, qb, out=buf[:, :N])
-    y, _ = oracle.gemm(oa, ob, want_bf16=False)
-    got = bf16_to_f64(host_bits(buf[:, :N]))
-    assert normwise_err(got, y) <= GEMM_TOL
+    _run_checked(qa, qb, oa, ob, out=buf[:, :N])
     assert torch.isnan(buf[:, N:]).all()  # nothing written past N
 
 
@@ -121,10 +135,7 @@ def test_epilogue_bias_gelu_modulate_gate_residual():
     for kw in (dict(bias=bias, act=nv.ACT_GELU_TANH), dict(mod_scale=ms, mod_shift=sh),
                dict(bias=bias, gate=gt, residual=res), dict(bias=bias, act=1, mod_scale=ms, mod_shift=sh,
                                                              gate=gt, residual=res)):
-        dk = {k: (dev_bf16(v) if isinstance(v, np.ndarray) else v) for k, v in kw.items()}
-        c = nv.gemm(qa, qb, **dk)
-        y, _ = oracle.gemm(oa, ob, want_bf16=False, **kw)
-        assert normwise_err(bf16_to_f64(host_bits(c)), y) <= GEMM_TOL, list(kw)
+        _run_checked(qa, qb, oa, ob, **kw)
 
 
 @pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 320, 512)])
@@ -142,7 +153,7 @@ def test_requant_epilogue_bit_exact_given_prequant_values(M, N, K):
     torch.cuda.synchronize()
     y = dy.cpu().numpy()
     assert normwise_err(y.astype(np.float64), y_ref) <= GEMM_TOL
-    assert normwise_err(bf16_to_f64(host_bits(c)), y_ref) <= GEMM_TOL
+    assert np.array_equal(host_bits(c), host_bits(dy.to(torch.bfloat16)))
     codes, scales, _ = oracle.quantize(np.ascontiguousarray(y), out_a32)
     assert np.array_equal(host_u8(rq.codes), codes)
     assert np.array_equal(host_u8(rq.scales), oracle.swizzle(scales))
@@ -170,11 +181,9 @@ def test_ffn_pair_up_requant_feeds_down():
     h = nv.empty_nvfp4(M, F)
     h.global_scale.copy_(amax / 2688.0)
     nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, requant=h, bf16_out=False)
-    out = nv.gemm(h, qd)
     torch.cuda.synchronize()
     oh = (host_u8(h.codes), oracle.unswizzle(host_u8(h.scales), M, F // 16), np.float32(h.global_scale.item()))
-    y, _ = oracle.gemm(oh, od, want_bf16=False)
-    assert normwise_err(bf16_to_f64(host_bits(out)), y) <= GEMM_TOL
+    _run_checked(h, qd, oh, od)
     # and the whole chain stays close to the fp64 chain of the oracle
     yu, _ = oracle.gemm(oa, ou, act=1, want_bf16=False)
     assert abs(float(amax.item()) - np.max(np.abs(yu))) <= 2e-3 * np.max(np.abs(yu))
@@ -187,8 +196,7 @@ def test_bounded_wait_records_timeout_and_context_survives():
     nv.gemm(qa, qb, debug_flags=nv.DBG_SKIP_LOADS, wait_limit_us=50000, ws=ws)
     code, info = nv.read_device_error(ws)
     assert code == nv.ERR_TIMEOUT and info in (2, 3, 4)
-    c = nv.gemm(qa, qb, ws=ws)
+    _run_checked(qa, qb, oa, ob)
+    nv.gemm(qa, qb, ws=ws)
     code, _ = nv.read_device_error(ws)
     assert code == nv.OK
-    y, _ = oracle.gemm(oa, ob, want_bf16=False)
-    assert normwise_err(bf16_to_f64(host_bits(c)), y) <= GEMM_TOL
