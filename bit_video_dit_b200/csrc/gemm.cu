@@ -171,45 +171,52 @@ drain:
 }
 
 // ---------------------------------------------------------------- MMA -------
+// One thread issues everything.  Descriptors are built once; a stage / k-block
+// step only adds to the 14-bit start-address field (shared memory addresses
+// are < 2^18, so the field never carries).  For each 64-wide k-block the scale
+// copies go out right before the MMA that reads them, so the tensor pipe can
+// start on k-block 0 while later copies are still queued.
 __device__ void mma_issuer(const Params& p, Smem* s, uint8_t* ring, uint32_t tmem) {
     volatile int* abort = &s->abort_flag;
+    const uint32_t ring_s = smem_u32(ring);
+    const uint64_t a_desc0 = smem_desc(ring_s, 16, 1024, kLayoutSw128);
+    const uint64_t b_desc0 = smem_desc(ring_s + A_BYTES, 16, 1024, kLayoutSw128);
+    const uint64_t sfa_desc0 = smem_desc(ring_s + A_BYTES + B_BYTES, 0, 128, kLayoutNone);
+    const uint64_t sfb_desc0 = smem_desc(ring_s + A_BYTES + B_BYTES + SFA_BYTES, 0, 128, kLayoutNone);
+    const uint32_t sfa_t = tmem + SFA_COL, sfb_t = tmem + SFB_COL;
     uint32_t it = 0;
     uint32_t tcount = 0;
     bool issued = false;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, tcount++) {
         int mb, nb;
         tile_coords(p, tile, mb, nb);
-        const int halves = ((int64_t)nb * BN + 128 < p.N) ? 2 : 1;
+        const bool two_halves = (int64_t)nb * BN + 128 < p.N;
         if (!mbar_wait_bounded(&s->tmem_empty, (tcount & 1) ^ 1, abort, p.limit_ns)) {
             if (!*abort) raise_abort(s, p, 2);
             goto drain;
         }
         tc_fence_after();
+        const uint32_t acc = tmem + ((tcount & 1) ? ACC1_COL : 0u);
         for (int kt = 0; kt < p.kt_count; kt++, it++) {
             const int st = it % STAGES;
-            const uint32_t round = it / STAGES;
-            if (!mbar_wait_bounded(&s->full[st], round & 1, abort, p.limit_ns)) {
+            if (!mbar_wait_bounded(&s->full[st], (it / STAGES) & 1, abort, p.limit_ns)) {
                 if (!*abort) raise_abort(s, p, 3);
                 goto drain;
             }
             tc_fence_after();
-            const uint32_t a_s = smem_u32(ring + st * STAGE_BYTES);
-            const uint32_t b_s = a_s + A_BYTES;
-            const uint32_t sfa_s = b_s + B_BYTES;
-            const uint32_t sfb_s = sfa_s + SFA_BYTES;
+            const uint64_t off = (uint64_t)((st * STAGE_BYTES) >> 4);
             const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
-            for (int kb = 0; kb < nkb; kb++) {
-                tc_cp_32x128b_x4(tmem + SFA_COL + 4 * kb, smem_desc(sfa_s + kb * 512, 0, 128, kLayoutNone));
-                for (int h = 0; h < halves; h++)
-                    tc_cp_32x128b_x4(tmem + SFB_COL + 8 * kb + 4 * h,
-                                     smem_desc(sfb_s + h * (KB_PER_STAGE * 512) + kb * 512, 0, 128, kLayoutNone));
-            }
-            const uint32_t acc = tmem + ((tcount & 1) ? ACC1_COL : 0u);
-            for (int kb = 0; kb < nkb; kb++) {
-                const uint64_t ad = smem_desc(a_s + kb * 32, 16, 1024, kLayoutSw128);
-                const uint64_t bd = smem_desc(b_s + kb * 32, 16, 1024, kLayoutSw128);
-                tc_mma_nvf4(acc, ad, bd, IDESC, tmem + SFA_COL + 4 * kb, tmem + SFB_COL + 8 * kb,
-                            (kt > 0 || kb > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kb = 0; kb < KB_PER_STAGE; kb++) {
+                if (kb < nkb) {
+                    tc_cp_32x128b_x4(sfa_t + 4 * kb, sfa_desc0 + off + kb * (512 >> 4));
+                    tc_cp_32x128b_x4(sfb_t + 8 * kb, sfb_desc0 + off + kb * (512 >> 4));
+                    if (two_halves)
+                        tc_cp_32x128b_x4(sfb_t + 8 * kb + 4,
+                                         sfb_desc0 + off + ((KB_PER_STAGE * 512) >> 4) + kb * (512 >> 4));
+                    tc_mma_nvf4(acc, a_desc0 + off + kb * (32 >> 4), b_desc0 + off + kb * (32 >> 4), IDESC,
+                                sfa_t + 4 * kb, sfb_t + 8 * kb, (kt > 0 || kb > 0) ? 1u : 0u);
+                }
             }
             issued = true;
             tc_commit(&s->empty[st]);
@@ -282,7 +289,7 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] = v[i] + y[i];
     }
-    if (row_ok) {
+    if (p.out_amax && row_ok) {
 #pragma unroll
         for (int i = 0; i < 32; i++)
             if (i < valid) amax_run = fmaxf(amax_run, fabsf(y[i]));

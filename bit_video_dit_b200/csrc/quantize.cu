@@ -219,7 +219,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
         __syncthreads();
         if (!s_ok) return;
     } else {
-        if (threadIdx.x < 2) s_alpha[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
+        const int nt = a.total_runs > a.runs_per_tensor ? 2 : 1;  // gscale[1] is NULL for one tensor
+        if (threadIdx.x < nt) s_alpha[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
         __syncthreads();
     }
 
