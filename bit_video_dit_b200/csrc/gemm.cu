@@ -12,11 +12,15 @@
 // fused adaLN kernels of the anzhuoshouzhuan.com article ("NVFP4 量化").
 //
 // Kernel design (B200):
-//  * persistent grid, one CTA per SM, static round-robin tile schedule over
-//    128 x 256 output tiles;
-//  * warp 0: TMA producer (A/B code tiles with 128B swizzle, scale tiles as
-//    plain bulk copies of the 512-byte scale-factor tiles); a 4-stage ring of
-//    K-slices of 256 elements (54 KB per stage);
+//  * persistent grid, one CTA per SM, static round-robin tile schedule.  Two
+//    variants of one template: a CTA pair (cluster of 2, tcgen05 cta_group::2)
+//    computing 256 x 256 tiles -- each CTA loads its 128 rows of A, its 128
+//    rows of B and all 256 rows of B's scales, the leader CTA issues the MMAs
+//    for both -- and a single-CTA 128 x 256 variant used when M <= 128;
+//  * warp 0: TMA producer (A/B code tiles with 128B swizzle, the 512-byte
+//    scale-factor tiles as 3-D boxes whose K tail the TMA zero-fills); a ring
+//    of K-slices of 256 elements (5 x 38 KB per CTA for the pair, 4 x 54 KB
+//    for one CTA);
 //  * warp 1: owns TMEM (512 columns: two overlapping 256-column accumulators
 //    and 48 scale columns) and issues, from one thread, tcgen05.cp of the
 //    scale tiles into TMEM and tcgen05.mma.kind::mxf4nvf4.block_scale (M=128,
@@ -35,20 +39,17 @@
 namespace nvfp4 {
 namespace gemm {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 256;        // K elements per stage
-constexpr int BKB = BK / 2;    // bytes per row per stage (128: one swizzle atom row)
+constexpr int BM = 128;  // rows of A per CTA
+constexpr int BN = 256;  // output columns per tile
+constexpr int BK = 256;  // K elements per stage
+constexpr int BKB = BK / 2;  // bytes per row per stage (128: one swizzle atom row)
 constexpr int KB_PER_STAGE = BK / 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BKB;            // 16 KB
-constexpr int B_BYTES = BN * BKB;            // 32 KB
-constexpr int SFA_BYTES = KB_PER_STAGE * 512;      // 2 KB
-constexpr int SFB_BYTES = 2 * KB_PER_STAGE * 512;  // 4 KB (two 128-row halves)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int A_BYTES = BM * BKB;                  // 16 KB
+constexpr int SFA_BYTES = KB_PER_STAGE * 512;      // 2 KB
+constexpr int SFB_BYTES = 2 * KB_PER_STAGE * 512;  // 4 KB (two 128-row halves of the tile's N)
+
 // Two accumulators of BN columns share TMEM with the 48 scale columns:
 // acc0 = [0, 256), acc1 = [192, 448), scales = [448, 496).  They overlap in
 // columns [192, 256); the epilogue drains those first (acc0: its chunks 6, 7;
@@ -59,26 +60,35 @@ constexpr uint32_t ACC1_COL = 192;
 constexpr uint32_t SFA_COL = ACC1_COL + BN;                        // 448
 constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;           // 464
 constexpr int OVERLAP_CHUNKS = (BN - (int)ACC1_COL) / 32;          // 2
-
-static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment for 128B swizzle");
 static_assert(SFA_COL + SF_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(ACC1_COL % 32 == 0 && OVERLAP_CHUNKS == 2, "overlap must be whole 32-column chunks");
 
 // instruction descriptor: E2M1 x E2M1, UE4M3 scales, f32 accumulate, K-major
-// A and B, M = 128, N = BN, K = 64 (dense).
+// A and B, M x N, K = 64 (dense).
 constexpr uint32_t make_idesc(int m, int n) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
-constexpr uint32_t IDESC = make_idesc(BM, BN);
+
+template <bool PAIR>
+struct Cfg {
+    static constexpr int CTAS = PAIR ? 2 : 1;
+    static constexpr int TILE_M = BM * CTAS;        // 256 or 128
+    static constexpr int B_ROWS = PAIR ? 128 : 256;  // rows of B each CTA loads
+    static constexpr int STAGES = PAIR ? 5 : 4;
+    static constexpr int B_BYTES = B_ROWS * BKB;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+    static constexpr uint32_t TX_BYTES = (uint32_t)(CTAS * STAGE_BYTES);  // per stage, both CTAs
+    static constexpr uint32_t IDESC = make_idesc(TILE_M, BN);
+    static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment for 128B swizzle");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
 
 struct Params {
     int M, N, K;
-    int tiles_m, tiles_n, num_tiles;
-    int kt_count;      // ceil(K / BK)
-    int kb_total;      // K / 64
-    int64_t sf_tiles_k;  // scale tiles per 128-row block along K (= K / 64)
-    const uint8_t* sfa;
-    const uint8_t* sfb;
+    int tiles_m, tiles_n, num_tiles;  // tiles_m counts TILE_M-row blocks
+    int kt_count;                     // ceil(K / BK)
+    int kb_total;                     // K / 64
     const float* ga;
     const float* gb;
     __nv_bfloat16* c;
@@ -100,6 +110,7 @@ struct Params {
     uint32_t dbg;
 };
 
+template <int STAGES>
 struct Smem {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
@@ -115,46 +126,76 @@ __device__ __forceinline__ void tile_coords(const Params& p, int tile, int& mb, 
     nb = tile / p.tiles_m;
 }
 
-__device__ __forceinline__ void raise_abort(Smem* s, const Params& p, uint32_t where) {
+template <class S>
+__device__ __forceinline__ void raise_abort(S* s, const Params& p, uint32_t where) {
     record_error(p.err, NVFP4_ERR_TIMEOUT, where);
     *(volatile int*)&s->abort_flag = 1;
 }
 
+// work unit of this CTA (pair: one per cluster) and the stride between them
+template <bool PAIR>
+__device__ __forceinline__ void tile_range(int& first, int& step) {
+    if (PAIR) {
+        first = blockIdx.x >> 1;
+        step = gridDim.x >> 1;
+    } else {
+        first = blockIdx.x;
+        step = gridDim.x;
+    }
+}
+
 // ---------------------------------------------------------------- producer --
-__device__ void producer(const Params& p, Smem* s, uint8_t* ring, const CUtensorMap* tma_a,
-                         const CUtensorMap* tma_b) {
+template <bool PAIR>
+__device__ void producer(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, const CUtensorMap* tma_a,
+                         const CUtensorMap* tma_b, const CUtensorMap* tma_sfa, const CUtensorMap* tma_sfb,
+                         uint32_t rank) {
+    using C = Cfg<PAIR>;
     prefetch_tmap(tma_a);
     prefetch_tmap(tma_b);
+    prefetch_tmap(tma_sfa);
+    prefetch_tmap(tma_sfb);
     volatile int* abort = &s->abort_flag;
     uint32_t issued_mask = 0, parity_mask = 0;  // per stage: a load was issued / its phase parity
     if (p.dbg & NVFP4_DBG_SKIP_LOADS) return;
+    int first, step;
+    tile_range<PAIR>(first, step);
     uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = first; tile < p.num_tiles; tile += step) {
         int mb, nb;
         tile_coords(p, tile, mb, nb);
-        const int halves = ((int64_t)nb * BN + 128 < p.N) ? 2 : 1;
+        const int a_row = mb * C::TILE_M + (int)rank * BM;
+        const int b_row = nb * BN + (int)rank * C::B_ROWS;
+        const int sfa_blk = mb * C::CTAS + (int)rank;
         for (int kt = 0; kt < p.kt_count; kt++, it++) {
-            const int st = it % STAGES;
-            const uint32_t round = it / STAGES;
+            const int st = it % C::STAGES;
+            const uint32_t round = it / C::STAGES;
             if (!mbar_wait_bounded(&s->empty[st], (round & 1) ^ 1, abort, p.limit_ns)) {
                 if (!*abort) raise_abort(s, p, 1);
                 goto drain;
             }
             {
-                uint8_t* a_s = ring + st * STAGE_BYTES;
+                uint8_t* a_s = ring + st * C::STAGE_BYTES;
                 uint8_t* b_s = a_s + A_BYTES;
-                uint8_t* sfa_s = b_s + B_BYTES;
+                uint8_t* sfa_s = b_s + C::B_BYTES;
                 uint8_t* sfb_s = sfa_s + SFA_BYTES;
-                const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
-                const uint32_t bytes = A_BYTES + B_BYTES + (uint32_t)nkb * 512u * (1u + halves);
-                mbar_expect_tx(&s->full[st], bytes);
-                tma_load_2d(a_s, tma_a, &s->full[st], kt * BKB, mb * BM);
-                tma_load_2d(b_s, tma_b, &s->full[st], kt * BKB, nb * BN);
-                const int64_t kt4 = (int64_t)kt * KB_PER_STAGE;
-                bulk_load(sfa_s, p.sfa + ((int64_t)mb * p.sf_tiles_k + kt4) * 512, nkb * 512, &s->full[st]);
-                for (int h = 0; h < halves; h++)
-                    bulk_load(sfb_s + h * (KB_PER_STAGE * 512),
-                              p.sfb + ((int64_t)(nb * 2 + h) * p.sf_tiles_k + kt4) * 512, nkb * 512, &s->full[st]);
+                const int kx = kt * BKB, ks = kt * KB_PER_STAGE;
+                if (PAIR) {
+                    // all transaction bytes of the pair are counted on the leader's barrier
+                    const uint32_t bar = mapa_shared(smem_u32(&s->full[st]), 0);
+                    if (rank == 0) mbar_expect_tx(&s->full[st], C::TX_BYTES);
+                    tma_load_2d_pair(a_s, tma_a, bar, kx, a_row);
+                    tma_load_2d_pair(b_s, tma_b, bar, kx, b_row);
+                    tma_load_3d_pair(sfa_s, tma_sfa, bar, 0, ks, sfa_blk);
+                    tma_load_3d_pair(sfb_s, tma_sfb, bar, 0, ks, nb * 2);
+                    tma_load_3d_pair(sfb_s + SFA_BYTES, tma_sfb, bar, 0, ks, nb * 2 + 1);
+                } else {
+                    mbar_expect_tx(&s->full[st], C::TX_BYTES);
+                    tma_load_2d(a_s, tma_a, &s->full[st], kx, a_row);
+                    tma_load_2d(b_s, tma_b, &s->full[st], kx, b_row);
+                    tma_load_3d(sfa_s, tma_sfa, &s->full[st], 0, ks, sfa_blk);
+                    tma_load_3d(sfb_s, tma_sfb, &s->full[st], 0, ks, nb * 2);
+                    tma_load_3d(sfb_s + SFA_BYTES, tma_sfb, &s->full[st], 0, ks, nb * 2 + 1);
+                }
                 issued_mask |= 1u << st;
                 parity_mask = (parity_mask & ~(1u << st)) | ((round & 1u) << st);
             }
@@ -163,34 +204,38 @@ __device__ void producer(const Params& p, Smem* s, uint8_t* ring, const CUtensor
     return;
 drain:
     // the only loads that can still be in flight are the last one per stage
-    for (int i = 0; i < STAGES; i++)
-        if (issued_mask & (1u << i)) {
-            volatile int never = 0;
-            mbar_wait_bounded(&s->full[i], (parity_mask >> i) & 1u, &never, p.limit_ns);
-        }
+    // (for the pair they are all counted on the leader's barriers)
+    if (!PAIR || rank == 0) {
+        for (int i = 0; i < C::STAGES; i++)
+            if (issued_mask & (1u << i)) {
+                volatile int never = 0;
+                mbar_wait_bounded(&s->full[i], (parity_mask >> i) & 1u, &never, p.limit_ns);
+            }
+    }
 }
 
 // ---------------------------------------------------------------- MMA -------
-// One thread issues everything.  Descriptors are built once; a stage / k-block
-// step only adds to the 14-bit start-address field (shared memory addresses
-// are < 2^18, so the field never carries).  For each 64-wide k-block the scale
-// copies go out right before the MMA that reads them, so the tensor pipe can
-// start on k-block 0 while later copies are still queued.
-__device__ void mma_issuer(const Params& p, Smem* s, uint8_t* ring, uint32_t tmem) {
+// One thread (of the leader CTA for the pair) issues everything.  Descriptors
+// are built once; a stage / k-block step only adds to the 14-bit start-address
+// field (shared memory addresses are < 2^18, so the field never carries).  For
+// each 64-wide k-block the scale copies go out right before the MMA that reads
+// them, so the tensor pipe can start on k-block 0 while later copies queue.
+template <bool PAIR>
+__device__ void mma_issuer(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, uint32_t tmem) {
+    using C = Cfg<PAIR>;
     volatile int* abort = &s->abort_flag;
     const uint32_t ring_s = smem_u32(ring);
     const uint64_t a_desc0 = smem_desc(ring_s, 16, 1024, kLayoutSw128);
     const uint64_t b_desc0 = smem_desc(ring_s + A_BYTES, 16, 1024, kLayoutSw128);
-    const uint64_t sfa_desc0 = smem_desc(ring_s + A_BYTES + B_BYTES, 0, 128, kLayoutNone);
-    const uint64_t sfb_desc0 = smem_desc(ring_s + A_BYTES + B_BYTES + SFA_BYTES, 0, 128, kLayoutNone);
+    const uint64_t sfa_desc0 = smem_desc(ring_s + A_BYTES + C::B_BYTES, 0, 128, kLayoutNone);
+    const uint64_t sfb_desc0 = smem_desc(ring_s + A_BYTES + C::B_BYTES + SFA_BYTES, 0, 128, kLayoutNone);
     const uint32_t sfa_t = tmem + SFA_COL, sfb_t = tmem + SFB_COL;
+    int first, step;
+    tile_range<PAIR>(first, step);
     uint32_t it = 0;
     uint32_t tcount = 0;
     bool issued = false;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, tcount++) {
-        int mb, nb;
-        tile_coords(p, tile, mb, nb);
-        const bool two_halves = (int64_t)nb * BN + 128 < p.N;
+    for (int tile = first; tile < p.num_tiles; tile += step, tcount++) {
         if (!mbar_wait_bounded(&s->tmem_empty, (tcount & 1) ^ 1, abort, p.limit_ns)) {
             if (!*abort) raise_abort(s, p, 2);
             goto drain;
@@ -198,36 +243,55 @@ __device__ void mma_issuer(const Params& p, Smem* s, uint8_t* ring, uint32_t tme
         tc_fence_after();
         const uint32_t acc = tmem + ((tcount & 1) ? ACC1_COL : 0u);
         for (int kt = 0; kt < p.kt_count; kt++, it++) {
-            const int st = it % STAGES;
-            if (!mbar_wait_bounded(&s->full[st], (it / STAGES) & 1, abort, p.limit_ns)) {
+            const int st = it % C::STAGES;
+            if (!mbar_wait_bounded(&s->full[st], (it / C::STAGES) & 1, abort, p.limit_ns)) {
                 if (!*abort) raise_abort(s, p, 3);
                 goto drain;
             }
             tc_fence_after();
-            const uint64_t off = (uint64_t)((st * STAGE_BYTES) >> 4);
+            const uint64_t off = (uint64_t)((st * C::STAGE_BYTES) >> 4);
             const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
 #pragma unroll
             for (int kb = 0; kb < KB_PER_STAGE; kb++) {
                 if (kb < nkb) {
-                    tc_cp_32x128b_x4(sfa_t + 4 * kb, sfa_desc0 + off + kb * (512 >> 4));
-                    tc_cp_32x128b_x4(sfb_t + 8 * kb, sfb_desc0 + off + kb * (512 >> 4));
-                    if (two_halves)
-                        tc_cp_32x128b_x4(sfb_t + 8 * kb + 4,
-                                         sfb_desc0 + off + ((KB_PER_STAGE * 512) >> 4) + kb * (512 >> 4));
-                    tc_mma_nvf4(acc, a_desc0 + off + kb * (32 >> 4), b_desc0 + off + kb * (32 >> 4), IDESC,
-                                sfa_t + 4 * kb, sfb_t + 8 * kb, (kt > 0 || kb > 0) ? 1u : 0u);
+                    const uint64_t sa = sfa_desc0 + off + kb * (512 >> 4);
+                    const uint64_t sb0 = sfb_desc0 + off + kb * (512 >> 4);
+                    const uint64_t sb1 = sb0 + (SFA_BYTES >> 4);
+                    const uint64_t ad = a_desc0 + off + kb * (32 >> 4);
+                    const uint64_t bd = b_desc0 + off + kb * (32 >> 4);
+                    const uint32_t acc_flag = (kt > 0 || kb > 0) ? 1u : 0u;
+                    if (PAIR) {
+                        tc_cp_32x128b_x4_pair(sfa_t + 4 * kb, sa);
+                        tc_cp_32x128b_x4_pair(sfb_t + 8 * kb, sb0);
+                        tc_cp_32x128b_x4_pair(sfb_t + 8 * kb + 4, sb1);
+                        tc_mma_nvf4_pair(acc, ad, bd, C::IDESC, sfa_t + 4 * kb, sfb_t + 8 * kb, acc_flag);
+                    } else {
+                        tc_cp_32x128b_x4(sfa_t + 4 * kb, sa);
+                        tc_cp_32x128b_x4(sfb_t + 8 * kb, sb0);
+                        tc_cp_32x128b_x4(sfb_t + 8 * kb + 4, sb1);
+                        tc_mma_nvf4(acc, ad, bd, C::IDESC, sfa_t + 4 * kb, sfb_t + 8 * kb, acc_flag);
+                    }
                 }
             }
             issued = true;
-            tc_commit(&s->empty[st]);
+            if (PAIR)
+                tc_commit_pair(&s->empty[st], 0x3);
+            else
+                tc_commit(&s->empty[st]);
         }
-        tc_commit(&s->tmem_full);
+        if (PAIR)
+            tc_commit_pair(&s->tmem_full, 0x3);
+        else
+            tc_commit(&s->tmem_full);
     }
     return;
 drain:
     if (issued) {
         // wait until every tcgen05 op issued so far has finished
-        tc_commit(&s->drain);
+        if (PAIR)
+            tc_commit_pair(&s->drain, 0x1);
+        else
+            tc_commit(&s->drain);
         volatile int never = 0;
         mbar_wait_bounded(&s->drain, 0, &never, p.limit_ns);
     }
@@ -336,21 +400,29 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
             *reinterpret_cast<uint4*>(p.out_codes + m * (p.N / 2) + n0 / 2) = w;
             sc2 = (uint16_t)(b0.code | (b1.code << 8));
         }
-        // rows past M inside the last 128-row tile are scale padding: zero
-        *reinterpret_cast<uint16_t*>(p.out_scales + swz_offset(m, bj, tiles_on)) = sc2;
+        // rows past M up to the next multiple of 128 are scale padding: zero
+        // (a 256-row pair tile can reach past that; those rows have no scales)
+        if (m < ((int64_t)p.M + 127) / 128 * 128)
+            *reinterpret_cast<uint16_t*>(p.out_scales + swz_offset(m, bj, tiles_on)) = sc2;
     }
 }
 
-__device__ void epilogue(const Params& p, Smem* s, uint32_t tmem, int warp, int lane) {
+template <bool PAIR>
+__device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t tmem, int warp, int lane, uint32_t rank) {
+    using C = Cfg<PAIR>;
     volatile int* abort = &s->abort_flag;
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
     const float oa32 = p.out_codes ? __ldg(p.out_gscale) : 0.0f;
     const int64_t tiles_on = (p.N + 63) / 64;  // scale tiles along N of the output
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    // the leader's MMA waits for the epilogue warps of both CTAs
+    const uint32_t empty_bar = PAIR ? mapa_shared(smem_u32(&s->tmem_empty), 0) : smem_u32(&s->tmem_empty);
+    int first, step;
+    tile_range<PAIR>(first, step);
     float amax_run = 0.0f;
     uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, tcount++) {
+    for (int tile = first; tile < p.num_tiles; tile += step, tcount++) {
         int mb, nb;
         tile_coords(p, tile, mb, nb);
         if (!mbar_wait_bounded(&s->tmem_full, tcount & 1, abort, p.limit_ns)) {
@@ -358,23 +430,23 @@ __device__ void epilogue(const Params& p, Smem* s, uint32_t tmem, int warp, int 
             return;
         }
         tc_fence_after();
-        const int64_t m = (int64_t)mb * BM + q * 32 + lane;
+        const int64_t m = (int64_t)mb * C::TILE_M + (int64_t)rank * BM + q * 32 + lane;
         const bool row_ok = m < p.M;
         const int ncols = min(BN, p.N - nb * BN);
         const int nchunks = (ncols + 31) / 32;
         const bool buf1 = tcount & 1;
         const uint32_t acc = lane_base + (buf1 ? ACC1_COL : 0u);
         // chunks of this buffer that the other buffer overlaps come first
-        const int first = buf1 ? 0 : (BN / 32 - OVERLAP_CHUNKS);
-        int n_overlap = buf1 ? min(nchunks, OVERLAP_CHUNKS) : max(0, nchunks - first);
+        const int first_ov = buf1 ? 0 : (BN / 32 - OVERLAP_CHUNKS);
+        const int n_overlap = buf1 ? min(nchunks, OVERLAP_CHUNKS) : max(0, nchunks - first_ov);
         if (n_overlap == 0) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s->tmem_empty);
+            if (lane == 0) mbar_arrive_cluster(empty_bar);
         }
         for (int i = 0; i < nchunks; i++) {
             // buffer 0 visits chunks 6, 7, 0, 1, ..., 5; buffer 1 visits 0..7
-            const int j = buf1 ? i : ((i < n_overlap) ? first + i : i - n_overlap);
+            const int j = buf1 ? i : ((i < n_overlap) ? first_ov + i : i - n_overlap);
             uint32_t r[32];
             tmem_ld_32cols(acc + j * 32, r);
             tmem_ld_wait();
@@ -382,7 +454,7 @@ __device__ void epilogue(const Params& p, Smem* s, uint32_t tmem, int warp, int 
                 // the overlapped columns are in registers: next tile may start
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s->tmem_empty);
+                if (lane == 0) mbar_arrive_cluster(empty_bar);
             }
             const int64_t n0 = (int64_t)nb * BN + j * 32;
             const int valid = (int)min((int64_t)32, p.N - n0);
@@ -396,50 +468,68 @@ __device__ void epilogue(const Params& p, Smem* s, uint32_t tmem, int warp, int 
     }
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
                 const __grid_constant__ Params p) {
+    using C = Cfg<PAIR>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Smem* s = reinterpret_cast<Smem*>(ring + STAGES * STAGE_BYTES);
+    Smem<C::STAGES>* s = reinterpret_cast<Smem<C::STAGES>*>(ring + C::STAGES * C::STAGE_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; i++) {
+        for (int i = 0; i < C::STAGES; i++) {
             mbar_init(&s->full[i], 1);
             mbar_init(&s->empty[i], 1);
         }
         mbar_init(&s->tmem_full, 1);
-        mbar_init(&s->tmem_empty, 4);
+        mbar_init(&s->tmem_empty, 4 * C::CTAS);
         mbar_init(&s->drain, 1);
         s->abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
     if (warp == 1) {
-        tmem_alloc(&s->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(&s->tmem_base, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&s->tmem_base, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync_all();  // peer barriers initialized before any remote arrive / multicast
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s->tmem_base;
 
     if (warp == 0) {
-        if (lane == 0) producer(p, s, ring, &tma_a, &tma_b);
+        if (lane == 0) producer<PAIR>(p, s, ring, &tma_a, &tma_b, &tma_sfa, &tma_sfb, rank);
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(p, s, ring, tmem);
+        if (lane == 0 && rank == 0) mma_issuer<PAIR>(p, s, ring, tmem);
         __syncwarp();
     } else {
-        epilogue(p, s, tmem, warp, lane);
+        epilogue<PAIR>(p, s, tmem, warp, lane, rank);
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR)
+        cluster_sync_all();  // neither CTA leaves while the pair's MMAs may touch it
+    else
+        __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        if (PAIR)
+            tmem_dealloc_pair(tmem, TMEM_COLS);
+        else
+            tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -453,10 +543,11 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn g_encode_tiled = nullptr;
+static int g_gemm_dev = -1;
 static int g_gemm_sms = 0;
-static int g_gemm_attr_dev = -1;
+static int g_gemm_pair_clusters = 0;
 
-static nvfp4_status gemm_setup(int& sms) {
+static nvfp4_status gemm_setup(int& sms, int& pair_clusters) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (g_encode_tiled == nullptr) {
@@ -467,22 +558,44 @@ static nvfp4_status gemm_setup(int& sms) {
             return NVFP4_ERR_CUDA;
         g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
     }
-    if (g_gemm_attr_dev != dev) {
+    if (g_gemm_dev != dev) {
         int major = 0, minor = 0, n = 0;
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
         if (major != 10 || minor != 0) return NVFP4_ERR_UNSUPPORTED;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NVFP4_ERR_CUDA;
-        if (cudaFuncSetAttribute(gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(gemm::gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::Cfg<false>::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm::gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::Cfg<true>::SMEM_BYTES) != cudaSuccess)
             return NVFP4_ERR_CUDA;
+        // how many CTA pairs can be resident at once (bounds the persistent grid)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (n / 2));
+        cfg.blockDim = dim3(gemm::THREADS);
+        cfg.dynamicSmemBytes = gemm::Cfg<true>::SMEM_BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm::gemm_kernel<true>, &cfg) != cudaSuccess || clusters < 1) {
+            cudaGetLastError();
+            clusters = 0;  // pair variant unavailable: single-CTA tiles only
+        }
         g_gemm_sms = n;
-        g_gemm_attr_dev = dev;
+        g_gemm_pair_clusters = clusters;
+        g_gemm_dev = dev;
     }
     sms = g_gemm_sms;
+    pair_clusters = g_gemm_pair_clusters;
     return NVFP4_OK;
 }
 
+// packed E2M1 codes [rows x K/2] bytes, 128-byte (256-element) boxes of box_rows rows
 static bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t K, int box_rows) {
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
@@ -490,6 +603,20 @@ static bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// swizzled scales viewed as [row blocks][K/64 tiles][128 x u32]; a box is the
+// 4 tiles (2 KB) of one stage of one 128-row block.  Tiles past K/64 read as 0.
+static bool make_scale_map(CUtensorMap* map, const void* scales, int64_t rows, int64_t K) {
+    const int64_t tiles_k = K / 64, blocks = (rows + 127) / 128;
+    cuuint64_t dims[3] = {128, (cuuint64_t)tiles_k, (cuuint64_t)blocks};
+    cuuint64_t strides[2] = {512, (cuuint64_t)(tiles_k * 512)};
+    cuuint32_t box[3] = {128, (cuuint32_t)gemm::KB_PER_STAGE, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(scales), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -532,26 +659,28 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
         if (ep->out_amax && (reinterpret_cast<uintptr_t>(ep->out_amax) & 3u)) return NVFP4_ERR_MISALIGNED;
         if (ep->debug_y && (reinterpret_cast<uintptr_t>(ep->debug_y) & 3u)) return NVFP4_ERR_MISALIGNED;
     }
-    int sms = 0;
-    nvfp4_status st = gemm_setup(sms);
+    int sms = 0, pair_clusters = 0;
+    nvfp4_status st = gemm_setup(sms, pair_clusters);
     if (st != NVFP4_OK) return st;
+    // CTA pairs (256-row tiles) whenever there is more than one 128-row block
+    const bool pair = M > gemm::BM && pair_clusters > 0;
 
-    CUtensorMap ma, mb;
-    if (!make_code_map(&ma, A->codes, M, K, gemm::BM) || !make_code_map(&mb, B->codes, N, K, gemm::BN))
+    CUtensorMap ma, mb, msa, msb;
+    if (!make_code_map(&ma, A->codes, M, K, gemm::BM) ||
+        !make_code_map(&mb, B->codes, N, K, pair ? gemm::Cfg<true>::B_ROWS : gemm::Cfg<false>::B_ROWS) ||
+        !make_scale_map(&msa, A->scales, M, K) || !make_scale_map(&msb, B->scales, N, K))
         return NVFP4_ERR_CUDA;
 
     gemm::Params p{};
     p.M = (int)M;
     p.N = (int)N;
     p.K = (int)K;
-    p.tiles_m = (int)((M + gemm::BM - 1) / gemm::BM);
+    const int tile_m = pair ? gemm::Cfg<true>::TILE_M : gemm::Cfg<false>::TILE_M;
+    p.tiles_m = (int)((M + tile_m - 1) / tile_m);
     p.tiles_n = (int)((N + gemm::BN - 1) / gemm::BN);
     p.num_tiles = p.tiles_m * p.tiles_n;
     p.kt_count = (int)((K + gemm::BK - 1) / gemm::BK);
     p.kb_total = (int)(K / 64);
-    p.sf_tiles_k = K / 64;
-    p.sfa = static_cast<const uint8_t*>(A->scales);
-    p.sfb = static_cast<const uint8_t*>(B->scales);
     p.ga = A->global_scale;
     p.gb = B->global_scale;
     p.c = static_cast<__nv_bfloat16*>(c_bf16);
@@ -575,7 +704,27 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
         p.limit_ns = 2000000000ull;
     }
     p.err = static_cast<DevError*>(workspace);
+    if (pair) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * std::min(p.num_tiles, pair_clusters));
+        cfg.blockDim = dim3(gemm::THREADS);
+        cfg.dynamicSmemBytes = gemm::Cfg<true>::SMEM_BYTES;
+        cfg.stream = (cudaStream_t)stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, gemm::gemm_kernel<true>, ma, mb, msa, msb, p) != cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_CUDA;
+        }
+        return NVFP4_OK;
+    }
     const int grid = std::min(p.num_tiles, sms);
-    gemm::gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, (cudaStream_t)stream>>>(ma, mb, p);
+    gemm::gemm_kernel<false><<<grid, gemm::THREADS, gemm::Cfg<false>::SMEM_BYTES, (cudaStream_t)stream>>>(ma, mb, msa,
+                                                                                                         msb, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
