@@ -213,18 +213,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended in hardware (not
+// spinning, so it takes no issue slots from the warps doing the work) for up
+// to `suspend_ns` nanoseconds or until the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on phase `parity` of `bar`.  Gives up (returns false) when
-// *abort becomes non-zero or after limit_ns nanoseconds.
+// *abort becomes non-zero or after limit_ns nanoseconds.  Between checks the
+// thread sleeps in hardware for at most 200 us (it wakes as soon as the phase
+// completes), so waiting warps do not compete with the working ones.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                   uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    for (uint32_t i = 1;; i++) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*abort) return false;
-            if (global_ns() - t0 > limit_ns) return false;
-        }
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
 }
 

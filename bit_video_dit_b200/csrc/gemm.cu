@@ -22,9 +22,11 @@
 //    of K-slices of 256 elements (5 x 38 KB per CTA for the pair, 4 x 54 KB
 //    for one CTA);
 //  * warp 1: owns TMEM (512 columns: two overlapping 256-column accumulators
-//    and 48 scale columns) and issues, from one thread, tcgen05.cp of the
-//    scale tiles into TMEM and tcgen05.mma.kind::mxf4nvf4.block_scale (M=128,
+//    and two 48-column scale buffers) and issues, from one thread,
+//    tcgen05.mma.kind::mxf4nvf4.block_scale (M=128 or 256 for the pair,
 //    N=256, K=64), releasing each stage with tcgen05.commit;
+//  * warps 6..8: tcgen05.cp of the stage's scale tiles into the free TMEM
+//    scale buffer, a stage ahead of the MMAs;
 //  * warps 2..5: epilogue, tcgen05.ld of 32 columns at a time, binary32 math,
 //    16-byte stores (and the NVFP4 requant with the same encoder as the
 //    quantize kernel); it drains the columns both accumulators share first,
@@ -44,24 +46,27 @@ constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 256;  // K elements per stage
 constexpr int BKB = BK / 2;  // bytes per row per stage (128: one swizzle atom row)
 constexpr int KB_PER_STAGE = BK / 64;
-constexpr int THREADS = 192;
+constexpr int THREADS = 288;  // producer, MMA, 4 epilogue warps, 3 scale-copy warps
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int A_BYTES = BM * BKB;                  // 16 KB
 constexpr int SFA_BYTES = KB_PER_STAGE * 512;      // 2 KB
 constexpr int SFB_BYTES = 2 * KB_PER_STAGE * 512;  // 4 KB (two 128-row halves of the tile's N)
 
-// Two accumulators of BN columns share TMEM with the 48 scale columns:
-// acc0 = [0, 256), acc1 = [192, 448), scales = [448, 496).  They overlap in
-// columns [192, 256); the epilogue drains those first (acc0: its chunks 6, 7;
-// acc1: its chunks 0, 1) and then lets the next tile's MMAs start, so the
-// rest of the epilogue overlaps the next mainloop.
-constexpr uint32_t SF_COLS = 4 * KB_PER_STAGE + 8 * KB_PER_STAGE;  // 48
-constexpr uint32_t ACC1_COL = 192;
-constexpr uint32_t SFA_COL = ACC1_COL + BN;                        // 448
-constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;           // 464
-constexpr int OVERLAP_CHUNKS = (BN - (int)ACC1_COL) / 32;          // 2
-static_assert(SFA_COL + SF_COLS <= TMEM_COLS, "TMEM budget");
-static_assert(ACC1_COL % 32 == 0 && OVERLAP_CHUNKS == 2, "overlap must be whole 32-column chunks");
+// Two accumulators of BN columns share TMEM with two 48-column scale buffers:
+// acc0 = [0, 256), acc1 = [160, 416), scales = [416, 512).  The accumulators
+// overlap in columns [160, 256); the epilogue drains those first (acc0: its
+// chunks 5..7, acc1: its chunks 0..2) and then lets the next tile's MMAs
+// start, so the rest of the epilogue overlaps the next mainloop.  The scale
+// buffers alternate by stage: the copy warps fill one while the MMAs read the
+// other.
+constexpr uint32_t SF_COLS = 4 * KB_PER_STAGE + 8 * KB_PER_STAGE;  // 48 per buffer
+constexpr uint32_t ACC1_COL = 160;
+constexpr uint32_t SFA_COL = ACC1_COL + BN;                        // 416 (+48: buffer 1)
+constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;           // 432 (+48: buffer 1)
+constexpr int OVERLAP_CHUNKS = (BN - (int)ACC1_COL) / 32;          // 3
+constexpr int COPY_WARPS = 3;  // SFA, SFB rows 0..127, SFB rows 128..255
+static_assert(SFA_COL + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(ACC1_COL % 32 == 0 && (BN - (int)ACC1_COL) % 32 == 0, "overlap must be whole 32-column chunks");
 
 // instruction descriptor: E2M1 x E2M1, UE4M3 scales, f32 accumulate, K-major
 // A and B, M x N, K = 64 (dense).
@@ -117,6 +122,8 @@ struct Smem {
     uint64_t tmem_full;
     uint64_t tmem_empty;
     uint64_t drain;
+    uint64_t sf_full[2];   // scale buffer filled (COPY_WARPS commits)
+    uint64_t sf_empty[2];  // scale buffer no longer read by the MMAs
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -215,11 +222,13 @@ drain:
 }
 
 // ---------------------------------------------------------------- MMA -------
-// One thread (of the leader CTA for the pair) issues everything.  Descriptors
-// are built once; a stage / k-block step only adds to the 14-bit start-address
-// field (shared memory addresses are < 2^18, so the field never carries).  For
-// each 64-wide k-block the scale copies go out right before the MMA that reads
-// them, so the tensor pipe can start on k-block 0 while later copies queue.
+// One thread (of the leader CTA for the pair) issues the MMAs; the scale-factor
+// copies into TMEM are issued by the copy warps below.  tcgen05.cp costs about
+// 50 cycles per instruction and a stage needs 12 of them against 512 cycles of
+// MMA work, so they run on other threads, a stage ahead, into the other scale
+// buffer.  Descriptors are built once; a stage / k-block step only adds to the
+// 14-bit start-address field (shared memory addresses are < 2^18, so the field
+// never carries).
 template <bool PAIR>
 __device__ void mma_issuer(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, uint32_t tmem) {
     using C = Cfg<PAIR>;
@@ -227,8 +236,6 @@ __device__ void mma_issuer(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t*
     const uint32_t ring_s = smem_u32(ring);
     const uint64_t a_desc0 = smem_desc(ring_s, 16, 1024, kLayoutSw128);
     const uint64_t b_desc0 = smem_desc(ring_s + A_BYTES, 16, 1024, kLayoutSw128);
-    const uint64_t sfa_desc0 = smem_desc(ring_s + A_BYTES + C::B_BYTES, 0, 128, kLayoutNone);
-    const uint64_t sfb_desc0 = smem_desc(ring_s + A_BYTES + C::B_BYTES + SFA_BYTES, 0, 128, kLayoutNone);
     const uint32_t sfa_t = tmem + SFA_COL, sfb_t = tmem + SFB_COL;
     int first, step;
     tile_range<PAIR>(first, step);
@@ -244,40 +251,36 @@ __device__ void mma_issuer(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t*
         const uint32_t acc = tmem + ((tcount & 1) ? ACC1_COL : 0u);
         for (int kt = 0; kt < p.kt_count; kt++, it++) {
             const int st = it % C::STAGES;
-            if (!mbar_wait_bounded(&s->full[st], (it / C::STAGES) & 1, abort, p.limit_ns)) {
+            const uint32_t sb = it & 1;
+            // the stage's scales are in TMEM (the copy warps saw its data arrive)
+            if (!mbar_wait_bounded(&s->sf_full[sb], (it >> 1) & 1, abort, p.limit_ns)) {
                 if (!*abort) raise_abort(s, p, 3);
                 goto drain;
             }
             tc_fence_after();
             const uint64_t off = (uint64_t)((st * C::STAGE_BYTES) >> 4);
             const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
+            const uint32_t sfo = sb ? SF_COLS : 0u;
 #pragma unroll
             for (int kb = 0; kb < KB_PER_STAGE; kb++) {
                 if (kb < nkb) {
-                    const uint64_t sa = sfa_desc0 + off + kb * (512 >> 4);
-                    const uint64_t sb0 = sfb_desc0 + off + kb * (512 >> 4);
-                    const uint64_t sb1 = sb0 + (SFA_BYTES >> 4);
                     const uint64_t ad = a_desc0 + off + kb * (32 >> 4);
                     const uint64_t bd = b_desc0 + off + kb * (32 >> 4);
                     const uint32_t acc_flag = (kt > 0 || kb > 0) ? 1u : 0u;
-                    if (PAIR) {
-                        tc_cp_32x128b_x4_pair(sfa_t + 4 * kb, sa);
-                        tc_cp_32x128b_x4_pair(sfb_t + 8 * kb, sb0);
-                        tc_cp_32x128b_x4_pair(sfb_t + 8 * kb + 4, sb1);
-                        tc_mma_nvf4_pair(acc, ad, bd, C::IDESC, sfa_t + 4 * kb, sfb_t + 8 * kb, acc_flag);
-                    } else {
-                        tc_cp_32x128b_x4(sfa_t + 4 * kb, sa);
-                        tc_cp_32x128b_x4(sfb_t + 8 * kb, sb0);
-                        tc_cp_32x128b_x4(sfb_t + 8 * kb + 4, sb1);
-                        tc_mma_nvf4(acc, ad, bd, C::IDESC, sfa_t + 4 * kb, sfb_t + 8 * kb, acc_flag);
-                    }
+                    if (PAIR)
+                        tc_mma_nvf4_pair(acc, ad, bd, C::IDESC, sfa_t + sfo + 4 * kb, sfb_t + sfo + 8 * kb, acc_flag);
+                    else
+                        tc_mma_nvf4(acc, ad, bd, C::IDESC, sfa_t + sfo + 4 * kb, sfb_t + sfo + 8 * kb, acc_flag);
                 }
             }
             issued = true;
-            if (PAIR)
+            if (PAIR) {
                 tc_commit_pair(&s->empty[st], 0x3);
-            else
+                tc_commit_pair(&s->sf_empty[sb], 0x1);
+            } else {
                 tc_commit(&s->empty[st]);
+                tc_commit(&s->sf_empty[sb]);
+            }
         }
         if (PAIR)
             tc_commit_pair(&s->tmem_full, 0x3);
@@ -294,6 +297,49 @@ drain:
             tc_commit(&s->drain);
         volatile int never = 0;
         mbar_wait_bounded(&s->drain, 0, &never, p.limit_ns);
+    }
+}
+
+// ---------------------------------------------------------------- copies ----
+// Copy warp `part` (0: SFA, 1: SFB rows 0..127, 2: SFB rows 128..255) moves its
+// 512-byte scale tiles of each stage from shared memory into the stage's TMEM
+// scale buffer (tcgen05.cp 32x128b.warpx4: one tile into lanes 0..31, copied
+// to all four lane quarters), then commits to sf_full.
+template <bool PAIR>
+__device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, uint32_t tmem, int part) {
+    using C = Cfg<PAIR>;
+    volatile int* abort = &s->abort_flag;
+    const uint32_t sf_s = smem_u32(ring) + A_BYTES + C::B_BYTES;  // SFA, then SFB rows 0..127, then 128..255
+    const uint64_t desc0 = smem_desc(sf_s + (uint32_t)part * SFA_BYTES, 0, 128, kLayoutNone);
+    const uint32_t tcol = tmem + (part == 0 ? SFA_COL : SFB_COL + 4u * (uint32_t)(part - 1));
+    const uint32_t kstride = part == 0 ? 4u : 8u;  // TMEM columns per k-block
+    int first, step;
+    tile_range<PAIR>(first, step);
+    uint32_t it = 0;
+    for (int tile = first; tile < p.num_tiles; tile += step) {
+        for (int kt = 0; kt < p.kt_count; kt++, it++) {
+            const int st = it % C::STAGES;
+            const uint32_t sb = it & 1;
+            if (!mbar_wait_bounded(&s->full[st], (it / C::STAGES) & 1, abort, p.limit_ns) ||
+                !mbar_wait_bounded(&s->sf_empty[sb], ((it >> 1) & 1) ^ 1, abort, p.limit_ns)) {
+                if (!*abort) raise_abort(s, p, 5);
+                return;
+            }
+            tc_fence_after();
+            const uint64_t d = desc0 + (uint64_t)((st * C::STAGE_BYTES) >> 4);
+            const uint32_t t = tcol + (sb ? SF_COLS : 0u);
+#pragma unroll
+            for (int kb = 0; kb < KB_PER_STAGE; kb++) {
+                if (PAIR)
+                    tc_cp_32x128b_x4_pair(t + kstride * kb, d + kb * (512 >> 4));
+                else
+                    tc_cp_32x128b_x4(t + kstride * kb, d + kb * (512 >> 4));
+            }
+            if (PAIR)
+                tc_commit_pair(&s->sf_full[sb], 0x1);
+            else
+                tc_commit(&s->sf_full[sb]);
+        }
     }
 }
 
@@ -489,6 +535,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(&s->tmem_full, 1);
         mbar_init(&s->tmem_empty, 4 * C::CTAS);
         mbar_init(&s->drain, 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&s->sf_full[i], COPY_WARPS);
+            mbar_init(&s->sf_empty[i], 1);
+        }
         s->abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -515,6 +565,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) mma_issuer<PAIR>(p, s, ring, tmem);
+        __syncwarp();
+    } else if (warp >= 6) {
+        if (lane == 0 && rank == 0) scale_copier<PAIR>(p, s, ring, tmem, warp - 6);
         __syncwarp();
     } else {
         epilogue<PAIR>(p, s, tmem, warp, lane, rank);
