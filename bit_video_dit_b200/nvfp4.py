@@ -24,7 +24,7 @@ DBG_SKIP_LOADS = 1
 
 EXPORTS = ("nvfp4_status_string", "nvfp4_version", "nvfp4_codes_bytes", "nvfp4_scales_bytes",
            "nvfp4_workspace_bytes", "nvfp4_read_device_error", "nvfp4_quantize", "nvfp4_gemm",
-           "nvfp4_kv_append", "nvfp4_kv_dequant", "nvfp4_test_encode")
+           "nvfp4_kv_append", "nvfp4_kv_dequant", "nvfp4_test_encode", "nvfp4_quantize_noalloc")
 
 
 class NVFP4Error(RuntimeError):
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_kv_dequant.restype = st
         L.nvfp4_test_encode.argtypes = [vp, i64, vp, vp, vp]
         L.nvfp4_test_encode.restype = st
+        L.nvfp4_quantize_noalloc.argtypes = [vp, i64, i64, i64, vp, vp, vp, ctypes.c_uint, vp]
+        L.nvfp4_quantize_noalloc.restype = st
         _lib = L
     return _lib
 

@@ -130,6 +130,27 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
                             void* scales, float* global_scale, unsigned flags, void* workspace,
                             size_t ws_bytes, nvfp4_stream_t stream);
 
+/* nvfp4_quantize without a workspace, for callers that cannot allocate
+ * device memory: code hosted inside a framework that owns every device
+ * allocation (an engine or server plugin handed only its input and output
+ * buffers), or a loop that must not call cudaMalloc because it would
+ * synchronize the device or break a fixed memory budget.  The pages have no
+ * counterpart of this call; it is a convenience of this library.
+ * Same arguments, rules and results as nvfp4_quantize, minus the workspace:
+ * the 256 bytes of scratch it needs live in one static device array of the
+ * library (NVFP4_NOALLOC_SCRATCH_BYTES; a problem that would need more is
+ * rejected with NVFP4_ERR_UNSUPPORTED), which every GPU that loads the
+ * library holds until the process exits.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress), so make that first
+ * call before any stream capture.  Each call clears the array (one
+ * cudaMemsetAsync on `stream`) and then launches the quantize kernel; it
+ * allocates nothing.  All calls share the array, so calls that can overlap
+ * on the GPU (different streams, different host threads) race: order them on
+ * one stream.  Errors found on the device are not reported by this call. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
+                                    void* scales, float* global_scale, unsigned flags, nvfp4_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* W4A4 GEMM  [RN-T] / [RN-I] W4A4 linears; [NEWS] fused adaLN epilogue        */
 /* ------------------------------------------------------------------------ */
