@@ -129,7 +129,7 @@ def kernel_hash() -> str:
 def recorded_traffic():
     """DRAM bytes per GEMM launch from the committed ncu summary, if it was
     taken on the current kernel sources."""
-    path = os.path.join(ROOT, "profiles", "gemm_qkv_traffic.json")
+    path = os.path.join(ROOT, "profiles", "gemm_qkv_traffic.txt")
     try:
         with open(path) as f:
             r = json.load(f)
@@ -304,6 +304,18 @@ def run_ours(args, rank: int, world: int) -> dict | None:
                      "frac_of_nominal_9pf": round(gemm_tflops / NOMINAL_FP4_TFLOPS, 4),
                      "traffic": None if tr is None else tr["dram_bytes_per_launch"],
                      "algorithmic_bytes": M * K // 2 + N * K // 2 + (M + N) * K // 16 + M * N * 2},
+        "roofline_by_kernel": {
+            "gemm": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4)},
+            "quantize": {"bound": "hbm", "achieved": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(quant_bytes / (q_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+            "kv_append": {"bound": "hbm", "achieved": round(append_bytes / (ap_ms * 1e-3) / 1e9, 1),
+                          "peak": pk["hbm_gbs"], "unit": "GB/s",
+                          "frac": round(append_bytes / (ap_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+            "kv_dequant": {"bound": "hbm", "achieved": round(dequant_bytes / (dq_ms * 1e-3) / 1e9, 1),
+                           "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": round(dequant_bytes / (dq_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}},
         "components_ms": {"quantize": round(q_ms, 4), "gemm": round(g_ms, 4), "kv_append": round(ap_ms, 4),
                           "kv_dequant": round(dq_ms, 4)},
         "quantize": {"GB/s": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),

@@ -4,9 +4,11 @@
 
 namespace {
 // Every call's workspace starts with a 256-byte control block: the device
-// error record (bytes 0..15) and, for quantize / KV append, the grid-barrier
-// words and tensor maxima of the fused kernel.
+// error record (bytes 0..15) and, for quantize / KV append, the launch epoch
+// of the fused kernel, which then keeps one 64-bit slot per CTA (1024 x 8
+// bytes) after the block.
 constexpr size_t kWsControl = 256;
+constexpr size_t kWsQuantize = kWsControl + 1024 * 8;
 }
 
 extern "C" const char* nvfp4_status_string(nvfp4_status s) {
@@ -43,11 +45,11 @@ extern "C" size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
     (void)k;
     switch (op) {
         case NVFP4_OP_QUANTIZE:
-        case NVFP4_OP_KV_APPEND:
+        case NVFP4_OP_KV_APPEND: return kWsQuantize;
         case NVFP4_OP_GEMM:
         case NVFP4_OP_KV_DEQUANT: return kWsControl;
     }
-    return kWsControl;
+    return kWsQuantize;
 }
 
 extern "C" nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int* code, uint32_t* info) {

@@ -1,8 +1,8 @@
 // noalloc.cu -- nvfp4_quantize_noalloc: nvfp4_quantize for callers that may
 // not allocate device memory (no workspace argument).
 //
-// The fused quantize kernel needs 256 bytes of device scratch besides its
-// inputs and outputs: its error record, grid-barrier words and tensor maxima.
+// The fused quantize kernel needs a little device scratch besides its inputs
+// and outputs: its error record, grid-barrier words and per-CTA maxima.
 // Here that scratch is one file-scope __device__ array instead of a caller
 // workspace.  Every GPU that loads the library holds the array until the
 // process exits.

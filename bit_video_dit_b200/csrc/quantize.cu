@@ -9,12 +9,9 @@
 //
 // All kernels here are HBM-bandwidth bound.  Layout of the work:
 //  * quantize / KV append: one cooperative launch (see quantize_fused_kernel):
-//    bulk copies into shared memory, |x| max on the bf16 bit patterns (two
-//    16-bit lanes per 32-bit SIMD max), a bounded grid barrier for the tensor
-//    scale, then the encode from shared memory.  In the encode a warp owns a
-//    512-element run of one row; lane i holds the 16-byte chunks i and i+32,
-//    a block of 16 elements is a lane pair (one shuffle for the block amax),
-//    and a warp's 4-byte code stores are 128 contiguous bytes.
+//    the input held in registers across a bounded grid barrier, |x| max on
+//    the bf16 bit patterns (two 16-bit lanes per 32-bit SIMD max), then the
+//    encode: a warp per 512-element run, a lane per 16-element block.
 //  * dequant-gather: a warp owns 512-element runs of a slot; lane i decodes
 //    elements 8i..8i+7 and 256+8i..256+8i+7 (4-byte code loads, 16-byte bf16
 //    stores, each warp-wide access contiguous), two runs in flight per lane.
@@ -27,27 +24,32 @@ namespace nvfp4 {
 constexpr int kThreads = 256;  // dequant / probe kernels
 
 // ---------------------------------------------------------------------------
-// Fused quantize: one cooperative launch, one CTA per SM.
-//   phase 1  every CTA bulk-copies (cp.async.bulk, no registers involved) its
-//            contiguous share of 512-element row runs into shared memory and
-//            takes the |x| max of it;
-//   barrier  the CTA maxima meet in one atomicMax word per tensor; the last
-//            CTA to arrive turns it into a32 = amax / 2688 and releases the
-//            grid (bounded wait everywhere else);
-//   phase 2  every CTA encodes its runs straight from shared memory.
-// HBM is read once and written once.  Runs that do not fit in shared memory
-// (tensors larger than ~#SMs x 200 KB) are read from global memory in both
-// phases instead.
+// Fused quantize: one cooperative launch, one CTA of 512 threads per SM.
+//   phase 1  every CTA loads its contiguous share of 512-element row runs
+//            straight into registers -- a lane holds one 16-element block of
+//            up to kMaxRuns runs, all loads in flight at once -- and takes the
+//            |x| max on the bf16 bit patterns;
+//   barrier  each CTA publishes its maxima in its own 64-bit slot, tagged
+//            with this launch's epoch; one warp per CTA polls all slots
+//            (bounded wait) and reduces them in the same pass, so no atomics
+//            and no second round trip: a32 = amax / 2688;
+//   phase 2  every CTA encodes the blocks it still holds in registers: one
+//            block scale per lane, 8-byte code stores (256 contiguous bytes
+//            per warp).
+// HBM is read once and written once.  Runs beyond kMaxRuns per warp (tensors
+// larger than ~#SMs x 176 KB) are read again in phase 2 (from L2 when the
+// tensor fits there).
 // ---------------------------------------------------------------------------
 constexpr int kQThreads = 512;
 constexpr int kQWarps = kQThreads / 32;
-constexpr int kRunBytes = 1024;  // one 512-element bf16 run
+constexpr int kMaxRuns = 11;   // runs held in registers per warp (11 x 32 B per lane)
+constexpr int kMaxGrid = 1024;
 
-// Control block in the first 256 bytes of the workspace (zero before first use).
-constexpr int kCtlCount = 8;   // uint32 index: CTAs arrived at the grid barrier
-constexpr int kCtlGen = 9;     // barrier generation
-constexpr int kCtlAmax = 10;   // [2] bf16 magnitude bit patterns, reset by the releasing CTA
-constexpr int kCtlAlpha = 12;  // [2] a32 bits
+// Workspace: a 256-byte control block (zero before first use), then one
+// 64-bit slot per CTA: epoch (high 32 bits) | tensor-1 max (bits 31..16) |
+// tensor-0 max (bits 15..0), maxima as bf16 magnitude bit patterns.
+constexpr int kCtlEpoch = 8;   // uint32 index: epoch of the last completed launch
+constexpr size_t kWsSlots = 256;
 
 struct QuantArgs {
     const uint8_t* x[2];
@@ -55,14 +57,15 @@ struct QuantArgs {
     uint8_t* scales[2];
     float* gscale[2];
     int64_t rows, cols, ld;   // per tensor, elements
-    int64_t upr;              // 512-element runs per row
-    int64_t runs_per_tensor;
-    int64_t total_runs;       // ntensors * runs_per_tensor
+    int upr;                  // 512-element runs per row
+    int runs_per_tensor;
+    int total_runs;           // ntensors * runs_per_tensor
+    int ntensors;
     int given;
     int swizzled;
     int64_t tiles_c;          // ceil(cols / 64)
-    int cap;                  // runs cached in shared memory per CTA
     uint32_t* ctl;
+    unsigned long long* slots;  // [kMaxGrid]
     DevError* err;
     uint64_t limit_ns;
 };
@@ -77,193 +80,170 @@ __device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
 }
 
 struct Run {
-    int t;            // tensor
-    int64_t r, c0;    // row, first column
-    int nchunks;      // valid 16-byte chunks (L / 8)
+    int t;        // tensor
+    int r;        // row
+    int c0;       // first column
+    int nblk;     // valid 16-element blocks (L / 16)
 };
 
-__device__ __forceinline__ Run run_of(const QuantArgs& a, int64_t g) {
+__device__ __forceinline__ Run run_of(const QuantArgs& a, int g) {
     Run u;
     u.t = g >= a.runs_per_tensor ? 1 : 0;
-    const int64_t gl = g - (u.t ? a.runs_per_tensor : 0);
+    const int gl = g - (u.t ? a.runs_per_tensor : 0);
     u.r = gl / a.upr;
     u.c0 = (gl - u.r * a.upr) * 512;
-    u.nchunks = (int)(min((int64_t)512, a.cols - u.c0) / 8);
+    u.nblk = (int)(min((int64_t)512, a.cols - u.c0) / 16);
     return u;
 }
 
 __device__ __forceinline__ const uint8_t* run_src(const QuantArgs& a, const Run& u) {
-    return (u.t ? a.x[1] : a.x[0]) + (u.r * a.ld + u.c0) * 2;
+    return (u.t ? a.x[1] : a.x[0]) + ((int64_t)u.r * a.ld + u.c0) * 2;
+}
+
+// encode one 16-element block (lane `lane` of run u) and store codes + scale
+__device__ __forceinline__ void encode_block(const QuantArgs& a, const Run& u, int lane, const uint4& q0,
+                                             const uint4& q1, float a32) {
+    // block max on the bf16 bit patterns (exact), widened once
+    const uint32_t mb = __vmaxu2(absmax_bits8(q0), absmax_bits8(q1));
+    const float amax_b = __uint_as_float(max(mb & 0xFFFFu, mb >> 16) << 16);
+    const BlockScale b = block_scale(amax_b, a32);
+    float f[16];
+    bf16x8_to_f32(q0, f);
+    bf16x8_to_f32(q1, f + 8);
+    const uint2 w = make_uint2(encode8(f, b.inv), encode8(f + 8, b.inv));
+    uint8_t* crow = (u.t ? a.codes[1] : a.codes[0]) + (int64_t)u.r * (a.cols / 2) + u.c0 / 2;
+    *reinterpret_cast<uint2*>(crow + 8 * lane) = w;
+    uint8_t* sb = u.t ? a.scales[1] : a.scales[0];
+    if (a.swizzled) {
+        // run base (warp-uniform) + lane part; c0 / 16 is a multiple of 32
+        const int64_t base = ((int64_t)(u.r >> 7) * a.tiles_c + (u.c0 >> 6)) * 512 + (u.r & 31) * 16 + ((u.r >> 5) & 3) * 4;
+        sb[base + (lane >> 2) * 512 + (lane & 3)] = (uint8_t)b.code;
+    } else {
+        sb[(int64_t)u.r * (a.cols / 16) + u.c0 / 16 + lane] = (uint8_t)b.code;
+    }
 }
 
 __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
-    extern __shared__ __align__(128) uint8_t qsmem[];
-    uint4* cache = reinterpret_cast<uint4*>(qsmem);  // [cap][64]
-    __shared__ __align__(8) uint64_t s_bar;
-    __shared__ uint32_t s_red[2][kQWarps];
+    __shared__ uint32_t s_red[kQWarps];
     __shared__ float s_alpha[2];
     __shared__ int s_ok;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t G = gridDim.x;
-    const int64_t begin = a.total_runs * (int64_t)blockIdx.x / G;
-    const int64_t end = a.total_runs * ((int64_t)blockIdx.x + 1) / G;
-    const int64_t ncached = min(end - begin, (int64_t)a.cap);
+    const int G = gridDim.x;
+    const int begin = (int)((int64_t)a.total_runs * blockIdx.x / G);
+    const int end = (int)((int64_t)a.total_runs * (blockIdx.x + 1) / G);
+    const uint32_t epoch = *(volatile uint32_t*)&a.ctl[kCtlEpoch] + 1u;  // same for every CTA of this launch
 
-    // ---- phase 1: bulk-copy this CTA's runs into shared memory
-    if (threadIdx.x == 0) {
-        mbar_init(&s_bar, 1);
-        fence_barrier_init();
-        fence_proxy_async_smem();
-        s_ok = 1;
-    }
-    __syncthreads();
-    {
-        // every thread announces its own bytes, then issues its copies; the
-        // single arrival comes after all announcements (the __syncthreads)
-        uint32_t mine = 0;
-        for (int64_t l = threadIdx.x; l < ncached; l += kQThreads) mine += (uint32_t)run_of(a, begin + l).nchunks * 16u;
-        if (mine) mbar_expect_tx_only(&s_bar, mine);
-        for (int64_t l = threadIdx.x; l < ncached; l += kQThreads) {
-            const Run u = run_of(a, begin + l);
-            bulk_load(cache + l * 64, run_src(a, u), (uint32_t)u.nchunks * 16u, &s_bar);
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) mbar_arrive(&s_bar);
-    if (ncached > 0) {
-        volatile int never = 0;
-        if (!mbar_wait_bounded(&s_bar, 0, &never, a.limit_ns)) {
-            record_error(a.err, NVFP4_ERR_TIMEOUT, 1);
-            s_ok = 0;  // the copies may still land: wait for them once more below
-        }
-    }
-    __syncthreads();
-    if (!s_ok) {
-        if (threadIdx.x == 0) {
-            volatile int never = 0;
-            mbar_wait_bounded(&s_bar, 0, &never, a.limit_ns);
-        }
-        return;
-    }
-
-    if (!a.given) {
-        uint32_t m0 = 0, m1 = 0;
-        for (int64_t g = begin + warp; g < end; g += kQWarps) {
+    // ---- phase 1: this warp's runs begin + warp + 16 k, one block per lane
+    uint4 q[kMaxRuns][2];
+#pragma unroll
+    for (int k = 0; k < kMaxRuns; k++) {
+        q[k][0] = q[k][1] = make_uint4(0, 0, 0, 0);
+        const int g = begin + warp + kQWarps * k;
+        if (g < end) {
             const Run u = run_of(a, g);
-            const int64_t l = g - begin;
-            const bool v0 = lane < u.nchunks, v1 = lane + 32 < u.nchunks;
-            uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-            if (l < ncached) {
-                if (v0) q0 = cache[l * 64 + lane];
-                if (v1) q1 = cache[l * 64 + 32 + lane];
-            } else {
-                const uint8_t* src = run_src(a, u);
-                if (v0) q0 = ld_stream16(src + lane * 16);
-                if (v1) q1 = ld_stream16(src + (lane + 32) * 16);
+            if (lane < u.nblk) {
+                const uint8_t* src = run_src(a, u) + lane * 32;
+                q[k][0] = ld_stream16(src);
+                q[k][1] = ld_stream16(src + 16);
             }
-            const uint32_t mm = __vmaxu2(absmax_bits8(q0), absmax_bits8(q1));
+        }
+    }
+    if (threadIdx.x == 0) s_ok = 1;
+    if (!a.given) {
+        uint32_t m0 = 0, m1 = 0;  // two bf16 magnitudes per word, per tensor
+#pragma unroll
+        for (int k = 0; k < kMaxRuns; k++) {
+            const int g = begin + warp + kQWarps * k;
+            const uint32_t mm = __vmaxu2(absmax_bits8(q[k][0]), absmax_bits8(q[k][1]));
+            if (g >= a.runs_per_tensor) m1 = __vmaxu2(m1, mm);
+            else m0 = __vmaxu2(m0, mm);
+        }
+        for (int g = begin + warp + kQWarps * kMaxRuns; g < end; g += kQWarps) {
+            const Run u = run_of(a, g);
+            uint32_t mm = 0;
+            if (lane < u.nblk) {
+                const uint8_t* src = run_src(a, u) + lane * 32;
+                mm = __vmaxu2(absmax_bits8(ld_stream16(src)), absmax_bits8(ld_stream16(src + 16)));
+            }
             if (u.t) m1 = __vmaxu2(m1, mm);
             else m0 = __vmaxu2(m0, mm);
         }
-        m0 = max(m0 & 0xFFFFu, m0 >> 16);
-        m1 = max(m1 & 0xFFFFu, m1 >> 16);
+        // one word per lane: tensor-1 max in the high half, tensor-0 in the low
+        uint32_t m = (max(m1 & 0xFFFFu, m1 >> 16) << 16) | max(m0 & 0xFFFFu, m0 >> 16);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            m0 = max(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
-            m1 = max(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
-        }
-        if (lane == 0) {
-            s_red[0][warp] = m0;
-            s_red[1][warp] = m1;
-        }
+        for (int o = 16; o > 0; o >>= 1) m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) s_red[warp] = m;
         __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t c0 = 0, c1 = 0;
-            for (int w = 0; w < kQWarps; w++) {
-                c0 = max(c0, s_red[0][w]);
-                c1 = max(c1, s_red[1][w]);
+        if (warp == 0) {
+            uint32_t c = lane < kQWarps ? s_red[lane] : 0u;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) c = __vmaxu2(c, __shfl_xor_sync(0xFFFFFFFFu, c, o));
+            if (lane == 0) {
+                const unsigned long long v = ((unsigned long long)epoch << 32) | c;
+                asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a.slots + blockIdx.x), "l"(v) : "memory");
             }
-            volatile uint32_t* vctl = a.ctl;
-            const uint32_t gen = vctl[kCtlGen];
-            atomicMax(&a.ctl[kCtlAmax + 0], c0);
-            atomicMax(&a.ctl[kCtlAmax + 1], c1);
-            __threadfence();
-            const uint32_t arrived = atomicAdd(&a.ctl[kCtlCount], 1u);
-            if (arrived == (uint32_t)G - 1) {
-                // last CTA: finish the tensor maxima and release the grid
-                __threadfence();
-                for (int t = 0; t < 2; t++) {
-                    const uint32_t bits = atomicExch(&a.ctl[kCtlAmax + t], 0u);
-                    const float a32 = __fdiv_rn(__uint_as_float(bits << 16), 2688.0f);  // amax / (6 * 448)
-                    vctl[kCtlAlpha + t] = __float_as_uint(a32);
-                    if (t < (a.total_runs > a.runs_per_tensor ? 2 : 1)) *(t ? a.gscale[1] : a.gscale[0]) = a32;
+            // wait until every CTA of this launch has published, reducing as we go
+            const uint64_t t0 = global_ns();
+            uint32_t it = 0;
+            uint32_t total;
+            while (true) {
+                bool all = true;
+                uint32_t mx = 0;
+                for (int i = lane; i < G; i += 32) {
+                    // relaxed loads pipeline; one acquire fence follows success
+                    unsigned long long v;
+                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a.slots + i) : "memory");
+                    if ((uint32_t)(v >> 32) != epoch) all = false;
+                    else mx = __vmaxu2(mx, (uint32_t)v);
                 }
-                vctl[kCtlCount] = 0;
-                __threadfence();
-                atomicAdd(&a.ctl[kCtlGen], 1u);
-            } else {
-                const uint64_t t0 = global_ns();
-                uint32_t it = 0;
-                while (vctl[kCtlGen] == gen) {
-                    if ((++it & 255u) == 0 && global_ns() - t0 > a.limit_ns) {
+                all = __all_sync(0xFFFFFFFFu, all);
+                if (all) {
+                    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx = __vmaxu2(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                    total = mx;
+                    break;
+                }
+                if ((++it & 15u) == 0 && global_ns() - t0 > a.limit_ns) {
+                    if (lane == 0) {
                         record_error(a.err, NVFP4_ERR_TIMEOUT, 2);
                         s_ok = 0;
-                        break;
                     }
+                    total = 0;
+                    break;
                 }
-                __threadfence();
             }
-            s_alpha[0] = __uint_as_float(vctl[kCtlAlpha + 0]);
-            s_alpha[1] = __uint_as_float(vctl[kCtlAlpha + 1]);
+            if (lane < a.ntensors) {
+                const uint32_t bits = lane ? (total >> 16) : (total & 0xFFFFu);
+                const float a32 = __fdiv_rn(__uint_as_float(bits << 16), 2688.0f);  // amax / (6 * 448)
+                s_alpha[lane] = a32;
+                if (blockIdx.x == 0 && s_ok) *(lane ? a.gscale[1] : a.gscale[0]) = a32;
+            }
+            // every CTA has read the epoch before publishing, so the next
+            // launch may now see the new one
+            if (blockIdx.x == 0 && lane == 0 && s_ok) *(volatile uint32_t*)&a.ctl[kCtlEpoch] = epoch;
         }
         __syncthreads();
         if (!s_ok) return;
     } else {
-        const int nt = a.total_runs > a.runs_per_tensor ? 2 : 1;  // gscale[1] is NULL for one tensor
-        if (threadIdx.x < nt) s_alpha[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
+        if (threadIdx.x < a.ntensors) s_alpha[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
         __syncthreads();
     }
 
     // ---- phase 2: encode
-    const int64_t sc_row = a.cols / 16;
-    for (int64_t g = begin + warp; g < end; g += kQWarps) {
-        const Run u = run_of(a, g);
-        const int64_t l = g - begin;
-        const bool v0 = lane < u.nchunks, v1 = lane + 32 < u.nchunks;
-        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-        if (l < ncached) {
-            if (v0) q0 = cache[l * 64 + lane];
-            if (v1) q1 = cache[l * 64 + 32 + lane];
-        } else {
-            const uint8_t* src = run_src(a, u);
-            if (v0) q0 = ld_stream16(src + lane * 16);
-            if (v1) q1 = ld_stream16(src + (lane + 32) * 16);
+#pragma unroll
+    for (int k = 0; k < kMaxRuns; k++) {
+        const int g = begin + warp + kQWarps * k;
+        if (g < end) {
+            const Run u = run_of(a, g);
+            if (lane < u.nblk) encode_block(a, u, lane, q[k][0], q[k][1], s_alpha[u.t]);
         }
-        const float a32 = s_alpha[u.t];
-        float f0[8], f1[8];
-        bf16x8_to_f32(q0, f0);
-        bf16x8_to_f32(q1, f1);
-        float am0 = absmax8(f0), am1 = absmax8(f1);
-        am0 = fmaxf(am0, __shfl_xor_sync(0xFFFFFFFFu, am0, 1));
-        am1 = fmaxf(am1, __shfl_xor_sync(0xFFFFFFFFu, am1, 1));
-        const BlockScale b0 = block_scale(am0, a32);
-        const BlockScale b1 = block_scale(am1, a32);
-        const uint32_t w0 = encode8(f0, b0.inv);
-        const uint32_t w1 = encode8(f1, b1.inv);
-        uint8_t* crow = (u.t ? a.codes[1] : a.codes[0]) + u.r * (a.cols / 2) + u.c0 / 2;
-        if (v0) *reinterpret_cast<uint32_t*>(crow + 4 * lane) = w0;
-        if (v1) *reinterpret_cast<uint32_t*>(crow + 128 + 4 * lane) = w1;
-        // even lanes store the scale of their first-half block, odd lanes
-        // the scale of their second-half block
-        const bool odd = lane & 1;
-        if (odd ? v1 : v0) {
-            const int64_t bj = u.c0 / 16 + (odd ? 16 : 0) + (lane >> 1);
-            const uint8_t code = (uint8_t)(odd ? b1.code : b0.code);
-            uint8_t* sb = u.t ? a.scales[1] : a.scales[0];
-            if (a.swizzled)
-                sb[swz_offset(u.r, bj, a.tiles_c)] = code;
-            else
-                sb[u.r * sc_row + bj] = code;
+    }
+    for (int g = begin + warp + kQWarps * kMaxRuns; g < end; g += kQWarps) {
+        const Run u = run_of(a, g);
+        if (lane < u.nblk) {
+            const uint8_t* src = run_src(a, u) + lane * 32;
+            encode_block(a, u, lane, ld_stream16(src), ld_stream16(src + 16), s_alpha[u.t]);
         }
     }
 
@@ -273,10 +253,9 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
         const int64_t rows_pad = (a.rows + 127) / 128 * 128;
         const int64_t sc_pad = a.tiles_c * 4;
         const int64_t npad = (rows_pad - a.rows) * sc_pad;
-        const int nt = a.total_runs > a.runs_per_tensor ? 2 : 1;
-        for (int t = 0; t < nt; t++) {
+        for (int t = 0; t < a.ntensors; t++) {
             uint8_t* sb = t ? a.scales[1] : a.scales[0];
-            for (int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x; i < npad; i += G * kQThreads) {
+            for (int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x; i < npad; i += (int64_t)G * kQThreads) {
                 const int64_t r = a.rows + i / sc_pad, c = i % sc_pad;
                 sb[swz_offset(r, c, a.tiles_c)] = 0;
             }
@@ -410,27 +389,10 @@ static nvfp4_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-static int g_q_dev = -1;
-static int g_q_smem = 0;
-
 // one fused, cooperative launch over one or two tensors of the same shape
 static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t rows, int64_t cols, int64_t ld,
                                   void* const* codes, void* const* scales, float* const* gscale, bool given,
                                   bool swizzled, void* workspace, cudaStream_t stream) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (g_q_dev != dev) {
-        int optin = 0;
-        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        // leave room for the kernel's static shared memory
-        const int smem = (optin - 2048) / kRunBytes * kRunBytes;
-        if (cudaFuncSetAttribute(quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        g_q_smem = smem;
-        g_q_dev = dev;
-    }
     QuantArgs a{};
     for (int t = 0; t < ntensors; t++) {
         a.x[t] = static_cast<const uint8_t*>(x[t]);
@@ -438,25 +400,27 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
         a.scales[t] = static_cast<uint8_t*>(scales[t]);
         a.gscale[t] = gscale[t];
     }
+    const int64_t upr = (cols + 511) / 512;
+    if (rows * upr * ntensors > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
     a.rows = rows;
     a.cols = cols;
     a.ld = ld;
-    a.upr = (cols + 511) / 512;
-    a.runs_per_tensor = rows * a.upr;
+    a.upr = (int)upr;
+    a.runs_per_tensor = (int)(rows * upr);
     a.total_runs = a.runs_per_tensor * ntensors;
+    a.ntensors = ntensors;
     a.given = given ? 1 : 0;
     a.swizzled = swizzled ? 1 : 0;
     a.tiles_c = (cols + 63) / 64;
     a.ctl = static_cast<uint32_t*>(workspace);
+    a.slots = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + kWsSlots);
     a.err = static_cast<DevError*>(workspace);
     a.limit_ns = 2000000000ull;
-    const int G = (int)std::min<int64_t>(num_sms(), a.total_runs);
-    const int64_t per_cta = (a.total_runs + G - 1) / G;
-    a.cap = (int)std::min<int64_t>(per_cta, g_q_smem / kRunBytes);
+    const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), a.total_runs);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kQThreads);
-    cfg.dynamicSmemBytes = (size_t)a.cap * kRunBytes;
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;

@@ -95,9 +95,9 @@ enum {
 /* Workspace bytes the caller must pass to the call `op` (device memory,
  * 256-byte aligned).  Never 0.  Its first 256 bytes are a control block (the
  * device error record in bytes 0..15; for quantize and KV append also the
- * grid-barrier words and tensor maxima of the fused kernel): they must be
- * zero before a workspace is first used, and the calls leave them ready for
- * the next call.  A workspace may be reused by calls that are ordered on one
+ * grid-barrier words of the fused kernel): they must be zero before a
+ * workspace is first used, and the calls leave them ready for the next call.
+ * Quantize and KV append also keep per-CTA maxima after the block.  A workspace may be reused by calls that are ordered on one
  * stream; calls that can run concurrently need their own workspaces. */
 size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k);
 
@@ -137,9 +137,10 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * synchronize the device or break a fixed memory budget.  The pages have no
  * counterpart of this call; it is a convenience of this library.
  * Same arguments, rules and results as nvfp4_quantize, minus the workspace:
- * the 256 bytes of scratch it needs live in one static device array of the
- * library (NVFP4_NOALLOC_SCRATCH_BYTES; a problem that would need more is
- * rejected with NVFP4_ERR_UNSUPPORTED), which every GPU that loads the
+ * the scratch it needs (8448 bytes: a control block and one maximum per CTA)
+ * lives in one static device array of the library
+ * (NVFP4_NOALLOC_SCRATCH_BYTES; a problem that would need more is rejected
+ * with NVFP4_ERR_UNSUPPORTED), which every GPU that loads the
  * library holds until the process exits.  The first call on a device looks
  * up the array's device address (cudaGetSymbolAddress), so make that first
  * call before any stream capture.  Each call clears the array (one
@@ -147,7 +148,7 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * allocates nothing.  All calls share the array, so calls that can overlap
  * on the GPU (different streams, different host threads) race: order them on
  * one stream.  Errors found on the device are not reported by this call. */
-#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+#define NVFP4_NOALLOC_SCRATCH_BYTES 8448
 nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
                                     void* scales, float* global_scale, unsigned flags, nvfp4_stream_t stream);
 
