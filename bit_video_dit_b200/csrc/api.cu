@@ -8,7 +8,7 @@ namespace {
 // of the fused kernel, which then keeps one 64-bit slot per CTA (1024 x 8
 // bytes) after the block.
 constexpr size_t kWsControl = 256;
-constexpr size_t kWsQuantize = kWsControl + 1024 * 8;
+constexpr size_t kWsQuantize = kWsControl;  // the grid-barrier words live in the control block
 }
 
 extern "C" const char* nvfp4_status_string(nvfp4_status s) {

@@ -427,6 +427,13 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t* r) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Ties 32 registers filled by tmem_ld_32cols to a preceding tmem_ld_wait: the
+// compiler sees them rewritten here, so no use of them moves above the wait.
+__device__ __forceinline__ void tmem_regs_ready(uint32_t* r) {
+#pragma unroll
+    for (int i = 0; i < 32; i++) asm volatile("" : "+r"(r[i]));
+}
+
 // Shared-memory matrix descriptor (sm_100 format, version 1).
 //   bits 0-13 start >> 4, 16-29 leading byte offset >> 4, 32-45 stride byte
 //   offset >> 4, 46-47 version = 1, 49-51 base offset, 61-63 layout type.

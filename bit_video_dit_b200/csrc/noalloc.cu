@@ -2,7 +2,7 @@
 // not allocate device memory (no workspace argument).
 //
 // The fused quantize kernel needs a little device scratch besides its inputs
-// and outputs: its error record, grid-barrier words and per-CTA maxima.
+// and outputs: its error record and grid-barrier words (a 256-byte block).
 // Here that scratch is one file-scope __device__ array instead of a caller
 // workspace.  Every GPU that loads the library holds the array until the
 // process exits.

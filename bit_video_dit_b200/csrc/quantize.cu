@@ -25,47 +25,51 @@ constexpr int kThreads = 256;  // dequant / probe kernels
 
 // ---------------------------------------------------------------------------
 // Fused quantize: one cooperative launch, one CTA of 512 threads per SM.
-//   phase 1  every CTA loads its contiguous share of 512-element row runs
-//            straight into registers -- a lane holds one 16-element block of
-//            up to kMaxRuns runs, all loads in flight at once -- and takes the
-//            |x| max on the bf16 bit patterns;
-//   barrier  each CTA publishes its maxima in its own 64-bit slot, tagged
-//            with this launch's epoch; one warp per CTA polls all slots
-//            (bounded wait) and reduces them in the same pass, so no atomics
-//            and no second round trip: a32 = amax / 2688;
-//   phase 2  every CTA encodes the blocks it still holds in registers: one
-//            block scale per lane, 8-byte code stores (256 contiguous bytes
-//            per warp).
-// HBM is read once and written once.  Runs beyond kMaxRuns per warp (tensors
-// larger than ~#SMs x 176 KB) are read again in phase 2 (from L2 when the
-// tensor fits there).
+//   phase 1  every warp takes a contiguous share of one tensor's 512-element
+//            row runs and loads up to kMaxRuns of them straight into
+//            registers -- a lane holds one 16-element block per run, all
+//            loads in flight at once -- keeping each block's |x| max (taken
+//            on the bf16 bit patterns) for phase 2;
+//   barrier  each CTA folds its maxima into two global maxima (fire-and-
+//            forget reductions) and counts itself in with an acquire-release
+//            add; every CTA polls the count (bounded wait), then reads the
+//            maxima: a32 = amax / 2688;
+//   phase 2  every warp encodes the blocks it holds: one block scale per
+//            lane (the reciprocal 1 / (s * a32) from a 256-entry table per
+//            tensor, built once per CTA), 8-byte code stores (256 contiguous
+//            bytes per warp).
+// A warp walks its runs with row pointers it advances, so no run needs an
+// integer division, and the scale layout is a template parameter.  HBM is
+// read once and written once; runs beyond kMaxRuns per warp (tensors larger
+// than ~#SMs x 176 KB) are read again in phase 2 (from L2 when the tensor
+// fits there).
 // ---------------------------------------------------------------------------
 constexpr int kQThreads = 512;
 constexpr int kQWarps = kQThreads / 32;
 constexpr int kMaxRuns = 11;   // runs held in registers per warp (11 x 32 B per lane)
 constexpr int kMaxGrid = 1024;
 
-// Workspace: a 256-byte control block (zero before first use), then one
-// 64-bit slot per CTA: epoch (high 32 bits) | tensor-1 max (bits 31..16) |
-// tensor-0 max (bits 15..0), maxima as bf16 magnitude bit patterns.
-constexpr int kCtlEpoch = 8;   // uint32 index: epoch of the last completed launch
-constexpr size_t kWsSlots = 256;
+// Control block (uint32 words of the workspace's first 256 bytes, zero before
+// first use; words 0..3 are the error record):
+constexpr int kCtlEpoch = 8;   // epoch of the last completed launch
+constexpr int kCtlCount = 16;  // [2] arrivals of the launch with epoch parity p
+constexpr int kCtlMax = 20;    // [2][2] bf16 magnitude maxima per parity, per tensor
 
 struct QuantArgs {
     const uint8_t* x[2];
     uint8_t* codes[2];
     uint8_t* scales[2];
     float* gscale[2];
-    int64_t rows, cols, ld;   // per tensor, elements
-    int upr;                  // 512-element runs per row
+    int64_t ld_bytes;      // row stride of x in bytes
+    int64_t code_ld;       // bytes per row of codes (cols / 2)
+    int64_t scale_ld;      // bytes per row of row-major scales (cols / 16)
+    int64_t tile_row;      // bytes per 128-row block of swizzled scales (cols / 64 * 512)
+    int upr;               // 512-element runs per row
+    int last_nblk;         // 16-element blocks in the last run of a row
     int runs_per_tensor;
-    int total_runs;           // ntensors * runs_per_tensor
     int ntensors;
     int given;
-    int swizzled;
-    int64_t tiles_c;          // ceil(cols / 64)
     uint32_t* ctl;
-    unsigned long long* slots;  // [kMaxGrid]
     DevError* err;
     uint64_t limit_ns;
 };
@@ -79,185 +83,238 @@ __device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
     return __vmaxu2(a, b);
 }
 
-struct Run {
-    int t;        // tensor
-    int r;        // row
-    int c0;       // first column
-    int nblk;     // valid 16-element blocks (L / 16)
+// 16-byte streaming load, or zeros when `pred` is false (no branch)
+__device__ __forceinline__ uint4 ld_stream16_if(const void* p, bool pred) {
+    uint4 v;
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+        "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+        "@q ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p), "r"((int)pred));
+    return v;
+}
+
+// A warp's position: run cr of row r of its tensor, with the row's pointers.
+template <bool SWZ>
+struct Walk {
+    int r, cr;
+    const uint8_t* xrow;
+    uint8_t* crow;
+    uint8_t* srow;  // SWZ: this row's base inside its 128-row block of tiles
+
+    __device__ __forceinline__ void seek(const QuantArgs& a, int t, int run) {
+        r = run / a.upr;
+        cr = run - r * a.upr;
+        xrow = a.x[t] + (int64_t)r * a.ld_bytes;
+        crow = a.codes[t] + (int64_t)r * a.code_ld;
+        srow = a.scales[t] + (SWZ ? (int64_t)(r >> 7) * a.tile_row + (r & 31) * 16 + ((r >> 5) & 3) * 4
+                                  : (int64_t)r * a.scale_ld);
+    }
+    __device__ __forceinline__ void next(const QuantArgs& a) {
+        if (++cr == a.upr) {
+            cr = 0;
+            ++r;
+            xrow += a.ld_bytes;
+            crow += a.code_ld;
+            if (SWZ) {
+                // rows 32 apart share a 16-byte tile row; a new 128-row block starts a new tile row
+                srow += (r & 127) == 0 ? a.tile_row - 3 * 4 - 31 * 16 : ((r & 31) == 0 ? 4 - 31 * 16 : 16);
+            } else {
+                srow += a.scale_ld;
+            }
+        }
+    }
+    __device__ __forceinline__ int nblk(const QuantArgs& a) const { return cr == a.upr - 1 ? a.last_nblk : 32; }
 };
 
-__device__ __forceinline__ Run run_of(const QuantArgs& a, int g) {
-    Run u;
-    u.t = g >= a.runs_per_tensor ? 1 : 0;
-    const int gl = g - (u.t ? a.runs_per_tensor : 0);
-    u.r = gl / a.upr;
-    u.c0 = (gl - u.r * a.upr) * 512;
-    u.nblk = (int)(min((int64_t)512, a.cols - u.c0) / 16);
-    return u;
-}
-
-__device__ __forceinline__ const uint8_t* run_src(const QuantArgs& a, const Run& u) {
-    return (u.t ? a.x[1] : a.x[0]) + ((int64_t)u.r * a.ld + u.c0) * 2;
-}
-
-// encode one 16-element block (lane `lane` of run u) and store codes + scale
-__device__ __forceinline__ void encode_block(const QuantArgs& a, const Run& u, int lane, const uint4& q0,
-                                             const uint4& q1, float a32) {
-    // block max on the bf16 bit patterns (exact), widened once
-    const uint32_t mb = __vmaxu2(absmax_bits8(q0), absmax_bits8(q1));
-    const float amax_b = __uint_as_float(max(mb & 0xFFFFu, mb >> 16) << 16);
-    const BlockScale b = block_scale(amax_b, a32);
+// encode one 16-element block (lane `lane` of the run at w) and store codes + scale
+template <bool SWZ>
+__device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool valid, const uint4& q0,
+                                             const uint4& q1, uint32_t bmax, float d6, const float* inv_tab) {
+    // s = E4M3(amax_b / (6 a32)); a zero tensor scale flushes every block
+    const float amax_b = __uint_as_float(bmax << 16);
+    const uint32_t code = d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, d6));
+    const float inv = inv_tab[code];
     float f[16];
     bf16x8_to_f32(q0, f);
     bf16x8_to_f32(q1, f + 8);
-    const uint2 w = make_uint2(encode8(f, b.inv), encode8(f + 8, b.inv));
-    uint8_t* crow = (u.t ? a.codes[1] : a.codes[0]) + (int64_t)u.r * (a.cols / 2) + u.c0 / 2;
-    *reinterpret_cast<uint2*>(crow + 8 * lane) = w;
-    uint8_t* sb = u.t ? a.scales[1] : a.scales[0];
-    if (a.swizzled) {
-        // run base (warp-uniform) + lane part; c0 / 16 is a multiple of 32
-        const int64_t base = ((int64_t)(u.r >> 7) * a.tiles_c + (u.c0 >> 6)) * 512 + (u.r & 31) * 16 + ((u.r >> 5) & 3) * 4;
-        sb[base + (lane >> 2) * 512 + (lane & 3)] = (uint8_t)b.code;
-    } else {
-        sb[(int64_t)u.r * (a.cols / 16) + u.c0 / 16 + lane] = (uint8_t)b.code;
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) y[i] = __fmul_rn(f[i], inv);
+    // a flushed block (inv == 0) is +0 codes
+    const uint32_t c0 = inv == 0.0f ? 0u : e2m1x8(y), c1 = inv == 0.0f ? 0u : e2m1x8(y + 8);
+    if (valid) {
+        *reinterpret_cast<uint2*>(w.crow + w.cr * 256 + 8 * lane) = make_uint2(c0, c1);
+        if (SWZ)
+            w.srow[(int64_t)(w.cr * 8 + (lane >> 2)) * 512 + (lane & 3)] = (uint8_t)code;
+        else
+            w.srow[w.cr * 32 + lane] = (uint8_t)code;
     }
 }
 
+template <bool SWZ>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
     __shared__ uint32_t s_red[kQWarps];
-    __shared__ float s_alpha[2];
+    __shared__ float s_d6[2];
+    __shared__ float s_inv[2][256];
+    __shared__ uint32_t s_total;
     __shared__ int s_ok;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
-    const int begin = (int)((int64_t)a.total_runs * blockIdx.x / G);
-    const int end = (int)((int64_t)a.total_runs * (blockIdx.x + 1) / G);
+    // warps [0, nw / ntensors) take tensor 0, the rest tensor 1
+    const int nw = G * kQWarps, nwt = nw / a.ntensors;
+    const int wg = blockIdx.x * kQWarps + warp;
+    const int t = wg / nwt;
+    const int wl = wg - t * nwt;
+    const int wb = (int)((int64_t)a.runs_per_tensor * wl / nwt);
+    const int we = (int)((int64_t)a.runs_per_tensor * (wl + 1) / nwt);
     const uint32_t epoch = *(volatile uint32_t*)&a.ctl[kCtlEpoch] + 1u;  // same for every CTA of this launch
+    const int par = (int)(epoch & 1u);
+    Walk<SWZ> w0;
+    w0.seek(a, t, min(wb, a.runs_per_tensor - 1));
 
-    // ---- phase 1: this warp's runs begin + warp + 16 k, one block per lane
+    // ---- phase 1: this warp's runs wb .. we-1 of tensor t, one block per lane
     uint4 q[kMaxRuns][2];
+    uint32_t bm[kMaxRuns];  // the lane's block max (bf16 magnitude bits) per run
+    {
+        Walk<SWZ> w = w0;
+#pragma unroll
+        for (int k = 0; k < kMaxRuns; k++) {
+            const bool have = wb + k < we;
+            const bool valid = have && lane < w.nblk(a);
+            const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
+            q[k][0] = ld_stream16_if(src, valid);
+            q[k][1] = ld_stream16_if(src + 16, valid);
+            if (have) w.next(a);
+        }
+    }
+    uint32_t m = 0;  // two bf16 magnitudes per word
 #pragma unroll
     for (int k = 0; k < kMaxRuns; k++) {
-        q[k][0] = q[k][1] = make_uint4(0, 0, 0, 0);
-        const int g = begin + warp + kQWarps * k;
-        if (g < end) {
-            const Run u = run_of(a, g);
-            if (lane < u.nblk) {
-                const uint8_t* src = run_src(a, u) + lane * 32;
-                q[k][0] = ld_stream16(src);
-                q[k][1] = ld_stream16(src + 16);
-            }
-        }
+        const uint32_t mm = __vmaxu2(absmax_bits8(q[k][0]), absmax_bits8(q[k][1]));
+        bm[k] = max(mm & 0xFFFFu, mm >> 16);
+        m = max(m, bm[k]);
     }
     if (threadIdx.x == 0) s_ok = 1;
     if (!a.given) {
-        uint32_t m0 = 0, m1 = 0;  // two bf16 magnitudes per word, per tensor
-#pragma unroll
-        for (int k = 0; k < kMaxRuns; k++) {
-            const int g = begin + warp + kQWarps * k;
-            const uint32_t mm = __vmaxu2(absmax_bits8(q[k][0]), absmax_bits8(q[k][1]));
-            if (g >= a.runs_per_tensor) m1 = __vmaxu2(m1, mm);
-            else m0 = __vmaxu2(m0, mm);
-        }
-        for (int g = begin + warp + kQWarps * kMaxRuns; g < end; g += kQWarps) {
-            const Run u = run_of(a, g);
-            uint32_t mm = 0;
-            if (lane < u.nblk) {
-                const uint8_t* src = run_src(a, u) + lane * 32;
-                mm = __vmaxu2(absmax_bits8(ld_stream16(src)), absmax_bits8(ld_stream16(src + 16)));
+        {
+            Walk<SWZ> w = w0;
+            for (int k = 0; k < kMaxRuns && wb + k < we; k++) w.next(a);
+            for (int g = wb + kMaxRuns; g < we; g++) {
+                const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
+                const bool valid = lane < w.nblk(a);
+                const uint32_t mm = __vmaxu2(absmax_bits8(ld_stream16_if(src, valid)),
+                                             absmax_bits8(ld_stream16_if(src + 16, valid)));
+                m = max(m, max(mm & 0xFFFFu, mm >> 16));
+                w.next(a);
             }
-            if (u.t) m1 = __vmaxu2(m1, mm);
-            else m0 = __vmaxu2(m0, mm);
         }
         // one word per lane: tensor-1 max in the high half, tensor-0 in the low
-        uint32_t m = (max(m1 & 0xFFFFu, m1 >> 16) << 16) | max(m0 & 0xFFFFu, m0 >> 16);
+        m = t ? (m << 16) : m;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
         if (lane == 0) s_red[warp] = m;
         __syncthreads();
-        if (warp == 0) {
-            uint32_t c = lane < kQWarps ? s_red[lane] : 0u;
+        if (threadIdx.x == 0) {
+            uint32_t c = 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) c = __vmaxu2(c, __shfl_xor_sync(0xFFFFFFFFu, c, o));
-            if (lane == 0) {
-                const unsigned long long v = ((unsigned long long)epoch << 32) | c;
-                asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a.slots + blockIdx.x), "l"(v) : "memory");
-            }
-            // wait until every CTA of this launch has published, reducing as we go
-            const uint64_t t0 = global_ns();
-            uint32_t it = 0;
-            uint32_t total;
-            while (true) {
-                bool all = true;
-                uint32_t mx = 0;
-                for (int i = lane; i < G; i += 32) {
-                    // relaxed loads pipeline; one acquire fence follows success
-                    unsigned long long v;
-                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a.slots + i) : "memory");
-                    if ((uint32_t)(v >> 32) != epoch) all = false;
-                    else mx = __vmaxu2(mx, (uint32_t)v);
-                }
-                all = __all_sync(0xFFFFFFFFu, all);
-                if (all) {
-                    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) mx = __vmaxu2(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-                    total = mx;
-                    break;
-                }
-                if ((++it & 15u) == 0 && global_ns() - t0 > a.limit_ns) {
-                    if (lane == 0) {
-                        record_error(a.err, NVFP4_ERR_TIMEOUT, 2);
-                        s_ok = 0;
-                    }
-                    total = 0;
+            for (int i = 0; i < kQWarps; i++) c = __vmaxu2(c, s_red[i]);
+            uint32_t* cnt = a.ctl + kCtlCount + par;
+            uint32_t* mx = a.ctl + kCtlMax + 2 * par;
+            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(c & 0xFFFFu) : "memory");
+            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx + 1), "r"(c >> 16) : "memory");
+            uint32_t old;
+            // acquire too: the last CTA to arrive reads the maxima without polling
+            asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
+            // wait for every CTA of this launch (bounded)
+            const uint64_t t_start = global_ns();
+            uint32_t n = old + 1u;
+            while (n < (uint32_t)G) {
+                __nanosleep(20);
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(cnt) : "memory");
+                if (n < (uint32_t)G && global_ns() - t_start > a.limit_ns) {
+                    record_error(a.err, NVFP4_ERR_TIMEOUT, 2);
+                    s_ok = 0;
                     break;
                 }
             }
-            if (lane < a.ntensors) {
-                const uint32_t bits = lane ? (total >> 16) : (total & 0xFFFFu);
-                const float a32 = __fdiv_rn(__uint_as_float(bits << 16), 2688.0f);  // amax / (6 * 448)
-                s_alpha[lane] = a32;
-                if (blockIdx.x == 0 && s_ok) *(lane ? a.gscale[1] : a.gscale[0]) = a32;
-            }
-            // every CTA has read the epoch before publishing, so the next
-            // launch may now see the new one
-            if (blockIdx.x == 0 && lane == 0 && s_ok) *(volatile uint32_t*)&a.ctl[kCtlEpoch] = epoch;
+            uint32_t t0, t1;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t0) : "l"(mx) : "memory");
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t1) : "l"(mx + 1) : "memory");
+            s_total = (t1 << 16) | t0;
         }
         __syncthreads();
         if (!s_ok) return;
+        if (threadIdx.x < a.ntensors) {
+            const uint32_t bits = threadIdx.x ? (s_total >> 16) : (s_total & 0xFFFFu);
+            const float a32 = __fdiv_rn(__uint_as_float(bits << 16), 2688.0f);  // amax / (6 * 448)
+            s_d6[threadIdx.x] = a32;  // a32 for now; the table below needs it
+            if (blockIdx.x == 0) *(threadIdx.x ? a.gscale[1] : a.gscale[0]) = a32;
+        }
+        // every CTA of this launch has counted itself in, and so has read the
+        // epoch and finished with the other parity's words: reset those for
+        // the next launch, then let it see the new epoch
+        if (blockIdx.x == 0 && threadIdx.x == 32) {
+            a.ctl[kCtlCount + (par ^ 1)] = 0u;
+            a.ctl[kCtlMax + 2 * (par ^ 1)] = 0u;
+            a.ctl[kCtlMax + 2 * (par ^ 1) + 1] = 0u;
+            __threadfence();
+            *(volatile uint32_t*)&a.ctl[kCtlEpoch] = epoch;
+        }
     } else {
-        if (threadIdx.x < a.ntensors) s_alpha[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
+        if (threadIdx.x < a.ntensors) s_d6[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
+    }
+    __syncthreads();
+    // per tensor: inv[code] = 1 / (s * a32) for every E4M3 code (0 when s = 0
+    // or a32 = 0), then d6 = 6 a32
+    {
+        const int tt = threadIdx.x >> 8, c = threadIdx.x & 255;
+        if (tt < a.ntensors) {
+            const float a32 = s_d6[tt];
+            const float sv = e4m3_value((uint32_t)c);
+            s_inv[tt][c] = (a32 == 0.0f || sv == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sv, a32));
+        }
+        __syncthreads();
+        if (threadIdx.x < a.ntensors) s_d6[threadIdx.x] = __fmul_rn(6.0f, s_d6[threadIdx.x]);
         __syncthreads();
     }
 
     // ---- phase 2: encode
+    {
+        const float d6 = s_d6[t];
+        const float* inv_tab = s_inv[t];
+        Walk<SWZ> w = w0;
 #pragma unroll
-    for (int k = 0; k < kMaxRuns; k++) {
-        const int g = begin + warp + kQWarps * k;
-        if (g < end) {
-            const Run u = run_of(a, g);
-            if (lane < u.nblk) encode_block(a, u, lane, q[k][0], q[k][1], s_alpha[u.t]);
+        for (int k = 0; k < kMaxRuns; k++) {
+            if (wb + k < we) {
+                encode_block<SWZ>(w, lane, lane < w.nblk(a), q[k][0], q[k][1], bm[k], d6, inv_tab);
+                w.next(a);
+            }
         }
-    }
-    for (int g = begin + warp + kQWarps * kMaxRuns; g < end; g += kQWarps) {
-        const Run u = run_of(a, g);
-        if (lane < u.nblk) {
-            const uint8_t* src = run_src(a, u) + lane * 32;
-            encode_block(a, u, lane, ld_stream16(src), ld_stream16(src + 16), s_alpha[u.t]);
+        for (int g = wb + kMaxRuns; g < we; g++) {
+            const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
+            const bool valid = lane < w.nblk(a);
+            const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
+            const uint32_t mm = __vmaxu2(absmax_bits8(v0), absmax_bits8(v1));
+            encode_block<SWZ>(w, lane, valid, v0, v1, max(mm & 0xFFFFu, mm >> 16), d6, inv_tab);
+            w.next(a);
         }
     }
 
     // zero the padding rows of the swizzled scale tiles (cols % 64 == 0, so
     // only the rows past `rows` up to the next multiple of 128 are padding)
-    if (a.swizzled) {
-        const int64_t rows_pad = (a.rows + 127) / 128 * 128;
-        const int64_t sc_pad = a.tiles_c * 4;
-        const int64_t npad = (rows_pad - a.rows) * sc_pad;
-        for (int t = 0; t < a.ntensors; t++) {
-            uint8_t* sb = t ? a.scales[1] : a.scales[0];
+    if (SWZ) {
+        const int64_t rows = a.runs_per_tensor / a.upr;
+        const int64_t tiles_c = a.tile_row / 512;
+        const int64_t rows_pad = (rows + 127) / 128 * 128;
+        const int64_t sc_pad = tiles_c * 4;
+        const int64_t npad = (rows_pad - rows) * sc_pad;
+        for (int tt = 0; tt < a.ntensors; tt++) {
+            uint8_t* sb = a.scales[tt];
             for (int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x; i < npad; i += (int64_t)G * kQThreads) {
-                const int64_t r = a.rows + i / sc_pad, c = i % sc_pad;
-                sb[swz_offset(r, c, a.tiles_c)] = 0;
+                const int64_t r = rows + i / sc_pad, c = i % sc_pad;
+                sb[swz_offset(r, c, tiles_c)] = 0;
             }
         }
     }
@@ -401,22 +458,20 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
         a.gscale[t] = gscale[t];
     }
     const int64_t upr = (cols + 511) / 512;
-    if (rows * upr * ntensors > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
-    a.rows = rows;
-    a.cols = cols;
-    a.ld = ld;
+    if (rows * upr > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
+    a.ld_bytes = ld * 2;
+    a.code_ld = cols / 2;
+    a.scale_ld = cols / 16;
+    a.tile_row = cols / 64 * 512;
     a.upr = (int)upr;
+    a.last_nblk = (int)((cols - (upr - 1) * 512) / 16);
     a.runs_per_tensor = (int)(rows * upr);
-    a.total_runs = a.runs_per_tensor * ntensors;
     a.ntensors = ntensors;
     a.given = given ? 1 : 0;
-    a.swizzled = swizzled ? 1 : 0;
-    a.tiles_c = (cols + 63) / 64;
     a.ctl = static_cast<uint32_t*>(workspace);
-    a.slots = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + kWsSlots);
     a.err = static_cast<DevError*>(workspace);
     a.limit_ns = 2000000000ull;
-    const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), a.total_runs);
+    const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), ((int64_t)a.runs_per_tensor * ntensors + kQWarps - 1) / kQWarps);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kQThreads);
@@ -427,7 +482,8 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, quantize_fused_kernel, a) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, swizzled ? quantize_fused_kernel<true> : quantize_fused_kernel<false>, a) !=
+        cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
     }
@@ -536,3 +592,4 @@ extern "C" nvfp4_status nvfp4_test_encode(const float* x, int64_t n, uint8_t* e2
     encoder_probe_kernel<<<g, 256, 0, (cudaStream_t)stream>>>(x, n, e2m1_out, e4m3_out);
     return launch_status();
 }
+

@@ -97,8 +97,8 @@ enum {
  * device error record in bytes 0..15; for quantize and KV append also the
  * grid-barrier words of the fused kernel): they must be zero before a
  * workspace is first used, and the calls leave them ready for the next call.
- * Quantize and KV append also keep per-CTA maxima after the block.  A workspace may be reused by calls that are ordered on one
- * stream; calls that can run concurrently need their own workspaces. */
+ * A workspace may be reused by calls that are ordered on one stream; calls
+ * that can run concurrently need their own workspaces. */
 size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k);
 
 /* Synchronizes `stream`, then reads and clears the device error record of
@@ -123,9 +123,9 @@ nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int
  * global_scale: device binary32, written (COMPUTE) or read (GIVEN).
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols) bytes.
  * One cooperative launch (one CTA per SM): the input is read from HBM once
- * (held in shared memory across a bounded grid barrier that turns the
- * per-CTA maxima into a32) unless it exceeds ~#SMs x 200 KB, in which case
- * the excess is read twice. */
+ * (held in registers across a bounded grid barrier that turns the CTAs'
+ * maxima into a32) unless it exceeds ~#SMs x 176 KB, in which case the
+ * excess is read twice. */
 nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
                             void* scales, float* global_scale, unsigned flags, void* workspace,
                             size_t ws_bytes, nvfp4_stream_t stream);
@@ -137,7 +137,7 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * synchronize the device or break a fixed memory budget.  The pages have no
  * counterpart of this call; it is a convenience of this library.
  * Same arguments, rules and results as nvfp4_quantize, minus the workspace:
- * the scratch it needs (8448 bytes: a control block and one maximum per CTA)
+ * the scratch it needs (the 256-byte control block of the grid barrier)
  * lives in one static device array of the library
  * (NVFP4_NOALLOC_SCRATCH_BYTES; a problem that would need more is rejected
  * with NVFP4_ERR_UNSUPPORTED), which every GPU that loads the
@@ -148,7 +148,7 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * allocates nothing.  All calls share the array, so calls that can overlap
  * on the GPU (different streams, different host threads) race: order them on
  * one stream.  Errors found on the device are not reported by this call. */
-#define NVFP4_NOALLOC_SCRATCH_BYTES 8448
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
 nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
                                     void* scales, float* global_scale, unsigned flags, nvfp4_stream_t stream);
 
