@@ -35,6 +35,7 @@
 //    records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
 //    drains what it issued and frees TMEM before returning.
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 
@@ -51,6 +52,16 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int A_BYTES = BM * BKB;                  // 16 KB
 constexpr int SFA_BYTES = KB_PER_STAGE * 512;      // 2 KB
 constexpr int SFB_BYTES = 2 * KB_PER_STAGE * 512;  // 4 KB (two 128-row halves of the tile's N)
+
+// Per-tile shared memory of the epilogue: the tile's per-column vectors
+// (bias, modulate scale, modulate shift, gate; bf16 pairs, two buffers by
+// tile parity) and each warp's two 32 x 32 bf16 staging buffers for the TMA
+// store of C (64-byte rows, 64B swizzle: 16-byte unit u of row r at
+// (u ^ (r / 2 % 4)) * 16).
+constexpr int EPI_BUF_BYTES = 32 * 64;
+constexpr int EPI_STAGE_BYTES = 4 * 2 * EPI_BUF_BYTES;  // 16 KB
+constexpr int VEC_WORDS = BN / 2;                        // bf16 pairs per vector per tile
+constexpr int VEC_BYTES = 2 * 4 * VEC_WORDS * 4;        // 4 KB
 
 // Two accumulators of BN columns share TMEM with two 48-column scale buffers:
 // acc0 = [0, 256), acc1 = [160, 416), scales = [416, 512).  The accumulators
@@ -79,10 +90,10 @@ struct Cfg {
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int TILE_M = BM * CTAS;        // 256 or 128
     static constexpr int B_ROWS = PAIR ? 128 : 256;  // rows of B each CTA loads
-    static constexpr int STAGES = PAIR ? 5 : 4;
+    static constexpr int STAGES = PAIR ? 5 : 3;
     static constexpr int B_BYTES = B_ROWS * BKB;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + VEC_BYTES + 1024 + 256;
     static constexpr uint32_t TX_BYTES = (uint32_t)(CTAS * STAGE_BYTES);  // per stage, both CTAs
     static constexpr uint32_t IDESC = make_idesc(TILE_M, BN);
     static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment for 128B swizzle");
@@ -344,9 +355,14 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
 }
 
 // ---------------------------------------------------------------- epilogue --
+// GELU, tanh form, with the hardware tanh (tanh.approx.f32, absolute error
+// about 2^-11): the GELU value moves by at most ~3e-4 |y|.
 __device__ __forceinline__ float gelu_tanh(float y) {
     const float k = 0.7978845608028654f;  // sqrt(2 / pi)
-    return 0.5f * y * (1.0f + tanhf(k * (y + 0.044715f * y * y * y)));
+    const float u = k * (y + 0.044715f * y * y * y);
+    float th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(u));
+    return 0.5f * y * (1.0f + th);
 }
 
 // 32 consecutive bf16 (as binary32), columns n0.. with `valid` of them in
@@ -362,16 +378,25 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* p, int valid, fl
     }
 }
 
-// One 32-column chunk of one output row: epilogue math and stores.
+// 32 bf16 of a staged per-column vector (shared memory, same for every lane)
+__device__ __forceinline__ void smem_vec32(const uint32_t* v, float* out) {
+    const uint4* q = reinterpret_cast<const uint4*>(v);
+#pragma unroll
+    for (int i = 0; i < 4; i++) bf16x8_to_f32(q[i], out + 8 * i);
+}
+
+// One 32-column chunk of one output row: epilogue math and outputs.  `r`
+// holds the accumulator (binary32 bits), `vec` the tile's staged vectors
+// (at this chunk's columns), `stage` this warp's staging buffer.
 __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* r, float alpha, int64_t m, bool row_ok,
-                                               int64_t n0, int valid, float oa32, int64_t tiles_on,
-                                               float& amax_run) {
+                                               int64_t n0, int valid, float oa32, int64_t tiles_on, float& amax_run,
+                                               const uint32_t* const* vec, uint8_t* stage, int lane) {
     float y[32];
 #pragma unroll
     for (int i = 0; i < 32; i++) y[i] = __uint_as_float(r[i]) * alpha;
     float v[32];
     if (p.bias) {
-        load_row32(p.bias + n0, valid, v);
+        smem_vec32(vec[0], v);
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] += v[i];
     }
@@ -380,17 +405,17 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
         for (int i = 0; i < 32; i++) y[i] = gelu_tanh(y[i]);
     }
     if (p.mod_scale) {
-        load_row32(p.mod_scale + n0, valid, v);
+        smem_vec32(vec[1], v);
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] = y[i] * (1.0f + v[i]);
     }
     if (p.mod_shift) {
-        load_row32(p.mod_shift + n0, valid, v);
+        smem_vec32(vec[2], v);
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] += v[i];
     }
     if (p.gate) {
-        load_row32(p.gate + n0, valid, v);
+        smem_vec32(vec[3], v);
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] = v[i] * y[i];
     }
@@ -410,23 +435,19 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
         for (int i = 0; i < 32; i++)
             if (i < valid) d[i] = y[i];
     }
-    if (p.c && row_ok) {
-        __nv_bfloat16* cp = p.c + m * p.ldc + n0;
-        if (valid == 32) {
-            uint32_t w[16];
+    if (p.c) {
+        // row `lane` of the staging buffer; the TMA store drops rows >= M and columns >= N
+        uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; i++) {
-                __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
-                w[i] = *reinterpret_cast<uint32_t*>(&b);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(cp);
-#pragma unroll
-            for (int i = 0; i < 4; i++) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; i++)
-                if (i < valid) cp[i] = __float2bfloat16_rn(y[i]);
+        for (int i = 0; i < 16; i++) {
+            __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&b);
         }
+        uint8_t* row = stage + lane * 64;
+        const int sw = (lane >> 1) & 3;
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+            *reinterpret_cast<uint4*>(row + ((u ^ sw) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     }
     if (p.out_codes) {
         // N % 64 == 0 for requant, so a 32-column chunk is whole
@@ -454,29 +475,49 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
 }
 
 template <bool PAIR>
-__device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t tmem, int warp, int lane, uint32_t rank) {
+__device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t tmem, int warp, int lane, uint32_t rank,
+                         const CUtensorMap* tma_c, uint8_t* epi_stage, uint32_t* vecs) {
     using C = Cfg<PAIR>;
     volatile int* abort = &s->abort_flag;
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int et = (warp - 2) * 32 + lane;  // 0..127 over the epilogue warps
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
     const float oa32 = p.out_codes ? __ldg(p.out_gscale) : 0.0f;
     const int64_t tiles_on = (p.N + 63) / 64;  // scale tiles along N of the output
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     // the leader's MMA waits for the epilogue warps of both CTAs
     const uint32_t empty_bar = PAIR ? mapa_shared(smem_u32(&s->tmem_empty), 0) : smem_u32(&s->tmem_empty);
+    const __nv_bfloat16* vsrc[4] = {p.bias, p.mod_scale, p.mod_shift, p.gate};
+    uint8_t* my_stage = epi_stage + (warp - 2) * 2 * EPI_BUF_BYTES;
+    if (p.c && lane == 0) prefetch_tmap(tma_c);
     int first, step;
     tile_range<PAIR>(first, step);
     float amax_run = 0.0f;
-    uint32_t tcount = 0;
+    uint32_t tcount = 0, nstored = 0;
     for (int tile = first; tile < p.num_tiles; tile += step, tcount++) {
         int mb, nb;
         tile_coords(p, tile, mb, nb);
-        if (!mbar_wait_bounded(&s->tmem_full, tcount & 1, abort, p.limit_ns)) {
-            if (!*abort) raise_abort(s, p, 4);
-            return;
+        // stage this tile's per-column vectors (zero past N)
+        uint32_t* tv = vecs + (tcount & 1) * 4 * VEC_WORDS;
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            if (vsrc[v]) {
+                const int64_t n = (int64_t)nb * BN + 2 * et;
+                uint32_t w2 = 0;
+                if (n + 1 < p.N)
+                    w2 = __ldg(reinterpret_cast<const uint32_t*>(vsrc[v] + n));
+                else if (n < p.N)
+                    w2 = (uint32_t)__bfloat16_as_ushort(vsrc[v][n]);
+                tv[v * VEC_WORDS + et] = w2;
+            }
         }
+        const bool ok = mbar_wait_bounded(&s->tmem_full, tcount & 1, abort, p.limit_ns);
+        if (!ok && !*abort) raise_abort(s, p, 4);
+        // the staged vectors are visible, and all four warps take the same exit
+        if (named_barrier_or(1, 128, !ok)) break;
         tc_fence_after();
-        const int64_t m = (int64_t)mb * C::TILE_M + (int64_t)rank * BM + q * 32 + lane;
+        const int64_t m0 = (int64_t)mb * C::TILE_M + (int64_t)rank * BM + q * 32;  // the warp's first row
+        const int64_t m = m0 + lane;
         const bool row_ok = m < p.M;
         const int ncols = min(BN, p.N - nb * BN);
         const int nchunks = (ncols + 31) / 32;
@@ -491,11 +532,12 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
             if (lane == 0) mbar_arrive_cluster(empty_bar);
         }
         for (int i = 0; i < nchunks; i++) {
-            // buffer 0 visits chunks 6, 7, 0, 1, ..., 5; buffer 1 visits 0..7
+            // buffer 0 visits chunks 5, 6, 7, 0, ..., 4; buffer 1 visits 0..7
             const int j = buf1 ? i : ((i < n_overlap) ? first_ov + i : i - n_overlap);
             uint32_t r[32];
             tmem_ld_32cols(acc + j * 32, r);
             tmem_ld_wait();
+            tmem_regs_ready(r);
             if (i == n_overlap - 1) {
                 // the overlapped columns are in registers: next tile may start
                 tc_fence_before();
@@ -504,9 +546,27 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
             }
             const int64_t n0 = (int64_t)nb * BN + j * 32;
             const int valid = (int)min((int64_t)32, p.N - n0);
-            epilogue_chunk(p, r, alpha, m, row_ok, n0, valid, oa32, tiles_on, amax_run);
+            uint8_t* stage = my_stage + (nstored & 1) * EPI_BUF_BYTES;
+            if (p.c) {
+                // the store issued two chunks ago has finished reading this buffer
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+            }
+            const uint32_t* vc[4] = {tv + j * 16, tv + VEC_WORDS + j * 16, tv + 2 * VEC_WORDS + j * 16,
+                                     tv + 3 * VEC_WORDS + j * 16};
+            epilogue_chunk(p, r, alpha, m, row_ok, n0, valid, oa32, tiles_on, amax_run, vc, stage, lane);
+            if (p.c) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(tma_c, stage, (int32_t)n0, (int32_t)m0);
+                    bulk_commit_group();
+                }
+                nstored++;
+            }
         }
     }
+    if (p.c && lane == 0) bulk_wait_group_all();
     if (p.out_amax) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax_run = fmaxf(amax_run, __shfl_xor_sync(0xFFFFFFFFu, amax_run, o));
@@ -518,11 +578,13 @@ template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                 const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
-                const __grid_constant__ Params p) {
+                const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ Params p) {
     using C = Cfg<PAIR>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Smem<C::STAGES>* s = reinterpret_cast<Smem<C::STAGES>*>(ring + C::STAGES * C::STAGE_BYTES);
+    uint8_t* epi_stage = ring + C::STAGES * C::STAGE_BYTES;  // 1024-aligned (STAGE_BYTES % 1024 == 0)
+    uint32_t* vecs = reinterpret_cast<uint32_t*>(epi_stage + EPI_STAGE_BYTES);
+    Smem<C::STAGES>* s = reinterpret_cast<Smem<C::STAGES>*>(epi_stage + EPI_STAGE_BYTES + VEC_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -570,7 +632,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0 && rank == 0) scale_copier<PAIR>(p, s, ring, tmem, warp - 6);
         __syncwarp();
     } else {
-        epilogue<PAIR>(p, s, tmem, warp, lane, rank);
+        epilogue<PAIR>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs);
     }
     tc_fence_before();
     if (PAIR)
@@ -660,6 +722,19 @@ static bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int
     return r == CUDA_SUCCESS;
 }
 
+// bf16 C [M x N], row stride ldc elements; a box is one epilogue warp's 32 rows
+// x 32 columns (64-byte rows, 64B swizzle)
+static bool make_c_map(CUtensorMap* map, void* c, int64_t M, int64_t N, int64_t ldc) {
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldc * 2)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // swizzled scales viewed as [row blocks][K/64 tiles][128 x u32]; a box is the
 // 4 tiles (2 KB) of one stage of one 128-row block.  Tiles past K/64 read as 0.
 static bool make_scale_map(CUtensorMap* map, const void* scales, int64_t rows, int64_t K) {
@@ -718,7 +793,9 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
     // CTA pairs (256-row tiles) whenever there is more than one 128-row block
     const bool pair = M > gemm::BM && pair_clusters > 0;
 
-    CUtensorMap ma, mb, msa, msb;
+    CUtensorMap ma, mb, msa, msb, mc;
+    memset(&mc, 0, sizeof(mc));
+    if (c_bf16 && !make_c_map(&mc, c_bf16, M, N, ldc)) return NVFP4_ERR_CUDA;
     if (!make_code_map(&ma, A->codes, M, K, gemm::BM) ||
         !make_code_map(&mb, B->codes, N, K, pair ? gemm::Cfg<true>::B_ROWS : gemm::Cfg<false>::B_ROWS) ||
         !make_scale_map(&msa, A->scales, M, K) || !make_scale_map(&msb, B->scales, N, K))
@@ -770,14 +847,14 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, gemm::gemm_kernel<true>, ma, mb, msa, msb, p) != cudaSuccess) {
+        if (cudaLaunchKernelEx(&cfg, gemm::gemm_kernel<true>, ma, mb, msa, msb, mc, p) != cudaSuccess) {
             cudaGetLastError();
             return NVFP4_ERR_CUDA;
         }
         return NVFP4_OK;
     }
     const int grid = std::min(p.num_tiles, sms);
-    gemm::gemm_kernel<false><<<grid, gemm::THREADS, gemm::Cfg<false>::SMEM_BYTES, (cudaStream_t)stream>>>(ma, mb, msa,
-                                                                                                         msb, p);
+    gemm::gemm_kernel<false><<<grid, gemm::THREADS, gemm::Cfg<false>::SMEM_BYTES, (cudaStream_t)stream>>>(
+        ma, mb, msa, msb, mc, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
