@@ -47,7 +47,13 @@ constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 256;  // K elements per stage
 constexpr int BKB = BK / 2;  // bytes per row per stage (128: one swizzle atom row)
 constexpr int KB_PER_STAGE = BK / 64;
-constexpr int THREADS = 288;  // producer, MMA, 4 epilogue warps, 3 scale-copy warps
+// Block: producer, MMA, 4 epilogue warps and NC scale-copy warps.  Two
+// variants: NC = 3 (SFA | SFB rows 0..127 | 128..255; 288 threads, so at
+// most 168 registers a thread) for long K, where the mainloop dominates, and
+// NC = 2 (SFA | all of SFB; 256 threads, up to 255 registers) for short K,
+// where the epilogue has the registers to take the shared accumulator
+// columns in one go and the next tile starts sooner.
+constexpr int threads_for(int nc) { return (6 + nc) * 32; }
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int A_BYTES = BM * BKB;                  // 16 KB
 constexpr int SFA_BYTES = KB_PER_STAGE * 512;      // 2 KB
@@ -75,7 +81,6 @@ constexpr uint32_t ACC1_COL = 160;
 constexpr uint32_t SFA_COL = ACC1_COL + BN;                        // 416 (+48: buffer 1)
 constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;           // 432 (+48: buffer 1)
 constexpr int OVERLAP_CHUNKS = (BN - (int)ACC1_COL) / 32;          // 3
-constexpr int COPY_WARPS = 3;  // SFA, SFB rows 0..127, SFB rows 128..255
 static_assert(SFA_COL + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(ACC1_COL % 32 == 0 && (BN - (int)ACC1_COL) % 32 == 0, "overlap must be whole 32-column chunks");
 
@@ -133,7 +138,7 @@ struct Smem {
     uint64_t tmem_full;
     uint64_t tmem_empty;
     uint64_t drain;
-    uint64_t sf_full[2];   // scale buffer filled (COPY_WARPS commits)
+    uint64_t sf_full[2];   // scale buffer filled (one commit per copy warp)
     uint64_t sf_empty[2];  // scale buffer no longer read by the MMAs
     uint32_t tmem_base;
     int abort_flag;
@@ -312,11 +317,12 @@ drain:
 }
 
 // ---------------------------------------------------------------- copies ----
-// Copy warp `part` (0: SFA, 1: SFB rows 0..127, 2: SFB rows 128..255) moves its
-// 512-byte scale tiles of each stage from shared memory into the stage's TMEM
-// scale buffer (tcgen05.cp 32x128b.warpx4: one tile into lanes 0..31, copied
-// to all four lane quarters), then commits to sf_full.
-template <bool PAIR>
+// Copy warp `part` (NC = 3: 0 SFA, 1 SFB rows 0..127, 2 SFB rows 128..255;
+// NC = 2: 0 SFA, 1 both SFB halves) moves its 512-byte scale tiles of each
+// stage from shared memory into the stage's TMEM scale buffer (tcgen05.cp
+// 32x128b.warpx4: one tile into lanes 0..31, copied to all four lane
+// quarters), then commits to sf_full.
+template <bool PAIR, int NC>
 __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, uint32_t tmem, int part) {
     using C = Cfg<PAIR>;
     volatile int* abort = &s->abort_flag;
@@ -324,6 +330,7 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
     const uint64_t desc0 = smem_desc(sf_s + (uint32_t)part * SFA_BYTES, 0, 128, kLayoutNone);
     const uint32_t tcol = tmem + (part == 0 ? SFA_COL : SFB_COL + 4u * (uint32_t)(part - 1));
     const uint32_t kstride = part == 0 ? 4u : 8u;  // TMEM columns per k-block
+    const int tiles = (NC == 2 && part == 1) ? 2 : 1;  // NC = 2: part 1 copies both SFB halves
     int first, step;
     tile_range<PAIR>(first, step);
     uint32_t it = 0;
@@ -341,10 +348,18 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
             const uint32_t t = tcol + (sb ? SF_COLS : 0u);
 #pragma unroll
             for (int kb = 0; kb < KB_PER_STAGE; kb++) {
-                if (PAIR)
-                    tc_cp_32x128b_x4_pair(t + kstride * kb, d + kb * (512 >> 4));
-                else
-                    tc_cp_32x128b_x4(t + kstride * kb, d + kb * (512 >> 4));
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    if (h < tiles) {
+                        // SFB rows 128..255 sit SFA_BYTES after rows 0..127 and go 4 columns right
+                        const uint32_t dst = t + kstride * kb + 4u * (uint32_t)h;
+                        const uint64_t src = d + kb * (512 >> 4) + (uint64_t)h * (SFA_BYTES >> 4);
+                        if (PAIR)
+                            tc_cp_32x128b_x4_pair(dst, src);
+                        else
+                            tc_cp_32x128b_x4(dst, src);
+                    }
+                }
             }
             if (PAIR)
                 tc_commit_pair(&s->sf_full[sb], 0x1);
@@ -474,7 +489,7 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
     }
 }
 
-template <bool PAIR>
+template <bool PAIR, bool EARLY>
 __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t tmem, int warp, int lane, uint32_t rank,
                          const CUtensorMap* tma_c, uint8_t* epi_stage, uint32_t* vecs) {
     using C = Cfg<PAIR>;
@@ -526,24 +541,7 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
         // chunks of this buffer that the other buffer overlaps come first
         const int first_ov = buf1 ? 0 : (BN / 32 - OVERLAP_CHUNKS);
         const int n_overlap = buf1 ? min(nchunks, OVERLAP_CHUNKS) : max(0, nchunks - first_ov);
-        if (n_overlap == 0) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(empty_bar);
-        }
-        for (int i = 0; i < nchunks; i++) {
-            // buffer 0 visits chunks 5, 6, 7, 0, ..., 4; buffer 1 visits 0..7
-            const int j = buf1 ? i : ((i < n_overlap) ? first_ov + i : i - n_overlap);
-            uint32_t r[32];
-            tmem_ld_32cols(acc + j * 32, r);
-            tmem_ld_wait();
-            tmem_regs_ready(r);
-            if (i == n_overlap - 1) {
-                // the overlapped columns are in registers: next tile may start
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(empty_bar);
-            }
+        auto out_chunk = [&](const uint32_t* r, int j) {
             const int64_t n0 = (int64_t)nb * BN + j * 32;
             const int valid = (int)min((int64_t)32, p.N - n0);
             uint8_t* stage = my_stage + (nstored & 1) * EPI_BUF_BYTES;
@@ -564,6 +562,57 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
                 }
                 nstored++;
             }
+        };
+        if (EARLY) {
+            // the overlapped chunks go to registers first; then the next tile may start
+            uint32_t ov[OVERLAP_CHUNKS][32];
+#pragma unroll
+            for (int c = 0; c < OVERLAP_CHUNKS; c++)
+                if (c < n_overlap) tmem_ld_32cols(acc + (first_ov + c) * 32, ov[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < OVERLAP_CHUNKS; c++) tmem_regs_ready(ov[c]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty_bar);
+            for (int i = 0; i < nchunks; i++) {
+                // buffer 0 visits chunks 5, 6, 7, 0, ..., 4; buffer 1 visits 0..7
+                const int j = buf1 ? i : ((i < n_overlap) ? first_ov + i : i - n_overlap);
+                uint32_t r[32];
+                if (i < n_overlap) {
+#pragma unroll
+                    for (int c = 0; c < OVERLAP_CHUNKS; c++)
+                        if (c == i)
+#pragma unroll
+                            for (int e = 0; e < 32; e++) r[e] = ov[c][e];
+                } else {
+                    tmem_ld_32cols(acc + j * 32, r);
+                    tmem_ld_wait();
+                    tmem_regs_ready(r);
+                }
+                out_chunk(r, j);
+            }
+        } else {
+            if (n_overlap == 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty_bar);
+            }
+            for (int i = 0; i < nchunks; i++) {
+                // buffer 0 visits chunks 5, 6, 7, 0, ..., 4; buffer 1 visits 0..7
+                const int j = buf1 ? i : ((i < n_overlap) ? first_ov + i : i - n_overlap);
+                uint32_t r[32];
+                tmem_ld_32cols(acc + j * 32, r);
+                tmem_ld_wait();
+                tmem_regs_ready(r);
+                if (i == n_overlap - 1) {
+                    // the overlapped columns are in registers: next tile may start
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(empty_bar);
+                }
+                out_chunk(r, j);
+            }
         }
     }
     if (p.c && lane == 0) bulk_wait_group_all();
@@ -574,8 +623,8 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
     }
 }
 
-template <bool PAIR>
-__global__ void __launch_bounds__(THREADS, 1)
+template <bool PAIR, int NC>
+__global__ void __launch_bounds__(threads_for(NC), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                 const __grid_constant__ CUtensorMap tma_sfa, const __grid_constant__ CUtensorMap tma_sfb,
                 const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ Params p) {
@@ -598,7 +647,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(&s->tmem_empty, 4 * C::CTAS);
         mbar_init(&s->drain, 1);
         for (int i = 0; i < 2; i++) {
-            mbar_init(&s->sf_full[i], COPY_WARPS);
+            mbar_init(&s->sf_full[i], NC);
             mbar_init(&s->sf_empty[i], 1);
         }
         s->abort_flag = 0;
@@ -629,10 +678,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0 && rank == 0) mma_issuer<PAIR>(p, s, ring, tmem);
         __syncwarp();
     } else if (warp >= 6) {
-        if (lane == 0 && rank == 0) scale_copier<PAIR>(p, s, ring, tmem, warp - 6);
+        if (lane == 0 && rank == 0) scale_copier<PAIR, NC>(p, s, ring, tmem, warp - 6);
         __syncwarp();
     } else {
-        epilogue<PAIR>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs);
+        epilogue<PAIR, NC == 2>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs);
     }
     tc_fence_before();
     if (PAIR)
@@ -679,15 +728,19 @@ static nvfp4_status gemm_setup(int& sms, int& pair_clusters) {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
         if (major != 10 || minor != 0) return NVFP4_ERR_UNSUPPORTED;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NVFP4_ERR_CUDA;
-        if (cudaFuncSetAttribute(gemm::gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm::gemm_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemm::Cfg<false>::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm::gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(gemm::gemm_kernel<false, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::Cfg<false>::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm::gemm_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::Cfg<true>::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm::gemm_kernel<true, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  gemm::Cfg<true>::SMEM_BYTES) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         // how many CTA pairs can be resident at once (bounds the persistent grid)
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (n / 2));
-        cfg.blockDim = dim3(gemm::THREADS);
+        cfg.blockDim = dim3(gemm::threads_for(3));
         cfg.dynamicSmemBytes = gemm::Cfg<true>::SMEM_BYTES;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -696,8 +749,8 @@ static nvfp4_status gemm_setup(int& sms, int& pair_clusters) {
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gemm::gemm_kernel<true>, &cfg) != cudaSuccess || clusters < 1) {
+        int clusters = 0;  // shared memory bounds both variants alike: one CTA per SM
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm::gemm_kernel<true, 3>, &cfg) != cudaSuccess || clusters < 1) {
             cudaGetLastError();
             clusters = 0;  // pair variant unavailable: single-CTA tiles only
         }
@@ -834,10 +887,13 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
         p.limit_ns = 2000000000ull;
     }
     p.err = static_cast<DevError*>(workspace);
+    // short K (at most 16 stages per tile): the epilogue bounds the tile rate,
+    // so take the variant whose epilogue frees the accumulator soonest
+    const int nc = p.kt_count <= 16 ? 2 : 3;
     if (pair) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * std::min(p.num_tiles, pair_clusters));
-        cfg.blockDim = dim3(gemm::THREADS);
+        cfg.blockDim = dim3(gemm::threads_for(nc));
         cfg.dynamicSmemBytes = gemm::Cfg<true>::SMEM_BYTES;
         cfg.stream = (cudaStream_t)stream;
         cudaLaunchAttribute attr[1];
@@ -847,14 +903,19 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, gemm::gemm_kernel<true>, ma, mb, msa, msb, mc, p) != cudaSuccess) {
+        if (cudaLaunchKernelEx(&cfg, nc == 2 ? gemm::gemm_kernel<true, 2> : gemm::gemm_kernel<true, 3>, ma, mb, msa, msb,
+                               mc, p) != cudaSuccess) {
             cudaGetLastError();
             return NVFP4_ERR_CUDA;
         }
         return NVFP4_OK;
     }
     const int grid = std::min(p.num_tiles, sms);
-    gemm::gemm_kernel<false><<<grid, gemm::THREADS, gemm::Cfg<false>::SMEM_BYTES, (cudaStream_t)stream>>>(
-        ma, mb, msa, msb, mc, p);
+    if (nc == 2)
+        gemm::gemm_kernel<false, 2><<<grid, gemm::threads_for(2), gemm::Cfg<false>::SMEM_BYTES, (cudaStream_t)stream>>>(
+            ma, mb, msa, msb, mc, p);
+    else
+        gemm::gemm_kernel<false, 3><<<grid, gemm::threads_for(3), gemm::Cfg<false>::SMEM_BYTES, (cudaStream_t)stream>>>(
+            ma, mb, msa, msb, mc, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -123,6 +123,63 @@ def test_ragged_shapes(M, N, K):
     assert torch.isnan(buf[:, N:]).all()  # nothing written past N
 
 
+@pytest.mark.parametrize("M,N,K", [(100, 264, 4160), (300, 520, 4352), (256, 256, 8192)])
+def test_long_k_shapes(M, N, K):
+    """More than 16 K-stages per tile: the kernel variant with three scale-copy
+    warps (single-CTA and CTA-pair tiles, a one-k-block K tail)."""
+    require_gpu()
+    qa, oa, qb, ob = _gemm_case(M, N, K, seed=M + N + K)
+    bias = syn.normal_bf16((N,), seed=7, std=0.02)
+    _run_checked(qa, qb, oa, ob, bias=bias)
+
+
+def _sampled_rows(M, seed):
+    return np.unique(np.concatenate([[0, 1, 127, 128, 255, 256, M - 1],
+                                     np.random.default_rng(seed).integers(0, M, 41)]))
+
+
+def test_ffn_full_size_up_gelu_requant_then_down_sampled_rows():
+    """DiT FFN pair at full size (8192 tokens, 3072 -> 14336 -> 3072): the
+    up-projection with GELU and the NVFP4 requant epilogue, then the
+    down-projection reading that NVFP4 output; checked on sampled rows."""
+    require_gpu()
+    M, D, F = syn.FFN_UP.M, syn.FFN_UP.K, syn.FFN_UP.N
+    qa, oa = _qboth(syn.activations_bf16(M, D, seed=51))
+    qu, ou = _qboth(syn.normal_bf16((F, D), seed=52, std=0.02))
+    qd, od = _qboth(syn.normal_bf16((D, F), seed=53, std=0.02))
+    rows = _sampled_rows(M, 54)
+    # output scale of the up-projection: delayed scaling from a calibration pass
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, out_amax=amax)
+    h = nv.empty_nvfp4(M, F)
+    h.global_scale.copy_(amax / 2688.0)
+    dy = torch.empty((M, F), dtype=torch.float32, device="cuda")
+    c = nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, requant=h, debug_y=dy)
+    torch.cuda.synchronize()
+    ref, _ = oracle.gemm(oa, ou, act=1, rows=rows, want_bf16=False)
+    y = dy.cpu().numpy()
+    assert normwise_err(y[rows].astype(np.float64), ref) <= GEMM_TOL
+    assert np.array_equal(host_bits(c)[rows], host_bits(dy.to(torch.bfloat16))[rows])
+    # requant of the sampled rows: the oracle's quantize of y with the given scale (row-local)
+    ha32 = np.float32(h.global_scale.item())
+    codes, scales, _ = oracle.quantize(np.ascontiguousarray(y[rows]), ha32)
+    assert np.array_equal(host_u8(h.codes)[rows], codes)
+    sc_dev = oracle.unswizzle(host_u8(h.scales), M, F // 16)
+    assert np.array_equal(sc_dev[rows], scales)
+    # down-projection over the NVFP4 hidden state (K = 14336: the long-K variant)
+    oh = (host_u8(h.codes), sc_dev, ha32)
+    _run_checked(h, qd, oh, od, rows=rows)
+
+
+def test_stack_layer_qkv_16384_tokens_sampled_rows():
+    """The QKV projection of the 16384-token linear stack (3072 -> 9216)."""
+    require_gpu()
+    M, N, K = 16384, 9216, 3072
+    qa, oa, qb, ob = _gemm_case(M, N, K, seed=61)
+    bias = syn.normal_bf16((N,), seed=62, std=0.02)
+    _run_checked(qa, qb, oa, ob, rows=_sampled_rows(M, 63), bias=bias)
+
+
 def test_epilogue_bias_gelu_modulate_gate_residual():
     require_gpu()
     M, N, K = 256, 512, 512
