@@ -10,8 +10,9 @@ One step = one pass of the whole path on seeded synthetic DiT-shaped inputs:
   4. nvfp4_kv_dequant of all 21 slots (ring order) back to bf16
 `value` is the W4A4 linear-layer throughput (2*M*N*K of step 2 per second of
 steps 1+2, device-timed with CUDA events); the KV rows are reported under
-"kv".  Each component is captured once in a CUDA graph and replayed, so the
-timed region holds device work only (no host launch gaps); `e2e` instead
+"kv".  The timed steps are captured as one CUDA graph, with the timing events
+between components as event-record nodes, so the timed region holds device
+work only (no host launch gaps); `e2e` instead
 calls the public Python API with host buffers every step.  The 681 MB bf16 output of step 4 overwrites L2 (126 MB) every step, so
 each step's GEMM and quantize read their inputs from HBM.
 
@@ -177,51 +178,59 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     v_out = torch.empty_like(k_out)
     stream = torch.cuda.current_stream()
 
-    # Each component of the step is captured once in a CUDA graph, so the
-    # timed loop replays device work back to back with no host gaps.
-    def capture(fn):
-        fn()  # warm: first calls set kernel attributes and resolve the driver entry point
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        return g
-
     do_quant = lambda: nv.quantize(a, out=qa, ws=ws_q)
     do_gemm = lambda: nv.gemm(qa, qw, out=c, bias=bias, ws=ws_g)
     do_append = [lambda s=s: cache.append(s, *chunks[s % n_chunks]) for s in range(S)]
     do_dequant = lambda: cache.dequant(ring, k_out, v_out)
-    if not args.direct:
-        g_quant, g_gemm = capture(do_quant), capture(do_gemm)
-        g_append = [capture(f) for f in do_append]
-        g_dequant = capture(do_dequant)
-        do_quant, do_gemm, do_dequant = g_quant.replay, g_gemm.replay, g_dequant.replay
-        do_append = [g.replay for g in g_append]
+    for f in (do_quant, do_gemm, do_append[0], do_dequant):
+        f()  # first calls set kernel attributes and resolve the driver entry point
     torch.cuda.synchronize()
 
     def step(i, ev=None):
         if ev:
-            ev[0].record(stream)
+            ev[0].record()  # the current (capture) stream
         do_quant()
         if ev:
-            ev[1].record(stream)
+            ev[1].record()  # the current (capture) stream
         do_gemm()
         if ev:
-            ev[2].record(stream)
+            ev[2].record()  # the current (capture) stream
         do_append[i % S]()
         if ev:
-            ev[3].record(stream)
+            ev[3].record()  # the current (capture) stream
         do_dequant()
         if ev:
-            ev[4].record(stream)
+            ev[4].record()  # the current (capture) stream
 
-    for i in range(args.warmup):
-        step(i)
+    # By default the warm-up steps and the timed steps are each captured as one
+    # CUDA graph (the timing events between the components become event-record
+    # nodes), so the timed region holds device work only: no host launch gaps
+    # and no per-component graph launches.  --direct launches every component
+    # on the stream instead.
+    evs = [[torch.cuda.Event(enable_timing=True, external=not args.direct) for _ in range(5)]
+           for _ in range(args.steps)]
+    if args.direct:
+        run_warmup = lambda: [step(i) for i in range(args.warmup)]
+        run_timed = lambda: [step(args.warmup + i, evs[i]) for i in range(args.steps)]
+        graphs = []
+    else:
+        g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_warm):
+            for i in range(args.warmup):
+                step(i)
+        with torch.cuda.graph(g_timed):
+            for i in range(args.steps):
+                step(args.warmup + i, evs[i])
+        run_warmup, run_timed = g_warm.replay, g_timed.replay
+        graphs = [g_warm, g_timed]
+    torch.cuda.synchronize()
+
+    run_warmup()
     torch.cuda.synchronize()
     code, _ = nv.read_device_error(ws_g)
     if code != nv.OK:
         raise RuntimeError(f"device error {code} during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
     clocks.start()
     time.sleep(0.3)
@@ -231,15 +240,13 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i, evs[i])
+    run_timed()
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    if not args.direct:
-        del g_quant, g_gemm, g_append, g_dequant
+    del graphs
 
     total_ms = t_start.elapsed_time(t_end)
     comp = np.zeros(4)
