@@ -132,12 +132,12 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def kernel_hash() -> str:
+def kernel_hash(files=("common.cuh", "gemm.cu")) -> str:
+    """Hash of the sources the GEMM kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_video_dit_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in files:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 

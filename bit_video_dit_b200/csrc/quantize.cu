@@ -111,19 +111,18 @@ struct Walk {
         srow = a.scales[t] + (SWZ ? (int64_t)(r >> 7) * a.tile_row + (r & 31) * 16 + ((r >> 5) & 3) * 4
                                   : (int64_t)r * a.scale_ld);
     }
-    // next run; branch-free (selects), so the unrolled loops stay straight lines
     __device__ __forceinline__ void next(const QuantArgs& a) {
-        const bool wrap = cr + 1 == a.upr;
-        cr = wrap ? 0 : cr + 1;
-        r += wrap ? 1 : 0;
-        xrow += wrap ? a.ld_bytes : 0;
-        crow += wrap ? a.code_ld : 0;
-        if (SWZ) {
-            // rows 32 apart share a 16-byte tile row; a new 128-row block starts a new tile row
-            const int64_t d = (r & 127) == 0 ? a.tile_row - 3 * 4 - 31 * 16 : ((r & 31) == 0 ? 4 - 31 * 16 : 16);
-            srow += wrap ? d : 0;
-        } else {
-            srow += wrap ? a.scale_ld : 0;
+        if (++cr == a.upr) {
+            cr = 0;
+            ++r;
+            xrow += a.ld_bytes;
+            crow += a.code_ld;
+            if (SWZ) {
+                // rows 32 apart share a 16-byte tile row; a new 128-row block starts a new tile row
+                srow += (r & 127) == 0 ? a.tile_row - 3 * 4 - 31 * 16 : ((r & 31) == 0 ? 4 - 31 * 16 : 16);
+            } else {
+                srow += a.scale_ld;
+            }
         }
     }
     __device__ __forceinline__ int nblk(const QuantArgs& a) const { return cr == a.upr - 1 ? a.last_nblk : 32; }
@@ -137,25 +136,14 @@ __device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool 
     const float amax_b = __uint_as_float(bmax << 16);
     const uint32_t code = d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, d6));
     const float inv = inv_tab[code];
-    // y = fl32(x * inv), two lanes per packed multiply (each lane rounds as a
-    // binary32 multiply), then E2M1 nearest-even, element 2i in the low nibble
-    const uint32_t wq[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    const float2 inv2 = make_float2(inv, inv);
-    const unsigned long long iv = *reinterpret_cast<const unsigned long long*>(&inv2);
-    uint32_t bytes[8];
+    float f[16];
+    bf16x8_to_f32(q0, f);
+    bf16x8_to_f32(q1, f + 8);
+    float y[16];
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const float2 xp = make_float2(__uint_as_float(wq[i] << 16), __uint_as_float(wq[i] & 0xFFFF0000u));
-        unsigned long long yp;
-        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(yp) : "l"(*reinterpret_cast<const unsigned long long*>(&xp)), "l"(iv));
-        const float2 y = *reinterpret_cast<const float2*>(&yp);
-        uint16_t b;
-        asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\tcvt.u16.u8 %0, t;\n\t}" : "=h"(b) : "f"(y.x), "f"(y.y));
-        bytes[i] = b;
-    }
+    for (int i = 0; i < 16; i++) y[i] = __fmul_rn(f[i], inv);
     // a flushed block (inv == 0) is +0 codes
-    const uint32_t c0 = inv == 0.0f ? 0u : (bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24));
-    const uint32_t c1 = inv == 0.0f ? 0u : (bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24));
+    const uint32_t c0 = inv == 0.0f ? 0u : e2m1x8(y), c1 = inv == 0.0f ? 0u : e2m1x8(y + 8);
     if (valid) {
         *reinterpret_cast<uint2*>(w.crow + w.cr * 256 + 8 * lane) = make_uint2(c0, c1);
         if (SWZ)
@@ -297,12 +285,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
         const float d6 = s_d6[t];
         const float* inv_tab = s_inv[t];
         Walk<SWZ> w = w0;
-        // a straight line over the held runs (stores predicated), so the
-        // compiler can overlap the encodes of neighbouring runs
 #pragma unroll
         for (int k = 0; k < kMaxRuns; k++) {
-            encode_block<SWZ>(w, lane, wb + k < we && lane < w.nblk(a), q[k][0], q[k][1], bm[k], d6, inv_tab);
-            w.next(a);
+            if (wb + k < we) {
+                encode_block<SWZ>(w, lane, lane < w.nblk(a), q[k][0], q[k][1], bm[k], d6, inv_tab);
+                w.next(a);
+            }
         }
         for (int g = wb + kMaxRuns; g < we; g++) {
             const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
