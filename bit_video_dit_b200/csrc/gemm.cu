@@ -48,11 +48,10 @@ constexpr int BK = 256;  // K elements per stage
 constexpr int BKB = BK / 2;  // bytes per row per stage (128: one swizzle atom row)
 constexpr int KB_PER_STAGE = BK / 64;
 // Block: producer, MMA, 4 epilogue warps and NC scale-copy warps.  Two
-// variants: NC = 3 (SFA | SFB rows 0..127 | 128..255; 288 threads, so at
-// most 168 registers a thread) for long K, where the mainloop dominates, and
-// NC = 2 (SFA | all of SFB; 256 threads, up to 255 registers) for short K,
-// where the epilogue has the registers to take the shared accumulator
-// columns in one go and the next tile starts sooner.
+// variants: NC = 3 (288 threads, so at most 168 registers a thread) for long
+// K, where the mainloop dominates, and NC = 2 (256 threads, up to 255
+// registers) for short K, where the epilogue has the registers to take the
+// shared accumulator columns in one go and the next tile starts sooner.
 constexpr int threads_for(int nc) { return (6 + nc) * 32; }
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int A_BYTES = BM * BKB;                  // 16 KB
@@ -317,20 +316,18 @@ drain:
 }
 
 // ---------------------------------------------------------------- copies ----
-// Copy warp `part` (NC = 3: 0 SFA, 1 SFB rows 0..127, 2 SFB rows 128..255;
-// NC = 2: 0 SFA, 1 both SFB halves) moves its 512-byte scale tiles of each
-// stage from shared memory into the stage's TMEM scale buffer (tcgen05.cp
-// 32x128b.warpx4: one tile into lanes 0..31, copied to all four lane
-// quarters), then commits to sf_full.
+// Copy warp `part` moves its share of the stage's twelve 512-byte scale tiles
+// (4 SFA, 4 SFB rows 0..127, 4 SFB rows 128..255; NC = 3: four each, NC = 2:
+// six each) from shared memory into the stage's TMEM scale buffer
+// (tcgen05.cp 32x128b.warpx4: one tile into lanes 0..31, copied to all four
+// lane quarters), then commits to sf_full.
 template <bool PAIR, int NC>
 __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, uint32_t tmem, int part) {
     using C = Cfg<PAIR>;
+    constexpr int PER = 3 * KB_PER_STAGE / NC;  // tiles per copy warp and stage: 6 (NC = 2) or 4 (NC = 3)
     volatile int* abort = &s->abort_flag;
     const uint32_t sf_s = smem_u32(ring) + A_BYTES + C::B_BYTES;  // SFA, then SFB rows 0..127, then 128..255
-    const uint64_t desc0 = smem_desc(sf_s + (uint32_t)part * SFA_BYTES, 0, 128, kLayoutNone);
-    const uint32_t tcol = tmem + (part == 0 ? SFA_COL : SFB_COL + 4u * (uint32_t)(part - 1));
-    const uint32_t kstride = part == 0 ? 4u : 8u;  // TMEM columns per k-block
-    const int tiles = (NC == 2 && part == 1) ? 2 : 1;  // NC = 2: part 1 copies both SFB halves
+    const uint64_t desc0 = smem_desc(sf_s, 0, 128, kLayoutNone);
     int first, step;
     tile_range<PAIR>(first, step);
     uint32_t it = 0;
@@ -345,21 +342,20 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
             }
             tc_fence_after();
             const uint64_t d = desc0 + (uint64_t)((st * C::STAGE_BYTES) >> 4);
-            const uint32_t t = tcol + (sb ? SF_COLS : 0u);
+            const uint32_t t = tmem + (sb ? SF_COLS : 0u);
 #pragma unroll
-            for (int kb = 0; kb < KB_PER_STAGE; kb++) {
-#pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    if (h < tiles) {
-                        // SFB rows 128..255 sit SFA_BYTES after rows 0..127 and go 4 columns right
-                        const uint32_t dst = t + kstride * kb + 4u * (uint32_t)h;
-                        const uint64_t src = d + kb * (512 >> 4) + (uint64_t)h * (SFA_BYTES >> 4);
-                        if (PAIR)
-                            tc_cp_32x128b_x4_pair(dst, src);
-                        else
-                            tc_cp_32x128b_x4(dst, src);
-                    }
-                }
+            for (int c = 0; c < PER; c++) {
+                // tile g of the stage: which = g / 4 (SFA, SFB rows 0..127, SFB rows
+                // 128..255: 2 KB apart in shared memory), k-block g % 4
+                const int g = part * PER + c;
+                const int which = g / KB_PER_STAGE, kb = g % KB_PER_STAGE;
+                const uint32_t dst =
+                    t + (which == 0 ? SFA_COL + 4u * kb : SFB_COL + 8u * kb + 4u * (uint32_t)(which - 1));
+                const uint64_t src = d + (uint64_t)((which * SFA_BYTES + kb * 512) >> 4);
+                if (PAIR)
+                    tc_cp_32x128b_x4_pair(dst, src);
+                else
+                    tc_cp_32x128b_x4(dst, src);
             }
             if (PAIR)
                 tc_commit_pair(&s->sf_full[sb], 0x1);
