@@ -28,6 +28,7 @@ _lib = None
 
 MODE_COMPUTE = 0
 MODE_GIVEN = 1
+MODE_SEARCH46 = 4  # OR-ed into the mode: adaptive scale search over {4, 6} (R18)
 
 
 def build(force: bool = False) -> str:
@@ -91,8 +92,9 @@ def lib():
             L.orc_gemm_exact_bf16.restype = ctypes.c_int
             L.orc_kv_slot_bytes.argtypes = [i64, i64, i64]
             L.orc_kv_slot_bytes.restype = i64
-            L.orc_kv_append.argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
-            L.orc_kv_append.restype = ctypes.c_int
+            for name in ("orc_kv_append", "orc_kv_append_search46"):
+                getattr(L, name).argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
+                getattr(L, name).restype = ctypes.c_int
             L.orc_kv_dequant.argtypes = [vp, vp, f32, i64, i64, i64, vp]
             _lib = L
     return _lib
@@ -141,11 +143,12 @@ def bf16_to_f32(h: int) -> float:
 
 # ---- array API ---------------------------------------------------------------
 
-def quantize(x: np.ndarray, alpha: float | None = None):
+def quantize(x: np.ndarray, alpha: float | None = None, search46: bool = False):
     """Quantize a 2-D array (uint16 bf16 bits or float32).
 
     Returns (codes uint8 [R, C/2], scales uint8 logical [R, C/16], alpha float32).
     alpha=None computes the tensor scale (R1); otherwise it is used as given.
+    search46 adds the per-block adaptive scale search over the targets {4, 6} (R18).
     """
     assert x.ndim == 2
     x = np.ascontiguousarray(x)
@@ -157,6 +160,8 @@ def quantize(x: np.ndarray, alpha: float | None = None):
     if alpha is not None:
         a[0] = np.float32(alpha)
         mode = MODE_GIVEN
+    if search46:
+        mode |= MODE_SEARCH46
     if x.dtype == np.uint16:
         fn = lib().orc_quantize_bf16
     elif x.dtype == np.float32:
@@ -265,14 +270,16 @@ def kv_slot_bytes(T: int, H: int, d: int) -> int:
     return int(lib().orc_kv_slot_bytes(T, H, d))
 
 
-def kv_append(x: np.ndarray):
-    """x: bf16 bits [T, H, d].  Returns (codes [T*H, d/2], scales [T*H, d/16], alpha)."""
+def kv_append(x: np.ndarray, search46: bool = False):
+    """x: bf16 bits [T, H, d].  Returns (codes [T*H, d/2], scales [T*H, d/16], alpha).
+    search46 adds the adaptive scale search over the targets {4, 6} (R18)."""
     T, H, d = x.shape
     x = np.ascontiguousarray(x)
     codes = np.zeros((T * H, d // 2), np.uint8)
     scales = np.zeros((T * H, d // 16), np.uint8)
     a = np.zeros(1, np.float32)
-    rc = lib().orc_kv_append(_p(x), T, H, d, d, _p(codes), _p(scales), _p(a))
+    fn = lib().orc_kv_append_search46 if search46 else lib().orc_kv_append
+    rc = fn(_p(x), T, H, d, d, _p(codes), _p(scales), _p(a))
     if rc != 0:
         raise ValueError(f"orc_kv_append failed ({rc})")
     return codes, scales, np.float32(a[0])

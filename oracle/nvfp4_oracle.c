@@ -38,6 +38,14 @@
  *      even (two roundings, in that order).
  *  R11 GELU is the tanh form.
  *  R15 KV: one a32 per (slot, K or V) over the whole chunk.
+ *  R18 adaptive scale search over the targets {4, 6} (optional mode): per
+ *      block, besides the standard encoding (block max aimed at 6: R3..R7),
+ *      encode with the block max aimed at 4 (r = fl32(amax_b / fl32(4 * a32)),
+ *      same rounding rules), and keep the one whose squared error is smaller;
+ *      a tie keeps the standard one.  The error is taken in binary32, in this
+ *      order: d = fl32(fl32(e2m1 * s) * a32) (R10's dequant product),
+ *      e = fl32(x - d), sum = fl32(sum + fl32(e * e)) over elements 0..15.
+ *      The tensor scale stays R1's.
  *  R16 KV slot = NVFP4 matrix of T*H rows x d columns, blocks along d, scales
  *      row-major (not swizzled).
  *
@@ -186,6 +194,41 @@ ORC_API unsigned orc_e4m3_encode(float r)
 /* ------------------------------------------------------------------------ */
 #define ORC_MODE_COMPUTE 0
 #define ORC_MODE_GIVEN 1
+#define ORC_MODE_SEARCH46 4 /* OR-ed into the mode: R18 */
+
+/* One candidate encoding of a 16-element block with the block max aimed at
+ * `target` (6: R3..R7; 4: R18): scale code and element codes. */
+static void encode_block(const float* xb, float amax_b, float a32, float target, uint8_t* sc, uint8_t* q)
+{
+    memset(q, 0, 16);
+    float d = target * a32;
+    float rb = amax_b / d;
+    *sc = (uint8_t)orc_e4m3_encode(rb); /* R3 */
+    float s = (float)orc_e4m3_value(*sc);
+    if (s != 0.0f) { /* R4 */
+        float denom = s * a32;
+        float inv = 1.0f / denom; /* R5 */
+        for (int i = 0; i < 16; i++) {
+            float y = xb[i] * inv;
+            q[i] = (uint8_t)orc_e2m1_encode(y); /* R6, R7 */
+        }
+    }
+}
+
+/* R18: binary32 squared error of a candidate, in the stated order. */
+static float block_sq_error(const float* xb, uint8_t sc, const uint8_t* q, float a32)
+{
+    float s = (float)orc_e4m3_value(sc);
+    float sum = 0.0f;
+    for (int i = 0; i < 16; i++) {
+        float e2 = (float)orc_e2m1_value(q[i]);
+        float dq = (e2 * s) * a32;
+        float e = xb[i] - dq;
+        float ee = e * e;
+        sum = sum + ee;
+    }
+    return sum;
+}
 
 /* x: binary32 [rows x cols], row stride ld elements.  cols % 16 == 0.
  * codes: [rows x cols/2] bytes (R8).  scales: logical [rows x cols/16] E4M3
@@ -196,6 +239,8 @@ ORC_API int orc_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t
     if (cols % 16 != 0 || ld < cols) return 1;
     init_tabs();
     float a32;
+    const int search = (mode & ORC_MODE_SEARCH46) != 0;
+    mode &= ~ORC_MODE_SEARCH46;
     if (mode == ORC_MODE_COMPUTE) {
         float amax = 0.0f;
         for (int64_t r = 0; r < rows; r++)
@@ -220,16 +265,13 @@ ORC_API int orc_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t
                 float amax_b = 0.0f;
                 for (int i = 0; i < 16; i++)
                     if (fabsf(xb[i]) > amax_b) amax_b = fabsf(xb[i]);
-                float d6 = 6.0f * a32;
-                float rb = amax_b / d6;
-                sc = (uint8_t)orc_e4m3_encode(rb); /* R3 */
-                float s = (float)orc_e4m3_value(sc);
-                if (s != 0.0f) { /* R4 */
-                    float denom = s * a32;
-                    float inv = 1.0f / denom; /* R5 */
-                    for (int i = 0; i < 16; i++) {
-                        float y = xb[i] * inv;
-                        q[i] = (uint8_t)orc_e2m1_encode(y); /* R6, R7 */
+                encode_block(xb, amax_b, a32, 6.0f, &sc, q);
+                if (search) {
+                    uint8_t sc4, q4[16];
+                    encode_block(xb, amax_b, a32, 4.0f, &sc4, q4);
+                    if (block_sq_error(xb, sc4, q4, a32) < block_sq_error(xb, sc, q, a32)) {
+                        sc = sc4;
+                        memcpy(q, q4, 16);
                     }
                 }
             }
@@ -488,6 +530,13 @@ ORC_API int orc_kv_append(const uint16_t* x, int64_t T, int64_t H, int64_t d, in
                           uint8_t* scales, float* alpha)
 {
     return orc_quantize_bf16(x, T * H, d, ld, ORC_MODE_COMPUTE, alpha, codes, scales);
+}
+
+/* As orc_kv_append with the R18 scale search. */
+ORC_API int orc_kv_append_search46(const uint16_t* x, int64_t T, int64_t H, int64_t d, int64_t ld, uint8_t* codes,
+                                   uint8_t* scales, float* alpha)
+{
+    return orc_quantize_bf16(x, T * H, d, ld, ORC_MODE_COMPUTE | ORC_MODE_SEARCH46, alpha, codes, scales);
 }
 
 ORC_API void orc_kv_dequant(const uint8_t* codes, const uint8_t* scales, float alpha, int64_t T, int64_t H,
