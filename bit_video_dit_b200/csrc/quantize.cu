@@ -128,24 +128,65 @@ struct Walk {
     __device__ __forceinline__ int nblk(const QuantArgs& a) const { return cr == a.upr - 1 ? a.last_nblk : 32; }
 };
 
-// encode one 16-element block (lane `lane` of the run at w) and store codes + scale
-template <bool SWZ>
-__device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool valid, const uint4& q0,
-                                             const uint4& q1, uint32_t bmax, float d6, const float* inv_tab) {
-    // s = E4M3(amax_b / (6 a32)); a zero tensor scale flushes every block
-    const float amax_b = __uint_as_float(bmax << 16);
-    const uint32_t code = d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, d6));
-    const float inv = inv_tab[code];
-    float f[16];
-    bf16x8_to_f32(q0, f);
-    bf16x8_to_f32(q1, f + 8);
+// Per-tensor constants of the encode: a32, 6 a32, 4 a32 (targets of the
+// block max) and the reciprocal 1 / (s * a32) of every E4M3 code s.
+struct EncodeConsts {
+    float a32, d6, d4;
+    const float* inv_tab;
+};
+
+// E2M1 codes of 16 binary32 ratios x * inv (two 32-bit words, element 2i in
+// the low nibble); a flushed block (inv == 0) is +0 codes.
+__device__ __forceinline__ uint2 encode16(const float* f, float inv) {
     float y[16];
 #pragma unroll
     for (int i = 0; i < 16; i++) y[i] = __fmul_rn(f[i], inv);
-    // a flushed block (inv == 0) is +0 codes
-    const uint32_t c0 = inv == 0.0f ? 0u : e2m1x8(y), c1 = inv == 0.0f ? 0u : e2m1x8(y + 8);
+    return make_uint2(inv == 0.0f ? 0u : e2m1x8(y), inv == 0.0f ? 0u : e2m1x8(y + 8));
+}
+
+// Squared error of an encoding of the block, binary32, in element order:
+// sum += (x - fl32(fl32(e2m1 * s) * a32))^2 (the dequant product, exact up to
+// the last multiply).
+__device__ __forceinline__ float block_sq_error(const float* f, uint2 c, float s, float a32) {
+    float sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 2; w++) {
+        const uint32_t word = w ? c.y : c.x;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float2 v = __half22float2(e2m1x2_to_half2((word >> (8 * j)) & 0xFFu));
+            const float d0 = __fmul_rn(__fmul_rn(v.x, s), a32), d1 = __fmul_rn(__fmul_rn(v.y, s), a32);
+            const float e0 = __fsub_rn(f[8 * w + 2 * j], d0), e1 = __fsub_rn(f[8 * w + 2 * j + 1], d1);
+            sum = __fadd_rn(sum, __fmul_rn(e0, e0));
+            sum = __fadd_rn(sum, __fmul_rn(e1, e1));
+        }
+    }
+    return sum;
+}
+
+// encode one 16-element block (lane `lane` of the run at w) and store codes +
+// scale.  SEARCH: also encode with the block max aimed at 4 instead of 6 and
+// keep that encoding when its squared error is smaller.
+template <bool SWZ, bool SEARCH>
+__device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool valid, const uint4& q0,
+                                             const uint4& q1, uint32_t bmax, const EncodeConsts& k) {
+    // s = E4M3(amax_b / (6 a32)); a zero tensor scale flushes every block
+    const float amax_b = __uint_as_float(bmax << 16);
+    uint32_t code = k.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, k.d6));
+    float f[16];
+    bf16x8_to_f32(q0, f);
+    bf16x8_to_f32(q1, f + 8);
+    uint2 c = encode16(f, k.inv_tab[code]);
+    if (SEARCH) {
+        const uint32_t code4 = k.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, k.d4));
+        const uint2 c4 = encode16(f, k.inv_tab[code4]);
+        if (block_sq_error(f, c4, e4m3_value(code4), k.a32) < block_sq_error(f, c, e4m3_value(code), k.a32)) {
+            code = code4;
+            c = c4;
+        }
+    }
     if (valid) {
-        *reinterpret_cast<uint2*>(w.crow + w.cr * 256 + 8 * lane) = make_uint2(c0, c1);
+        *reinterpret_cast<uint2*>(w.crow + w.cr * 256 + 8 * lane) = c;
         if (SWZ)
             w.srow[(int64_t)(w.cr * 8 + (lane >> 2)) * 512 + (lane & 3)] = (uint8_t)code;
         else
@@ -153,10 +194,10 @@ __device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool 
     }
 }
 
-template <bool SWZ>
+template <bool SWZ, bool SEARCH>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
     __shared__ uint32_t s_red[kQWarps];
-    __shared__ float s_d6[2];
+    __shared__ float s_d6[2], s_d4[2], s_a32[2];
     __shared__ float s_inv[2][256];
     __shared__ uint32_t s_total;
     __shared__ int s_ok;
@@ -267,7 +308,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
     }
     __syncthreads();
     // per tensor: inv[code] = 1 / (s * a32) for every E4M3 code (0 when s = 0
-    // or a32 = 0), then d6 = 6 a32
+    // or a32 = 0), then 6 a32 and 4 a32
     {
         const int tt = threadIdx.x >> 8, c = threadIdx.x & 255;
         if (tt < a.ntensors) {
@@ -276,19 +317,23 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             s_inv[tt][c] = (a32 == 0.0f || sv == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sv, a32));
         }
         __syncthreads();
-        if (threadIdx.x < a.ntensors) s_d6[threadIdx.x] = __fmul_rn(6.0f, s_d6[threadIdx.x]);
+        if (threadIdx.x < a.ntensors) {
+            const float a32 = s_d6[threadIdx.x];
+            s_a32[threadIdx.x] = a32;
+            s_d6[threadIdx.x] = __fmul_rn(6.0f, a32);
+            s_d4[threadIdx.x] = __fmul_rn(4.0f, a32);
+        }
         __syncthreads();
     }
 
     // ---- phase 2: encode
     {
-        const float d6 = s_d6[t];
-        const float* inv_tab = s_inv[t];
+        const EncodeConsts kc{s_a32[t], s_d6[t], s_d4[t], s_inv[t]};
         Walk<SWZ> w = w0;
 #pragma unroll
         for (int k = 0; k < kMaxRuns; k++) {
             if (wb + k < we) {
-                encode_block<SWZ>(w, lane, lane < w.nblk(a), q[k][0], q[k][1], bm[k], d6, inv_tab);
+                encode_block<SWZ, SEARCH>(w, lane, lane < w.nblk(a), q[k][0], q[k][1], bm[k], kc);
                 w.next(a);
             }
         }
@@ -297,7 +342,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             const bool valid = lane < w.nblk(a);
             const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
             const uint32_t mm = __vmaxu2(absmax_bits8(v0), absmax_bits8(v1));
-            encode_block<SWZ>(w, lane, valid, v0, v1, max(mm & 0xFFFFu, mm >> 16), d6, inv_tab);
+            encode_block<SWZ, SEARCH>(w, lane, valid, v0, v1, max(mm & 0xFFFFu, mm >> 16), kc);
             w.next(a);
         }
     }
@@ -449,7 +494,7 @@ static nvfp4_status launch_status() {
 // one fused, cooperative launch over one or two tensors of the same shape
 static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t rows, int64_t cols, int64_t ld,
                                   void* const* codes, void* const* scales, float* const* gscale, bool given,
-                                  bool swizzled, void* workspace, cudaStream_t stream) {
+                                  bool swizzled, bool search, void* workspace, cudaStream_t stream) {
     QuantArgs a{};
     for (int t = 0; t < ntensors; t++) {
         a.x[t] = static_cast<const uint8_t*>(x[t]);
@@ -482,8 +527,9 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, swizzled ? quantize_fused_kernel<true> : quantize_fused_kernel<false>, a) !=
-        cudaSuccess) {
+    void (*kern)(QuantArgs) = swizzled ? (search ? quantize_fused_kernel<true, true> : quantize_fused_kernel<true, false>)
+                                       : (search ? quantize_fused_kernel<false, true> : quantize_fused_kernel<false, false>);
+    if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
     }
@@ -497,7 +543,7 @@ using namespace nvfp4;
 extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
                                        void* scales, float* global_scale, unsigned flags, void* workspace,
                                        size_t ws_bytes, nvfp4_stream_t stream) {
-    if (flags & ~(NVFP4_Q_GIVEN_GLOBAL | NVFP4_Q_ROWMAJOR_SCALES)) return NVFP4_ERR_INVALID_ARG;
+    if (flags & ~(NVFP4_Q_GIVEN_GLOBAL | NVFP4_Q_ROWMAJOR_SCALES | NVFP4_Q_SCALE_SEARCH)) return NVFP4_ERR_INVALID_ARG;
     if (rows < 0 || cols <= 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
     if (cols % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
     if (rows > ((int64_t)1 << 31) || cols > ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED;
@@ -513,7 +559,8 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     void* ss[1] = {scales};
     float* gs[1] = {global_scale};
     return quantize_impl(1, xs, rows, cols, ld, cs, ss, gs, (flags & NVFP4_Q_GIVEN_GLOBAL) != 0,
-                         (flags & NVFP4_Q_ROWMAJOR_SCALES) == 0, workspace, (cudaStream_t)stream);
+                         (flags & NVFP4_Q_ROWMAJOR_SCALES) == 0, (flags & NVFP4_Q_SCALE_SEARCH) != 0, workspace,
+                         (cudaStream_t)stream);
 }
 
 static nvfp4_status check_cache(const nvfp4_kv_cache* c) {
@@ -522,6 +569,7 @@ static nvfp4_status check_cache(const nvfp4_kv_cache* c) {
         return NVFP4_ERR_INVALID_ARG;
     if (c->n_slots <= 0 || c->tokens_per_slot <= 0 || c->heads <= 0 || c->head_dim <= 0) return NVFP4_ERR_INVALID_ARG;
     if (c->head_dim % 16 != 0) return NVFP4_ERR_UNSUPPORTED;
+    if (c->flags & ~NVFP4_KV_SCALE_SEARCH) return NVFP4_ERR_INVALID_ARG;
     const int64_t e = (int64_t)c->tokens_per_slot * c->heads * c->head_dim;
     if (e % 64 != 0 || e > ((int64_t)1 << 40)) return NVFP4_ERR_UNSUPPORTED;
     if (!aligned16(c->k_codes) || !aligned16(c->k_scales) || !aligned16(c->v_codes) || !aligned16(c->v_scales) ||
@@ -549,7 +597,8 @@ extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slo
     void* ss[2] = {static_cast<uint8_t*>(cache->k_scales) + (int64_t)slot * (e / 16),
                    static_cast<uint8_t*>(cache->v_scales) + (int64_t)slot * (e / 16)};
     float* gs[2] = {cache->k_global + slot, cache->v_global + slot};
-    return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, workspace, (cudaStream_t)stream);
+    return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, (cache->flags & NVFP4_KV_SCALE_SEARCH) != 0,
+                         workspace, (cudaStream_t)stream);
 }
 
 extern "C" nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n,

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
 OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT = range(4)
-Q_COMPUTE_GLOBAL, Q_GIVEN_GLOBAL, Q_ROWMAJOR_SCALES = 0, 1, 2
+Q_COMPUTE_GLOBAL, Q_GIVEN_GLOBAL, Q_ROWMAJOR_SCALES, Q_SCALE_SEARCH = 0, 1, 2, 4
+KV_SCALE_SEARCH = 1
 ACT_NONE, ACT_GELU_TANH = 0, 1
 DBG_SKIP_LOADS = 1
 
@@ -50,7 +51,7 @@ class CKVCache(ctypes.Structure):
     _fields_ = [("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
                 ("v_scales", ctypes.c_void_p), ("k_global", ctypes.c_void_p), ("v_global", ctypes.c_void_p),
                 ("n_slots", ctypes.c_int32), ("tokens_per_slot", ctypes.c_int32), ("heads", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32)]
+                ("head_dim", ctypes.c_int32), ("flags", ctypes.c_uint32)]
 
 
 _lib = None
@@ -166,7 +167,8 @@ def empty_nvfp4(rows: int, cols: int, device="cuda", swizzled: bool = True) -> N
 
 
 def quantize(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, out: NVFP4Tensor | None = None,
-             rowmajor_scales: bool = False, ws: torch.Tensor | None = None, stream=None) -> NVFP4Tensor:
+             rowmajor_scales: bool = False, scale_search: bool = False, ws: torch.Tensor | None = None,
+             stream=None) -> NVFP4Tensor:
     """bf16 [rows, cols] (row stride x.stride(0)) -> NVFP4Tensor.  With
     global_scale given, that tensor scale is used (delayed scaling); otherwise
     it is computed as amax / 2688 and written to out.global_scale."""
@@ -176,7 +178,7 @@ def quantize(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, out: 
     rows, cols = x.shape
     if out is None:
         out = empty_nvfp4(rows, cols, x.device, swizzled=not rowmajor_scales)
-    flags = Q_ROWMAJOR_SCALES if rowmajor_scales else 0
+    flags = (Q_ROWMAJOR_SCALES if rowmajor_scales else 0) | (Q_SCALE_SEARCH if scale_search else 0)
     if global_scale is not None:
         out.global_scale.copy_(global_scale.reshape(1))
         flags |= Q_GIVEN_GLOBAL
@@ -226,8 +228,10 @@ class KVCache:
     K and V each stored as codes + row-major E4M3 scales + one binary32 tensor
     scale per slot (9/16 byte per element per tensor)."""
 
-    def __init__(self, n_slots: int, tokens: int, heads: int, head_dim: int, device="cuda"):
+    def __init__(self, n_slots: int, tokens: int, heads: int, head_dim: int, device="cuda",
+                 scale_search: bool = False):
         self.n_slots, self.tokens, self.heads, self.head_dim = n_slots, tokens, heads, head_dim
+        self.flags = KV_SCALE_SEARCH if scale_search else 0
         e = tokens * heads * head_dim
         self.slot_elems = e
         u8 = torch.uint8
@@ -243,7 +247,7 @@ class KVCache:
     def c(self) -> CKVCache:
         return CKVCache(self.k_codes.data_ptr(), self.k_scales.data_ptr(), self.v_codes.data_ptr(),
                         self.v_scales.data_ptr(), self.k_global.data_ptr(), self.v_global.data_ptr(),
-                        self.n_slots, self.tokens, self.heads, self.head_dim)
+                        self.n_slots, self.tokens, self.heads, self.head_dim, self.flags)
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in

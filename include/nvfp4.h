@@ -115,6 +115,14 @@ nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int
 #define NVFP4_Q_COMPUTE_GLOBAL 0u /* compute a32 = amax / 2688 and write *global_scale */
 #define NVFP4_Q_GIVEN_GLOBAL 1u   /* read a32 from *global_scale (delayed scaling) */
 #define NVFP4_Q_ROWMAJOR_SCALES 2u /* write row-major scales instead of the swizzled tiles */
+/* Adaptive scale search over the block-max targets {4, 6} ([RN] "NVFP4 训练的
+ *工程细节" and "推理底座": "adaptive scale search" / "adaptive scale 选择"):
+ * per 16-element block, also encode with the block max aimed at 4, i.e.
+ * s4 = E4M3(amax_b / fl32(4 * a32)), and keep that encoding when its squared
+ * error is smaller.  The error is binary32, summed over the block's elements
+ * in order: sum += (x - fl32(fl32(e2m1 * s) * a32))^2; a tie keeps the
+ * standard encoding.  The tensor scale a32 is unchanged. */
+#define NVFP4_Q_SCALE_SEARCH 4u
 
 /* x_bf16: bf16 [rows x cols], row stride ld elements (ld >= cols, ld % 8 == 0).
  * cols % 64 == 0, rows >= 0.
@@ -223,11 +231,15 @@ typedef struct {
     float* k_global; /* [n_slots] device binary32 */
     float* v_global; /* [n_slots] device binary32 */
     int32_t n_slots, tokens_per_slot, heads, head_dim;
+    uint32_t flags; /* NVFP4_KV_* (0: the standard encoding) */
 } nvfp4_kv_cache;
+
+#define NVFP4_KV_SCALE_SEARCH 1u /* appends use the scale search of NVFP4_Q_SCALE_SEARCH */
 
 /* Quantizes one chunk's K and V (bf16, token-major [T][H][d], contiguous)
  * in place into slot `slot`: one tensor scale per (slot, K|V) = amax / 2688
- * over the whole chunk, then the quantize rule above with row-major scales.
+ * over the whole chunk, then the quantize rule above with row-major scales
+ * (with the scale search when cache->flags has NVFP4_KV_SCALE_SEARCH).
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_KV_APPEND, T*H, 0, d) bytes.
  * One cooperative launch covering K and V (as nvfp4_quantize). */
 nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,

@@ -86,3 +86,29 @@ def test_out_of_range_slot_is_reported():
     assert bool((ko[0] == ko[2]).all())
     code, _ = nv.read_device_error(cache.ws_dequant)  # the record was cleared
     assert code == nv.OK
+
+
+def test_full_chunk_append_with_scale_search():
+    """KV append with the adaptive scale search ({4, 6}) on the full chunk: codes,
+    scales and tensor scales bit for bit against the oracle, and the bf16 dequant."""
+    require_gpu()
+    T, H, d = syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    cache = nv.KVCache(2, T, H, d, scale_search=True)
+    k, v = syn.kv_chunk_bf16(T, H, d, seed=4)
+    cache.append(1, dev_bf16(k), dev_bf16(v))
+    torch.cuda.synchronize()
+    for which, x in ((0, k), (1, v)):
+        codes, scales, a32 = oracle.kv_append(x, search46=True)
+        c = cache.k_codes if which == 0 else cache.v_codes
+        s = cache.k_scales if which == 0 else cache.v_scales
+        g = cache.k_global if which == 0 else cache.v_global
+        assert f32_bits(g[1].cpu().numpy()) == f32_bits(a32)
+        assert np.array_equal(host_u8(c[1]), codes.reshape(-1))
+        assert np.array_equal(host_u8(s[1]), scales.reshape(-1))
+    slots = torch.tensor([1], dtype=torch.int32, device="cuda")
+    ko, vo = cache.dequant(slots)
+    torch.cuda.synchronize()
+    for x, o in ((k, ko), (v, vo)):
+        codes, scales, a32 = oracle.kv_append(x, search46=True)
+        want = oracle.kv_dequant(codes, scales, a32, T, H, d)
+        assert np.array_equal(host_bits(o[0]), want)

@@ -13,7 +13,7 @@ from .gpu_util import dev_bf16, f32_bits, host_u8, require_gpu
 pytestmark = pytest.mark.gpu
 
 
-def _check(x_bits, *, ld=None, alpha=None, rowmajor=False):
+def _check(x_bits, *, ld=None, alpha=None, rowmajor=False, search=False):
     require_gpu()
     rows, cols = x_bits.shape
     if ld is None:
@@ -23,9 +23,9 @@ def _check(x_bits, *, ld=None, alpha=None, rowmajor=False):
         buf[:, :cols] = x_bits
         xd = dev_bf16(buf)[:, :cols]
     gs = None if alpha is None else torch.tensor([alpha], dtype=torch.float32, device="cuda")
-    q = nv.quantize(xd, global_scale=gs, rowmajor_scales=rowmajor)
+    q = nv.quantize(xd, global_scale=gs, rowmajor_scales=rowmajor, scale_search=search)
     torch.cuda.synchronize()
-    codes, scales, a32 = oracle.quantize(x_bits, alpha)
+    codes, scales, a32 = oracle.quantize(x_bits, alpha, search46=search)
     assert f32_bits(q.global_scale.cpu().numpy()) == f32_bits(a32)
     gc = host_u8(q.codes)
     bad = np.argwhere(gc != codes)
@@ -78,3 +78,25 @@ def test_zero_rows_is_a_noop():
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     q = nv.quantize(x)
     assert q.codes.numel() == 0
+
+
+# ---- adaptive scale search over the targets {4, 6} (NVFP4_Q_SCALE_SEARCH) ----
+
+def test_scale_search_activation_full_size():
+    q = _check(syn.activations_bf16(4096, 3072, seed=2), search=True)
+    # it does pick the target-4 encoding for part of the blocks
+    std = nv.quantize(dev_bf16(syn.activations_bf16(4096, 3072, seed=2)))
+    torch.cuda.synchronize()
+    frac = (q.scales != std.scales).float().mean().item()
+    assert 0.01 < frac < 0.99
+
+
+@pytest.mark.parametrize("rows,cols,ld,rowmajor", [(200, 320, None, False), (129, 576, 640, True), (1, 64, None, False)])
+def test_scale_search_ragged(rows, cols, ld, rowmajor):
+    _check(syn.activations_bf16(rows, cols, seed=rows * 7 + cols), ld=ld, rowmajor=rowmajor, search=True)
+
+
+def test_scale_search_given_scale_and_zero_tensor():
+    x = syn.normal_bf16((128, 256), seed=5)
+    _check(x, alpha=0.01, search=True)
+    _check(np.zeros((64, 128), np.uint16), search=True)
