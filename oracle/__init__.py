@@ -92,6 +92,10 @@ def lib():
             L.orc_gemm_exact_bf16.restype = ctypes.c_int
             L.orc_kv_slot_bytes.argtypes = [i64, i64, i64]
             L.orc_kv_slot_bytes.restype = i64
+            L.orc_ln_modulate.argtypes = [vp, i64, i64, i64, vp, vp, f32, vp]
+            L.orc_ln_modulate.restype = ctypes.c_int
+            L.orc_ln_modulate_quantize.argtypes = [vp, i64, i64, i64, vp, vp, f32, ctypes.c_int, vp, vp, vp]
+            L.orc_ln_modulate_quantize.restype = ctypes.c_int
             for name in ("orc_kv_append", "orc_kv_append_search46"):
                 getattr(L, name).argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
                 getattr(L, name).restype = ctypes.c_int
@@ -290,3 +294,39 @@ def kv_dequant(codes, scales, alpha, T: int, H: int, d: int) -> np.ndarray:
     lib().orc_kv_dequant(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)), float(alpha),
                          T, H, d, _p(out))
     return out
+
+
+def ln_modulate(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6) -> np.ndarray:
+    """LayerNorm of each row of bf16 bits x [R, C] (no affine), then
+    m = h * (1 + scale) + shift (bf16 bits [C] or None), binary32 (R19)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    R, C = x.shape
+    m = np.zeros((R, C), np.float32)
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.uint16)
+    sh = None if shift is None else np.ascontiguousarray(shift, dtype=np.uint16)
+    rc = lib().orc_ln_modulate(_p(x), R, C, C, None if sc is None else _p(sc), None if sh is None else _p(sh),
+                               float(eps), _p(m))
+    if rc != 0:
+        raise ValueError(f"orc_ln_modulate failed ({rc})")
+    return m
+
+
+def ln_modulate_quantize(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6, alpha: float | None = None):
+    """ln_modulate then quantize (R19, R1..R8).  Returns (codes, logical scales, alpha)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    R, C = x.shape
+    codes = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    a = np.zeros(1, np.float32)
+    mode = MODE_COMPUTE
+    if alpha is not None:
+        a[0] = np.float32(alpha)
+        mode = MODE_GIVEN
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.uint16)
+    sh = None if shift is None else np.ascontiguousarray(shift, dtype=np.uint16)
+    rc = lib().orc_ln_modulate_quantize(_p(x), R, C, C, None if sc is None else _p(sc),
+                                        None if sh is None else _p(sh), float(eps), mode, _p(a), _p(codes),
+                                        _p(scales))
+    if rc != 0:
+        raise ValueError(f"orc_ln_modulate_quantize failed ({rc})")
+    return codes, scales, np.float32(a[0])

@@ -46,6 +46,8 @@
  *      order: d = fl32(fl32(e2m1 * s) * a32) (R10's dequant product),
  *      e = fl32(x - d), sum = fl32(sum + fl32(e * e)) over elements 0..15.
  *      The tensor scale stays R1's.
+ *  R19 LayerNorm + adaLN modulate before the quantize (optional path): see
+ *      orc_ln_modulate for the operations, their binary32 order and eps.
  *  R16 KV slot = NVFP4 matrix of T*H rows x d columns, blocks along d, scales
  *      row-major (not swizzled).
  *
@@ -543,4 +545,75 @@ ORC_API void orc_kv_dequant(const uint8_t* codes, const uint8_t* scales, float a
                             int64_t d, uint16_t* out)
 {
     orc_dequant_bf16(codes, scales, alpha, T * H, d, out);
+}
+
+/* ------------------------------------------------------------------------ */
+/* LayerNorm + adaLN modulate + quantize (the step before the linear layer)  */
+/* ------------------------------------------------------------------------ */
+/* R19: per row r of x (bf16 [rows x cols], cols % 16 == 0), in binary32:
+ *   mean = S1 / cols, var = S2 / cols with S1 = sum x, S2 = sum fl32(x - mean)^2,
+ *   rstd = 1 / sqrt(var + eps)  (each operation correctly rounded),
+ *   m = fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale[c])) + shift[c]
+ *   (scale, shift bf16 [cols] or absent: 0),
+ * then m is quantized as a binary32 tensor (R1..R8).  Sums run in a fixed
+ * order: 32 partial sums, partial j over the 16-element blocks j, j+32,
+ * j+64, ... of the row (blocks and their elements in order), then combined
+ * by a butterfly: for o = 16, 8, 4, 2, 1, partial[j] = partial[j] +
+ * partial[j ^ o] (all j at once). */
+static float row_sum32(const float* v, int64_t cols)
+{
+    float part[32], next[32];
+    const int64_t nb = cols / 16;
+    for (int j = 0; j < 32; j++) {
+        float s = 0.0f;
+        for (int64_t b = j; b < nb; b += 32)
+            for (int i = 0; i < 16; i++) s = s + v[b * 16 + i];
+        part[j] = s;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        for (int j = 0; j < 32; j++) next[j] = part[j] + part[j ^ o];
+        memcpy(part, next, sizeof part);
+    }
+    return part[0];
+}
+
+ORC_API int orc_ln_modulate(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, const uint16_t* scale,
+                            const uint16_t* shift, float eps, float* m)
+{
+    if (cols % 16 != 0 || ld < cols) return 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t r = 0; r < rows; r++) {
+        float* xr = (float*)malloc((size_t)cols * sizeof(float));
+        float* dr = (float*)malloc((size_t)cols * sizeof(float));
+        for (int64_t c = 0; c < cols; c++) xr[c] = orc_bf16_to_f32(x[r * ld + c]);
+        const float n = (float)cols;
+        const float mean = row_sum32(xr, cols) / n;
+        for (int64_t c = 0; c < cols; c++) {
+            float d = xr[c] - mean;
+            dr[c] = d * d;
+        }
+        const float var = row_sum32(dr, cols) / n;
+        const float rstd = 1.0f / sqrtf(var + eps);
+        for (int64_t c = 0; c < cols; c++) {
+            float h = (xr[c] - mean) * rstd;
+            float g = 1.0f + (scale ? orc_bf16_to_f32(scale[c]) : 0.0f);
+            float t = h * g;
+            m[r * cols + c] = t + (shift ? orc_bf16_to_f32(shift[c]) : 0.0f);
+        }
+        free(xr);
+        free(dr);
+    }
+    return 0;
+}
+
+ORC_API int orc_ln_modulate_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                     const uint16_t* scale, const uint16_t* shift, float eps, int mode, float* alpha,
+                                     uint8_t* codes, uint8_t* scales)
+{
+    float* m = (float*)malloc((size_t)(rows * cols) * sizeof(float) + 1);
+    if (!m) return 2;
+    int rc = orc_ln_modulate(x, rows, cols, ld, scale, shift, eps, m);
+    if (rc == 0) rc = orc_quantize_f32(m, rows, cols, cols, mode, alpha, codes, scales);
+    free(m);
+    return rc;
 }
