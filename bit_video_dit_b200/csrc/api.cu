@@ -40,7 +40,6 @@ extern "C" size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int swizzled) {
 }
 
 extern "C" size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k) {
-    (void)m;
     (void)n;
     (void)k;
     switch (op) {
@@ -48,6 +47,8 @@ extern "C" size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
         case NVFP4_OP_KV_APPEND: return kWsQuantize;
         case NVFP4_OP_GEMM:
         case NVFP4_OP_KV_DEQUANT: return kWsControl;
+        case NVFP4_OP_LN_QUANTIZE:  // control block, then (mean, rstd) per row
+            return kWsControl + (size_t)(m > 0 ? m : 0) * 8;
     }
     return kWsQuantize;
 }

@@ -69,6 +69,12 @@ struct QuantArgs {
     int runs_per_tensor;
     int ntensors;
     int given;
+    // LayerNorm + modulate ahead of the quantize (LN kernels only): per-row
+    // (mean, rstd) and the bf16 [cols] modulation vectors (NULL: 0)
+    const float2* ln_stats;
+    const __nv_bfloat16* mod_scale;
+    const __nv_bfloat16* mod_shift;
+    int cols;
     uint32_t* ctl;
     DevError* err;
     uint64_t limit_ns;
@@ -168,14 +174,10 @@ __device__ __forceinline__ float block_sq_error(const float* f, uint2 c, float s
 // scale.  SEARCH: also encode with the block max aimed at 4 instead of 6 and
 // keep that encoding when its squared error is smaller.
 template <bool SWZ, bool SEARCH>
-__device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool valid, const uint4& q0,
-                                             const uint4& q1, uint32_t bmax, const EncodeConsts& k) {
+__device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool valid, const float* f, float amax_b,
+                                             const EncodeConsts& k) {
     // s = E4M3(amax_b / (6 a32)); a zero tensor scale flushes every block
-    const float amax_b = __uint_as_float(bmax << 16);
     uint32_t code = k.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, k.d6));
-    float f[16];
-    bf16x8_to_f32(q0, f);
-    bf16x8_to_f32(q1, f + 8);
     uint2 c = encode16(f, k.inv_tab[code]);
     if (SEARCH) {
         const uint32_t code4 = k.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, k.d4));
@@ -194,8 +196,58 @@ __device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool 
     }
 }
 
-template <bool SWZ, bool SEARCH>
+// The 16 binary32 values of the lane's block of the run at w: the bf16 input,
+// or with LN its LayerNorm + modulate, in this order and rounding:
+// m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift).
+template <bool LN, bool SWZ>
+__device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>& w, int lane, bool valid,
+                                             const uint4& q0, const uint4& q1, float* f) {
+    bf16x8_to_f32(q0, f);
+    bf16x8_to_f32(q1, f + 8);
+    if (LN) {
+        const float2 st = __ldg(a.ln_stats + w.r);
+        const int c0 = w.cr * 512 + lane * 16;
+        float sc[16], sh[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) sc[i] = sh[i] = 0.0f;
+        if (valid && a.mod_scale) {
+            const uint4* p = reinterpret_cast<const uint4*>(a.mod_scale + c0);
+            bf16x8_to_f32(__ldg(p), sc);
+            bf16x8_to_f32(__ldg(p + 1), sc + 8);
+        }
+        if (valid && a.mod_shift) {
+            const uint4* p = reinterpret_cast<const uint4*>(a.mod_shift + c0);
+            bf16x8_to_f32(__ldg(p), sh);
+            bf16x8_to_f32(__ldg(p + 1), sh + 8);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const float h = __fmul_rn(__fsub_rn(f[i], st.x), st.y);
+            f[i] = __fadd_rn(__fmul_rn(h, __fadd_rn(1.0f, sc[i])), sh[i]);
+        }
+    }
+}
+
+// a block's |x| max as an order-preserving 32-bit key: the bf16 magnitude
+// bits (LN: the binary32 magnitude bits of the modulated values)
+template <bool LN>
+__device__ __forceinline__ uint32_t block_max_key(const uint4& q0, const uint4& q1, const float* f) {
+    if (LN) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; i++) mx = fmaxf(mx, fabsf(f[i]));
+        return __float_as_uint(mx);
+    }
+    const uint32_t mm = __vmaxu2(absmax_bits8(q0), absmax_bits8(q1));
+    return max(mm & 0xFFFFu, mm >> 16);
+}
+
+template <bool LN>
+__device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float(LN ? key : key << 16); }
+
+template <bool SWZ, bool SEARCH, bool LN>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
+    constexpr int kRuns = LN ? 4 : kMaxRuns;  // LN needs registers for the transform
     __shared__ uint32_t s_red[kQWarps];
     __shared__ float s_d6[2], s_d4[2], s_a32[2];
     __shared__ float s_inv[2][256];
@@ -216,12 +268,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
     w0.seek(a, t, min(wb, a.runs_per_tensor - 1));
 
     // ---- phase 1: this warp's runs wb .. we-1 of tensor t, one block per lane
-    uint4 q[kMaxRuns][2];
-    uint32_t bm[kMaxRuns];  // the lane's block max (bf16 magnitude bits) per run
+    uint4 q[kRuns][2];
+    uint32_t bm[kRuns];  // the lane's block max key per run
     {
         Walk<SWZ> w = w0;
 #pragma unroll
-        for (int k = 0; k < kMaxRuns; k++) {
+        for (int k = 0; k < kRuns; k++) {
             const bool have = wb + k < we;
             const bool valid = have && lane < w.nblk(a);
             const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
@@ -230,41 +282,60 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             if (have) w.next(a);
         }
     }
-    uint32_t m = 0;  // two bf16 magnitudes per word
+    uint32_t m = 0;  // the lane's max key over its runs
+    if constexpr (!LN) {
+        // blocks past the data were loaded as zeros: key 0
 #pragma unroll
-    for (int k = 0; k < kMaxRuns; k++) {
-        const uint32_t mm = __vmaxu2(absmax_bits8(q[k][0]), absmax_bits8(q[k][1]));
-        bm[k] = max(mm & 0xFFFFu, mm >> 16);
-        m = max(m, bm[k]);
+        for (int k = 0; k < kRuns; k++) {
+            const uint32_t mm = __vmaxu2(absmax_bits8(q[k][0]), absmax_bits8(q[k][1]));
+            bm[k] = max(mm & 0xFFFFu, mm >> 16);
+            m = max(m, bm[k]);
+        }
+    } else {
+        Walk<SWZ> w = w0;
+#pragma unroll
+        for (int k = 0; k < kRuns; k++) {
+            float f[16];
+            const bool have = wb + k < we;
+            block_values<LN>(a, w, lane, have && lane < w.nblk(a), q[k][0], q[k][1], f);
+            bm[k] = have && lane < w.nblk(a) ? block_max_key<LN>(q[k][0], q[k][1], f) : 0u;
+            m = max(m, bm[k]);
+            if (have) w.next(a);
+        }
     }
     if (threadIdx.x == 0) s_ok = 1;
     if (!a.given) {
         {
             Walk<SWZ> w = w0;
-            for (int k = 0; k < kMaxRuns && wb + k < we; k++) w.next(a);
-            for (int g = wb + kMaxRuns; g < we; g++) {
+            for (int k = 0; k < kRuns && wb + k < we; k++) w.next(a);
+            for (int g = wb + kRuns; g < we; g++) {
                 const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
                 const bool valid = lane < w.nblk(a);
-                const uint32_t mm = __vmaxu2(absmax_bits8(ld_stream16_if(src, valid)),
-                                             absmax_bits8(ld_stream16_if(src + 16, valid)));
-                m = max(m, max(mm & 0xFFFFu, mm >> 16));
+                const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
+                float f[16];
+                block_values<LN>(a, w, lane, valid, v0, v1, f);
+                if (valid) m = max(m, block_max_key<LN>(v0, v1, f));
                 w.next(a);
             }
         }
-        // one word per lane: tensor-1 max in the high half, tensor-0 in the low
-        m = t ? (m << 16) : m;
+        // one word per lane: for two tensors, tensor-1 max in the high half,
+        // tensor-0 in the low (16-bit keys); LN has one tensor and 32-bit keys
+        if (!LN) m = t ? (m << 16) : m;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+            m = LN ? max(m, other) : __vmaxu2(m, other);
+        }
         if (lane == 0) s_red[warp] = m;
         __syncthreads();
         if (threadIdx.x == 0) {
             uint32_t c = 0;
 #pragma unroll
-            for (int i = 0; i < kQWarps; i++) c = __vmaxu2(c, s_red[i]);
+            for (int i = 0; i < kQWarps; i++) c = LN ? max(c, s_red[i]) : __vmaxu2(c, s_red[i]);
             uint32_t* cnt = a.ctl + kCtlCount + par;
             uint32_t* mx = a.ctl + kCtlMax + 2 * par;
-            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(c & 0xFFFFu) : "memory");
-            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx + 1), "r"(c >> 16) : "memory");
+            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(LN ? c : c & 0xFFFFu) : "memory");
+            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx + 1), "r"(LN ? 0u : c >> 16) : "memory");
             uint32_t old;
             // acquire too: the last CTA to arrive reads the maxima without polling
             asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
@@ -283,13 +354,13 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             uint32_t t0, t1;
             asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t0) : "l"(mx) : "memory");
             asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t1) : "l"(mx + 1) : "memory");
-            s_total = (t1 << 16) | t0;
+            s_total = LN ? t0 : ((t1 << 16) | t0);
         }
         __syncthreads();
         if (!s_ok) return;
         if (threadIdx.x < a.ntensors) {
-            const uint32_t bits = threadIdx.x ? (s_total >> 16) : (s_total & 0xFFFFu);
-            const float a32 = __fdiv_rn(__uint_as_float(bits << 16), 2688.0f);  // amax / (6 * 448)
+            const uint32_t key = LN ? s_total : (threadIdx.x ? (s_total >> 16) : (s_total & 0xFFFFu));
+            const float a32 = __fdiv_rn(key_value<LN>(key), 2688.0f);  // amax / (6 * 448)
             s_d6[threadIdx.x] = a32;  // a32 for now; the table below needs it
             if (blockIdx.x == 0) *(threadIdx.x ? a.gscale[1] : a.gscale[0]) = a32;
         }
@@ -331,18 +402,22 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
         const EncodeConsts kc{s_a32[t], s_d6[t], s_d4[t], s_inv[t]};
         Walk<SWZ> w = w0;
 #pragma unroll
-        for (int k = 0; k < kMaxRuns; k++) {
+        for (int k = 0; k < kRuns; k++) {
             if (wb + k < we) {
-                encode_block<SWZ, SEARCH>(w, lane, lane < w.nblk(a), q[k][0], q[k][1], bm[k], kc);
+                const bool valid = lane < w.nblk(a);
+                float f[16];
+                block_values<LN>(a, w, lane, valid, q[k][0], q[k][1], f);
+                encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<LN>(bm[k]), kc);
                 w.next(a);
             }
         }
-        for (int g = wb + kMaxRuns; g < we; g++) {
+        for (int g = wb + kRuns; g < we; g++) {
             const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
             const bool valid = lane < w.nblk(a);
             const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
-            const uint32_t mm = __vmaxu2(absmax_bits8(v0), absmax_bits8(v1));
-            encode_block<SWZ, SEARCH>(w, lane, valid, v0, v1, max(mm & 0xFFFFu, mm >> 16), kc);
+            float f[16];
+            block_values<LN>(a, w, lane, valid, v0, v1, f);
+            encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<LN>(block_max_key<LN>(v0, v1, f)), kc);
             w.next(a);
         }
     }
@@ -363,6 +438,50 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             }
         }
     }
+}
+
+// LayerNorm statistics of each row (one warp per row), in the fixed order of
+// the fused LayerNorm + modulate + quantize: lane j sums the 16-element
+// blocks j, j+32, ... of the row in order, the 32 partial sums meet in an
+// xor butterfly (16, 8, 4, 2, 1); mean = S1 / cols, var = S2 / cols with S2
+// over fl32(x - mean)^2, rstd = 1 / sqrt(var + eps), every step correctly
+// rounded binary32.
+__device__ __forceinline__ float warp_butterfly_sum(float s) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
+    return s;
+}
+
+__global__ void __launch_bounds__(256) ln_stats_kernel(const uint8_t* x, int64_t ld_bytes, int rows, int cols,
+                                                       float eps, float2* out) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const uint8_t* xr = x + (int64_t)row * ld_bytes;
+    const int nb = cols / 16;
+    const float n = (float)cols;
+    float s = 0.0f;
+    for (int b = lane; b < nb; b += 32) {
+        float f[16];
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
+#pragma unroll
+        for (int i = 0; i < 16; i++) s = __fadd_rn(s, f[i]);
+    }
+    const float mean = __fdiv_rn(warp_butterfly_sum(s), n);
+    float s2 = 0.0f;
+    for (int b = lane; b < nb; b += 32) {
+        float f[16];
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const float d = __fsub_rn(f[i], mean);
+            s2 = __fadd_rn(s2, __fmul_rn(d, d));
+        }
+    }
+    const float var = __fdiv_rn(warp_butterfly_sum(s2), n);
+    if (lane == 0) out[row] = make_float2(mean, __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps))));
 }
 
 struct DequantArgs {
@@ -494,7 +613,9 @@ static nvfp4_status launch_status() {
 // one fused, cooperative launch over one or two tensors of the same shape
 static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t rows, int64_t cols, int64_t ld,
                                   void* const* codes, void* const* scales, float* const* gscale, bool given,
-                                  bool swizzled, bool search, void* workspace, cudaStream_t stream) {
+                                  bool swizzled, bool search, void* workspace, cudaStream_t stream,
+                                  const float2* ln_stats = nullptr, const void* mod_scale = nullptr,
+                                  const void* mod_shift = nullptr) {
     QuantArgs a{};
     for (int t = 0; t < ntensors; t++) {
         a.x[t] = static_cast<const uint8_t*>(x[t]);
@@ -516,6 +637,10 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     a.ctl = static_cast<uint32_t*>(workspace);
     a.err = static_cast<DevError*>(workspace);
     a.limit_ns = 2000000000ull;
+    a.ln_stats = ln_stats;
+    a.mod_scale = static_cast<const __nv_bfloat16*>(mod_scale);
+    a.mod_shift = static_cast<const __nv_bfloat16*>(mod_shift);
+    a.cols = (int)cols;
     const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), ((int64_t)a.runs_per_tensor * ntensors + kQWarps - 1) / kQWarps);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
@@ -527,8 +652,13 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void (*kern)(QuantArgs) = swizzled ? (search ? quantize_fused_kernel<true, true> : quantize_fused_kernel<true, false>)
-                                       : (search ? quantize_fused_kernel<false, true> : quantize_fused_kernel<false, false>);
+    void (*kern)(QuantArgs);
+    if (ln_stats)
+        kern = swizzled ? (search ? quantize_fused_kernel<true, true, true> : quantize_fused_kernel<true, false, true>)
+                        : (search ? quantize_fused_kernel<false, true, true> : quantize_fused_kernel<false, false, true>);
+    else
+        kern = swizzled ? (search ? quantize_fused_kernel<true, true, false> : quantize_fused_kernel<true, false, false>)
+                        : (search ? quantize_fused_kernel<false, true, false> : quantize_fused_kernel<false, false, false>);
     if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
@@ -561,6 +691,36 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     return quantize_impl(1, xs, rows, cols, ld, cs, ss, gs, (flags & NVFP4_Q_GIVEN_GLOBAL) != 0,
                          (flags & NVFP4_Q_ROWMAJOR_SCALES) == 0, (flags & NVFP4_Q_SCALE_SEARCH) != 0, workspace,
                          (cudaStream_t)stream);
+}
+
+extern "C" nvfp4_status nvfp4_ln_modulate_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                                   const void* mod_scale, const void* mod_shift, float eps,
+                                                   void* codes, void* scales, float* global_scale, unsigned flags,
+                                                   void* workspace, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (flags & ~(NVFP4_Q_GIVEN_GLOBAL | NVFP4_Q_ROWMAJOR_SCALES | NVFP4_Q_SCALE_SEARCH)) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols <= 0 || ld < cols || !(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
+    if (rows > ((int64_t)1 << 30) || cols > ((int64_t)1 << 24)) return NVFP4_ERR_UNSUPPORTED;
+    if (!global_scale || !workspace) return NVFP4_ERR_INVALID_ARG;
+    if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_LN_QUANTIZE, rows, 0, cols)) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0) return NVFP4_OK;
+    if (!x_bf16 || !codes || !scales) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales) || (ld % 8) != 0 ||
+        (mod_scale && !aligned16(mod_scale)) || (mod_shift && !aligned16(mod_shift)) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return NVFP4_ERR_MISALIGNED;
+    // the row statistics follow the 256-byte control block
+    float2* stats = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + 256);
+    ln_stats_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, (cudaStream_t)stream>>>(
+        static_cast<const uint8_t*>(x_bf16), ld * 2, (int)rows, (int)cols, eps, stats);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    const void* xs[1] = {x_bf16};
+    void* cs[1] = {codes};
+    void* ss[1] = {scales};
+    float* gs[1] = {global_scale};
+    return quantize_impl(1, xs, rows, cols, ld, cs, ss, gs, (flags & NVFP4_Q_GIVEN_GLOBAL) != 0,
+                         (flags & NVFP4_Q_ROWMAJOR_SCALES) == 0, (flags & NVFP4_Q_SCALE_SEARCH) != 0, workspace,
+                         (cudaStream_t)stream, stats, mod_scale, mod_shift);
 }
 
 static nvfp4_status check_cache(const nvfp4_kv_cache* c) {

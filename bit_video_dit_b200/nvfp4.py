@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
-OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT = range(4)
+OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT, OP_LN_QUANTIZE = range(5)
 Q_COMPUTE_GLOBAL, Q_GIVEN_GLOBAL, Q_ROWMAJOR_SCALES, Q_SCALE_SEARCH = 0, 1, 2, 4
 KV_SCALE_SEARCH = 1
 ACT_NONE, ACT_GELU_TANH = 0, 1
@@ -25,7 +25,8 @@ DBG_SKIP_LOADS = 1
 
 EXPORTS = ("nvfp4_status_string", "nvfp4_version", "nvfp4_codes_bytes", "nvfp4_scales_bytes",
            "nvfp4_workspace_bytes", "nvfp4_read_device_error", "nvfp4_quantize", "nvfp4_gemm",
-           "nvfp4_kv_append", "nvfp4_kv_dequant", "nvfp4_test_encode", "nvfp4_quantize_noalloc")
+           "nvfp4_kv_append", "nvfp4_kv_dequant", "nvfp4_test_encode", "nvfp4_quantize_noalloc",
+           "nvfp4_ln_modulate_quantize")
 
 
 class NVFP4Error(RuntimeError):
@@ -90,6 +91,9 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_test_encode.restype = st
         L.nvfp4_quantize_noalloc.argtypes = [vp, i64, i64, i64, vp, vp, vp, ctypes.c_uint, vp]
         L.nvfp4_quantize_noalloc.restype = st
+        L.nvfp4_ln_modulate_quantize.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_float, vp, vp, vp,
+                                                 ctypes.c_uint, vp, sz, vp]
+        L.nvfp4_ln_modulate_quantize.restype = st
         _lib = L
     return _lib
 
@@ -187,6 +191,35 @@ def quantize(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, out: 
     _check("nvfp4_quantize", lib().nvfp4_quantize(
         x.data_ptr(), rows, cols, x.stride(0), out.codes.data_ptr(), out.scales.data_ptr(),
         out.global_scale.data_ptr(), flags, ws.data_ptr(), ws.numel(), _stream(stream)))
+    return out
+
+
+def ln_modulate_quantize(x: torch.Tensor, *, mod_scale: torch.Tensor | None = None,
+                         mod_shift: torch.Tensor | None = None, eps: float = 1e-6,
+                         global_scale: torch.Tensor | None = None, out: NVFP4Tensor | None = None,
+                         rowmajor_scales: bool = False, scale_search: bool = False, ws: torch.Tensor | None = None,
+                         stream=None) -> NVFP4Tensor:
+    """LayerNorm (no affine) of each row of bf16 x [rows, cols], then
+    h * (1 + mod_scale) + mod_shift (bf16 [cols] each, optional), quantized to
+    NVFP4 in the same pass (tensor scale from max |m| unless global_scale is given)."""
+    _require_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("ln_modulate_quantize takes a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    for v in (mod_scale, mod_shift):
+        if v is not None and (v.dtype != torch.bfloat16 or v.numel() != cols or not v.is_contiguous()):
+            raise ValueError("mod_scale / mod_shift are contiguous bf16 [cols]")
+    if out is None:
+        out = empty_nvfp4(rows, cols, x.device, swizzled=not rowmajor_scales)
+    flags = (Q_ROWMAJOR_SCALES if rowmajor_scales else 0) | (Q_SCALE_SEARCH if scale_search else 0)
+    if global_scale is not None:
+        out.global_scale.copy_(global_scale.reshape(1))
+        flags |= Q_GIVEN_GLOBAL
+    if ws is None:
+        ws = workspace(OP_LN_QUANTIZE, rows, 0, cols, x.device)
+    _check("nvfp4_ln_modulate_quantize", lib().nvfp4_ln_modulate_quantize(
+        x.data_ptr(), rows, cols, x.stride(0), _ptr(mod_scale), _ptr(mod_shift), float(eps), out.codes.data_ptr(),
+        out.scales.data_ptr(), out.global_scale.data_ptr(), flags, ws.data_ptr(), ws.numel(), _stream(stream)))
     return out
 
 

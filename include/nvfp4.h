@@ -89,7 +89,8 @@ enum {
     NVFP4_OP_QUANTIZE = 0,  /* nvfp4_quantize: m = rows, k = cols, n unused */
     NVFP4_OP_GEMM = 1,      /* nvfp4_gemm */
     NVFP4_OP_KV_APPEND = 2, /* nvfp4_kv_append */
-    NVFP4_OP_KV_DEQUANT = 3 /* nvfp4_kv_dequant */
+    NVFP4_OP_KV_DEQUANT = 3, /* nvfp4_kv_dequant */
+    NVFP4_OP_LN_QUANTIZE = 4 /* nvfp4_ln_modulate_quantize (m = rows) */
 };
 
 /* Workspace bytes the caller must pass to the call `op` (device memory,
@@ -137,6 +138,28 @@ nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int
 nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
                             void* scales, float* global_scale, unsigned flags, void* workspace,
                             size_t ws_bytes, nvfp4_stream_t stream);
+
+/* LayerNorm + adaLN modulate + quantize, the step before a DiT linear layer
+ * (the pages' fused adaLN kernels, [NEWS] "NVFP4 量化"; here fused with the
+ * NVFP4 quantize so the modulated activation never goes to memory in bf16).
+ * Per row of x (bf16 [rows x cols], row stride ld): LayerNorm without affine
+ * parameters (population variance, eps inside the square root), then
+ * m = h * (1 + mod_scale[c]) + mod_shift[c] (bf16 [cols] each, or NULL for
+ * 0), all in binary32:
+ *   mean = S1 / cols, var = S2 / cols, rstd = 1 / sqrt(var + eps),
+ *   m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift),
+ * where S1 = sum x and S2 = sum fl32(x - mean)^2 are summed as 32 partial
+ * sums (partial j over the 16-element blocks j, j+32, ... in order) combined
+ * by an xor butterfly over 16, 8, 4, 2, 1.  m is then quantized exactly as
+ * nvfp4_quantize quantizes a tensor (flags as there), a32 from max |m|.
+ * cols % 64 == 0; pointers 16-byte aligned.
+ * workspace: nvfp4_workspace_bytes(NVFP4_OP_LN_QUANTIZE, rows, 0, cols)
+ * bytes (the control block, then 8 bytes of row statistics per row).
+ * Two launches: the row statistics, then the fused quantize. */
+nvfp4_status nvfp4_ln_modulate_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                        const void* mod_scale, const void* mod_shift, float eps, void* codes,
+                                        void* scales, float* global_scale, unsigned flags, void* workspace,
+                                        size_t ws_bytes, nvfp4_stream_t stream);
 
 /* nvfp4_quantize without a workspace, for callers that cannot allocate
  * device memory: code hosted inside a framework that owns every device
