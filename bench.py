@@ -179,7 +179,25 @@ def measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, rep
     q_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
     ap_ms = float(np.median([e[2].elapsed_time(e[3]) for e in ev]))
     del g
-    return {"quantize_ms": q_ms, "kv_append_ms": ap_ms}
+    # the fused LayerNorm + modulate + quantize of A (the step before the linear layer)
+    sc = torch.randn(a.shape[1], device=a.device).mul_(0.1).to(torch.bfloat16)
+    sh = torch.randn(a.shape[1], device=a.device).mul_(0.1).to(torch.bfloat16)
+    ws_ln = nv.workspace(nv.OP_LN_QUANTIZE, a.shape[0], 0, a.shape[1], a.device)
+    nv.ln_modulate_quantize(a, mod_scale=sc, mod_shift=sh, out=qs, ws=ws_ln)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            cache.dequant(ring, k_out, v_out)
+            ev[i][0].record()
+            nv.ln_modulate_quantize(a, mod_scale=sc, mod_shift=sh, out=qs, ws=ws_ln)
+            ev[i][1].record()
+    g.replay()
+    torch.cuda.synchronize()
+    ln_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
+    del g
+    return {"quantize_ms": q_ms, "kv_append_ms": ap_ms, "ln_quantize_ms": ln_ms}
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
@@ -390,6 +408,10 @@ def run_ours(args, rank: int, world: int) -> dict | None:
             "quantize_GB/s": round(quant_bytes / (search["quantize_ms"] * 1e-3) / 1e9, 1),
             "kv_append_ms": round(search["kv_append_ms"], 4),
             "kv_append_GB/s": round(append_bytes / (search["kv_append_ms"] * 1e-3) / 1e9, 1)},
+        "ln_modulate_quantize": {
+            "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A, two launches, outside the step",
+            "ms": round(search["ln_quantize_ms"], 4),
+            "GB/s": round(quant_bytes / (search["ln_quantize_ms"] * 1e-3) / 1e9, 1)},
         "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
                 "what": "pinned host A -> device, quantize, gemm+bias, C -> pinned host"},
