@@ -498,74 +498,113 @@ struct DequantArgs {
 
 // 8 E2M1 codes (32 bits) with one block scale and the slot's a32 -> 8 bf16
 // (16 bytes): bf16_rne(fl32(fl32(e2m1 * s) * a32)); e2m1 * s is exact in
-// binary16, so the only roundings are the two the definition has.
-__device__ __forceinline__ uint4 dequant8(uint32_t q, uint8_t sc, float a32) {
+// binary16, so the only roundings are the two the definition has.  The
+// binary32 products go two at a time (mul.rn.f32x2, each lane rounded as a
+// binary32 multiply).
+__device__ __forceinline__ uint4 dequant8(uint32_t q, uint8_t sc, unsigned long long a2) {
     const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         const __half2 v = __hmul2(e2m1x2_to_half2((q >> (8 * j)) & 0xFFu), s2);  // exact
         const float2 f = __half22float2(v);
-        const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(f.x, a32), __fmul_rn(f.y, a32));
+        unsigned long long p;
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(p) : "l"(*reinterpret_cast<const unsigned long long*>(&f)), "l"(a2));
+        const float2 y = *reinterpret_cast<const float2*>(&p);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(y.x, y.y);
         o[j] = *reinterpret_cast<const uint32_t*>(&b);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__global__ void __launch_bounds__(kThreads) kv_dequant_kernel(DequantArgs a) {
+// 16 bytes to global memory with the streaming hint: the dequantized output
+// is written once and not read back by this kernel, so it should not push the
+// codes out of L2.
+__device__ __forceinline__ void st_stream16(void* p, const uint4& v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// One resident wave of warps (at most 32 registers a thread, so 8 blocks of
+// 256 fit an SM); each warp walks units (512-element runs of the listed
+// slots) two at a time with a stride of twice the warp count.  A lane loads
+// 4 code bytes and a scale byte per half unit and stores 16 bytes, so every
+// warp store covers 512 contiguous bytes.  Positions are 32-bit: the list
+// index is below 2^31 and the run index below slot_elems / 512 <= 2^31.
+__global__ void __launch_bounds__(kThreads, 8) kv_dequant_kernel(DequantArgs a) {
     const int t = blockIdx.y;
     const int lane = threadIdx.x & 31;
     const int64_t ups = (a.slot_elems + 511) / 512;  // 512-element runs per slot
-    const int64_t units = (int64_t)a.n * ups;
     const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
     const uint8_t* cb = t ? a.codes[1] : a.codes[0];
     const uint8_t* sb = t ? a.scales[1] : a.scales[0];
     const float* gb = t ? a.gscale[1] : a.gscale[0];
     uint8_t* ob = t ? a.out[1] : a.out[0];
     const int64_t w0 = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    for (int64_t base = w0; base < units; base += 2 * nwarps) {
-        // two runs per iteration: all loads first, then decode and store
-        uint32_t q[2][2];
-        uint8_t sc[2][2];
+    const uint32_t ups32 = (uint32_t)ups;
+    const uint32_t qs = (uint32_t)(2 * nwarps / ups), rs = (uint32_t)(2 * nwarps - (int64_t)qs * ups);
+    const uint32_t n = (uint32_t)a.n;
+    uint32_t pi[2], pu[2];
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+        const int64_t unit = w0 + k * nwarps;
+        pi[k] = (uint32_t)(unit / ups);
+        pu[k] = (uint32_t)(unit - (int64_t)pi[k] * ups);
+    }
+    while (pi[0] < n) {
+        // both units' loads first, then decode and store
+        uint32_t q[2][2], sc[2];
         float a32[2];
-        bool ok[2][2];
-        int64_t obase[2], e0[2];
+        int64_t o0[2];
+        int halves[2];
 #pragma unroll
         for (int k = 0; k < 2; k++) {
-            const int64_t unit = base + k * nwarps;
-            ok[k][0] = ok[k][1] = false;
-            a32[k] = 0.0f;
-            obase[k] = e0[k] = 0;
             q[k][0] = q[k][1] = 0;
-            sc[k][0] = sc[k][1] = 0;
-            if (unit >= units) continue;
-            const int64_t i = unit / ups;
-            const int64_t u = unit - i * ups;
-            const int32_t s = __ldg(a.slots + i);
+            sc[k] = 0;
+            a32[k] = 0.0f;
+            o0[k] = 0;
+            halves[k] = 0;
+            if (pi[k] >= n) continue;
+            const int32_t s = __ldg(a.slots + pi[k]);
             if (s < 0 || s >= a.n_slots) {
-                if (lane == 0 && u == 0 && t == 0) record_error(a.err, NVFP4_ERR_DEVICE, (uint32_t)i);
+                if (lane == 0 && pu[k] == 0 && t == 0) record_error(a.err, NVFP4_ERR_DEVICE, pi[k]);
                 continue;
             }
-            const int64_t sbase = (int64_t)s * a.slot_elems;
-            e0[k] = u * 512 + 8 * lane;
-            obase[k] = (int64_t)i * a.slot_elems;
+            const int64_t e0 = (int64_t)pu[k] * 512 + 8 * lane;
+            const int64_t src = (int64_t)s * a.slot_elems + e0;
+            o0[k] = (int64_t)pi[k] * a.slot_elems + e0;
             a32[k] = __ldg(gb + s);
-#pragma unroll
-            for (int h = 0; h < 2; h++) {
-                const int64_t e = e0[k] + 256 * h;
-                ok[k][h] = e < a.slot_elems;
-                if (ok[k][h]) {
-                    q[k][h] = __ldg(reinterpret_cast<const uint32_t*>(cb + (sbase + e) / 2));
-                    sc[k][h] = __ldg(sb + (sbase + e) / 16);
-                }
+            // slot_elems is a multiple of 64 and e0 of 8: a word that starts
+            // inside the slot ends inside it
+            if (e0 < a.slot_elems) {
+                q[k][0] = __ldg(reinterpret_cast<const uint32_t*>(cb + src / 2));
+                sc[k] = __ldg(sb + src / 16);
+                halves[k] = 1;
+            }
+            if (e0 + 256 < a.slot_elems) {
+                q[k][1] = __ldg(reinterpret_cast<const uint32_t*>(cb + (src + 256) / 2));
+                sc[k] |= (uint32_t)__ldg(sb + (src + 256) / 16) << 8;
+                halves[k] = 2;
             }
         }
 #pragma unroll
-        for (int k = 0; k < 2; k++)
+        for (int k = 0; k < 2; k++) {
+            const float2 aa = make_float2(a32[k], a32[k]);
+            const unsigned long long a2 = *reinterpret_cast<const unsigned long long*>(&aa);
 #pragma unroll
             for (int h = 0; h < 2; h++)
-                if (ok[k][h])
-                    *reinterpret_cast<uint4*>(ob + (obase[k] + e0[k] + 256 * h) * 2) = dequant8(q[k][h], sc[k][h], a32[k]);
+                if (h < halves[k])
+                    st_stream16(ob + (o0[k] + 256 * h) * 2, dequant8(q[k][h], (uint8_t)(sc[k] >> (8 * h)), a2));
+        }
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            pi[k] += qs;
+            pu[k] += rs;
+            if (pu[k] >= ups32) {
+                pu[k] -= ups32;
+                pi[k] += 1;
+            }
+        }
     }
 }
 
@@ -787,8 +826,16 @@ extern "C" nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int3
     a.n_slots = cache->n_slots;
     a.slot_elems = (int64_t)cache->tokens_per_slot * cache->heads * cache->head_dim;
     a.err = static_cast<DevError*>(workspace);
+    // one resident wave over K and V together (blockIdx.y picks the tensor)
+    static int resident = 0;
+    if (resident == 0) {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kv_dequant_kernel, kThreads, 0) != cudaSuccess || b < 2)
+            b = 2;
+        resident = b;
+    }
     const int64_t units = (int64_t)n * ((a.slot_elems + 511) / 512);
-    const int g = grid_for(units, 2 * (kThreads / 32), num_sms() * 8);
+    const int g = grid_for(units, 2 * (kThreads / 32), num_sms() * resident / 2);
     kv_dequant_kernel<<<dim3(g, 2), kThreads, 0, (cudaStream_t)stream>>>(a);
     return launch_status();
 }
