@@ -100,6 +100,10 @@ def lib():
                 getattr(L, name).argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
                 getattr(L, name).restype = ctypes.c_int
             L.orc_kv_dequant.argtypes = [vp, vp, f32, i64, i64, i64, vp]
+            L.orc_channel_mean.argtypes = [vp, i64, i64, vp]
+            L.orc_kv_append_smooth.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp]
+            L.orc_kv_append_smooth.restype = ctypes.c_int
+            L.orc_kv_dequant_smooth.argtypes = [vp, vp, f32, vp, i64, i64, i64, vp]
             _lib = L
     return _lib
 
@@ -293,6 +297,42 @@ def kv_dequant(codes, scales, alpha, T: int, H: int, d: int) -> np.ndarray:
     out = np.zeros((T, H, d), np.uint16)
     lib().orc_kv_dequant(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)), float(alpha),
                          T, H, d, _p(out))
+    return out
+
+
+def channel_mean(x: np.ndarray) -> np.ndarray:
+    """Binary32 mean over the first axis of bf16 bits x [T, C...] for every
+    channel, in R20's fixed order (32 strided partial sums, butterfly)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    T = x.shape[0]
+    C = x.size // T
+    mean = np.zeros(C, np.float32)
+    lib().orc_channel_mean(_p(x), T, C, _p(mean))
+    return mean
+
+
+def kv_append_smooth(x: np.ndarray, search46: bool = False):
+    """K-smoothing append (R20): x bf16 bits [T, H, d].  Returns (codes, scales,
+    alpha, mean [H*d]); the quantized values are fl32(x - mean[channel])."""
+    T, H, d = x.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    codes = np.zeros((T * H, d // 2), np.uint8)
+    scales = np.zeros((T * H, d // 16), np.uint8)
+    a = np.zeros(1, np.float32)
+    mean = np.zeros(H * d, np.float32)
+    rc = lib().orc_kv_append_smooth(_p(x), T, H, d, MODE_SEARCH46 if search46 else 0, _p(codes), _p(scales),
+                                    _p(a), _p(mean))
+    if rc != 0:
+        raise ValueError(f"orc_kv_append_smooth failed ({rc})")
+    return codes, scales, np.float32(a[0]), mean
+
+
+def kv_dequant_smooth(codes, scales, alpha, mean, T: int, H: int, d: int) -> np.ndarray:
+    """R20 dequant: bf16 of fl32(fl32(fl32(e2m1 * s) * alpha) + mean[channel])."""
+    out = np.zeros((T, H, d), np.uint16)
+    mean = np.ascontiguousarray(mean, dtype=np.float32)
+    lib().orc_kv_dequant_smooth(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)), float(alpha),
+                                _p(mean), T, H, d, _p(out))
     return out
 
 

@@ -50,6 +50,9 @@
  *      orc_ln_modulate for the operations, their binary32 order and eps.
  *  R16 KV slot = NVFP4 matrix of T*H rows x d columns, blocks along d, scales
  *      row-major (not swizzled).
+ *  R20 K-smoothing of a KV chunk (optional, per tensor): subtract each
+ *      channel's mean over the chunk's tokens before the quantize and add it
+ *      back in the dequant; see orc_channel_mean for the order.
  *
  * Every floating-point step that the GPU must reproduce bit for bit is done in
  * IEEE binary32 (compile with -ffp-contract=off so nothing fuses); the GEMM
@@ -560,9 +563,19 @@ ORC_API void orc_kv_dequant(const uint8_t* codes, const uint8_t* scales, float a
  * j+64, ... of the row (blocks and their elements in order), then combined
  * by a butterfly: for o = 16, 8, 4, 2, 1, partial[j] = partial[j] +
  * partial[j ^ o] (all j at once). */
+static float butterfly32(float* part)
+{
+    float next[32];
+    for (int o = 16; o > 0; o >>= 1) {
+        for (int j = 0; j < 32; j++) next[j] = part[j] + part[j ^ o];
+        memcpy(part, next, 32 * sizeof(float));
+    }
+    return part[0];
+}
+
 static float row_sum32(const float* v, int64_t cols)
 {
-    float part[32], next[32];
+    float part[32];
     const int64_t nb = cols / 16;
     for (int j = 0; j < 32; j++) {
         float s = 0.0f;
@@ -570,11 +583,7 @@ static float row_sum32(const float* v, int64_t cols)
             for (int i = 0; i < 16; i++) s = s + v[b * 16 + i];
         part[j] = s;
     }
-    for (int o = 16; o > 0; o >>= 1) {
-        for (int j = 0; j < 32; j++) next[j] = part[j] + part[j ^ o];
-        memcpy(part, next, sizeof part);
-    }
-    return part[0];
+    return butterfly32(part);
 }
 
 ORC_API int orc_ln_modulate(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, const uint16_t* scale,
@@ -616,4 +625,61 @@ ORC_API int orc_ln_modulate_quantize(const uint16_t* x, int64_t rows, int64_t co
     if (rc == 0) rc = orc_quantize_f32(m, rows, cols, cols, mode, alpha, codes, scales);
     free(m);
     return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* KV K-smoothing [RN-I] (R20): per chunk and tensor, each channel's mean     */
+/* over the tokens is taken out before the quantize and put back at dequant  */
+/* ------------------------------------------------------------------------ */
+/* x: bf16 [T][C] (C = H*d channels, token t at x + t*C).  mean[c] in
+ * binary32, fixed order: 32 partial sums, partial p over the tokens p, p+32,
+ * p+64, ... in increasing order (starting from +0), combined by the same
+ * butterfly as R19 (o = 16, 8, 4, 2, 1: part[p] = part[p] + part[p ^ o]);
+ * mean = fl32(S / T). */
+ORC_API void orc_channel_mean(const uint16_t* x, int64_t T, int64_t C, float* mean)
+{
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t c = 0; c < C; c++) {
+        float part[32];
+        for (int p = 0; p < 32; p++) {
+            float s = 0.0f;
+            for (int64_t t = p; t < T; t += 32) s = s + orc_bf16_to_f32(x[t * C + c]);
+            part[p] = s;
+        }
+        mean[c] = butterfly32(part) / (float)T;
+    }
+}
+
+/* x: bf16 chunk [T][H][d] (contiguous).  Writes mean [H*d] (orc_channel_mean),
+ * then quantizes v = fl32(x - mean[h*d + j]) as orc_kv_append does (R15, R16;
+ * mode may carry ORC_MODE_SEARCH46). */
+ORC_API int orc_kv_append_smooth(const uint16_t* x, int64_t T, int64_t H, int64_t d, int mode, uint8_t* codes,
+                                 uint8_t* scales, float* alpha, float* mean)
+{
+    const int64_t C = H * d;
+    if (d % 16 != 0) return 1;
+    orc_channel_mean(x, T, C, mean);
+    float* v = (float*)malloc((size_t)(T * C) * sizeof(float) + 1);
+    if (!v) return 2;
+    for (int64_t t = 0; t < T; t++)
+        for (int64_t c = 0; c < C; c++) v[t * C + c] = orc_bf16_to_f32(x[t * C + c]) - mean[c];
+    int rc = orc_quantize_f32(v, T * H, d, d, ORC_MODE_COMPUTE | (mode & ORC_MODE_SEARCH46), alpha, codes, scales);
+    free(v);
+    return rc;
+}
+
+/* R20 dequant: x^ = bf16_rne(fl32(fl32(fl32(e2m1 * s) * a32) + mean[h*d + j]))
+ * for row r = t*H + h, column j. */
+ORC_API void orc_kv_dequant_smooth(const uint8_t* codes, const uint8_t* scales, float alpha, const float* mean,
+                                   int64_t T, int64_t H, int64_t d, uint16_t* out)
+{
+    const int64_t rows = T * H, nb = d / 16;
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < d; c++) {
+            float qs = (float)(code_at(codes, d, r, c) * orc_e4m3_value(scales[r * nb + c / 16]));
+            float v = qs * alpha;
+            float y = v + mean[(r % H) * d + c];
+            out[r * d + c] = orc_f32_to_bf16(y);
+        }
 }
