@@ -197,7 +197,30 @@ def measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, rep
     torch.cuda.synchronize()
     ln_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
     del g
-    return {"quantize_ms": q_ms, "kv_append_ms": ap_ms, "ln_quantize_ms": ln_ms}
+    # the pages' per-chunk KV variant: K-smoothing of K, the scale search on K and V
+    cache_k = nv.KVCache(cache.n_slots, cache.tokens, cache.heads, cache.head_dim, scale_search=True,
+                         smooth_k=True)
+    for s in range(cache_k.n_slots):
+        cache_k.append(s, *chunks[s % len(chunks)])
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            cache.dequant(ring, k_out, v_out)
+            ev[i][0].record()
+            cache_k.append(i % cache_k.n_slots, *chunks[i % len(chunks)])
+            ev[i][1].record()
+            ev[i][2].record()
+            cache_k.dequant(ring, k_out, v_out)
+            ev[i][3].record()
+    g.replay()
+    torch.cuda.synchronize()
+    sm_ap_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
+    sm_dq_ms = float(np.median([e[2].elapsed_time(e[3]) for e in ev]))
+    del g
+    return {"quantize_ms": q_ms, "kv_append_ms": ap_ms, "ln_quantize_ms": ln_ms,
+            "smooth_append_ms": sm_ap_ms, "smooth_dequant_ms": sm_dq_ms}
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
@@ -408,6 +431,13 @@ def run_ours(args, rank: int, world: int) -> dict | None:
             "quantize_GB/s": round(quant_bytes / (search["quantize_ms"] * 1e-3) / 1e9, 1),
             "kv_append_ms": round(search["kv_append_ms"], 4),
             "kv_append_GB/s": round(append_bytes / (search["kv_append_ms"] * 1e-3) / 1e9, 1)},
+        "kv_smoothing": {
+            "what": "KV append with K-smoothing of K and the scale search on K and V (channel means + quantize, "
+                    "two launches), and the dequant of all slots with the means added back, outside the step",
+            "append_ms": round(search["smooth_append_ms"], 4),
+            "append_GB/s": round(append_bytes / (search["smooth_append_ms"] * 1e-3) / 1e9, 1),
+            "dequant_ms": round(search["smooth_dequant_ms"], 4),
+            "dequant_GB/s": round(dequant_bytes / (search["smooth_dequant_ms"] * 1e-3) / 1e9, 1)},
         "ln_modulate_quantize": {
             "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A, two launches, outside the step",
             "ms": round(search["ln_quantize_ms"], 4),

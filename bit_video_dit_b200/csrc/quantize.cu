@@ -75,6 +75,11 @@ struct QuantArgs {
     const __nv_bfloat16* mod_scale;
     const __nv_bfloat16* mod_shift;
     int cols;
+    // K-smoothing ahead of the quantize (smoothing kernels only, one row per
+    // tensor): binary32 channel means [smooth_hd] per tensor (NULL: none);
+    // the element at flat index i belongs to channel i mod smooth_hd
+    const float* smooth_mean[2];
+    int smooth_hd;
     uint32_t* ctl;
     DevError* err;
     uint64_t limit_ns;
@@ -196,15 +201,39 @@ __device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool 
     }
 }
 
-// The 16 binary32 values of the lane's block of the run at w: the bf16 input,
-// or with LN its LayerNorm + modulate, in this order and rounding:
-// m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift).
-template <bool LN, bool SWZ>
-__device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>& w, int lane, bool valid,
+// Value transforms ahead of the encode (a template parameter of the kernel).
+constexpr int kXfNone = 0;    // the bf16 input as is
+constexpr int kXfLn = 1;      // LayerNorm + adaLN modulate of each row
+constexpr int kXfSmooth = 2;  // minus the channel mean (K-smoothing of a KV chunk)
+
+// The 16 binary32 values of the lane's block of the run at w (tensor t): the
+// bf16 input; with LN its LayerNorm + modulate, in this order and rounding:
+// m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift);
+// with smoothing fl32(x - mean[channel]).
+template <int XF, bool SWZ>
+__device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>& w, int t, int lane, bool valid,
                                              const uint4& q0, const uint4& q1, float* f) {
     bf16x8_to_f32(q0, f);
     bf16x8_to_f32(q1, f + 8);
-    if (LN) {
+    if (XF == kXfSmooth) {
+        const float* mean = t ? a.smooth_mean[1] : a.smooth_mean[0];
+        if (valid && mean) {
+            // one row per tensor, fewer than 2^31 elements: the block's first
+            // flat index is w.cr * 512 + lane * 16, and its 16 channels are
+            // consecutive (smooth_hd is a multiple of 16)
+            const uint32_t c0 = (uint32_t)(w.cr * 512 + lane * 16) % (uint32_t)a.smooth_hd;
+            const float4* p = reinterpret_cast<const float4*>(mean + c0);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const float4 v = __ldg(p + j);
+                f[4 * j] = __fsub_rn(f[4 * j], v.x);
+                f[4 * j + 1] = __fsub_rn(f[4 * j + 1], v.y);
+                f[4 * j + 2] = __fsub_rn(f[4 * j + 2], v.z);
+                f[4 * j + 3] = __fsub_rn(f[4 * j + 3], v.w);
+            }
+        }
+    }
+    if (XF == kXfLn) {
         const float2 st = __ldg(a.ln_stats + w.r);
         const int c0 = w.cr * 512 + lane * 16;
         float sc[16], sh[16];
@@ -229,10 +258,10 @@ __device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>
 }
 
 // a block's |x| max as an order-preserving 32-bit key: the bf16 magnitude
-// bits (LN: the binary32 magnitude bits of the modulated values)
-template <bool LN>
+// bits (F32, after a transform: the binary32 magnitude bits of the values)
+template <bool F32>
 __device__ __forceinline__ uint32_t block_max_key(const uint4& q0, const uint4& q1, const float* f) {
-    if (LN) {
+    if (F32) {
         float mx = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; i++) mx = fmaxf(mx, fabsf(f[i]));
@@ -242,16 +271,17 @@ __device__ __forceinline__ uint32_t block_max_key(const uint4& q0, const uint4& 
     return max(mm & 0xFFFFu, mm >> 16);
 }
 
-template <bool LN>
-__device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float(LN ? key : key << 16); }
+template <bool F32>
+__device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float(F32 ? key : key << 16); }
 
-template <bool SWZ, bool SEARCH, bool LN>
+template <bool SWZ, bool SEARCH, int XF>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
-    constexpr int kRuns = LN ? 4 : kMaxRuns;  // LN needs registers for the transform
+    constexpr bool F32 = XF != kXfNone;       // 32-bit keys of transformed values
+    constexpr int kRuns = F32 ? 4 : kMaxRuns;  // a transform needs registers
     __shared__ uint32_t s_red[kQWarps];
     __shared__ float s_d6[2], s_d4[2], s_a32[2];
     __shared__ float s_inv[2][256];
-    __shared__ uint32_t s_total;
+    __shared__ uint32_t s_total[2];
     __shared__ int s_ok;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
@@ -283,7 +313,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
         }
     }
     uint32_t m = 0;  // the lane's max key over its runs
-    if constexpr (!LN) {
+    if constexpr (!F32) {
         // blocks past the data were loaded as zeros: key 0
 #pragma unroll
         for (int k = 0; k < kRuns; k++) {
@@ -297,8 +327,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
         for (int k = 0; k < kRuns; k++) {
             float f[16];
             const bool have = wb + k < we;
-            block_values<LN>(a, w, lane, have && lane < w.nblk(a), q[k][0], q[k][1], f);
-            bm[k] = have && lane < w.nblk(a) ? block_max_key<LN>(q[k][0], q[k][1], f) : 0u;
+            block_values<XF>(a, w, t, lane, have && lane < w.nblk(a), q[k][0], q[k][1], f);
+            bm[k] = have && lane < w.nblk(a) ? block_max_key<F32>(q[k][0], q[k][1], f) : 0u;
             m = max(m, bm[k]);
             if (have) w.next(a);
         }
@@ -313,29 +343,44 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
                 const bool valid = lane < w.nblk(a);
                 const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
                 float f[16];
-                block_values<LN>(a, w, lane, valid, v0, v1, f);
-                if (valid) m = max(m, block_max_key<LN>(v0, v1, f));
+                block_values<XF>(a, w, t, lane, valid, v0, v1, f);
+                if (valid) m = max(m, block_max_key<F32>(v0, v1, f));
                 w.next(a);
             }
         }
-        // one word per lane: for two tensors, tensor-1 max in the high half,
-        // tensor-0 in the low (16-bit keys); LN has one tensor and 32-bit keys
-        if (!LN) m = t ? (m << 16) : m;
+        // 16-bit keys: one word per lane, tensor-1 max in the high half and
+        // tensor-0 in the low, reduced as pairs; 32-bit keys (after a
+        // transform): a warp covers one tensor, so its max, then per tensor
+        // over the CTA's warps
+        if (!F32) m = t ? (m << 16) : m;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-            m = LN ? max(m, other) : __vmaxu2(m, other);
+            m = F32 ? max(m, other) : __vmaxu2(m, other);
         }
         if (lane == 0) s_red[warp] = m;
         __syncthreads();
         if (threadIdx.x == 0) {
-            uint32_t c = 0;
+            uint32_t c0 = 0u, c1 = 0u;
+            if (F32) {
 #pragma unroll
-            for (int i = 0; i < kQWarps; i++) c = LN ? max(c, s_red[i]) : __vmaxu2(c, s_red[i]);
+                for (int i = 0; i < kQWarps; i++) {
+                    if ((blockIdx.x * kQWarps + i) / nwt)
+                        c1 = max(c1, s_red[i]);
+                    else
+                        c0 = max(c0, s_red[i]);
+                }
+            } else {
+                uint32_t c = 0u;
+#pragma unroll
+                for (int i = 0; i < kQWarps; i++) c = __vmaxu2(c, s_red[i]);
+                c0 = c & 0xFFFFu;
+                c1 = c >> 16;
+            }
             uint32_t* cnt = a.ctl + kCtlCount + par;
             uint32_t* mx = a.ctl + kCtlMax + 2 * par;
-            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(LN ? c : c & 0xFFFFu) : "memory");
-            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx + 1), "r"(LN ? 0u : c >> 16) : "memory");
+            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(c0) : "memory");
+            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx + 1), "r"(c1) : "memory");
             uint32_t old;
             // acquire too: the last CTA to arrive reads the maxima without polling
             asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
@@ -354,13 +399,13 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             uint32_t t0, t1;
             asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t0) : "l"(mx) : "memory");
             asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t1) : "l"(mx + 1) : "memory");
-            s_total = LN ? t0 : ((t1 << 16) | t0);
+            s_total[0] = t0;
+            s_total[1] = t1;
         }
         __syncthreads();
         if (!s_ok) return;
         if (threadIdx.x < a.ntensors) {
-            const uint32_t key = LN ? s_total : (threadIdx.x ? (s_total >> 16) : (s_total & 0xFFFFu));
-            const float a32 = __fdiv_rn(key_value<LN>(key), 2688.0f);  // amax / (6 * 448)
+            const float a32 = __fdiv_rn(key_value<F32>(s_total[threadIdx.x]), 2688.0f);  // amax / (6 * 448)
             s_d6[threadIdx.x] = a32;  // a32 for now; the table below needs it
             if (blockIdx.x == 0) *(threadIdx.x ? a.gscale[1] : a.gscale[0]) = a32;
         }
@@ -406,8 +451,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             if (wb + k < we) {
                 const bool valid = lane < w.nblk(a);
                 float f[16];
-                block_values<LN>(a, w, lane, valid, q[k][0], q[k][1], f);
-                encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<LN>(bm[k]), kc);
+                block_values<XF>(a, w, t, lane, valid, q[k][0], q[k][1], f);
+                encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<F32>(bm[k]), kc);
                 w.next(a);
             }
         }
@@ -416,8 +461,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             const bool valid = lane < w.nblk(a);
             const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
             float f[16];
-            block_values<LN>(a, w, lane, valid, v0, v1, f);
-            encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<LN>(block_max_key<LN>(v0, v1, f)), kc);
+            block_values<XF>(a, w, t, lane, valid, v0, v1, f);
+            encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<F32>(block_max_key<F32>(v0, v1, f)), kc);
             w.next(a);
         }
     }
@@ -484,6 +529,54 @@ __global__ void __launch_bounds__(256) ln_stats_kernel(const uint8_t* x, int64_t
     if (lane == 0) out[row] = make_float2(mean, __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps))));
 }
 
+// Channel means of a KV chunk for K-smoothing, in a fixed binary32 order:
+// channel c = h * d + j of the chunk [T][H*d]; partial p (p = 0..31) sums
+// tokens p, p+32, p+64, ... in increasing order from +0, the 32 partials meet
+// in an xor butterfly (16, 8, 4, 2, 1), and mean = S / T, each step one
+// correctly rounded binary32 operation.  A block of 1024 threads covers 64
+// channels of one tensor: warp p computes partial p of two adjacent channels
+// per lane (one 4-byte load a token, 128 contiguous bytes a warp), the
+// partials meet in shared memory, and warp w finishes channels 2w and 2w + 1.
+struct MeanArgs {
+    const uint8_t* x[2];  // bf16 [T][hd]
+    float* mean[2];       // [hd], NULL: tensor not smoothed
+    int T;
+    int hd;               // H * d, a multiple of 16
+};
+
+__global__ void __launch_bounds__(1024) kv_channel_mean_kernel(MeanArgs a) {
+    __shared__ float part[32][65];
+    const int t = blockIdx.y;
+    const uint8_t* x = t ? a.x[1] : a.x[0];
+    float* out = t ? a.mean[1] : a.mean[0];
+    if (out == nullptr) return;  // the whole block
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * 64 + 2 * lane;
+    float s0 = 0.0f, s1 = 0.0f;
+    if (c < a.hd) {
+        const uint8_t* p = x + ((int64_t)warp * a.hd + c) * 2;
+        const int64_t stride = (int64_t)32 * a.hd * 2;
+#pragma unroll 8
+        for (int tok = warp; tok < a.T; tok += 32, p += stride) {
+            const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p));
+            s0 = __fadd_rn(s0, __uint_as_float(v << 16));
+            s1 = __fadd_rn(s1, __uint_as_float(v & 0xFFFF0000u));
+        }
+    }
+    part[warp][2 * lane] = s0;
+    part[warp][2 * lane + 1] = s1;
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+        const int ch = 2 * warp + k;
+        float sum = part[lane][ch];  // lane p holds partial p
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, o));
+        const int cc = blockIdx.x * 64 + ch;
+        if (lane == 0 && cc < a.hd) out[cc] = __fdiv_rn(sum, (float)a.T);
+    }
+}
+
 struct DequantArgs {
     const uint8_t* codes[2];
     const uint8_t* scales[2];
@@ -494,15 +587,25 @@ struct DequantArgs {
     int32_t n_slots;
     int64_t slot_elems;      // T * H * d
     DevError* err;
+    const float* mean[2];    // K-smoothing channel means [n_slots][hd] (NULL: none)
+    int hd;                  // H * d
 };
 
 // 8 E2M1 codes (32 bits) with one block scale and the slot's a32 -> 8 bf16
 // (16 bytes): bf16_rne(fl32(fl32(e2m1 * s) * a32)); e2m1 * s is exact in
 // binary16, so the only roundings are the two the definition has.  The
 // binary32 products go two at a time (mul.rn.f32x2, each lane rounded as a
-// binary32 multiply).
-__device__ __forceinline__ uint4 dequant8(uint32_t q, uint8_t sc, unsigned long long a2) {
+// binary32 multiply).  ADD (K-smoothing): the 8 channel means m are added to
+// the products first, bf16_rne(fl32(fl32(fl32(e2m1 * s) * a32) + m)).
+template <bool ADD>
+__device__ __forceinline__ uint4 dequant8(uint32_t q, uint8_t sc, unsigned long long a2, const float4* m) {
     const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
+    float mv[8];
+    if (ADD) {
+        const float4 m0 = __ldg(m), m1 = __ldg(m + 1);
+        mv[0] = m0.x; mv[1] = m0.y; mv[2] = m0.z; mv[3] = m0.w;
+        mv[4] = m1.x; mv[5] = m1.y; mv[6] = m1.z; mv[7] = m1.w;
+    }
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; j++) {
@@ -510,7 +613,14 @@ __device__ __forceinline__ uint4 dequant8(uint32_t q, uint8_t sc, unsigned long 
         const float2 f = __half22float2(v);
         unsigned long long p;
         asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(p) : "l"(*reinterpret_cast<const unsigned long long*>(&f)), "l"(a2));
-        const float2 y = *reinterpret_cast<const float2*>(&p);
+        float2 y = *reinterpret_cast<const float2*>(&p);
+        if (ADD) {
+            // scalar adds: the compiler may contract a packed multiply and a
+            // packed add into one fused multiply-add, which would skip the
+            // product's own rounding; __fadd_rn is never contracted
+            y.x = __fadd_rn(y.x, mv[2 * j]);
+            y.y = __fadd_rn(y.y, mv[2 * j + 1]);
+        }
         const __nv_bfloat162 b = __floats2bfloat162_rn(y.x, y.y);
         o[j] = *reinterpret_cast<const uint32_t*>(&b);
     }
@@ -531,7 +641,9 @@ __device__ __forceinline__ void st_stream16(void* p, const uint4& v) {
 // 4 code bytes and a scale byte per half unit and stores 16 bytes, so every
 // warp store covers 512 contiguous bytes.  Positions are 32-bit: the list
 // index is below 2^31 and the run index below slot_elems / 512 <= 2^31.
-__global__ void __launch_bounds__(kThreads, 8) kv_dequant_kernel(DequantArgs a) {
+// SMOOTH: the tensor's channel means (when it has them) are added back.
+template <bool SMOOTH>
+__global__ void __launch_bounds__(kThreads, SMOOTH ? 6 : 8) kv_dequant_kernel(DequantArgs a) {
     const int t = blockIdx.y;
     const int lane = threadIdx.x & 31;
     const int64_t ups = (a.slot_elems + 511) / 512;  // 512-element runs per slot
@@ -540,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, 8) kv_dequant_kernel(DequantArgs a) 
     const uint8_t* sb = t ? a.scales[1] : a.scales[0];
     const float* gb = t ? a.gscale[1] : a.gscale[0];
     uint8_t* ob = t ? a.out[1] : a.out[0];
+    const float* mb = SMOOTH ? (t ? a.mean[1] : a.mean[0]) : nullptr;
     const int64_t w0 = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     const uint32_t ups32 = (uint32_t)ups;
     const uint32_t qs = (uint32_t)(2 * nwarps / ups), rs = (uint32_t)(2 * nwarps - (int64_t)qs * ups);
@@ -556,6 +669,7 @@ __global__ void __launch_bounds__(kThreads, 8) kv_dequant_kernel(DequantArgs a) 
         uint32_t q[2][2], sc[2];
         float a32[2];
         int64_t o0[2];
+        const float* mk[2];  // SMOOTH: the slot's channel means
         int halves[2];
 #pragma unroll
         for (int k = 0; k < 2; k++) {
@@ -564,6 +678,7 @@ __global__ void __launch_bounds__(kThreads, 8) kv_dequant_kernel(DequantArgs a) 
             a32[k] = 0.0f;
             o0[k] = 0;
             halves[k] = 0;
+            mk[k] = nullptr;
             if (pi[k] >= n) continue;
             const int32_t s = __ldg(a.slots + pi[k]);
             if (s < 0 || s >= a.n_slots) {
@@ -574,6 +689,7 @@ __global__ void __launch_bounds__(kThreads, 8) kv_dequant_kernel(DequantArgs a) 
             const int64_t src = (int64_t)s * a.slot_elems + e0;
             o0[k] = (int64_t)pi[k] * a.slot_elems + e0;
             a32[k] = __ldg(gb + s);
+            if (SMOOTH && mb) mk[k] = mb + (int64_t)s * a.hd;
             // slot_elems is a multiple of 64 and e0 of 8: a word that starts
             // inside the slot ends inside it
             if (e0 < a.slot_elems) {
@@ -592,9 +708,20 @@ __global__ void __launch_bounds__(kThreads, 8) kv_dequant_kernel(DequantArgs a) 
             const float2 aa = make_float2(a32[k], a32[k]);
             const unsigned long long a2 = *reinterpret_cast<const unsigned long long*>(&aa);
 #pragma unroll
-            for (int h = 0; h < 2; h++)
-                if (h < halves[k])
-                    st_stream16(ob + (o0[k] + 256 * h) * 2, dequant8(q[k][h], (uint8_t)(sc[k] >> (8 * h)), a2));
+            for (int h = 0; h < 2; h++) {
+                if (h >= halves[k]) continue;
+                uint4 v;
+                if (SMOOTH && mk[k]) {
+                    // fewer than 2^31 elements a slot (checked on the host): the
+                    // lane's 8 channels are consecutive (hd is a multiple of 16)
+                    const uint32_t e = (uint32_t)(pu[k] * 512 + 8 * lane + 256 * h);
+                    const float4* m = reinterpret_cast<const float4*>(mk[k] + e % (uint32_t)a.hd);
+                    v = dequant8<true>(q[k][h], (uint8_t)(sc[k] >> (8 * h)), a2, m);
+                } else {
+                    v = dequant8<false>(q[k][h], (uint8_t)(sc[k] >> (8 * h)), a2, nullptr);
+                }
+                st_stream16(ob + (o0[k] + 256 * h) * 2, v);
+            }
         }
 #pragma unroll
         for (int k = 0; k < 2; k++) {
@@ -654,7 +781,8 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
                                   void* const* codes, void* const* scales, float* const* gscale, bool given,
                                   bool swizzled, bool search, void* workspace, cudaStream_t stream,
                                   const float2* ln_stats = nullptr, const void* mod_scale = nullptr,
-                                  const void* mod_shift = nullptr) {
+                                  const void* mod_shift = nullptr, const float* const* smooth_mean = nullptr,
+                                  int smooth_hd = 0) {
     QuantArgs a{};
     for (int t = 0; t < ntensors; t++) {
         a.x[t] = static_cast<const uint8_t*>(x[t]);
@@ -680,6 +808,11 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     a.mod_scale = static_cast<const __nv_bfloat16*>(mod_scale);
     a.mod_shift = static_cast<const __nv_bfloat16*>(mod_shift);
     a.cols = (int)cols;
+    if (smooth_mean) {
+        a.smooth_mean[0] = smooth_mean[0];
+        a.smooth_mean[1] = ntensors > 1 ? smooth_mean[1] : nullptr;
+        a.smooth_hd = smooth_hd;
+    }
     const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), ((int64_t)a.runs_per_tensor * ntensors + kQWarps - 1) / kQWarps);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
@@ -693,11 +826,13 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     cfg.numAttrs = 1;
     void (*kern)(QuantArgs);
     if (ln_stats)
-        kern = swizzled ? (search ? quantize_fused_kernel<true, true, true> : quantize_fused_kernel<true, false, true>)
-                        : (search ? quantize_fused_kernel<false, true, true> : quantize_fused_kernel<false, false, true>);
+        kern = swizzled ? (search ? quantize_fused_kernel<true, true, kXfLn> : quantize_fused_kernel<true, false, kXfLn>)
+                        : (search ? quantize_fused_kernel<false, true, kXfLn> : quantize_fused_kernel<false, false, kXfLn>);
+    else if (smooth_mean)  // KV chunks only: row-major scales
+        kern = search ? quantize_fused_kernel<false, true, kXfSmooth> : quantize_fused_kernel<false, false, kXfSmooth>;
     else
-        kern = swizzled ? (search ? quantize_fused_kernel<true, true, false> : quantize_fused_kernel<true, false, false>)
-                        : (search ? quantize_fused_kernel<false, true, false> : quantize_fused_kernel<false, false, false>);
+        kern = swizzled ? (search ? quantize_fused_kernel<true, true, kXfNone> : quantize_fused_kernel<true, false, kXfNone>)
+                        : (search ? quantize_fused_kernel<false, true, kXfNone> : quantize_fused_kernel<false, false, kXfNone>);
     if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
@@ -768,9 +903,21 @@ static nvfp4_status check_cache(const nvfp4_kv_cache* c) {
         return NVFP4_ERR_INVALID_ARG;
     if (c->n_slots <= 0 || c->tokens_per_slot <= 0 || c->heads <= 0 || c->head_dim <= 0) return NVFP4_ERR_INVALID_ARG;
     if (c->head_dim % 16 != 0) return NVFP4_ERR_UNSUPPORTED;
-    if (c->flags & ~NVFP4_KV_SCALE_SEARCH) return NVFP4_ERR_INVALID_ARG;
+    if (c->flags & ~(NVFP4_KV_SCALE_SEARCH | NVFP4_KV_SMOOTH_K | NVFP4_KV_SMOOTH_V)) return NVFP4_ERR_INVALID_ARG;
     const int64_t e = (int64_t)c->tokens_per_slot * c->heads * c->head_dim;
     if (e % 64 != 0 || e > ((int64_t)1 << 40)) return NVFP4_ERR_UNSUPPORTED;
+    if (c->flags & (NVFP4_KV_SMOOTH_K | NVFP4_KV_SMOOTH_V)) {
+        // smoothing indexes channels with 32-bit arithmetic
+        // and divides by the token count in binary32 (exact below 2^24)
+        if (e >= ((int64_t)1 << 31) || (int64_t)c->heads * c->head_dim >= ((int64_t)1 << 24) ||
+            c->tokens_per_slot >= (1 << 24))
+            return NVFP4_ERR_UNSUPPORTED;
+        if (((c->flags & NVFP4_KV_SMOOTH_K) && !c->k_mean) || ((c->flags & NVFP4_KV_SMOOTH_V) && !c->v_mean))
+            return NVFP4_ERR_INVALID_ARG;
+        if (((c->flags & NVFP4_KV_SMOOTH_K) && !aligned16(c->k_mean)) ||
+            ((c->flags & NVFP4_KV_SMOOTH_V) && !aligned16(c->v_mean)))
+            return NVFP4_ERR_MISALIGNED;
+    }
     if (!aligned16(c->k_codes) || !aligned16(c->k_scales) || !aligned16(c->v_codes) || !aligned16(c->v_scales) ||
         (reinterpret_cast<uintptr_t>(c->k_global) & 3u) || (reinterpret_cast<uintptr_t>(c->v_global) & 3u))
         return NVFP4_ERR_MISALIGNED;
@@ -796,8 +943,24 @@ extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slo
     void* ss[2] = {static_cast<uint8_t*>(cache->k_scales) + (int64_t)slot * (e / 16),
                    static_cast<uint8_t*>(cache->v_scales) + (int64_t)slot * (e / 16)};
     float* gs[2] = {cache->k_global + slot, cache->v_global + slot};
-    return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, (cache->flags & NVFP4_KV_SCALE_SEARCH) != 0,
-                         workspace, (cudaStream_t)stream);
+    const bool search = (cache->flags & NVFP4_KV_SCALE_SEARCH) != 0;
+    const bool sk = (cache->flags & NVFP4_KV_SMOOTH_K) != 0, sv = (cache->flags & NVFP4_KV_SMOOTH_V) != 0;
+    if (!sk && !sv)
+        return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, search, workspace, (cudaStream_t)stream);
+    // K-smoothing: the slot's channel means first, then the quantize of x - mean
+    const int hd = cache->heads * cache->head_dim;
+    MeanArgs m{};
+    m.x[0] = static_cast<const uint8_t*>(k_bf16);
+    m.x[1] = static_cast<const uint8_t*>(v_bf16);
+    m.mean[0] = sk ? cache->k_mean + (int64_t)slot * hd : nullptr;
+    m.mean[1] = sv ? cache->v_mean + (int64_t)slot * hd : nullptr;
+    m.T = cache->tokens_per_slot;
+    m.hd = hd;
+    kv_channel_mean_kernel<<<dim3((unsigned)((hd + 63) / 64), 2), 1024, 0, (cudaStream_t)stream>>>(m);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+    const float* means[2] = {m.mean[0], m.mean[1]};
+    return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, search, workspace, (cudaStream_t)stream, nullptr,
+                         nullptr, nullptr, means, hd);
 }
 
 extern "C" nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n,
@@ -826,17 +989,23 @@ extern "C" nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int3
     a.n_slots = cache->n_slots;
     a.slot_elems = (int64_t)cache->tokens_per_slot * cache->heads * cache->head_dim;
     a.err = static_cast<DevError*>(workspace);
+    const bool smooth = (cache->flags & (NVFP4_KV_SMOOTH_K | NVFP4_KV_SMOOTH_V)) != 0;
+    if (smooth) {
+        a.mean[0] = (cache->flags & NVFP4_KV_SMOOTH_K) ? cache->k_mean : nullptr;
+        a.mean[1] = (cache->flags & NVFP4_KV_SMOOTH_V) ? cache->v_mean : nullptr;
+        a.hd = cache->heads * cache->head_dim;
+    }
     // one resident wave over K and V together (blockIdx.y picks the tensor)
-    static int resident = 0;
-    if (resident == 0) {
+    static int resident[2] = {0, 0};
+    void (*kern)(DequantArgs) = smooth ? kv_dequant_kernel<true> : kv_dequant_kernel<false>;
+    if (resident[smooth] == 0) {
         int b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kv_dequant_kernel, kThreads, 0) != cudaSuccess || b < 2)
-            b = 2;
-        resident = b;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, 0) != cudaSuccess || b < 2) b = 2;
+        resident[smooth] = b;
     }
     const int64_t units = (int64_t)n * ((a.slot_elems + 511) / 512);
-    const int g = grid_for(units, 2 * (kThreads / 32), num_sms() * resident / 2);
-    kv_dequant_kernel<<<dim3(g, 2), kThreads, 0, (cudaStream_t)stream>>>(a);
+    const int g = grid_for(units, 2 * (kThreads / 32), num_sms() * resident[smooth] / 2);
+    kern<<<dim3(g, 2), kThreads, 0, (cudaStream_t)stream>>>(a);
     return launch_status();
 }
 

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
 OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT, OP_LN_QUANTIZE = range(5)
 Q_COMPUTE_GLOBAL, Q_GIVEN_GLOBAL, Q_ROWMAJOR_SCALES, Q_SCALE_SEARCH = 0, 1, 2, 4
-KV_SCALE_SEARCH = 1
+KV_SCALE_SEARCH, KV_SMOOTH_K, KV_SMOOTH_V = 1, 2, 4
 ACT_NONE, ACT_GELU_TANH = 0, 1
 DBG_SKIP_LOADS = 1
 
@@ -52,7 +52,8 @@ class CKVCache(ctypes.Structure):
     _fields_ = [("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
                 ("v_scales", ctypes.c_void_p), ("k_global", ctypes.c_void_p), ("v_global", ctypes.c_void_p),
                 ("n_slots", ctypes.c_int32), ("tokens_per_slot", ctypes.c_int32), ("heads", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+                ("head_dim", ctypes.c_int32), ("flags", ctypes.c_uint32), ("k_mean", ctypes.c_void_p),
+                ("v_mean", ctypes.c_void_p)]
 
 
 _lib = None
@@ -259,12 +260,14 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, *, out: torch.Tensor | None = None, bia
 class KVCache:
     """Paged NVFP4 KV cache: n_slots frame-chunks of tokens x heads x head_dim,
     K and V each stored as codes + row-major E4M3 scales + one binary32 tensor
-    scale per slot (9/16 byte per element per tensor)."""
+    scale per slot (9/16 byte per element per tensor).  smooth_k / smooth_v
+    add K-smoothing: one binary32 mean per channel (heads x head_dim) per slot."""
 
     def __init__(self, n_slots: int, tokens: int, heads: int, head_dim: int, device="cuda",
-                 scale_search: bool = False):
+                 scale_search: bool = False, smooth_k: bool = False, smooth_v: bool = False):
         self.n_slots, self.tokens, self.heads, self.head_dim = n_slots, tokens, heads, head_dim
-        self.flags = KV_SCALE_SEARCH if scale_search else 0
+        self.flags = ((KV_SCALE_SEARCH if scale_search else 0) | (KV_SMOOTH_K if smooth_k else 0) |
+                      (KV_SMOOTH_V if smooth_v else 0))
         e = tokens * heads * head_dim
         self.slot_elems = e
         u8 = torch.uint8
@@ -274,17 +277,23 @@ class KVCache:
         self.v_scales = torch.zeros((n_slots, e // 16), dtype=u8, device=device)
         self.k_global = torch.zeros(n_slots, dtype=torch.float32, device=device)
         self.v_global = torch.zeros(n_slots, dtype=torch.float32, device=device)
+        f32 = torch.float32
+        self.k_mean = torch.zeros((n_slots, heads * head_dim), dtype=f32, device=device) if smooth_k else None
+        self.v_mean = torch.zeros((n_slots, heads * head_dim), dtype=f32, device=device) if smooth_v else None
         self.ws_append = workspace(OP_KV_APPEND, tokens * heads, 0, head_dim, device)
         self.ws_dequant = workspace(OP_KV_DEQUANT, device=device)
 
     def c(self) -> CKVCache:
         return CKVCache(self.k_codes.data_ptr(), self.k_scales.data_ptr(), self.v_codes.data_ptr(),
                         self.v_scales.data_ptr(), self.k_global.data_ptr(), self.v_global.data_ptr(),
-                        self.n_slots, self.tokens, self.heads, self.head_dim, self.flags)
+                        self.n_slots, self.tokens, self.heads, self.head_dim, self.flags,
+                        None if self.k_mean is None else self.k_mean.data_ptr(),
+                        None if self.v_mean is None else self.v_mean.data_ptr())
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
-                   (self.k_codes, self.v_codes, self.k_scales, self.v_scales, self.k_global, self.v_global))
+                   (self.k_codes, self.v_codes, self.k_scales, self.v_scales, self.k_global, self.v_global,
+                    self.k_mean, self.v_mean) if t is not None)
 
     def append(self, slot: int, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
         """Quantize one chunk's K and V (bf16 [T, H, d], contiguous) into `slot` in place."""

@@ -255,9 +255,21 @@ typedef struct {
     float* v_global; /* [n_slots] device binary32 */
     int32_t n_slots, tokens_per_slot, heads, head_dim;
     uint32_t flags; /* NVFP4_KV_* (0: the standard encoding) */
+    float* k_mean;  /* [n_slots][H*d] device binary32, with NVFP4_KV_SMOOTH_K (else unused, may be NULL) */
+    float* v_mean;  /* [n_slots][H*d] device binary32, with NVFP4_KV_SMOOTH_V (else unused, may be NULL) */
 } nvfp4_kv_cache;
 
 #define NVFP4_KV_SCALE_SEARCH 1u /* appends use the scale search of NVFP4_Q_SCALE_SEARCH */
+/* K-smoothing [RN-I] (K and V each, independently): the append takes each
+ * channel's mean over the chunk's tokens (channel c = h*d + j; binary32:
+ * partial p sums tokens p, p+32, ... in order, the 32 partials meet in an xor
+ * butterfly 16, 8, 4, 2, 1, mean = S / T), stores it at *_mean[slot][c] and
+ * quantizes fl32(x - mean[c]) (tensor scale from max |x - mean|); the dequant
+ * returns bf16_rne(fl32(fl32(fl32(e2m1 * s) * a32) + mean[c])).  Needs
+ * T*H*d < 2^31, T < 2^24 and the mean array 16-byte aligned; the append is then
+ * two launches (the means, then the quantize). */
+#define NVFP4_KV_SMOOTH_K 2u
+#define NVFP4_KV_SMOOTH_V 4u
 
 /* Quantizes one chunk's K and V (bf16, token-major [T][H][d], contiguous)
  * in place into slot `slot`: one tensor scale per (slot, K|V) = amax / 2688
@@ -270,7 +282,8 @@ nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const vo
 
 /* Gathers the n slots listed in slots_dev (device int32 [n], values in
  * [0, n_slots)) back to bf16: output i covers rows i*T*H .. of k_out / v_out
- * (bf16 [n][T][H][d]).  Each value is bf16_rne(fl32(fl32(e2m1 * s) * a32)).
+ * (bf16 [n][T][H][d]).  Each value is bf16_rne(fl32(fl32(e2m1 * s) * a32))
+ * (plus the channel mean before the bf16 rounding for a smoothed tensor).
  * An out-of-range slot index records NVFP4_ERR_DEVICE (info = list position)
  * in the workspace and leaves that output chunk unwritten.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_KV_DEQUANT, 0, 0, 0) bytes. */

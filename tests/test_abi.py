@@ -88,6 +88,19 @@ def test_host_side_argument_checks(L):
     assert st == nv.ERR_INVALID_ARG  # slot out of range
     st = L.nvfp4_kv_dequant(ctypes.byref(kv), fake, -1, fake, fake, fake, 1 << 16, None)
     assert st == nv.ERR_INVALID_ARG
+    # K-smoothing: the flagged tensor's mean array is required and 16-byte aligned
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32, nv.KV_SMOOTH_K)
+    st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 16, None)
+    assert st == nv.ERR_INVALID_ARG  # no k_mean
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32, nv.KV_SMOOTH_V, fake, fake + 4)
+    st = L.nvfp4_kv_dequant(ctypes.byref(kv), fake, 1, fake, fake, fake, 1 << 16, None)
+    assert st == nv.ERR_MISALIGNED  # v_mean not 16-byte aligned
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 1 << 24, 1, 16, nv.KV_SMOOTH_K, fake, fake)
+    st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 30, None)
+    assert st == nv.ERR_UNSUPPORTED  # T = 2^24 tokens: not exact as a binary32 divisor
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32, 8)
+    st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 16, None)
+    assert st == nv.ERR_INVALID_ARG  # unknown flag
 
 
 def test_product_path_does_not_import_the_oracle():

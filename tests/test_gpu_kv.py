@@ -112,3 +112,115 @@ def test_full_chunk_append_with_scale_search():
         codes, scales, a32 = oracle.kv_append(x, search46=True)
         want = oracle.kv_dequant(codes, scales, a32, T, H, d)
         assert np.array_equal(host_bits(o[0]), want)
+
+
+def _check_smoothed(cache, slot, x, which, smoothed, search):
+    """Codes, scales, tensor scale and (smoothed) channel means of one slot's K or V
+    bit for bit against the oracle; returns what the oracle's dequant needs."""
+    T, H, d = x.shape
+    if smoothed:
+        codes, scales, a32, mean = oracle.kv_append_smooth(x, search46=search)
+        m = cache.k_mean if which == 0 else cache.v_mean
+        assert np.array_equal(m[slot].cpu().numpy().view(np.uint32), mean.view(np.uint32))
+    else:
+        codes, scales, a32 = oracle.kv_append(x, search46=search)
+        mean = None
+    c = cache.k_codes if which == 0 else cache.v_codes
+    s = cache.k_scales if which == 0 else cache.v_scales
+    g = cache.k_global if which == 0 else cache.v_global
+    assert f32_bits(g[slot].cpu().numpy()) == f32_bits(a32)
+    assert np.array_equal(host_u8(c[slot]), codes.reshape(-1))
+    assert np.array_equal(host_u8(s[slot]), scales.reshape(-1))
+    if smoothed:
+        return oracle.kv_dequant_smooth(codes, scales, a32, mean, T, H, d)
+    return oracle.kv_dequant(codes, scales, a32, T, H, d)
+
+
+def _channel_biased(x, seed, scale=2.0):
+    """bf16 bits [T, H, d] plus a per-channel offset ~ N(0, scale) (bf16 nearest-even)."""
+    T, H, d = x.shape
+    g = torch.Generator().manual_seed(seed)
+    bias = torch.randn((H, d), generator=g) * scale
+    xf = torch.from_numpy(x.astype(np.int32) << 16).view(torch.float32)
+    return (xf + bias).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("smooth_k,smooth_v,search", [(True, False, False), (True, True, True), (False, True, False)])
+def test_full_chunk_append_and_dequant_with_smoothing(smooth_k, smooth_v, search):
+    """K-smoothing on the workload's 2640 x 24 x 128 chunk (K with per-channel offsets):
+    channel means, codes, scales and tensor scales bit for bit, and the bf16 dequant with
+    the means added back."""
+    require_gpu()
+    T, H, d = syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    cache = nv.KVCache(3, T, H, d, scale_search=search, smooth_k=smooth_k, smooth_v=smooth_v)
+    k, v = syn.kv_chunk_bf16(T, H, d, seed=21)
+    k = _channel_biased(k, seed=22)
+    cache.append(1, dev_bf16(k), dev_bf16(v))
+    slots = torch.tensor([1, 1], dtype=torch.int32, device="cuda")
+    ko, vo = cache.dequant(slots)
+    torch.cuda.synchronize()
+    for which, x, sm, o in ((0, k, smooth_k, ko), (1, v, smooth_v, vo)):
+        want = _check_smoothed(cache, 1, x, which, sm, search)
+        got = host_bits(o)
+        assert np.array_equal(got[0], want) and np.array_equal(got[1], want)
+
+
+@pytest.mark.parametrize("T,H,d", [(4, 3, 16), (12, 3, 16), (33, 2, 64), (64, 5, 32)])
+def test_smoothed_ring_with_ragged_shapes(T, H, d):
+    """Smoothed K and V over a ring with a page table, on shapes with fewer tokens than
+    partial sums, channel counts that are not a multiple of 64, and short last runs."""
+    require_gpu()
+    n_slots = 4
+    cache = nv.KVCache(n_slots, T, H, d, smooth_k=True, smooth_v=True)
+    latest = {}
+    for step in range(6):
+        k, v = syn.kv_chunk_bf16(T, H, d, seed=300 + step)
+        k = _channel_biased(k, seed=400 + step)
+        slot = step % n_slots
+        cache.append(slot, dev_bf16(k), dev_bf16(v))
+        latest[slot] = (k, v)
+    order = [2, 3, 0, 1, 3]
+    ko, vo = cache.dequant(torch.tensor(order, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    ko, vo = host_bits(ko), host_bits(vo)
+    for i, s in enumerate(order):
+        for which, x in enumerate(latest[s]):
+            want = _check_smoothed(cache, s, x, which, True, False)
+            assert np.array_equal((ko if which == 0 else vo)[i], want), (i, s, which)
+
+
+def test_smoothing_makes_a_channel_constant_chunk_lossless():
+    """Every token the same per channel: the smoothed values are 0, so the tensor scale
+    is 0, all codes are 0, and the dequant returns the chunk bit for bit."""
+    require_gpu()
+    T, H, d = 40, 6, 32
+    g = np.random.default_rng(5)
+    b = (g.integers(-64, 65, size=(H, d)) / 8.0).astype(np.float32)
+    x = np.broadcast_to(b, (T, H, d)).copy()
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    cache = nv.KVCache(2, T, H, d, smooth_k=True, smooth_v=True)
+    cache.append(0, dev_bf16(xb), dev_bf16(xb))
+    ko, vo = cache.dequant(torch.tensor([0], dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert float(cache.k_global[0]) == 0.0 and float(cache.v_global[0]) == 0.0
+    assert not bool(cache.k_codes[0].any()) and not bool(cache.k_scales[0].any())
+    assert np.array_equal(host_bits(ko)[0], xb) and np.array_equal(host_bits(vo)[0], xb)
+
+
+def test_smoothing_reduces_the_error_of_channel_biased_keys():
+    """Not parity: on K with per-channel offsets larger than its spread, the smoothed
+    store's dequant error is several times smaller than the plain store's."""
+    require_gpu()
+    T, H, d = 256, 8, 128
+    k, v = syn.kv_chunk_bf16(T, H, d, seed=31)
+    k = _channel_biased(k, seed=32, scale=8.0)
+    slots = torch.tensor([0], dtype=torch.int32, device="cuda")
+    errs = []
+    for smooth in (False, True):
+        cache = nv.KVCache(1, T, H, d, smooth_k=smooth)
+        cache.append(0, dev_bf16(k), dev_bf16(v))
+        ko, _ = cache.dequant(slots)
+        ref = torch.from_numpy(k.astype(np.int32) << 16).view(torch.float32)
+        got = ko[0].float().cpu()
+        errs.append(float(((got - ref) ** 2).mean()))
+    assert errs[1] * 3 < errs[0], errs
