@@ -104,6 +104,12 @@ def lib():
             L.orc_kv_append_smooth.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp]
             L.orc_kv_append_smooth.restype = ctypes.c_int
             L.orc_kv_dequant_smooth.argtypes = [vp, vp, f32, vp, i64, i64, i64, vp]
+            for name in ("orc_quantize_2d_f32", "orc_quantize_2d_bf16"):
+                getattr(L, name).argtypes = [vp, i64, i64, ctypes.c_int, vp, vp, vp, vp, vp]
+                getattr(L, name).restype = ctypes.c_int
+            L.orc_rht16_f32.argtypes = [vp, i64, vp, vp]
+            L.orc_quantize_t_bf16.argtypes = [vp, i64, i64, i64, vp, ctypes.c_int, vp, vp, vp]
+            L.orc_quantize_t_bf16.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -334,6 +340,59 @@ def kv_dequant_smooth(codes, scales, alpha, mean, T: int, H: int, d: int) -> np.
     lib().orc_kv_dequant_smooth(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)), float(alpha),
                                 _p(mean), T, H, d, _p(out))
     return out
+
+
+def quantize_2d(x: np.ndarray, alpha: float | None = None):
+    """2D block scaling (R21) of a 2-D array (bf16 bits or float32), rows and cols
+    multiples of 16.  Returns (codes [R, C/2], scales [R, C/16], codes_t [C, R/2],
+    scales_t [C, R/16], alpha): the row-wise operand and the transposed one."""
+    x = np.ascontiguousarray(x)
+    R, C = x.shape
+    codes = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    codes_t = np.zeros((C, R // 2), np.uint8)
+    scales_t = np.zeros((C, R // 16), np.uint8)
+    a = np.zeros(1, np.float32)
+    mode = MODE_COMPUTE
+    if alpha is not None:
+        a[0] = np.float32(alpha)
+        mode = MODE_GIVEN
+    fn = {np.dtype(np.uint16): lib().orc_quantize_2d_bf16, np.dtype(np.float32): lib().orc_quantize_2d_f32}[x.dtype]
+    rc = fn(_p(x), R, C, mode, _p(a), _p(codes), _p(scales), _p(codes_t), _p(scales_t))
+    if rc != 0:
+        raise ValueError(f"orc_quantize_2d failed ({rc})")
+    return codes, scales, codes_t, scales_t, np.float32(a[0])
+
+
+def rht16(x: np.ndarray, sign) -> np.ndarray:
+    """R22 on each consecutive 16-element block of float32 x (size % 16 == 0)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    sg = np.ascontiguousarray(sign, dtype=np.int8)
+    assert sg.size == 16 and x.size % 16 == 0
+    out = np.zeros_like(x)
+    lib().orc_rht16_f32(_p(x), x.size // 16, _p(sg), _p(out))
+    return out
+
+
+def quantize_t(x: np.ndarray, sign=None, alpha: float | None = None):
+    """Transposed operand of bf16 bits x [R, C] (R % 16 == 0): x^T quantized with
+    1D blocks along R, after R22 when sign (16 entries of +1/-1) is given.
+    Returns (codes_t [C, R/2], scales_t [C, R/16], alpha)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    R, C = x.shape
+    codes = np.zeros((C, R // 2), np.uint8)
+    scales = np.zeros((C, R // 16), np.uint8)
+    a = np.zeros(1, np.float32)
+    mode = MODE_COMPUTE
+    if alpha is not None:
+        a[0] = np.float32(alpha)
+        mode = MODE_GIVEN
+    sg = None if sign is None else np.ascontiguousarray(sign, dtype=np.int8)
+    rc = lib().orc_quantize_t_bf16(_p(x), R, C, C, None if sg is None else _p(sg), mode, _p(a), _p(codes),
+                                   _p(scales))
+    if rc != 0:
+        raise ValueError(f"orc_quantize_t failed ({rc})")
+    return codes, scales, np.float32(a[0])
 
 
 def ln_modulate(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6) -> np.ndarray:

@@ -53,6 +53,11 @@
  *  R20 K-smoothing of a KV chunk (optional, per tensor): subtract each
  *      channel's mean over the chunk's tokens before the quantize and add it
  *      back in the dequant; see orc_channel_mean for the order.
+ *  R21 2D block scaling of weights [RN-T]: one E4M3 scale per 16 x 16 block
+ *      from the block's amax; see orc_quantize_2d_f32.
+ *  R22 Random Hadamard Transform ahead of the weight-gradient quantize
+ *      [RN-T]: 16-point, normalised, Sylvester order, one sign vector; see
+ *      rht16.
  *
  * Every floating-point step that the GPU must reproduce bit for bit is done in
  * IEEE binary32 (compile with -ffp-contract=off so nothing fuses); the GEMM
@@ -682,4 +687,127 @@ ORC_API void orc_kv_dequant_smooth(const uint8_t* codes, const uint8_t* scales, 
             float y = v + mean[(r % H) * d + c];
             out[r * d + c] = orc_f32_to_bf16(y);
         }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Training-side NVFP4 [RN-T]: 2D block scaling of weights (R21), and the     */
+/* transposed quantize with the Random Hadamard Transform (R22) for the      */
+/* weight-gradient GEMM                                                      */
+/* ------------------------------------------------------------------------ */
+/* R21: x binary32 [rows x cols], rows and cols multiples of 16.  One E4M3
+ * scale per 16 x 16 block: amax_b over its 256 elements, s = R3 of
+ * fl32(amax_b / fl32(6 a32)), every element encoded with it (R4..R8); a32 from
+ * the tensor amax (R1, mode COMPUTE) or given.  Outputs, either pair may be
+ * NULL: codes [rows x cols/2] with logical scales [rows x cols/16] (row r,
+ * column block j holds the scale of block (r/16, j): the per-row view the
+ * block-scaled GEMM reads), and the transposed operand codes_t [cols x rows/2]
+ * with scales_t [cols x rows/16] (the same codes and scales, transposed). */
+ORC_API int orc_quantize_2d_f32(const float* x, int64_t rows, int64_t cols, int mode, float* alpha, uint8_t* codes,
+                                uint8_t* scales, uint8_t* codes_t, uint8_t* scales_t)
+{
+    if (rows % 16 != 0 || cols % 16 != 0) return 1;
+    init_tabs();
+    float a32;
+    if ((mode & ~ORC_MODE_SEARCH46) == ORC_MODE_COMPUTE) {
+        float amax = 0.0f;
+        for (int64_t i = 0; i < rows * cols; i++)
+            if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+        a32 = amax / 2688.0f; /* R1 */
+        *alpha = a32;
+    } else {
+        a32 = *alpha;
+    }
+    const int64_t br = rows / 16, bc = cols / 16;
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t bi = 0; bi < br; bi++) {
+        for (int64_t bj = 0; bj < bc; bj++) {
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; i++)
+                for (int j = 0; j < 16; j++) {
+                    float v = fabsf(x[(bi * 16 + i) * cols + bj * 16 + j]);
+                    if (v > amax_b) amax_b = v;
+                }
+            uint8_t sc = 0, q[16][16];
+            memset(q, 0, sizeof q);
+            if (a32 != 0.0f) /* R2 */
+                for (int i = 0; i < 16; i++) encode_block(x + (bi * 16 + i) * cols + bj * 16, amax_b, a32, 6.0f, &sc, q[i]);
+            for (int i = 0; i < 16; i++) {
+                const int64_t r = bi * 16 + i, c = bj * 16 + i;
+                if (codes) {
+                    for (int j = 0; j < 8; j++)
+                        codes[r * (cols / 2) + bj * 8 + j] = (uint8_t)(q[i][2 * j] | (q[i][2 * j + 1] << 4));
+                    scales[r * bc + bj] = sc;
+                }
+                if (codes_t) { /* row c of x^T: column bj*16 + i of x, its 16 rows bi*16 .. */
+                    for (int j = 0; j < 8; j++)
+                        codes_t[c * (rows / 2) + bi * 8 + j] = (uint8_t)(q[2 * j][i] | (q[2 * j + 1][i] << 4));
+                    scales_t[c * br + bi] = sc;
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+ORC_API int orc_quantize_2d_bf16(const uint16_t* x, int64_t rows, int64_t cols, int mode, float* alpha,
+                                 uint8_t* codes, uint8_t* scales, uint8_t* codes_t, uint8_t* scales_t)
+{
+    float* xf = (float*)malloc((size_t)(rows * cols) * sizeof(float) + 1);
+    if (!xf) return 2;
+    for (int64_t i = 0; i < rows * cols; i++) xf[i] = orc_bf16_to_f32(x[i]);
+    int rc = orc_quantize_2d_f32(xf, rows, cols, mode, alpha, codes, scales, codes_t, scales_t);
+    free(xf);
+    return rc;
+}
+
+/* R22: the 16-point Random Hadamard Transform of one block, in binary32:
+ * v_i = v_i * sign_i (sign_i = +1 or -1: exact), then the Walsh-Hadamard
+ * butterflies for h = 1, 2, 4, 8: for every i with (i & h) == 0,
+ * (v_i, v_{i+h}) <- (fl32(v_i + v_{i+h}), fl32(v_i - v_{i+h})), then
+ * v_i = fl32(v_i * 0.25).  In exact arithmetic y = (1/4) H diag(sign) v with H
+ * the 16 x 16 Sylvester Hadamard matrix (H_ij = (-1)^popcount(i & j)), an
+ * orthogonal map. */
+static void rht16(float* v, const int8_t* sign)
+{
+    for (int i = 0; i < 16; i++) v[i] = sign[i] < 0 ? -v[i] : v[i];
+    for (int h = 1; h < 16; h <<= 1)
+        for (int i = 0; i < 16; i++)
+            if ((i & h) == 0) {
+                float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+    for (int i = 0; i < 16; i++) v[i] = v[i] * 0.25f;
+}
+
+ORC_API void orc_rht16_f32(const float* in, int64_t n_blocks, const int8_t* sign, float* out)
+{
+    for (int64_t b = 0; b < n_blocks; b++) {
+        float v[16];
+        memcpy(v, in + b * 16, sizeof v);
+        rht16(v, sign);
+        memcpy(out + b * 16, v, sizeof v);
+    }
+}
+
+/* x bf16 [rows x cols] (rows % 16 == 0, row stride ld): the operand of a GEMM
+ * that contracts over x's rows (the weight-gradient GEMM contracts over the
+ * tokens).  x^T [cols x rows] is quantized with 1D blocks of 16 along the rows
+ * of x (R1..R8); with sign != NULL each block first goes through rht16 (R22),
+ * and the tensor scale comes from the transformed values.  Codes
+ * [cols x rows/2], logical scales [cols x rows/16]. */
+ORC_API int orc_quantize_t_bf16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, const int8_t* sign, int mode,
+                                float* alpha, uint8_t* codes_t, uint8_t* scales_t)
+{
+    if (rows % 16 != 0 || ld < cols) return 1;
+    float* xt = (float*)malloc((size_t)(rows * cols) * sizeof(float) + 1);
+    if (!xt) return 2;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) xt[c * rows + r] = orc_bf16_to_f32(x[r * ld + c]);
+    if (sign)
+        for (int64_t c = 0; c < cols; c++)
+            for (int64_t b = 0; b < rows / 16; b++) rht16(xt + c * rows + b * 16, sign);
+    int rc = orc_quantize_f32(xt, cols, rows, rows, mode, alpha, codes_t, scales_t);
+    free(xt);
+    return rc;
 }
