@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
-OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT, OP_LN_QUANTIZE = range(5)
+OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT, OP_LN_QUANTIZE, OP_QUANTIZE_2D, OP_QUANTIZE_T = range(7)
 Q_COMPUTE_GLOBAL, Q_GIVEN_GLOBAL, Q_ROWMAJOR_SCALES, Q_SCALE_SEARCH = 0, 1, 2, 4
 KV_SCALE_SEARCH, KV_SMOOTH_K, KV_SMOOTH_V = 1, 2, 4
 ACT_NONE, ACT_GELU_TANH = 0, 1
@@ -26,7 +26,7 @@ DBG_SKIP_LOADS = 1
 EXPORTS = ("nvfp4_status_string", "nvfp4_version", "nvfp4_codes_bytes", "nvfp4_scales_bytes",
            "nvfp4_workspace_bytes", "nvfp4_read_device_error", "nvfp4_quantize", "nvfp4_gemm",
            "nvfp4_kv_append", "nvfp4_kv_dequant", "nvfp4_test_encode", "nvfp4_quantize_noalloc",
-           "nvfp4_ln_modulate_quantize")
+           "nvfp4_ln_modulate_quantize", "nvfp4_quantize_2d", "nvfp4_quantize_t")
 
 
 class NVFP4Error(RuntimeError):
@@ -95,6 +95,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_ln_modulate_quantize.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_float, vp, vp, vp,
                                                  ctypes.c_uint, vp, sz, vp]
         L.nvfp4_ln_modulate_quantize.restype = st
+        L.nvfp4_quantize_2d.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, ctypes.c_uint, vp, sz, vp]
+        L.nvfp4_quantize_2d.restype = st
+        L.nvfp4_quantize_t.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, ctypes.c_uint, vp, sz, vp]
+        L.nvfp4_quantize_t.restype = st
         _lib = L
     return _lib
 
@@ -192,6 +196,59 @@ def quantize(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, out: 
     _check("nvfp4_quantize", lib().nvfp4_quantize(
         x.data_ptr(), rows, cols, x.stride(0), out.codes.data_ptr(), out.scales.data_ptr(),
         out.global_scale.data_ptr(), flags, ws.data_ptr(), ws.numel(), _stream(stream)))
+    return out
+
+
+def quantize_2d(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, want_rows: bool = True,
+                want_t: bool = True, ws: torch.Tensor | None = None, stream=None):
+    """2D (16 x 16 block) scaling of a bf16 weight [rows, cols]: returns
+    (operand of x, operand of x^T), either None when not wanted; both share the
+    tensor scale (computed as amax / 2688 unless global_scale is given)."""
+    _require_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("quantize_2d takes a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    a = empty_nvfp4(rows, cols, x.device) if want_rows else None
+    t = empty_nvfp4(cols, rows, x.device) if want_t else None
+    gs = (a or t).global_scale
+    flags = 0
+    if global_scale is not None:
+        gs.copy_(global_scale.reshape(1))
+        flags |= Q_GIVEN_GLOBAL
+    if ws is None:
+        ws = workspace(OP_QUANTIZE_2D, rows, 0, cols, x.device)
+    _check("nvfp4_quantize_2d", lib().nvfp4_quantize_2d(
+        x.data_ptr(), rows, cols, x.stride(0), _ptr(a.codes if a else None), _ptr(a.scales if a else None),
+        _ptr(t.codes if t else None), _ptr(t.scales if t else None), gs.data_ptr(), flags, ws.data_ptr(),
+        ws.numel(), _stream(stream)))
+    if a is not None and t is not None:
+        t.global_scale = a.global_scale
+    return a, t
+
+
+def quantize_t(x: torch.Tensor, *, rht_sign=None, global_scale: torch.Tensor | None = None,
+               out: NVFP4Tensor | None = None, ws: torch.Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """The operand of a GEMM contracting over x's rows (bf16 [rows, cols]):
+    x^T quantized with 1D blocks along the rows, after the 16-point Random
+    Hadamard Transform when rht_sign (16 values of +1 / -1) is given."""
+    _require_cuda(x)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("quantize_t takes a 2-D bf16 tensor with unit column stride")
+    rows, cols = x.shape
+    if out is None:
+        out = empty_nvfp4(cols, rows, x.device)
+    flags = 0
+    if global_scale is not None:
+        out.global_scale.copy_(global_scale.reshape(1))
+        flags |= Q_GIVEN_GLOBAL
+    if ws is None:
+        ws = workspace(OP_QUANTIZE_T, rows, 0, cols, x.device)
+    sign = None
+    if rht_sign is not None:
+        sign = (ctypes.c_int8 * 16)(*[int(v) for v in rht_sign])
+    _check("nvfp4_quantize_t", lib().nvfp4_quantize_t(
+        x.data_ptr(), rows, cols, x.stride(0), out.codes.data_ptr(), out.scales.data_ptr(),
+        out.global_scale.data_ptr(), sign, flags, ws.data_ptr(), ws.numel(), _stream(stream)))
     return out
 
 

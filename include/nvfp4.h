@@ -90,7 +90,9 @@ enum {
     NVFP4_OP_GEMM = 1,      /* nvfp4_gemm */
     NVFP4_OP_KV_APPEND = 2, /* nvfp4_kv_append */
     NVFP4_OP_KV_DEQUANT = 3, /* nvfp4_kv_dequant */
-    NVFP4_OP_LN_QUANTIZE = 4 /* nvfp4_ln_modulate_quantize (m = rows) */
+    NVFP4_OP_LN_QUANTIZE = 4, /* nvfp4_ln_modulate_quantize (m = rows) */
+    NVFP4_OP_QUANTIZE_2D = 5, /* nvfp4_quantize_2d */
+    NVFP4_OP_QUANTIZE_T = 6   /* nvfp4_quantize_t */
 };
 
 /* Workspace bytes the caller must pass to the call `op` (device memory,
@@ -290,6 +292,38 @@ nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const vo
 nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n, void* k_out_bf16,
                               void* v_out_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 
+
+/* ------------------------------------------------------------------------ */
+/* Training-side operands  [RN-T] "NVFP4 训练的工程细节"                        */
+/* ------------------------------------------------------------------------ */
+/* 2D block scaling of a weight x (bf16 [rows x cols], row stride ld elements;
+ * rows % 64 == 0, cols % 64 == 0): one E4M3 scale per 16 x 16 block,
+ * s = E4M3_rne_sat(amax_block / (6 * a32)), every element encoded with it as
+ * in nvfp4_quantize (a32 = amax / 2688 over the tensor, or given with
+ * NVFP4_Q_GIVEN_GLOBAL).  Writes the GEMM operand of x (codes [rows x cols/2],
+ * swizzled scales of [rows x cols/16], each row holding its block's scale)
+ * and/or the operand of x^T (codes_t [cols x rows/2], swizzled scales_t of
+ * [cols x rows/16]): the same codes and scales, transposed (pass NULL for a
+ * pair not wanted, not both).  Two launches (amax, encode); workspace:
+ * nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_2D, rows, 0, cols) bytes. */
+nvfp4_status nvfp4_quantize_2d(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
+                               void* scales, void* codes_t, void* scales_t, float* global_scale, unsigned flags,
+                               void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* The operand of a GEMM that contracts over x's rows (the weight gradient
+ * dW = dY^T X contracts over tokens): x^T [cols x rows] quantized with 1D
+ * blocks of 16 along the rows of x (codes_t [cols x rows/2], swizzled
+ * scales_t of [cols x rows/16]).  With rht_sign (host array of 16 int8 values,
+ * each +1 or -1; NULL: no transform), each 16-element block along the rows
+ * first goes through the Random Hadamard Transform y = (1/4) H_16 diag(sign) v
+ * in binary32 (signs, then butterflies h = 1, 2, 4, 8 with (a + b, a - b),
+ * then * 0.25), and a32 comes from max |y|.  Use the same signs for both
+ * operands of the product so the transform cancels.  rows % 64 == 0,
+ * cols % 16 == 0.  Two launches; workspace:
+ * nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_T, rows, 0, cols) bytes. */
+nvfp4_status nvfp4_quantize_t(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes_t,
+                              void* scales_t, float* global_scale, const int8_t* rht_sign, unsigned flags,
+                              void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Test support                                                              */

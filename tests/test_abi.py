@@ -101,6 +101,20 @@ def test_host_side_argument_checks(L):
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32, 8)
     st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 16, None)
     assert st == nv.ERR_INVALID_ARG  # unknown flag
+    # training-side operands: shapes, outputs, signs and alignment are checked before any launch
+    q2 = L.nvfp4_quantize_2d
+    assert q2(fake, 96, 64, 64, fake, fake, fake, fake, fake, 0, fake, 256, None) == nv.ERR_UNSUPPORTED  # rows % 64
+    assert q2(fake, 64, 48, 48, fake, fake, fake, fake, fake, 0, fake, 256, None) == nv.ERR_UNSUPPORTED  # cols % 64
+    assert q2(fake, 64, 64, 64, None, None, None, None, fake, 0, fake, 256, None) == nv.ERR_INVALID_ARG  # no output
+    assert q2(fake, 64, 64, 64, fake, None, None, None, fake, 0, fake, 256, None) == nv.ERR_INVALID_ARG  # half a pair
+    assert q2(fake, 64, 64, 64, fake + 8, fake, None, None, fake, 0, fake, 256, None) == nv.ERR_MISALIGNED
+    assert q2(fake, 64, 64, 64, fake, fake, None, None, fake, 0, fake, 16, None) == nv.ERR_INVALID_ARG  # workspace
+    qt = L.nvfp4_quantize_t
+    assert qt(fake, 64, 24, 24, fake, fake, fake, None, 0, fake, 256, None) == nv.ERR_UNSUPPORTED  # cols % 16
+    bad = (ctypes.c_int8 * 16)(*([1] * 15 + [2]))
+    assert qt(fake, 64, 32, 32, fake, fake, fake, bad, 0, fake, 256, None) == nv.ERR_INVALID_ARG  # sign not +-1
+    assert qt(fake, 64, 32, 32, fake, fake, fake, None, 2, fake, 256, None) == nv.ERR_INVALID_ARG  # unknown flag
+    assert qt(fake, 64, 32, 36, fake, fake, fake, None, 0, fake, 256, None) == nv.ERR_MISALIGNED  # ld % 8
 
 
 def test_product_path_does_not_import_the_oracle():
