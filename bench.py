@@ -223,6 +223,52 @@ def measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, rep
             "smooth_append_ms": sm_ap_ms, "smooth_dequant_ms": sm_dq_ms}
 
 
+RHT_SIGN = (1, -1, -1, 1, 1, 1, -1, 1, -1, -1, 1, -1, 1, 1, -1, -1)
+
+
+def measure_training(nv, a, w, cache, ring, k_out, v_out, reps: int) -> dict:
+    """ms per launch pair of the training-side operands and the weight-gradient GEMM on
+    the QKV shapes: 2D scaling of W [9216 x 3072] (both operands), the RHT transposed
+    operands of X [4096 x 3072] and dY [4096 x 9216], and dW = dY^T X (231.9 GFLOP)."""
+    M, K = a.shape
+    N = w.shape[0]
+    g = torch.Generator(device=a.device).manual_seed(77)
+    dy = torch.randn((M, N), generator=g, device=a.device).to(torch.bfloat16)
+    w2, w2t = nv.quantize_2d(w)
+    ws2 = nv.workspace(nv.OP_QUANTIZE_2D, N, 0, K, a.device)
+    xt = nv.quantize_t(a, rht_sign=RHT_SIGN)
+    dyt = nv.quantize_t(dy, rht_sign=RHT_SIGN)
+    wst = nv.workspace(nv.OP_QUANTIZE_T, M, 0, K, a.device)
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device=a.device)
+    wsg = nv.workspace(nv.OP_GEMM, N, K, M, a.device)
+    nv.gemm(dyt, xt, out=dw, ws=wsg)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(8)] for _ in range(reps)]
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for i in range(reps):
+            cache.dequant(ring, k_out, v_out)
+            ev[i][0].record()
+            nv.quantize_2d(w, out=w2, out_t=w2t, ws=ws2)
+            ev[i][1].record()
+            cache.dequant(ring, k_out, v_out)
+            ev[i][2].record()
+            nv.quantize_t(a, rht_sign=RHT_SIGN, out=xt, ws=wst)
+            ev[i][3].record()
+            nv.quantize_t(dy, rht_sign=RHT_SIGN, out=dyt, ws=wst)
+            ev[i][4].record()
+            cache.dequant(ring, k_out, v_out)
+            ev[i][5].record()
+            nv.gemm(dyt, xt, out=dw, ws=wsg)
+            ev[i][6].record()
+    gr.replay()
+    torch.cuda.synchronize()
+    med = lambda j: float(np.median([e[j].elapsed_time(e[j + 1]) for e in ev]))
+    out = {"quantize_2d_ms": med(0), "quantize_t_x_ms": med(2), "quantize_t_dy_ms": med(3), "wgrad_ms": med(5)}
+    del gr
+    return out
+
+
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
@@ -334,6 +380,9 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     # timed the same way (inside a graph, each after a dequant of all slots so
     # that its input comes from HBM); reported beside the step, not part of it.
     search = measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, reps=5)
+    # the training-side operands (2D weight scaling, RHT transposed operands) and the
+    # weight-gradient GEMM on the same layer shapes, also beside the step
+    train = measure_training(nv, a, dev_bf16(w_host), cache, ring, k_out, v_out, reps=5)
 
     total_ms = t_start.elapsed_time(t_end)
     comp = np.zeros(4)
@@ -438,6 +487,18 @@ def run_ours(args, rank: int, world: int) -> dict | None:
             "append_GB/s": round(append_bytes / (search["smooth_append_ms"] * 1e-3) / 1e9, 1),
             "dequant_ms": round(search["smooth_dequant_ms"], 4),
             "dequant_GB/s": round(dequant_bytes / (search["smooth_dequant_ms"] * 1e-3) / 1e9, 1)},
+        "training": {
+            "what": "training-side NVFP4 on the QKV layer shapes, outside the step: 2D (16x16) scaling of W "
+                    "[9216x3072] writing W and W^T operands; RHT + transposed 1D quantize of X [4096x3072] and "
+                    "dY [4096x9216] (weight-gradient operands); dW = dY^T X (9216x3072x4096) on those operands",
+            "quantize_2d_ms": round(train["quantize_2d_ms"], 4),
+            "quantize_2d_GB/s": round(N * K * 3.125 / (train["quantize_2d_ms"] * 1e-3) / 1e9, 1),
+            "quantize_t_x_ms": round(train["quantize_t_x_ms"], 4),
+            "quantize_t_x_GB/s": round(M * K * 2.5625 / (train["quantize_t_x_ms"] * 1e-3) / 1e9, 1),
+            "quantize_t_dy_ms": round(train["quantize_t_dy_ms"], 4),
+            "quantize_t_dy_GB/s": round(M * N * 2.5625 / (train["quantize_t_dy_ms"] * 1e-3) / 1e9, 1),
+            "wgrad_ms": round(train["wgrad_ms"], 4),
+            "wgrad_TFLOP/s": round(2.0 * N * K * M / (train["wgrad_ms"] * 1e-3) / 1e12, 1)},
         "ln_modulate_quantize": {
             "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A, two launches, outside the step",
             "ms": round(search["ln_quantize_ms"], 4),

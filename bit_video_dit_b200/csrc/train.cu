@@ -6,14 +6,14 @@
 //
 // Both run as two launches on the caller's stream: an amax pass (the tensor
 // scale a32 = amax / 2688 needs the whole tensor) and an encode pass.  A warp
-// owns a 64-row x 64-column tile of x (rows % 64 == 0): lane l holds columns
-// 2l and 2l + 1 of the tile for all 64 rows (64 four-byte loads, each warp
+// owns a 32-row x 64-column tile of x (rows % 64 == 0): lane l holds columns
+// 2l and 2l + 1 of the tile for all 32 rows (32 four-byte loads, each warp
 // load 128 contiguous bytes), so a 16-element block along the rows is one
 // lane's register column and a 16 x 16 block is eight lanes.  Per column the
-// lane writes the transposed operand's 32 code bytes (two 16-byte stores) and
-// its 4 scale bytes (one 4-byte store into the swizzled tile); the 2D mode
+// lane writes the transposed operand's 16 code bytes (one 16-byte store) and
+// its 2 scale bytes (one 2-byte store into the swizzled tile); the 2D mode
 // also writes the row-wise operand (a byte per row and lane, 32 contiguous
-// bytes per warp store) and its scales.
+// bytes per warp store) and its scales.  The grid is one resident wave.
 #include <algorithm>
 #include <cstdint>
 
@@ -24,6 +24,7 @@ namespace train {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
+constexpr int kTileRows = 32;
 
 struct TrainArgs {
     const uint8_t* x;      // bf16 [rows][ld]
@@ -52,25 +53,40 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
     return out;
 }
 
-// The 16-point Random Hadamard Transform of one block, binary32: the signs
+// The 16-point Random Hadamard Transform of a block, binary32: the signs
 // (exact), butterflies h = 1, 2, 4, 8 with (a + b, a - b), then * 0.25 (the
 // 1 / sqrt(16) normalisation): y = (1/4) H_16 diag(sign) v, H_16 the
 // Sylvester Hadamard matrix.
-__device__ __forceinline__ void rht16(float* v, uint32_t sign_mask) {
+// The same transform on two blocks at once (columns c and c + 1 of a lane):
+// element i of both blocks in one 64-bit pair, the packed binary32 add, sub
+// and multiply rounding each lane as the scalar operation does.
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ void rht16x2(float* f0, float* f1, uint32_t sign_mask) {
+    uint64_t v[16];
 #pragma unroll
-    for (int i = 0; i < 16; i++)
-        v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((sign_mask >> i) & 1u) << 31));
+    for (int i = 0; i < 16; i++) {
+        const uint64_t flip = (uint64_t)((sign_mask >> i) & 1u) * 0x8000000080000000ull;
+        v[i] = pk(f0[i], f1[i]) ^ flip;
+    }
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1)
 #pragma unroll
         for (int i = 0; i < 16; i++)
             if ((i & h) == 0) {
-                const float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
+                const uint64_t a = v[i], b = v[i + h];
+                asm("add.rn.f32x2 %0, %1, %2;" : "=l"(v[i]) : "l"(a), "l"(b));
+                asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(v[i + h]) : "l"(a), "l"(b));
             }
+    const uint64_t q = pk(0.25f, 0.25f);
 #pragma unroll
-    for (int i = 0; i < 16; i++) v[i] = __fmul_rn(v[i], 0.25f);
+    for (int i = 0; i < 16; i++) {
+        uint64_t r;
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(v[i]), "l"(q));
+        f0[i] = __uint_as_float((uint32_t)r);
+        f1[i] = __uint_as_float((uint32_t)(r >> 32));
+    }
 }
 
 __device__ __forceinline__ float absmax16(const float* f) {
@@ -94,7 +110,7 @@ __device__ __forceinline__ float block_inv(uint32_t code, float a32) {
 // with 1D blocks along the rows (RHT: after the transform).  ENCODE = false
 // is the amax pass.
 template <bool TWO_D, bool RHT, bool ENCODE>
-__global__ void __launch_bounds__(kThreads) train_quant_kernel(const __grid_constant__ TrainArgs a) {
+__global__ void __launch_bounds__(kThreads, (RHT && ENCODE) ? 2 : 3) train_quant_kernel(const __grid_constant__ TrainArgs a) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * kWarps;
     float a32 = 0.0f, d6 = 0.0f;
@@ -109,27 +125,24 @@ __global__ void __launch_bounds__(kThreads) train_quant_kernel(const __grid_cons
     const int64_t tiles_c_r = a.cols / 64;          // row-wise operand (2D)
     for (int64_t t = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); t < a.ntiles; t += nwarps) {
         const int tr = (int)(t / a.tiles_c), tc = (int)(t - (int64_t)tr * a.tiles_c);
-        const int r0 = tr * 64, c = tc * 64 + 2 * lane;
+        const int r0 = tr * kTileRows, c = tc * 64 + 2 * lane;
         const bool active = c < a.cols;  // cols % 16 == 0: whole 8-lane groups
-        uint32_t v[64];
+        uint32_t v[kTileRows];
         const uint8_t* src = a.x + ((int64_t)r0 * a.ld + c) * 2;
 #pragma unroll
-        for (int i = 0; i < 64; i++)
+        for (int i = 0; i < kTileRows; i++)
             v[i] = active ? __ldg(reinterpret_cast<const uint32_t*>(src + (int64_t)i * a.ld * 2)) : 0u;
-        uint32_t ct[2][8];  // transposed codes of the two columns: 64 rows -> 8 words each
+        uint32_t ct[2][4];  // transposed codes of the two columns: 32 rows -> 4 words each
         uint32_t st[2] = {0u, 0u};
 #pragma unroll
-        for (int b = 0; b < 4; b++) {
+        for (int b = 0; b < kTileRows / 16; b++) {
             float f0[16], f1[16];
 #pragma unroll
             for (int i = 0; i < 16; i++) {
                 f0[i] = __uint_as_float(v[16 * b + i] << 16);
                 f1[i] = __uint_as_float(v[16 * b + i] & 0xFFFF0000u);
             }
-            if (RHT) {
-                rht16(f0, a.sign_mask);
-                rht16(f1, a.sign_mask);
-            }
+            if (RHT) rht16x2(f0, f1, a.sign_mask);
             const float m0 = absmax16(f0), m1 = absmax16(f1);
             if (!ENCODE) {
                 lane_max = fmaxf(lane_max, fmaxf(m0, m1));
@@ -148,10 +161,13 @@ __global__ void __launch_bounds__(kThreads) train_quant_kernel(const __grid_cons
             }
             const float inv0 = block_inv(code0, a32), inv1 = block_inv(code1, a32);
             float y0[16], y1[16];
+            const uint64_t inv2 = pk(inv0, inv1);
 #pragma unroll
             for (int i = 0; i < 16; i++) {
-                y0[i] = __fmul_rn(f0[i], inv0);
-                y1[i] = __fmul_rn(f1[i], inv1);
+                uint64_t r;
+                asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(f0[i], f1[i])), "l"(inv2));
+                y0[i] = __uint_as_float((uint32_t)r);
+                y1[i] = __uint_as_float((uint32_t)(r >> 32));
             }
             ct[0][2 * b] = inv0 == 0.0f ? 0u : e2m1x8(y0);
             ct[0][2 * b + 1] = inv0 == 0.0f ? 0u : e2m1x8(y0 + 8);
@@ -179,9 +195,9 @@ __global__ void __launch_bounds__(kThreads) train_quant_kernel(const __grid_cons
             for (int j = 0; j < 2; j++) {
                 uint8_t* dst = a.codes_t + (int64_t)(c + j) * code_ld_t + r0 / 2;
                 *reinterpret_cast<uint4*>(dst) = make_uint4(ct[j][0], ct[j][1], ct[j][2], ct[j][3]);
-                *reinterpret_cast<uint4*>(dst + 16) = make_uint4(ct[j][4], ct[j][5], ct[j][6], ct[j][7]);
-                // scale columns r0/16 .. r0/16 + 3 of row c + j: 4 contiguous bytes
-                *reinterpret_cast<uint32_t*>(a.scales_t + swz_offset(c + j, r0 / 16, tiles_c_t)) = st[j];
+                // scale columns r0/16 and r0/16 + 1 of row c + j: 2 contiguous
+                // bytes (r0/16 is even, so they share a 4-byte group)
+                *reinterpret_cast<uint16_t*>(a.scales_t + swz_offset(c + j, r0 / 16, tiles_c_t)) = (uint16_t)st[j];
             }
         }
     }
@@ -226,14 +242,24 @@ nvfp4_status zero_padding(uint8_t* scales, int64_t rows, int64_t sc, cudaStream_
 template <bool TWO_D, bool RHT>
 nvfp4_status run(TrainArgs& a, cudaStream_t s) {
     a.tiles_c = (a.cols + 63) / 64;
-    a.ntiles = (a.rows / 64) * a.tiles_c;
+    a.ntiles = (a.rows / kTileRows) * a.tiles_c;
     const int64_t want = ((int64_t)a.ntiles + kWarps - 1) / kWarps;
-    const int g = (int)std::min<int64_t>(want, (int64_t)sm_count() * 4);
+    // one resident wave of each pass (blocks per SM from the occupancy query)
+    static int resident[2] = {0, 0};
+    for (int e = 0; e < 2; e++)
+        if (resident[e] == 0) {
+            int b = 0;
+            auto k = e ? train_quant_kernel<TWO_D, RHT, true> : train_quant_kernel<TWO_D, RHT, false>;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, kThreads, 0) != cudaSuccess || b < 1) b = 1;
+            resident[e] = b;
+        }
     if (!a.given) {
         if (cudaMemsetAsync(a.amax_word, 0, 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+        const int g = (int)std::min<int64_t>(want, (int64_t)sm_count() * resident[0]);
         train_quant_kernel<TWO_D, RHT, false><<<g, kThreads, 0, s>>>(a);
         if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     }
+    const int g = (int)std::min<int64_t>(want, (int64_t)sm_count() * resident[1]);
     train_quant_kernel<TWO_D, RHT, true><<<g, kThreads, 0, s>>>(a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

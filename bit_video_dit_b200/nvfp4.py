@@ -200,7 +200,8 @@ def quantize(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, out: 
 
 
 def quantize_2d(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, want_rows: bool = True,
-                want_t: bool = True, ws: torch.Tensor | None = None, stream=None):
+                want_t: bool = True, out: NVFP4Tensor | None = None, out_t: NVFP4Tensor | None = None,
+                ws: torch.Tensor | None = None, stream=None):
     """2D (16 x 16 block) scaling of a bf16 weight [rows, cols]: returns
     (operand of x, operand of x^T), either None when not wanted; both share the
     tensor scale (computed as amax / 2688 unless global_scale is given)."""
@@ -208,8 +209,8 @@ def quantize_2d(x: torch.Tensor, *, global_scale: torch.Tensor | None = None, wa
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("quantize_2d takes a 2-D bf16 tensor with unit column stride")
     rows, cols = x.shape
-    a = empty_nvfp4(rows, cols, x.device) if want_rows else None
-    t = empty_nvfp4(cols, rows, x.device) if want_t else None
+    a = (out or empty_nvfp4(rows, cols, x.device)) if want_rows else None
+    t = (out_t or empty_nvfp4(cols, rows, x.device)) if want_t else None
     gs = (a or t).global_scale
     flags = 0
     if global_scale is not None:
