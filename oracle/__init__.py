@@ -6,7 +6,9 @@ path (``bit_video_dit_b200``) never imports it and shares no code with it.
 
 The arithmetic lives in ``nvfp4_oracle.c`` (plain C, binary32 steps with
 ``-ffp-contract=off``, binary64 GEMM accumulation); this module only builds
-that file with gcc and marshals numpy arrays through ctypes.  Format source:
+that file with gcc and marshals numpy arrays through ctypes; the attention over
+the cache (its chunk set and fp64 softmax attention) is written out in plain
+numpy below.  Format source:
 "LongLive-2.0：用 NVFP4 并行底座做长视频生成" (yingwang.github.io reading note),
 section 二 方法 / "NVFP4 量化格式" (E2M1 codes, per-16 E4M3 block scale, FP32
 tensor scale, the Dequant equation) and "推理底座" (per-chunk KV quantization).
@@ -393,6 +395,32 @@ def quantize_t(x: np.ndarray, sign=None, alpha: float | None = None):
     if rc != 0:
         raise ValueError(f"orc_quantize_t failed ({rc})")
     return codes, scales, np.float32(a[0])
+
+
+def attention_chunks(t: int, sink_global: int, shot_start: int, sink_shot: int, window: int) -> list[int]:
+    """The chunk indices chunk t attends to in the cache (reading note, section 二, the multi-shot anchors):
+    A_g = the video's first sink_global chunks, A_s = the current shot's first sink_shot chunks (the shot starts
+    at chunk shot_start), and the window KV[t - window, t); their union without repeats, only chunks already
+    made (index < t), ascending."""
+    s = set(range(0, sink_global)) | set(range(shot_start, shot_start + sink_shot)) | set(range(t - window, t))
+    return sorted(c for c in s if 0 <= c < t)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
+    """fp64 softmax attention of bf16 bits q [Tq, H, d] over bf16 bits k, v [L, H, d] (every query sees every
+    key): O[i, h] = sum_j softmax_j(scale * q[i, h] . k[j, h]) v[j, h].  Returns float64 [Tq, H, d]."""
+    qf = (q.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    kf = (k.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    vf = (v.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    Tq, H, d = qf.shape
+    out = np.zeros((Tq, H, d), np.float64)
+    for h in range(H):
+        s = (qf[:, h, :] @ kf[:, h, :].T) * scale
+        s -= s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=1, keepdims=True)
+        out[:, h, :] = p @ vf[:, h, :]
+    return out
 
 
 def ln_modulate(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6) -> np.ndarray:
