@@ -48,7 +48,8 @@ extern "C" size_t nvfp4_workspace_bytes(int op, int64_t m, int64_t n, int64_t k)
         case NVFP4_OP_GEMM:
         case NVFP4_OP_KV_DEQUANT:
         case NVFP4_OP_QUANTIZE_2D:  // error record, then the amax word at byte 128
-        case NVFP4_OP_QUANTIZE_T: return kWsControl;
+        case NVFP4_OP_QUANTIZE_T:
+        case NVFP4_OP_KV_ATTENTION: return kWsControl;
         case NVFP4_OP_LN_QUANTIZE:  // control block, then (mean, rstd) per row
             return kWsControl + (size_t)(m > 0 ? m : 0) * 8;
     }

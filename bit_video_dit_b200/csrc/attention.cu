@@ -1,0 +1,414 @@
+// Attention of bf16 queries over NVFP4 KV-cache slots, reading the cache
+// directly (the reading note's KV store, section 二 推理底座, and its attention
+// anchors: the caller lists the slots of A_g | A_s | KV[t - W, t)).
+//
+// One CTA per (128-query tile, head), 128 threads: thread i owns query row i
+// and TMEM lane i.  K and V tiles of 128 tokens are dequantized from the slot
+// (E2M1 codes, E4M3 block scales, the slot's a32, the K-smoothing mean when
+// the cache has one) straight into shared memory in the layouts the tensor
+// cores read, with each thread writing its token's row as 16-byte chunks:
+//   Q, K, P: K-major, no swizzle: element (row r, column c) at
+//            (c / 8) * 2048 + r * 16 + (c % 8) * 2 (8-row core matrices 128
+//            bytes apart, 8-column chunks 2048 bytes apart);
+//   V:       MN-major (the d columns are the MMA's N): element (token t, dim j)
+//            at (j / 8) * 2048 + t * 16 + (j % 8) * 2.
+// S = Q K^T and O += P V run as tcgen05.mma kind::f16 (bf16 operands, binary32
+// accumulators in TMEM: S in columns [0, 128), O in [128, 256)), issued by
+// thread 0 and waited on through an mbarrier.  The softmax takes two passes
+// over the keys: the first finds each row's max and sum of exponentials, the
+// second forms P = exp(scale * (s - max)) in bf16 and accumulates P V, so the
+// output never needs rescaling; O / sum is stored as bf16.  Every wait is
+// bounded; a timeout records NVFP4_ERR_TIMEOUT and the CTA stops.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace attn {
+
+constexpr int kD = 128;       // head_dim (the tile's K for Q K^T, N for P V)
+constexpr int kTile = 128;    // queries per CTA, keys per KV tile
+constexpr int kThreads = 128;
+constexpr int kOperandBytes = kTile * kD * 2;  // 32 KB per bf16 128 x 128 operand
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kSCol = 0, kOCol = 128;
+
+struct AttnArgs {
+    const uint8_t* q;            // bf16 [Tq][H][d]
+    uint8_t* o;                  // bf16 [Tq][H][d]
+    const uint8_t* codes[2];     // K, V codes of slot 0 (slot s at + s * slot_elems / 2)
+    const uint8_t* scales[2];    // K, V row-major scales
+    const float* gscale[2];      // [n_slots]
+    const float* mean[2];        // K-smoothing means [n_slots][H * d] or NULL
+    const int32_t* slots;
+    int n, n_slots, tq, tokens, heads;
+    int64_t slot_elems;
+    float scale_log2;            // softmax scale * log2(e)
+    DevError* err;
+    uint64_t limit_ns;
+};
+
+// instruction descriptor of kind::f16: binary32 accumulator, bf16 A and B,
+// A K-major, B K-major (b_mn = 0) or MN-major (1), M = N = 128
+__host__ __device__ constexpr uint32_t idesc_f16(int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(kTile >> 3) << 17) |
+           ((uint32_t)(kTile >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void st_shared16(uint32_t addr, const uint4& v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// 8 E2M1 codes with their block scale and the slot's a32 -> 8 bf16, as the
+// cache's dequant: bf16_rne(fl32(fl32(e2m1 * s) * a32) [+ mean]).
+__device__ __forceinline__ uint4 dq8(uint32_t q, uint32_t sc, float a32, const float* m) {
+    const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const float2 f = __half22float2(__hmul2(e2m1x2_to_half2((q >> (8 * j)) & 0xFFu), s2));
+        float y0 = __fmul_rn(f.x, a32), y1 = __fmul_rn(f.y, a32);
+        if (m) {
+            y0 = __fadd_rn(y0, __ldg(m + 2 * j));
+            y1 = __fadd_rn(y1, __ldg(m + 2 * j + 1));
+        }
+        const __nv_bfloat162 b = __floats2bfloat162_rn(y0, y1);
+        o[j] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Thread i's token row (token `tok` of slot s, head h) of K or V into the
+// operand at `base` (K-major and MN-major layouts put a row at the same
+// places); zeros when the token is past the slot's end.
+__device__ __forceinline__ void load_kv_row(const AttnArgs& a, int t, int s, int tok, int h, uint32_t base, int row) {
+    uint4 v[16];
+    if (tok < a.tokens) {
+        const int64_t e = (int64_t)s * a.slot_elems + ((int64_t)tok * a.heads + h) * kD;
+        const uint4* cp = reinterpret_cast<const uint4*>(a.codes[t] + e / 2);
+        const uint2 sp = __ldg(reinterpret_cast<const uint2*>(a.scales[t] + e / 16));
+        const float a32 = __ldg(a.gscale[t] + s);
+        const float* m = a.mean[t] ? a.mean[t] + ((int64_t)s * a.heads + h) * kD : nullptr;
+        const uint32_t sw[2] = {sp.x, sp.y};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const uint4 c = __ldg(cp + k);
+            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int chunk = 4 * k + j;  // elements 8 * chunk .. + 7; block chunk / 2
+                const uint32_t sc = (sw[chunk / 8] >> (8 * ((chunk / 2) % 4))) & 0xFFu;
+                v[chunk] = dq8(cw[j], sc, a32, m ? m + 8 * chunk : nullptr);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 16; c++) v[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int c = 0; c < 16; c++) st_shared16(base + c * 2048 + row * 16, v[c]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_constant__ AttnArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ uint64_t bar_s, bar_o;
+    __shared__ uint32_t tmem_base;
+    __shared__ int s_abort;
+    const int i = threadIdx.x;  // query row, TMEM lane
+    const int warp = i >> 5;
+    const int qt = blockIdx.x, h = blockIdx.y;
+    const uint32_t q_s = smem_u32(smem), k_s = q_s + kOperandBytes, v_s = k_s + kOperandBytes,
+                   p_s = v_s + kOperandBytes;
+    if (i == 0) {
+        mbar_init(&bar_s, 1);
+        mbar_init(&bar_o, 1);
+        s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    // Q row i (zeros past the last query)
+    {
+        const int qrow = qt * kTile + i;
+        uint4 v[16];
+        if (qrow < a.tq) {
+            const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)qrow * a.heads + h) * kD * 2);
+#pragma unroll
+            for (int c = 0; c < 16; c++) v[c] = __ldg(src + c);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 16; c++) v[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int c = 0; c < 16; c++) st_shared16(q_s + c * 2048 + i * 16, v[c]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    const uint32_t t_s = tmem + kSCol, t_o = tmem + kOCol;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    constexpr uint32_t ID_QK = idesc_f16(0), ID_PV = idesc_f16(1);
+    const int tiles_per_slot = (a.tokens + kTile - 1) / kTile;
+    uint32_t ph_s = 0, ph_o = 0;
+    bool ok = true;
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool first_pv = true;
+
+    for (int pass = 0; pass < 2 && ok; pass++) {
+        for (int si = 0; si < a.n && ok; si++) {
+            const int s = __ldg(a.slots + si);
+            if (s < 0 || s >= a.n_slots) {
+                if (pass == 0 && i == 0 && qt == 0 && h == 0) record_error(a.err, NVFP4_ERR_DEVICE, (uint32_t)si);
+                continue;  // uniform over the CTA
+            }
+            for (int kt = 0; kt < tiles_per_slot && ok; kt++) {
+                const int tok = kt * kTile + i;
+                const int valid = min(kTile, a.tokens - kt * kTile);
+                // the previous P V product must be done with K, V and P
+                // (every wait's outcome is made uniform over the CTA before
+                // anyone acts on it, so all threads take the same barriers)
+                if (pass == 1 && !first_pv) {
+                    const bool got = mbar_wait_bounded(&bar_o, ph_o, &s_abort, a.limit_ns);
+                    ph_o ^= 1u;
+                    if (!__syncthreads_and(got)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                load_kv_row(a, 0, s, tok, h, k_s, i);
+                if (pass == 1) load_kv_row(a, 1, s, tok, h, v_s, i);
+                fence_proxy_async_smem();
+                __syncthreads();
+                if (i == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kD / 16; k++)
+                        mma_f16(t_s, smem_desc(q_s + k * 4096, 2048, 128, kLayoutNone),
+                                smem_desc(k_s + k * 4096, 2048, 128, kLayoutNone), ID_QK, k > 0);
+                    tc_commit(&bar_s);
+                }
+                {
+                    const bool got = mbar_wait_bounded(&bar_s, ph_s, &s_abort, a.limit_ns);
+                    ph_s ^= 1u;
+                    if (!__syncthreads_and(got)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                tc_fence_after();
+                uint32_t r[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; c++) tmem_ld_32cols(t_s + lane_off + 32 * c, r[c]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
+                if (pass == 0) {
+                    float mt = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 4; c++)
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (32 * c + j < valid) mt = fmaxf(mt, __uint_as_float(r[c][j]));
+                    const float m_new = fmaxf(m_run, mt);
+                    float sum = 0.0f;
+#pragma unroll
+                    for (int c = 0; c < 4; c++)
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (32 * c + j < valid) sum += ex2((__uint_as_float(r[c][j]) - m_new) * a.scale_log2);
+                    l_run = l_run * ex2((m_run - m_new) * a.scale_log2) + sum;
+                    m_run = m_new;
+                } else {
+                    // P row i: exp(scale * (s - max)) in bf16, zero for keys past the slot's end
+#pragma unroll
+                    for (int c = 0; c < 4; c++)
+#pragma unroll
+                        for (int g = 0; g < 4; g++) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; e++) {
+                                const int j0 = 32 * c + 8 * g + 2 * e;
+                                const float p0 = j0 < valid ? ex2((__uint_as_float(r[c][8 * g + 2 * e]) - m_run) * a.scale_log2) : 0.0f;
+                                const float p1 = j0 + 1 < valid ? ex2((__uint_as_float(r[c][8 * g + 2 * e + 1]) - m_run) * a.scale_log2) : 0.0f;
+                                const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
+                                w[e] = *reinterpret_cast<const uint32_t*>(&b);
+                            }
+                            st_shared16(p_s + (4 * c + g) * 2048 + i * 16, make_uint4(w[0], w[1], w[2], w[3]));
+                        }
+                }
+                // every row's S is read before the next Q K^T overwrites it
+                tc_fence_before();
+                fence_proxy_async_smem();
+                __syncthreads();
+                if (pass == 1 && i == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kTile / 16; k++)
+                        mma_f16(t_o, smem_desc(p_s + k * 4096, 2048, 128, kLayoutNone),
+                                smem_desc(v_s + k * 256, 128, 2048, kLayoutNone), ID_PV, (!first_pv || k > 0) ? 1u : 0u);
+                    tc_commit(&bar_o);
+                }
+                if (pass == 1) first_pv = false;
+            }
+        }
+    }
+    // O row i / l -> bf16
+    if (ok && !first_pv) {
+        const bool got = mbar_wait_bounded(&bar_o, ph_o, &s_abort, a.limit_ns);
+        ok = __syncthreads_and(got) != 0;
+        tc_fence_after();
+    }
+    if (!ok) {
+        if (i == 0) record_error(a.err, NVFP4_ERR_TIMEOUT, 3);
+    } else {
+        const int qrow = qt * kTile + i;
+        const float inv_l = l_run > 0.0f ? __frcp_rn(l_run) : 0.0f;
+        uint32_t r[4][32];
+        if (!first_pv) {
+#pragma unroll
+            for (int c = 0; c < 4; c++) tmem_ld_32cols(t_o + lane_off + 32 * c, r[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+#pragma unroll
+                for (int j = 0; j < 32; j++) r[c][j] = 0u;
+        }
+        if (qrow < a.tq) {
+            uint4* dst = reinterpret_cast<uint4*>(a.o + ((int64_t)qrow * a.heads + h) * kD * 2);
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+#pragma unroll
+                for (int g = 0; g < 4; g++) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const __nv_bfloat162 b =
+                            __floats2bfloat162_rn(__uint_as_float(r[c][8 * g + 2 * e]) * inv_l,
+                                                  __uint_as_float(r[c][8 * g + 2 * e + 1]) * inv_l);
+                        w[e] = *reinterpret_cast<const uint32_t*>(&b);
+                    }
+                    dst[4 * c + g] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace attn
+}  // namespace nvfp4
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+using namespace nvfp4;
+using namespace nvfp4::attn;
+
+extern "C" int32_t nvfp4_attention_chunks(int32_t t, int32_t sink_global, int32_t shot_start, int32_t sink_shot,
+                                          int32_t window, int32_t* out, int32_t max_out) {
+    if (t < 0 || sink_global < 0 || sink_shot < 0 || window < 0 || shot_start < 0 || max_out < 0 ||
+        (max_out > 0 && !out))
+        return -1;
+    // ascending walk over [0, t): a chunk is in the set when it lies in any of
+    // the three ranges (so each appears once)
+    int32_t n = 0;
+    const int64_t w0 = (int64_t)t - window;
+    for (int64_t c = 0; c < t; c++) {
+        const bool in = c < sink_global || (c >= shot_start && c < (int64_t)shot_start + sink_shot) || c >= w0;
+        if (!in) {
+            // skip the gap up to the next range start in one step
+            int64_t next = t;
+            if (c < shot_start) next = std::min<int64_t>(next, shot_start);
+            if (c < w0) next = std::min<int64_t>(next, w0);
+            c = next - 1;
+            continue;
+        }
+        if (n >= max_out) return -1;
+        out[n++] = (int32_t)c;
+    }
+    return n;
+}
+
+extern "C" nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n,
+                                           const void* q_bf16, int32_t tq, float scale, void* o_bf16, void* workspace,
+                                           size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!cache || n < 0 || tq < 0 || !workspace || !(scale >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
+    if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_KV_ATTENTION, 0, 0, 0)) return NVFP4_ERR_INVALID_ARG;
+    if (!cache->k_codes || !cache->k_scales || !cache->v_codes || !cache->v_scales || !cache->k_global ||
+        !cache->v_global || cache->n_slots <= 0 || cache->tokens_per_slot <= 0 || cache->heads <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (cache->head_dim != kD) return NVFP4_ERR_UNSUPPORTED;
+    if (cache->flags & ~(NVFP4_KV_SCALE_SEARCH | NVFP4_KV_SMOOTH_K | NVFP4_KV_SMOOTH_V)) return NVFP4_ERR_INVALID_ARG;
+    const bool sk = (cache->flags & NVFP4_KV_SMOOTH_K) != 0, sv = (cache->flags & NVFP4_KV_SMOOTH_V) != 0;
+    if ((sk && !cache->k_mean) || (sv && !cache->v_mean)) return NVFP4_ERR_INVALID_ARG;
+    if (tq == 0) return NVFP4_OK;
+    if (!q_bf16 || !o_bf16 || (n > 0 && !slots_dev)) return NVFP4_ERR_INVALID_ARG;
+    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!a16(q_bf16) || !a16(o_bf16) || !a16(cache->k_codes) || !a16(cache->v_codes) || !a16(cache->k_scales) ||
+        !a16(cache->v_scales) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        (reinterpret_cast<uintptr_t>(slots_dev) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    AttnArgs a{};
+    a.q = static_cast<const uint8_t*>(q_bf16);
+    a.o = static_cast<uint8_t*>(o_bf16);
+    a.codes[0] = static_cast<const uint8_t*>(cache->k_codes);
+    a.codes[1] = static_cast<const uint8_t*>(cache->v_codes);
+    a.scales[0] = static_cast<const uint8_t*>(cache->k_scales);
+    a.scales[1] = static_cast<const uint8_t*>(cache->v_scales);
+    a.gscale[0] = cache->k_global;
+    a.gscale[1] = cache->v_global;
+    a.mean[0] = sk ? cache->k_mean : nullptr;
+    a.mean[1] = sv ? cache->v_mean : nullptr;
+    a.slots = slots_dev;
+    a.n = n;
+    a.n_slots = cache->n_slots;
+    a.tq = tq;
+    a.tokens = cache->tokens_per_slot;
+    a.heads = cache->heads;
+    a.slot_elems = (int64_t)cache->tokens_per_slot * cache->heads * cache->head_dim;
+    const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)kD);
+    a.scale_log2 = sc * 1.4426950408889634f;  // log2(e)
+    a.err = static_cast<DevError*>(workspace);
+    a.limit_ns = 2000000000ull;
+    const int smem = 4 * kOperandBytes;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(kv_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        attr = true;
+    }
+    const dim3 grid((unsigned)((tq + kTile - 1) / kTile), (unsigned)cache->heads);
+    kv_attention_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}

@@ -17,7 +17,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
-OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT, OP_LN_QUANTIZE, OP_QUANTIZE_2D, OP_QUANTIZE_T = range(7)
+(OP_QUANTIZE, OP_GEMM, OP_KV_APPEND, OP_KV_DEQUANT, OP_LN_QUANTIZE, OP_QUANTIZE_2D, OP_QUANTIZE_T,
+ OP_KV_ATTENTION) = range(8)
 Q_COMPUTE_GLOBAL, Q_GIVEN_GLOBAL, Q_ROWMAJOR_SCALES, Q_SCALE_SEARCH = 0, 1, 2, 4
 KV_SCALE_SEARCH, KV_SMOOTH_K, KV_SMOOTH_V = 1, 2, 4
 ACT_NONE, ACT_GELU_TANH = 0, 1
@@ -26,7 +27,8 @@ DBG_SKIP_LOADS = 1
 EXPORTS = ("nvfp4_status_string", "nvfp4_version", "nvfp4_codes_bytes", "nvfp4_scales_bytes",
            "nvfp4_workspace_bytes", "nvfp4_read_device_error", "nvfp4_quantize", "nvfp4_gemm",
            "nvfp4_kv_append", "nvfp4_kv_dequant", "nvfp4_test_encode", "nvfp4_quantize_noalloc",
-           "nvfp4_ln_modulate_quantize", "nvfp4_quantize_2d", "nvfp4_quantize_t")
+           "nvfp4_ln_modulate_quantize", "nvfp4_quantize_2d", "nvfp4_quantize_t", "nvfp4_attention_chunks",
+           "nvfp4_kv_attention")
 
 
 class NVFP4Error(RuntimeError):
@@ -99,6 +101,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize_2d.restype = st
         L.nvfp4_quantize_t.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, ctypes.c_uint, vp, sz, vp]
         L.nvfp4_quantize_t.restype = st
+        L.nvfp4_attention_chunks.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int32), i32]
+        L.nvfp4_attention_chunks.restype = i32
+        L.nvfp4_kv_attention.argtypes = [ctypes.POINTER(CKVCache), vp, i32, vp, i32, ctypes.c_float, vp, vp, sz, vp]
+        L.nvfp4_kv_attention.restype = st
         _lib = L
     return _lib
 
@@ -380,6 +386,35 @@ class KVCache:
             ctypes.byref(cc), slots.data_ptr(), n, k_out.data_ptr(), v_out.data_ptr(),
             self.ws_dequant.data_ptr(), self.ws_dequant.numel(), _stream(stream)))
         return k_out, v_out
+
+    def attention(self, slots: torch.Tensor, q: torch.Tensor, *, scale: float = 0.0, out: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """softmax(scale Q K^T) V over every key of the listed slots (device int32), K and V read from
+        the NVFP4 cache; q and the result are bf16 [Tq, H, d]; scale 0 means 1 / sqrt(d)."""
+        _require_cuda(slots, q)
+        if q.dtype != torch.bfloat16 or not q.is_contiguous() or q.dim() != 3 or q.shape[1:] != (self.heads,
+                                                                                               self.head_dim):
+            raise ValueError("attention takes contiguous bf16 q [Tq, heads, head_dim]")
+        if out is None:
+            out = torch.empty_like(q)
+        if ws is None:
+            ws = workspace(OP_KV_ATTENTION, device=q.device)
+        cc = self.c()
+        _check("nvfp4_kv_attention", lib().nvfp4_kv_attention(
+            ctypes.byref(cc), slots.data_ptr(), slots.numel(), q.data_ptr(), q.shape[0], float(scale),
+            out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)))
+        return out
+
+
+def attention_chunks(t: int, sink_global: int, shot_start: int, sink_shot: int, window: int) -> list[int]:
+    """Chunk indices step t attends to: the global sink, the shot sink and the window, without
+    repeats, ascending (computed by the library's host function)."""
+    cap = max(1, t)
+    buf = (ctypes.c_int32 * cap)()
+    n = lib().nvfp4_attention_chunks(t, sink_global, shot_start, sink_shot, window, buf, cap)
+    if n < 0:
+        raise ValueError("nvfp4_attention_chunks: bad arguments")
+    return list(buf[:n])
 
 
 def test_encode(x: torch.Tensor, e2m1: bool = True, e4m3: bool = True, stream=None):

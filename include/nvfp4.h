@@ -92,7 +92,8 @@ enum {
     NVFP4_OP_KV_DEQUANT = 3, /* nvfp4_kv_dequant */
     NVFP4_OP_LN_QUANTIZE = 4, /* nvfp4_ln_modulate_quantize (m = rows) */
     NVFP4_OP_QUANTIZE_2D = 5, /* nvfp4_quantize_2d */
-    NVFP4_OP_QUANTIZE_T = 6   /* nvfp4_quantize_t */
+    NVFP4_OP_QUANTIZE_T = 6,  /* nvfp4_quantize_t */
+    NVFP4_OP_KV_ATTENTION = 7 /* nvfp4_kv_attention */
 };
 
 /* Workspace bytes the caller must pass to the call `op` (device memory,
@@ -292,6 +293,30 @@ nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const vo
 nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n, void* k_out_bf16,
                               void* v_out_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 
+
+/* Attention over the cache [RN-I, RN multi-shot anchors].  The chunk set of
+ * step t: A_g (the first sink_global chunks) | A_s (the current shot's first
+ * sink_shot chunks; the shot starts at chunk shot_start) | KV[t - window, t),
+ * without repeats, only chunks < t, ascending, written to the host array out
+ * (at most max_out).  Returns the count, or -1 on a negative argument or a
+ * full array.  Host only; mapping chunks to slots is the caller's page table. */
+int32_t nvfp4_attention_chunks(int32_t t, int32_t sink_global, int32_t shot_start, int32_t sink_shot,
+                               int32_t window, int32_t* out, int32_t max_out);
+
+/* O = softmax(scale * Q K^T) V over every key of the n slots listed in
+ * slots_dev (device int32, values in [0, n_slots)), reading K and V from the
+ * cache: each key and value is the cache's bf16 dequant (with the smoothing
+ * mean added for a smoothed tensor), no mask inside the set.  q_bf16 and
+ * o_bf16 are bf16 [tq][heads][head_dim] (token-major like the cache's chunks);
+ * scale = 0 means 1 / sqrt(head_dim).  head_dim must be 128.  Products on the
+ * tensor cores in bf16 with binary32 accumulation, softmax in binary32 (two
+ * passes over the keys), P rounded to bf16; one launch of
+ * ceil(tq / 128) x heads CTAs.  An out-of-range slot records NVFP4_ERR_DEVICE
+ * (info = list position) and is skipped.  workspace:
+ * nvfp4_workspace_bytes(NVFP4_OP_KV_ATTENTION, 0, 0, 0) bytes. */
+nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n, const void* q_bf16,
+                                int32_t tq, float scale, void* o_bf16, void* workspace, size_t ws_bytes,
+                                nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Training-side operands  [RN-T] "NVFP4 训练的工程细节"                        */

@@ -1,0 +1,104 @@
+"""GPU parity of nvfp4_kv_attention (softmax attention of bf16 queries over NVFP4
+cache slots read directly by the kernel) against the oracle's fp64 attention over
+the oracle's bf16 dequant of the same slots (reading R23: max |O - O_ref| /
+max |O_ref| <= 1e-2)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_video_dit_b200 import nvfp4 as nv
+from bit_video_dit_b200 import synthetic as syn
+
+from .gpu_util import dev_bf16, host_bits, normwise_err, require_gpu
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-2
+
+
+def _bits_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _case(T, H, Tq, slot_chunks, n_slots, seed, smooth_k=False, smooth_v=False, scale=0.0, rows=None):
+    """Fill a cache with seeded chunks, attend with seeded queries over the listed slots;
+    compare against the oracle (on sampled query rows when `rows` is given)."""
+    d = 128
+    cache = nv.KVCache(n_slots, T, H, d, smooth_k=smooth_k, smooth_v=smooth_v)
+    kh, vh = {}, {}
+    for s in range(n_slots):
+        k, v = syn.kv_chunk_bf16(T, H, d, seed=seed + s)
+        cache.append(s, dev_bf16(k), dev_bf16(v))
+        for name, x, sm, store in (("k", k, smooth_k, kh), ("v", v, smooth_v, vh)):
+            if sm:
+                c, sc, a, m = oracle.kv_append_smooth(x)
+                store[s] = oracle.kv_dequant_smooth(c, sc, a, m, T, H, d)
+            else:
+                c, sc, a = oracle.kv_append(x)
+                store[s] = oracle.kv_dequant(c, sc, a, T, H, d)
+    q = syn.kv_chunk_bf16(Tq, H, d, seed=seed + 1000)[0]
+    slots = torch.tensor(slot_chunks, dtype=torch.int32, device="cuda")
+    o = cache.attention(slots, dev_bf16(q), scale=scale)
+    torch.cuda.synchronize()
+    got = _bits_to_f64(host_bits(o))
+    if not slot_chunks:
+        return got, None, cache
+    kk = np.concatenate([kh[s] for s in slot_chunks], axis=0)
+    vv = np.concatenate([vh[s] for s in slot_chunks], axis=0)
+    sc = scale if scale > 0 else 1.0 / np.sqrt(d)
+    qs = q if rows is None else q[rows]
+    ref = oracle.attention(qs, kk, vv, sc)
+    gs = got if rows is None else got[rows]
+    err = normwise_err(gs.reshape(-1), ref.reshape(-1))
+    assert err <= TOL, err
+    return got, ref, cache
+
+
+@pytest.mark.parametrize("T,Tq", [(256, 200), (200, 128), (130, 7)])
+def test_small_sets_with_ragged_tiles(T, Tq):
+    require_gpu()
+    _case(T, 2, Tq, [0, 2], 3, seed=40 + T)
+
+
+def test_sink_and_window_set_from_the_chunk_builder():
+    """Step t = 9 of a ring of 6 slots: global sink 1, shot sink 1 (shot from chunk 4), window 3;
+    chunk c lives in slot c mod 6 except the pinned sink in slot 0."""
+    require_gpu()
+    chunks = nv.attention_chunks(9, 1, 4, 1, 3)
+    assert chunks == [0, 4, 6, 7, 8]
+    slots = [0 if c == 0 else 1 + (c - 1) % 5 for c in chunks]
+    _case(160, 3, 150, slots, 6, seed=60)
+
+
+@pytest.mark.parametrize("smooth_k,smooth_v", [(True, False), (True, True)])
+def test_smoothed_cache(smooth_k, smooth_v):
+    require_gpu()
+    _case(192, 2, 140, [1, 0], 2, seed=80, smooth_k=smooth_k, smooth_v=smooth_v)
+
+
+def test_given_scale_and_repeated_slot():
+    require_gpu()
+    _case(128, 2, 64, [1, 1, 0], 2, seed=90, scale=0.05)
+
+
+def test_full_chunk_workload_on_sampled_queries():
+    """The KV workload's chunk (2640 tokens x 24 heads x 128) attending over three slots
+    (a sink and a two-chunk window) with a full 2640-token query chunk; 48 sampled rows."""
+    require_gpu()
+    rows = np.sort(np.random.default_rng(7).choice(2640, 48, replace=False))
+    _case(syn.KV_TOKENS, syn.KV_HEADS, syn.KV_TOKENS, [0, 2, 3], 4, seed=100, rows=rows)
+
+
+def test_empty_list_gives_zeros_and_bad_slot_is_reported():
+    require_gpu()
+    got, _, _ = _case(128, 2, 32, [], 2, seed=110)
+    assert not np.any(got)
+    T, H, d = 128, 2, 128
+    cache = nv.KVCache(2, T, H, d)
+    k, v = syn.kv_chunk_bf16(T, H, d, seed=111)
+    cache.append(0, dev_bf16(k), dev_bf16(v))
+    q = dev_bf16(syn.kv_chunk_bf16(16, H, d, seed=112)[0])
+    ws = nv.workspace(nv.OP_KV_ATTENTION, device="cuda")
+    cache.attention(torch.tensor([0, 5], dtype=torch.int32, device="cuda"), q, ws=ws)
+    code, info = nv.read_device_error(ws)
+    assert code == nv.ERR_DEVICE and info == 1
