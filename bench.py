@@ -269,6 +269,40 @@ def measure_training(nv, a, w, cache, ring, k_out, v_out, reps: int) -> dict:
     return out
 
 
+def measure_attention(nv, cache, ring, k_out, v_out, reps: int) -> dict:
+    """ms per launch of the attention of one 2640-token query chunk over the NVFP4 cache:
+    all 21 slots (the set the dequant gathers) and a sink + window set of 5 slots."""
+    g = torch.Generator(device=k_out.device).manual_seed(91)
+    q = torch.randn((cache.tokens, cache.heads, cache.head_dim), generator=g, device=k_out.device)
+    q = q.to(torch.bfloat16)
+    o = torch.empty_like(q)
+    ws = nv.workspace(nv.OP_KV_ATTENTION, device=k_out.device)
+    chunks = nv.attention_chunks(30, 1, 24, 1, 3)  # global sink, shot sink, window of 3
+    small = torch.tensor([c % cache.n_slots for c in chunks], dtype=torch.int32, device=k_out.device)
+    sets = {"all": ring, "sink_window": small}
+    out = {}
+    for name, sl in sets.items():
+        cache.attention(sl, q, out=o, ws=ws)
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(reps)]
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for i in range(reps):
+                cache.dequant(ring, k_out, v_out)
+                ev[i][0].record()
+                cache.attention(sl, q, out=o, ws=ws)
+                ev[i][1].record()
+        gr.replay()
+        torch.cuda.synchronize()
+        ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
+        keys = sl.numel() * cache.tokens
+        flops = 4.0 * cache.tokens * keys * cache.head_dim * cache.heads
+        out[name] = {"slots": int(sl.numel()), "keys": keys, "ms": round(ms, 4),
+                     "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1)}
+        del gr
+    return out
+
+
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
@@ -383,6 +417,8 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     # the training-side operands (2D weight scaling, RHT transposed operands) and the
     # weight-gradient GEMM on the same layer shapes, also beside the step
     train = measure_training(nv, a, dev_bf16(w_host), cache, ring, k_out, v_out, reps=5)
+    # attention reading the NVFP4 cache directly (one query chunk), beside the step
+    attn = measure_attention(nv, cache, ring, k_out, v_out, reps=3)
 
     total_ms = t_start.elapsed_time(t_end)
     comp = np.zeros(4)
@@ -499,6 +535,11 @@ def run_ours(args, rank: int, world: int) -> dict | None:
             "quantize_t_dy_GB/s": round(M * N * 2.5625 / (train["quantize_t_dy_ms"] * 1e-3) / 1e9, 1),
             "wgrad_ms": round(train["wgrad_ms"], 4),
             "wgrad_TFLOP/s": round(2.0 * N * K * M / (train["wgrad_ms"] * 1e-3) / 1e12, 1)},
+        "kv_attention": {
+            "what": "softmax attention of one 2640x24x128 bf16 query chunk over NVFP4 cache slots read directly "
+                    "(dequant into the tensor-core tiles, tcgen05 bf16 MMAs, two-pass softmax), outside the step; "
+                    "TFLOP/s counts 4*Tq*keys*d*H",
+            "bf16_peak_TFLOP/s": pk.get("bf16_tflops"), **attn},
         "ln_modulate_quantize": {
             "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A, two launches, outside the step",
             "ms": round(search["ln_quantize_ms"], 4),

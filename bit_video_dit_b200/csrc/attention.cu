@@ -7,7 +7,8 @@
 // (E2M1 codes, E4M3 block scales, the slot's a32, the K-smoothing mean when
 // the cache has one) straight into shared memory in the layouts the tensor
 // cores read, with each thread writing its token's row as 16-byte chunks:
-//   Q, K, P: K-major, no swizzle: element (row r, column c) at
+//   Q, K, P: K-major, no swizzle (P is written over K, which the Q K^T
+//            product has finished with): element (row r, column c) at
 //            (c / 8) * 2048 + r * 16 + (c % 8) * 2 (8-row core matrices 128
 //            bytes apart, 8-column chunks 2048 bytes apart);
 //   V:       MN-major (the d columns are the MMA's N): element (token t, dim j)
@@ -98,38 +99,55 @@ __device__ __forceinline__ uint4 dq8(uint32_t q, uint32_t sc, float a32, const f
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Thread i's token row (token `tok` of slot s, head h) of K or V into the
-// operand at `base` (K-major and MN-major layouts put a row at the same
-// places); zeros when the token is past the slot's end.
-__device__ __forceinline__ void load_kv_row(const AttnArgs& a, int t, int s, int tok, int h, uint32_t base, int row) {
-    uint4 v[16];
-    if (tok < a.tokens) {
+// One token row (token `tok` of slot s, head h) of K or V as stored: 64 code
+// bytes, 8 scale bytes and the slot's a32; zeros when the token is past the
+// slot's end.  Fetched a tile ahead so the loads overlap the tile in flight.
+struct RowRaw {
+    uint4 c[4];
+    uint2 sc;
+    float a32;
+    bool valid;
+};
+
+__device__ __forceinline__ RowRaw fetch_row(const AttnArgs& a, int t, int s, int tok, int h) {
+    RowRaw r;
+    r.valid = tok < a.tokens;
+    if (r.valid) {
         const int64_t e = (int64_t)s * a.slot_elems + ((int64_t)tok * a.heads + h) * kD;
         const uint4* cp = reinterpret_cast<const uint4*>(a.codes[t] + e / 2);
-        const uint2 sp = __ldg(reinterpret_cast<const uint2*>(a.scales[t] + e / 16));
-        const float a32 = __ldg(a.gscale[t] + s);
-        const float* m = a.mean[t] ? a.mean[t] + ((int64_t)s * a.heads + h) * kD : nullptr;
-        const uint32_t sw[2] = {sp.x, sp.y};
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-            const uint4 c = __ldg(cp + k);
-            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int chunk = 4 * k + j;  // elements 8 * chunk .. + 7; block chunk / 2
-                const uint32_t sc = (sw[chunk / 8] >> (8 * ((chunk / 2) % 4))) & 0xFFu;
-                v[chunk] = dq8(cw[j], sc, a32, m ? m + 8 * chunk : nullptr);
-            }
-        }
+        for (int k = 0; k < 4; k++) r.c[k] = __ldg(cp + k);
+        r.sc = __ldg(reinterpret_cast<const uint2*>(a.scales[t] + e / 16));
+        r.a32 = __ldg(a.gscale[t] + s);
     } else {
 #pragma unroll
-        for (int c = 0; c < 16; c++) v[c] = make_uint4(0u, 0u, 0u, 0u);
+        for (int k = 0; k < 4; k++) r.c[k] = make_uint4(0u, 0u, 0u, 0u);
+        r.sc = make_uint2(0u, 0u);
+        r.a32 = 0.0f;
     }
-#pragma unroll
-    for (int c = 0; c < 16; c++) st_shared16(base + c * 2048 + row * 16, v[c]);
+    return r;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_constant__ AttnArgs a) {
+// The row's 128 dequantized bf16 values into the operand at `base` (K-major
+// and MN-major layouts put a row at the same places); a row past the slot's
+// end (codes 0, a32 0, no mean) decodes to zeros.
+__device__ __forceinline__ void store_row(const AttnArgs& a, int t, int s, int h, const RowRaw& r, uint32_t base,
+                                         int row) {
+    const float* m = (a.mean[t] && r.valid) ? a.mean[t] + ((int64_t)s * a.heads + h) * kD : nullptr;
+    const uint32_t sw[2] = {r.sc.x, r.sc.y};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const uint32_t cw[4] = {r.c[k].x, r.c[k].y, r.c[k].z, r.c[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int chunk = 4 * k + j;  // elements 8 * chunk .. + 7; block chunk / 2
+            const uint32_t sc = (sw[chunk / 8] >> (8 * ((chunk / 2) % 4))) & 0xFFu;
+            st_shared16(base + chunk * 2048 + row * 16, dq8(cw[j], sc, r.a32, m ? m + 8 * chunk : nullptr));
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_constant__ AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint64_t bar_s, bar_o;
     __shared__ uint32_t tmem_base;
@@ -137,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
     const int i = threadIdx.x;  // query row, TMEM lane
     const int warp = i >> 5;
     const int qt = blockIdx.x, h = blockIdx.y;
-    const uint32_t q_s = smem_u32(smem), k_s = q_s + kOperandBytes, v_s = k_s + kOperandBytes,
-                   p_s = v_s + kOperandBytes;
+    // P is written over K: the Q K^T product is done with K before P is formed
+    const uint32_t q_s = smem_u32(smem), k_s = q_s + kOperandBytes, v_s = k_s + kOperandBytes, p_s = k_s;
     if (i == 0) {
         mbar_init(&bar_s, 1);
         mbar_init(&bar_o, 1);
@@ -177,103 +195,129 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
     float m_run = -INFINITY, l_run = 0.0f;
     bool first_pv = true;
 
-    for (int pass = 0; pass < 2 && ok; pass++) {
-        for (int si = 0; si < a.n && ok; si++) {
+    if (i == 0 && qt == 0 && h == 0)
+        for (int si = 0; si < a.n; si++) {
             const int s = __ldg(a.slots + si);
-            if (s < 0 || s >= a.n_slots) {
-                if (pass == 0 && i == 0 && qt == 0 && h == 0) record_error(a.err, NVFP4_ERR_DEVICE, (uint32_t)si);
-                continue;  // uniform over the CTA
-            }
-            for (int kt = 0; kt < tiles_per_slot && ok; kt++) {
-                const int tok = kt * kTile + i;
-                const int valid = min(kTile, a.tokens - kt * kTile);
-                // the previous P V product must be done with K, V and P
-                // (every wait's outcome is made uniform over the CTA before
-                // anyone acts on it, so all threads take the same barriers)
-                if (pass == 1 && !first_pv) {
-                    const bool got = mbar_wait_bounded(&bar_o, ph_o, &s_abort, a.limit_ns);
-                    ph_o ^= 1u;
-                    if (!__syncthreads_and(got)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                }
-                load_kv_row(a, 0, s, tok, h, k_s, i);
-                if (pass == 1) load_kv_row(a, 1, s, tok, h, v_s, i);
-                fence_proxy_async_smem();
-                __syncthreads();
-                if (i == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < kD / 16; k++)
-                        mma_f16(t_s, smem_desc(q_s + k * 4096, 2048, 128, kLayoutNone),
-                                smem_desc(k_s + k * 4096, 2048, 128, kLayoutNone), ID_QK, k > 0);
-                    tc_commit(&bar_s);
-                }
-                {
-                    const bool got = mbar_wait_bounded(&bar_s, ph_s, &s_abort, a.limit_ns);
-                    ph_s ^= 1u;
-                    if (!__syncthreads_and(got)) {
-                        ok = false;
-                        break;
-                    }
+            if (s < 0 || s >= a.n_slots) record_error(a.err, NVFP4_ERR_DEVICE, (uint32_t)si);
+        }
+    // the key tiles: tile g is tile g % tiles_per_slot of list entry g / tiles_per_slot;
+    // entries with an out-of-range slot are skipped (uniform over the CTA)
+    const int G = a.n * tiles_per_slot;
+    auto slot_of = [&](int g) { return __ldg(a.slots + g / tiles_per_slot); };
+    auto next_tile = [&](int g) {
+        while (g < G) {
+            const int s = slot_of(g);
+            if (s >= 0 && s < a.n_slots) break;
+            g += tiles_per_slot - g % tiles_per_slot;
+        }
+        return g;
+    };
+    for (int pass = 0; pass < 2 && ok; pass++) {
+        int g = next_tile(0);
+        RowRaw kr, vr;
+        if (g < G) {
+            kr = fetch_row(a, 0, slot_of(g), (g % tiles_per_slot) * kTile + i, h);
+            if (pass == 1) vr = fetch_row(a, 1, slot_of(g), (g % tiles_per_slot) * kTile + i, h);
+        }
+        while (g < G && ok) {
+            const int s = slot_of(g), kt = g % tiles_per_slot;
+            const int valid = min(kTile, a.tokens - kt * kTile);
+            const int gn = next_tile(g + 1);
+            // the previous P V product must be done with K, V and P
+            // (every wait's outcome is made uniform over the CTA before
+            // anyone acts on it, so all threads take the same barriers)
+            if (pass == 1 && !first_pv) {
+                const bool got = mbar_wait_bounded(&bar_o, ph_o, &s_abort, a.limit_ns);
+                ph_o ^= 1u;
+                if (!__syncthreads_and(got)) {
+                    ok = false;
+                    break;
                 }
                 tc_fence_after();
-                uint32_t r[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; c++) tmem_ld_32cols(t_s + lane_off + 32 * c, r[c]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
-                if (pass == 0) {
-                    float mt = -INFINITY;
-#pragma unroll
-                    for (int c = 0; c < 4; c++)
-#pragma unroll
-                        for (int j = 0; j < 32; j++)
-                            if (32 * c + j < valid) mt = fmaxf(mt, __uint_as_float(r[c][j]));
-                    const float m_new = fmaxf(m_run, mt);
-                    float sum = 0.0f;
-#pragma unroll
-                    for (int c = 0; c < 4; c++)
-#pragma unroll
-                        for (int j = 0; j < 32; j++)
-                            if (32 * c + j < valid) sum += ex2((__uint_as_float(r[c][j]) - m_new) * a.scale_log2);
-                    l_run = l_run * ex2((m_run - m_new) * a.scale_log2) + sum;
-                    m_run = m_new;
-                } else {
-                    // P row i: exp(scale * (s - max)) in bf16, zero for keys past the slot's end
-#pragma unroll
-                    for (int c = 0; c < 4; c++)
-#pragma unroll
-                        for (int g = 0; g < 4; g++) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; e++) {
-                                const int j0 = 32 * c + 8 * g + 2 * e;
-                                const float p0 = j0 < valid ? ex2((__uint_as_float(r[c][8 * g + 2 * e]) - m_run) * a.scale_log2) : 0.0f;
-                                const float p1 = j0 + 1 < valid ? ex2((__uint_as_float(r[c][8 * g + 2 * e + 1]) - m_run) * a.scale_log2) : 0.0f;
-                                const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
-                                w[e] = *reinterpret_cast<const uint32_t*>(&b);
-                            }
-                            st_shared16(p_s + (4 * c + g) * 2048 + i * 16, make_uint4(w[0], w[1], w[2], w[3]));
-                        }
-                }
-                // every row's S is read before the next Q K^T overwrites it
-                tc_fence_before();
-                fence_proxy_async_smem();
-                __syncthreads();
-                if (pass == 1 && i == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < kTile / 16; k++)
-                        mma_f16(t_o, smem_desc(p_s + k * 4096, 2048, 128, kLayoutNone),
-                                smem_desc(v_s + k * 256, 128, 2048, kLayoutNone), ID_PV, (!first_pv || k > 0) ? 1u : 0u);
-                    tc_commit(&bar_o);
-                }
-                if (pass == 1) first_pv = false;
             }
+            store_row(a, 0, s, h, kr, k_s, i);
+            if (pass == 1) store_row(a, 1, s, h, vr, v_s, i);
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (i == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < kD / 16; k++)
+                    mma_f16(t_s, smem_desc(q_s + k * 4096, 2048, 128, kLayoutNone),
+                            smem_desc(k_s + k * 4096, 2048, 128, kLayoutNone), ID_QK, k > 0);
+                tc_commit(&bar_s);
+            }
+            // the next tile's rows load while the product and the softmax run
+            if (gn < G) {
+                kr = fetch_row(a, 0, slot_of(gn), (gn % tiles_per_slot) * kTile + i, h);
+                if (pass == 1) vr = fetch_row(a, 1, slot_of(gn), (gn % tiles_per_slot) * kTile + i, h);
+            }
+            {
+                const bool got = mbar_wait_bounded(&bar_s, ph_s, &s_abort, a.limit_ns);
+                ph_s ^= 1u;
+                if (!__syncthreads_and(got)) {
+                    ok = false;
+                    break;
+                }
+            }
+            tc_fence_after();
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; c++) tmem_ld_32cols(t_s + lane_off + 32 * c, r[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
+            if (pass == 0) {
+                float mt = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; c++)
+#pragma unroll
+                    for (int j = 0; j < 32; j++)
+                        if (32 * c + j < valid) mt = fmaxf(mt, __uint_as_float(r[c][j]));
+                const float m_new = fmaxf(m_run, mt);
+                float sum = 0.0f;
+#pragma unroll
+                for (int c = 0; c < 4; c++)
+#pragma unroll
+                    for (int j = 0; j < 32; j++)
+                        if (32 * c + j < valid) sum += ex2((__uint_as_float(r[c][j]) - m_new) * a.scale_log2);
+                l_run = l_run * ex2((m_run - m_new) * a.scale_log2) + sum;
+                m_run = m_new;
+            } else {
+                // P row i: exp(scale * (s - max)) in bf16, zero for keys past the slot's end
+#pragma unroll
+                for (int c = 0; c < 4; c++)
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; q4++) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const int j0 = 32 * c + 8 * q4 + 2 * e;
+                            const float p0 =
+                                j0 < valid ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e]) - m_run) * a.scale_log2) : 0.0f;
+                            const float p1 = j0 + 1 < valid
+                                                 ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e + 1]) - m_run) * a.scale_log2)
+                                                 : 0.0f;
+                            const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
+                            w[e] = *reinterpret_cast<const uint32_t*>(&b);
+                        }
+                        st_shared16(p_s + (4 * c + q4) * 2048 + i * 16, make_uint4(w[0], w[1], w[2], w[3]));
+                    }
+            }
+            // every row's S is read before the next Q K^T overwrites it
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (pass == 1 && i == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < kTile / 16; k++)
+                    mma_f16(t_o, smem_desc(p_s + k * 4096, 2048, 128, kLayoutNone),
+                            smem_desc(v_s + k * 256, 128, 2048, kLayoutNone), ID_PV, (!first_pv || k > 0) ? 1u : 0u);
+                tc_commit(&bar_o);
+            }
+            if (pass == 1) first_pv = false;
+            g = gn;
         }
     }
     // O row i / l -> bf16
@@ -401,7 +445,7 @@ extern "C" nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const in
     a.scale_log2 = sc * 1.4426950408889634f;  // log2(e)
     a.err = static_cast<DevError*>(workspace);
     a.limit_ns = 2000000000ull;
-    const int smem = 4 * kOperandBytes;
+    const int smem = 3 * kOperandBytes;
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(kv_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)

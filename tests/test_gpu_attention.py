@@ -102,3 +102,23 @@ def test_empty_list_gives_zeros_and_bad_slot_is_reported():
     cache.attention(torch.tensor([0, 5], dtype=torch.int32, device="cuda"), q, ws=ws)
     code, info = nv.read_device_error(ws)
     assert code == nv.ERR_DEVICE and info == 1
+
+
+def test_smoothed_channel_constant_slot_with_zero_tensor_scale():
+    """A smoothed K chunk that is constant per channel has tensor scale 0 and all codes 0;
+    its keys are the means, which the attention must still add."""
+    require_gpu()
+    T, H, d = 96, 2, 128
+    cache = nv.KVCache(1, T, H, d, smooth_k=True)
+    rng = np.random.default_rng(3)
+    b = (rng.integers(-16, 17, size=(H, d)) / 8.0).astype(np.float32)
+    kb = (np.broadcast_to(b, (T, H, d)).copy().view(np.uint32) >> 16).astype(np.uint16)
+    _, v = syn.kv_chunk_bf16(T, H, d, seed=5)
+    cache.append(0, dev_bf16(kb), dev_bf16(v))
+    assert float(cache.k_global[0]) == 0.0
+    q = syn.kv_chunk_bf16(40, H, d, seed=6)[0]
+    o = cache.attention(torch.tensor([0], dtype=torch.int32, device="cuda"), dev_bf16(q))
+    torch.cuda.synchronize()
+    c, sc, a = oracle.kv_append(v)
+    ref = oracle.attention(q, kb, oracle.kv_dequant(c, sc, a, T, H, d), 1.0 / np.sqrt(d))
+    assert normwise_err(_bits_to_f64(host_bits(o)).reshape(-1), ref.reshape(-1)) <= TOL
