@@ -16,9 +16,9 @@
 // S = Q K^T and O += P V run as tcgen05.mma kind::f16 (bf16 operands, binary32
 // accumulators in TMEM: S in columns [0, 128), O in [128, 256)), issued by
 // thread 0 and waited on through an mbarrier.  The softmax takes two passes
-// over the keys: the first finds each row's max and sum of exponentials, the
-// second forms P = exp(scale * (s - max)) in bf16 and accumulates P V, so the
-// output never needs rescaling; O / sum is stored as bf16.  Every wait is
+// over the keys: the first finds each row's max, the second forms
+// P = exp(scale * (s - max)), sums it (binary32) and accumulates P V with P in
+// bf16, so the output never needs rescaling; O / sum is stored as bf16.  Every wait is
 // bounded; a timeout records NVFP4_ERR_TIMEOUT and the CTA stops.
 #include <algorithm>
 #include <cmath>
@@ -268,21 +268,11 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
 #pragma unroll
             for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
             if (pass == 0) {
-                float mt = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; c++)
 #pragma unroll
                     for (int j = 0; j < 32; j++)
-                        if (32 * c + j < valid) mt = fmaxf(mt, __uint_as_float(r[c][j]));
-                const float m_new = fmaxf(m_run, mt);
-                float sum = 0.0f;
-#pragma unroll
-                for (int c = 0; c < 4; c++)
-#pragma unroll
-                    for (int j = 0; j < 32; j++)
-                        if (32 * c + j < valid) sum += ex2((__uint_as_float(r[c][j]) - m_new) * a.scale_log2);
-                l_run = l_run * ex2((m_run - m_new) * a.scale_log2) + sum;
-                m_run = m_new;
+                        if (32 * c + j < valid) m_run = fmaxf(m_run, __uint_as_float(r[c][j]));
             } else {
                 // P row i: exp(scale * (s - max)) in bf16, zero for keys past the slot's end
 #pragma unroll
@@ -298,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
                             const float p1 = j0 + 1 < valid
                                                  ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e + 1]) - m_run) * a.scale_log2)
                                                  : 0.0f;
+                            l_run += p0 + p1;
                             const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
                             w[e] = *reinterpret_cast<const uint32_t*>(&b);
                         }
