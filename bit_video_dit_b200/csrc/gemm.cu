@@ -68,20 +68,30 @@ constexpr int EPI_STAGE_BYTES = 4 * 2 * EPI_BUF_BYTES;  // 16 KB
 constexpr int VEC_WORDS = BN / 2;                        // bf16 pairs per vector per tile
 constexpr int VEC_BYTES = 2 * 4 * VEC_WORDS * 4;        // 4 KB
 
-// Two accumulators of BN columns share TMEM with two 48-column scale buffers:
-// acc0 = [0, 256), acc1 = [160, 416), scales = [416, 512).  The accumulators
-// overlap in columns [160, 256); the epilogue drains those first (acc0: its
-// chunks 5..7, acc1: its chunks 0..2) and then lets the next tile's MMAs
-// start, so the rest of the epilogue overlaps the next mainloop.  The scale
-// buffers alternate by stage: the copy warps fill one while the MMAs read the
-// other.
+// Two accumulators of BN columns share TMEM with NSF 48-column scale buffers
+// that the stages take in turn (the copy warps fill one while the MMAs read
+// another).  The accumulators overlap; the epilogue drains the shared columns
+// first and then lets the next tile's MMAs start, so the rest of the
+// epilogue overlaps the next mainloop.  Short K (NC = 2): two scale buffers,
+// acc0 = [0, 256), acc1 = [160, 416), scales = [416, 512), 3 shared chunks
+// (acc0: its chunks 5..7, acc1: 0..2).  Long K (NC = 3): three scale buffers,
+// so the copy warps can run two stages ahead of the MMAs and the tensor pipe
+// never waits for a copy to be seen; acc1 = [96, 352), scales = [352, 496),
+// 5 shared chunks -- a longer hand-over between tiles, which long K
+// amortises.
 constexpr uint32_t SF_COLS = 4 * KB_PER_STAGE + 8 * KB_PER_STAGE;  // 48 per buffer
-constexpr uint32_t ACC1_COL = 160;
-constexpr uint32_t SFA_COL = ACC1_COL + BN;                        // 416 (+48: buffer 1)
-constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;           // 432 (+48: buffer 1)
-constexpr int OVERLAP_CHUNKS = (BN - (int)ACC1_COL) / 32;          // 3
-static_assert(SFA_COL + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
-static_assert(ACC1_COL % 32 == 0 && (BN - (int)ACC1_COL) % 32 == 0, "overlap must be whole 32-column chunks");
+constexpr int MAX_NSF = 3;
+template <int NC>
+struct Tm {
+    static constexpr int NSF = NC == 3 ? 3 : 2;
+    static constexpr uint32_t ACC1_COL = NC == 3 ? 96 : 160;
+    static constexpr uint32_t SFA_COL = ACC1_COL + BN;               // scale buffer 0
+    static constexpr uint32_t SFB_COL = SFA_COL + 4 * KB_PER_STAGE;
+    static constexpr int OVERLAP_CHUNKS = (BN - (int)ACC1_COL) / 32;
+    static_assert(SFA_COL + NSF * SF_COLS <= TMEM_COLS, "TMEM budget");
+    static_assert(NSF <= MAX_NSF, "scale-buffer barriers");
+    static_assert(ACC1_COL % 32 == 0 && (BN - (int)ACC1_COL) % 32 == 0, "overlap must be whole 32-column chunks");
+};
 
 // instruction descriptor: E2M1 x E2M1, UE4M3 scales, f32 accumulate, K-major
 // A and B, M x N, K = 64 (dense).
@@ -137,8 +147,8 @@ struct Smem {
     uint64_t tmem_full;
     uint64_t tmem_empty;
     uint64_t drain;
-    uint64_t sf_full[2];   // scale buffer filled (one commit per copy warp)
-    uint64_t sf_empty[2];  // scale buffer no longer read by the MMAs
+    uint64_t sf_full[MAX_NSF];   // scale buffer filled (one commit per copy warp)
+    uint64_t sf_empty[MAX_NSF];  // scale buffer no longer read by the MMAs
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -244,14 +254,15 @@ drain:
 // buffer.  Descriptors are built once; a stage / k-block step only adds to the
 // 14-bit start-address field (shared memory addresses are < 2^18, so the field
 // never carries).
-template <bool PAIR>
+template <bool PAIR, int NC>
 __device__ void mma_issuer(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, uint32_t tmem) {
     using C = Cfg<PAIR>;
+    using T = Tm<NC>;
     volatile int* abort = &s->abort_flag;
     const uint32_t ring_s = smem_u32(ring);
     const uint64_t a_desc0 = smem_desc(ring_s, 16, 1024, kLayoutSw128);
     const uint64_t b_desc0 = smem_desc(ring_s + A_BYTES, 16, 1024, kLayoutSw128);
-    const uint32_t sfa_t = tmem + SFA_COL, sfb_t = tmem + SFB_COL;
+    const uint32_t sfa_t = tmem + T::SFA_COL, sfb_t = tmem + T::SFB_COL;
     int first, step;
     tile_range<PAIR>(first, step);
     uint32_t it = 0;
@@ -263,19 +274,19 @@ __device__ void mma_issuer(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t*
             goto drain;
         }
         tc_fence_after();
-        const uint32_t acc = tmem + ((tcount & 1) ? ACC1_COL : 0u);
+        const uint32_t acc = tmem + ((tcount & 1) ? T::ACC1_COL : 0u);
         for (int kt = 0; kt < p.kt_count; kt++, it++) {
             const int st = it % C::STAGES;
-            const uint32_t sb = it & 1;
+            const uint32_t sb = it % T::NSF;
             // the stage's scales are in TMEM (the copy warps saw its data arrive)
-            if (!mbar_wait_bounded(&s->sf_full[sb], (it >> 1) & 1, abort, p.limit_ns)) {
+            if (!mbar_wait_bounded(&s->sf_full[sb], (it / T::NSF) & 1, abort, p.limit_ns)) {
                 if (!*abort) raise_abort(s, p, 3);
                 goto drain;
             }
             tc_fence_after();
             const uint64_t off = (uint64_t)((st * C::STAGE_BYTES) >> 4);
             const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
-            const uint32_t sfo = sb ? SF_COLS : 0u;
+            const uint32_t sfo = sb * SF_COLS;
 #pragma unroll
             for (int kb = 0; kb < KB_PER_STAGE; kb++) {
                 if (kb < nkb) {
@@ -324,6 +335,7 @@ drain:
 template <bool PAIR, int NC>
 __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_t* ring, uint32_t tmem, int part) {
     using C = Cfg<PAIR>;
+    using T = Tm<NC>;
     constexpr int PER = 3 * KB_PER_STAGE / NC;  // tiles per copy warp and stage: 6 (NC = 2) or 4 (NC = 3)
     volatile int* abort = &s->abort_flag;
     const uint32_t sf_s = smem_u32(ring) + A_BYTES + C::B_BYTES;  // SFA, then SFB rows 0..127, then 128..255
@@ -334,15 +346,15 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
     for (int tile = first; tile < p.num_tiles; tile += step) {
         for (int kt = 0; kt < p.kt_count; kt++, it++) {
             const int st = it % C::STAGES;
-            const uint32_t sb = it & 1;
+            const uint32_t sb = it % T::NSF;
             if (!mbar_wait_bounded(&s->full[st], (it / C::STAGES) & 1, abort, p.limit_ns) ||
-                !mbar_wait_bounded(&s->sf_empty[sb], ((it >> 1) & 1) ^ 1, abort, p.limit_ns)) {
+                !mbar_wait_bounded(&s->sf_empty[sb], ((it / T::NSF) & 1) ^ 1, abort, p.limit_ns)) {
                 if (!*abort) raise_abort(s, p, 5);
                 return;
             }
             tc_fence_after();
             const uint64_t d = desc0 + (uint64_t)((st * C::STAGE_BYTES) >> 4);
-            const uint32_t t = tmem + (sb ? SF_COLS : 0u);
+            const uint32_t t = tmem + sb * SF_COLS;
 #pragma unroll
             for (int c = 0; c < PER; c++) {
                 // tile g of the stage: which = g / 4 (SFA, SFB rows 0..127, SFB rows
@@ -350,7 +362,7 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
                 const int g = part * PER + c;
                 const int which = g / KB_PER_STAGE, kb = g % KB_PER_STAGE;
                 const uint32_t dst =
-                    t + (which == 0 ? SFA_COL + 4u * kb : SFB_COL + 8u * kb + 4u * (uint32_t)(which - 1));
+                    t + (which == 0 ? T::SFA_COL + 4u * kb : T::SFB_COL + 8u * kb + 4u * (uint32_t)(which - 1));
                 const uint64_t src = d + (uint64_t)((which * SFA_BYTES + kb * 512) >> 4);
                 if (PAIR)
                     tc_cp_32x128b_x4_pair(dst, src);
@@ -485,7 +497,7 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
     }
 }
 
-template <bool PAIR, bool EARLY>
+template <bool PAIR, int NC, bool EARLY>
 __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t tmem, int warp, int lane, uint32_t rank,
                          const CUtensorMap* tma_c, uint8_t* epi_stage, uint32_t* vecs) {
     using C = Cfg<PAIR>;
@@ -533,7 +545,8 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
         const int ncols = min(BN, p.N - nb * BN);
         const int nchunks = (ncols + 31) / 32;
         const bool buf1 = tcount & 1;
-        const uint32_t acc = lane_base + (buf1 ? ACC1_COL : 0u);
+        constexpr int OVERLAP_CHUNKS = Tm<NC>::OVERLAP_CHUNKS;
+        const uint32_t acc = lane_base + (buf1 ? Tm<NC>::ACC1_COL : 0u);
         // chunks of this buffer that the other buffer overlaps come first
         const int first_ov = buf1 ? 0 : (BN / 32 - OVERLAP_CHUNKS);
         const int n_overlap = buf1 ? min(nchunks, OVERLAP_CHUNKS) : max(0, nchunks - first_ov);
@@ -642,7 +655,7 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
         mbar_init(&s->tmem_full, 1);
         mbar_init(&s->tmem_empty, 4 * C::CTAS);
         mbar_init(&s->drain, 1);
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < Tm<NC>::NSF; i++) {
             mbar_init(&s->sf_full[i], NC);
             mbar_init(&s->sf_empty[i], 1);
         }
@@ -671,13 +684,13 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
         if (lane == 0) producer<PAIR>(p, s, ring, &tma_a, &tma_b, &tma_sfa, &tma_sfb, rank);
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) mma_issuer<PAIR>(p, s, ring, tmem);
+        if (lane == 0 && rank == 0) mma_issuer<PAIR, NC>(p, s, ring, tmem);
         __syncwarp();
     } else if (warp >= 6) {
         if (lane == 0 && rank == 0) scale_copier<PAIR, NC>(p, s, ring, tmem, warp - 6);
         __syncwarp();
     } else {
-        epilogue<PAIR, NC == 2>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs);
+        epilogue<PAIR, NC, NC == 2>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs);
     }
     tc_fence_before();
     if (PAIR)
