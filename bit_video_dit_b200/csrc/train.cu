@@ -59,17 +59,18 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
 // Sylvester Hadamard matrix.
 // The same transform on two blocks at once (columns c and c + 1 of a lane):
 // element i of both blocks in one 64-bit pair, the packed binary32 add, sub
-// and multiply rounding each lane as the scalar operation does.
+// and multiply rounding each lane as the scalar operation does.  The signs
+// are applied by the caller (on the packed bf16 words, exact), and SCALE =
+// false leaves out the final * 0.25, which the amax pass applies to its
+// maximum instead (exact: rounding is monotone, so it commutes with max).
 __device__ __forceinline__ uint64_t pk(float lo, float hi) {
     return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
 }
-__device__ __forceinline__ void rht16x2(float* f0, float* f1, uint32_t sign_mask) {
+template <bool SCALE>
+__device__ __forceinline__ void rht16x2(float* f0, float* f1) {
     uint64_t v[16];
 #pragma unroll
-    for (int i = 0; i < 16; i++) {
-        const uint64_t flip = (uint64_t)((sign_mask >> i) & 1u) * 0x8000000080000000ull;
-        v[i] = pk(f0[i], f1[i]) ^ flip;
-    }
+    for (int i = 0; i < 16; i++) v[i] = pk(f0[i], f1[i]);
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1)
 #pragma unroll
@@ -82,8 +83,8 @@ __device__ __forceinline__ void rht16x2(float* f0, float* f1, uint32_t sign_mask
     const uint64_t q = pk(0.25f, 0.25f);
 #pragma unroll
     for (int i = 0; i < 16; i++) {
-        uint64_t r;
-        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(v[i]), "l"(q));
+        uint64_t r = v[i];
+        if (SCALE) asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(v[i]), "l"(q));
         f0[i] = __uint_as_float((uint32_t)r);
         f1[i] = __uint_as_float((uint32_t)(r >> 32));
     }
@@ -139,10 +140,12 @@ __global__ void __launch_bounds__(kThreads, (RHT && ENCODE) ? 2 : 3) train_quant
             float f0[16], f1[16];
 #pragma unroll
             for (int i = 0; i < 16; i++) {
-                f0[i] = __uint_as_float(v[16 * b + i] << 16);
-                f1[i] = __uint_as_float(v[16 * b + i] & 0xFFFF0000u);
+                // RHT signs on the packed bf16 pair (both columns share row i's sign)
+                const uint32_t w = RHT ? v[16 * b + i] ^ (((a.sign_mask >> i) & 1u) * 0x80008000u) : v[16 * b + i];
+                f0[i] = __uint_as_float(w << 16);
+                f1[i] = __uint_as_float(w & 0xFFFF0000u);
             }
-            if (RHT) rht16x2(f0, f1, a.sign_mask);
+            if (RHT) rht16x2<ENCODE>(f0, f1);
             const float m0 = absmax16(f0), m1 = absmax16(f1);
             if (!ENCODE) {
                 lane_max = fmaxf(lane_max, fmaxf(m0, m1));
@@ -202,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, (RHT && ENCODE) ? 2 : 3) train_quant
         }
     }
     if (!ENCODE) {
+        if (RHT) lane_max = __fmul_rn(lane_max, 0.25f);  // the transform's normalisation, left out above
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) lane_max = fmaxf(lane_max, __shfl_xor_sync(0xFFFFFFFFu, lane_max, o));
         if (lane == 0 && lane_max > 0.0f) atomicMax(a.amax_word, __float_as_uint(lane_max));
