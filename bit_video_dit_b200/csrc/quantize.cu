@@ -497,6 +497,8 @@ __device__ __forceinline__ float warp_butterfly_sum(float s) {
     return s;
 }
 
+constexpr int kStatRegBlocks = 8;  // 16-element blocks a lane holds in registers (rows up to 4096 columns)
+
 __global__ void __launch_bounds__(256) ln_stats_kernel(const uint8_t* x, int64_t ld_bytes, int rows, int cols,
                                                        float eps, float2* out) {
     const int lane = threadIdx.x & 31;
@@ -505,24 +507,57 @@ __global__ void __launch_bounds__(256) ln_stats_kernel(const uint8_t* x, int64_t
     const uint8_t* xr = x + (int64_t)row * ld_bytes;
     const int nb = cols / 16;
     const float n = (float)cols;
-    float s = 0.0f;
-    for (int b = lane; b < nb; b += 32) {
-        float f[16];
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
+    float s = 0.0f, s2 = 0.0f, mean;
+    if (nb <= 32 * kStatRegBlocks) {
+        // the lane's blocks (lane, lane + 32, ...) loaded at once and kept for both sums
+        uint4 v[kStatRegBlocks][2];
 #pragma unroll
-        for (int i = 0; i < 16; i++) s = __fadd_rn(s, f[i]);
-    }
-    const float mean = __fdiv_rn(warp_butterfly_sum(s), n);
-    float s2 = 0.0f;
-    for (int b = lane; b < nb; b += 32) {
-        float f[16];
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
+        for (int k = 0; k < kStatRegBlocks; k++) {
+            const int b = lane + 32 * k;
+            const bool ok = b < nb;
+            v[k][0] = ok ? __ldg(reinterpret_cast<const uint4*>(xr + b * 32)) : make_uint4(0u, 0u, 0u, 0u);
+            v[k][1] = ok ? __ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
-            const float d = __fsub_rn(f[i], mean);
-            s2 = __fadd_rn(s2, __fmul_rn(d, d));
+        for (int k = 0; k < kStatRegBlocks; k++) {
+            if (lane + 32 * k >= nb) break;
+            float f[16];
+            bf16x8_to_f32(v[k][0], f);
+            bf16x8_to_f32(v[k][1], f + 8);
+#pragma unroll
+            for (int i = 0; i < 16; i++) s = __fadd_rn(s, f[i]);
+        }
+        mean = __fdiv_rn(warp_butterfly_sum(s), n);
+#pragma unroll
+        for (int k = 0; k < kStatRegBlocks; k++) {
+            if (lane + 32 * k >= nb) break;
+            float f[16];
+            bf16x8_to_f32(v[k][0], f);
+            bf16x8_to_f32(v[k][1], f + 8);
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const float d = __fsub_rn(f[i], mean);
+                s2 = __fadd_rn(s2, __fmul_rn(d, d));
+            }
+        }
+    } else {
+        for (int b = lane; b < nb; b += 32) {
+            float f[16];
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
+#pragma unroll
+            for (int i = 0; i < 16; i++) s = __fadd_rn(s, f[i]);
+        }
+        mean = __fdiv_rn(warp_butterfly_sum(s), n);
+        for (int b = lane; b < nb; b += 32) {
+            float f[16];
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const float d = __fsub_rn(f[i], mean);
+                s2 = __fadd_rn(s2, __fmul_rn(d, d));
+            }
         }
     }
     const float var = __fdiv_rn(warp_butterfly_sum(s2), n);
@@ -533,10 +568,10 @@ __global__ void __launch_bounds__(256) ln_stats_kernel(const uint8_t* x, int64_t
 // channel c = h * d + j of the chunk [T][H*d]; partial p (p = 0..31) sums
 // tokens p, p+32, p+64, ... in increasing order from +0, the 32 partials meet
 // in an xor butterfly (16, 8, 4, 2, 1), and mean = S / T, each step one
-// correctly rounded binary32 operation.  A block of 1024 threads covers 64
-// channels of one tensor: warp p computes partial p of two adjacent channels
-// per lane (one 4-byte load a token, 128 contiguous bytes a warp), the
-// partials meet in shared memory, and warp w finishes channels 2w and 2w + 1.
+// correctly rounded binary32 operation.  A block of 1024 threads covers 32
+// channels of one tensor: warp p computes partial p of one channel per lane
+// (a 2-byte load a token, 64 contiguous bytes a warp), the partials meet in
+// shared memory, and warp w finishes channel w.
 struct MeanArgs {
     const uint8_t* x[2];  // bf16 [T][hd]
     float* mean[2];       // [hd], NULL: tensor not smoothed
@@ -545,36 +580,28 @@ struct MeanArgs {
 };
 
 __global__ void __launch_bounds__(1024) kv_channel_mean_kernel(MeanArgs a) {
-    __shared__ float part[32][65];
+    __shared__ float part[32][33];
     const int t = blockIdx.y;
     const uint8_t* x = t ? a.x[1] : a.x[0];
     float* out = t ? a.mean[1] : a.mean[0];
     if (out == nullptr) return;  // the whole block
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x * 64 + 2 * lane;
-    float s0 = 0.0f, s1 = 0.0f;
+    const int c = blockIdx.x * 32 + lane;
+    float s0 = 0.0f;
     if (c < a.hd) {
         const uint8_t* p = x + ((int64_t)warp * a.hd + c) * 2;
         const int64_t stride = (int64_t)32 * a.hd * 2;
 #pragma unroll 8
-        for (int tok = warp; tok < a.T; tok += 32, p += stride) {
-            const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p));
-            s0 = __fadd_rn(s0, __uint_as_float(v << 16));
-            s1 = __fadd_rn(s1, __uint_as_float(v & 0xFFFF0000u));
-        }
+        for (int tok = warp; tok < a.T; tok += 32, p += stride)
+            s0 = __fadd_rn(s0, __uint_as_float((uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p)) << 16));
     }
-    part[warp][2 * lane] = s0;
-    part[warp][2 * lane + 1] = s1;
+    part[warp][lane] = s0;
     __syncthreads();
+    float sum = part[lane][warp];  // lane p holds partial p of channel `warp`
 #pragma unroll
-    for (int k = 0; k < 2; k++) {
-        const int ch = 2 * warp + k;
-        float sum = part[lane][ch];  // lane p holds partial p
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, o));
-        const int cc = blockIdx.x * 64 + ch;
-        if (lane == 0 && cc < a.hd) out[cc] = __fdiv_rn(sum, (float)a.T);
-    }
+    for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xFFFFFFFFu, sum, o));
+    const int cc = blockIdx.x * 32 + warp;
+    if (lane == 0 && cc < a.hd) out[cc] = __fdiv_rn(sum, (float)a.T);
 }
 
 struct DequantArgs {
@@ -956,7 +983,7 @@ extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slo
     m.mean[1] = sv ? cache->v_mean + (int64_t)slot * hd : nullptr;
     m.T = cache->tokens_per_slot;
     m.hd = hd;
-    kv_channel_mean_kernel<<<dim3((unsigned)((hd + 63) / 64), 2), 1024, 0, (cudaStream_t)stream>>>(m);
+    kv_channel_mean_kernel<<<dim3((unsigned)((hd + 31) / 32), 2), 1024, 0, (cudaStream_t)stream>>>(m);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     const float* means[2] = {m.mean[0], m.mean[1]};
     return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, search, workspace, (cudaStream_t)stream, nullptr,
