@@ -591,8 +591,16 @@ __global__ void __launch_bounds__(1024) kv_channel_mean_kernel(MeanArgs a) {
     if (c < a.hd) {
         const uint8_t* p = x + ((int64_t)warp * a.hd + c) * 2;
         const int64_t stride = (int64_t)32 * a.hd * 2;
-#pragma unroll 8
-        for (int tok = warp; tok < a.T; tok += 32, p += stride)
+        // up to 24 tokens' loads in flight before their (in-order) adds
+        int tok = warp;
+        for (; tok + 23 * 32 < a.T; tok += 24 * 32, p += 24 * stride) {
+            uint32_t v[24];
+#pragma unroll
+            for (int k = 0; k < 24; k++) v[k] = __ldg(reinterpret_cast<const uint16_t*>(p + k * stride));
+#pragma unroll
+            for (int k = 0; k < 24; k++) s0 = __fadd_rn(s0, __uint_as_float(v[k] << 16));
+        }
+        for (; tok < a.T; tok += 32, p += stride)
             s0 = __fadd_rn(s0, __uint_as_float((uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p)) << 16));
     }
     part[warp][lane] = s0;
