@@ -15,10 +15,11 @@
 //            at (j / 8) * 2048 + t * 16 + (j % 8) * 2.
 // S = Q K^T and O += P V run as tcgen05.mma kind::f16 (bf16 operands, binary32
 // accumulators in TMEM: S in columns [0, 128), O in [128, 256)), issued by
-// thread 0 and waited on through an mbarrier.  The softmax takes two passes
-// over the keys: the first finds each row's max, the second forms
-// P = exp(scale * (s - max)), sums it (binary32) and accumulates P V with P in
-// bf16, so the output never needs rescaling; O / sum is stored as bf16.  Every wait is
+// thread 0 and waited on through an mbarrier.  The softmax is one pass with a
+// lazy row maximum: P = exp(scale * (s - m)) in bf16 against a reference max m
+// that moves only when a tile exceeds it by more than 2^8 (then the row of O
+// in TMEM and the running sum are rescaled by the thread that owns the row),
+// and O / sum is stored as bf16.  Every wait is
 // bounded; a timeout records NVFP4_ERR_TIMEOUT and the CTA stops.
 #include <algorithm>
 #include <cmath>
@@ -35,6 +36,7 @@ constexpr int kThreads = 128;
 constexpr int kOperandBytes = kTile * kD * 2;  // 32 KB per bf16 128 x 128 operand
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kSCol = 0, kOCol = 128;
+constexpr float kLazyLog2 = 8.0f;  // a row's reference max moves when exceeded by more than 2^8
 
 struct AttnArgs {
     const uint8_t* q;            // bf16 [Tq][H][d]
@@ -212,104 +214,125 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
         }
         return g;
     };
-    for (int pass = 0; pass < 2 && ok; pass++) {
-        int g = next_tile(0);
-        RowRaw kr, vr;
-        if (g < G) {
-            kr = fetch_row(a, 0, slot_of(g), (g % tiles_per_slot) * kTile + i, h);
-            if (pass == 1) vr = fetch_row(a, 1, slot_of(g), (g % tiles_per_slot) * kTile + i, h);
-        }
-        while (g < G && ok) {
-            const int s = slot_of(g), kt = g % tiles_per_slot;
-            const int valid = min(kTile, a.tokens - kt * kTile);
-            const int gn = next_tile(g + 1);
-            // the previous P V product must be done with K, V and P
-            // (every wait's outcome is made uniform over the CTA before
-            // anyone acts on it, so all threads take the same barriers)
-            if (pass == 1 && !first_pv) {
-                const bool got = mbar_wait_bounded(&bar_o, ph_o, &s_abort, a.limit_ns);
-                ph_o ^= 1u;
-                if (!__syncthreads_and(got)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-            }
-            store_row(a, 0, s, h, kr, k_s, i);
-            if (pass == 1) store_row(a, 1, s, h, vr, v_s, i);
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (i == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kD / 16; k++)
-                    mma_f16(t_s, smem_desc(q_s + k * 4096, 2048, 128, kLayoutNone),
-                            smem_desc(k_s + k * 4096, 2048, 128, kLayoutNone), ID_QK, k > 0);
-                tc_commit(&bar_s);
-            }
-            // the next tile's rows load while the product and the softmax run
-            if (gn < G) {
-                kr = fetch_row(a, 0, slot_of(gn), (gn % tiles_per_slot) * kTile + i, h);
-                if (pass == 1) vr = fetch_row(a, 1, slot_of(gn), (gn % tiles_per_slot) * kTile + i, h);
-            }
-            {
-                const bool got = mbar_wait_bounded(&bar_s, ph_s, &s_abort, a.limit_ns);
-                ph_s ^= 1u;
-                if (!__syncthreads_and(got)) {
-                    ok = false;
-                    break;
-                }
+    int g = next_tile(0);
+    RowRaw kr, vr;
+    if (g < G) {
+        kr = fetch_row(a, 0, slot_of(g), (g % tiles_per_slot) * kTile + i, h);
+        vr = fetch_row(a, 1, slot_of(g), (g % tiles_per_slot) * kTile + i, h);
+    }
+    while (g < G && ok) {
+        const int s = slot_of(g), kt = g % tiles_per_slot;
+        const int valid = min(kTile, a.tokens - kt * kTile);
+        const int gn = next_tile(g + 1);
+        // the previous P V product must be done with K, V and P and with O
+        // (every wait's outcome is made uniform over the CTA before anyone
+        // acts on it, so all threads take the same barriers)
+        if (!first_pv) {
+            const bool got = mbar_wait_bounded(&bar_o, ph_o, &s_abort, a.limit_ns);
+            ph_o ^= 1u;
+            if (!__syncthreads_and(got)) {
+                ok = false;
+                break;
             }
             tc_fence_after();
-            uint32_t r[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; c++) tmem_ld_32cols(t_s + lane_off + 32 * c, r[c]);
-            tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
-            if (pass == 0) {
-#pragma unroll
-                for (int c = 0; c < 4; c++)
-#pragma unroll
-                    for (int j = 0; j < 32; j++)
-                        if (32 * c + j < valid) m_run = fmaxf(m_run, __uint_as_float(r[c][j]));
-            } else {
-                // P row i: exp(scale * (s - max)) in bf16, zero for keys past the slot's end
-#pragma unroll
-                for (int c = 0; c < 4; c++)
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; q4++) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; e++) {
-                            const int j0 = 32 * c + 8 * q4 + 2 * e;
-                            const float p0 =
-                                j0 < valid ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e]) - m_run) * a.scale_log2) : 0.0f;
-                            const float p1 = j0 + 1 < valid
-                                                 ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e + 1]) - m_run) * a.scale_log2)
-                                                 : 0.0f;
-                            l_run += p0 + p1;
-                            const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
-                            w[e] = *reinterpret_cast<const uint32_t*>(&b);
-                        }
-                        st_shared16(p_s + (4 * c + q4) * 2048 + i * 16, make_uint4(w[0], w[1], w[2], w[3]));
-                    }
-            }
-            // every row's S is read before the next Q K^T overwrites it
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (pass == 1 && i == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kTile / 16; k++)
-                    mma_f16(t_o, smem_desc(p_s + k * 4096, 2048, 128, kLayoutNone),
-                            smem_desc(v_s + k * 256, 128, 2048, kLayoutNone), ID_PV, (!first_pv || k > 0) ? 1u : 0u);
-                tc_commit(&bar_o);
-            }
-            if (pass == 1) first_pv = false;
-            g = gn;
         }
+        store_row(a, 0, s, h, kr, k_s, i);
+        store_row(a, 1, s, h, vr, v_s, i);
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (i == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < kD / 16; k++)
+                mma_f16(t_s, smem_desc(q_s + k * 4096, 2048, 128, kLayoutNone),
+                        smem_desc(k_s + k * 4096, 2048, 128, kLayoutNone), ID_QK, k > 0);
+            tc_commit(&bar_s);
+        }
+        // the next tile's rows load while the product and the softmax run
+        if (gn < G) {
+            kr = fetch_row(a, 0, slot_of(gn), (gn % tiles_per_slot) * kTile + i, h);
+            vr = fetch_row(a, 1, slot_of(gn), (gn % tiles_per_slot) * kTile + i, h);
+        }
+        {
+            const bool got = mbar_wait_bounded(&bar_s, ph_s, &s_abort, a.limit_ns);
+            ph_s ^= 1u;
+            if (!__syncthreads_and(got)) {
+                ok = false;
+                break;
+            }
+        }
+        tc_fence_after();
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; c++) tmem_ld_32cols(t_s + lane_off + 32 * c, r[c]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
+        // online softmax with a lazy maximum: the row's reference max moves
+        // only when this tile exceeds it by more than 2^8 in exp(scale * s),
+        // and then O (in TMEM) and the running sum are rescaled; otherwise P
+        // stays below 2^8, which bf16 and the binary32 accumulators carry
+        float mt = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+#pragma unroll
+            for (int j = 0; j < 32; j++)
+                if (32 * c + j < valid) mt = fmaxf(mt, __uint_as_float(r[c][j]));
+        float factor = 1.0f;  // O's rescale, applied after P is formed (S's registers are free then)
+        if ((mt - m_run) * a.scale_log2 > kLazyLog2) {
+            factor = ex2((m_run - mt) * a.scale_log2);  // 0 on the first tile (m_run = -inf)
+            l_run *= factor;
+            m_run = mt;
+        }
+        // P row i: exp(scale * (s - m_run)) in bf16, zero for keys past the slot's end
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+#pragma unroll
+            for (int q4 = 0; q4 < 4; q4++) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int j0 = 32 * c + 8 * q4 + 2 * e;
+                    const float p0 =
+                        j0 < valid ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e]) - m_run) * a.scale_log2) : 0.0f;
+                    const float p1 = j0 + 1 < valid
+                                         ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e + 1]) - m_run) * a.scale_log2)
+                                         : 0.0f;
+                    l_run += p0 + p1;
+                    const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
+                    w[e] = *reinterpret_cast<const uint32_t*>(&b);
+                }
+                st_shared16(p_s + (4 * c + q4) * 2048 + i * 16, make_uint4(w[0], w[1], w[2], w[3]));
+            }
+        // tcgen05.ld / st are warp-collective: the warp rescales together when any
+        // of its rows needs it (the others multiply by exactly 1)
+        if (__any_sync(0xFFFFFFFFu, factor != 1.0f) && !first_pv) {
+            uint32_t o[32];
+#pragma unroll 1
+            for (int c = 0; c < 4; c++) {
+                tmem_ld_32cols(t_o + lane_off + 32 * c, o);
+                tmem_ld_wait();
+                tmem_regs_ready(o);
+#pragma unroll
+                for (int j = 0; j < 32; j++) o[j] = __float_as_uint(__uint_as_float(o[j]) * factor);
+                tmem_st_32cols(t_o + lane_off + 32 * c, o);
+            }
+            tmem_st_wait();
+        }
+        // every row's S is read (and O rescaled) before the next MMAs
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (i == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < kTile / 16; k++)
+                mma_f16(t_o, smem_desc(p_s + k * 4096, 2048, 128, kLayoutNone),
+                        smem_desc(v_s + k * 256, 128, 2048, kLayoutNone), ID_PV, (!first_pv || k > 0) ? 1u : 0u);
+            tc_commit(&bar_o);
+        }
+        first_pv = false;
+        g = gn;
     }
     // O row i / l -> bf16
     if (ok && !first_pv) {
