@@ -562,8 +562,8 @@ def run_ours(args, rank: int, world: int) -> dict | None:
             "wgrad_TFLOP/s": round(2.0 * N * K * M / (train["wgrad_ms"] * 1e-3) / 1e12, 1)},
         "kv_attention": {
             "what": "softmax attention of one 2640x24x128 bf16 query chunk over NVFP4 cache slots read directly "
-                    "(dequant into the tensor-core tiles, tcgen05 bf16 MMAs, two-pass softmax), outside the step; "
-                    "TFLOP/s counts 4*Tq*keys*d*H",
+                    "(e2m1 * s tiles in binary16, tcgen05 f16 MMAs with binary32 accumulators, one-pass softmax), "
+                    "outside the step; TFLOP/s counts 4*Tq*keys*d*H",
             "bf16_peak_TFLOP/s": pk.get("bf16_tflops"), **attn},
         "ln_modulate_quantize": {
             "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A, two launches, outside the step",

@@ -53,11 +53,12 @@ struct AttnArgs {
     uint64_t limit_ns;
 };
 
-// instruction descriptor of kind::f16: binary32 accumulator, bf16 A and B,
-// A K-major, B K-major (b_mn = 0) or MN-major (1), M = N = 128
-__host__ __device__ constexpr uint32_t idesc_f16(int b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(kTile >> 3) << 17) |
-           ((uint32_t)(kTile >> 4) << 24);
+// instruction descriptor of kind::f16: binary32 accumulator, A and B both
+// binary16 (bf = 0) or both bf16 (bf = 1), A K-major, B K-major (b_mn = 0) or
+// MN-major (1), M = N = 128
+__host__ __device__ constexpr uint32_t idesc_f16(int b_mn, int bf) {
+    return (1u << 4) | ((uint32_t)bf << 7) | ((uint32_t)bf << 10) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(kTile >> 3) << 17) | ((uint32_t)(kTile >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -101,6 +102,21 @@ __device__ __forceinline__ uint4 dq8(uint32_t q, uint32_t sc, float a32, const f
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// 8 E2M1 codes times their block scale, exactly, as binary16 (every product
+// e2m1 * s of an E2M1 value and an E4M3 scale is exact in binary16): the
+// operand values of the binary16 path, whose tensor scale a32 is applied to
+// the products instead.
+__device__ __forceinline__ uint4 raw8(uint32_t q, uint32_t sc) {
+    const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const __half2 v = __hmul2(e2m1x2_to_half2((q >> (8 * j)) & 0xFFu), s2);
+        o[j] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // One token row (token `tok` of slot s, head h) of K or V as stored: 64 code
 // bytes, 8 scale bytes and the slot's a32; zeros when the token is past the
 // slot's end.  Fetched a tile ahead so the loads overlap the tile in flight.
@@ -133,6 +149,7 @@ __device__ __forceinline__ RowRaw fetch_row(const AttnArgs& a, int t, int s, int
 // The row's 128 dequantized bf16 values into the operand at `base` (K-major
 // and MN-major layouts put a row at the same places); a row past the slot's
 // end (codes 0, a32 0, no mean) decodes to zeros.
+template <bool RAW>
 __device__ __forceinline__ void store_row(const AttnArgs& a, int t, int s, int h, const RowRaw& r, uint32_t base,
                                          int row) {
     const float* m = (a.mean[t] && r.valid) ? a.mean[t] + ((int64_t)s * a.heads + h) * kD : nullptr;
@@ -144,11 +161,20 @@ __device__ __forceinline__ void store_row(const AttnArgs& a, int t, int s, int h
         for (int j = 0; j < 4; j++) {
             const int chunk = 4 * k + j;  // elements 8 * chunk .. + 7; block chunk / 2
             const uint32_t sc = (sw[chunk / 8] >> (8 * ((chunk / 2) % 4))) & 0xFFu;
-            st_shared16(base + chunk * 2048 + row * 16, dq8(cw[j], sc, r.a32, m ? m + 8 * chunk : nullptr));
+            st_shared16(base + chunk * 2048 + row * 16,
+                        RAW ? raw8(cw[j], sc) : dq8(cw[j], sc, r.a32, m ? m + 8 * chunk : nullptr));
         }
     }
 }
 
+// RAW (no smoothing mean on either tensor): binary16 operands.  Each Q row is
+// scaled by a power of two 2^k (exact) so that its largest magnitude lies in
+// [2^14, 2^15), then rounded to binary16; K and V tiles hold e2m1 * s exactly;
+// the row's 2^-k and the slot's K scale a32_K multiply the products inside the
+// exponent, and P carries a32_V / a32_ref (a32_ref: the largest V scale of the
+// listed slots), O being multiplied by a32_ref at the end.  Otherwise: bf16
+// operands holding the cache's bf16 dequant (with the smoothing means).
+template <bool RAW>
 __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_constant__ AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint64_t bar_s, bar_o;
@@ -169,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
         tmem_alloc(&tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    // Q row i (zeros past the last query)
+    // Q row i (zeros past the last query); RAW: times 2^k into binary16
+    float q_inv = 1.0f;  // RAW: 2^-k
     {
         const int qrow = qt * kTile + i;
         uint4 v[16];
@@ -181,8 +208,40 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
 #pragma unroll
             for (int c = 0; c < 16; c++) v[c] = make_uint4(0u, 0u, 0u, 0u);
         }
+        if (RAW) {
+            uint32_t mx = 0u;  // largest bf16 magnitude bits of the row
+#pragma unroll
+            for (int c = 0; c < 16; c++)
+                mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v[c].x & 0x7FFF7FFFu, v[c].y & 0x7FFF7FFFu),
+                                           __vmaxu2(v[c].z & 0x7FFF7FFFu, v[c].w & 0x7FFF7FFFu)));
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            // 2^k brings the largest magnitude into [2^14, 2^15): k = 141 - its biased exponent
+            const int k = mx == 0u ? 0 : min(100, max(-100, 141 - (int)(mx >> 7)));
+            const float pk = __uint_as_float((uint32_t)(127 + k) << 23);
+            q_inv = __uint_as_float((uint32_t)(127 - k) << 23);
+#pragma unroll
+            for (int c = 0; c < 16; c++) {
+                uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const __half2 hv = __floats2half2_rn(__uint_as_float(w[e] << 16) * pk,
+                                                         __uint_as_float(w[e] & 0xFFFF0000u) * pk);
+                    w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+                }
+                v[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
 #pragma unroll
         for (int c = 0; c < 16; c++) st_shared16(q_s + c * 2048 + i * 16, v[c]);
+    }
+    // RAW: the largest V tensor scale of the listed slots (the same in every thread)
+    float a_ref = 1.0f;
+    if (RAW) {
+        a_ref = 0.0f;
+        for (int si = 0; si < a.n; si++) {
+            const int s = __ldg(a.slots + si);
+            if (s >= 0 && s < a.n_slots) a_ref = fmaxf(a_ref, __ldg(a.gscale[1] + s));
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -190,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
     const uint32_t tmem = tmem_base;
     const uint32_t t_s = tmem + kSCol, t_o = tmem + kOCol;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    constexpr uint32_t ID_QK = idesc_f16(0), ID_PV = idesc_f16(1);
+    constexpr uint32_t ID_QK = idesc_f16(0, RAW ? 0 : 1), ID_PV = idesc_f16(1, RAW ? 0 : 1);
     const int tiles_per_slot = (a.tokens + kTile - 1) / kTile;
     uint32_t ph_s = 0, ph_o = 0;
     bool ok = true;
@@ -236,8 +295,8 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
             }
             tc_fence_after();
         }
-        store_row(a, 0, s, h, kr, k_s, i);
-        store_row(a, 1, s, h, vr, v_s, i);
+        store_row<RAW>(a, 0, s, h, kr, k_s, i);
+        store_row<RAW>(a, 1, s, h, vr, v_s, i);
         fence_proxy_async_smem();
         __syncthreads();
         if (i == 0) {
@@ -268,23 +327,28 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 4; c++) tmem_regs_ready(r[c]);
-        // online softmax with a lazy maximum: the row's reference max moves
-        // only when this tile exceeds it by more than 2^8 in exp(scale * s),
-        // and then O (in TMEM) and the running sum are rescaled; otherwise P
-        // stays below 2^8, which bf16 and the binary32 accumulators carry
-        float mt = -INFINITY;
+        // online softmax with a lazy maximum, in exponent units t = c_s * S
+        // (exp(scale * q.k) = 2^t; RAW: c_s also carries the row's 2^-k and the
+        // slot's a32_K): the row's reference max moves only when this tile
+        // exceeds it by more than 8, and then O (in TMEM) and the running sum
+        // are rescaled; otherwise P stays below 2^8
+        const float c_s = RAW ? q_inv * __ldg(a.gscale[0] + s) * a.scale_log2 : a.scale_log2;
+        const float w_s = RAW ? (a_ref > 0.0f ? __fdiv_rn(__ldg(a.gscale[1] + s), a_ref) : 0.0f) : 1.0f;
+        float smax = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; c++)
 #pragma unroll
             for (int j = 0; j < 32; j++)
-                if (32 * c + j < valid) mt = fmaxf(mt, __uint_as_float(r[c][j]));
+                if (32 * c + j < valid) smax = fmaxf(smax, __uint_as_float(r[c][j]));
+        const float mt = smax * c_s;  // c_s >= 0
         float factor = 1.0f;  // O's rescale, applied after P is formed (S's registers are free then)
-        if ((mt - m_run) * a.scale_log2 > kLazyLog2) {
-            factor = ex2((m_run - mt) * a.scale_log2);  // 0 on the first tile (m_run = -inf)
+        if (mt - m_run > kLazyLog2) {
+            factor = ex2(m_run - mt);  // 0 on the first tile (m_run = -inf)
             l_run *= factor;
             m_run = mt;
         }
-        // P row i: exp(scale * (s - m_run)) in bf16, zero for keys past the slot's end
+        // P row i: 2^(t - m_run) times w_s (RAW: a32_V / a32_ref) in binary16
+        // (RAW) or bf16, zero for keys past the slot's end
 #pragma unroll
         for (int c = 0; c < 4; c++)
 #pragma unroll
@@ -293,14 +357,17 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
                     const int j0 = 32 * c + 8 * q4 + 2 * e;
-                    const float p0 =
-                        j0 < valid ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e]) - m_run) * a.scale_log2) : 0.0f;
-                    const float p1 = j0 + 1 < valid
-                                         ? ex2((__uint_as_float(r[c][8 * q4 + 2 * e + 1]) - m_run) * a.scale_log2)
-                                         : 0.0f;
+                    const float p0 = j0 < valid ? ex2(fmaf(__uint_as_float(r[c][8 * q4 + 2 * e]), c_s, -m_run)) : 0.0f;
+                    const float p1 =
+                        j0 + 1 < valid ? ex2(fmaf(__uint_as_float(r[c][8 * q4 + 2 * e + 1]), c_s, -m_run)) : 0.0f;
                     l_run += p0 + p1;
-                    const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
-                    w[e] = *reinterpret_cast<const uint32_t*>(&b);
+                    if (RAW) {
+                        const __half2 hv = __floats2half2_rn(p0 * w_s, p1 * w_s);
+                        w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+                    } else {
+                        const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
+                        w[e] = *reinterpret_cast<const uint32_t*>(&b);
+                    }
                 }
                 st_shared16(p_s + (4 * c + q4) * 2048 + i * 16, make_uint4(w[0], w[1], w[2], w[3]));
             }
@@ -344,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
         if (i == 0) record_error(a.err, NVFP4_ERR_TIMEOUT, 3);
     } else {
         const int qrow = qt * kTile + i;
-        const float inv_l = l_run > 0.0f ? __frcp_rn(l_run) : 0.0f;
+        const float inv_l = l_run > 0.0f ? __fdiv_rn(a_ref, l_run) : 0.0f;  // a_ref = 1 unless RAW
         uint32_t r[4][32];
         if (!first_pv) {
 #pragma unroll
@@ -460,13 +527,16 @@ extern "C" nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const in
     a.err = static_cast<DevError*>(workspace);
     a.limit_ns = 2000000000ull;
     const int smem = 3 * kOperandBytes;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(kv_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    // caches without smoothing means take the binary16 path
+    const bool raw = !sk && !sv;
+    void (*kern)(AttnArgs) = raw ? kv_attention_kernel<true> : kv_attention_kernel<false>;
+    static bool attr[2] = {false, false};
+    if (!attr[raw]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return NVFP4_ERR_CUDA;
-        attr = true;
+        attr[raw] = true;
     }
     const dim3 grid((unsigned)((tq + kTile - 1) / kTile), (unsigned)cache->heads);
-    kv_attention_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(a);
+    kern<<<grid, kThreads, smem, (cudaStream_t)stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

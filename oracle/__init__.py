@@ -406,12 +406,17 @@ def attention_chunks(t: int, sink_global: int, shot_start: int, sink_shot: int, 
     return sorted(c for c in s if 0 <= c < t)
 
 
+def _as_f64(x: np.ndarray) -> np.ndarray:
+    """bf16 bits (uint16) or binary32 values -> float64."""
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.asarray(x, dtype=np.float64)
+
+
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
-    """fp64 softmax attention of bf16 bits q [Tq, H, d] over bf16 bits k, v [L, H, d] (every query sees every
-    key): O[i, h] = sum_j softmax_j(scale * q[i, h] . k[j, h]) v[j, h].  Returns float64 [Tq, H, d]."""
-    qf = (q.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    kf = (k.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    vf = (v.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    """fp64 softmax attention of q [Tq, H, d] over k, v [L, H, d] (bf16 bits or binary32 values; every query
+    sees every key): O[i, h] = sum_j softmax_j(scale * q[i, h] . k[j, h]) v[j, h].  Returns float64 [Tq, H, d]."""
+    qf, kf, vf = _as_f64(q), _as_f64(k), _as_f64(v)
     Tq, H, d = qf.shape
     out = np.zeros((Tq, H, d), np.float64)
     for h in range(H):

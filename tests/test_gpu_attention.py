@@ -1,7 +1,8 @@
 """GPU parity of nvfp4_kv_attention (softmax attention of bf16 queries over NVFP4
 cache slots read directly by the kernel) against the oracle's fp64 attention over
-the oracle's bf16 dequant of the same slots (reading R23: max |O - O_ref| /
-max |O_ref| <= 1e-2)."""
+the same slots' values -- exact e2m1 * s * a32 for a cache without smoothing, the
+bf16 dequant with the means otherwise (reading R23: max |O - O_ref| / max |O_ref|
+<= 1e-2)."""
 import numpy as np
 import pytest
 import torch
@@ -25,6 +26,10 @@ def _case(T, H, Tq, slot_chunks, n_slots, seed, smooth_k=False, smooth_v=False, 
     compare against the oracle (on sampled query rows when `rows` is given)."""
     d = 128
     cache = nv.KVCache(n_slots, T, H, d, smooth_k=smooth_k, smooth_v=smooth_v)
+    # keys and values as the kernel reads them (reading R23): without smoothing the cache's
+    # exact values e2m1 * s * a32 (binary16 path); with smoothing on either tensor the
+    # cache's bf16 dequant (plus the means) for both
+    raw = not (smooth_k or smooth_v)
     kh, vh = {}, {}
     for s in range(n_slots):
         k, v = syn.kv_chunk_bf16(T, H, d, seed=seed + s)
@@ -35,7 +40,8 @@ def _case(T, H, Tq, slot_chunks, n_slots, seed, smooth_k=False, smooth_v=False, 
                 store[s] = oracle.kv_dequant_smooth(c, sc, a, m, T, H, d)
             else:
                 c, sc, a = oracle.kv_append(x)
-                store[s] = oracle.kv_dequant(c, sc, a, T, H, d)
+                store[s] = (oracle.dequant_f32(c, sc, a).reshape(T, H, d) if raw
+                            else oracle.kv_dequant(c, sc, a, T, H, d))
     q = syn.kv_chunk_bf16(Tq, H, d, seed=seed + 1000)[0]
     slots = torch.tensor(slot_chunks, dtype=torch.int32, device="cuda")
     o = cache.attention(slots, dev_bf16(q), scale=scale)
@@ -119,6 +125,6 @@ def test_smoothed_channel_constant_slot_with_zero_tensor_scale():
     q = syn.kv_chunk_bf16(40, H, d, seed=6)[0]
     o = cache.attention(torch.tensor([0], dtype=torch.int32, device="cuda"), dev_bf16(q))
     torch.cuda.synchronize()
-    c, sc, a = oracle.kv_append(v)
+    c, sc, a = oracle.kv_append(v)  # smoothed cache: the bf16 path for both tensors
     ref = oracle.attention(q, kb, oracle.kv_dequant(c, sc, a, T, H, d), 1.0 / np.sqrt(d))
     assert normwise_err(_bits_to_f64(host_bits(o)).reshape(-1), ref.reshape(-1)) <= TOL
