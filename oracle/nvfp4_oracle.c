@@ -19,7 +19,7 @@
  *        frame-chunk's K and V are quantized separately; storage goes from
  *        4*T_c*H*d to 9/8*T_c*H*d bytes.
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent:
  *  R1  tensor scale  a32 = fl32(amax / 2688), 2688 = 6 * 448 (E2M1 max times
  *      E4M3 max), so the tensor's largest block gets the largest block scale.
  *  R2  a32 == 0 (all-zero tensor): every scale code and element code is 0.
