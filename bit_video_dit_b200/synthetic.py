@@ -75,6 +75,37 @@ def kv_chunk_bf16(T: int, H: int, d: int, seed: int):
     return out[0], out[1]
 
 
+def rope_table(T: int, d: int, seed: int | None = None, start: int = 0, base: float = 10000.0):
+    """A rotary angle table, cos and sin as binary32 [T, d/2]: seeded uniform
+    angles in [-pi, pi) when `seed` is given, else token positions start ..
+    start + T - 1 times the frequencies base^(-2p/d) (float64, then rounded)."""
+    if seed is not None:
+        ang = rng(seed).uniform(-np.pi, np.pi, size=(T, d // 2))
+    else:
+        pos = np.arange(start, start + T, dtype=np.float64)
+        ang = pos[:, None] * base ** (-2.0 * np.arange(d // 2, dtype=np.float64) / d)[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def rope_table_3d(frames: int, hh: int, ww: int, d: int, frame0: int = 0, base: float = 10000.0):
+    """The 3D (frame, row, column) angle table of a chunk of frames x hh x ww
+    latent patches, tokens frame-major: the head's d/2 pairs split into a frame
+    band of d/2 - 2*floor(d/6) pairs, then a row band and a column band of
+    floor(d/6) pairs each (22, 21, 21 for d = 128); pair i of a band of n pairs
+    turns by its axis position times base^(-i/n).  cos and sin as binary32
+    [frames*hh*ww, d/2]."""
+    npair = d // 2
+    nb = d // 6  # pairs per spatial band
+    nt = npair - 2 * nb
+    f, r, c = np.meshgrid(np.arange(frame0, frame0 + frames), np.arange(hh), np.arange(ww), indexing="ij")
+    parts = []
+    for pos, n in ((f, nt), (r, nb), (c, nb)):
+        freq = base ** (-2.0 * np.arange(n, dtype=np.float64) / (2 * n))
+        parts.append(pos.reshape(-1, 1).astype(np.float64) * freq[None, :])
+    ang = np.concatenate(parts, axis=1)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
 @dataclass(frozen=True)
 class GemmShape:
     M: int
@@ -94,3 +125,5 @@ STACK_LAYER = (GemmShape(STACK_M, 9216, 3072), GemmShape(STACK_M, 3072, 3072),
 
 # NVFP4 KV cache: 21 ring slots (frame-chunks) x 2640 tokens x 24 heads x 128.
 KV_SLOTS, KV_TOKENS, KV_HEADS, KV_DIM = 21, 2640, 24, 128
+# a chunk's tokens as a latent grid: 3 frames x 22 x 40 patches (720p)
+KV_GRID = (3, 22, 40)

@@ -110,6 +110,10 @@ def lib():
                 getattr(L, name).argtypes = [vp, i64, i64, ctypes.c_int, vp, vp, vp, vp, vp]
                 getattr(L, name).restype = ctypes.c_int
             L.orc_rht16_f32.argtypes = [vp, i64, vp, vp]
+            L.orc_rope.argtypes = [vp, i64, i64, i64, vp, vp, vp]
+            L.orc_channel_mean_f32.argtypes = [vp, i64, i64, vp]
+            L.orc_kv_append_rope.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, vp, vp]
+            L.orc_kv_append_rope.restype = ctypes.c_int
             L.orc_quantize_t_bf16.argtypes = [vp, i64, i64, i64, vp, ctypes.c_int, vp, vp, vp]
             L.orc_quantize_t_bf16.restype = ctypes.c_int
             _lib = L
@@ -342,6 +346,53 @@ def kv_dequant_smooth(codes, scales, alpha, mean, T: int, H: int, d: int) -> np.
     lib().orc_kv_dequant_smooth(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)), float(alpha),
                                 _p(mean), T, H, d, _p(out))
     return out
+
+
+def _rope_tables(cos, sin, T: int, d: int):
+    cs = np.ascontiguousarray(cos, dtype=np.float32)
+    sn = np.ascontiguousarray(sin, dtype=np.float32)
+    if cs.shape != (T, d // 2) or sn.shape != (T, d // 2):
+        raise ValueError("cos / sin must be [T, d/2]")
+    return cs, sn
+
+
+def rope(x: np.ndarray, cos, sin) -> np.ndarray:
+    """R24: bf16 bits x [T, H, d] with every head's interleaved pairs (2p, 2p+1)
+    turned by the binary32 angle table (cos, sin [T, d/2]); binary32 [T, H, d]."""
+    T, H, d = x.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    cs, sn = _rope_tables(cos, sin, T, d)
+    y = np.zeros((T, H, d), np.float32)
+    lib().orc_rope(_p(x), T, H, d, _p(cs), _p(sn), _p(y))
+    return y
+
+
+def channel_mean_f32(v: np.ndarray) -> np.ndarray:
+    """R20's channel mean of binary32 values v [T, C...] (same order as channel_mean)."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    T = v.shape[0]
+    C = v.size // T
+    mean = np.zeros(C, np.float32)
+    lib().orc_channel_mean_f32(_p(v), T, C, _p(mean))
+    return mean
+
+
+def kv_append_rope(x: np.ndarray, cos, sin, smooth: bool = False, search46: bool = False):
+    """The keys' append with R24 (x bf16 bits [T, H, d]): rope, then (smooth) the
+    channel means of the rotated keys taken out (R20), then the quantize.
+    Returns (codes, scales, alpha, mean [H*d] or None)."""
+    T, H, d = x.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    cs, sn = _rope_tables(cos, sin, T, d)
+    codes = np.zeros((T * H, d // 2), np.uint8)
+    scales = np.zeros((T * H, d // 16), np.uint8)
+    a = np.zeros(1, np.float32)
+    mean = np.zeros(H * d, np.float32) if smooth else None
+    rc = lib().orc_kv_append_rope(_p(x), T, H, d, _p(cs), _p(sn), MODE_SEARCH46 if search46 else 0, _p(codes),
+                                  _p(scales), _p(a), _p(mean))
+    if rc != 0:
+        raise ValueError(f"orc_kv_append_rope failed ({rc})")
+    return codes, scales, np.float32(a[0]), mean
 
 
 def quantize_2d(x: np.ndarray, alpha: float | None = None):

@@ -58,6 +58,12 @@
  *  R22 Random Hadamard Transform ahead of the weight-gradient quantize
  *      [RN-T]: 16-point, normalised, Sylvester order, one sign vector; see
  *      rht16.
+ *  R24 rotary position embedding of a KV chunk's keys ahead of their
+ *      quantize (optional; the fused RoPE ahead of the in-place KV update of
+ *      the anzhuoshouzhuan.com article, "NVFP4 量化"): the interleaved pairs
+ *      (2p, 2p+1) of every head turn by the angle of (token, p), given as a
+ *      binary32 cos / sin table; see orc_rope for the order.  Values are never
+ *      rounded to bf16 between the rotation and the quantize.
  *
  * Every floating-point step that the GPU must reproduce bit for bit is done in
  * IEEE binary32 (compile with -ffp-contract=off so nothing fuses); the GEMM
@@ -687,6 +693,72 @@ ORC_API void orc_kv_dequant_smooth(const uint8_t* codes, const uint8_t* scales, 
             float y = v + mean[(r % H) * d + c];
             out[r * d + c] = orc_f32_to_bf16(y);
         }
+}
+
+/* ------------------------------------------------------------------------ */
+/* R24: rotary position embedding of a chunk's keys before the quantize       */
+/* ------------------------------------------------------------------------ */
+/* x: bf16 [T][H][d] (d even); cs, sn: binary32 [T][d/2], the cosine and sine
+ * of the angle of token t's pair p.  For every token t, head h and pair p
+ * (channels 2p and 2p+1 of the head), with c = cs[t][p], s = sn[t][p]:
+ *   y[2p]   = fl32(fl32(x[2p] * c) - fl32(x[2p+1] * s))
+ *   y[2p+1] = fl32(fl32(x[2p] * s) + fl32(x[2p+1] * c))
+ * i.e. the complex product (x[2p] + i x[2p+1]) (c + i s), each product and
+ * the sum rounded once in binary32. */
+ORC_API void orc_rope(const uint16_t* x, int64_t T, int64_t H, int64_t d, const float* cs, const float* sn, float* y)
+{
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t t = 0; t < T; t++)
+        for (int64_t h = 0; h < H; h++) {
+            const int64_t base = (t * H + h) * d;
+            for (int64_t p = 0; p < d / 2; p++) {
+                const float x0 = orc_bf16_to_f32(x[base + 2 * p]);
+                const float x1 = orc_bf16_to_f32(x[base + 2 * p + 1]);
+                const float c = cs[t * (d / 2) + p], s = sn[t * (d / 2) + p];
+                const float a = x0 * c, b = x1 * s, e = x0 * s, f = x1 * c;
+                y[base + 2 * p] = a - b;
+                y[base + 2 * p + 1] = e + f;
+            }
+        }
+}
+
+/* R20's channel mean of binary32 values v [T][C], same order as
+ * orc_channel_mean. */
+ORC_API void orc_channel_mean_f32(const float* v, int64_t T, int64_t C, float* mean)
+{
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t c = 0; c < C; c++) {
+        float part[32];
+        for (int p = 0; p < 32; p++) {
+            float s = 0.0f;
+            for (int64_t t = p; t < T; t += 32) s = s + v[t * C + c];
+            part[p] = s;
+        }
+        mean[c] = butterfly32(part) / (float)T;
+    }
+}
+
+/* The keys' append with R24: y = orc_rope(x); with K-smoothing (mean != NULL)
+ * the channel means of y (R20's order) and the quantize of fl32(y - mean),
+ * else the quantize of y; a32 from the quantized values (R1), blocks and
+ * layout as orc_kv_append (R15, R16; mode may carry ORC_MODE_SEARCH46). */
+ORC_API int orc_kv_append_rope(const uint16_t* x, int64_t T, int64_t H, int64_t d, const float* cs,
+                               const float* sn, int mode, uint8_t* codes, uint8_t* scales, float* alpha,
+                               float* mean)
+{
+    const int64_t C = H * d;
+    if (d % 16 != 0) return 1;
+    float* y = (float*)malloc((size_t)(T * C) * sizeof(float) + 1);
+    if (!y) return 2;
+    orc_rope(x, T, H, d, cs, sn, y);
+    if (mean) {
+        orc_channel_mean_f32(y, T, C, mean);
+        for (int64_t t = 0; t < T; t++)
+            for (int64_t c = 0; c < C; c++) y[t * C + c] = y[t * C + c] - mean[c];
+    }
+    int rc = orc_quantize_f32(y, T * H, d, d, ORC_MODE_COMPUTE | (mode & ORC_MODE_SEARCH46), alpha, codes, scales);
+    free(y);
+    return rc;
 }
 
 /* ------------------------------------------------------------------------ */
