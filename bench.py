@@ -219,8 +219,33 @@ def measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, rep
     sm_ap_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
     sm_dq_ms = float(np.median([e[2].elapsed_time(e[3]) for e in ev]))
     del g
+    # the keys' RoPE fused ahead of their quantize (3-frame x 22 x 40 angle table), on the
+    # plain cache and on the smoothed + searched one (means of the turned keys)
+    cs, sn = syn.rope_table_3d(*syn.KV_GRID, cache.head_dim)
+    rope = (torch.from_numpy(cs).to(a.device), torch.from_numpy(sn).to(a.device))
+    cache.append(0, *chunks[0], rope=rope)
+    cache_k.append(0, *chunks[0], rope=rope)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            cache.dequant(ring, k_out, v_out)
+            ev[i][0].record()
+            cache.append(i % cache.n_slots, *chunks[i % len(chunks)], rope=rope)
+            ev[i][1].record()
+            cache.dequant(ring, k_out, v_out)
+            ev[i][2].record()
+            cache_k.append(i % cache_k.n_slots, *chunks[i % len(chunks)], rope=rope)
+            ev[i][3].record()
+    g.replay()
+    torch.cuda.synchronize()
+    rp_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
+    rp_sm_ms = float(np.median([e[2].elapsed_time(e[3]) for e in ev]))
+    del g
     return {"quantize_ms": q_ms, "kv_append_ms": ap_ms, "ln_quantize_ms": ln_ms,
-            "smooth_append_ms": sm_ap_ms, "smooth_dequant_ms": sm_dq_ms}
+            "smooth_append_ms": sm_ap_ms, "smooth_dequant_ms": sm_dq_ms,
+            "rope_append_ms": rp_ms, "rope_smooth_append_ms": rp_sm_ms}
 
 
 RHT_SIGN = (1, -1, -1, 1, 1, 1, -1, 1, -1, -1, 1, -1, 1, 1, -1, -1)
@@ -548,6 +573,14 @@ def run_ours(args, rank: int, world: int) -> dict | None:
             "append_GB/s": round(append_bytes / (search["smooth_append_ms"] * 1e-3) / 1e9, 1),
             "dequant_ms": round(search["smooth_dequant_ms"], 4),
             "dequant_GB/s": round(dequant_bytes / (search["smooth_dequant_ms"] * 1e-3) / 1e9, 1)},
+        "kv_rope": {
+            "what": "KV append with the keys' rotary embedding fused ahead of their quantize (3-frame x 22 x 40 "
+                    "angle table read from L2), plain and with K-smoothing + scale search (means of the turned "
+                    "keys, two launches), outside the step; GB/s counts the append's algorithmic bytes",
+            "append_ms": round(search["rope_append_ms"], 4),
+            "append_GB/s": round(append_bytes / (search["rope_append_ms"] * 1e-3) / 1e9, 1),
+            "smooth_search_append_ms": round(search["rope_smooth_append_ms"], 4),
+            "smooth_search_append_GB/s": round(append_bytes / (search["rope_smooth_append_ms"] * 1e-3) / 1e9, 1)},
         "training": {
             "what": "training-side NVFP4 on the QKV layer shapes, outside the step: 2D (16x16) scaling of W "
                     "[9216x3072] writing W and W^T operands; RHT + transposed 1D quantize of X [4096x3072] and "

@@ -80,6 +80,14 @@ struct QuantArgs {
     // the element at flat index i belongs to channel i mod smooth_hd
     const float* smooth_mean[2];
     int smooth_hd;
+    // rotary position embedding of tensor 0 (the keys) ahead of the quantize
+    // (smoothing kernels only, one row per tensor): binary32 cos / sin
+    // [tokens][rope_d / 2]; the element at flat index i is channel i mod rope_d
+    // of a head of token i / rope_hd (NULL: none)
+    const float* rope_cos;
+    const float* rope_sin;
+    int rope_d;
+    int rope_hd;
     uint32_t* ctl;
     DevError* err;
     uint64_t limit_ns;
@@ -204,17 +212,39 @@ __device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool 
 // Value transforms ahead of the encode (a template parameter of the kernel).
 constexpr int kXfNone = 0;    // the bf16 input as is
 constexpr int kXfLn = 1;      // LayerNorm + adaLN modulate of each row
-constexpr int kXfSmooth = 2;  // minus the channel mean (K-smoothing of a KV chunk)
+constexpr int kXfSmooth = 2;  // RoPE of the keys, then minus the channel mean (KV chunk)
 
 // The 16 binary32 values of the lane's block of the run at w (tensor t): the
 // bf16 input; with LN its LayerNorm + modulate, in this order and rounding:
 // m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift);
-// with smoothing fl32(x - mean[channel]).
+// for a KV chunk, the keys' rotary embedding where a table is given (pair
+// (x0, x1) -> (fl32(fl32(x0 c) - fl32(x1 s)), fl32(fl32(x0 s) + fl32(x1 c))),
+// c and s of the element's token and pair), then fl32(y - mean[channel]) where
+// means are given.
 template <int XF, bool SWZ>
 __device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>& w, int t, int lane, bool valid,
                                              const uint4& q0, const uint4& q1, float* f) {
     bf16x8_to_f32(q0, f);
     bf16x8_to_f32(q1, f + 8);
+    if (XF == kXfSmooth && t == 0 && a.rope_cos && valid) {
+        // one row per tensor, fewer than 2^31 elements: the block's 16
+        // elements are 8 whole pairs of one head of one token (rope_d % 16 == 0)
+        const uint32_t i0 = (uint32_t)(w.cr * 512 + lane * 16);
+        const uint32_t tok = i0 / (uint32_t)a.rope_hd;
+        const uint32_t p0 = (i0 % (uint32_t)a.rope_d) >> 1;
+        const size_t off = (size_t)tok * (uint32_t)(a.rope_d >> 1) + p0;  // a multiple of 8 floats
+        const float4* pc = reinterpret_cast<const float4*>(a.rope_cos + off);
+        const float4* ps = reinterpret_cast<const float4*>(a.rope_sin + off);
+        const float4 c0 = __ldg(pc), c1 = __ldg(pc + 1), s0 = __ldg(ps), s1 = __ldg(ps + 1);
+        const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const float x0 = f[2 * k], x1 = f[2 * k + 1];
+            f[2 * k] = __fsub_rn(__fmul_rn(x0, c[k]), __fmul_rn(x1, sn[k]));
+            f[2 * k + 1] = __fadd_rn(__fmul_rn(x0, sn[k]), __fmul_rn(x1, c[k]));
+        }
+    }
     if (XF == kXfSmooth) {
         const float* mean = t ? a.smooth_mean[1] : a.smooth_mean[0];
         if (valid && mean) {
@@ -577,8 +607,18 @@ struct MeanArgs {
     float* mean[2];       // [hd], NULL: tensor not smoothed
     int T;
     int hd;               // H * d, a multiple of 16
+    // ROPE kernels: the keys (tensor 0) are turned first, as the quantize does
+    const float* rope_cos;  // [T][d / 2]
+    const float* rope_sin;
+    int d;
 };
 
+// the bf16 value at p as binary32
+__device__ __forceinline__ float ldg_bf16(const uint8_t* p) {
+    return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p)) << 16);
+}
+
+template <bool ROPE>
 __global__ void __launch_bounds__(1024) kv_channel_mean_kernel(MeanArgs a) {
     __shared__ float part[32][33];
     const int t = blockIdx.y;
@@ -588,7 +628,41 @@ __global__ void __launch_bounds__(1024) kv_channel_mean_kernel(MeanArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x * 32 + lane;
     float s0 = 0.0f;
-    if (c < a.hd) {
+    if (ROPE && t == 0) {
+        // each key is turned with its pair partner, the neighbouring lane's
+        // channel (channels 2p, 2p + 1 sit in lanes 2i, 2i + 1; hd is even, so
+        // both are in range or neither), by its token's angle.  Every lane
+        // loads (lanes past hd read channel 0 and their sums are dropped), so
+        // the exchanges are warp-wide; token loops are uniform per warp.
+        const int cc = c < a.hd ? c : 0;
+        const int hp = a.d >> 1;
+        const int pr = (cc % a.d) >> 1;
+        const bool odd = (lane & 1) != 0;
+        const int64_t stride = (int64_t)32 * a.hd * 2;
+        const uint8_t* p = x + ((int64_t)warp * a.hd + cc) * 2;
+        const float* pc = a.rope_cos + (int64_t)warp * hp + pr;
+        const float* ps = a.rope_sin + (int64_t)warp * hp + pr;
+        const int64_t tstride = (int64_t)32 * hp;
+        auto turn = [&](float xv, float cs, float sn) {
+            const float xp = __shfl_xor_sync(0xFFFFFFFFu, xv, 1);
+            return odd ? __fadd_rn(__fmul_rn(xp, sn), __fmul_rn(xv, cs))
+                       : __fsub_rn(__fmul_rn(xv, cs), __fmul_rn(xp, sn));
+        };
+        int tok = warp;
+        for (; tok + 7 * 32 < a.T; tok += 8 * 32, p += 8 * stride, pc += 8 * tstride, ps += 8 * tstride) {
+            float xv[8], cs[8], sn[8];
+#pragma unroll
+            for (int k = 0; k < 8; k++) {
+                xv[k] = ldg_bf16(p + k * stride);
+                cs[k] = __ldg(pc + k * tstride);
+                sn[k] = __ldg(ps + k * tstride);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; k++) s0 = __fadd_rn(s0, turn(xv[k], cs[k], sn[k]));
+        }
+        for (; tok < a.T; tok += 32, p += stride, pc += tstride, ps += tstride)
+            s0 = __fadd_rn(s0, turn(ldg_bf16(p), __ldg(pc), __ldg(ps)));
+    } else if (c < a.hd) {
         const uint8_t* p = x + ((int64_t)warp * a.hd + c) * 2;
         const int64_t stride = (int64_t)32 * a.hd * 2;
         // up to 24 tokens' loads in flight before their (in-order) adds
@@ -817,7 +891,8 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
                                   bool swizzled, bool search, void* workspace, cudaStream_t stream,
                                   const float2* ln_stats = nullptr, const void* mod_scale = nullptr,
                                   const void* mod_shift = nullptr, const float* const* smooth_mean = nullptr,
-                                  int smooth_hd = 0) {
+                                  int smooth_hd = 0, const float* rope_cos = nullptr, const float* rope_sin = nullptr,
+                                  int rope_d = 0) {
     QuantArgs a{};
     for (int t = 0; t < ntensors; t++) {
         a.x[t] = static_cast<const uint8_t*>(x[t]);
@@ -848,6 +923,12 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
         a.smooth_mean[1] = ntensors > 1 ? smooth_mean[1] : nullptr;
         a.smooth_hd = smooth_hd;
     }
+    if (rope_cos) {
+        a.rope_cos = rope_cos;
+        a.rope_sin = rope_sin;
+        a.rope_d = rope_d;
+        a.rope_hd = smooth_hd;
+    }
     const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), ((int64_t)a.runs_per_tensor * ntensors + kQWarps - 1) / kQWarps);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
@@ -863,7 +944,7 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     if (ln_stats)
         kern = swizzled ? (search ? quantize_fused_kernel<true, true, kXfLn> : quantize_fused_kernel<true, false, kXfLn>)
                         : (search ? quantize_fused_kernel<false, true, kXfLn> : quantize_fused_kernel<false, false, kXfLn>);
-    else if (smooth_mean)  // KV chunks only: row-major scales
+    else if (smooth_mean || rope_cos)  // KV chunks only: row-major scales
         kern = search ? quantize_fused_kernel<false, true, kXfSmooth> : quantize_fused_kernel<false, false, kXfSmooth>;
     else
         kern = swizzled ? (search ? quantize_fused_kernel<true, true, kXfNone> : quantize_fused_kernel<true, false, kXfNone>)
@@ -959,8 +1040,11 @@ static nvfp4_status check_cache(const nvfp4_kv_cache* c) {
     return NVFP4_OK;
 }
 
-extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
-                                        const void* v_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream) {
+// The chunk's append: channel means first where a tensor is smoothed (of
+// the turned keys where a RoPE table is given), then the fused quantize.
+static nvfp4_status kv_append_impl(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
+                                   const void* v_bf16, const float* rope_cos, const float* rope_sin,
+                                   void* workspace, size_t ws_bytes, cudaStream_t stream) {
     nvfp4_status st = check_cache(cache);
     if (st != NVFP4_OK) return st;
     if (slot < 0 || slot >= cache->n_slots) return NVFP4_ERR_INVALID_ARG;
@@ -970,6 +1054,13 @@ extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slo
     if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_KV_APPEND, rows, 0, cache->head_dim)) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(k_bf16) || !aligned16(v_bf16) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return NVFP4_ERR_MISALIGNED;
+    const bool rope = rope_cos != nullptr;
+    if (rope) {
+        // flat element and channel indexes are 32-bit in the kernels
+        if (e >= ((int64_t)1 << 31) || (int64_t)cache->heads * cache->head_dim >= ((int64_t)1 << 24))
+            return NVFP4_ERR_UNSUPPORTED;
+        if (!aligned16(rope_cos) || !aligned16(rope_sin)) return NVFP4_ERR_MISALIGNED;
+    }
     // The chunk is quantized as one flat row of T*H*d elements: with
     // row-major scales over rows of head_dim this is the same byte layout.
     const void* xs[2] = {k_bf16, v_bf16};
@@ -980,10 +1071,11 @@ extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slo
     float* gs[2] = {cache->k_global + slot, cache->v_global + slot};
     const bool search = (cache->flags & NVFP4_KV_SCALE_SEARCH) != 0;
     const bool sk = (cache->flags & NVFP4_KV_SMOOTH_K) != 0, sv = (cache->flags & NVFP4_KV_SMOOTH_V) != 0;
-    if (!sk && !sv)
-        return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, search, workspace, (cudaStream_t)stream);
-    // K-smoothing: the slot's channel means first, then the quantize of x - mean
     const int hd = cache->heads * cache->head_dim;
+    if (!sk && !sv)
+        return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, search, workspace, stream, nullptr, nullptr,
+                             nullptr, nullptr, hd, rope_cos, rope_sin, cache->head_dim);
+    // K-smoothing: the slot's channel means first, then the quantize of x - mean
     MeanArgs m{};
     m.x[0] = static_cast<const uint8_t*>(k_bf16);
     m.x[1] = static_cast<const uint8_t*>(v_bf16);
@@ -991,11 +1083,31 @@ extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slo
     m.mean[1] = sv ? cache->v_mean + (int64_t)slot * hd : nullptr;
     m.T = cache->tokens_per_slot;
     m.hd = hd;
-    kv_channel_mean_kernel<<<dim3((unsigned)((hd + 31) / 32), 2), 1024, 0, (cudaStream_t)stream>>>(m);
+    m.rope_cos = rope_cos;
+    m.rope_sin = rope_sin;
+    m.d = cache->head_dim;
+    const dim3 grid((unsigned)((hd + 31) / 32), 2);
+    if (rope && sk)
+        kv_channel_mean_kernel<true><<<grid, 1024, 0, stream>>>(m);
+    else
+        kv_channel_mean_kernel<false><<<grid, 1024, 0, stream>>>(m);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
     const float* means[2] = {m.mean[0], m.mean[1]};
-    return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, search, workspace, (cudaStream_t)stream, nullptr,
-                         nullptr, nullptr, means, hd);
+    return quantize_impl(2, xs, 1, e, e, cs, ss, gs, false, false, search, workspace, stream, nullptr, nullptr,
+                         nullptr, means, hd, rope_cos, rope_sin, cache->head_dim);
+}
+
+extern "C" nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
+                                        const void* v_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream) {
+    return kv_append_impl(cache, slot, k_bf16, v_bf16, nullptr, nullptr, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+extern "C" nvfp4_status nvfp4_kv_append_rope(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
+                                             const void* v_bf16, const float* rope_cos, const float* rope_sin,
+                                             void* workspace, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!rope_cos || !rope_sin) return NVFP4_ERR_INVALID_ARG;
+    return kv_append_impl(cache, slot, k_bf16, v_bf16, rope_cos, rope_sin, workspace, ws_bytes,
+                          (cudaStream_t)stream);
 }
 
 extern "C" nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n,

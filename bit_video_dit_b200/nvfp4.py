@@ -28,7 +28,7 @@ EXPORTS = ("nvfp4_status_string", "nvfp4_version", "nvfp4_codes_bytes", "nvfp4_s
            "nvfp4_workspace_bytes", "nvfp4_read_device_error", "nvfp4_quantize", "nvfp4_gemm",
            "nvfp4_kv_append", "nvfp4_kv_dequant", "nvfp4_test_encode", "nvfp4_quantize_noalloc",
            "nvfp4_ln_modulate_quantize", "nvfp4_quantize_2d", "nvfp4_quantize_t", "nvfp4_attention_chunks",
-           "nvfp4_kv_attention")
+           "nvfp4_kv_attention", "nvfp4_kv_append_rope")
 
 
 class NVFP4Error(RuntimeError):
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_gemm.restype = st
         L.nvfp4_kv_append.argtypes = [ctypes.POINTER(CKVCache), i32, vp, vp, vp, sz, vp]
         L.nvfp4_kv_append.restype = st
+        L.nvfp4_kv_append_rope.argtypes = [ctypes.POINTER(CKVCache), i32, vp, vp, vp, vp, vp, sz, vp]
+        L.nvfp4_kv_append_rope.restype = st
         L.nvfp4_kv_dequant.argtypes = [ctypes.POINTER(CKVCache), vp, i32, vp, vp, vp, sz, vp]
         L.nvfp4_kv_dequant.restype = st
         L.nvfp4_test_encode.argtypes = [vp, i64, vp, vp, vp]
@@ -359,16 +361,28 @@ class KVCache:
                    (self.k_codes, self.v_codes, self.k_scales, self.v_scales, self.k_global, self.v_global,
                     self.k_mean, self.v_mean) if t is not None)
 
-    def append(self, slot: int, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
-        """Quantize one chunk's K and V (bf16 [T, H, d], contiguous) into `slot` in place."""
+    def append(self, slot: int, k: torch.Tensor, v: torch.Tensor, stream=None, rope=None) -> None:
+        """Quantize one chunk's K and V (bf16 [T, H, d], contiguous) into `slot` in place.
+        rope = (cos, sin), device float32 [T, d/2] each: the keys' rotary embedding
+        (interleaved pairs) is applied ahead of their quantize (nvfp4_kv_append_rope)."""
         _require_cuda(k, v)
         for t in (k, v):
             if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.numel() != self.slot_elems:
                 raise ValueError("append takes contiguous bf16 [T, H, d] chunks")
         cc = self.c()
-        _check("nvfp4_kv_append", lib().nvfp4_kv_append(
-            ctypes.byref(cc), int(slot), k.data_ptr(), v.data_ptr(), self.ws_append.data_ptr(),
-            self.ws_append.numel(), _stream(stream)))
+        if rope is None:
+            _check("nvfp4_kv_append", lib().nvfp4_kv_append(
+                ctypes.byref(cc), int(slot), k.data_ptr(), v.data_ptr(), self.ws_append.data_ptr(),
+                self.ws_append.numel(), _stream(stream)))
+            return
+        cos, sin = rope
+        _require_cuda(cos, sin)
+        for t in (cos, sin):
+            if t.dtype != torch.float32 or not t.is_contiguous() or t.shape != (self.tokens, self.head_dim // 2):
+                raise ValueError("rope tables are contiguous float32 [T, d/2]")
+        _check("nvfp4_kv_append_rope", lib().nvfp4_kv_append_rope(
+            ctypes.byref(cc), int(slot), k.data_ptr(), v.data_ptr(), cos.data_ptr(), sin.data_ptr(),
+            self.ws_append.data_ptr(), self.ws_append.numel(), _stream(stream)))
 
     def dequant(self, slots: torch.Tensor, k_out: torch.Tensor | None = None, v_out: torch.Tensor | None = None,
                 stream=None):

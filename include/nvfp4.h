@@ -283,6 +283,23 @@ typedef struct {
 nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
                              const void* v_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 
+/* nvfp4_kv_append with the keys' rotary position embedding fused ahead of
+ * their quantize ([NEWS]: fused RoPE and the in-place KV update).  rope_cos,
+ * rope_sin: device binary32 [T][d/2], row t the token's cos / sin per pair,
+ * 16-byte aligned, read only.  In every head of token t, pair p (channels 2p
+ * and 2p+1, interleaved) becomes, with c = rope_cos[t][p], s = rope_sin[t][p]:
+ *   y[2p]   = fl32(fl32(x[2p] * c) - fl32(x[2p+1] * s))
+ *   y[2p+1] = fl32(fl32(x[2p] * s) + fl32(x[2p+1] * c))
+ * and the slot holds the quantize of y (binary32, never rounded to bf16):
+ * tensor scale from max |y|, and with NVFP4_KV_SMOOTH_K the channel means of y
+ * (the cache's dequant then returns the turned keys).  V is stored as by
+ * nvfp4_kv_append.  Angles (positions, 1D or 3D frequency bands) are the
+ * caller's.  Needs T*H*d < 2^31; NULL tables: NVFP4_ERR_INVALID_ARG.
+ * Same workspace and launches as nvfp4_kv_append. */
+nvfp4_status nvfp4_kv_append_rope(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
+                                  const void* v_bf16, const float* rope_cos, const float* rope_sin,
+                                  void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
+
 /* Gathers the n slots listed in slots_dev (device int32 [n], values in
  * [0, n_slots)) back to bf16: output i covers rows i*T*H .. of k_out / v_out
  * (bf16 [n][T][H][d]).  Each value is bf16_rne(fl32(fl32(e2m1 * s) * a32))

@@ -101,6 +101,13 @@ def test_host_side_argument_checks(L):
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32, 8)
     st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 16, None)
     assert st == nv.ERR_INVALID_ARG  # unknown flag
+    # the keys' RoPE tables: present, 16-byte aligned, and 32-bit flat indexes
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32)
+    rope = L.nvfp4_kv_append_rope
+    assert rope(ctypes.byref(kv), 0, fake, fake, None, fake, fake, 1 << 16, None) == nv.ERR_INVALID_ARG
+    assert rope(ctypes.byref(kv), 0, fake, fake, fake + 4, fake, fake, 1 << 16, None) == nv.ERR_MISALIGNED
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 1 << 20, 16, 128)
+    assert rope(ctypes.byref(kv), 0, fake, fake, fake, fake, fake, 1 << 30, None) == nv.ERR_UNSUPPORTED
     # training-side operands: shapes, outputs, signs and alignment are checked before any launch
     q2 = L.nvfp4_quantize_2d
     assert q2(fake, 96, 64, 64, fake, fake, fake, fake, fake, 0, fake, 256, None) == nv.ERR_UNSUPPORTED  # rows % 64
