@@ -251,6 +251,51 @@ def measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, rep
 RHT_SIGN = (1, -1, -1, 1, 1, 1, -1, 1, -1, -1, 1, -1, 1, 1, -1, -1)
 
 
+def measure_ffn(nv, cache, ring, k_out, v_out, reps: int) -> dict:
+    """ms per launch of the 8192-token FFN pair: quantize A [8192 x 3072], the up
+    projection 3072 -> 14336 with GELU and the NVFP4 requant of its output (output
+    scale from one calibration pass), and the down projection 14336 -> 3072 to bf16
+    on that NVFP4 output (721.6 GFLOP each)."""
+    dev = k_out.device
+    up, dn = syn.FFN_UP, syn.FFN_DOWN
+    a = torch.from_numpy(syn.activations_bf16(up.M, up.K, seed=5).view(np.int16)).to(dev).view(torch.bfloat16)
+    wu = torch.from_numpy(syn.normal_bf16((up.N, up.K), seed=6, std=0.02).view(np.int16)).to(dev).view(torch.bfloat16)
+    wd = torch.from_numpy(syn.normal_bf16((dn.N, dn.K), seed=7, std=0.02).view(np.int16)).to(dev).view(torch.bfloat16)
+    qu, qd = nv.quantize(wu), nv.quantize(wd)
+    del wu, wd
+    qa = nv.empty_nvfp4(up.M, up.K, dev)
+    ws_q = nv.workspace(nv.OP_QUANTIZE, up.M, 0, up.K, dev)
+    ws_u = nv.workspace(nv.OP_GEMM, up.M, up.N, up.K, dev)
+    ws_d = nv.workspace(nv.OP_GEMM, dn.M, dn.N, dn.K, dev)
+    nv.quantize(a, out=qa, ws=ws_q)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, out_amax=amax, ws=ws_u)  # calibration pass (bf16 output dropped)
+    h = nv.empty_nvfp4(up.M, up.N, dev)
+    h.global_scale.copy_(amax / 2688.0)
+    c = torch.empty((dn.M, dn.N), dtype=torch.bfloat16, device=dev)
+    nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, requant=h, bf16_out=False, ws=ws_u)
+    nv.gemm(h, qd, out=c, ws=ws_d)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            cache.dequant(ring, k_out, v_out)  # L2 flush between repetitions
+            ev[i][0].record()
+            nv.quantize(a, out=qa, ws=ws_q)
+            ev[i][1].record()
+            nv.gemm(qa, qu, act=nv.ACT_GELU_TANH, requant=h, bf16_out=False, ws=ws_u)
+            ev[i][2].record()
+            nv.gemm(h, qd, out=c, ws=ws_d)
+            ev[i][3].record()
+    g.replay()
+    torch.cuda.synchronize()
+    out = {k: float(np.median([e[j].elapsed_time(e[j + 1]) for e in ev]))
+           for j, k in enumerate(("quantize_ms", "up_ms", "down_ms"))}
+    del g
+    return out
+
+
 def measure_training(nv, a, w, cache, ring, k_out, v_out, reps: int) -> dict:
     """ms per launch pair of the training-side operands and the weight-gradient GEMM on
     the QKV shapes: 2D scaling of W [9216 x 3072] (both operands), the RHT transposed
@@ -444,6 +489,8 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     train = measure_training(nv, a, dev_bf16(w_host), cache, ring, k_out, v_out, reps=5)
     # attention reading the NVFP4 cache directly (one query chunk), beside the step
     attn = measure_attention(nv, cache, ring, k_out, v_out, reps=3)
+    # the 8192-token FFN pair (up with GELU + requant, down to bf16), beside the step
+    ffn = measure_ffn(nv, cache, ring, k_out, v_out, reps=5)
 
     total_ms = t_start.elapsed_time(t_end)
     comp = np.zeros(4)
@@ -581,6 +628,20 @@ def run_ours(args, rank: int, world: int) -> dict | None:
             "append_GB/s": round(append_bytes / (search["rope_append_ms"] * 1e-3) / 1e9, 1),
             "smooth_search_append_ms": round(search["rope_smooth_append_ms"], 4),
             "smooth_search_append_GB/s": round(append_bytes / (search["rope_smooth_append_ms"] * 1e-3) / 1e9, 1)},
+        "ffn_8192": {
+            "what": "the FFN pair at 8192 tokens, outside the step: quantize A [8192x3072], up 3072->14336 with GELU "
+                    "and the NVFP4 requant of its output (output scale from a calibration pass), down 14336->3072 to "
+                    "bf16 on that NVFP4 output; each 2*M*N*K = 721.6 GFLOP",
+            "quantize_ms": round(ffn["quantize_ms"], 4),
+            "up_ms": round(ffn["up_ms"], 4),
+            "up_TFLOP/s": round(2 * syn.FFN_UP.M * syn.FFN_UP.N * syn.FFN_UP.K / (ffn["up_ms"] * 1e-3) / 1e12, 1),
+            "up_frac_fp4_peak": round(2 * syn.FFN_UP.M * syn.FFN_UP.N * syn.FFN_UP.K / (ffn["up_ms"] * 1e-3) / 1e12
+                                      / fp4_peak, 4),
+            "down_ms": round(ffn["down_ms"], 4),
+            "down_TFLOP/s": round(2 * syn.FFN_DOWN.M * syn.FFN_DOWN.N * syn.FFN_DOWN.K / (ffn["down_ms"] * 1e-3)
+                                  / 1e12, 1),
+            "down_frac_fp4_peak": round(2 * syn.FFN_DOWN.M * syn.FFN_DOWN.N * syn.FFN_DOWN.K
+                                        / (ffn["down_ms"] * 1e-3) / 1e12 / fp4_peak, 4)},
         "training": {
             "what": "training-side NVFP4 on the QKV layer shapes, outside the step: 2D (16x16) scaling of W "
                     "[9216x3072] writing W and W^T operands; RHT + transposed 1D quantize of X [4096x3072] and "
