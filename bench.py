@@ -251,12 +251,12 @@ def measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, rep
 RHT_SIGN = (1, -1, -1, 1, 1, 1, -1, 1, -1, -1, 1, -1, 1, 1, -1, -1)
 
 
-def measure_ffn(nv, cache, ring, k_out, v_out, reps: int) -> dict:
+def measure_ffn(nv, flush, dev, reps: int) -> dict:
     """ms per launch of the 8192-token FFN pair: quantize A [8192 x 3072], the up
     projection 3072 -> 14336 with GELU and the NVFP4 requant of its output (output
     scale from one calibration pass), and the down projection 14336 -> 3072 to bf16
-    on that NVFP4 output (721.6 GFLOP each)."""
-    dev = k_out.device
+    on that NVFP4 output (721.6 GFLOP each).  `flush()` evicts L2 before each
+    repetition (it is captured into the timing graph)."""
     up, dn = syn.FFN_UP, syn.FFN_DOWN
     a = torch.from_numpy(syn.activations_bf16(up.M, up.K, seed=5).view(np.int16)).to(dev).view(torch.bfloat16)
     wu = torch.from_numpy(syn.normal_bf16((up.N, up.K), seed=6, std=0.02).view(np.int16)).to(dev).view(torch.bfloat16)
@@ -280,7 +280,7 @@ def measure_ffn(nv, cache, ring, k_out, v_out, reps: int) -> dict:
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(reps):
-            cache.dequant(ring, k_out, v_out)  # L2 flush between repetitions
+            flush()  # L2 flush between repetitions
             ev[i][0].record()
             nv.quantize(a, out=qa, ws=ws_q)
             ev[i][1].record()
@@ -490,7 +490,7 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     # attention reading the NVFP4 cache directly (one query chunk), beside the step
     attn = measure_attention(nv, cache, ring, k_out, v_out, reps=3)
     # the 8192-token FFN pair (up with GELU + requant, down to bf16), beside the step
-    ffn = measure_ffn(nv, cache, ring, k_out, v_out, reps=5)
+    ffn = measure_ffn(nv, lambda: cache.dequant(ring, k_out, v_out), k_out.device, reps=5)
 
     total_ms = t_start.elapsed_time(t_end)
     comp = np.zeros(4)
@@ -738,6 +738,9 @@ def main(argv=None) -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--direct", action="store_true",
                     help="launch each component on the stream instead of replaying it from a CUDA graph")
+    ap.add_argument("--ffn-only", action="store_true",
+                    help="time only the 8192-token FFN pair (under 1 GB on the device: the small case for "
+                         "profiling its GEMMs) and print its numbers")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -754,6 +757,15 @@ def main(argv=None) -> int:
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
     torch.cuda.set_device(local)
+    if args.ffn_only:
+        from bit_video_dit_b200 import build as nvbuild
+        from bit_video_dit_b200 import nvfp4 as nv
+        nvbuild.build()
+        flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # 256 MB > L2
+        ffn = measure_ffn(nv, lambda: flush_buf.fill_(1), flush_buf.device, reps=max(1, args.steps))
+        if rank == 0:
+            print(json.dumps({"ffn_8192": {k: round(v, 4) for k, v in ffn.items()}}), flush=True)
+        return 0
     if world > 1:
         import datetime
 
