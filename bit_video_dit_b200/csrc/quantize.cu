@@ -15,6 +15,12 @@
 //  * dequant-gather: a warp owns 512-element runs of a slot; lane i decodes
 //    elements 8i..8i+7 and 256+8i..256+8i+7 (4-byte code loads, 16-byte bf16
 //    stores, each warp-wide access contiguous), two runs in flight per lane.
+//  * value transforms ahead of the encode (template variants of the fused
+//    kernel): LayerNorm + adaLN modulate of activation rows; for a KV chunk the
+//    keys' rotary embedding (the article's fused RoPE; interleaved pairs turned
+//    by a per-token cos / sin table) and the K-smoothing mean subtraction, whose
+//    channel means come from a separate fixed-order kernel (of the turned keys
+//    when both apply).
 #include <algorithm>
 
 #include "common.cuh"
