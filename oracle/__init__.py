@@ -23,8 +23,10 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
-_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+# The planted-mistake tests point these at a modified copy of the C source (and
+# a library path of their own) in a child process; nothing else sets them.
+_SRC = os.environ.get("NVFP4_ORACLE_SRC") or os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB_PATH = os.environ.get("NVFP4_ORACLE_LIB") or os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 

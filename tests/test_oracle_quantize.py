@@ -179,3 +179,46 @@ def test_swizzle_is_a_bijection_with_zero_padding(rows, sc):
     assert np.count_nonzero(swz) == rows * sc  # padding bytes stay zero
     offs = {oracle.swizzle_offset(r, c, sc) for r in range(0, rows, 7) for c in range(sc)}
     assert len(offs) == len(range(0, rows, 7)) * sc
+
+
+def test_reciprocal_form_decides_a_midpoint():
+    """R5: the element is multiplied by the binary32 reciprocal of s * a32, not divided by it.  With a32 = 1
+    (given) and a block max of 0.17578125 the block scale is s = 0.029296875 (E4M3 1.875 * 2^-6) exactly, and
+    the element 0.0732421875 = 2.5 * s sits on the E2M1 midpoint between 2 and 3: divided by s it is 2.5 and
+    ties to 2 (code 4); times fl32(1 / s) it is 2.5000002 and rounds to 3 (code 5).  The expected codes come
+    from numpy binary32 arithmetic and ml_dtypes' E4M3 / E2M1 conversions (round to nearest even)."""
+    import ml_dtypes
+
+    xf = np.zeros((1, 16), np.float32)
+    xf[0, 0], xf[0, 1] = 0.17578125, 0.0732421875
+    codes, scales, _ = oracle.quantize(xf, alpha=np.float32(1.0))
+    r = np.array([np.float32(0.17578125) / np.float32(6.0)], np.float32)
+    s = r.astype(ml_dtypes.float8_e4m3fn).astype(np.float32)[0]
+    assert s == np.float32(0.029296875) and scales[0, 0] == r.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)[0]
+    inv = np.float32(1.0) / (s * np.float32(1.0))
+    want = (np.minimum(xf[0] * inv, np.float32(6.0)).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF).tolist()
+    q = _codes_unpacked(codes)[0].tolist()
+    assert q == want and q[1] == 5
+    # the division form would have given code 4 for that element
+    yd = np.array([xf[0, 1] / s], np.float32)
+    assert int(yd.astype(ml_dtypes.float4_e2m1fn).view(np.uint8)[0] & 0xF) == 4
+
+
+def test_dequant_rounds_to_binary32_then_to_bf16():
+    """R10: two roundings, binary32 then bf16.  With sixteen elements of 1.5, scale 1 and a32 = 0.66927087307
+    (binary32), the exact product 1.5 * a32 = 1.0039063096... rounds in binary32 to 1 + 2^-8, the midpoint
+    between the bf16 values 1 and 1 + 2^-7, which ties to 1 (bf16 0x3F80); one rounding of the exact product
+    would give 1 + 2^-7 (0x3F81).  The expected value is torch's binary32 -> bf16 conversion of numpy's
+    binary32 product."""
+    import torch
+
+    a32 = np.float32(0.6692708730697632)
+    codes = np.full((1, 8), 0x33, np.uint8)  # elements 1.5 (code 3) in both nibbles
+    scales = np.array([[0x38]], np.uint8)    # E4M3 0x38 = 1.0
+    got = oracle.dequant_bf16(codes, scales, a32)[0]
+    p32 = np.float32(1.5) * a32
+    want = torch.tensor([p32]).to(torch.bfloat16).view(torch.int16).item() & 0xFFFF
+    assert p32 == np.float32(1.0 + 2.0 ** -8) and want == 0x3F80
+    assert all(int(v) == want for v in got)
+    # the exact product lies above the midpoint, so a single rounding would go up
+    assert Fraction(3, 2) * Fraction(float(a32)) > Fraction(1) + Fraction(1, 256)
