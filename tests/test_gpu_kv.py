@@ -224,3 +224,26 @@ def test_smoothing_reduces_the_error_of_channel_biased_keys():
         got = ko[0].float().cpu()
         errs.append(float(((got - ref) ** 2).mean()))
     assert errs[1] * 3 < errs[0], errs
+
+
+def test_dequant_rounds_to_binary32_then_to_bf16():
+    """A slot of codes 1.5 with scale 1.0 and a32 = 0.66927087307 (binary32): 1.5 * a32 rounds in binary32 to
+    1 + 2^-8, the bf16 midpoint between 1 and 1 + 2^-7, which ties to 1 (0x3F80); a single rounding of the
+    exact product would give 0x3F81 (reading R10, two roundings)."""
+    require_gpu()
+    T, H, d = 4, 1, 16
+    a32 = np.float32(0.6692708730697632)
+    cache = nv.KVCache(1, T, H, d)
+    for t in (cache.k_codes, cache.v_codes):
+        t.fill_(0x33)
+    for t in (cache.k_scales, cache.v_scales):
+        t.fill_(0x38)
+    for t in (cache.k_global, cache.v_global):
+        t.fill_(float(a32))
+    ko, vo = cache.dequant(torch.tensor([0], dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    codes = np.full((T * H, d // 2), 0x33, np.uint8)
+    scales = np.full((T * H, d // 16), 0x38, np.uint8)
+    want = oracle.kv_dequant(codes, scales, a32, T, H, d)
+    assert np.all(want == 0x3F80)
+    assert np.array_equal(host_bits(ko)[0], want) and np.array_equal(host_bits(vo)[0], want)

@@ -100,3 +100,18 @@ def test_scale_search_given_scale_and_zero_tensor():
     x = syn.normal_bf16((128, 256), seed=5)
     _check(x, alpha=0.01, search=True)
     _check(np.zeros((64, 128), np.uint16), search=True)
+
+
+def test_rounding_boundary_blocks():
+    """The blocks the oracle pins on rounding boundaries (given a32 = 1), with and without the scale search: an
+    element on an E2M1 midpoint where the binary32 reciprocal of s * a32 and a division disagree (R5), sixteen
+    6.0 that both search targets represent exactly (a tie keeps the standard encoding, R18), and blocks exact
+    under one target only."""
+    xf = np.zeros((4, 64), np.float32)
+    xf[0, 0], xf[0, 1] = 0.17578125, 0.0732421875
+    xf[1, 0:16] = 6.0
+    xf[2, 0:16] = [4, 3, 2, 1.5, 1, 0.5, 0, -4, -3, -2, -1.5, -1, -0.5, 4, 2, 1]
+    xf[3, 0:16] = [6, 3, 1.5, 0.5, 0, -6, 2, 1, -0.5, 4, -3, 1.5, 0, 0, 6, -1]
+    x = syn.f32_to_bf16_bits(xf)
+    for search in (False, True):
+        _check(x, alpha=1.0, search=search)

@@ -186,6 +186,20 @@ ORACLE_MUTATIONS = {
     "R22 signs inverted": [("v[i] = sign[i] < 0 ? -v[i] : v[i];", "v[i] = sign[i] > 0 ? -v[i] : v[i];")],
     "R22 normalised by 1/2": [("for (int i = 0; i < 16; i++) v[i] = v[i] * 0.25f;",
                                "for (int i = 0; i < 16; i++) v[i] = v[i] * 0.5f;")],
+    "R1 tensor scale amax / 448": [
+        ("        a32 = amax / 2688.0f; /* R1 */\n        *alpha = a32;\n    } else {\n        a32 = *alpha;\n"
+         "    }\n    const int64_t nb = cols / 16;",
+         "        a32 = amax / 448.0f; /* R1 */\n        *alpha = a32;\n    } else {\n        a32 = *alpha;\n"
+         "    }\n    const int64_t nb = cols / 16;")],
+    "R8 nibbles swapped": [("(uint8_t)(q[2 * i] | (q[2 * i + 1] << 4)); /* R8 */",
+                            "(uint8_t)((q[2 * i] << 4) | q[2 * i + 1]); /* R8 */")],
+    "R11 GELU cube dropped to a square": [("0.044715 * y * y * y", "0.044715 * y * y")],
+    "R18 a tie takes the target-4 candidate": [
+        ("block_sq_error(xb, sc4, q4, a32) < block_sq_error(xb, sc, q, a32)",
+         "block_sq_error(xb, sc4, q4, a32) <= block_sq_error(xb, sc, q, a32)")],
+    "R21 2D block max over its first row only": [
+        ("            for (int i = 0; i < 16; i++)\n                for (int j = 0; j < 16; j++) {",
+         "            for (int i = 0; i < 1; i++)\n                for (int j = 0; j < 16; j++) {")],
 }
 
 

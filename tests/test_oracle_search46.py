@@ -57,6 +57,20 @@ def test_block_exact_under_target_6_keeps_it():
     assert np.array_equal(deq[0], x[0].astype(np.float64))
 
 
+def test_a_tie_keeps_the_standard_encoding():
+    """Sixteen 6.0 with a32 = 1 are exact under both targets: aimed at 6 the scale is 1.0 and every code
+    is 6; aimed at 4 the scale is 1.5 and every code is 4.  Both squared errors are 0, and a tie keeps the
+    standard encoding (scale E4M3 0x38 = 1.0, not 0x3C = 1.5)."""
+    x = _block([6.0] * 16)
+    c46, s46, _ = oracle.quantize(x, alpha=1.0, search46=True)
+    one = np.array([1.0], np.float32).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)[0]
+    assert s46[0, 0] == one == 0x38
+    deq, _ = _decode(c46, s46, 1.0)
+    assert np.array_equal(deq[0], x[0].astype(np.float64))
+    # the target-4 candidate is exact too: its scale 6 / 4 = 1.5 is an E4M3 value
+    assert np.array([1.5], np.float32).astype(ml_dtypes.float8_e4m3fn).astype(np.float32)[0] == 1.5
+
+
 def test_zero_tensor_and_flushed_blocks_unchanged():
     x = np.zeros((3, 64), np.float32)
     assert all(np.array_equal(a, b) for a, b in zip(oracle.quantize(x)[:2], oracle.quantize(x, search46=True)[:2]))
