@@ -17,7 +17,6 @@ transform cancel in the weight-gradient product.
 from fractions import Fraction
 
 import numpy as np
-import pytest
 import scipy.linalg
 
 import oracle

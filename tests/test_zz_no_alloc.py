@@ -7,7 +7,6 @@ on consecutive calls, since every call reuses the same static scratch.
 This file is named to be collected last, so a failure here comes after every
 other test has run.
 """
-import ctypes
 
 import numpy as np
 import pytest
