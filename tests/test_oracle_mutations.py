@@ -9,18 +9,23 @@ RoPE of the anzhuoshouzhuan.com LongLive 2.0 article, section "NVFP4 量化"), w
 the pins of test_oracle_rope.py restated against a library handle; and the rest of
 the oracle (the format and scaling rules R3-R10 of "LongLive-2.0：用 NVFP4 并行底座做
 长视频生成", section "NVFP4 量化格式", the GEMM and its epilogue, R19, R20, R22),
-each mutant run against every other oracle pin file in a child process."""
+each mutant run against every other oracle pin file in a child process; and the
+numpy attention and chunk-set functions (section 二's sink + window set), each
+mutant compiled from the function's source and patched in for the test."""
 import ctypes
+import inspect
 import os
 import shutil
 import subprocess
 import sys
+import textwrap
 
 import numpy as np
 import pytest
 
 import oracle
 
+from . import test_oracle_attention as _ta
 from .test_oracle_rope import U, _f32, _nonzero_chunk, _quarter_turned_bits, _turn
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "nvfp4_oracle.c")
@@ -229,3 +234,57 @@ def test_planted_mistake_in_the_oracle_fails_a_pin(gcc, tmp_path, name):
     # tests ran and at least one failed (exit status 1), or a pin's input crashed the
     # modified copy (killed by a signal); not a build, collection or usage error
     assert (rc == 1 and " failed" in out) or rc < 0, f"no pin caught: {name} (exit {rc})\n{out}"
+
+
+# ---------------------------------------------------------------------------
+# The attention part of the oracle is Python: a mutant is the function's source
+# with one mistake, compiled into the oracle module's namespace and patched in
+# for the duration of the test; the attention pins are then called directly.
+PY_MUTATIONS = {
+    "softmax over the queries": ("attention", "p /= p.sum(axis=1, keepdims=True)",
+                                 "p /= p.sum(axis=0, keepdims=True)"),
+    "scores without the scale": ("attention", "s = (qf[:, h, :] @ kf[:, h, :].T) * scale",
+                                 "s = (qf[:, h, :] @ kf[:, h, :].T)"),
+    "keys in place of values": ("attention", "out[:, h, :] = p @ vf[:, h, :]", "out[:, h, :] = p @ kf[:, h, :]"),
+    "window one chunk short": ("attention_chunks", "set(range(t - window, t))", "set(range(t - window + 1, t))"),
+    "the current chunk included": ("attention_chunks", "if 0 <= c < t)", "if 0 <= c <= t)"),
+    "shot sink from the first chunk": ("attention_chunks", "set(range(shot_start, shot_start + sink_shot))",
+                                       "set(range(0, sink_shot))"),
+}
+
+
+def _py_mutant(fn_name, old, new):
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, fn_name)))
+    assert src.count(old) == 1, old
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<planted {fn_name}>", "exec"), ns)
+    return ns[fn_name]
+
+
+def _attention_pins():
+    yield _ta.test_attention_matches_torch_sdpa_in_float64
+    yield _ta.test_equal_keys_average_the_values
+    yield _ta.test_a_dominant_key_selects_its_value
+    for args, want in _ta._golden():
+        yield lambda args=args, want=want: _ta.test_attention_chunks_hand_worked(args, want)
+
+
+def _failing_attention_pins():
+    failed = 0
+    for pin in _attention_pins():
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    return failed
+
+
+def test_attention_pins_pass_on_the_unchanged_functions():
+    assert _failing_attention_pins() == 0
+
+
+@pytest.mark.parametrize("name", list(PY_MUTATIONS))
+def test_planted_mistake_in_the_attention_oracle_fails_a_pin(monkeypatch, name):
+    fn_name, old, new = PY_MUTATIONS[name]
+    monkeypatch.setattr(oracle, fn_name, _py_mutant(fn_name, old, new))
+    assert _failing_attention_pins() > 0, f"no pin caught: {name}"
