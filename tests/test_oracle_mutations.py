@@ -202,6 +202,10 @@ ORACLE_MUTATIONS = {
     "R18 a tie takes the target-4 candidate": [
         ("block_sq_error(xb, sc4, q4, a32) < block_sq_error(xb, sc, q, a32)",
          "block_sq_error(xb, sc4, q4, a32) <= block_sq_error(xb, sc, q, a32)")],
+    "R19 sample variance (n - 1)": [("const float var = row_sum32(dr, cols) / n;",
+                                     "const float var = row_sum32(dr, cols) / (n - 1.0f);")],
+    "R21 transposed operand not transposed": [
+        ("(uint8_t)(q[2 * j][i] | (q[2 * j + 1][i] << 4));", "(uint8_t)(q[i][2 * j] | (q[i][2 * j + 1] << 4));")],
     "R21 2D block max over its first row only": [
         ("            for (int i = 0; i < 16; i++)\n                for (int j = 0; j < 16; j++) {",
          "            for (int i = 0; i < 1; i++)\n                for (int j = 0; j < 16; j++) {")],
