@@ -908,6 +908,9 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     }
     const int64_t upr = (cols + 511) / 512;
     if (rows * upr > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
+    // the kernel's byte offsets inside a row are 32-bit: at most 2^30 elements
+    // per row (a KV chunk is one row of T*H*d elements)
+    if (cols > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
     a.ld_bytes = ld * 2;
     a.code_ld = cols / 2;
     a.scale_ld = cols / 16;

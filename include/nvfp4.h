@@ -129,7 +129,8 @@ nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int
 #define NVFP4_Q_SCALE_SEARCH 4u
 
 /* x_bf16: bf16 [rows x cols], row stride ld elements (ld >= cols, ld % 8 == 0).
- * cols % 64 == 0, rows >= 0.
+ * cols % 64 == 0, rows >= 0; cols <= 2^30 and rows * ceil(cols / 512) <= 2^30,
+ * else NVFP4_ERR_UNSUPPORTED.
  * codes: nvfp4_codes_bytes(rows, cols) bytes, rows of cols/2 bytes.
  * scales: nvfp4_scales_bytes(rows, cols, swizzled) bytes (padding zeroed).
  * global_scale: device binary32, written (COMPUTE) or read (GIVEN).
@@ -279,7 +280,9 @@ typedef struct {
  * over the whole chunk, then the quantize rule above with row-major scales
  * (with the scale search when cache->flags has NVFP4_KV_SCALE_SEARCH).
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_KV_APPEND, T*H, 0, d) bytes.
- * One cooperative launch covering K and V (as nvfp4_quantize). */
+ * One cooperative launch covering K and V (as nvfp4_quantize), which takes
+ * the chunk as one row of T*H*d elements: T*H*d <= 2^30, else
+ * NVFP4_ERR_UNSUPPORTED (the dequant takes slots of up to 2^40 elements). */
 nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
                              const void* v_bf16, void* workspace, size_t ws_bytes, nvfp4_stream_t stream);
 

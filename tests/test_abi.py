@@ -101,6 +101,11 @@ def test_host_side_argument_checks(L):
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32, 8)
     st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 16, None)
     assert st == nv.ERR_INVALID_ARG  # unknown flag
+    # rows longer than 2^30 elements (a KV chunk is one row of T*H*d) are refused before any launch
+    st = L.nvfp4_quantize(fake, 1, (1 << 30) + 64, (1 << 30) + 64, fake, fake, fake, 0, fake, 1 << 16, None)
+    assert st == nv.ERR_UNSUPPORTED
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 1, (1 << 23) + 1, 1, 128)  # (2^23 + 1) * 128 > 2^30
+    assert L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 30, None) == nv.ERR_UNSUPPORTED
     # the keys' RoPE tables: present, 16-byte aligned, and 32-bit flat indexes
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32)
     rope = L.nvfp4_kv_append_rope
