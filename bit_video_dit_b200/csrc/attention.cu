@@ -497,6 +497,9 @@ extern "C" nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const in
     if (cache->flags & ~(NVFP4_KV_SCALE_SEARCH | NVFP4_KV_SMOOTH_K | NVFP4_KV_SMOOTH_V)) return NVFP4_ERR_INVALID_ARG;
     const bool sk = (cache->flags & NVFP4_KV_SMOOTH_K) != 0, sv = (cache->flags & NVFP4_KV_SMOOTH_V) != 0;
     if ((sk && !cache->k_mean) || (sv && !cache->v_mean)) return NVFP4_ERR_INVALID_ARG;
+    // the kernel counts key tiles over the whole list in 32 bits
+    if ((int64_t)n * ((cache->tokens_per_slot + kTile - 1) / kTile) >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED;
     if (tq == 0) return NVFP4_OK;
     if (!q_bf16 || !o_bf16 || (n > 0 && !slots_dev)) return NVFP4_ERR_INVALID_ARG;
     auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };

@@ -325,12 +325,16 @@ int32_t nvfp4_attention_chunks(int32_t t, int32_t sink_global, int32_t shot_star
 
 /* O = softmax(scale * Q K^T) V over every key of the n slots listed in
  * slots_dev (device int32, values in [0, n_slots)), reading K and V from the
- * cache: each key and value is the cache's bf16 dequant (with the smoothing
- * mean added for a smoothed tensor), no mask inside the set.  q_bf16 and
- * o_bf16 are bf16 [tq][heads][head_dim] (token-major like the cache's chunks);
- * scale = 0 means 1 / sqrt(head_dim).  head_dim must be 128.  Products on the
- * tensor cores in bf16 with binary32 accumulation, softmax in binary32 (two
- * passes over the keys), P rounded to bf16; one launch of
+ * cache directly, no mask inside the set.  For a cache without smoothing the
+ * keys and values are the exact e2m1 * s * a32 (tiles of e2m1 * s in binary16,
+ * the slot's a32 applied to the products); with K- or V-smoothing they are the
+ * cache's bf16 dequant with the means added (bf16 tiles).  q_bf16 and o_bf16
+ * are bf16 [tq][heads][head_dim] (token-major like the cache's chunks); scale
+ * = 0 means 1 / sqrt(head_dim).  head_dim must be 128, and n * ceil(T / 128)
+ * < 2^31 (else NVFP4_ERR_UNSUPPORTED).  Products on the tensor cores with
+ * binary32 accumulation, a one-pass softmax in binary32 whose reference
+ * maximum moves only when a tile exceeds it by more than 2^8 (O rescaled in
+ * TMEM then), P rounded to the tiles' 16-bit type; one launch of
  * ceil(tq / 128) x heads CTAs.  An out-of-range slot records NVFP4_ERR_DEVICE
  * (info = list position) and is skipped.  workspace:
  * nvfp4_workspace_bytes(NVFP4_OP_KV_ATTENTION, 0, 0, 0) bytes. */

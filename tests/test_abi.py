@@ -106,6 +106,10 @@ def test_host_side_argument_checks(L):
     assert st == nv.ERR_UNSUPPORTED
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 1, (1 << 23) + 1, 1, 128)  # (2^23 + 1) * 128 > 2^30
     assert L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 30, None) == nv.ERR_UNSUPPORTED
+    # attention: the key tiles of the whole list are counted in 32 bits
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 1, 1 << 18, 1, 128)  # 2048 tiles per slot
+    st = L.nvfp4_kv_attention(ctypes.byref(kv), fake, 1 << 20, fake, 128, ctypes.c_float(0.0), fake, fake, 256, None)
+    assert st == nv.ERR_UNSUPPORTED
     # the keys' RoPE tables: present, 16-byte aligned, and 32-bit flat indexes
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32)
     rope = L.nvfp4_kv_append_rope
