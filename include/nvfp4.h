@@ -156,7 +156,7 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * sums (partial j over the 16-element blocks j, j+32, ... in order) combined
  * by an xor butterfly over 16, 8, 4, 2, 1.  m is then quantized exactly as
  * nvfp4_quantize quantizes a tensor (flags as there), a32 from max |m|.
- * cols % 64 == 0; pointers 16-byte aligned.
+ * cols % 64 == 0, cols <= 2^24, rows <= 2^30; pointers 16-byte aligned.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_LN_QUANTIZE, rows, 0, cols)
  * bytes (the control block, then 8 bytes of row statistics per row).
  * Two launches: the row statistics, then the fused quantize. */
@@ -234,10 +234,11 @@ typedef struct {
 
 /* C[M x N] = a32_A * a32_B * (A_q . S_A)(B_q . S_B)^T, then the epilogue.
  * A: [M x K] activations, B: [N x K] weights (both K-major, K = A->cols =
- * B->cols, K % 64 == 0).  M, N >= 1, arbitrary (tails handled).
+ * B->cols, K % 64 == 0).  M, N >= 1, arbitrary (tails handled); M, N, K
+ * <= 2^30 (else NVFP4_ERR_UNSUPPORTED).
  * c_bf16: [M x N] with row stride ldc (ldc >= N, ldc % 8 == 0) or NULL when
  * ep->out_codes is set.  ep may be NULL (plain bf16 output).
- * Requant needs N % 16 == 0.
+ * Requant needs N % 64 == 0 (else NVFP4_ERR_UNSUPPORTED).
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM, M, N, K) bytes.
  * One persistent launch (tcgen05 block-scaled MMA, TMEM accumulators, TMA). */
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* c_bf16, int64_t ldc,
@@ -270,8 +271,9 @@ typedef struct {
  * butterfly 16, 8, 4, 2, 1, mean = S / T), stores it at *_mean[slot][c] and
  * quantizes fl32(x - mean[c]) (tensor scale from max |x - mean|); the dequant
  * returns bf16_rne(fl32(fl32(fl32(e2m1 * s) * a32) + mean[c])).  Needs
- * T*H*d < 2^31, T < 2^24 and the mean array 16-byte aligned; the append is then
- * two launches (the means, then the quantize). */
+ * T*H*d < 2^31 (the append, as any append, T*H*d <= 2^30), T < 2^24 and the
+ * mean array 16-byte aligned; the append is then two launches (the means, then
+ * the quantize). */
 #define NVFP4_KV_SMOOTH_K 2u
 #define NVFP4_KV_SMOOTH_V 4u
 
@@ -297,7 +299,8 @@ nvfp4_status nvfp4_kv_append(const nvfp4_kv_cache* cache, int32_t slot, const vo
  * tensor scale from max |y|, and with NVFP4_KV_SMOOTH_K the channel means of y
  * (the cache's dequant then returns the turned keys).  V is stored as by
  * nvfp4_kv_append.  Angles (positions, 1D or 3D frequency bands) are the
- * caller's.  Needs T*H*d < 2^31; NULL tables: NVFP4_ERR_INVALID_ARG.
+ * caller's.  T*H*d <= 2^30 as for nvfp4_kv_append; NULL tables:
+ * NVFP4_ERR_INVALID_ARG.
  * Same workspace and launches as nvfp4_kv_append. */
 nvfp4_status nvfp4_kv_append_rope(const nvfp4_kv_cache* cache, int32_t slot, const void* k_bf16,
                                   const void* v_bf16, const float* rope_cos, const float* rope_sin,
