@@ -349,7 +349,7 @@ nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const int32_t* slot
 /* Training-side operands  [RN-T] "NVFP4 训练的工程细节"                        */
 /* ------------------------------------------------------------------------ */
 /* 2D block scaling of a weight x (bf16 [rows x cols], row stride ld elements;
- * rows % 64 == 0, cols % 64 == 0): one E4M3 scale per 16 x 16 block,
+ * rows % 64 == 0, cols % 64 == 0, both <= 2^30): one E4M3 scale per 16 x 16 block,
  * s = E4M3_rne_sat(amax_block / (6 * a32)), every element encoded with it as
  * in nvfp4_quantize (a32 = amax / 2688 over the tensor, or given with
  * NVFP4_Q_GIVEN_GLOBAL).  Writes the GEMM operand of x (codes [rows x cols/2],
@@ -371,7 +371,7 @@ nvfp4_status nvfp4_quantize_2d(const void* x_bf16, int64_t rows, int64_t cols, i
  * in binary32 (signs, then butterflies h = 1, 2, 4, 8 with (a + b, a - b),
  * then * 0.25), and a32 comes from max |y|.  Use the same signs for both
  * operands of the product so the transform cancels.  rows % 64 == 0,
- * cols % 16 == 0.  Two launches; workspace:
+ * cols % 16 == 0, both <= 2^30.  Two launches; workspace:
  * nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_T, rows, 0, cols) bytes. */
 nvfp4_status nvfp4_quantize_t(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes_t,
                               void* scales_t, float* global_scale, const int8_t* rht_sign, unsigned flags,
