@@ -206,6 +206,10 @@ ORACLE_MUTATIONS = {
                                      "const float var = row_sum32(dr, cols) / (n - 1.0f);")],
     "R21 transposed operand not transposed": [
         ("(uint8_t)(q[2 * j][i] | (q[2 * j + 1][i] << 4));", "(uint8_t)(q[i][2 * j] | (q[i][2 * j + 1] << 4));")],
+    "R20 mean subtracted again in the dequant": [("float y = v + mean[(r % H) * d + c];",
+                                                  "float y = v - mean[(r % H) * d + c];")],
+    "R20 mean indexed by token instead of head": [("float y = v + mean[(r % H) * d + c];",
+                                                   "float y = v + mean[(r / H % H) * d + c];")],
     "R21 2D block max over its first row only": [
         ("            for (int i = 0; i < 16; i++)\n                for (int j = 0; j < 16; j++) {",
          "            for (int i = 0; i < 1; i++)\n                for (int j = 0; j < 16; j++) {")],
