@@ -96,16 +96,20 @@ def lib():
             L.orc_gemm_exact_bf16.restype = ctypes.c_int
             L.orc_kv_slot_bytes.argtypes = [i64, i64, i64]
             L.orc_kv_slot_bytes.restype = i64
+            L.orc_ln_stats.argtypes = [vp, i64, i64, i64, f32, vp]
+            L.orc_ln_stats.restype = ctypes.c_int
+            L.orc_ln_modulate_given.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
+            L.orc_ln_modulate_given.restype = ctypes.c_int
             L.orc_ln_modulate.argtypes = [vp, i64, i64, i64, vp, vp, f32, vp]
             L.orc_ln_modulate.restype = ctypes.c_int
-            L.orc_ln_modulate_quantize.argtypes = [vp, i64, i64, i64, vp, vp, f32, ctypes.c_int, vp, vp, vp]
+            L.orc_ln_modulate_quantize.argtypes = [vp, i64, i64, i64, vp, vp, f32, vp, ctypes.c_int, vp, vp, vp]
             L.orc_ln_modulate_quantize.restype = ctypes.c_int
             for name in ("orc_kv_append", "orc_kv_append_search46"):
                 getattr(L, name).argtypes = [vp, i64, i64, i64, i64, vp, vp, vp]
                 getattr(L, name).restype = ctypes.c_int
             L.orc_kv_dequant.argtypes = [vp, vp, f32, i64, i64, i64, vp]
             L.orc_channel_mean.argtypes = [vp, i64, i64, vp]
-            L.orc_kv_append_smooth.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp]
+            L.orc_kv_append_smooth.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp, ctypes.c_int]
             L.orc_kv_append_smooth.restype = ctypes.c_int
             L.orc_kv_dequant_smooth.argtypes = [vp, vp, f32, vp, i64, i64, i64, vp]
             for name in ("orc_quantize_2d_f32", "orc_quantize_2d_bf16"):
@@ -114,7 +118,7 @@ def lib():
             L.orc_rht16_f32.argtypes = [vp, i64, vp, vp]
             L.orc_rope.argtypes = [vp, i64, i64, i64, vp, vp, vp]
             L.orc_channel_mean_f32.argtypes = [vp, i64, i64, vp]
-            L.orc_kv_append_rope.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, vp, vp]
+            L.orc_kv_append_rope.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, vp, vp, ctypes.c_int]
             L.orc_kv_append_rope.restype = ctypes.c_int
             L.orc_quantize_t_bf16.argtypes = [vp, i64, i64, i64, vp, ctypes.c_int, vp, vp, vp]
             L.orc_quantize_t_bf16.restype = ctypes.c_int
@@ -316,7 +320,7 @@ def kv_dequant(codes, scales, alpha, T: int, H: int, d: int) -> np.ndarray:
 
 def channel_mean(x: np.ndarray) -> np.ndarray:
     """Binary32 mean over the first axis of bf16 bits x [T, C...] for every
-    channel, in R20's fixed order (32 strided partial sums, butterfly)."""
+    channel (R20: the binary64 mean rounded once)."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     T = x.shape[0]
     C = x.size // T
@@ -325,17 +329,20 @@ def channel_mean(x: np.ndarray) -> np.ndarray:
     return mean
 
 
-def kv_append_smooth(x: np.ndarray, search46: bool = False):
+def kv_append_smooth(x: np.ndarray, search46: bool = False, mean=None):
     """K-smoothing append (R20): x bf16 bits [T, H, d].  Returns (codes, scales,
-    alpha, mean [H*d]); the quantized values are fl32(x - mean[channel])."""
+    alpha, mean [H*d]); the quantized values are fl32(x - mean[channel]).  With
+    `mean` given (binary32 [H*d], e.g. the means a kernel stored) those are
+    used instead of the oracle's own."""
     T, H, d = x.shape
     x = np.ascontiguousarray(x, dtype=np.uint16)
     codes = np.zeros((T * H, d // 2), np.uint8)
     scales = np.zeros((T * H, d // 16), np.uint8)
     a = np.zeros(1, np.float32)
-    mean = np.zeros(H * d, np.float32)
+    given = mean is not None
+    mean = np.array(mean, np.float32).reshape(H * d) if given else np.zeros(H * d, np.float32)
     rc = lib().orc_kv_append_smooth(_p(x), T, H, d, MODE_SEARCH46 if search46 else 0, _p(codes), _p(scales),
-                                    _p(a), _p(mean))
+                                    _p(a), _p(mean), 1 if given else 0)
     if rc != 0:
         raise ValueError(f"orc_kv_append_smooth failed ({rc})")
     return codes, scales, np.float32(a[0]), mean
@@ -370,7 +377,7 @@ def rope(x: np.ndarray, cos, sin) -> np.ndarray:
 
 
 def channel_mean_f32(v: np.ndarray) -> np.ndarray:
-    """R20's channel mean of binary32 values v [T, C...] (same order as channel_mean)."""
+    """R20's channel mean of binary32 values v [T, C...] (the binary64 mean rounded once)."""
     v = np.ascontiguousarray(v, dtype=np.float32)
     T = v.shape[0]
     C = v.size // T
@@ -379,9 +386,10 @@ def channel_mean_f32(v: np.ndarray) -> np.ndarray:
     return mean
 
 
-def kv_append_rope(x: np.ndarray, cos, sin, smooth: bool = False, search46: bool = False):
+def kv_append_rope(x: np.ndarray, cos, sin, smooth: bool = False, search46: bool = False, mean=None):
     """The keys' append with R24 (x bf16 bits [T, H, d]): rope, then (smooth) the
-    channel means of the rotated keys taken out (R20), then the quantize.
+    channel means of the rotated keys taken out (R20; the given binary32 [H*d]
+    `mean` instead of the oracle's own when passed), then the quantize.
     Returns (codes, scales, alpha, mean [H*d] or None)."""
     T, H, d = x.shape
     x = np.ascontiguousarray(x, dtype=np.uint16)
@@ -389,9 +397,13 @@ def kv_append_rope(x: np.ndarray, cos, sin, smooth: bool = False, search46: bool
     codes = np.zeros((T * H, d // 2), np.uint8)
     scales = np.zeros((T * H, d // 16), np.uint8)
     a = np.zeros(1, np.float32)
-    mean = np.zeros(H * d, np.float32) if smooth else None
+    given = smooth and mean is not None
+    if smooth:
+        mean = np.array(mean, np.float32).reshape(H * d) if given else np.zeros(H * d, np.float32)
+    else:
+        mean = None
     rc = lib().orc_kv_append_rope(_p(x), T, H, d, _p(cs), _p(sn), MODE_SEARCH46 if search46 else 0, _p(codes),
-                                  _p(scales), _p(a), _p(mean))
+                                  _p(scales), _p(a), _p(mean), 1 if given else 0)
     if rc != 0:
         raise ValueError(f"orc_kv_append_rope failed ({rc})")
     return codes, scales, np.float32(a[0]), mean
@@ -481,22 +493,46 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.n
     return out
 
 
-def ln_modulate(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6) -> np.ndarray:
+def ln_stats(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """R19's row statistics of bf16 bits x [R, C]: binary32 [R, 2] holding
+    (mean, rstd) = (fl32(mu), fl32(1 / sqrt(var + eps))), mu and var taken in
+    binary64 (population variance)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    R, C = x.shape
+    st = np.zeros((R, 2), np.float32)
+    rc = lib().orc_ln_stats(_p(x), R, C, C, float(eps), _p(st))
+    if rc != 0:
+        raise ValueError(f"orc_ln_stats failed ({rc})")
+    return st
+
+
+def _ln_vecs(scale, shift):
+    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.uint16)
+    sh = None if shift is None else np.ascontiguousarray(shift, dtype=np.uint16)
+    return sc, sh
+
+
+def ln_modulate(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6, stats=None) -> np.ndarray:
     """LayerNorm of each row of bf16 bits x [R, C] (no affine), then
-    m = h * (1 + scale) + shift (bf16 bits [C] or None), binary32 (R19)."""
+    m = h * (1 + scale) + shift (bf16 bits [C] or None), binary32 (R19).  With
+    `stats` (binary32 [R, 2] of (mean, rstd), e.g. a kernel's) those row
+    statistics are used instead of ln_stats'."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     R, C = x.shape
     m = np.zeros((R, C), np.float32)
-    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.uint16)
-    sh = None if shift is None else np.ascontiguousarray(shift, dtype=np.uint16)
-    rc = lib().orc_ln_modulate(_p(x), R, C, C, None if sc is None else _p(sc), None if sh is None else _p(sh),
-                               float(eps), _p(m))
+    sc, sh = _ln_vecs(scale, shift)
+    if stats is None:
+        rc = lib().orc_ln_modulate(_p(x), R, C, C, _p(sc), _p(sh), float(eps), _p(m))
+    else:
+        st = np.ascontiguousarray(stats, dtype=np.float32).reshape(R, 2)
+        rc = lib().orc_ln_modulate_given(_p(x), R, C, C, _p(st), _p(sc), _p(sh), _p(m))
     if rc != 0:
         raise ValueError(f"orc_ln_modulate failed ({rc})")
     return m
 
 
-def ln_modulate_quantize(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6, alpha: float | None = None):
+def ln_modulate_quantize(x: np.ndarray, scale=None, shift=None, eps: float = 1e-6, alpha: float | None = None,
+                         stats=None):
     """ln_modulate then quantize (R19, R1..R8).  Returns (codes, logical scales, alpha)."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     R, C = x.shape
@@ -507,10 +543,9 @@ def ln_modulate_quantize(x: np.ndarray, scale=None, shift=None, eps: float = 1e-
     if alpha is not None:
         a[0] = np.float32(alpha)
         mode = MODE_GIVEN
-    sc = None if scale is None else np.ascontiguousarray(scale, dtype=np.uint16)
-    sh = None if shift is None else np.ascontiguousarray(shift, dtype=np.uint16)
-    rc = lib().orc_ln_modulate_quantize(_p(x), R, C, C, None if sc is None else _p(sc),
-                                        None if sh is None else _p(sh), float(eps), mode, _p(a), _p(codes),
+    sc, sh = _ln_vecs(scale, shift)
+    st = None if stats is None else np.ascontiguousarray(stats, dtype=np.float32).reshape(R, 2)
+    rc = lib().orc_ln_modulate_quantize(_p(x), R, C, C, _p(sc), _p(sh), float(eps), _p(st), mode, _p(a), _p(codes),
                                         _p(scales))
     if rc != 0:
         raise ValueError(f"orc_ln_modulate_quantize failed ({rc})")

@@ -46,13 +46,15 @@
  *      order: d = fl32(fl32(e2m1 * s) * a32) (R10's dequant product),
  *      e = fl32(x - d), sum = fl32(sum + fl32(e * e)) over elements 0..15.
  *      The tensor scale stays R1's.
- *  R19 LayerNorm + adaLN modulate before the quantize (optional path): see
- *      orc_ln_modulate for the operations, their binary32 order and eps.
+ *  R19 LayerNorm + adaLN modulate before the quantize (optional path): row
+ *      statistics by their definition (binary64, rounded once to binary32),
+ *      then the modulation in binary32 steps; see orc_ln_stats.
  *  R16 KV slot = NVFP4 matrix of T*H rows x d columns, blocks along d, scales
  *      row-major (not swizzled).
  *  R20 K-smoothing of a KV chunk (optional, per tensor): subtract each
- *      channel's mean over the chunk's tokens before the quantize and add it
- *      back in the dequant; see orc_channel_mean for the order.
+ *      channel's mean over the chunk's tokens (binary64, rounded once to
+ *      binary32) before the quantize and add it back in the dequant; see
+ *      orc_channel_mean.
  *  R21 2D block scaling of weights [RN-T]: one E4M3 scale per 16 x 16 block
  *      from the block's amax; see orc_quantize_2d_f32.
  *  R22 Random Hadamard Transform ahead of the weight-gradient quantize
@@ -564,75 +566,80 @@ ORC_API void orc_kv_dequant(const uint8_t* codes, const uint8_t* scales, float a
 /* ------------------------------------------------------------------------ */
 /* LayerNorm + adaLN modulate + quantize (the step before the linear layer)  */
 /* ------------------------------------------------------------------------ */
-/* R19: per row r of x (bf16 [rows x cols], cols % 16 == 0), in binary32:
- *   mean = S1 / cols, var = S2 / cols with S1 = sum x, S2 = sum fl32(x - mean)^2,
- *   rstd = 1 / sqrt(var + eps)  (each operation correctly rounded),
- *   m = fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale[c])) + shift[c]
+/* R19: per row r of x (bf16 [rows x cols], cols % 16 == 0), LayerNorm without
+ * affine parameters, population variance, eps inside the square root:
+ *   mu = (1/cols) sum_c x[c],  var = (1/cols) sum_c (x[c] - mu)^2,
+ *   mean = fl32(mu),  rstd = fl32(1 / sqrt(var + eps)),
+ * the sums, mu, var and the root taken in binary64 and each statistic rounded
+ * once to binary32 (the definition, with no summation order of its own: a
+ * binary64 sum of bf16 values is exact unless the row spans more than ~2^40 in
+ * magnitude, and otherwise off by far less than a binary32 unit).  Then, with
+ * (mean, rstd) as binary32 inputs, every element in binary32:
+ *   m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale[c])) + shift[c])
  *   (scale, shift bf16 [cols] or absent: 0),
- * then m is quantized as a binary32 tensor (R1..R8).  Sums run in a fixed
- * order: 32 partial sums, partial j over the 16-element blocks j, j+32,
- * j+64, ... of the row (blocks and their elements in order), then combined
- * by a butterfly: for o = 16, 8, 4, 2, 1, partial[j] = partial[j] +
- * partial[j ^ o] (all j at once). */
-static float butterfly32(float* part)
+ * and m is quantized as a binary32 tensor (R1..R8).  The statistics are an
+ * input of the second part (orc_ln_modulate_given), so a kernel whose binary32
+ * reductions land on slightly different statistics can be checked twice: its
+ * statistics against orc_ln_stats within a summation bound, and its codes bit
+ * for bit against the quantize of m built from its own statistics. */
+ORC_API int orc_ln_stats(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, float eps, float* stats)
 {
-    float next[32];
-    for (int o = 16; o > 0; o >>= 1) {
-        for (int j = 0; j < 32; j++) next[j] = part[j] + part[j ^ o];
-        memcpy(part, next, 32 * sizeof(float));
+    if (cols <= 0 || ld < cols) return 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t r = 0; r < rows; r++) {
+        double s1 = 0.0;
+        for (int64_t c = 0; c < cols; c++) s1 += (double)orc_bf16_to_f32(x[r * ld + c]);
+        const double mu = s1 / (double)cols;
+        double s2 = 0.0;
+        for (int64_t c = 0; c < cols; c++) {
+            const double d = (double)orc_bf16_to_f32(x[r * ld + c]) - mu;
+            s2 += d * d;
+        }
+        const double var = s2 / (double)cols;
+        stats[2 * r] = (float)mu;
+        stats[2 * r + 1] = (float)(1.0 / sqrt(var + (double)eps));
     }
-    return part[0];
+    return 0;
 }
 
-static float row_sum32(const float* v, int64_t cols)
+ORC_API int orc_ln_modulate_given(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, const float* stats,
+                                  const uint16_t* scale, const uint16_t* shift, float* m)
 {
-    float part[32];
-    const int64_t nb = cols / 16;
-    for (int j = 0; j < 32; j++) {
-        float s = 0.0f;
-        for (int64_t b = j; b < nb; b += 32)
-            for (int i = 0; i < 16; i++) s = s + v[b * 16 + i];
-        part[j] = s;
+    if (cols % 16 != 0 || ld < cols) return 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads())
+    for (int64_t r = 0; r < rows; r++) {
+        const float mean = stats[2 * r], rstd = stats[2 * r + 1];
+        for (int64_t c = 0; c < cols; c++) {
+            float h = (orc_bf16_to_f32(x[r * ld + c]) - mean) * rstd;
+            float g = 1.0f + (scale ? orc_bf16_to_f32(scale[c]) : 0.0f);
+            float t = h * g;
+            m[r * cols + c] = t + (shift ? orc_bf16_to_f32(shift[c]) : 0.0f);
+        }
     }
-    return butterfly32(part);
+    return 0;
 }
 
 ORC_API int orc_ln_modulate(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, const uint16_t* scale,
                             const uint16_t* shift, float eps, float* m)
 {
     if (cols % 16 != 0 || ld < cols) return 1;
-#pragma omp parallel for schedule(static) num_threads(nthreads())
-    for (int64_t r = 0; r < rows; r++) {
-        float* xr = (float*)malloc((size_t)cols * sizeof(float));
-        float* dr = (float*)malloc((size_t)cols * sizeof(float));
-        for (int64_t c = 0; c < cols; c++) xr[c] = orc_bf16_to_f32(x[r * ld + c]);
-        const float n = (float)cols;
-        const float mean = row_sum32(xr, cols) / n;
-        for (int64_t c = 0; c < cols; c++) {
-            float d = xr[c] - mean;
-            dr[c] = d * d;
-        }
-        const float var = row_sum32(dr, cols) / n;
-        const float rstd = 1.0f / sqrtf(var + eps);
-        for (int64_t c = 0; c < cols; c++) {
-            float h = (xr[c] - mean) * rstd;
-            float g = 1.0f + (scale ? orc_bf16_to_f32(scale[c]) : 0.0f);
-            float t = h * g;
-            m[r * cols + c] = t + (shift ? orc_bf16_to_f32(shift[c]) : 0.0f);
-        }
-        free(xr);
-        free(dr);
-    }
-    return 0;
+    float* st = (float*)malloc((size_t)(rows > 0 ? rows : 1) * 2 * sizeof(float));
+    if (!st) return 2;
+    int rc = orc_ln_stats(x, rows, cols, ld, eps, st);
+    if (rc == 0) rc = orc_ln_modulate_given(x, rows, cols, ld, st, scale, shift, m);
+    free(st);
+    return rc;
 }
 
+/* stats: binary32 (mean, rstd) per row to use, or NULL for orc_ln_stats' */
 ORC_API int orc_ln_modulate_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
-                                     const uint16_t* scale, const uint16_t* shift, float eps, int mode, float* alpha,
-                                     uint8_t* codes, uint8_t* scales)
+                                     const uint16_t* scale, const uint16_t* shift, float eps, const float* stats,
+                                     int mode, float* alpha, uint8_t* codes, uint8_t* scales)
 {
     float* m = (float*)malloc((size_t)(rows * cols) * sizeof(float) + 1);
     if (!m) return 2;
-    int rc = orc_ln_modulate(x, rows, cols, ld, scale, shift, eps, m);
+    int rc = stats ? orc_ln_modulate_given(x, rows, cols, ld, stats, scale, shift, m)
+                   : orc_ln_modulate(x, rows, cols, ld, scale, shift, eps, m);
     if (rc == 0) rc = orc_quantize_f32(m, rows, cols, cols, mode, alpha, codes, scales);
     free(m);
     return rc;
@@ -642,34 +649,31 @@ ORC_API int orc_ln_modulate_quantize(const uint16_t* x, int64_t rows, int64_t co
 /* KV K-smoothing [RN-I] (R20): per chunk and tensor, each channel's mean     */
 /* over the tokens is taken out before the quantize and put back at dequant  */
 /* ------------------------------------------------------------------------ */
-/* x: bf16 [T][C] (C = H*d channels, token t at x + t*C).  mean[c] in
- * binary32, fixed order: 32 partial sums, partial p over the tokens p, p+32,
- * p+64, ... in increasing order (starting from +0), combined by the same
- * butterfly as R19 (o = 16, 8, 4, 2, 1: part[p] = part[p] + part[p ^ o]);
- * mean = fl32(S / T). */
+/* x: bf16 [T][C] (C = H*d channels, token t at x + t*C).  R20:
+ * mean[c] = fl32((1/T) sum_t x[t][c]), the sum and the quotient in binary64
+ * and rounded once to binary32 (the definition; a binary64 sum of bf16 values
+ * is exact for any chunk of realistic range). */
 ORC_API void orc_channel_mean(const uint16_t* x, int64_t T, int64_t C, float* mean)
 {
 #pragma omp parallel for schedule(static) num_threads(nthreads())
     for (int64_t c = 0; c < C; c++) {
-        float part[32];
-        for (int p = 0; p < 32; p++) {
-            float s = 0.0f;
-            for (int64_t t = p; t < T; t += 32) s = s + orc_bf16_to_f32(x[t * C + c]);
-            part[p] = s;
-        }
-        mean[c] = butterfly32(part) / (float)T;
+        double s = 0.0;
+        for (int64_t t = 0; t < T; t++) s += (double)orc_bf16_to_f32(x[t * C + c]);
+        mean[c] = (float)(s / (double)T);
     }
 }
 
-/* x: bf16 chunk [T][H][d] (contiguous).  Writes mean [H*d] (orc_channel_mean),
- * then quantizes v = fl32(x - mean[h*d + j]) as orc_kv_append does (R15, R16;
- * mode may carry ORC_MODE_SEARCH46). */
+/* x: bf16 chunk [T][H][d] (contiguous).  mean [H*d]: with mean_given == 0
+ * written here (orc_channel_mean), else read as given (the means a kernel
+ * stored, so its codes can be checked bit for bit against them); then
+ * quantizes v = fl32(x - mean[h*d + j]) as orc_kv_append does (R15, R16; mode
+ * may carry ORC_MODE_SEARCH46). */
 ORC_API int orc_kv_append_smooth(const uint16_t* x, int64_t T, int64_t H, int64_t d, int mode, uint8_t* codes,
-                                 uint8_t* scales, float* alpha, float* mean)
+                                 uint8_t* scales, float* alpha, float* mean, int mean_given)
 {
     const int64_t C = H * d;
     if (d % 16 != 0) return 1;
-    orc_channel_mean(x, T, C, mean);
+    if (!mean_given) orc_channel_mean(x, T, C, mean);
     float* v = (float*)malloc((size_t)(T * C) * sizeof(float) + 1);
     if (!v) return 2;
     for (int64_t t = 0; t < T; t++)
@@ -722,29 +726,26 @@ ORC_API void orc_rope(const uint16_t* x, int64_t T, int64_t H, int64_t d, const 
         }
 }
 
-/* R20's channel mean of binary32 values v [T][C], same order as
- * orc_channel_mean. */
+/* R20's channel mean of binary32 values v [T][C]: fl32 of the binary64
+ * mean, as orc_channel_mean. */
 ORC_API void orc_channel_mean_f32(const float* v, int64_t T, int64_t C, float* mean)
 {
 #pragma omp parallel for schedule(static) num_threads(nthreads())
     for (int64_t c = 0; c < C; c++) {
-        float part[32];
-        for (int p = 0; p < 32; p++) {
-            float s = 0.0f;
-            for (int64_t t = p; t < T; t += 32) s = s + v[t * C + c];
-            part[p] = s;
-        }
-        mean[c] = butterfly32(part) / (float)T;
+        double s = 0.0;
+        for (int64_t t = 0; t < T; t++) s += (double)v[t * C + c];
+        mean[c] = (float)(s / (double)T);
     }
 }
 
 /* The keys' append with R24: y = orc_rope(x); with K-smoothing (mean != NULL)
- * the channel means of y (R20's order) and the quantize of fl32(y - mean),
- * else the quantize of y; a32 from the quantized values (R1), blocks and
- * layout as orc_kv_append (R15, R16; mode may carry ORC_MODE_SEARCH46). */
+ * the channel means of y (R20; computed here, or read as given when
+ * mean_given != 0) and the quantize of fl32(y - mean), else the quantize of
+ * y; a32 from the quantized values (R1), blocks and layout as orc_kv_append
+ * (R15, R16; mode may carry ORC_MODE_SEARCH46). */
 ORC_API int orc_kv_append_rope(const uint16_t* x, int64_t T, int64_t H, int64_t d, const float* cs,
                                const float* sn, int mode, uint8_t* codes, uint8_t* scales, float* alpha,
-                               float* mean)
+                               float* mean, int mean_given)
 {
     const int64_t C = H * d;
     if (d % 16 != 0) return 1;
@@ -752,7 +753,7 @@ ORC_API int orc_kv_append_rope(const uint16_t* x, int64_t T, int64_t H, int64_t 
     if (!y) return 2;
     orc_rope(x, T, H, d, cs, sn, y);
     if (mean) {
-        orc_channel_mean_f32(y, T, C, mean);
+        if (!mean_given) orc_channel_mean_f32(y, T, C, mean);
         for (int64_t t = 0; t < T; t++)
             for (int64_t c = 0; c < C; c++) y[t * C + c] = y[t * C + c] - mean[c];
     }

@@ -36,7 +36,10 @@ def _case(T, H, Tq, slot_chunks, n_slots, seed, smooth_k=False, smooth_v=False, 
         cache.append(s, dev_bf16(k), dev_bf16(v))
         for name, x, sm, store in (("k", k, smooth_k, kh), ("v", v, smooth_v, vh)):
             if sm:
-                c, sc, a, m = oracle.kv_append_smooth(x)
+                # the codes follow the kernel's stored means (checked against the oracle's
+                # within their summation bound in the KV tests)
+                km = (cache.k_mean if name == "k" else cache.v_mean)[s].cpu().numpy()
+                c, sc, a, m = oracle.kv_append_smooth(x, mean=km)
                 store[s] = oracle.kv_dequant_smooth(c, sc, a, m, T, H, d)
             else:
                 c, sc, a = oracle.kv_append(x)

@@ -9,7 +9,7 @@ import oracle
 from bit_video_dit_b200 import nvfp4 as nv
 from bit_video_dit_b200 import synthetic as syn
 
-from .gpu_util import dev_bf16, f32_bits, host_bits, host_u8, require_gpu
+from .gpu_util import check_channel_means, dev_bf16, f32_bits, host_bits, host_u8, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -115,13 +115,16 @@ def test_full_chunk_append_with_scale_search():
 
 
 def _check_smoothed(cache, slot, x, which, smoothed, search):
-    """Codes, scales, tensor scale and (smoothed) channel means of one slot's K or V
-    bit for bit against the oracle; returns what the oracle's dequant needs."""
+    """One slot's K or V against the oracle: the stored channel means (when
+    smoothed) within the summation bound of the kernel's stated order around the
+    oracle's correctly rounded means, then codes, scales and tensor scale bit for
+    bit against the oracle's smoothed store built from the kernel's means; returns
+    what the oracle's dequant needs."""
     T, H, d = x.shape
     if smoothed:
-        codes, scales, a32, mean = oracle.kv_append_smooth(x, search46=search)
         m = cache.k_mean if which == 0 else cache.v_mean
-        assert np.array_equal(m[slot].cpu().numpy().view(np.uint32), mean.view(np.uint32))
+        km = check_channel_means(m[slot], syn.bf16_bits_to_f32(x).reshape(T, -1), oracle.channel_mean(x))
+        codes, scales, a32, mean = oracle.kv_append_smooth(x, search46=search, mean=km)
     else:
         codes, scales, a32 = oracle.kv_append(x, search46=search)
         mean = None

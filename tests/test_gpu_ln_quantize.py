@@ -1,6 +1,10 @@
 """GPU parity of nvfp4_ln_modulate_quantize (LayerNorm + adaLN modulate +
-NVFP4 quantize, reading R19) against the oracle: codes, scales and the tensor
-scale bit for bit."""
+NVFP4 quantize, reading R19) against the oracle, in two parts: the kernel's
+binary32 row statistics (mean, rstd) against the oracle's definition within
+the bounds of the kernel's stated summation order, then codes, scales and the
+tensor scale bit for bit against the oracle's modulate + quantize built from
+the kernel's own statistics (its binary32 reductions may land a unit away
+from the correctly rounded statistics, and the codes follow them)."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +13,7 @@ import oracle
 from bit_video_dit_b200 import nvfp4 as nv
 from bit_video_dit_b200 import synthetic as syn
 
-from .gpu_util import dev_bf16, f32_bits, host_u8, require_gpu
+from .gpu_util import check_ln_stats, dev_bf16, f32_bits, host_u8, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -24,15 +28,18 @@ def _check(x_bits, scale=None, shift=None, *, eps=1e-6, ld=None, alpha=None, row
         buf[:, :cols] = x_bits
         xd = dev_bf16(buf)[:, :cols]
     gs = None if alpha is None else torch.tensor([alpha], dtype=torch.float32, device="cuda")
+    ws = nv.workspace(nv.OP_LN_QUANTIZE, rows, 0, cols)
     q = nv.ln_modulate_quantize(xd, mod_scale=None if scale is None else dev_bf16(scale),
                                 mod_shift=None if shift is None else dev_bf16(shift), eps=eps, global_scale=gs,
-                                rowmajor_scales=rowmajor, scale_search=search)
+                                rowmajor_scales=rowmajor, scale_search=search, ws=ws)
     torch.cuda.synchronize()
+    # the row statistics follow the 256-byte control block of the workspace
+    st = check_ln_stats(ws[256:256 + 8 * rows].view(torch.float32), x_bits, eps)
     if search:
-        m = oracle.ln_modulate(x_bits, scale, shift, eps=eps)
+        m = oracle.ln_modulate(x_bits, scale, shift, eps=eps, stats=st)
         codes, scales, a32 = oracle.quantize(m, alpha, search46=True)
     else:
-        codes, scales, a32 = oracle.ln_modulate_quantize(x_bits, scale, shift, eps=eps, alpha=alpha)
+        codes, scales, a32 = oracle.ln_modulate_quantize(x_bits, scale, shift, eps=eps, alpha=alpha, stats=st)
     assert f32_bits(q.global_scale.cpu().numpy()) == f32_bits(a32)
     gc = host_u8(q.codes)
     bad = np.argwhere(gc != codes)

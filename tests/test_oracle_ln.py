@@ -1,7 +1,9 @@
 """Pins of the oracle's LayerNorm + adaLN modulate before the quantize
 (reading R19: population variance, eps inside the square root, no affine
 LayerNorm parameters, m = h * (1 + scale) + shift), against a float64 numpy
-LayerNorm and closed-form rows."""
+LayerNorm, exact rational statistics and closed-form rows."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
@@ -55,3 +57,64 @@ def test_quantize_of_the_modulated_rows_is_the_binary32_quantize():
     assert a32 == np.float32(np.abs(m).max() / np.float32(2688.0))
     c2, s2, a2 = oracle.quantize(m)
     assert np.array_equal(codes, c2) and np.array_equal(scales, s2) and a2 == a32
+
+
+def _f32_round(q: Fraction) -> np.float32:
+    """Correctly rounded (nearest, ties to even) binary32 of the rational q."""
+    f = np.float32(float(q))
+    best = None
+    for c in (np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))):
+        key = (abs(Fraction(float(c)) - q), int(np.array(c, np.float32).view(np.uint32)) & 1)
+        if best is None or key < best[0]:
+            best = (key, c)
+    return np.float32(best[1])
+
+
+@pytest.mark.parametrize("rows,cols", [(6, 3072), (4, 64), (3, 1040)])
+def test_row_mean_is_the_correctly_rounded_exact_mean(rows, cols):
+    # the mean statistic is fl32 of the exact rational mean (bf16 sums are exact in binary64 here)
+    bits = syn.activations_bf16(rows, cols, seed=3 * rows + cols)
+    st = oracle.ln_stats(bits, eps=1e-6)
+    x = syn.bf16_bits_to_f32(bits)
+    for r in range(rows):
+        mu = sum(Fraction(float(v)) for v in x[r]) / cols
+        assert st[r, 0] == _f32_round(mu), r
+
+
+@pytest.mark.parametrize("rows,cols", [(6, 3072), (4, 64)])
+def test_row_rstd_is_within_one_unit_of_the_exact_value(rows, cols):
+    # rstd = 1 / sqrt(var + eps) with the exact population variance: the binary64 route is within one
+    # binary32 unit of it (a block left out, n - 1, or squares about 0 move it by far more)
+    bits = syn.activations_bf16(rows, cols, seed=5 * rows + cols)
+    eps = 1e-6
+    st = oracle.ln_stats(bits, eps=eps)
+    x = syn.bf16_bits_to_f32(bits)
+    for r in range(rows):
+        xs = [Fraction(float(v)) for v in x[r]]
+        mu = sum(xs) / cols
+        var = sum((v - mu) ** 2 for v in xs) / cols
+        want = 1.0 / np.sqrt(float(var + Fraction(eps)))
+        got = float(st[r, 1])
+        assert abs(got - want) <= float(np.spacing(np.float32(want))), r
+
+
+def test_modulation_given_statistics_is_the_binary32_expression():
+    # with (mean, rstd) given, every element is fl32(fl32(fl32(fl32(x - mean) rstd) fl32(1 + sc)) + sh),
+    # restated here with numpy binary32 operations (each correctly rounded, no fusion)
+    rows, cols = 5, 320
+    bits = syn.activations_bf16(rows, cols, seed=21)
+    sc = syn.normal_bf16((cols,), seed=22, std=0.1)
+    sh = syn.normal_bf16((cols,), seed=23, std=0.1)
+    rng = np.random.default_rng(24)
+    st = np.stack([rng.standard_normal(rows), rng.uniform(0.5, 2.0, rows)], axis=1).astype(np.float32)
+    m = oracle.ln_modulate(bits, sc, sh, stats=st)
+    x = syn.bf16_bits_to_f32(bits)
+    f = np.float32
+    h = (x - st[:, :1].astype(f)).astype(f) * st[:, 1:].astype(f)
+    g = (f(1.0) + syn.bf16_bits_to_f32(sc)).astype(f)
+    want = (h.astype(f) * g).astype(f) + syn.bf16_bits_to_f32(sh)
+    assert np.array_equal(m, want.astype(f))
+    # and the quantize of it is the binary32 quantize of m
+    c1, s1, a1 = oracle.ln_modulate_quantize(bits, sc, sh, stats=st)
+    c2, s2, a2 = oracle.quantize(m)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2) and a1 == a2

@@ -44,7 +44,7 @@ def _build(tmp_path, replacements):
     L = ctypes.CDLL(str(so))
     vp, i64 = ctypes.c_void_p, ctypes.c_int64
     L.orc_rope.argtypes = [vp, i64, i64, i64, vp, vp, vp]
-    L.orc_kv_append_rope.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, vp, vp]
+    L.orc_kv_append_rope.argtypes = [vp, i64, i64, i64, vp, vp, ctypes.c_int, vp, vp, vp, vp, ctypes.c_int]
     L.orc_kv_append_rope.restype = ctypes.c_int
     return L
 
@@ -72,7 +72,7 @@ def _append(L, x, cs, sn, smooth):
     scales = np.zeros((T * H, d // 16), np.uint8)
     a = np.zeros(1, np.float32)
     mean = np.zeros(H * d, np.float32) if smooth else None
-    assert L.orc_kv_append_rope(_p(x), T, H, d, _p(cs), _p(sn), 0, _p(codes), _p(scales), _p(a), _p(mean)) == 0
+    assert L.orc_kv_append_rope(_p(x), T, H, d, _p(cs), _p(sn), 0, _p(codes), _p(scales), _p(a), _p(mean), 0) == 0
     return codes, scales, np.float32(a[0]), mean
 
 
@@ -138,8 +138,8 @@ MUTATIONS = {
          "                const float x1 = orc_bf16_to_f32(x[base + 2 * p + 1]);",
          "const float x0 = orc_bf16_to_f32(x[base + p]);\n"
          "                const float x1 = orc_bf16_to_f32(x[base + p + d / 2]);")],
-    "means of the unturned keys": [("        orc_channel_mean_f32(y, T, C, mean);",
-                                    "        orc_channel_mean(x, T, C, mean);")],
+    "means of the unturned keys": [("if (!mean_given) orc_channel_mean_f32(y, T, C, mean);",
+                                    "if (!mean_given) orc_channel_mean(x, T, C, mean);")],
 }
 
 
@@ -183,11 +183,20 @@ ORACLE_MUTATIONS = {
     "R10 one rounding instead of two": [
         ("            float v = qs * alpha;\n            out[r * cols + c] = orc_f32_to_bf16(v);",
          "            out[r * cols + c] = orc_f64_to_bf16((double)qs * (double)alpha);")],
-    "R19 eps outside the root": [("const float rstd = 1.0f / sqrtf(var + eps);",
-                                  "const float rstd = 1.0f / (sqrtf(var) + eps);")],
+    "R19 eps outside the root": [("stats[2 * r + 1] = (float)(1.0 / sqrt(var + (double)eps));",
+                                  "stats[2 * r + 1] = (float)(1.0 / (sqrt(var) + (double)eps));")],
+    "R19 one 16-element block in 32 left out of the row sum": [
+        ("for (int64_t c = 0; c < cols; c++) s1 += (double)orc_bf16_to_f32(x[r * ld + c]);",
+         "for (int64_t c = 0; c < cols; c++) if ((c / 16) % 32 != 31) s1 += (double)orc_bf16_to_f32(x[r * ld + c]);")],
+    "R19 squares taken about 0 instead of the mean": [
+        ("const double d = (double)orc_bf16_to_f32(x[r * ld + c]) - mu;",
+         "const double d = (double)orc_bf16_to_f32(x[r * ld + c]);")],
     "R20 first 32 tokens dropped": [
-        ("for (int64_t t = p; t < T; t += 32) s = s + orc_bf16_to_f32(x[t * C + c]);",
-         "for (int64_t t = p + 32; t < T; t += 32) s = s + orc_bf16_to_f32(x[t * C + c]);")],
+        ("for (int64_t t = 0; t < T; t++) s += (double)orc_bf16_to_f32(x[t * C + c]);",
+         "for (int64_t t = 32; t < T; t++) s += (double)orc_bf16_to_f32(x[t * C + c]);")],
+    "R20 one token in 32 left out of the sum": [
+        ("for (int64_t t = 0; t < T; t++) s += (double)orc_bf16_to_f32(x[t * C + c]);",
+         "for (int64_t t = 0; t < T; t++) if (t % 32 != 31) s += (double)orc_bf16_to_f32(x[t * C + c]);")],
     "R22 signs inverted": [("v[i] = sign[i] < 0 ? -v[i] : v[i];", "v[i] = sign[i] > 0 ? -v[i] : v[i];")],
     "R22 normalised by 1/2": [("for (int i = 0; i < 16; i++) v[i] = v[i] * 0.25f;",
                                "for (int i = 0; i < 16; i++) v[i] = v[i] * 0.5f;")],
@@ -202,8 +211,8 @@ ORACLE_MUTATIONS = {
     "R18 a tie takes the target-4 candidate": [
         ("block_sq_error(xb, sc4, q4, a32) < block_sq_error(xb, sc, q, a32)",
          "block_sq_error(xb, sc4, q4, a32) <= block_sq_error(xb, sc, q, a32)")],
-    "R19 sample variance (n - 1)": [("const float var = row_sum32(dr, cols) / n;",
-                                     "const float var = row_sum32(dr, cols) / (n - 1.0f);")],
+    "R19 sample variance (n - 1)": [("const double var = s2 / (double)cols;",
+                                     "const double var = s2 / (double)(cols - 1);")],
     "R21 transposed operand not transposed": [
         ("(uint8_t)(q[2 * j][i] | (q[2 * j + 1][i] << 4));", "(uint8_t)(q[i][2 * j] | (q[i][2 * j + 1] << 4));")],
     "R20 mean subtracted again in the dequant": [("float y = v + mean[(r % H) * d + c];",

@@ -71,18 +71,52 @@ def test_channel_mean_of_a_constant_channel_is_that_constant():
 
 
 @pytest.mark.parametrize("T", [1, 31, 33, 100, 2640])
-def test_channel_mean_is_within_the_summation_error_bound(T):
-    # a token dropped or counted twice, or a wrong channel stride, moves the mean by ~|x| / T,
-    # far outside this bound (at most ceil(T/32) + 5 rounded additions per result, then a division)
+def test_channel_mean_is_the_correctly_rounded_exact_mean(T):
+    # R20 is the definition: fl32 of the exact mean, whatever the data (a token dropped or counted
+    # twice, or a wrong channel stride, moves it by ~|x| / T)
     rng = np.random.default_rng(T)
     C = 3 * 32
     x = bf16_value(bf16_rne(rng.standard_normal((T, C)).astype(np.float32)))
-    m = oracle.channel_mean(bf16_bits(x)).astype(np.float64)
-    exact = np.array([float(sum(Fraction(float(v)) for v in x[:, c]) / T) for c in range(C)])
-    n_add = -(-T // 32) + 5
+    m = oracle.channel_mean(bf16_bits(x))
+    for c in range(C):
+        assert m[c] == f32_round(sum(Fraction(float(v)) for v in x[:, c]) / T), c
+
+
+def summation_bound(x: np.ndarray, mean: np.ndarray) -> np.ndarray:
+    """Bound on |m - mean| for binary32 channel means m summed as 32 strided
+    partial sums (each over ceil(T/32) tokens in order) met in 5 pairwise
+    levels, then divided by T: every term passes through at most
+    ceil(T/32) + 5 rounded additions, and the division adds one rounding."""
+    T = x.shape[0]
     u = 2.0 ** -24
-    bound = n_add * u * np.abs(x.astype(np.float64)).sum(0) / T * 1.01 + u * np.abs(exact) + 1e-300
-    assert np.all(np.abs(m - exact) <= bound)
+    depth = -(-T // 32) + 5
+    return (depth + 1) * u * np.abs(x.astype(np.float64)).sum(0) / T + u * np.abs(mean)
+
+
+@pytest.mark.parametrize("T", [1, 33, 2640])
+def test_summation_bound_holds_for_strided_partials_and_catches_a_dropped_token(T):
+    # The GPU tests hold a kernel's channel means to summation_bound.  A binary32 sum in that
+    # shape (32 strided partials, pairwise levels) stays inside it; the same sum with one
+    # token left out does not.
+    rng = np.random.default_rng(100 + T)
+    C = 64
+    x = bf16_value(bf16_rne((rng.standard_normal((T, C)) + 3.0).astype(np.float32)))
+    mean = oracle.channel_mean(bf16_bits(x)).astype(np.float64)
+    bound = summation_bound(x, mean)
+
+    def strided(xs):
+        part = np.zeros((32, C), np.float32)
+        for t in range(xs.shape[0]):
+            part[t % 32] = (part[t % 32] + xs[t]).astype(np.float32)
+        while part.shape[0] > 1:
+            h = part.shape[0] // 2
+            part = (part[:h] + part[h:]).astype(np.float32)
+        return (part[0] / np.float32(T)).astype(np.float32).astype(np.float64)
+
+    assert np.all(np.abs(strided(x) - mean) <= bound)
+    if T > 1:
+        short = strided(np.delete(x, T // 2, axis=0))
+        assert np.all(np.abs(short - mean) > bound)
 
 
 def test_channel_constant_chunk_round_trips_exactly_with_smoothing_only():
