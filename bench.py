@@ -1,20 +1,19 @@
 """Throughput of the NVFP4 hot path on B200.
 
-One step = one pass of the whole path on seeded synthetic DiT-shaped inputs:
-  1. nvfp4_quantize  of the activation A [4096 x 3072] bf16 (tensor amax,
-     block scales, E2M1 codes, swizzled scale tiles)
-  2. nvfp4_gemm      QKV projection 4096 x 9216 x 3072, W pre-quantized once,
-     bias epilogue, bf16 out
-  3. nvfp4_kv_append of one frame-chunk's K and V [2640 x 24 x 128] into ring
-     slot step % 21
-  4. nvfp4_kv_dequant of all 21 slots (ring order) back to bf16
-`value` is the W4A4 linear-layer throughput (2*M*N*K of step 2 per second of
-steps 1+2, device-timed with CUDA events); the KV rows are reported under
-"kv".  The timed steps are captured as one CUDA graph, with the timing events
-between components as event-record nodes, so the timed region holds device
-work only (no host launch gaps); `e2e` instead
-calls the public Python API with host buffers every step.  The 681 MB bf16 output of step 4 overwrites L2 (126 MB) every step, so
-each step's GEMM and quantize read their inputs from HBM.
+One step = one forward of the DiT linear stack on seeded synthetic inputs:
+30 layers at 16384 tokens, hidden 3072, FFN 14336, every linear W4A4 NVFP4:
+  nvfp4_quantize of the bf16 input [16384 x 3072], then per layer
+  QKV 3072->9216 + bias (bf16 Q, K, V; its V third requantized in the same
+  epilogue as the stand-in attention output) -> out-projection 3072->3072 +
+  bias -> FFN up 3072->14336 + bias + GELU -> FFN down 14336->3072 + bias,
+  each GEMM's epilogue writing the next GEMM's NVFP4 input (output tensor
+  scales fixed by one calibration pass: delayed scaling).
+`value` = 123.7 TFLOP of GEMM work per step / the step's device time (CUDA
+events; the timed steps replayed from one CUDA graph with an event before
+every launch, so per-GEMM times come from the same run).  Beside it: the
+single-layer QKV workload (quantize + 4096 x 9216 x 3072 GEMM), the NVFP4 KV
+cache (append, dequant of 21 slots), the 8192-token FFN pair and the next-row
+kernels.  `e2e` runs the stack through the public API with host buffers.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -44,7 +43,7 @@ import torch  # noqa: E402
 from bit_video_dit_b200 import synthetic as syn  # noqa: E402
 
 METRIC = "W4A4 GEMM TFLOPS (% B200 FP4 peak); quantize/KV-append GB/s (% HBM peak)"
-WORKLOAD = "dit_qkv_4096x9216x3072_bias+kv_append_dequant_21x2640x24x128"
+WORKLOAD = "dit_stack_30x4_16384"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput (9 / 2.25 PFLOP/s)
 NOMINAL_FP4_TFLOPS = 9000.0
 NOMINAL_HBM_GBS = 8000.0
@@ -378,91 +377,218 @@ def dev_bf16(bits: np.ndarray) -> torch.Tensor:
 
 
 # --------------------------------------------------------------------------- ours
+STACK_NAMES = ("qkv", "out", "up", "down")
+
+
+def build_stack(nv, dev, layers: int, rank: int):
+    """The 16384-token DiT linear stack with seeded N(0, 0.02) weights (the same
+    generator as the parity test), its first-layer input and the calibrated
+    output scales."""
+    from bit_video_dit_b200.stack import LinearStack
+
+    M, D, F = syn.STACK_M, syn.STACK_LAYER[0].K, syn.STACK_LAYER[2].N
+    st = LinearStack(M, D, F, dev)
+    for l in range(layers):
+        w, b = syn.stack_layer_bf16(l, D, F)
+        st.add_layer({k: dev_bf16(v) for k, v in w.items()}, {k: dev_bf16(v) for k, v in b.items()})
+        del w
+    x_host = syn.activations_bf16(M, D, seed=80 + 1000 * rank)
+    x = dev_bf16(x_host)
+    st.calibrate(x)
+    torch.cuda.synchronize()
+    return st, x, x_host
+
+
+def time_stack(st, x, steps: int, warmup: int, direct: bool):
+    """Warm-up steps, then `steps` timed forwards of the stack (input quantize +
+    every GEMM), captured as one CUDA graph each unless `direct`, with an event
+    before every launch (event-record nodes inside the graph).  Returns the
+    total ms and the per-launch-class mean ms."""
+    n = st.launches_per_forward()
+    L = len(st.layers)
+    evs = [[torch.cuda.Event(enable_timing=True, external=not direct) for _ in range(n + 1)] for _ in range(steps)]
+
+    def fwd(ev=None):
+        if ev:
+            ev[0].record()
+        st.quantize_input(x)
+        k = 1
+        for l in range(L):
+            for g in range(4):
+                if ev:
+                    ev[k].record()
+                st.gemm(l, g)
+                k += 1
+        if ev:
+            ev[k].record()
+
+    if direct:
+        run_warm = lambda: [fwd() for _ in range(warmup)]
+        run_timed = lambda: [fwd(evs[i]) for i in range(steps)]
+        graphs = []
+    else:
+        gw, gt = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gw):
+            for _ in range(warmup):
+                fwd()
+        with torch.cuda.graph(gt):
+            for i in range(steps):
+                fwd(evs[i])
+        run_warm, run_timed = gw.replay, gt.replay
+        graphs = [gw, gt]
+    torch.cuda.synchronize()
+    run_warm()
+    torch.cuda.synchronize()
+    return run_timed, evs, graphs
+
+
+def stack_components(evs, L: int) -> dict:
+    """Mean ms per launch of the input quantize and of each GEMM of a layer."""
+    q = np.mean([e[0].elapsed_time(e[1]) for e in evs])
+    per = {name: [] for name in STACK_NAMES}
+    for e in evs:
+        k = 1
+        for _ in range(L):
+            for g in range(4):
+                per[STACK_NAMES[g]].append(e[k].elapsed_time(e[k + 1]))
+                k += 1
+    return {"input_quantize": float(q), **{k: float(np.mean(v)) for k, v in per.items()}}
+
+
+def measure_linear_kv(nv, dev, rank: int, steps: int, warmup: int) -> dict:
+    """The single-layer and KV-cache workloads beside the stack: quantize A
+    [4096 x 3072] + the QKV projection 4096 x 9216 x 3072 with bias to bf16
+    (W pre-quantized once), the KV append of one 2640 x 24 x 128 K/V chunk into
+    ring slot (step mod 21) and the dequant of all 21 slots, each step captured
+    in a graph with events between the four launches (the 681 MB dequant output
+    overwrites L2 every step)."""
+    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
+    S, T, H, D = syn.KV_SLOTS, syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    a_host = syn.activations_bf16(M, K, seed=2 + 1000 * rank)
+    w_host = syn.normal_bf16((N, K), seed=3, std=0.02)
+    a = dev_bf16(a_host)
+    w = dev_bf16(w_host)
+    bias = dev_bf16(syn.normal_bf16((N,), seed=4, std=0.02))
+    qw = nv.quantize(w)
+    qa = nv.empty_nvfp4(M, K, dev)
+    ws_q = nv.workspace(nv.OP_QUANTIZE, M, 0, K, dev)
+    ws_g = nv.workspace(nv.OP_GEMM, M, N, K, dev)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    cache = nv.KVCache(S, T, H, D, dev)
+    chunks = [tuple(dev_bf16(x) for x in syn.kv_chunk_bf16(T, H, D, seed=50 + i + 1000 * rank)) for i in range(4)]
+    for s_ in range(S):
+        cache.append(s_, *chunks[s_ % 4])
+    ring = torch.arange(S, dtype=torch.int32, device=dev)
+    k_out = torch.empty((S, T, H, D), dtype=torch.bfloat16, device=dev)
+    v_out = torch.empty_like(k_out)
+    nv.quantize(a, out=qa, ws=ws_q)
+    nv.gemm(qa, qw, out=c, bias=bias, ws=ws_g)
+    cache.dequant(ring, k_out, v_out)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(steps)]
+
+    def step(i, ev=None):
+        for j, f in enumerate((lambda: nv.quantize(a, out=qa, ws=ws_q),
+                               lambda: nv.gemm(qa, qw, out=c, bias=bias, ws=ws_g),
+                               lambda: cache.append(i % S, *chunks[i % 4]),
+                               lambda: cache.dequant(ring, k_out, v_out))):
+            if ev:
+                ev[j].record()
+            f()
+        if ev:
+            ev[4].record()
+
+    gw, gt = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw):
+        for i in range(warmup):
+            step(i)
+    with torch.cuda.graph(gt):
+        for i in range(steps):
+            step(warmup + i, evs[i])
+    gw.replay()
+    gt.replay()
+    torch.cuda.synchronize()
+    comp = np.mean([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs], axis=0)
+    code, _ = nv.read_device_error(ws_g)
+    if code != nv.OK:
+        raise RuntimeError(f"device error {code} in the QKV GEMM")
+    del gw, gt
+    return {"comp": comp, "a": a, "w": w, "qa": qa, "ws_q": ws_q, "chunks": chunks, "cache": cache, "ring": ring,
+            "k_out": k_out, "v_out": v_out}
+
+
+def e2e_stack(nv, st, x_host, steps: int) -> float:
+    """ms per step of the stack through the public API with host buffers: each
+    step copies its bf16 input [16384 x 3072] from pinned host memory to the
+    device, runs the stack, and copies the final NVFP4 output (codes, scales,
+    tensor scale) back to pinned host memory.  Copies run on their own streams
+    with double-buffered device inputs, so a step's copies overlap the
+    neighbouring steps' compute."""
+    dev = st.device
+    stream = torch.cuda.current_stream()
+    x_pin = torch.from_numpy(x_host.view(np.int16)).pin_memory()
+    outs = [(torch.empty(st.x.codes.shape, dtype=torch.uint8).pin_memory(),
+             torch.empty(st.x.scales.shape, dtype=torch.uint8).pin_memory(),
+             torch.empty(1, dtype=torch.float32).pin_memory()) for _ in range(2)]
+    x_devs = [torch.empty(x_host.shape, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    res = [nv.empty_nvfp4(st.M, st.D, dev) for _ in range(2)]
+
+    def run(n_steps):
+        ev_in = [torch.cuda.Event() for _ in range(n_steps)]
+        ev_cmp = [torch.cuda.Event() for _ in range(n_steps)]
+        ev_out = [torch.cuda.Event() for _ in range(n_steps)]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        for k in range(n_steps):
+            b = k % 2
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(ev_cmp[k - 2])
+                x_devs[b].view(torch.int16).copy_(x_pin, non_blocking=True)
+                ev_in[k].record(s_in)
+            stream.wait_event(ev_in[k])
+            if k >= 2:
+                stream.wait_event(ev_out[k - 2])
+            out = st.forward(x_devs[b])
+            # the result leaves the stack's buffer for this step's own (the next step overwrites it)
+            res[b].codes.copy_(out.codes)
+            res[b].scales.copy_(out.scales)
+            res[b].global_scale.copy_(out.global_scale)
+            ev_cmp[k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[k])
+                outs[b][0].copy_(res[b].codes, non_blocking=True)
+                outs[b][1].copy_(res[b].scales, non_blocking=True)
+                outs[b][2].copy_(res[b].global_scale, non_blocking=True)
+                ev_out[k].record(s_out)
+        stream.wait_event(ev_out[n_steps - 1])
+        stream.wait_event(ev_in[n_steps - 1])
+        end.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / n_steps
+
+    run(2)
+    return run(steps)
+
+
 def run_ours(args, rank: int, world: int) -> dict | None:
     from bit_video_dit_b200 import build as nvbuild
     from bit_video_dit_b200 import nvfp4 as nv
 
     nvbuild.build()
     dev = torch.device("cuda", torch.cuda.current_device())
-    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
-    S, T, H, D = syn.KV_SLOTS, syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
-
-    a_host = syn.activations_bf16(M, K, seed=2 + 1000 * rank)
-    w_host = syn.normal_bf16((N, K), seed=3, std=0.02)
-    bias_host = syn.normal_bf16((N,), seed=4, std=0.02)
-    a = dev_bf16(a_host)
-    w = dev_bf16(w_host)
-    bias = dev_bf16(bias_host)
-    qw = nv.quantize(w)  # weights quantized once
-    del w
-    qa = nv.empty_nvfp4(M, K, dev)
-    ws_q = nv.workspace(nv.OP_QUANTIZE, M, 0, K, dev)
-    ws_g = nv.workspace(nv.OP_GEMM, M, N, K, dev)
-    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    cache = nv.KVCache(S, T, H, D, dev)
-    n_chunks = 4  # distinct K/V chunks cycled through the ring
-    chunks = [tuple(dev_bf16(x) for x in syn.kv_chunk_bf16(T, H, D, seed=50 + i + 1000 * rank))
-              for i in range(n_chunks)]
-    for s in range(S):
-        cache.append(s, *chunks[s % n_chunks])
-    ring = torch.arange(S, dtype=torch.int32, device=dev)
-    k_out = torch.empty((S, T, H, D), dtype=torch.bfloat16, device=dev)
-    v_out = torch.empty_like(k_out)
-    stream = torch.cuda.current_stream()
-
-    do_quant = lambda: nv.quantize(a, out=qa, ws=ws_q)
-    do_gemm = lambda: nv.gemm(qa, qw, out=c, bias=bias, ws=ws_g)
-    do_append = [lambda s=s: cache.append(s, *chunks[s % n_chunks]) for s in range(S)]
-    do_dequant = lambda: cache.dequant(ring, k_out, v_out)
-    for f in (do_quant, do_gemm, do_append[0], do_dequant):
-        f()  # first calls set kernel attributes and resolve the driver entry point
-    torch.cuda.synchronize()
-
-    def step(i, ev=None):
-        if ev:
-            ev[0].record()  # the current (capture) stream
-        do_quant()
-        if ev:
-            ev[1].record()  # the current (capture) stream
-        do_gemm()
-        if ev:
-            ev[2].record()  # the current (capture) stream
-        do_append[i % S]()
-        if ev:
-            ev[3].record()  # the current (capture) stream
-        do_dequant()
-        if ev:
-            ev[4].record()  # the current (capture) stream
-
-    # By default the warm-up steps and the timed steps are each captured as one
-    # CUDA graph (the timing events between the components become event-record
-    # nodes), so the timed region holds device work only: no host launch gaps
-    # and no per-component graph launches.  --direct launches every component
-    # on the stream instead.
-    evs = [[torch.cuda.Event(enable_timing=True, external=not args.direct) for _ in range(5)]
-           for _ in range(args.steps)]
-    if args.direct:
-        run_warmup = lambda: [step(i) for i in range(args.warmup)]
-        run_timed = lambda: [step(args.warmup + i, evs[i]) for i in range(args.steps)]
-        graphs = []
-    else:
-        g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_warm):
-            for i in range(args.warmup):
-                step(i)
-        with torch.cuda.graph(g_timed):
-            for i in range(args.steps):
-                step(args.warmup + i, evs[i])
-        run_warmup, run_timed = g_warm.replay, g_timed.replay
-        graphs = [g_warm, g_timed]
-    torch.cuda.synchronize()
-
-    run_warmup()
-    torch.cuda.synchronize()
-    code, _ = nv.read_device_error(ws_g)
+    L = args.layers
+    st, x, x_host = build_stack(nv, dev, L, rank)
+    code, _ = nv.read_device_error(st.ws_g)
     if code != nv.OK:
-        raise RuntimeError(f"device error {code} during warm-up")
+        raise RuntimeError(f"device error {code} during calibration")
+    run_timed, evs, graphs = time_stack(st, x, args.steps, args.warmup, args.direct)
 
+    stream = torch.cuda.current_stream()
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
     clocks.start()
     time.sleep(0.3)
@@ -479,88 +605,60 @@ def run_ours(args, rank: int, world: int) -> dict | None:
         torch.distributed.barrier()
     clk = clocks.stop()
     del graphs
-
-    # The adaptive scale search ({4, 6}) variants of the two quantize launches,
-    # timed the same way (inside a graph, each after a dequant of all slots so
-    # that its input comes from HBM); reported beside the step, not part of it.
-    search = measure_scale_search(nv, a, qa, ws_q, chunks, cache, ring, k_out, v_out, reps=5)
-    # the training-side operands (2D weight scaling, RHT transposed operands) and the
-    # weight-gradient GEMM on the same layer shapes, also beside the step
-    train = measure_training(nv, a, dev_bf16(w_host), cache, ring, k_out, v_out, reps=5)
-    # attention reading the NVFP4 cache directly (one query chunk), beside the step
-    attn = measure_attention(nv, cache, ring, k_out, v_out, reps=3)
-    # the 8192-token FFN pair (up with GELU + requant, down to bf16), beside the step
-    ffn = measure_ffn(nv, lambda: cache.dequant(ring, k_out, v_out), k_out.device, reps=5)
-
+    code, _ = nv.read_device_error(st.ws_g)
+    if code != nv.OK:
+        raise RuntimeError(f"device error {code} in the timed stack")
     total_ms = t_start.elapsed_time(t_end)
-    comp = np.zeros(4)
-    for e in evs:
-        comp += [e[j].elapsed_time(e[j + 1]) for j in range(4)]
-    comp /= args.steps  # ms per step per component: quantize, gemm, append, dequant
+    comp = stack_components(evs, L)
+    e2e_ms = e2e_stack(nv, st, x_host, max(3, min(args.steps, 10)))
 
-    # --- e2e through the public API with host buffers (linear layer) -------
-    # Every step copies its own A from pinned host memory and its C back to
-    # pinned host memory inside the timed region.  The copies run on their own
-    # streams with double-buffered device tensors, so step k+1's host->device
-    # copy and step k-1's device->host copy overlap step k's compute (PCIe is
-    # full duplex: one copy engine per direction).
-    a_pin = torch.from_numpy(a_host.view(np.int16)).pin_memory()
-    c_pins = [torch.empty((M, N), dtype=torch.int16).pin_memory() for _ in range(2)]
-    a_devs = [torch.empty((M, K), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    c_devs = [c, torch.empty_like(c)]
-    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    e2e_steps = max(3, min(args.steps, 10))
+    sub = None
+    if not args.stack_only:
+        lk = measure_linear_kv(nv, dev, rank, max(5, min(args.steps, 20)), args.warmup)
+        flush = lambda: lk["cache"].dequant(lk["ring"], lk["k_out"], lk["v_out"])
+        sub = {"lk": lk,
+               "search": measure_scale_search(nv, lk["a"], lk["qa"], lk["ws_q"], lk["chunks"], lk["cache"],
+                                              lk["ring"], lk["k_out"], lk["v_out"], reps=5),
+               "train": measure_training(nv, lk["a"], lk["w"], lk["cache"], lk["ring"], lk["k_out"], lk["v_out"],
+                                         reps=5),
+               "attn": measure_attention(nv, lk["cache"], lk["ring"], lk["k_out"], lk["v_out"], reps=3),
+               "ffn": measure_ffn(nv, flush, dev, reps=5)}
 
-    def e2e_run(n_steps):
-        ev_in = [torch.cuda.Event() for _ in range(n_steps)]
-        ev_cmp = [torch.cuda.Event() for _ in range(n_steps)]
-        ev_out = [torch.cuda.Event() for _ in range(n_steps)]
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-        s_in.wait_event(start)
-        s_out.wait_event(start)
-        for k in range(n_steps):
-            b = k % 2
-            with torch.cuda.stream(s_in):
-                if k >= 2:
-                    s_in.wait_event(ev_cmp[k - 2])  # a_devs[b] is free once step k-2 has read it
-                a_devs[b].view(torch.int16).copy_(a_pin, non_blocking=True)
-                ev_in[k].record(s_in)
-            stream.wait_event(ev_in[k])
-            if k >= 2:
-                stream.wait_event(ev_out[k - 2])  # c_devs[b] is free once step k-2's result is on the host
-            nv.quantize(a_devs[b], out=qa, ws=ws_q)
-            nv.gemm(qa, qw, out=c_devs[b], bias=bias, ws=ws_g)
-            ev_cmp[k].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_cmp[k])
-                c_pins[b].copy_(c_devs[b].view(torch.int16), non_blocking=True)
-                ev_out[k].record(s_out)
-        stream.wait_event(ev_out[n_steps - 1])
-        stream.wait_event(ev_in[n_steps - 1])
-        end.record(stream)
-        torch.cuda.synchronize()
-        return start.elapsed_time(end) / n_steps
-
-    e2e_run(2)
-    e2e_ms = e2e_run(e2e_steps)
-
-    times = torch.tensor([total_ms, *comp.tolist(), e2e_ms], dtype=torch.float64, device=dev)
-    total_ms, q_ms, g_ms, ap_ms, dq_ms, e2e_ms = max_over_ranks(times, world)
+    keys = ["input_quantize", *STACK_NAMES]
+    times = torch.tensor([total_ms, *[comp[k] for k in keys], e2e_ms,
+                          *(sub["lk"]["comp"].tolist() if sub else [0.0] * 4)], dtype=torch.float64, device=dev)
+    vals = max_over_ranks(times, world)
+    total_ms, e2e_ms = vals[0], vals[1 + len(keys)]
+    comp = dict(zip(keys, vals[1:1 + len(keys)]))
+    q2_ms, g2_ms, ap_ms, dq_ms = vals[2 + len(keys):]
     if rank != 0:
         return None
+    return report(args, world, st, total_ms, comp, e2e_ms, clk, sub, (q2_ms, g2_ms, ap_ms, dq_ms))
 
+
+def _rl(bound, achieved, peak, unit, **kw):
+    return {"bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
+            "frac": round(achieved / peak, 4), **kw}
+
+
+def report(args, world, st, total_ms, comp, e2e_ms, clk, sub, lin) -> dict:
     pk = peaks()
-    flops = 2.0 * M * N * K
-    lin_ms = q_ms + g_ms
-    value = job_tflops(world, flops, lin_ms)
-    gemm_tflops = flops / (g_ms * 1e-3) / 1e12
     fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
-    quant_bytes = M * K * 2.5625
-    kv_elems = T * H * D
-    append_bytes = 2 * kv_elems * 2.5625
-    dequant_bytes = 2 * S * kv_elems * (0.5625 + 2.0)
+    L, M, D, F = len(st.layers), st.M, st.D, st.F
+    ms_step = total_ms / args.steps
+    flops = st.flops()
+    value = job_tflops(world, flops, ms_step)
+    shapes = {"qkv": (3 * D, D), "out": (D, D), "up": (F, D), "down": (D, F)}
+    gemm_ms = sum(comp[k] for k in STACK_NAMES)  # per layer
+    gemm_tflops = flops / L / (gemm_ms * 1e-3) / 1e12
+    by = {}
+    for k in STACK_NAMES:
+        N, K = shapes[k]
+        t = 2.0 * M * N * K / (comp[k] * 1e-3) / 1e12
+        by[f"gemm_{k}"] = _rl("tensor", t, fp4_peak, "TFLOP/s", ms=round(comp[k], 4), shape=[M, N, K])
+    qbytes = M * D * 2.5625
+    by["input_quantize"] = _rl("hbm", qbytes / (comp["input_quantize"] * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s",
+                               ms=round(comp["input_quantize"], 4))
     tr = recorded_traffic()
     out = {
         "metric": METRIC,
@@ -569,163 +667,212 @@ def run_ours(args, rank: int, world: int) -> dict | None:
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(total_ms / args.steps, 4),
+        "ms_per_step": round(ms_step, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate); bf16 in/out",
-        "data": "synthetic (seeded N(0,1) activations with 0.1% x20 outlier channels, N(0,0.02) weights)",
-        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "kv_slots": S, "kv_tokens": T, "kv_heads": H,
-                   "kv_head_dim": D, "parallelism": f"dp{world} (independent replicas, no collective)",
-                   "l2": "inputs larger than L2: each step's 681 MB KV dequant output overwrites the 126 MB L2"},
-        "roofline": {"kernel": "nvfp4 gemm (tcgen05 mxf4nvf4)", "bound": "tensor",
-                     "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(gemm_tflops / fp4_peak, 4),
-                     "peak_source": f"{pk['source']} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16)",
-                     "frac_of_nominal_9pf": round(gemm_tflops / NOMINAL_FP4_TFLOPS, 4),
-                     "traffic": None if tr is None else tr["dram_bytes_per_launch"],
-                     "algorithmic_bytes": M * K // 2 + N * K // 2 + (M + N) * K // 16 + M * N * 2},
-        "roofline_by_kernel": {
-            "gemm": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4)},
-            "quantize": {"bound": "hbm", "achieved": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
-                         "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(quant_bytes / (q_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
-            "kv_append": {"bound": "hbm", "achieved": round(append_bytes / (ap_ms * 1e-3) / 1e9, 1),
-                          "peak": pk["hbm_gbs"], "unit": "GB/s",
-                          "frac": round(append_bytes / (ap_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
-            "kv_dequant": {"bound": "hbm", "achieved": round(dequant_bytes / (dq_ms * 1e-3) / 1e9, 1),
-                           "peak": pk["hbm_gbs"], "unit": "GB/s",
-                           "frac": round(dequant_bytes / (dq_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}},
-        "components_ms": {"quantize": round(q_ms, 4), "gemm": round(g_ms, 4), "kv_append": round(ap_ms, 4),
-                          "kv_dequant": round(dq_ms, 4)},
-        "quantize": {"GB/s": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
-                     "frac_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                     "bytes_per_call": quant_bytes},
-        "kv": {"append_GB/s": round(append_bytes / (ap_ms * 1e-3) / 1e9, 1),
-               "append_frac_hbm": round(append_bytes / (ap_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-               "dequant_GB/s": round(dequant_bytes / (dq_ms * 1e-3) / 1e9, 1),
-               "dequant_frac_hbm": round(dequant_bytes / (dq_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-               "hbm_peak_GB/s": pk["hbm_gbs"], "cache_bytes": cache.nbytes()},
-        "scale_search": {
-            "what": "adaptive per-block scale search over the targets {4, 6}, outside the step",
-            "quantize_ms": round(search["quantize_ms"], 4),
-            "quantize_GB/s": round(quant_bytes / (search["quantize_ms"] * 1e-3) / 1e9, 1),
-            "kv_append_ms": round(search["kv_append_ms"], 4),
-            "kv_append_GB/s": round(append_bytes / (search["kv_append_ms"] * 1e-3) / 1e9, 1)},
-        "kv_smoothing": {
-            "what": "KV append with K-smoothing of K and the scale search on K and V (channel means + quantize, "
-                    "two launches), and the dequant of all slots with the means added back, outside the step",
-            "append_ms": round(search["smooth_append_ms"], 4),
-            "append_GB/s": round(append_bytes / (search["smooth_append_ms"] * 1e-3) / 1e9, 1),
-            "dequant_ms": round(search["smooth_dequant_ms"], 4),
-            "dequant_GB/s": round(dequant_bytes / (search["smooth_dequant_ms"] * 1e-3) / 1e9, 1)},
-        "kv_rope": {
-            "what": "KV append with the keys' rotary embedding fused ahead of their quantize (3-frame x 22 x 40 "
-                    "angle table read from L2), plain and with K-smoothing + scale search (means of the turned "
-                    "keys, two launches), outside the step; GB/s counts the append's algorithmic bytes",
-            "append_ms": round(search["rope_append_ms"], 4),
-            "append_GB/s": round(append_bytes / (search["rope_append_ms"] * 1e-3) / 1e9, 1),
-            "smooth_search_append_ms": round(search["rope_smooth_append_ms"], 4),
-            "smooth_search_append_GB/s": round(append_bytes / (search["rope_smooth_append_ms"] * 1e-3) / 1e9, 1)},
-        "ffn_8192": {
-            "what": "the FFN pair at 8192 tokens, outside the step: quantize A [8192x3072], up 3072->14336 with GELU "
-                    "and the NVFP4 requant of its output (output scale from a calibration pass), down 14336->3072 to "
-                    "bf16 on that NVFP4 output; each 2*M*N*K = 721.6 GFLOP",
-            "quantize_ms": round(ffn["quantize_ms"], 4),
-            "up_ms": round(ffn["up_ms"], 4),
-            "up_TFLOP/s": round(2 * syn.FFN_UP.M * syn.FFN_UP.N * syn.FFN_UP.K / (ffn["up_ms"] * 1e-3) / 1e12, 1),
-            "up_frac_fp4_peak": round(2 * syn.FFN_UP.M * syn.FFN_UP.N * syn.FFN_UP.K / (ffn["up_ms"] * 1e-3) / 1e12
-                                      / fp4_peak, 4),
-            "down_ms": round(ffn["down_ms"], 4),
-            "down_TFLOP/s": round(2 * syn.FFN_DOWN.M * syn.FFN_DOWN.N * syn.FFN_DOWN.K / (ffn["down_ms"] * 1e-3)
-                                  / 1e12, 1),
-            "down_frac_fp4_peak": round(2 * syn.FFN_DOWN.M * syn.FFN_DOWN.N * syn.FFN_DOWN.K
-                                        / (ffn["down_ms"] * 1e-3) / 1e12 / fp4_peak, 4)},
-        "training": {
-            "what": "training-side NVFP4 on the QKV layer shapes, outside the step: 2D (16x16) scaling of W "
-                    "[9216x3072] writing W and W^T operands; RHT + transposed 1D quantize of X [4096x3072] and "
-                    "dY [4096x9216] (weight-gradient operands); dW = dY^T X (9216x3072x4096) on those operands",
-            "quantize_2d_ms": round(train["quantize_2d_ms"], 4),
-            "quantize_2d_GB/s": round(N * K * 3.125 / (train["quantize_2d_ms"] * 1e-3) / 1e9, 1),
-            "quantize_t_x_ms": round(train["quantize_t_x_ms"], 4),
-            "quantize_t_x_GB/s": round(M * K * 2.5625 / (train["quantize_t_x_ms"] * 1e-3) / 1e9, 1),
-            "quantize_t_dy_ms": round(train["quantize_t_dy_ms"], 4),
-            "quantize_t_dy_GB/s": round(M * N * 2.5625 / (train["quantize_t_dy_ms"] * 1e-3) / 1e9, 1),
-            "wgrad_ms": round(train["wgrad_ms"], 4),
-            "wgrad_TFLOP/s": round(2.0 * N * K * M / (train["wgrad_ms"] * 1e-3) / 1e12, 1)},
-        "kv_attention": {
-            "what": "softmax attention of one 2640x24x128 bf16 query chunk over NVFP4 cache slots read directly "
-                    "(e2m1 * s tiles in binary16, tcgen05 f16 MMAs with binary32 accumulators, one-pass softmax), "
-                    "outside the step; TFLOP/s counts 4*Tq*keys*d*H",
-            "bf16_peak_TFLOP/s": pk.get("bf16_tflops"), **attn},
-        "ln_modulate_quantize": {
-            "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A, two launches, outside the step",
-            "ms": round(search["ln_quantize_ms"], 4),
-            "GB/s": round(quant_bytes / (search["ln_quantize_ms"] * 1e-3) / 1e9, 1)},
-        "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
-                "what": "pinned host A -> device, quantize, gemm+bias, C -> pinned host, every step; the copies "
-                        "run on their own streams (double-buffered) and overlap the neighbouring steps' compute"},
-        "gpu_launches": 4 * args.steps,  # quantize, GEMM, KV append, KV dequant per step
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, fp32 accumulate); bf16 input and QKV output",
+        "data": "synthetic (seeded N(0,1) activations with 0.1% x20 outlier channels, N(0,0.02) random-init "
+                "weights and biases)",
+        "config": {"workload": WORKLOAD, "layers": L, "M": M, "D": D, "F": F,
+                   "per_layer": "QKV 3072->9216 +bias (bf16 out, V third requantized) -> out 3072->3072 +bias "
+                                "requant -> up 3072->14336 +bias GELU requant -> down 14336->3072 +bias requant",
+                   "step": "nvfp4_quantize of the input + 4 nvfp4_gemm per layer",
+                   "parallelism": f"dp{world} (independent replicas, no collective)",
+                   "l2": "inputs larger than L2: every step streams 2.1 GB of NVFP4 weights and ~10 GB of "
+                         "activations through the 126 MB L2"},
+        "roofline": _rl("tensor", gemm_tflops, fp4_peak, "TFLOP/s",
+                        kernel="gemm_kernel (tcgen05 mxf4nvf4), all 4 GEMMs of a layer: 2*M*N*K per launch "
+                               "over the launches' mean duration",
+                        peak_source=f"{pk['source']} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16)",
+                        frac_of_nominal_9pf=round(gemm_tflops / NOMINAL_FP4_TFLOPS, 4),
+                        traffic=None if tr is None else tr.get("dram_bytes_per_launch")),
+        "roofline_by_kernel": by,
+        "components_ms": {k: round(v, 4) for k, v in comp.items()},
+        "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * D * 2,
+                "d2h_bytes_per_step": M * D // 2 + int(st.x.scales.numel()) + 4,
+                "what": "pinned host bf16 input -> device, quantize + the 30-layer stack, final NVFP4 output "
+                        "(codes, scales, tensor scale) -> pinned host, every step; copies on their own streams "
+                        "(double-buffered), overlapping the neighbouring steps' compute"},
+        "gpu_launches": st.launches_per_forward() * args.steps,
         "clocks": clk,
     }
+    if sub:
+        out.update(sub_report(sub, lin, pk, fp4_peak))
     return out
 
 
-# --------------------------------------------------------------------------- oracle
-def oracle_linear_rows(rows: int, w_codes, a_host, bias_host, seed_rows: int):
-    """Time the CPU oracle on `rows` rows of the QKV layer: quantize those rows
-    of A (with the full tensor scale), then their GEMM rows with bias."""
-    import oracle
-
+def sub_report(sub, lin, pk, fp4_peak) -> dict:
+    q_ms, g_ms, ap_ms, dq_ms = lin
     M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
-    sub = np.ascontiguousarray(a_host[:rows])
+    S, T, H, D = syn.KV_SLOTS, syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    flops = 2.0 * M * N * K
+    quant_bytes = M * K * 2.5625
+    kv_elems = T * H * D
+    append_bytes = 2 * kv_elems * 2.5625
+    dequant_bytes = 2 * S * kv_elems * (0.5625 + 2.0)
+    gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
+    search, train, attn, ffn = sub["search"], sub["train"], sub["attn"], sub["ffn"]
+    up, dn = syn.FFN_UP, syn.FFN_DOWN
+    return {
+        "linear_4096": {
+            "what": "config QKV: quantize A [4096x3072] per call + QKV GEMM 4096x9216x3072 + bias -> bf16, W "
+                    "pre-quantized; graph with events, the KV dequant's 681 MB output flushing L2 every step",
+            "TFLOP/s": round(flops / ((q_ms + g_ms) * 1e-3) / 1e12, 1),
+            "gemm": _rl("tensor", flops / (g_ms * 1e-3) / 1e12, fp4_peak, "TFLOP/s", ms=round(g_ms, 4)),
+            "quantize": _rl("hbm", gbs(quant_bytes, q_ms), pk["hbm_gbs"], "GB/s", ms=round(q_ms, 4))},
+        "kv": {
+            "what": "NVFP4 KV cache of 21 slots x 2640 x 24 x 128: append of one K/V chunk (in place into ring "
+                    "slot step mod 21), dequant-gather of all 21 slots to bf16",
+            "append": _rl("hbm", gbs(append_bytes, ap_ms), pk["hbm_gbs"], "GB/s", ms=round(ap_ms, 4)),
+            "dequant": _rl("hbm", gbs(dequant_bytes, dq_ms), pk["hbm_gbs"], "GB/s", ms=round(dq_ms, 4)),
+            "cache_bytes": sub["lk"]["cache"].nbytes()},
+        "scale_search": {
+            "what": "adaptive per-block scale search over the targets {4, 6}",
+            "quantize_ms": round(search["quantize_ms"], 4),
+            "quantize_GB/s": round(gbs(quant_bytes, search["quantize_ms"]), 1),
+            "kv_append_ms": round(search["kv_append_ms"], 4),
+            "kv_append_GB/s": round(gbs(append_bytes, search["kv_append_ms"]), 1)},
+        "kv_smoothing": {
+            "what": "KV append with K-smoothing of K and the scale search on K and V (channel means + quantize), "
+                    "and the dequant of all slots with the means added back",
+            "append_ms": round(search["smooth_append_ms"], 4),
+            "append_GB/s": round(gbs(append_bytes, search["smooth_append_ms"]), 1),
+            "dequant_ms": round(search["smooth_dequant_ms"], 4),
+            "dequant_GB/s": round(gbs(dequant_bytes, search["smooth_dequant_ms"]), 1)},
+        "kv_rope": {
+            "what": "KV append with the keys' rotary embedding fused ahead of their quantize (3-frame x 22 x 40 "
+                    "angle table), plain and with K-smoothing + scale search; GB/s of the append's bytes",
+            "append_ms": round(search["rope_append_ms"], 4),
+            "append_GB/s": round(gbs(append_bytes, search["rope_append_ms"]), 1),
+            "smooth_search_append_ms": round(search["rope_smooth_append_ms"], 4),
+            "smooth_search_append_GB/s": round(gbs(append_bytes, search["rope_smooth_append_ms"]), 1)},
+        "ffn_8192": {
+            "what": "config FFN: quantize A [8192x3072], up 3072->14336 with GELU and the NVFP4 requant of its "
+                    "output, down 14336->3072 to bf16 on that output; each 2*M*N*K = 721.6 GFLOP",
+            "quantize_ms": round(ffn["quantize_ms"], 4),
+            "up": _rl("tensor", 2 * up.M * up.N * up.K / (ffn["up_ms"] * 1e-3) / 1e12, fp4_peak, "TFLOP/s",
+                      ms=round(ffn["up_ms"], 4)),
+            "down": _rl("tensor", 2 * dn.M * dn.N * dn.K / (ffn["down_ms"] * 1e-3) / 1e12, fp4_peak, "TFLOP/s",
+                        ms=round(ffn["down_ms"], 4))},
+        "training": {
+            "what": "training-side NVFP4 on the QKV layer shapes: 2D (16x16) scaling of W [9216x3072] writing W "
+                    "and W^T operands; RHT + transposed 1D quantize of X [4096x3072] and dY [4096x9216]; "
+                    "dW = dY^T X (9216x3072x4096) on those operands",
+            "quantize_2d_ms": round(train["quantize_2d_ms"], 4),
+            "quantize_2d_GB/s": round(gbs(N * K * 3.125, train["quantize_2d_ms"]), 1),
+            "quantize_t_x_ms": round(train["quantize_t_x_ms"], 4),
+            "quantize_t_x_GB/s": round(gbs(M * K * 2.5625, train["quantize_t_x_ms"]), 1),
+            "quantize_t_dy_ms": round(train["quantize_t_dy_ms"], 4),
+            "quantize_t_dy_GB/s": round(gbs(M * N * 2.5625, train["quantize_t_dy_ms"]), 1),
+            "wgrad_ms": round(train["wgrad_ms"], 4),
+            "wgrad_TFLOP/s": round(2.0 * N * K * M / (train["wgrad_ms"] * 1e-3) / 1e12, 1)},
+        "kv_attention": {
+            "what": "softmax attention of one 2640x24x128 bf16 query chunk over NVFP4 cache slots read directly; "
+                    "TFLOP/s counts 4*Tq*keys*d*H", "bf16_peak_TFLOP/s": pk.get("bf16_tflops"), **attn},
+        "ln_modulate_quantize": {
+            "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A [4096x3072]",
+            "ms": round(search["ln_quantize_ms"], 4),
+            "GB/s": round(gbs(quant_bytes, search["ln_quantize_ms"]), 1)},
+    }
+
+
+# --------------------------------------------------------------------------- oracle
+def _timed(f):
     t0 = time.perf_counter()
-    codes, scales, a32 = oracle.quantize(sub)
-    oracle.gemm((codes, scales, a32), w_codes, bias=bias_host, want_bf16=True)
+    f()
     return time.perf_counter() - t0
 
 
-def cpu_baseline(steps: int = 1, rows: int = 8) -> dict:
+def oracle_stack_rows(rows: int, layer_w, x_rows_bits):
+    """The oracle on `rows` token rows through one layer of the stack: the
+    quantize of those input rows, then the four fp64 GEMMs with their epilogues
+    and the binary32 requants between them (output scales from the rows
+    themselves).  Returns seconds."""
     import oracle
 
-    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
-    a_host = syn.activations_bf16(M, K, seed=2)
-    w_host = syn.normal_bf16((N, K), seed=3, std=0.02)
-    bias_host = syn.normal_bf16((N,), seed=4, std=0.02)
-    wq = oracle.quantize(w_host)
-    ts = [oracle_linear_rows(rows, wq, a_host, bias_host, i) for i in range(steps)]
-    t = min(ts)
-    return {"value": round(2.0 * rows * N * K / t / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
-            "kind": "oracle", "host_cores": os.cpu_count(),
-            "sample": f"{rows} of {M} token rows of the QKV layer per step (quantize rows + fp64 GEMM rows + bias)",
-            "seconds_per_step": round(t, 3)}
+    def run():
+        codes, scales, a32 = oracle.quantize(x_rows_bits)
+        a = (codes, scales, a32)
+        D = x_rows_bits.shape[1]
+        for g, (w, b) in enumerate(layer_w):
+            y, _ = oracle.gemm(a, w, bias=b, act=1 if g == 2 else 0, want_bf16=False)
+            if g == 0:
+                y = y[:, 2 * D:]
+            y = np.ascontiguousarray(y.astype(np.float32))
+            a = oracle.quantize(y)
+    return _timed(run)
+
+
+def oracle_layer_weights(layer: int):
+    import oracle
+
+    D, F = syn.STACK_LAYER[0].K, syn.STACK_LAYER[2].N
+    w, b = syn.stack_layer_bf16(layer, D, F)
+    return [(oracle.quantize(w[n]), b[n]) for n in STACK_NAMES]
+
+
+def cpu_baseline(rows: int = 4) -> dict:
+    """The oracle on the host cores: the stack's rate on `rows` token rows of
+    one layer (the headline's sample, extrapolated to the full stack), and the
+    codec work of the KV workload and the activation quantize timed in full."""
+    import oracle
+
+    D = syn.STACK_LAYER[0].K
+    lw = oracle_layer_weights(0)
+    x = syn.activations_bf16(rows, D, seed=80)
+    t = oracle_stack_rows(rows, lw, x)
+    per_row = 2.0 * (3 * D * D + D * D + 2 * syn.STACK_LAYER[2].N * D)
+    value = rows * per_row / t / 1e12
+    full_stack_s = syn.STACK_LAYERS * syn.STACK_M * per_row / (value * 1e12)
+    # codec work in full: quantize of A [4096 x 3072], a KV append of one chunk, the dequant of 21 slots
+    M, K = syn.QKV.M, syn.QKV.K
+    a = syn.activations_bf16(M, K, seed=2)
+    tq = _timed(lambda: oracle.quantize(a))
+    T, H, Dh = syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    k, v = syn.kv_chunk_bf16(T, H, Dh, seed=50)
+    res = {}
+    ta = _timed(lambda: res.update(k=oracle.kv_append(k), v=oracle.kv_append(v)))
+    td = _timed(lambda: [oracle.kv_dequant(*res["k"], T, H, Dh) for _ in range(syn.KV_SLOTS)] +
+                [oracle.kv_dequant(*res["v"], T, H, Dh) for _ in range(syn.KV_SLOTS)])
+    kv_elems = T * H * Dh
+    return {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "host_cores": os.cpu_count(),
+            "sample": f"{rows} of {syn.STACK_M} token rows through one layer of the stack (input quantize, 4 fp64 "
+                      "GEMMs with epilogues, 4 binary32 requants)",
+            "extrapolated_full_stack_s": round(full_stack_s, 1),
+            "codecs_in_full": {
+                "quantize_4096x3072_GB/s": round(M * K * 2.5625 / tq / 1e9, 4),
+                "kv_append_GB/s": round(2 * kv_elems * 2.5625 / ta / 1e9, 4),
+                "kv_dequant_21_slots_GB/s": round(2 * syn.KV_SLOTS * kv_elems * 2.5625 / td / 1e9, 4),
+                "seconds": round(tq + ta + td, 2)}}
 
 
 def run_reference(args) -> dict:
+    """--impl reference: the oracle, as it stands, on the stack's metric: each
+    step one layer (cycling over two seeded layers) on a few token rows."""
     import oracle
 
-    M, N, K = syn.QKV.M, syn.QKV.N, syn.QKV.K
-    rows = 8
-    a_host = syn.activations_bf16(M, K, seed=2)
-    w_host = syn.normal_bf16((N, K), seed=3, std=0.02)
-    bias_host = syn.normal_bf16((N,), seed=4, std=0.02)
-    wq = oracle.quantize(w_host)
+    D = syn.STACK_LAYER[0].K
+    rows = 4
+    lws = [oracle_layer_weights(l) for l in range(2)]
+    x = syn.activations_bf16(rows, D, seed=80)
     for i in range(args.warmup):
-        oracle_linear_rows(rows, wq, a_host, bias_host, i)
-    t = 0.0
-    for i in range(args.steps):
-        t += oracle_linear_rows(rows, wq, a_host, bias_host, i)
-    value = args.steps * 2.0 * rows * N * K / t / 1e12
-    cb = {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(), "kind": "oracle",
-          "sample": f"{rows} of {M} token rows of the QKV layer per step (quantize rows + fp64 GEMM rows + bias)"}
+        oracle_stack_rows(rows, lws[i % 2], x)
+    t = sum(oracle_stack_rows(rows, lws[i % 2], x) for i in range(args.steps))
+    per_row = 2.0 * (3 * D * D + D * D + 2 * syn.STACK_LAYER[2].N * D)
+    value = args.steps * rows * per_row / t / 1e12
+    sample = (f"{rows} of {syn.STACK_M} token rows through one layer of the stack per step (layers 0 and 1 in turn): "
+              "input quantize, 4 fp64 GEMMs with epilogues, 4 binary32 requants")
     return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 GEMM over NVFP4 operands; f32 quantize",
             "data": "synthetic (seeded, same generators as the GPU arm)", "impl": "reference",
-            "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "parallelism": "cpu oracle, rank 0"},
-            "cpu_baseline": cb,
+            "config": {"workload": WORKLOAD, "layers": syn.STACK_LAYERS, "M": syn.STACK_M,
+                       "parallelism": "cpu oracle, rank 0"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -741,6 +888,10 @@ def main(argv=None) -> int:
     ap.add_argument("--ffn-only", action="store_true",
                     help="time only the 8192-token FFN pair (under 1 GB on the device: the small case for "
                          "profiling its GEMMs) and print its numbers")
+    ap.add_argument("--layers", type=int, default=syn.STACK_LAYERS,
+                    help="layers of the stack (default 30, the workload; fewer only for profiling)")
+    ap.add_argument("--stack-only", action="store_true",
+                    help="time the stack alone (skip the single-layer, KV and next-row measurements)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -776,6 +927,8 @@ def main(argv=None) -> int:
         if rank == 0 and out is not None:
             if not args.no_cpu_baseline and world == 1:
                 out["cpu_baseline"] = cpu_baseline()
+            if args.layers != syn.STACK_LAYERS:
+                out["config"]["workload"] = f"dit_stack_{args.layers}x4_16384 (reduced: not the workload)"
             print(json.dumps(out), flush=True)
     finally:
         if world > 1:

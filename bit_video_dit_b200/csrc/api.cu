@@ -4,11 +4,14 @@
 
 namespace {
 // Every call's workspace starts with a 256-byte control block: the device
-// error record (bytes 0..15) and, for quantize / KV append, the launch epoch
-// of the fused kernel, which then keeps one 64-bit slot per CTA (1024 x 8
-// bytes) after the block.
+// error record (bytes 0..15) and, for quantize / KV append, the fused
+// kernel's grid-barrier words (the launch epoch at word 8, the two arrival
+// counters at words 16..17, the per-parity tensor maxima at words 20..23).
+// Nothing follows the block for those calls: their whole workspace is 256
+// bytes, which is also what the no-allocation quantize keeps in its static
+// array.  The LayerNorm quantize keeps its row statistics after the block.
 constexpr size_t kWsControl = 256;
-constexpr size_t kWsQuantize = kWsControl;  // the grid-barrier words live in the control block
+constexpr size_t kWsQuantize = kWsControl;
 }
 
 extern "C" const char* nvfp4_status_string(nvfp4_status s) {

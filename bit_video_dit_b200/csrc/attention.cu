@@ -533,12 +533,19 @@ extern "C" nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const in
     // caches without smoothing means take the binary16 path
     const bool raw = !sk && !sv;
     void (*kern)(AttnArgs) = raw ? kv_attention_kernel<true> : kv_attention_kernel<false>;
-    static bool attr[2] = {false, false};
-    if (!attr[raw]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    // the shared-memory attribute of both variants, set once per device
+    static PerDevice<bool> attr_set;
+    bool done = false;
+    const nvfp4_status ast = attr_set.get(&done, [smem](int, bool& v) {
+        if (cudaFuncSetAttribute(kv_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kv_attention_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
             return NVFP4_ERR_CUDA;
-        attr[raw] = true;
-    }
+        v = true;
+        return NVFP4_OK;
+    });
+    if (ast != NVFP4_OK) return ast;
     const dim3 grid((unsigned)((tq + kTile - 1) / kTile), (unsigned)cache->heads);
     kern<<<grid, kThreads, smem, (cudaStream_t)stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

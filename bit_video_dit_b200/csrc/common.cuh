@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/nvfp4.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -16,6 +18,43 @@
 #endif
 
 namespace nvfp4 {
+
+// ---------------------------------------------------------------------------
+// Host: a value kept per device (SM counts, occupancy, kernel attributes set),
+// filled on the first call made with that device current and shared by every
+// host thread.  A fill that fails is not kept, so the next call retries it.
+// ---------------------------------------------------------------------------
+template <class T>
+class PerDevice {
+  public:
+    // *out = the current device's value; init(dev, T&) -> nvfp4_status fills it once
+    template <class F>
+    nvfp4_status get(T* out, F&& init) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+        if (dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_UNSUPPORTED;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (!ok_[dev]) {
+            T v{};
+            const nvfp4_status st = init(dev, v);
+            if (st != NVFP4_OK) return st;
+            val_[dev] = v;
+            ok_[dev] = true;
+        }
+        *out = val_[dev];
+        return NVFP4_OK;
+    }
+
+  private:
+    static constexpr int kMaxDevices = 64;
+    std::mutex mu_;
+    T val_[kMaxDevices]{};
+    bool ok_[kMaxDevices]{};
+};
+
+// Host: nvfp4_quantize's argument checks other than the workspace's (quantize.cu).
+nvfp4_status quantize_check_args(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, const void* codes,
+                                 const void* scales, const float* global_scale, unsigned flags);
 
 // ---------------------------------------------------------------------------
 // Device error record: the first 16 bytes of every call's workspace.

@@ -133,6 +133,7 @@ struct Params {
     uint8_t* out_codes;
     uint8_t* out_scales;
     const float* out_gscale;
+    int q_col0, q_col1;  // requant / out_amax window [q_col0, q_col1): multiples of 64 (requant)
     float* out_amax;
     float* debug_y;
     DevError* err;
@@ -410,7 +411,11 @@ __device__ __forceinline__ void smem_vec32(const uint32_t* v, float* out) {
 
 // One 32-column chunk of one output row: epilogue math and outputs.  `r`
 // holds the accumulator (binary32 bits), `vec` the tile's staged vectors
-// (at this chunk's columns), `stage` this warp's staging buffer.
+// (at this chunk's columns), `stage` this warp's staging buffer.  The NVFP4
+// requant and out_amax cover the column window [q_col0, q_col1) only (its
+// ends are multiples of 64 when requantizing, so a chunk is inside or
+// outside it as a whole); requant column n lands at n - q_col0 of an
+// [M x (q_col1 - q_col0)] operand with tiles_on scale tiles along its row.
 __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* r, float alpha, int64_t m, bool row_ok,
                                                int64_t n0, int valid, float oa32, int64_t tiles_on, float& amax_run,
                                                const uint32_t* const* vec, uint8_t* stage, int lane) {
@@ -447,10 +452,12 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
 #pragma unroll
         for (int i = 0; i < 32; i++) y[i] = v[i] + y[i];
     }
-    if (p.out_amax && row_ok) {
+    const bool in_win = n0 >= p.q_col0 && n0 < p.q_col1;
+    if (p.out_amax && row_ok && in_win) {
+        const int wv = (int)min((int64_t)valid, (int64_t)p.q_col1 - n0);
 #pragma unroll
         for (int i = 0; i < 32; i++)
-            if (i < valid) amax_run = fmaxf(amax_run, fabsf(y[i]));
+            if (i < wv) amax_run = fmaxf(amax_run, fabsf(y[i]));
     }
     if (p.debug_y && row_ok) {
         float* d = p.debug_y + m * p.N + n0;
@@ -472,9 +479,10 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
         for (int u = 0; u < 4; u++)
             *reinterpret_cast<uint4*>(row + ((u ^ sw) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     }
-    if (p.out_codes) {
-        // N % 64 == 0 for requant, so a 32-column chunk is whole
-        const int64_t bj = n0 / 16;
+    if (p.out_codes && in_win) {
+        // the window's ends are multiples of 64, so a 32-column chunk inside it is whole
+        const int64_t nq = n0 - p.q_col0;
+        const int64_t bj = nq / 16;
         uint16_t sc2 = 0;
         if (row_ok) {
             float am0 = 0.0f, am1 = 0.0f;
@@ -487,7 +495,7 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
             const BlockScale b1 = block_scale(am1, oa32);
             const uint4 w = make_uint4(encode8(y, b0.inv), encode8(y + 8, b0.inv), encode8(y + 16, b1.inv),
                                        encode8(y + 24, b1.inv));
-            *reinterpret_cast<uint4*>(p.out_codes + m * (p.N / 2) + n0 / 2) = w;
+            *reinterpret_cast<uint4*>(p.out_codes + m * ((p.q_col1 - p.q_col0) / 2) + nq / 2) = w;
             sc2 = (uint16_t)(b0.code | (b1.code << 8));
         }
         // rows past M up to the next multiple of 128 are scale padding: zero
@@ -506,7 +514,7 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
     const int et = (warp - 2) * 32 + lane;  // 0..127 over the epilogue warps
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
     const float oa32 = p.out_codes ? __ldg(p.out_gscale) : 0.0f;
-    const int64_t tiles_on = (p.N + 63) / 64;  // scale tiles along N of the output
+    const int64_t tiles_on = ((int64_t)(p.q_col1 - p.q_col0) + 63) / 64;  // scale tiles along the requant window
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     // the leader's MMA waits for the epilogue warps of both CTAs
     const uint32_t empty_bar = PAIR ? mapa_shared(smem_u32(&s->tmem_empty), 0) : smem_u32(&s->tmem_empty);
@@ -715,23 +723,28 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-static EncodeTiledFn g_encode_tiled = nullptr;
-static int g_gemm_dev = -1;
-static int g_gemm_sms = 0;
-static int g_gemm_pair_clusters = 0;
+static EncodeTiledFn g_encode_tiled = nullptr;  // driver entry point, looked up once per process
+static std::once_flag g_encode_once;
+
+struct GemmDevice {
+    int sms;
+    int pair_clusters;
+};
+static PerDevice<GemmDevice> g_gemm_dev;
 
 static nvfp4_status gemm_setup(int& sms, int& pair_clusters) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (g_encode_tiled == nullptr) {
+    std::call_once(g_encode_once, [] {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess || fn == nullptr)
-            return NVFP4_ERR_CUDA;
-        g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
-    }
-    if (g_gemm_dev != dev) {
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && fn != nullptr)
+            g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
+        else
+            cudaGetLastError();
+    });
+    if (g_encode_tiled == nullptr) return NVFP4_ERR_CUDA;
+    GemmDevice gd{};
+    const nvfp4_status st = g_gemm_dev.get(&gd, [](int dev, GemmDevice& v) {
         int major = 0, minor = 0, n = 0;
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
@@ -763,12 +776,13 @@ static nvfp4_status gemm_setup(int& sms, int& pair_clusters) {
             cudaGetLastError();
             clusters = 0;  // pair variant unavailable: single-CTA tiles only
         }
-        g_gemm_sms = n;
-        g_gemm_pair_clusters = clusters;
-        g_gemm_dev = dev;
-    }
-    sms = g_gemm_sms;
-    pair_clusters = g_gemm_pair_clusters;
+        v.sms = n;
+        v.pair_clusters = clusters;
+        return NVFP4_OK;
+    });
+    if (st != NVFP4_OK) return st;
+    sms = gd.sms;
+    pair_clusters = gd.pair_clusters;
     return NVFP4_OK;
 }
 
@@ -831,7 +845,11 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
     const bool requant = ep && ep->out_codes;
     if (!c_bf16 && !requant) return NVFP4_ERR_INVALID_ARG;
     if (requant && (!ep->out_scales || !ep->out_global_scale)) return NVFP4_ERR_INVALID_ARG;
-    if (requant && N % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
+    // the requant / out_amax column window (out_cols == 0: all N columns)
+    const int64_t win0 = ep ? ep->out_col0 : 0;
+    const int64_t wcols = (ep && ep->out_cols) ? ep->out_cols : N - win0;
+    if (win0 < 0 || wcols <= 0 || win0 + wcols > N) return NVFP4_ERR_INVALID_ARG;
+    if (requant && (win0 % 64 != 0 || wcols % 64 != 0)) return NVFP4_ERR_UNSUPPORTED;
     if (ep && ep->act != NVFP4_ACT_NONE && ep->act != NVFP4_ACT_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
     if (ep && (ep->debug_flags & ~NVFP4_DBG_SKIP_LOADS)) return NVFP4_ERR_INVALID_ARG;
     if (ep && ep->residual && ep->ld_residual < N) return NVFP4_ERR_INVALID_ARG;
@@ -889,11 +907,15 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
         p.out_scales = static_cast<uint8_t*>(ep->out_scales);
         p.out_gscale = ep->out_global_scale;
         p.out_amax = ep->out_amax;
+        p.q_col0 = (int)win0;
+        p.q_col1 = (int)(win0 + wcols);
         p.debug_y = ep->debug_y;
         p.dbg = ep->debug_flags;
         p.limit_ns = (uint64_t)(ep->wait_limit_us ? ep->wait_limit_us : 2000000u) * 1000ull;
     } else {
         p.limit_ns = 2000000000ull;
+        p.q_col0 = 0;
+        p.q_col1 = (int)N;
     }
     p.err = static_cast<DevError*>(workspace);
     // short K (at most 16 stages per tile): the epilogue bounds the tile rate,

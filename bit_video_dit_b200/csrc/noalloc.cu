@@ -49,8 +49,13 @@ nvfp4_status scratch_for_current_device(void** out) {
 extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                                void* codes, void* scales, float* global_scale, unsigned flags,
                                                nvfp4_stream_t stream) {
-    if (rows < 0 || cols <= 0) return NVFP4_ERR_INVALID_ARG;
+    // every argument check first: a rejected call puts nothing on the stream
+    // and leaves the shared array alone (another stream may be using it)
+    const nvfp4_status chk = nvfp4::quantize_check_args(x_bf16, rows, cols, ld, codes, scales, global_scale, flags);
+    if (chk != NVFP4_OK) return chk;
+    if (rows == 0) return NVFP4_OK;
     if (nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols) > kNoAllocScratchBytes) return NVFP4_ERR_UNSUPPORTED;
+    if (rows * ((cols + 511) / 512) > ((int64_t)1 << 30) || cols > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
     void* scratch = nullptr;
     const nvfp4_status st = scratch_for_current_device(&scratch);
     if (st != NVFP4_OK) return st;

@@ -865,18 +865,23 @@ __global__ void encoder_probe_kernel(const float* x, int64_t n, uint8_t* e2m1, u
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static int g_sms = 0;
+static PerDevice<int> g_sms;
 
+// SMs of the current device (148 on B200 if the query fails)
 static int num_sms() {
-    if (g_sms == 0) {
-        int dev = 0, n = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-            g_sms = n;
-        else
-            return 148;
-    }
-    return g_sms;
+    int n = 0;
+    const nvfp4_status st = g_sms.get(&n, [](int dev, int& v) {
+        return cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? NVFP4_OK
+                                                                                               : NVFP4_ERR_CUDA;
+    });
+    return st == NVFP4_OK && n > 0 ? n : 148;
 }
+
+// resident 256-thread blocks per SM of the two dequant kernels on the current device
+struct DequantResidency {
+    int blocks[2];
+};
+static PerDevice<DequantResidency> g_dequant_resident;
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -969,20 +974,36 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
 
 using namespace nvfp4;
 
-extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
-                                       void* scales, float* global_scale, unsigned flags, void* workspace,
-                                       size_t ws_bytes, nvfp4_stream_t stream) {
+namespace nvfp4 {
+// nvfp4_quantize's argument checks apart from the workspace (shared with the
+// no-allocation entry point, which must run them before touching its scratch).
+nvfp4_status quantize_check_args(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, const void* codes,
+                                 const void* scales, const float* global_scale, unsigned flags) {
     if (flags & ~(NVFP4_Q_GIVEN_GLOBAL | NVFP4_Q_ROWMAJOR_SCALES | NVFP4_Q_SCALE_SEARCH)) return NVFP4_ERR_INVALID_ARG;
     if (rows < 0 || cols <= 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
     if (cols % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
     if (rows > ((int64_t)1 << 31) || cols > ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED;
-    if (!global_scale || !workspace) return NVFP4_ERR_INVALID_ARG;
-    if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols)) return NVFP4_ERR_INVALID_ARG;
+    if (!global_scale) return NVFP4_ERR_INVALID_ARG;
     if (rows == 0) return NVFP4_OK;
     if (!x_bf16 || !codes || !scales) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales) || (ld % 8) != 0 ||
-        (reinterpret_cast<uintptr_t>(global_scale) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u))
         return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+}  // namespace nvfp4
+
+extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
+                                       void* scales, float* global_scale, unsigned flags, void* workspace,
+                                       size_t ws_bytes, nvfp4_stream_t stream) {
+    const nvfp4_status chk = quantize_check_args(x_bf16, rows, cols, ld, codes, scales, global_scale, flags);
+    if (chk != NVFP4_OK) return chk;
+    if (!workspace) return NVFP4_ERR_INVALID_ARG;
+    if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols)) return NVFP4_ERR_INVALID_ARG;
+    if (rows == 0) return NVFP4_OK;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return NVFP4_ERR_MISALIGNED;
+    // the row and run counts the kernel indexes in 32 bits (also refused inside quantize_impl)
+    if (rows * ((cols + 511) / 512) > ((int64_t)1 << 30) || cols > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
     const void* xs[1] = {x_bf16};
     void* cs[1] = {codes};
     void* ss[1] = {scales};
@@ -1152,15 +1173,23 @@ extern "C" nvfp4_status nvfp4_kv_dequant(const nvfp4_kv_cache* cache, const int3
         a.hd = cache->heads * cache->head_dim;
     }
     // one resident wave over K and V together (blockIdx.y picks the tensor)
-    static int resident[2] = {0, 0};
     void (*kern)(DequantArgs) = smooth ? kv_dequant_kernel<true> : kv_dequant_kernel<false>;
-    if (resident[smooth] == 0) {
-        int b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, 0) != cudaSuccess || b < 2) b = 2;
-        resident[smooth] = b;
-    }
+    DequantResidency res{};
+    st = g_dequant_resident.get(&res, [](int, DequantResidency& v) {
+        for (int sm = 0; sm < 2; sm++) {
+            int b = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, sm ? kv_dequant_kernel<true> : kv_dequant_kernel<false>,
+                                                              kThreads, 0) != cudaSuccess || b < 2) {
+                cudaGetLastError();
+                b = 2;
+            }
+            v.blocks[sm] = b;
+        }
+        return NVFP4_OK;
+    });
+    if (st != NVFP4_OK) return st;
     const int64_t units = (int64_t)n * ((a.slot_elems + 511) / 512);
-    const int g = grid_for(units, 2 * (kThreads / 32), num_sms() * resident[smooth] / 2);
+    const int g = grid_for(units, 2 * (kThreads / 32), num_sms() * res.blocks[smooth] / 2);
     kern<<<dim3(g, 2), kThreads, 0, (cudaStream_t)stream>>>(a);
     return launch_status();
 }

@@ -225,15 +225,21 @@ using namespace nvfp4::train;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+PerDevice<int> g_train_sms;
+
+// SMs of the current device (148 on B200 if the query fails)
 int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            n = 148;
-    }
-    return n;
+    int n = 0;
+    const nvfp4_status st = g_train_sms.get(&n, [](int dev, int& v) {
+        return cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? NVFP4_OK
+                                                                                               : NVFP4_ERR_CUDA;
+    });
+    return st == NVFP4_OK && n > 0 ? n : 148;
 }
+
+struct TrainResidency {
+    int blocks[2];  // resident blocks per SM of the amax pass and of the encode pass
+};
 
 // Zero a swizzled scale buffer when its layout has padding rows (rows not a
 // multiple of 128): the kernels write only real rows.
@@ -248,15 +254,23 @@ nvfp4_status run(TrainArgs& a, cudaStream_t s) {
     a.tiles_c = (a.cols + 63) / 64;
     a.ntiles = (a.rows / kTileRows) * a.tiles_c;
     const int64_t want = ((int64_t)a.ntiles + kWarps - 1) / kWarps;
-    // one resident wave of each pass (blocks per SM from the occupancy query)
-    static int resident[2] = {0, 0};
-    for (int e = 0; e < 2; e++)
-        if (resident[e] == 0) {
+    // one resident wave of each pass (blocks per SM from the occupancy query, per device)
+    static PerDevice<TrainResidency> g_resident;
+    TrainResidency res{};
+    const nvfp4_status rst = g_resident.get(&res, [](int, TrainResidency& v) {
+        for (int e = 0; e < 2; e++) {
             int b = 0;
             auto k = e ? train_quant_kernel<TWO_D, RHT, true> : train_quant_kernel<TWO_D, RHT, false>;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, kThreads, 0) != cudaSuccess || b < 1) b = 1;
-            resident[e] = b;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, kThreads, 0) != cudaSuccess || b < 1) {
+                cudaGetLastError();
+                b = 1;
+            }
+            v.blocks[e] = b;
         }
+        return NVFP4_OK;
+    });
+    if (rst != NVFP4_OK) return rst;
+    const int* resident = res.blocks;
     if (!a.given) {
         if (cudaMemsetAsync(a.amax_word, 0, 4, s) != cudaSuccess) return NVFP4_ERR_CUDA;
         const int g = (int)std::min<int64_t>(want, (int64_t)sm_count() * resident[0]);

@@ -47,7 +47,8 @@ class CEpilogue(ctypes.Structure):
                 ("gate", ctypes.c_void_p), ("residual", ctypes.c_void_p), ("ld_residual", ctypes.c_int64),
                 ("act", ctypes.c_int), ("out_codes", ctypes.c_void_p), ("out_scales", ctypes.c_void_p),
                 ("out_global_scale", ctypes.c_void_p), ("out_amax", ctypes.c_void_p),
-                ("debug_y", ctypes.c_void_p), ("debug_flags", ctypes.c_uint), ("wait_limit_us", ctypes.c_uint32)]
+                ("debug_y", ctypes.c_void_p), ("debug_flags", ctypes.c_uint), ("wait_limit_us", ctypes.c_uint32),
+                ("out_col0", ctypes.c_int64), ("out_cols", ctypes.c_int64)]
 
 
 class CKVCache(ctypes.Structure):
@@ -292,28 +293,32 @@ def ln_modulate_quantize(x: torch.Tensor, *, mod_scale: torch.Tensor | None = No
 
 def make_epilogue(*, bias=None, mod_scale=None, mod_shift=None, gate=None, residual=None, act: int = ACT_NONE,
                   requant: NVFP4Tensor | None = None, out_amax=None, debug_y=None, debug_flags: int = 0,
-                  wait_limit_us: int = 0) -> CEpilogue:
+                  wait_limit_us: int = 0, out_window: tuple[int, int] | None = None) -> CEpilogue:
+    col0, cols = out_window if out_window is not None else (0, 0)
     return CEpilogue(_ptr(bias), _ptr(mod_scale), _ptr(mod_shift), _ptr(gate), _ptr(residual),
                      0 if residual is None else residual.stride(0), int(act),
                      None if requant is None else requant.codes.data_ptr(),
                      None if requant is None else requant.scales.data_ptr(),
                      None if requant is None else requant.global_scale.data_ptr(),
-                     _ptr(out_amax), _ptr(debug_y), int(debug_flags), int(wait_limit_us))
+                     _ptr(out_amax), _ptr(debug_y), int(debug_flags), int(wait_limit_us), int(col0), int(cols))
 
 
 def gemm(a: NVFP4Tensor, b: NVFP4Tensor, *, out: torch.Tensor | None = None, bias=None, mod_scale=None,
          mod_shift=None, gate=None, residual=None, act: int = ACT_NONE, requant: NVFP4Tensor | None = None,
          out_amax=None, debug_y=None, debug_flags: int = 0, wait_limit_us: int = 0, bf16_out: bool = True,
-         ws: torch.Tensor | None = None, stream=None) -> torch.Tensor | None:
+         out_window: tuple[int, int] | None = None, ws: torch.Tensor | None = None,
+         stream=None) -> torch.Tensor | None:
     """C[M, N] = a32_A a32_B (A . S_A)(B . S_B)^T -> epilogue -> bf16 `out`
-    and/or NVFP4 `requant` (whose global_scale holds the output tensor scale)."""
+    and/or NVFP4 `requant` (whose global_scale holds the output tensor scale).
+    out_window = (col0, cols): the requant and out_amax cover columns
+    col0 .. col0 + cols - 1 only (requant is then an [M, cols] operand)."""
     M, N = a.rows, b.rows
     dev = a.codes.device
     if out is None and bf16_out:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ep = make_epilogue(bias=bias, mod_scale=mod_scale, mod_shift=mod_shift, gate=gate, residual=residual, act=act,
                        requant=requant, out_amax=out_amax, debug_y=debug_y, debug_flags=debug_flags,
-                       wait_limit_us=wait_limit_us)
+                       wait_limit_us=wait_limit_us, out_window=out_window)
     if ws is None:
         ws = workspace(OP_GEMM, M, N, a.cols, dev)
     ca, cb = a.c(), b.c()

@@ -19,11 +19,11 @@ import numpy as np
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round binary32 values to bf16 (nearest-even) and return the uint16 bits."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return r.astype(np.uint16)
+    """Round finite binary32 values to bf16 (nearest-even) and return the uint16
+    bits (32-bit arithmetic: the largest finite pattern plus the rounding
+    increment stays below 2^32)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_bits_to_f32(h: np.ndarray) -> np.ndarray:
@@ -37,6 +37,42 @@ def rng(seed: int) -> np.random.Generator:
 def normal_bf16(shape, seed: int, std: float = 1.0) -> np.ndarray:
     g = rng(seed)
     return f32_to_bf16_bits((g.standard_normal(size=shape, dtype=np.float32) * np.float32(std)))
+
+
+_BLOCK_ROWS = 1024
+
+
+def normal_bf16_blocks(shape, seed: int, std: float = 1.0, threads: int | None = None) -> np.ndarray:
+    """N(0, std^2) bf16 bits [rows, cols] for large tensors: row block i (1024
+    rows) is drawn from its own PCG64 stream seeded with (seed, i), blocks in
+    parallel threads; the result depends only on (shape, seed, std)."""
+    import concurrent.futures as cf
+    import os
+
+    rows, cols = shape
+    out = np.empty((rows, cols), np.uint16)
+
+    def fill(i):
+        r0, r1 = i * _BLOCK_ROWS, min(rows, (i + 1) * _BLOCK_ROWS)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, i])))
+        x = g.standard_normal(size=(r1 - r0, cols), dtype=np.float32)
+        x *= np.float32(std)
+        out[r0:r1] = f32_to_bf16_bits(x)
+
+    n = -(-rows // _BLOCK_ROWS)
+    with cf.ThreadPoolExecutor(max_workers=threads or min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(n)))
+    return out
+
+
+def stack_layer_bf16(layer: int, D: int = 3072, F: int = 14336):
+    """One layer of the DiT linear stack: weights N(0, 0.02) of the QKV
+    [3D x D], out-projection [D x D], FFN up [F x D] and FFN down [D x F]
+    linears and their N(0, 0.02) biases, as bf16 bits, seeded by the layer."""
+    names = (("qkv", 3 * D, D), ("out", D, D), ("up", F, D), ("down", D, F))
+    w = {n: normal_bf16_blocks((r, c), seed=10_000 + 8 * layer + i, std=0.02) for i, (n, r, c) in enumerate(names)}
+    b = {n: normal_bf16((r,), seed=20_000 + 8 * layer + i, std=0.02) for i, (n, r, _) in enumerate(names)}
+    return w, b
 
 
 def activations_bf16(rows: int, cols: int, seed: int, outlier_frac: float = 0.001,

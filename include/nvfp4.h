@@ -180,9 +180,14 @@ nvfp4_status nvfp4_ln_modulate_quantize(const void* x_bf16, int64_t rows, int64_
  * up the array's device address (cudaGetSymbolAddress), so make that first
  * call before any stream capture.  Each call clears the array (one
  * cudaMemsetAsync on `stream`) and then launches the quantize kernel; it
- * allocates nothing.  All calls share the array, so calls that can overlap
- * on the GPU (different streams, different host threads) race: order them on
- * one stream.  Errors found on the device are not reported by this call. */
+ * allocates nothing.  Every argument check runs before the clear, so a
+ * rejected call enqueues nothing and leaves the array alone.  All calls share
+ * the array, so calls that can overlap on the GPU (different streams,
+ * different host threads) race: order them on one stream.  Errors found on
+ * the device are not reported by this call: if the kernel's bounded
+ * grid-barrier wait ever ran out, it would return without writing the codes,
+ * scales or tensor scale, leaving those outputs as they were, and the next
+ * call's clear erases the record. */
 #define NVFP4_NOALLOC_SCRATCH_BYTES 256
 nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld, void* codes,
                                     void* scales, float* global_scale, unsigned flags, nvfp4_stream_t stream);
@@ -209,10 +214,14 @@ typedef struct {
  *   y += bias[n];  y = act(y);  y = y * (1 + mod_scale[n]) + mod_shift[n];
  *   y = gate[n] * y;  y = residual[m, n] + y
  * (each step skipped when its pointer is NULL / act is NONE).  Then y is
- * stored as bf16 to c (if non-NULL) and/or re-quantized to NVFP4 with the
- * given output tensor scale (if out_codes is non-NULL): blocks of 16 along N,
- * swizzled scales for an [M x N] operand, exactly the quantize rule above.
- * out_amax (optional) receives atomically max(|y|) over the output, for
+ * stored as bf16 to c (if non-NULL; every column) and/or re-quantized to
+ * NVFP4 with the given output tensor scale (if out_codes is non-NULL):
+ * blocks of 16 along N, exactly the quantize rule above, over the column
+ * window [out_col0, out_col0 + out_cols) (out_cols == 0: every column from
+ * out_col0 on; both multiples of 64 for a requant), written as an
+ * [M x out_cols] operand: codes [M x out_cols/2], swizzled scales.  A DiT
+ * QKV projection can so hand its V third straight to the next GEMM.
+ * out_amax (optional) receives atomically max(|y|) over the same window, for
  * calibrating out_global_scale; the caller initializes it.
  * debug_y (optional, tests) receives y as binary32 [M x N] before the store. */
 typedef struct {
@@ -223,13 +232,15 @@ typedef struct {
     const void* residual;  /* bf16 [M x N], row stride ld_residual, or NULL */
     int64_t ld_residual;
     int act;               /* NVFP4_ACT_* */
-    void* out_codes;       /* NVFP4 requant: codes [M x N/2] or NULL */
-    void* out_scales;      /* swizzled scales for [M x N] */
+    void* out_codes;       /* NVFP4 requant: codes [M x out_cols/2] or NULL */
+    void* out_scales;      /* swizzled scales for [M x out_cols] */
     const float* out_global_scale; /* device binary32 a32 of the output */
     float* out_amax;       /* device binary32 or NULL */
     float* debug_y;        /* device binary32 [M x N] or NULL */
     unsigned debug_flags;  /* NVFP4_DBG_*, 0 in production */
     uint32_t wait_limit_us; /* bound of every device-side wait; 0 = default (2 s) */
+    int64_t out_col0;      /* first column of the requant / out_amax window (0: from column 0) */
+    int64_t out_cols;      /* columns in the window (0: through column N - 1) */
 } nvfp4_epilogue;
 
 /* C[M x N] = a32_A * a32_B * (A_q . S_A)(B_q . S_B)^T, then the epilogue.
@@ -238,7 +249,8 @@ typedef struct {
  * <= 2^30 (else NVFP4_ERR_UNSUPPORTED).
  * c_bf16: [M x N] with row stride ldc (ldc >= N, ldc % 8 == 0) or NULL when
  * ep->out_codes is set.  ep may be NULL (plain bf16 output).
- * Requant needs N % 64 == 0 (else NVFP4_ERR_UNSUPPORTED).
+ * A requant window that is not a multiple of 64 at both ends returns
+ * NVFP4_ERR_UNSUPPORTED; one outside [0, N), NVFP4_ERR_INVALID_ARG.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM, M, N, K) bytes.
  * One persistent launch (tcgen05 block-scaled MMA, TMEM accumulators, TMA). */
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, void* c_bf16, int64_t ldc,

@@ -66,6 +66,14 @@ def test_host_side_argument_checks(L):
     assert st == nv.ERR_MISALIGNED
     st = L.nvfp4_quantize(fake, 16, 64, 64, fake, fake, fake, 0, fake, 16, None)
     assert st == nv.ERR_INVALID_ARG  # workspace too small
+    # the no-allocation quantize runs the same checks before touching its shared scratch (here,
+    # with no GPU, any CUDA call would fail with NVFP4_ERR_CUDA instead)
+    nq = L.nvfp4_quantize_noalloc
+    assert nq(fake, 16, 48, 48, fake, fake, fake, 0, None) == nv.ERR_UNSUPPORTED  # cols % 64
+    assert nq(fake, 16, 64, 64, fake, fake, fake, 8, None) == nv.ERR_INVALID_ARG  # unknown flag
+    assert nq(fake + 8, 16, 64, 64, fake, fake, fake, 0, None) == nv.ERR_MISALIGNED
+    assert nq(fake, 16, 64, 64, fake, fake, None, 0, None) == nv.ERR_INVALID_ARG  # no tensor scale
+    assert nq(fake, 0, 64, 64, fake, fake, fake, 0, None) == nv.OK  # nothing to do, nothing enqueued
     a = nv.CTensor(fake, fake, fake, 64, 256)
     b = nv.CTensor(fake, fake, fake, 128, 192)
     st = L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), fake, 128, None, fake, 4096, None)
@@ -80,6 +88,15 @@ def test_host_side_argument_checks(L):
     assert st == nv.ERR_INVALID_ARG  # no output at all
     st = L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), fake + 16, 100, None, fake, 4096, None)
     assert st == nv.ERR_INVALID_ARG  # ldc < N
+    # the requant / out_amax column window: inside [0, N), multiples of 64 for a requant
+    b = nv.CTensor(fake, fake, fake, 512, 256)
+    for window, want in (((64, 0), nv.OK), ((96, 64), nv.ERR_UNSUPPORTED), ((64, 96), nv.ERR_UNSUPPORTED),
+                         ((448, 128), nv.ERR_INVALID_ARG), ((-64, 64), nv.ERR_INVALID_ARG),
+                         ((512, 0), nv.ERR_INVALID_ARG)):
+        ep = nv.CEpilogue(out_codes=fake, out_scales=fake, out_global_scale=fake, out_col0=window[0],
+                          out_cols=window[1], ld_residual=0, act=9)  # act 9: rejected after the window checks
+        st = L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), None, 512, ctypes.byref(ep), fake, 4096, None)
+        assert st == (nv.ERR_INVALID_ARG if want == nv.OK else want), window
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 24)
     st = L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 16, None)
     assert st == nv.ERR_UNSUPPORTED  # head_dim % 16

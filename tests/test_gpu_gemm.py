@@ -257,3 +257,36 @@ def test_bounded_wait_records_timeout_and_context_survives():
     nv.gemm(qa, qb, ws=ws)
     code, _ = nv.read_device_error(ws)
     assert code == nv.OK
+
+
+@pytest.mark.parametrize("M,N,K,col0,cols", [(200, 512, 256, 128, 192), (300, 9216 // 8, 512, 768, 384),
+                                            (129, 256, 256, 0, 64)])
+def test_requant_of_a_column_window(M, N, K, col0, cols):
+    """The requant (and out_amax) of columns col0 .. col0 + cols - 1 only, as an
+    [M, cols] operand (a QKV projection's V third): bit for bit the oracle's
+    quantize of those columns of y; the bf16 output still covers every column."""
+    require_gpu()
+    qa, oa, qb, ob = _gemm_case(M, N, K, seed=91 + col0)
+    bias = syn.normal_bf16((N,), seed=92, std=0.1)
+    y_ref, _ = oracle.gemm(oa, ob, bias=bias, want_bf16=False)
+    out_a32 = np.float32(np.max(np.abs(y_ref[:, col0:col0 + cols])) / 2688.0)
+    rq = nv.empty_nvfp4(M, cols)
+    rq.global_scale.fill_(float(out_a32))
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    dy = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    c = nv.gemm(qa, qb, bias=dev_bf16(bias), requant=rq, out_amax=amax, debug_y=dy, out_window=(col0, cols))
+    torch.cuda.synchronize()
+    y = dy.cpu().numpy()
+    assert normwise_err(y.astype(np.float64), y_ref) <= GEMM_TOL
+    assert np.array_equal(host_bits(c), host_bits(dy.to(torch.bfloat16)))
+    yw = np.ascontiguousarray(y[:, col0:col0 + cols])
+    codes, scales, _ = oracle.quantize(yw, out_a32)
+    assert np.array_equal(host_u8(rq.codes), codes)
+    assert np.array_equal(host_u8(rq.scales), oracle.swizzle(scales))
+    assert float(amax.item()) == float(np.max(np.abs(yw)))
+    # the same window without a bf16 output gives the same operand
+    rq2 = nv.empty_nvfp4(M, cols)
+    rq2.global_scale.fill_(float(out_a32))
+    nv.gemm(qa, qb, bias=dev_bf16(bias), requant=rq2, bf16_out=False, out_window=(col0, cols))
+    torch.cuda.synchronize()
+    assert torch.equal(rq2.codes, rq.codes) and torch.equal(rq2.scales, rq.scales)
