@@ -12,25 +12,27 @@
 // fused adaLN kernels of the anzhuoshouzhuan.com article ("NVFP4 量化").
 //
 // Kernel design (B200):
-//  * persistent grid, one CTA per SM, static round-robin tile schedule.  Two
-//    variants of one template: a CTA pair (cluster of 2, tcgen05 cta_group::2)
-//    computing 256 x 256 tiles -- each CTA loads its 128 rows of A, its 128
-//    rows of B and all 256 rows of B's scales, the leader CTA issues the MMAs
-//    for both -- and a single-CTA 128 x 256 variant used when M <= 128;
+//  * persistent grid, one CTA per SM, static tile schedule with the N blocks
+//    of an M block consecutive.  Two variants of one template: a CTA pair
+//    (cluster of 2, tcgen05 cta_group::2) computing 256 x 256 tiles -- each
+//    CTA loads its 128 rows of A, its 128 rows of B and all 256 rows of B's
+//    scales, the leader CTA issues the MMAs for both -- and a single-CTA
+//    128 x 256 variant used when M <= 128;
 //  * warp 0: TMA producer (A/B code tiles with 128B swizzle, the 512-byte
 //    scale-factor tiles as 3-D boxes whose K tail the TMA zero-fills); a ring
-//    of K-slices of 256 elements (5 x 38 KB per CTA for the pair, 4 x 54 KB
+//    of K-slices of 256 elements (5 x 38 KB per CTA for the pair, 3 x 54 KB
 //    for one CTA);
 //  * warp 1: owns TMEM (512 columns: two overlapping 256-column accumulators
-//    and two 48-column scale buffers) and issues, from one thread,
+//    and two or three 48-column scale buffers) and issues, from one thread,
 //    tcgen05.mma.kind::mxf4nvf4.block_scale (M=128 or 256 for the pair,
 //    N=256, K=64), releasing each stage with tcgen05.commit;
-//  * warps 6..8: tcgen05.cp of the stage's scale tiles into the free TMEM
-//    scale buffer, a stage ahead of the MMAs;
-//  * warps 2..5: epilogue, tcgen05.ld of 32 columns at a time, binary32 math,
-//    16-byte stores (and the NVFP4 requant with the same encoder as the
-//    quantize kernel); it drains the columns both accumulators share first,
-//    so the next tile's MMAs run while the rest of the epilogue proceeds;
+//  * warps 10..: tcgen05.cp of the stage's scale tiles into a free TMEM scale
+//    buffer, a stage ahead of the MMAs;
+//  * warps 2..9: epilogue, two warps per TMEM lane quarter, each taking every
+//    other 32-column chunk: tcgen05.ld, binary32 math, bf16 through TMA stores
+//    and/or the NVFP4 requant with the same encoder as the quantize kernel;
+//    the columns both accumulators share are drained first, so the next
+//    tile's MMAs run while the rest of the epilogue proceeds;
 //  * every mbarrier wait is bounded (globaltimer); on expiry the kernel
 //    records NVFP4_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag,
 //    drains what it issued and frees TMEM before returning.
@@ -47,12 +49,17 @@ constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 256;  // K elements per stage
 constexpr int BKB = BK / 2;  // bytes per row per stage (128: one swizzle atom row)
 constexpr int KB_PER_STAGE = BK / 64;
-// Block: producer, MMA, 4 epilogue warps and NC scale-copy warps.  Two
-// variants: NC = 3 (288 threads, so at most 168 registers a thread) for long
-// K, where the mainloop dominates, and NC = 2 (256 threads, up to 255
-// registers) for short K, where the epilogue has the registers to take the
-// shared accumulator columns in one go and the next tile starts sooner.
-constexpr int threads_for(int nc) { return (6 + nc) * 32; }
+// Block: producer, MMA, 8 epilogue warps (two per TMEM lane quarter, each
+// taking every other 32-column chunk, so every scheduler has two epilogue
+// warps to switch between) and NC scale-copy warps.  Two variants: NC = 3
+// (416 threads, at most 152 registers a thread) for long K, where the
+// mainloop dominates, and NC = 2 (384 threads, 168 registers) for short K,
+// where the epilogue takes its shared accumulator columns into registers at
+// once so the next tile starts sooner.
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int FIRST_COPY_WARP = 2 + EPI_WARPS;
+constexpr int threads_for(int nc) { return (FIRST_COPY_WARP + nc) * 32; }
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int A_BYTES = BM * BKB;                  // 16 KB
 constexpr int SFA_BYTES = KB_PER_STAGE * 512;      // 2 KB
@@ -60,11 +67,11 @@ constexpr int SFB_BYTES = 2 * KB_PER_STAGE * 512;  // 4 KB (two 128-row halves o
 
 // Per-tile shared memory of the epilogue: the tile's per-column vectors
 // (bias, modulate scale, modulate shift, gate; bf16 pairs, two buffers by
-// tile parity) and each warp's two 32 x 32 bf16 staging buffers for the TMA
-// store of C (64-byte rows, 64B swizzle: 16-byte unit u of row r at
+// tile parity) and each warp's 32 x 32 bf16 staging buffer for the TMA store
+// of C (64-byte rows, 64B swizzle: 16-byte unit u of row r at
 // (u ^ (r / 2 % 4)) * 16).
 constexpr int EPI_BUF_BYTES = 32 * 64;
-constexpr int EPI_STAGE_BYTES = 4 * 2 * EPI_BUF_BYTES;  // 16 KB
+constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BUF_BYTES;  // 16 KB
 constexpr int VEC_WORDS = BN / 2;                        // bf16 pairs per vector per tile
 constexpr int VEC_BYTES = 2 * 4 * VEC_WORDS * 4;        // 4 KB
 
@@ -154,9 +161,13 @@ struct Smem {
     int abort_flag;
 };
 
+// Tile order: the N blocks of one M block are consecutive, so the tiles
+// running at once share a few A row blocks (each fetched from HBM once and
+// then read from L2 by every N block) while the whole weight B stays in L2
+// across waves when it fits (a DiT linear's weight is at most ~25 MB).
 __device__ __forceinline__ void tile_coords(const Params& p, int tile, int& mb, int& nb) {
-    mb = tile % p.tiles_m;
-    nb = tile / p.tiles_m;
+    nb = tile % p.tiles_n;
+    mb = tile / p.tiles_n;
 }
 
 template <class S>
@@ -505,13 +516,22 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
     }
 }
 
+// Epilogue warp w (2..9) reads TMEM lane quarter w % 4 (rows 32 (w % 4) ..
+// of the CTA's 128) and the 32-column chunks j = h, h + 2, h + 4, h + 6 of
+// the tile (h = (w - 2) / 4).  The chunks this accumulator shares with the
+// other one (Tm::OVERLAP_CHUNKS at the high end of buffer 0, at the low end
+// of buffer 1) come first; once they are in registers the warp arrives on
+// tmem_empty (8 warps per CTA), so the next tile's MMAs can start.
 template <bool PAIR, int NC, bool EARLY>
 __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t tmem, int warp, int lane, uint32_t rank,
                          const CUtensorMap* tma_c, uint8_t* epi_stage, uint32_t* vecs) {
     using C = Cfg<PAIR>;
+    constexpr int OV = Tm<NC>::OVERLAP_CHUNKS;
+    static_assert(!EARLY || OV <= 4, "an early warp holds at most two shared chunks");
     volatile int* abort = &s->abort_flag;
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int et = (warp - 2) * 32 + lane;  // 0..127 over the epilogue warps
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;          // column chunks h, h + 2, h + 4, h + 6
+    const int et = (warp - 2) * 32 + lane;  // 0..255 over the epilogue warps
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
     const float oa32 = p.out_codes ? __ldg(p.out_gscale) : 0.0f;
     const int64_t tiles_on = ((int64_t)(p.q_col1 - p.q_col0) + 63) / 64;  // scale tiles along the requant window
@@ -519,52 +539,56 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
     // the leader's MMA waits for the epilogue warps of both CTAs
     const uint32_t empty_bar = PAIR ? mapa_shared(smem_u32(&s->tmem_empty), 0) : smem_u32(&s->tmem_empty);
     const __nv_bfloat16* vsrc[4] = {p.bias, p.mod_scale, p.mod_shift, p.gate};
-    uint8_t* my_stage = epi_stage + (warp - 2) * 2 * EPI_BUF_BYTES;
+    uint8_t* stage = epi_stage + (warp - 2) * EPI_BUF_BYTES;
     if (p.c && lane == 0) prefetch_tmap(tma_c);
     int first, step;
     tile_range<PAIR>(first, step);
     float amax_run = 0.0f;
-    uint32_t tcount = 0, nstored = 0;
+    uint32_t tcount = 0;
     for (int tile = first; tile < p.num_tiles; tile += step, tcount++) {
         int mb, nb;
         tile_coords(p, tile, mb, nb);
-        // stage this tile's per-column vectors (zero past N)
+        // stage this tile's per-column vectors (zero past N): one bf16 pair per thread of the first 128
         uint32_t* tv = vecs + (tcount & 1) * 4 * VEC_WORDS;
+        if (et < VEC_WORDS) {
 #pragma unroll
-        for (int v = 0; v < 4; v++) {
-            if (vsrc[v]) {
-                const int64_t n = (int64_t)nb * BN + 2 * et;
-                uint32_t w2 = 0;
-                if (n + 1 < p.N)
-                    w2 = __ldg(reinterpret_cast<const uint32_t*>(vsrc[v] + n));
-                else if (n < p.N)
-                    w2 = (uint32_t)__bfloat16_as_ushort(vsrc[v][n]);
-                tv[v * VEC_WORDS + et] = w2;
+            for (int v = 0; v < 4; v++) {
+                if (vsrc[v]) {
+                    const int64_t n = (int64_t)nb * BN + 2 * et;
+                    uint32_t w2 = 0;
+                    if (n + 1 < p.N)
+                        w2 = __ldg(reinterpret_cast<const uint32_t*>(vsrc[v] + n));
+                    else if (n < p.N)
+                        w2 = (uint32_t)__bfloat16_as_ushort(vsrc[v][n]);
+                    tv[v * VEC_WORDS + et] = w2;
+                }
             }
         }
         const bool ok = mbar_wait_bounded(&s->tmem_full, tcount & 1, abort, p.limit_ns);
         if (!ok && !*abort) raise_abort(s, p, 4);
-        // the staged vectors are visible, and all four warps take the same exit
-        if (named_barrier_or(1, 128, !ok)) break;
+        // the staged vectors are visible, and all epilogue warps take the same exit
+        if (named_barrier_or(1, EPI_THREADS, !ok)) break;
         tc_fence_after();
         const int64_t m0 = (int64_t)mb * C::TILE_M + (int64_t)rank * BM + q * 32;  // the warp's first row
         const int64_t m = m0 + lane;
         const bool row_ok = m < p.M;
         const int ncols = min(BN, p.N - nb * BN);
         const int nchunks = (ncols + 31) / 32;
+        const int nmy = (nchunks - h + 1) >> 1;  // this warp's chunks: i = 0 .. nmy - 1, j = h + 2 i
         const bool buf1 = tcount & 1;
-        constexpr int OVERLAP_CHUNKS = Tm<NC>::OVERLAP_CHUNKS;
         const uint32_t acc = lane_base + (buf1 ? Tm<NC>::ACC1_COL : 0u);
-        // chunks of this buffer that the other buffer overlaps come first
-        const int first_ov = buf1 ? 0 : (BN / 32 - OVERLAP_CHUNKS);
-        const int n_overlap = buf1 ? min(nchunks, OVERLAP_CHUNKS) : max(0, nchunks - first_ov);
+        // shared chunks: buffer 1's first OV, buffer 0's last OV; as indices i of this warp's
+        // chunks they are a prefix (buffer 1) or a suffix starting at s0 (buffer 0)
+        const int s0 = (BN / 32 - OV - h + 1) >> 1;
+        const int n_ov = buf1 ? min(nmy, (OV - h + 1) >> 1) : max(0, nmy - s0);
+        // processing order t = 0 .. nmy - 1: shared chunks first
+        auto chunk_of = [&](int t) { return h + 2 * (buf1 ? t : (t < n_ov ? s0 + t : t - n_ov)); };
         auto out_chunk = [&](const uint32_t* r, int j) {
             const int64_t n0 = (int64_t)nb * BN + j * 32;
             const int valid = (int)min((int64_t)32, p.N - n0);
-            uint8_t* stage = my_stage + (nstored & 1) * EPI_BUF_BYTES;
             if (p.c) {
-                // the store issued two chunks ago has finished reading this buffer
-                if (lane == 0) bulk_wait_group_read<1>();
+                // the previous store has finished reading the staging buffer
+                if (lane == 0) bulk_wait_group_read<0>();
                 __syncwarp();
             }
             const uint32_t* vc[4] = {tv + j * 16, tv + VEC_WORDS + j * 16, tv + 2 * VEC_WORDS + j * 16,
@@ -577,31 +601,25 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
                     tma_store_2d(tma_c, stage, (int32_t)n0, (int32_t)m0);
                     bulk_commit_group();
                 }
-                nstored++;
             }
         };
         if (EARLY) {
-            // the overlapped chunks go to registers first; then the next tile may start
-            uint32_t ov[OVERLAP_CHUNKS][32];
-#pragma unroll
-            for (int c = 0; c < OVERLAP_CHUNKS; c++)
-                if (c < n_overlap) tmem_ld_32cols(acc + (first_ov + c) * 32, ov[c]);
+            // the shared chunks (at most two) go to registers first; then the next tile may start
+            uint32_t ov0[32], ov1[32];
+            if (n_ov > 0) tmem_ld_32cols(acc + chunk_of(0) * 32, ov0);
+            if (n_ov > 1) tmem_ld_32cols(acc + chunk_of(1) * 32, ov1);
             tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < OVERLAP_CHUNKS; c++) tmem_regs_ready(ov[c]);
+            tmem_regs_ready(ov0);
+            tmem_regs_ready(ov1);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_bar);
-            for (int i = 0; i < nchunks; i++) {
-                // buffer 0 visits chunks 5, 6, 7, 0, ..., 4; buffer 1 visits 0..7
-                const int j = buf1 ? i : ((i < n_overlap) ? first_ov + i : i - n_overlap);
+            for (int t = 0; t < nmy; t++) {
+                const int j = chunk_of(t);
                 uint32_t r[32];
-                if (i < n_overlap) {
+                if (t < n_ov) {
 #pragma unroll
-                    for (int c = 0; c < OVERLAP_CHUNKS; c++)
-                        if (c == i)
-#pragma unroll
-                            for (int e = 0; e < 32; e++) r[e] = ov[c][e];
+                    for (int e = 0; e < 32; e++) r[e] = t == 0 ? ov0[e] : ov1[e];
                 } else {
                     tmem_ld_32cols(acc + j * 32, r);
                     tmem_ld_wait();
@@ -610,20 +628,19 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
                 out_chunk(r, j);
             }
         } else {
-            if (n_overlap == 0) {
+            if (n_ov == 0) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(empty_bar);
             }
-            for (int i = 0; i < nchunks; i++) {
-                // buffer 0 visits chunks 5, 6, 7, 0, ..., 4; buffer 1 visits 0..7
-                const int j = buf1 ? i : ((i < n_overlap) ? first_ov + i : i - n_overlap);
+            for (int t = 0; t < nmy; t++) {
+                const int j = chunk_of(t);
                 uint32_t r[32];
                 tmem_ld_32cols(acc + j * 32, r);
                 tmem_ld_wait();
                 tmem_regs_ready(r);
-                if (i == n_overlap - 1) {
-                    // the overlapped columns are in registers: next tile may start
+                if (t == n_ov - 1) {
+                    // this warp's shared columns are in registers: the next tile may start
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(empty_bar);
@@ -661,7 +678,7 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
             mbar_init(&s->empty[i], 1);
         }
         mbar_init(&s->tmem_full, 1);
-        mbar_init(&s->tmem_empty, 4 * C::CTAS);
+        mbar_init(&s->tmem_empty, EPI_WARPS * C::CTAS);
         mbar_init(&s->drain, 1);
         for (int i = 0; i < Tm<NC>::NSF; i++) {
             mbar_init(&s->sf_full[i], NC);
@@ -694,8 +711,8 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) mma_issuer<PAIR, NC>(p, s, ring, tmem);
         __syncwarp();
-    } else if (warp >= 6) {
-        if (lane == 0 && rank == 0) scale_copier<PAIR, NC>(p, s, ring, tmem, warp - 6);
+    } else if (warp >= FIRST_COPY_WARP) {
+        if (lane == 0 && rank == 0) scale_copier<PAIR, NC>(p, s, ring, tmem, warp - FIRST_COPY_WARP);
         __syncwarp();
     } else {
         epilogue<PAIR, NC, NC == 2>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs);
