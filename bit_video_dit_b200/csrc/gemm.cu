@@ -72,8 +72,8 @@ constexpr int SFB_BYTES = 2 * KB_PER_STAGE * 512;  // 4 KB (two 128-row halves o
 // (u ^ (r / 2 % 4)) * 16).
 constexpr int EPI_BUF_BYTES = 32 * 64;
 constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BUF_BYTES;  // 16 KB
-constexpr int VEC_WORDS = BN / 2;                        // bf16 pairs per vector per tile
-constexpr int VEC_BYTES = 2 * 4 * VEC_WORDS * 4;        // 4 KB
+constexpr int VEC_BYTES = 2 * 4 * BN * 4;  // two tile parities x 4 binary32 vectors x BN: 8 KB
+constexpr int INV_TAB_BYTES = 256 * 4;    // requant reciprocal per E4M3 code
 
 // Two accumulators of BN columns share TMEM with NSF 48-column scale buffers
 // that the stages take in turn (the copy warps fill one while the MMAs read
@@ -114,7 +114,7 @@ struct Cfg {
     static constexpr int STAGES = PAIR ? 5 : 3;
     static constexpr int B_BYTES = B_ROWS * BKB;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + VEC_BYTES + 1024 + 256;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + VEC_BYTES + INV_TAB_BYTES + 1024 + 256;
     static constexpr uint32_t TX_BYTES = (uint32_t)(CTAS * STAGE_BYTES);  // per stage, both CTAs
     static constexpr uint32_t IDESC = make_idesc(TILE_M, BN);
     static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment for 128B swizzle");
@@ -390,14 +390,43 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
 }
 
 // ---------------------------------------------------------------- epilogue --
-// GELU, tanh form, with the hardware tanh (tanh.approx.f32, absolute error
-// about 2^-11): the GELU value moves by at most ~3e-4 |y|.
-__device__ __forceinline__ float gelu_tanh(float y) {
-    const float k = 0.7978845608028654f;  // sqrt(2 / pi)
-    const float u = k * (y + 0.044715f * y * y * y);
-    float th;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(u));
-    return 0.5f * y * (1.0f + th);
+// Packed binary32 pairs (f32x2): each lane rounded as its own binary32
+// operation, two elements per instruction.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)));
+    return *reinterpret_cast<const float2*>(&r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)));
+    return *reinterpret_cast<const float2*>(&r);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)), "l"(*reinterpret_cast<const unsigned long long*>(&c)));
+    return *reinterpret_cast<const float2*>(&r);
+}
+
+// GELU, tanh form, on a pair: (y / 2) (1 + tanh(u)) with u = sqrt(2/pi) (y +
+// 0.044715 y^3) = y * (sqrt(2/pi) + sqrt(2/pi) 0.044715 y^2) and the hardware
+// tanh (tanh.approx.f32): the value moves by at most ~3e-4 |y| from the exact
+// tanh form.  The product form keeps the sign of a negative y whose tanh
+// rounds to -1 (a -0 result, as the exact value's tiny negative), which a
+// fused h + h tanh(u) would turn into +0.
+__device__ __forceinline__ float2 gelu2(float2 y) {
+    const float2 k = make_float2(0.7978845608028654f, 0.7978845608028654f);       // sqrt(2 / pi)
+    const float2 kc = make_float2(0.0356774081363001f, 0.0356774081363001f);      // sqrt(2 / pi) * 0.044715
+    const float2 half = make_float2(0.5f, 0.5f);
+    const float2 one = make_float2(1.0f, 1.0f);
+    const float2 u = mul2(y, fma2(kc, mul2(y, y), k));
+    float2 th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(u.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(u.y));
+    return mul2(mul2(half, y), add2(one, th));
 }
 
 // 32 consecutive bf16 (as binary32), columns n0.. with `valid` of them in
@@ -413,76 +442,125 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* p, int valid, fl
     }
 }
 
-// 32 bf16 of a staged per-column vector (shared memory, same for every lane)
-__device__ __forceinline__ void smem_vec32(const uint32_t* v, float* out) {
-    const uint4* q = reinterpret_cast<const uint4*>(v);
+// Per-tile staged column vectors in shared memory, binary32 [VEC_N][BN]:
+// bias, 1 + modulate scale (fl32 of the sum), modulate shift, gate.
+constexpr int VEC_BIAS = 0, VEC_SCALE1 = 1, VEC_SHIFT = 2, VEC_GATE = 3, VEC_N = 4;
+
+// 32 binary32 of a staged vector (the same for every lane: broadcast loads)
+__device__ __forceinline__ void smem_vec32(const float* v, float2* out) {
+    const float4* q = reinterpret_cast<const float4*>(v);
 #pragma unroll
-    for (int i = 0; i < 4; i++) bf16x8_to_f32(q[i], out + 8 * i);
+    for (int i = 0; i < 8; i++) {
+        const float4 f = q[i];
+        out[2 * i] = make_float2(f.x, f.y);
+        out[2 * i + 1] = make_float2(f.z, f.w);
+    }
+}
+
+// Requant constants of one launch: the output tensor scale a32, 6 a32, and
+// the reciprocal 1 / (s * a32) of every E4M3 code s (0 for s == 0 or
+// a32 == 0), a table each CTA fills once.
+struct RequantConsts {
+    float a32, d6;
+    const float* inv_tab;
+};
+
+// E4M3 code of the block max and the block's reciprocal scale: the quantize
+// rule s = E4M3_rne_satfinite(amax / (6 a32)), 1 / (s a32) from the table.
+__device__ __forceinline__ uint32_t requant_scale(float amax_b, const RequantConsts& k, float& inv) {
+    const uint32_t code = k.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, k.d6));
+    inv = k.inv_tab[code];
+    return code;
+}
+
+// Eight pairs (16 elements of one block) times inv -> 64 bits of E2M1 codes.
+__device__ __forceinline__ uint2 encode16x2(const float2* y, float inv) {
+    const float2 iv = make_float2(inv, inv);
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float2 t = mul2(y[i], iv);
+        q[2 * i] = t.x;
+        q[2 * i + 1] = t.y;
+    }
+    // a flushed block (s == 0 or a32 == 0: inv == 0) is +0 codes (not the -0
+    // that negative values times 0 would give)
+    return inv == 0.0f ? make_uint2(0u, 0u) : make_uint2(e2m1x8(q), e2m1x8(q + 8));
 }
 
 // One 32-column chunk of one output row: epilogue math and outputs.  `r`
-// holds the accumulator (binary32 bits), `vec` the tile's staged vectors
-// (at this chunk's columns), `stage` this warp's staging buffer.  The NVFP4
-// requant and out_amax cover the column window [q_col0, q_col1) only (its
-// ends are multiples of 64 when requantizing, so a chunk is inside or
-// outside it as a whole); requant column n lands at n - q_col0 of an
-// [M x (q_col1 - q_col0)] operand with tiles_on scale tiles along its row.
+// holds the accumulator (binary32 bits), `tv` the tile's staged vectors,
+// `stage` this warp's staging buffer.  The arithmetic is binary32 on pairs:
+// y = fma(acc, a32_A a32_B, bias) (one rounding), then GELU, y (1 + scale),
+// + shift, gate * y, residual + y as the header states.  The NVFP4 requant and
+// out_amax cover the column window [q_col0, q_col1) only (its ends are
+// multiples of 64 when requantizing, so a chunk is inside or outside it as a
+// whole); requant column n lands at n - q_col0 of an [M x (q_col1 - q_col0)]
+// operand with tiles_on scale tiles along its row.
 __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* r, float alpha, int64_t m, bool row_ok,
-                                               int64_t n0, int valid, float oa32, int64_t tiles_on, float& amax_run,
-                                               const uint32_t* const* vec, uint8_t* stage, int lane) {
-    float y[32];
-#pragma unroll
-    for (int i = 0; i < 32; i++) y[i] = __uint_as_float(r[i]) * alpha;
-    float v[32];
+                                               int64_t n0, int j, int valid, const RequantConsts& rq,
+                                               int64_t tiles_on, float& amax_run, const float* tv, uint8_t* stage,
+                                               int lane) {
+    float2 y[16];
+    float2 v[16];
+    const float2 al = make_float2(alpha, alpha);
     if (p.bias) {
-        smem_vec32(vec[0], v);
+        smem_vec32(tv + VEC_BIAS * BN + j * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; i++) y[i] += v[i];
+        for (int i = 0; i < 16; i++) y[i] = fma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), al, v[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; i++) y[i] = mul2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), al);
     }
     if (p.act == NVFP4_ACT_GELU_TANH) {
 #pragma unroll
-        for (int i = 0; i < 32; i++) y[i] = gelu_tanh(y[i]);
+        for (int i = 0; i < 16; i++) y[i] = gelu2(y[i]);
     }
     if (p.mod_scale) {
-        smem_vec32(vec[1], v);
+        smem_vec32(tv + VEC_SCALE1 * BN + j * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; i++) y[i] = y[i] * (1.0f + v[i]);
+        for (int i = 0; i < 16; i++) y[i] = mul2(y[i], v[i]);
     }
     if (p.mod_shift) {
-        smem_vec32(vec[2], v);
+        smem_vec32(tv + VEC_SHIFT * BN + j * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; i++) y[i] += v[i];
+        for (int i = 0; i < 16; i++) y[i] = add2(y[i], v[i]);
     }
     if (p.gate) {
-        smem_vec32(vec[3], v);
+        smem_vec32(tv + VEC_GATE * BN + j * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; i++) y[i] = v[i] * y[i];
+        for (int i = 0; i < 16; i++) y[i] = mul2(v[i], y[i]);
     }
     if (p.residual && row_ok) {
-        load_row32(p.residual + m * p.ld_res + n0, valid, v);
+        float rv[32];
+        load_row32(p.residual + m * p.ld_res + n0, valid, rv);
 #pragma unroll
-        for (int i = 0; i < 32; i++) y[i] = v[i] + y[i];
+        for (int i = 0; i < 16; i++) y[i] = add2(make_float2(rv[2 * i], rv[2 * i + 1]), y[i]);
     }
     const bool in_win = n0 >= p.q_col0 && n0 < p.q_col1;
     if (p.out_amax && row_ok && in_win) {
         const int wv = (int)min((int64_t)valid, (int64_t)p.q_col1 - n0);
 #pragma unroll
-        for (int i = 0; i < 32; i++)
-            if (i < wv) amax_run = fmaxf(amax_run, fabsf(y[i]));
+        for (int i = 0; i < 16; i++) {
+            if (2 * i < wv) amax_run = fmaxf(amax_run, fabsf(y[i].x));
+            if (2 * i + 1 < wv) amax_run = fmaxf(amax_run, fabsf(y[i].y));
+        }
     }
     if (p.debug_y && row_ok) {
         float* d = p.debug_y + m * p.N + n0;
 #pragma unroll
-        for (int i = 0; i < 32; i++)
-            if (i < valid) d[i] = y[i];
+        for (int i = 0; i < 16; i++) {
+            if (2 * i < valid) d[2 * i] = y[i].x;
+            if (2 * i + 1 < valid) d[2 * i + 1] = y[i].y;
+        }
     }
     if (p.c) {
         // row `lane` of the staging buffer; the TMA store drops rows >= M and columns >= N
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; i++) {
-            __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t*>(&b);
+            __nv_bfloat162 bb = __floats2bfloat162_rn(y[i].x, y[i].y);
+            w[i] = *reinterpret_cast<uint32_t*>(&bb);
         }
         uint8_t* row = stage + lane * 64;
         const int sw = (lane >> 1) & 3;
@@ -498,16 +576,18 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
         if (row_ok) {
             float am0 = 0.0f, am1 = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; i++) {
-                am0 = fmaxf(am0, fabsf(y[i]));
-                am1 = fmaxf(am1, fabsf(y[16 + i]));
+            for (int i = 0; i < 8; i++) {
+                am0 = fmaxf(am0, fmaxf(fabsf(y[i].x), fabsf(y[i].y)));
+                am1 = fmaxf(am1, fmaxf(fabsf(y[8 + i].x), fabsf(y[8 + i].y)));
             }
-            const BlockScale b0 = block_scale(am0, oa32);
-            const BlockScale b1 = block_scale(am1, oa32);
-            const uint4 w = make_uint4(encode8(y, b0.inv), encode8(y + 8, b0.inv), encode8(y + 16, b1.inv),
-                                       encode8(y + 24, b1.inv));
-            *reinterpret_cast<uint4*>(p.out_codes + m * ((p.q_col1 - p.q_col0) / 2) + nq / 2) = w;
-            sc2 = (uint16_t)(b0.code | (b1.code << 8));
+            float inv0, inv1;
+            const uint32_t c0 = requant_scale(am0, rq, inv0);
+            const uint32_t c1 = requant_scale(am1, rq, inv1);
+            const uint2 w0 = encode16x2(y, inv0);
+            const uint2 w1 = encode16x2(y + 8, inv1);
+            *reinterpret_cast<uint4*>(p.out_codes + m * ((p.q_col1 - p.q_col0) / 2) + nq / 2) =
+                make_uint4(w0.x, w0.y, w1.x, w1.y);
+            sc2 = (uint16_t)(c0 | (c1 << 8));
         }
         // rows past M up to the next multiple of 128 are scale padding: zero
         // (a 256-row pair tile can reach past that; those rows have no scales)
@@ -524,7 +604,7 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const uint32_t* 
 // tmem_empty (8 warps per CTA), so the next tile's MMAs can start.
 template <bool PAIR, int NC, bool EARLY>
 __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t tmem, int warp, int lane, uint32_t rank,
-                         const CUtensorMap* tma_c, uint8_t* epi_stage, uint32_t* vecs) {
+                         const CUtensorMap* tma_c, uint8_t* epi_stage, float* vecs, float* inv_tab) {
     using C = Cfg<PAIR>;
     constexpr int OV = Tm<NC>::OVERLAP_CHUNKS;
     static_assert(!EARLY || OV <= 4, "an early warp holds at most two shared chunks");
@@ -534,6 +614,12 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
     const int et = (warp - 2) * 32 + lane;  // 0..255 over the epilogue warps
     const float alpha = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
     const float oa32 = p.out_codes ? __ldg(p.out_gscale) : 0.0f;
+    // the requant's reciprocal table: one entry per epilogue thread (256 codes)
+    if (p.out_codes) {
+        const float sv = e4m3_value((uint32_t)et);
+        inv_tab[et] = (oa32 == 0.0f || sv == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sv, oa32));
+    }
+    const RequantConsts rq{oa32, __fmul_rn(6.0f, oa32), inv_tab};
     const int64_t tiles_on = ((int64_t)(p.q_col1 - p.q_col0) + 63) / 64;  // scale tiles along the requant window
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     // the leader's MMA waits for the epilogue warps of both CTAs
@@ -548,19 +634,16 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
     for (int tile = first; tile < p.num_tiles; tile += step, tcount++) {
         int mb, nb;
         tile_coords(p, tile, mb, nb);
-        // stage this tile's per-column vectors (zero past N): one bf16 pair per thread of the first 128
-        uint32_t* tv = vecs + (tcount & 1) * 4 * VEC_WORDS;
-        if (et < VEC_WORDS) {
+        // stage this tile's per-column vectors as binary32 (one column per
+        // epilogue thread; past N: 0, and 1 + scale = 1)
+        float* tv = vecs + (tcount & 1) * VEC_N * BN;
+        {
+            const int64_t n = (int64_t)nb * BN + et;
 #pragma unroll
-            for (int v = 0; v < 4; v++) {
+            for (int v = 0; v < VEC_N; v++) {
                 if (vsrc[v]) {
-                    const int64_t n = (int64_t)nb * BN + 2 * et;
-                    uint32_t w2 = 0;
-                    if (n + 1 < p.N)
-                        w2 = __ldg(reinterpret_cast<const uint32_t*>(vsrc[v] + n));
-                    else if (n < p.N)
-                        w2 = (uint32_t)__bfloat16_as_ushort(vsrc[v][n]);
-                    tv[v * VEC_WORDS + et] = w2;
+                    const float x = n < p.N ? __bfloat162float(vsrc[v][n]) : 0.0f;
+                    tv[v * BN + et] = v == VEC_SCALE1 ? __fadd_rn(1.0f, x) : x;
                 }
             }
         }
@@ -591,9 +674,7 @@ __device__ void epilogue(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint32_t t
                 if (lane == 0) bulk_wait_group_read<0>();
                 __syncwarp();
             }
-            const uint32_t* vc[4] = {tv + j * 16, tv + VEC_WORDS + j * 16, tv + 2 * VEC_WORDS + j * 16,
-                                     tv + 3 * VEC_WORDS + j * 16};
-            epilogue_chunk(p, r, alpha, m, row_ok, n0, valid, oa32, tiles_on, amax_run, vc, stage, lane);
+            epilogue_chunk(p, r, alpha, m, row_ok, n0, j, valid, rq, tiles_on, amax_run, tv, stage, lane);
             if (p.c) {
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -666,8 +747,9 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_stage = ring + C::STAGES * C::STAGE_BYTES;  // 1024-aligned (STAGE_BYTES % 1024 == 0)
-    uint32_t* vecs = reinterpret_cast<uint32_t*>(epi_stage + EPI_STAGE_BYTES);
-    Smem<C::STAGES>* s = reinterpret_cast<Smem<C::STAGES>*>(epi_stage + EPI_STAGE_BYTES + VEC_BYTES);
+    float* vecs = reinterpret_cast<float*>(epi_stage + EPI_STAGE_BYTES);
+    float* inv_tab = reinterpret_cast<float*>(epi_stage + EPI_STAGE_BYTES + VEC_BYTES);
+    Smem<C::STAGES>* s = reinterpret_cast<Smem<C::STAGES>*>(epi_stage + EPI_STAGE_BYTES + VEC_BYTES + INV_TAB_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -715,7 +797,7 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
         if (lane == 0 && rank == 0) scale_copier<PAIR, NC>(p, s, ring, tmem, warp - FIRST_COPY_WARP);
         __syncwarp();
     } else {
-        epilogue<PAIR, NC, NC == 2>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs);
+        epilogue<PAIR, NC, NC == 2>(p, s, tmem, warp, lane, rank, &tma_c, epi_stage, vecs, inv_tab);
     }
     tc_fence_before();
     if (PAIR)

@@ -210,10 +210,12 @@ typedef struct {
 #define NVFP4_DBG_SKIP_LOADS 1u /* producer issues no loads: the consumer's bounded wait
                                    must run out and record NVFP4_ERR_TIMEOUT (tests only) */
 
-/* Epilogue, applied in binary32 to y = a32_A * a32_B * acc, in this order:
- *   y += bias[n];  y = act(y);  y = y * (1 + mod_scale[n]) + mod_shift[n];
- *   y = gate[n] * y;  y = residual[m, n] + y
- * (each step skipped when its pointer is NULL / act is NONE).  Then y is
+/* Epilogue, in binary32, in this order:
+ *   y = a32_A * a32_B * acc + bias[n]  (one fused multiply-add; y = a32_A *
+ *   a32_B * acc without a bias);  y = act(y);  y = y * (1 + mod_scale[n]);
+ *   y = y + mod_shift[n];  y = gate[n] * y;  y = residual[m, n] + y
+ * (each step skipped when its pointer is NULL / act is NONE; a32_A * a32_B
+ * and 1 + mod_scale[n] rounded to binary32 first).  Then y is
  * stored as bf16 to c (if non-NULL; every column) and/or re-quantized to
  * NVFP4 with the given output tensor scale (if out_codes is non-NULL):
  * blocks of 16 along N, exactly the quantize rule above, over the column
