@@ -50,6 +50,7 @@ struct AttnArgs {
     int64_t slot_elems;
     float scale_log2;            // softmax scale * log2(e)
     DevError* err;
+    uint32_t* rescales;          // count of warp-level rescales of O (diagnostic)
     uint64_t limit_ns;
 };
 
@@ -374,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
         // tcgen05.ld / st are warp-collective: the warp rescales together when any
         // of its rows needs it (the others multiply by exactly 1)
         if (__any_sync(0xFFFFFFFFu, factor != 1.0f) && !first_pv) {
+            if ((i & 31) == 0) atomicAdd(a.rescales, 1u);
             uint32_t o[32];
 #pragma unroll 1
             for (int c = 0; c < 4; c++) {
@@ -528,6 +530,7 @@ extern "C" nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const in
     const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)kD);
     a.scale_log2 = sc * 1.4426950408889634f;  // log2(e)
     a.err = static_cast<DevError*>(workspace);
+    a.rescales = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + 16);
     a.limit_ns = 2000000000ull;
     const int smem = 3 * kOperandBytes;
     // caches without smoothing means take the binary16 path

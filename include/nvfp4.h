@@ -354,7 +354,10 @@ int32_t nvfp4_attention_chunks(int32_t t, int32_t sink_global, int32_t shot_star
  * TMEM then), P rounded to the tiles' 16-bit type; one launch of
  * ceil(tq / 128) x heads CTAs.  An out-of-range slot records NVFP4_ERR_DEVICE
  * (info = list position) and is skipped.  workspace:
- * nvfp4_workspace_bytes(NVFP4_OP_KV_ATTENTION, 0, 0, 0) bytes. */
+ * nvfp4_workspace_bytes(NVFP4_OP_KV_ATTENTION, 0, 0, 0) bytes; its bytes
+ * 16..19 (a uint32 after the error record) count the rescales of O, one per
+ * warp and key tile in which a row's reference maximum moved after the first
+ * tile (a diagnostic: each call adds to it, the caller clears it). */
 nvfp4_status nvfp4_kv_attention(const nvfp4_kv_cache* cache, const int32_t* slots_dev, int32_t n, const void* q_bf16,
                                 int32_t tq, float scale, void* o_bf16, void* workspace, size_t ws_bytes,
                                 nvfp4_stream_t stream);

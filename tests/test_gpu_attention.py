@@ -60,7 +60,25 @@ def _case(T, H, Tq, slot_chunks, n_slots, seed, smooth_k=False, smooth_v=False, 
     gs = got if rows is None else got[rows]
     err = normwise_err(gs.reshape(-1), ref.reshape(-1))
     assert err <= TOL, err
+    check_rows(gs, qs, kk, vv, sc, ref)
     return got, ref, cache
+
+
+def check_rows(got, q, k, v, scale, ref):
+    """Per element of every output row (reading R23's error sources): P rounded
+    to its 16-bit type moves each weight by at most 2^-9 of itself, so the
+    numerator by at most 2^-9 of sum_j p_j |v_j|; O's bf16 store and the
+    binary32 row sum add at most ~2^-9 |O|.  Bound, with a factor 2 of room:
+      |O - O_ref| <= 2^-8 (softmax-weighted |V|) + 2^-8 |O_ref| + 2^-24 max|V|
+    (the last term: binary16 weights below its normal range, absolute 2^-25)."""
+    vf = _bits_to_f64(v) if v.dtype == np.uint16 else np.asarray(v, np.float64)
+    wabs = oracle.attention(q, k, np.abs(vf), scale)
+    vmax = np.max(np.abs(vf))
+    bound = 2.0 ** -8 * wabs + 2.0 ** -8 * np.abs(ref) + 2.0 ** -24 * vmax
+    excess = np.abs(got - ref) - bound
+    worst = np.unravel_index(np.argmax(excess), excess.shape)
+    assert np.all(excess <= 0), (f"row element outside the bound at {worst}: got {got[worst]} ref {ref[worst]} "
+                                 f"bound {bound[worst]}")
 
 
 @pytest.mark.parametrize("T,Tq", [(256, 200), (200, 128), (130, 7)])
@@ -131,3 +149,48 @@ def test_smoothed_channel_constant_slot_with_zero_tensor_scale():
     c, sc, a = oracle.kv_append(v)  # smoothed cache: the bf16 path for both tensors
     ref = oracle.attention(q, kb, oracle.kv_dequant(c, sc, a, T, H, d), 1.0 / np.sqrt(d))
     assert normwise_err(_bits_to_f64(host_bits(o)).reshape(-1), ref.reshape(-1)) <= TOL
+
+
+def test_lazy_maximum_rescale_is_forced_and_counted():
+    """Even query rows align with one late key (token 300 of a 384-token slot, in the
+    third key tile) whose score exceeds every earlier one by far more than 2^8 in the
+    exponent, so those rows move their reference maximum and O is rescaled in TMEM;
+    odd rows of the same warps do not (they multiply by exactly 1).  The workspace's
+    rescale counter records it, and O matches the oracle per element."""
+    require_gpu()
+    T, H, d, Tq = 384, 2, 128, 128
+    rng = np.random.default_rng(17)
+    kf = (rng.standard_normal((T, H, d)) * 0.1).astype(np.float32)
+    kf[300] = 0.5
+    vf = rng.standard_normal((T, H, d)).astype(np.float32)
+    qf = (rng.standard_normal((Tq, H, d)) * 0.3).astype(np.float32)
+    qf[0::2] = 2.0
+    kb, vb, qb = (syn.f32_to_bf16_bits(x) for x in (kf, vf, qf))
+    cache = nv.KVCache(1, T, H, d)
+    cache.append(0, dev_bf16(kb), dev_bf16(vb))
+    ws = nv.workspace(nv.OP_KV_ATTENTION, device="cuda")
+    o = cache.attention(torch.tensor([0], dtype=torch.int32, device="cuda"), dev_bf16(qb), ws=ws)
+    torch.cuda.synchronize()
+    rescales = int(ws[16:20].view(torch.int32).item())
+    # 1 query tile x 2 heads x 4 warps, each with even rows that move at the third key tile
+    assert rescales >= 8, rescales
+    kc, ksc, ka = oracle.kv_append(kb)
+    vc, vsc, va = oracle.kv_append(vb)
+    kk = oracle.dequant_f32(kc, ksc, ka).reshape(T, H, d)
+    vv = oracle.dequant_f32(vc, vsc, va).reshape(T, H, d)
+    sc = 1.0 / np.sqrt(d)
+    ref = oracle.attention(qb, kk, vv, sc)
+    got = _bits_to_f64(host_bits(o))
+    assert normwise_err(got.reshape(-1), ref.reshape(-1)) <= TOL
+    check_rows(got, qb, kk, vv, sc, ref)
+    # the even rows are dominated by value row 300 (the rescale really mattered)
+    assert np.allclose(ref[0::2], vv[300][None].astype(np.float64), rtol=0, atol=5e-2 * np.abs(vv[300]).max())
+
+
+def test_twenty_one_slot_workload_set_on_sampled_rows():
+    """The bench's attention: one 2640 x 24 x 128 query chunk over all 21 ring slots
+    (55,440 keys per head) of the KV workload's cache, checked on 32 sampled query rows
+    normwise and per element."""
+    require_gpu()
+    rows = np.sort(np.random.default_rng(21).choice(syn.KV_TOKENS, 32, replace=False))
+    _case(syn.KV_TOKENS, syn.KV_HEADS, syn.KV_TOKENS, list(range(syn.KV_SLOTS)), syn.KV_SLOTS, seed=200, rows=rows)
