@@ -784,6 +784,52 @@ def sub_report(sub, lin, pk, fp4_peak) -> dict:
     }
 
 
+def measure_codecs(nv, dev, reps: int) -> dict:
+    """ms per launch (median over `reps`, each after a 256 MB L2 flush, inside
+    one graph) of the codec kernels on their workloads: quantize of A
+    [4096 x 3072], the KV append of one 2640 x 24 x 128 K/V chunk, the dequant
+    of 21 slots, and the LayerNorm + modulate + quantize of A.  Also the small
+    case for profiling those kernels (under 2 GB on the device)."""
+    M, K = syn.QKV.M, syn.QKV.K
+    S, T, H, D = syn.KV_SLOTS, syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    a = dev_bf16(syn.activations_bf16(M, K, seed=2))
+    qa = nv.empty_nvfp4(M, K, dev)
+    ws_q = nv.workspace(nv.OP_QUANTIZE, M, 0, K, dev)
+    ws_ln = nv.workspace(nv.OP_LN_QUANTIZE, M, 0, K, dev)
+    sc = dev_bf16(syn.normal_bf16((K,), seed=72, std=0.1))
+    sh = dev_bf16(syn.normal_bf16((K,), seed=73, std=0.1))
+    cache = nv.KVCache(S, T, H, D, dev)
+    k, v = (dev_bf16(x) for x in syn.kv_chunk_bf16(T, H, D, seed=50))
+    for s_ in range(S):
+        cache.append(s_, k, v)
+    ring = torch.arange(S, dtype=torch.int32, device=dev)
+    k_out = torch.empty((S, T, H, D), dtype=torch.bfloat16, device=dev)
+    v_out = torch.empty_like(k_out)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls = {"quantize_ms": lambda: nv.quantize(a, out=qa, ws=ws_q),
+             "kv_append_ms": lambda: cache.append(0, k, v),
+             "kv_dequant_ms": lambda: cache.dequant(ring, k_out, v_out),
+             "ln_quantize_ms": lambda: nv.ln_modulate_quantize(a, mod_scale=sc, mod_shift=sh, out=qa, ws=ws_ln)}
+    for f in calls.values():
+        f()
+    torch.cuda.synchronize()
+    ev = {name: [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(reps)]
+          for name in calls}
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            for name, f in calls.items():
+                flush.fill_(1)
+                ev[name][i][0].record()
+                f()
+                ev[name][i][1].record()
+    g.replay()
+    torch.cuda.synchronize()
+    out = {name: float(np.median([e[0].elapsed_time(e[1]) for e in evs])) for name, evs in ev.items()}
+    del g
+    return out
+
+
 # --------------------------------------------------------------------------- oracle
 def _timed(f):
     t0 = time.perf_counter()
@@ -894,6 +940,9 @@ def main(argv=None) -> int:
     ap.add_argument("--ffn-only", action="store_true",
                     help="time only the 8192-token FFN pair (under 1 GB on the device: the small case for "
                          "profiling its GEMMs) and print its numbers")
+    ap.add_argument("--codecs-only", action="store_true",
+                    help="time only the codec kernels (quantize, KV append / dequant, LayerNorm quantize) on their "
+                         "workloads and print their numbers (also the small case for profiling them)")
     ap.add_argument("--layers", type=int, default=syn.STACK_LAYERS,
                     help="layers of the stack (default 30, the workload; fewer only for profiling)")
     ap.add_argument("--stack-only", action="store_true",
@@ -922,6 +971,20 @@ def main(argv=None) -> int:
         ffn = measure_ffn(nv, lambda: flush_buf.fill_(1), flush_buf.device, reps=max(1, args.steps))
         if rank == 0:
             print(json.dumps({"ffn_8192": {k: round(v, 4) for k, v in ffn.items()}}), flush=True)
+        return 0
+    if args.codecs_only:
+        from bit_video_dit_b200 import build as nvbuild
+        from bit_video_dit_b200 import nvfp4 as nv
+        nvbuild.build()
+        res = measure_codecs(nv, torch.device("cuda", local), reps=max(3, args.steps))
+        pk = peaks()
+        b = {"quantize_ms": syn.QKV.M * syn.QKV.K * 2.5625, "ln_quantize_ms": syn.QKV.M * syn.QKV.K * 2.5625,
+             "kv_append_ms": 2 * syn.KV_TOKENS * syn.KV_HEADS * syn.KV_DIM * 2.5625,
+             "kv_dequant_ms": 2 * syn.KV_SLOTS * syn.KV_TOKENS * syn.KV_HEADS * syn.KV_DIM * 2.5625}
+        if rank == 0:
+            print(json.dumps({k: {"ms": round(v, 4), "GB/s": round(b[k] / (v * 1e-3) / 1e9, 1),
+                                  "frac_hbm": round(b[k] / (v * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+                              for k, v in res.items()}), flush=True)
         return 0
     if world > 1:
         import datetime

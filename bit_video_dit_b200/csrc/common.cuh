@@ -166,6 +166,27 @@ __device__ __forceinline__ uint32_t encode8(const float* x, float inv) {
     return e2m1x8(y);
 }
 
+// Packed binary32 pairs (f32x2): each lane rounded as its own binary32
+// operation, two elements per instruction.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)));
+    return *reinterpret_cast<const float2*>(&r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)));
+    return *reinterpret_cast<const float2*>(&r);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&b)), "l"(*reinterpret_cast<const unsigned long long*>(&c)));
+    return *reinterpret_cast<const float2*>(&r);
+}
+
 // bf16x8 (one uint4) -> 8 binary32
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float* f) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};

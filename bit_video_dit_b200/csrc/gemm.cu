@@ -390,27 +390,6 @@ __device__ void scale_copier(const Params& p, Smem<Cfg<PAIR>::STAGES>* s, uint8_
 }
 
 // ---------------------------------------------------------------- epilogue --
-// Packed binary32 pairs (f32x2): each lane rounded as its own binary32
-// operation, two elements per instruction.
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    unsigned long long r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
-        "l"(*reinterpret_cast<const unsigned long long*>(&b)));
-    return *reinterpret_cast<const float2*>(&r);
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-    unsigned long long r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
-        "l"(*reinterpret_cast<const unsigned long long*>(&b)));
-    return *reinterpret_cast<const float2*>(&r);
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-    unsigned long long r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(*reinterpret_cast<const unsigned long long*>(&a)),
-        "l"(*reinterpret_cast<const unsigned long long*>(&b)), "l"(*reinterpret_cast<const unsigned long long*>(&c)));
-    return *reinterpret_cast<const float2*>(&r);
-}
-
 // GELU, tanh form, on a pair: (y / 2) (1 + tanh(u)) with u = sqrt(2/pi) (y +
 // 0.044715 y^3) = y * (sqrt(2/pi) + sqrt(2/pi) 0.044715 y^2) and the hardware
 // tanh (tanh.approx.f32): the value moves by at most ~3e-4 |y| from the exact

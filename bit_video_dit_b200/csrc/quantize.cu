@@ -164,8 +164,13 @@ struct EncodeConsts {
 // the low nibble); a flushed block (inv == 0) is +0 codes.
 __device__ __forceinline__ uint2 encode16(const float* f, float inv) {
     float y[16];
+    const float2 iv = make_float2(inv, inv);
 #pragma unroll
-    for (int i = 0; i < 16; i++) y[i] = __fmul_rn(f[i], inv);
+    for (int i = 0; i < 8; i++) {
+        const float2 t = mul2(make_float2(f[2 * i], f[2 * i + 1]), iv);
+        y[2 * i] = t.x;
+        y[2 * i + 1] = t.y;
+    }
     return make_uint2(inv == 0.0f ? 0u : e2m1x8(y), inv == 0.0f ? 0u : e2m1x8(y + 8));
 }
 
@@ -517,6 +522,249 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
                 const int64_t r = rows + i / sc_pad, c = i % sc_pad;
                 sb[swz_offset(r, c, tiles_c)] = 0;
             }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// LayerNorm + adaLN modulate + quantize in one cooperative launch, for inputs
+// whose rows fit in shared memory (one CTA of 512 threads per SM holds
+// ceil(rows / #SMs) rows):
+//   load     thread 0 bulk-copies the CTA's contiguous rows into shared
+//            memory (one cp.async.bulk per row) while the threads stage
+//            fl32(1 + scale[c]) and shift[c] as binary32;
+//   phase 1  a warp per row: the row statistics from shared memory in the
+//            fixed order of the two-launch path (lane j sums the 16-element
+//            blocks j, j+32, ... in order, the 32 partials meet in an xor
+//            butterfly; S2 over fl32(x - mean)^2), so both paths give the same
+//            bits; then the block maxima of the modulated values
+//            m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift)
+//            and the CTA's maximum;
+//   barrier  the fused quantize's bounded grid barrier turns the CTAs' maxima
+//            into a32 = max |m| / 2688;
+//   phase 2  every block of m is recomputed from shared memory and encoded.
+// HBM: the input is read once and the codes and scales written once.
+// ---------------------------------------------------------------------------
+struct LnArgs {
+    const uint8_t* x;
+    int64_t ld_bytes;
+    int rows, cols;
+    float eps;
+    const __nv_bfloat16* mod_scale;  // NULL: 0
+    const __nv_bfloat16* mod_shift;  // NULL: 0
+    uint8_t* codes;
+    uint8_t* scales;
+    float* gscale;
+    int given;
+    int swizzled;
+    int64_t tile_row;  // swizzled scales: bytes per 128-row block (cols / 64 * 512)
+    float2* stats;     // (mean, rstd) per row, written for the caller
+    uint32_t* ctl;
+    DevError* err;
+    uint64_t limit_ns;
+};
+
+__device__ __forceinline__ float ln_butterfly(float s) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
+    return s;
+}
+
+// the 16 bf16 of block b of a row staged in shared memory, as binary32
+__device__ __forceinline__ void ln_block(const uint8_t* row, int b, float* f) {
+    const uint4* p = reinterpret_cast<const uint4*>(row + b * 32);
+    bf16x8_to_f32(p[0], f);
+    bf16x8_to_f32(p[1], f + 8);
+}
+
+// the block's modulated values m (in place over x) and their |m| max
+__device__ __forceinline__ float ln_modulate16(float* f, float mean, float rstd, const float* sc1, const float* sh) {
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const float h = __fmul_rn(__fsub_rn(f[i], mean), rstd);
+        f[i] = __fadd_rn(__fmul_rn(h, sc1[i]), sh[i]);
+        mx = fmaxf(mx, fabsf(f[i]));
+    }
+    return mx;
+}
+
+template <bool SEARCH>
+__global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __grid_constant__ LnArgs a) {
+    extern __shared__ __align__(16) uint8_t ln_smem[];
+    __shared__ uint64_t bar;
+    __shared__ uint32_t s_red[kQWarps];
+    __shared__ float s_inv[256];
+    __shared__ float s_a32, s_d6, s_d4;
+    __shared__ uint32_t s_total;
+    __shared__ int s_ok;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x;
+    const int r0 = (int)((int64_t)a.rows * blockIdx.x / G), r1 = (int)((int64_t)a.rows * (blockIdx.x + 1) / G);
+    const int nr = r1 - r0, cols = a.cols, nb = cols / 16;
+    const int64_t row_bytes = (int64_t)cols * 2;
+    uint8_t* xs = ln_smem;                                              // [nr][cols] bf16
+    float* sc1 = reinterpret_cast<float*>(ln_smem + (int64_t)nr * row_bytes);  // [cols] fl32(1 + scale)
+    float* sh = sc1 + cols;                                             // [cols] shift
+    float2* st = reinterpret_cast<float2*>(sh + cols);                  // [nr] (mean, rstd)
+    const uint32_t epoch = *(volatile uint32_t*)&a.ctl[kCtlEpoch] + 1u;  // same for every CTA of this launch
+    const int par = (int)(epoch & 1u);
+    if (threadIdx.x == 0) {
+        s_ok = 1;
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        mbar_expect_tx(&bar, (uint32_t)(nr * row_bytes));
+        for (int r = 0; r < nr; r++) bulk_load(xs + r * row_bytes, a.x + (int64_t)(r0 + r) * a.ld_bytes, (uint32_t)row_bytes, &bar);
+    }
+    for (int c = threadIdx.x; c < cols; c += kQThreads) {
+        sc1[c] = a.mod_scale ? __fadd_rn(1.0f, __bfloat162float(a.mod_scale[c])) : 1.0f;
+        sh[c] = a.mod_shift ? __bfloat162float(a.mod_shift[c]) : 0.0f;
+    }
+    __syncthreads();
+    {
+        volatile int never = 0;
+        const bool got = nr == 0 || mbar_wait_bounded(&bar, 0, &never, a.limit_ns);
+        if (!__syncthreads_and(got)) {
+            if (threadIdx.x == 0) record_error(a.err, NVFP4_ERR_TIMEOUT, 6);
+            return;
+        }
+    }
+    // ---- phase 1: statistics and the block maxima of m, a warp per row
+    const float n = (float)cols;
+    float lmax = 0.0f;
+    for (int r = warp; r < nr; r += kQWarps) {
+        const uint8_t* row = xs + r * row_bytes;
+        float s1 = 0.0f;
+        for (int b = lane; b < nb; b += 32) {
+            float f[16];
+            ln_block(row, b, f);
+#pragma unroll
+            for (int i = 0; i < 16; i++) s1 = __fadd_rn(s1, f[i]);
+        }
+        const float mean = __fdiv_rn(ln_butterfly(s1), n);
+        float s2 = 0.0f;
+        for (int b = lane; b < nb; b += 32) {
+            float f[16];
+            ln_block(row, b, f);
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const float d = __fsub_rn(f[i], mean);
+                s2 = __fadd_rn(s2, __fmul_rn(d, d));
+            }
+        }
+        const float var = __fdiv_rn(ln_butterfly(s2), n);
+        const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+        if (lane == 0) {
+            st[r] = make_float2(mean, rstd);
+            a.stats[r0 + r] = make_float2(mean, rstd);
+        }
+        if (!a.given) {
+            for (int b = lane; b < nb; b += 32) {
+                float f[16];
+                ln_block(row, b, f);
+                lmax = fmaxf(lmax, ln_modulate16(f, mean, rstd, sc1 + b * 16, sh + b * 16));
+            }
+        }
+    }
+    if (!a.given) {
+        uint32_t m = __float_as_uint(lmax);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) s_red[warp] = m;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t c0 = 0u;
+#pragma unroll
+            for (int i = 0; i < kQWarps; i++) c0 = max(c0, s_red[i]);
+            uint32_t* cnt = a.ctl + kCtlCount + par;
+            uint32_t* mx = a.ctl + kCtlMax + 2 * par;
+            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(c0) : "memory");
+            uint32_t old;
+            asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
+            const uint64_t t_start = global_ns();
+            uint32_t cnt_now = old + 1u;
+            while (cnt_now < (uint32_t)G) {
+                __nanosleep(20);
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cnt_now) : "l"(cnt) : "memory");
+                if (cnt_now < (uint32_t)G && global_ns() - t_start > a.limit_ns) {
+                    record_error(a.err, NVFP4_ERR_TIMEOUT, 2);
+                    s_ok = 0;
+                    break;
+                }
+            }
+            uint32_t t0;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t0) : "l"(mx) : "memory");
+            s_total = t0;
+        }
+        __syncthreads();
+        if (!s_ok) return;
+        if (threadIdx.x == 0) {
+            const float a32 = __fdiv_rn(__uint_as_float(s_total), 2688.0f);  // amax / (6 * 448)
+            s_a32 = a32;
+            if (blockIdx.x == 0) *a.gscale = a32;
+        }
+        // every CTA has counted itself in: reset the other parity's words, then publish the epoch
+        if (blockIdx.x == 0 && threadIdx.x == 32) {
+            a.ctl[kCtlCount + (par ^ 1)] = 0u;
+            a.ctl[kCtlMax + 2 * (par ^ 1)] = 0u;
+            a.ctl[kCtlMax + 2 * (par ^ 1) + 1] = 0u;
+            __threadfence();
+            *(volatile uint32_t*)&a.ctl[kCtlEpoch] = epoch;
+        }
+    } else if (threadIdx.x == 0) {
+        s_a32 = *a.gscale;
+    }
+    __syncthreads();
+    {
+        const int c = threadIdx.x;
+        if (c < 256) {
+            const float sv = e4m3_value((uint32_t)c);
+            s_inv[c] = (s_a32 == 0.0f || sv == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sv, s_a32));
+        }
+        if (threadIdx.x == 0) {
+            s_d6 = __fmul_rn(6.0f, s_a32);
+            s_d4 = __fmul_rn(4.0f, s_a32);
+        }
+        __syncthreads();
+    }
+    // ---- phase 2: encode every block of m
+    const EncodeConsts kc{s_a32, s_d6, s_d4, s_inv};
+    const int64_t tiles_c = cols / 64;
+    for (int r = warp; r < nr; r += kQWarps) {
+        const uint8_t* row = xs + r * row_bytes;
+        const float2 rs = st[r];
+        const int64_t gr = r0 + r;
+        uint8_t* crow = a.codes + gr * (cols / 2);
+        for (int b = lane; b < nb; b += 32) {
+            float f[16];
+            ln_block(row, b, f);
+            const float amax_b = ln_modulate16(f, rs.x, rs.y, sc1 + b * 16, sh + b * 16);
+            uint32_t code = kc.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, kc.d6));
+            uint2 cw = encode16(f, kc.inv_tab[code]);
+            if (SEARCH) {
+                const uint32_t code4 = kc.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, kc.d4));
+                const uint2 c4 = encode16(f, kc.inv_tab[code4]);
+                if (block_sq_error(f, c4, e4m3_value(code4), kc.a32) < block_sq_error(f, cw, e4m3_value(code), kc.a32)) {
+                    code = code4;
+                    cw = c4;
+                }
+            }
+            *reinterpret_cast<uint2*>(crow + b * 8) = cw;
+            if (a.swizzled)
+                a.scales[swz_offset(gr, b, tiles_c)] = (uint8_t)code;
+            else
+                a.scales[gr * nb + b] = (uint8_t)code;
+        }
+    }
+    // zero the padding rows of the swizzled scale tiles (rows past `rows` up to the next multiple of 128)
+    if (a.swizzled) {
+        const int64_t rows_pad = ((int64_t)a.rows + 127) / 128 * 128;
+        const int64_t sc_pad = tiles_c * 4;
+        const int64_t npad = (rows_pad - a.rows) * sc_pad;
+        for (int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x; i < npad; i += (int64_t)G * kQThreads) {
+            const int64_t r = a.rows + i / sc_pad, c = i % sc_pad;
+            a.scales[swz_offset(r, c, tiles_c)] = 0;
         }
     }
 }
@@ -885,6 +1133,11 @@ static PerDevice<DequantResidency> g_dequant_resident;
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// dynamic shared memory of the one-launch LayerNorm quantize (rows, vectors,
+// statistics); larger inputs take the two-launch path
+constexpr int64_t kLnSmemMax = 200 * 1024;
+static PerDevice<bool> g_ln_attr;
+
 static int grid_for(int64_t work_items, int per_cta, int cap) {
     int64_t g = (work_items + per_cta - 1) / per_cta;
     if (g < 1) g = 1;
@@ -1031,6 +1284,58 @@ extern "C" nvfp4_status nvfp4_ln_modulate_quantize(const void* x_bf16, int64_t r
         return NVFP4_ERR_MISALIGNED;
     // the row statistics follow the 256-byte control block
     float2* stats = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + 256);
+    // one launch when each CTA's rows fit in shared memory with the staged vectors
+    const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), rows);
+    const int64_t rows_per_cta = (rows + G - 1) / G;
+    const int64_t smem = rows_per_cta * cols * 2 + cols * 8 + rows_per_cta * 8;
+    if (smem <= kLnSmemMax) {
+        LnArgs la{};
+        la.x = static_cast<const uint8_t*>(x_bf16);
+        la.ld_bytes = ld * 2;
+        la.rows = (int)rows;
+        la.cols = (int)cols;
+        la.eps = eps;
+        la.mod_scale = static_cast<const __nv_bfloat16*>(mod_scale);
+        la.mod_shift = static_cast<const __nv_bfloat16*>(mod_shift);
+        la.codes = static_cast<uint8_t*>(codes);
+        la.scales = static_cast<uint8_t*>(scales);
+        la.gscale = global_scale;
+        la.given = (flags & NVFP4_Q_GIVEN_GLOBAL) != 0;
+        la.swizzled = (flags & NVFP4_Q_ROWMAJOR_SCALES) == 0;
+        la.tile_row = cols / 64 * 512;
+        la.stats = stats;
+        la.ctl = static_cast<uint32_t*>(workspace);
+        la.err = static_cast<DevError*>(workspace);
+        la.limit_ns = 2000000000ull;
+        const bool search = (flags & NVFP4_Q_SCALE_SEARCH) != 0;
+        void (*kern)(LnArgs) = search ? ln_quantize_smem_kernel<true> : ln_quantize_smem_kernel<false>;
+        bool attr_ok = false;
+        const nvfp4_status ast = g_ln_attr.get(&attr_ok, [](int, bool& v) {
+            if (cudaFuncSetAttribute(ln_quantize_smem_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kLnSmemMax) != cudaSuccess ||
+                cudaFuncSetAttribute(ln_quantize_smem_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kLnSmemMax) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+            v = true;
+            return NVFP4_OK;
+        });
+        if (ast != NVFP4_OK) return ast;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(G);
+        cfg.blockDim = dim3(kQThreads);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cfg.stream = (cudaStream_t)stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, la) != cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_CUDA;
+        }
+        return NVFP4_OK;
+    }
     ln_stats_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, (cudaStream_t)stream>>>(
         static_cast<const uint8_t*>(x_bf16), ld * 2, (int)rows, (int)cols, eps, stats);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_CUDA;

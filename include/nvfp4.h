@@ -158,8 +158,13 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * nvfp4_quantize quantizes a tensor (flags as there), a32 from max |m|.
  * cols % 64 == 0, cols <= 2^24, rows <= 2^30; pointers 16-byte aligned.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_LN_QUANTIZE, rows, 0, cols)
- * bytes (the control block, then 8 bytes of row statistics per row).
- * Two launches: the row statistics, then the fused quantize. */
+ * bytes (the control block, then the binary32 (mean, rstd) of every row,
+ * which the call leaves there).  One cooperative launch when ceil(rows /
+ * #SMs) rows fit in a CTA's shared memory (about 200 KB: 4096 x 3072 does,
+ * 8192 x 3072 does not): the rows are bulk-copied in once, the statistics,
+ * the tensor maximum and the encode all read them there.  Otherwise two
+ * launches: the row statistics, then the fused quantize.  Both give the same
+ * bits. */
 nvfp4_status nvfp4_ln_modulate_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                         const void* mod_scale, const void* mod_shift, float eps, void* codes,
                                         void* scales, float* global_scale, unsigned flags, void* workspace,

@@ -50,9 +50,17 @@ def _check(x_bits, scale=None, shift=None, *, eps=1e-6, ld=None, alpha=None, row
 
 
 def test_dit_activation_full_size():
+    """4096 x 3072: each CTA's rows fit in shared memory, so one launch."""
     D = syn.QKV.K
     _check(syn.activations_bf16(4096, D, seed=71), syn.normal_bf16((D,), seed=72, std=0.1),
            syn.normal_bf16((D,), seed=73, std=0.1))
+
+
+def test_rows_beyond_shared_memory_take_the_two_launch_path():
+    """8192 x 3072 (56 rows a CTA, 344 KB): the statistics kernel, then the fused quantize."""
+    D = syn.QKV.K
+    _check(syn.activations_bf16(8192, D, seed=74), syn.normal_bf16((D,), seed=75, std=0.1),
+           syn.normal_bf16((D,), seed=76, std=0.1))
 
 
 @pytest.mark.parametrize("rows,cols,ld", [(200, 320, None), (129, 576, 640), (1, 64, None), (3, 14336, None)])
