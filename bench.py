@@ -141,9 +141,10 @@ def kernel_hash(files=("common.cuh", "gemm.cu")) -> str:
 
 
 def recorded_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current kernel sources."""
-    path = os.path.join(ROOT, "profiles", "gemm_qkv_traffic.txt")
+    """DRAM bytes per GEMM launch of the stack (mean over a layer's four, and
+    per GEMM) from the committed ncu summary, if it was taken on the current
+    kernel sources."""
+    path = os.path.join(ROOT, "profiles", "gemm_stack_traffic.txt")
     try:
         with open(path) as f:
             r = json.load(f)
@@ -622,7 +623,8 @@ def run_ours(args, rank: int, world: int) -> dict | None:
                "train": measure_training(nv, lk["a"], lk["w"], lk["cache"], lk["ring"], lk["k_out"], lk["v_out"],
                                          reps=5),
                "attn": measure_attention(nv, lk["cache"], lk["ring"], lk["k_out"], lk["v_out"], reps=3),
-               "ffn": measure_ffn(nv, flush, dev, reps=5)}
+               "ffn": measure_ffn(nv, flush, dev, reps=5),
+               "stream": measure_codec_stream(nv, dev, rounds=4)}
 
     keys = ["input_quantize", *STACK_NAMES]
     times = torch.tensor([total_ms, *[comp[k] for k in keys], e2e_ms,
@@ -654,16 +656,18 @@ def report(args, world, st, total_ms, comp, e2e_ms, clk, sub, lin) -> dict:
     shapes = {"qkv": (3 * D, D), "out": (D, D), "up": (F, D), "down": (D, F)}
     gemm_ms = sum(comp[k] for k in STACK_NAMES)  # per layer
     gemm_tflops = flops / L / (gemm_ms * 1e-3) / 1e12
+    tr = recorded_traffic()
     by = {}
     for k in STACK_NAMES:
         N, K = shapes[k]
         t = 2.0 * M * N * K / (comp[k] * 1e-3) / 1e12
+        g = None if tr is None else tr["per_gemm"][k]
         by[f"gemm_{k}"] = _rl("tensor", t, fp4_sus, "TFLOP/s", ms=round(comp[k], 4), shape=[M, N, K],
-                              frac_of_burst=round(t / fp4_peak, 4))
+                              frac_of_burst=round(t / fp4_peak, 4),
+                              traffic=None if g is None else g["dram_read"] + g["dram_write"])
     qbytes = M * D * 2.5625
     by["input_quantize"] = _rl("hbm", qbytes / (comp["input_quantize"] * 1e-3) / 1e9, pk["hbm_gbs"], "GB/s",
                                ms=round(comp["input_quantize"], 4))
-    tr = recorded_traffic()
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -727,11 +731,21 @@ def sub_report(sub, lin, pk, fp4_peak) -> dict:
                     "pre-quantized; graph with events, the KV dequant's 681 MB output flushing L2 every step",
             "TFLOP/s": round(flops / ((q_ms + g_ms) * 1e-3) / 1e12, 1),
             "gemm": _rl("tensor", flops / (g_ms * 1e-3) / 1e12, fp4_peak, "TFLOP/s", ms=round(g_ms, 4)),
-            "quantize": _rl("hbm", gbs(quant_bytes, q_ms), pk["hbm_gbs"], "GB/s", ms=round(q_ms, 4))},
+            "quantize": _rl("hbm", gbs(quant_bytes, q_ms), pk["hbm_gbs"], "GB/s", ms=round(q_ms, 4),
+                            timing="inside the step graph, events around the launch (their own ~5.5 us included)"),
+            "quantize_back_to_back": _rl("hbm", gbs(quant_bytes, sub["stream"]["quantize_ms"]), pk["hbm_gbs"],
+                                         "GB/s", ms=round(sub["stream"]["quantize_ms"], 4),
+                                         timing="32 launches back to back over 8 rotating 25 MB inputs (201 MB > "
+                                                "L2), one pair of events")},
         "kv": {
             "what": "NVFP4 KV cache of 21 slots x 2640 x 24 x 128: append of one K/V chunk (in place into ring "
                     "slot step mod 21), dequant-gather of all 21 slots to bf16",
-            "append": _rl("hbm", gbs(append_bytes, ap_ms), pk["hbm_gbs"], "GB/s", ms=round(ap_ms, 4)),
+            "append": _rl("hbm", gbs(append_bytes, ap_ms), pk["hbm_gbs"], "GB/s", ms=round(ap_ms, 4),
+                          timing="inside the step graph, events around the launch (their own ~5.5 us included)"),
+            "append_back_to_back": _rl("hbm", gbs(append_bytes, sub["stream"]["kv_append_ms"]), pk["hbm_gbs"],
+                                       "GB/s", ms=round(sub["stream"]["kv_append_ms"], 4),
+                                       timing="32 appends back to back over 8 rotating 32 MB K/V chunks (260 MB > "
+                                              "L2) into 8 slots, one pair of events"),
             "dequant": _rl("hbm", gbs(dequant_bytes, dq_ms), pk["hbm_gbs"], "GB/s", ms=round(dq_ms, 4)),
             "cache_bytes": sub["lk"]["cache"].nbytes()},
         "scale_search": {
@@ -780,7 +794,9 @@ def sub_report(sub, lin, pk, fp4_peak) -> dict:
         "ln_modulate_quantize": {
             "what": "LayerNorm + adaLN modulate + NVFP4 quantize of A [4096x3072]",
             "ms": round(search["ln_quantize_ms"], 4),
-            "GB/s": round(gbs(quant_bytes, search["ln_quantize_ms"]), 1)},
+            "GB/s": round(gbs(quant_bytes, search["ln_quantize_ms"]), 1),
+            "back_to_back_ms": round(sub["stream"]["ln_quantize_ms"], 4),
+            "back_to_back_GB/s": round(gbs(quant_bytes, sub["stream"]["ln_quantize_ms"]), 1)},
     }
 
 
@@ -827,6 +843,54 @@ def measure_codecs(nv, dev, reps: int) -> dict:
     torch.cuda.synchronize()
     out = {name: float(np.median([e[0].elapsed_time(e[1]) for e in evs])) for name, evs in ev.items()}
     del g
+    return out
+
+
+def measure_codec_stream(nv, dev, rounds: int) -> dict:
+    """ms per launch of the codec kernels launched back to back inside one
+    graph, every launch on its own buffers from a set larger than L2 (8 copies
+    of A [4096 x 3072], 201 MB; 8 K/V chunk pairs, 260 MB; the outputs rotate
+    too), so each launch reads its inputs from HBM; one pair of events brackets
+    `rounds` x 8 launches, so the events' own cost per kernel (~5.5 us here
+    between two events around even a one-element kernel) is not charged to
+    each launch, only the gaps between launches."""
+    M, K = syn.QKV.M, syn.QKV.K
+    T, H, D = syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    nb = 8
+    a0 = dev_bf16(syn.activations_bf16(M, K, seed=2))
+    acts = [a0.clone() for _ in range(nb)]
+    outs = [nv.empty_nvfp4(M, K, dev) for _ in range(nb)]
+    ws_q = nv.workspace(nv.OP_QUANTIZE, M, 0, K, dev)
+    ws_ln = nv.workspace(nv.OP_LN_QUANTIZE, M, 0, K, dev)
+    sc = dev_bf16(syn.normal_bf16((K,), seed=72, std=0.1))
+    sh = dev_bf16(syn.normal_bf16((K,), seed=73, std=0.1))
+    k0, v0 = (dev_bf16(x) for x in syn.kv_chunk_bf16(T, H, D, seed=50))
+    chunks = [(k0.clone(), v0.clone()) for _ in range(nb)]
+    cache = nv.KVCache(nb, T, H, D, dev)
+    calls = {"quantize_ms": lambda i: nv.quantize(acts[i], out=outs[i], ws=ws_q),
+             "kv_append_ms": lambda i: cache.append(i, *chunks[i]),
+             "ln_quantize_ms": lambda i: nv.ln_modulate_quantize(acts[i], mod_scale=sc, mod_shift=sh, out=outs[i],
+                                                                 ws=ws_ln)}
+    out = {}
+    for name, f in calls.items():
+        for i in range(nb):
+            f(i)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            e0.record()
+            for _ in range(rounds):
+                for i in range(nb):
+                    f(i)
+            e1.record()
+        g.replay()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / (rounds * nb)
+        del g
     return out
 
 
@@ -976,15 +1040,17 @@ def main(argv=None) -> int:
         from bit_video_dit_b200 import build as nvbuild
         from bit_video_dit_b200 import nvfp4 as nv
         nvbuild.build()
-        res = measure_codecs(nv, torch.device("cuda", local), reps=max(3, args.steps))
+        dev = torch.device("cuda", local)
+        res = measure_codecs(nv, dev, reps=max(3, args.steps))
+        stream_res = measure_codec_stream(nv, dev, rounds=max(2, args.steps))
         pk = peaks()
         b = {"quantize_ms": syn.QKV.M * syn.QKV.K * 2.5625, "ln_quantize_ms": syn.QKV.M * syn.QKV.K * 2.5625,
              "kv_append_ms": 2 * syn.KV_TOKENS * syn.KV_HEADS * syn.KV_DIM * 2.5625,
              "kv_dequant_ms": 2 * syn.KV_SLOTS * syn.KV_TOKENS * syn.KV_HEADS * syn.KV_DIM * 2.5625}
+        line = lambda r: {k: {"ms": round(v, 4), "GB/s": round(b[k] / (v * 1e-3) / 1e9, 1),
+                              "frac_hbm": round(b[k] / (v * 1e-3) / 1e9 / pk["hbm_gbs"], 4)} for k, v in r.items()}
         if rank == 0:
-            print(json.dumps({k: {"ms": round(v, 4), "GB/s": round(b[k] / (v * 1e-3) / 1e9, 1),
-                                  "frac_hbm": round(b[k] / (v * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
-                              for k, v in res.items()}), flush=True)
+            print(json.dumps({"flushed_each": line(res), "back_to_back": line(stream_res)}), flush=True)
         return 0
     if world > 1:
         import datetime

@@ -55,7 +55,6 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows,
     if (chk != NVFP4_OK) return chk;
     if (rows == 0) return NVFP4_OK;
     if (nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols) > kNoAllocScratchBytes) return NVFP4_ERR_UNSUPPORTED;
-    if (rows * ((cols + 511) / 512) > ((int64_t)1 << 30) || cols > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
     void* scratch = nullptr;
     const nvfp4_status st = scratch_for_current_device(&scratch);
     if (st != NVFP4_OK) return st;

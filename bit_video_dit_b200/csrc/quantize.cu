@@ -32,10 +32,10 @@ constexpr int kThreads = 256;  // dequant / probe kernels
 // ---------------------------------------------------------------------------
 // Fused quantize: one cooperative launch, one CTA of 512 threads per SM.
 //   phase 1  every warp takes a contiguous share of one tensor's 512-element
-//            row runs and loads up to kMaxRuns of them straight into
-//            registers -- a lane holds one 16-element block per run, all
-//            loads in flight at once -- keeping each block's |x| max (taken
-//            on the bf16 bit patterns) for phase 2;
+//            runs (the tensor's elements in row order, 32 blocks of 16 a run)
+//            and loads up to kMaxRuns of them straight into registers -- a
+//            lane holds one 16-element block per run, all loads in flight at
+//            once -- and takes their |x| max (on the bf16 bit patterns);
 //   barrier  each CTA folds its maxima into two global maxima (fire-and-
 //            forget reductions) and counts itself in with an acquire-release
 //            add; every CTA polls the count (bounded wait), then reads the
@@ -44,22 +44,25 @@ constexpr int kThreads = 256;  // dequant / probe kernels
 //            lane (the reciprocal 1 / (s * a32) from a 256-entry table per
 //            tensor, built once per CTA), 8-byte code stores (256 contiguous
 //            bytes per warp).
-// A warp walks its runs with row pointers it advances, so no run needs an
-// integer division, and the scale layout is a template parameter.  HBM is
-// read once and written once; runs beyond kMaxRuns per warp (tensors larger
-// than ~#SMs x 176 KB) are read again in phase 2 (from L2 when the tensor
-// fits there).
+// A block's row comes from its index by a multiply-high with a per-shape
+// magic number (no division, no state carried from run to run), so the runs
+// a lane holds are independent and their encodes interleave; the scale
+// layout is a template parameter.  HBM is read once and written once; runs
+// beyond kMaxRuns per warp (tensors larger than ~#SMs x 176 KB) are read
+// again in phase 2, several at a time (from L2 when the tensor fits there).
 // ---------------------------------------------------------------------------
 constexpr int kQThreads = 512;
 constexpr int kQWarps = kQThreads / 32;
 constexpr int kMaxRuns = 11;   // runs held in registers per warp (11 x 32 B per lane)
+constexpr int kBatch = 2;      // runs past the held ones, loaded together (phase 1)
+constexpr int kBatch2 = 6;     // the same in phase 2, once the held runs are encoded
 constexpr int kMaxGrid = 1024;
 
 // Control block (uint32 words of the workspace's first 256 bytes, zero before
 // first use; words 0..3 are the error record):
 constexpr int kCtlEpoch = 8;   // epoch of the last completed launch
 constexpr int kCtlCount = 16;  // [2] arrivals of the launch with epoch parity p
-constexpr int kCtlMax = 20;    // [2][2] bf16 magnitude maxima per parity, per tensor
+constexpr int kCtlMax = 20;    // [2][2] magnitude maxima per parity, per tensor
 
 struct QuantArgs {
     const uint8_t* x[2];
@@ -67,12 +70,12 @@ struct QuantArgs {
     uint8_t* scales[2];
     float* gscale[2];
     int64_t ld_bytes;      // row stride of x in bytes
-    int64_t code_ld;       // bytes per row of codes (cols / 2)
-    int64_t scale_ld;      // bytes per row of row-major scales (cols / 16)
-    int64_t tile_row;      // bytes per 128-row block of swizzled scales (cols / 64 * 512)
-    int upr;               // 512-element runs per row
-    int last_nblk;         // 16-element blocks in the last run of a row
-    int runs_per_tensor;
+    int64_t tiles_c;       // swizzled scales: 4-column tiles per row block (cols / 64)
+    uint32_t nblk;         // 16-element blocks per tensor (rows * cols / 16 < 2^31)
+    uint32_t nb;           // blocks per row (cols / 16)
+    uint32_t nb_magic;     // block b's row = umulhi(b, nb_magic) >> nb_shift
+    int nb_shift;
+    int runs_per_tensor;   // ceil(nblk / 32)
     int ntensors;
     int given;
     // LayerNorm + modulate ahead of the quantize (LN kernels only): per-row
@@ -80,7 +83,6 @@ struct QuantArgs {
     const float2* ln_stats;
     const __nv_bfloat16* mod_scale;
     const __nv_bfloat16* mod_shift;
-    int cols;
     // K-smoothing ahead of the quantize (smoothing kernels only, one row per
     // tensor): binary32 channel means [smooth_hd] per tensor (NULL: none);
     // the element at flat index i belongs to channel i mod smooth_hd
@@ -120,37 +122,20 @@ __device__ __forceinline__ uint4 ld_stream16_if(const void* p, bool pred) {
     return v;
 }
 
-// A warp's position: run cr of row r of its tensor, with the row's pointers.
-template <bool SWZ>
-struct Walk {
-    int r, cr;
-    const uint8_t* xrow;
-    uint8_t* crow;
-    uint8_t* srow;  // SWZ: this row's base inside its 128-row block of tiles
-
-    __device__ __forceinline__ void seek(const QuantArgs& a, int t, int run) {
-        r = run / a.upr;
-        cr = run - r * a.upr;
-        xrow = a.x[t] + (int64_t)r * a.ld_bytes;
-        crow = a.codes[t] + (int64_t)r * a.code_ld;
-        srow = a.scales[t] + (SWZ ? (int64_t)(r >> 7) * a.tile_row + (r & 31) * 16 + ((r >> 5) & 3) * 4
-                                  : (int64_t)r * a.scale_ld);
+// Where the lane's block of run `run` (tensor t) lives: block index b in the
+// tensor, its row r and block column cb; valid when b is inside the tensor.
+struct Blk {
+    uint32_t b, r, cb;
+    bool valid;
+    __device__ __forceinline__ Blk(const QuantArgs& a, int run, int lane) {
+        b = (uint32_t)run * 32u + (uint32_t)lane;
+        valid = b < a.nblk;
+        r = __umulhi(b, a.nb_magic) >> a.nb_shift;
+        cb = b - r * a.nb;
     }
-    __device__ __forceinline__ void next(const QuantArgs& a) {
-        if (++cr == a.upr) {
-            cr = 0;
-            ++r;
-            xrow += a.ld_bytes;
-            crow += a.code_ld;
-            if (SWZ) {
-                // rows 32 apart share a 16-byte tile row; a new 128-row block starts a new tile row
-                srow += (r & 127) == 0 ? a.tile_row - 3 * 4 - 31 * 16 : ((r & 31) == 0 ? 4 - 31 * 16 : 16);
-            } else {
-                srow += a.scale_ld;
-            }
-        }
+    __device__ __forceinline__ const uint8_t* src(const QuantArgs& a, int t) const {
+        return (t ? a.x[1] : a.x[0]) + (int64_t)r * a.ld_bytes + (int64_t)cb * 32;
     }
-    __device__ __forceinline__ int nblk(const QuantArgs& a) const { return cr == a.upr - 1 ? a.last_nblk : 32; }
 };
 
 // Per-tensor constants of the encode: a32, 6 a32, 4 a32 (targets of the
@@ -194,29 +179,30 @@ __device__ __forceinline__ float block_sq_error(const float* f, uint2 c, float s
     return sum;
 }
 
-// encode one 16-element block (lane `lane` of the run at w) and store codes +
-// scale.  SEARCH: also encode with the block max aimed at 4 instead of 6 and
-// keep that encoding when its squared error is smaller.
+// encode the lane's 16-element block and store its codes + scale.  SEARCH:
+// also encode with the block max aimed at 4 instead of 6 and keep that
+// encoding when its squared error is smaller.
 template <bool SWZ, bool SEARCH>
-__device__ __forceinline__ void encode_block(const Walk<SWZ>& w, int lane, bool valid, const float* f, float amax_b,
-                                             const EncodeConsts& k) {
+__device__ __forceinline__ void encode_block(const QuantArgs& a, int t, const Blk& k, const float* f, float amax_b,
+                                             const EncodeConsts& kc) {
     // s = E4M3(amax_b / (6 a32)); a zero tensor scale flushes every block
-    uint32_t code = k.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, k.d6));
-    uint2 c = encode16(f, k.inv_tab[code]);
+    uint32_t code = kc.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, kc.d6));
+    uint2 c = encode16(f, kc.inv_tab[code]);
     if (SEARCH) {
-        const uint32_t code4 = k.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, k.d4));
-        const uint2 c4 = encode16(f, k.inv_tab[code4]);
-        if (block_sq_error(f, c4, e4m3_value(code4), k.a32) < block_sq_error(f, c, e4m3_value(code), k.a32)) {
+        const uint32_t code4 = kc.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, kc.d4));
+        const uint2 c4 = encode16(f, kc.inv_tab[code4]);
+        if (block_sq_error(f, c4, e4m3_value(code4), kc.a32) < block_sq_error(f, c, e4m3_value(code), kc.a32)) {
             code = code4;
             c = c4;
         }
     }
-    if (valid) {
-        *reinterpret_cast<uint2*>(w.crow + w.cr * 256 + 8 * lane) = c;
+    if (k.valid) {
+        *reinterpret_cast<uint2*>((t ? a.codes[1] : a.codes[0]) + (int64_t)k.b * 8) = c;
+        uint8_t* sc = t ? a.scales[1] : a.scales[0];
         if (SWZ)
-            w.srow[(int64_t)(w.cr * 8 + (lane >> 2)) * 512 + (lane & 3)] = (uint8_t)code;
+            sc[swz_offset(k.r, k.cb, a.tiles_c)] = (uint8_t)code;
         else
-            w.srow[w.cr * 32 + lane] = (uint8_t)code;
+            sc[k.b] = (uint8_t)code;
     }
 }
 
@@ -225,22 +211,22 @@ constexpr int kXfNone = 0;    // the bf16 input as is
 constexpr int kXfLn = 1;      // LayerNorm + adaLN modulate of each row
 constexpr int kXfSmooth = 2;  // RoPE of the keys, then minus the channel mean (KV chunk)
 
-// The 16 binary32 values of the lane's block of the run at w (tensor t): the
-// bf16 input; with LN its LayerNorm + modulate, in this order and rounding:
+// The 16 binary32 values of the lane's block k (tensor t): the bf16 input;
+// with LN its LayerNorm + modulate, in this order and rounding:
 // m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift);
 // for a KV chunk, the keys' rotary embedding where a table is given (pair
 // (x0, x1) -> (fl32(fl32(x0 c) - fl32(x1 s)), fl32(fl32(x0 s) + fl32(x1 c))),
 // c and s of the element's token and pair), then fl32(y - mean[channel]) where
 // means are given.
-template <int XF, bool SWZ>
-__device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>& w, int t, int lane, bool valid,
-                                             const uint4& q0, const uint4& q1, float* f) {
+template <int XF>
+__device__ __forceinline__ void block_values(const QuantArgs& a, const Blk& k, int t, const uint4& q0, const uint4& q1,
+                                             float* f) {
     bf16x8_to_f32(q0, f);
     bf16x8_to_f32(q1, f + 8);
-    if (XF == kXfSmooth && t == 0 && a.rope_cos && valid) {
+    if (XF == kXfSmooth && t == 0 && a.rope_cos && k.valid) {
         // one row per tensor, fewer than 2^31 elements: the block's 16
         // elements are 8 whole pairs of one head of one token (rope_d % 16 == 0)
-        const uint32_t i0 = (uint32_t)(w.cr * 512 + lane * 16);
+        const uint32_t i0 = k.cb * 16u;
         const uint32_t tok = i0 / (uint32_t)a.rope_hd;
         const uint32_t p0 = (i0 % (uint32_t)a.rope_d) >> 1;
         const size_t off = (size_t)tok * (uint32_t)(a.rope_d >> 1) + p0;  // a multiple of 8 floats
@@ -250,19 +236,18 @@ __device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>
         const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-        for (int k = 0; k < 8; k++) {
-            const float x0 = f[2 * k], x1 = f[2 * k + 1];
-            f[2 * k] = __fsub_rn(__fmul_rn(x0, c[k]), __fmul_rn(x1, sn[k]));
-            f[2 * k + 1] = __fadd_rn(__fmul_rn(x0, sn[k]), __fmul_rn(x1, c[k]));
+        for (int j = 0; j < 8; j++) {
+            const float x0 = f[2 * j], x1 = f[2 * j + 1];
+            f[2 * j] = __fsub_rn(__fmul_rn(x0, c[j]), __fmul_rn(x1, sn[j]));
+            f[2 * j + 1] = __fadd_rn(__fmul_rn(x0, sn[j]), __fmul_rn(x1, c[j]));
         }
     }
     if (XF == kXfSmooth) {
         const float* mean = t ? a.smooth_mean[1] : a.smooth_mean[0];
-        if (valid && mean) {
-            // one row per tensor, fewer than 2^31 elements: the block's first
-            // flat index is w.cr * 512 + lane * 16, and its 16 channels are
-            // consecutive (smooth_hd is a multiple of 16)
-            const uint32_t c0 = (uint32_t)(w.cr * 512 + lane * 16) % (uint32_t)a.smooth_hd;
+        if (k.valid && mean) {
+            // one row per tensor: the block's 16 channels are consecutive
+            // (smooth_hd is a multiple of 16)
+            const uint32_t c0 = (k.cb * 16u) % (uint32_t)a.smooth_hd;
             const float4* p = reinterpret_cast<const float4*>(mean + c0);
 #pragma unroll
             for (int j = 0; j < 4; j++) {
@@ -275,17 +260,17 @@ __device__ __forceinline__ void block_values(const QuantArgs& a, const Walk<SWZ>
         }
     }
     if (XF == kXfLn) {
-        const float2 st = __ldg(a.ln_stats + w.r);
-        const int c0 = w.cr * 512 + lane * 16;
+        const float2 st = k.valid ? __ldg(a.ln_stats + k.r) : make_float2(0.0f, 0.0f);
+        const uint32_t c0 = k.cb * 16u;
         float sc[16], sh[16];
 #pragma unroll
         for (int i = 0; i < 16; i++) sc[i] = sh[i] = 0.0f;
-        if (valid && a.mod_scale) {
+        if (k.valid && a.mod_scale) {
             const uint4* p = reinterpret_cast<const uint4*>(a.mod_scale + c0);
             bf16x8_to_f32(__ldg(p), sc);
             bf16x8_to_f32(__ldg(p + 1), sc + 8);
         }
-        if (valid && a.mod_shift) {
+        if (k.valid && a.mod_shift) {
             const uint4* p = reinterpret_cast<const uint4*>(a.mod_shift + c0);
             bf16x8_to_f32(__ldg(p), sh);
             bf16x8_to_f32(__ldg(p + 1), sh + 8);
@@ -315,6 +300,49 @@ __device__ __forceinline__ uint32_t block_max_key(const uint4& q0, const uint4& 
 template <bool F32>
 __device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float(F32 ? key : key << 16); }
 
+// ---------------------------------------------------------------------------
+// Grid-wide maximum of the cooperative quantize kernels (thread 0 of each
+// CTA): fold the CTA's per-tensor maxima into the launch's global maxima and
+// count the CTA in (acquire-release), wait until every CTA of the launch has
+// (bounded), then read the maxima into total[2].  False when the wait ran out
+// (error recorded).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool grid_max_exchange(uint32_t* ctl, DevError* err, uint64_t limit_ns, int par, int G,
+                                                  uint32_t c0, uint32_t c1, uint32_t* total) {
+    uint32_t* cnt = ctl + kCtlCount + par;
+    uint32_t* mx = ctl + kCtlMax + 2 * par;
+    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(c0) : "memory");
+    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx + 1), "r"(c1) : "memory");
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
+    const uint64_t t_start = global_ns();
+    uint32_t n = old + 1u;
+    bool ok = true;
+    while (n < (uint32_t)G) {
+        __nanosleep(20);
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(cnt) : "memory");
+        if (n < (uint32_t)G && global_ns() - t_start > limit_ns) {
+            record_error(err, NVFP4_ERR_TIMEOUT, 2);
+            ok = false;
+            break;
+        }
+    }
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(total[0]) : "l"(mx) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(total[1]) : "l"(mx + 1) : "memory");
+    return ok;
+}
+
+// After every CTA has counted itself in (so has read the epoch and is done
+// with the other parity's words): reset those for the next launch, then
+// publish this launch's epoch.  One thread of one CTA.
+__device__ __forceinline__ void grid_barrier_retire(uint32_t* ctl, int par, uint32_t epoch) {
+    ctl[kCtlCount + (par ^ 1)] = 0u;
+    ctl[kCtlMax + 2 * (par ^ 1)] = 0u;
+    ctl[kCtlMax + 2 * (par ^ 1) + 1] = 0u;
+    __threadfence();
+    *(volatile uint32_t*)&ctl[kCtlEpoch] = epoch;
+}
+
 template <bool SWZ, bool SEARCH, int XF>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
     constexpr bool F32 = XF != kXfNone;       // 32-bit keys of transformed values
@@ -335,58 +363,50 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
     const int we = (int)((int64_t)a.runs_per_tensor * (wl + 1) / nwt);
     const uint32_t epoch = *(volatile uint32_t*)&a.ctl[kCtlEpoch] + 1u;  // same for every CTA of this launch
     const int par = (int)(epoch & 1u);
-    Walk<SWZ> w0;
-    w0.seek(a, t, min(wb, a.runs_per_tensor - 1));
 
     // ---- phase 1: this warp's runs wb .. we-1 of tensor t, one block per lane
     uint4 q[kRuns][2];
-    uint32_t bm[kRuns];  // the lane's block max key per run
-    {
-        Walk<SWZ> w = w0;
 #pragma unroll
-        for (int k = 0; k < kRuns; k++) {
-            const bool have = wb + k < we;
-            const bool valid = have && lane < w.nblk(a);
-            const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
-            q[k][0] = ld_stream16_if(src, valid);
-            q[k][1] = ld_stream16_if(src + 16, valid);
-            if (have) w.next(a);
-        }
+    for (int k = 0; k < kRuns; k++) {
+        const Blk kb(a, wb + k, lane);
+        const bool ld = wb + k < we && kb.valid;
+        const uint8_t* src = kb.src(a, t);
+        q[k][0] = ld_stream16_if(src, ld);
+        q[k][1] = ld_stream16_if(src + 16, ld);
     }
-    uint32_t m = 0;  // the lane's max key over its runs
-    if constexpr (!F32) {
-        // blocks past the data were loaded as zeros: key 0
+    uint32_t m = 0;  // the lane's max key over its runs (each block's max is taken again in phase 2)
 #pragma unroll
-        for (int k = 0; k < kRuns; k++) {
+    for (int k = 0; k < kRuns; k++) {
+        if constexpr (!F32) {
+            // blocks past the data were loaded as zeros: key 0
             const uint32_t mm = __vmaxu2(absmax_bits8(q[k][0]), absmax_bits8(q[k][1]));
-            bm[k] = max(mm & 0xFFFFu, mm >> 16);
-            m = max(m, bm[k]);
-        }
-    } else {
-        Walk<SWZ> w = w0;
-#pragma unroll
-        for (int k = 0; k < kRuns; k++) {
+            m = max(m, max(mm & 0xFFFFu, mm >> 16));
+        } else {
+            const Blk kb(a, wb + k, lane);
             float f[16];
-            const bool have = wb + k < we;
-            block_values<XF>(a, w, t, lane, have && lane < w.nblk(a), q[k][0], q[k][1], f);
-            bm[k] = have && lane < w.nblk(a) ? block_max_key<F32>(q[k][0], q[k][1], f) : 0u;
-            m = max(m, bm[k]);
-            if (have) w.next(a);
+            block_values<XF>(a, kb, t, q[k][0], q[k][1], f);
+            if (wb + k < we && kb.valid) m = max(m, block_max_key<F32>(q[k][0], q[k][1], f));
         }
     }
     if (threadIdx.x == 0) s_ok = 1;
     if (!a.given) {
-        {
-            Walk<SWZ> w = w0;
-            for (int k = 0; k < kRuns && wb + k < we; k++) w.next(a);
-            for (int g = wb + kRuns; g < we; g++) {
-                const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
-                const bool valid = lane < w.nblk(a);
-                const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
+        // the runs past the held ones, kBatch loads in flight per lane
+        for (int g = wb + kRuns; g < we; g += kBatch) {
+            uint4 v[kBatch][2];
+#pragma unroll
+            for (int u = 0; u < kBatch; u++) {
+                const Blk kb(a, g + u, lane);
+                const bool ld = g + u < we && kb.valid;
+                const uint8_t* src = kb.src(a, t);
+                v[u][0] = ld_stream16_if(src, ld);
+                v[u][1] = ld_stream16_if(src + 16, ld);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; u++) {
+                const Blk kb(a, g + u, lane);
                 float f[16];
-                block_values<XF>(a, w, t, lane, valid, v0, v1, f);
-                if (valid) m = max(m, block_max_key<F32>(v0, v1, f));
-                w.next(a);
+                block_values<XF>(a, kb, t, v[u][0], v[u][1], f);
+                if (g + u < we && kb.valid) m = max(m, block_max_key<F32>(v[u][0], v[u][1], f));
             }
         }
         // 16-bit keys: one word per lane, tensor-1 max in the high half and
@@ -418,30 +438,10 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
                 c0 = c & 0xFFFFu;
                 c1 = c >> 16;
             }
-            uint32_t* cnt = a.ctl + kCtlCount + par;
-            uint32_t* mx = a.ctl + kCtlMax + 2 * par;
-            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(c0) : "memory");
-            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx + 1), "r"(c1) : "memory");
-            uint32_t old;
-            // acquire too: the last CTA to arrive reads the maxima without polling
-            asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
-            // wait for every CTA of this launch (bounded)
-            const uint64_t t_start = global_ns();
-            uint32_t n = old + 1u;
-            while (n < (uint32_t)G) {
-                __nanosleep(20);
-                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(cnt) : "memory");
-                if (n < (uint32_t)G && global_ns() - t_start > a.limit_ns) {
-                    record_error(a.err, NVFP4_ERR_TIMEOUT, 2);
-                    s_ok = 0;
-                    break;
-                }
-            }
-            uint32_t t0, t1;
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t0) : "l"(mx) : "memory");
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t1) : "l"(mx + 1) : "memory");
-            s_total[0] = t0;
-            s_total[1] = t1;
+            uint32_t tot[2];
+            if (!grid_max_exchange(a.ctl, a.err, a.limit_ns, par, G, c0, c1, tot)) s_ok = 0;
+            s_total[0] = tot[0];
+            s_total[1] = tot[1];
         }
         __syncthreads();
         if (!s_ok) return;
@@ -450,16 +450,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
             s_d6[threadIdx.x] = a32;  // a32 for now; the table below needs it
             if (blockIdx.x == 0) *(threadIdx.x ? a.gscale[1] : a.gscale[0]) = a32;
         }
-        // every CTA of this launch has counted itself in, and so has read the
-        // epoch and finished with the other parity's words: reset those for
-        // the next launch, then let it see the new epoch
-        if (blockIdx.x == 0 && threadIdx.x == 32) {
-            a.ctl[kCtlCount + (par ^ 1)] = 0u;
-            a.ctl[kCtlMax + 2 * (par ^ 1)] = 0u;
-            a.ctl[kCtlMax + 2 * (par ^ 1) + 1] = 0u;
-            __threadfence();
-            *(volatile uint32_t*)&a.ctl[kCtlEpoch] = epoch;
-        }
+        if (blockIdx.x == 0 && threadIdx.x == 32) grid_barrier_retire(a.ctl, par, epoch);
     } else {
         if (threadIdx.x < a.ntensors) s_d6[threadIdx.x] = *(threadIdx.x ? a.gscale[1] : a.gscale[0]);
     }
@@ -486,41 +477,49 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
     // ---- phase 2: encode
     {
         const EncodeConsts kc{s_a32[t], s_d6[t], s_d4[t], s_inv[t]};
-        Walk<SWZ> w = w0;
 #pragma unroll
         for (int k = 0; k < kRuns; k++) {
             if (wb + k < we) {
-                const bool valid = lane < w.nblk(a);
+                const Blk kb(a, wb + k, lane);
                 float f[16];
-                block_values<XF>(a, w, t, lane, valid, q[k][0], q[k][1], f);
-                encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<F32>(bm[k]), kc);
-                w.next(a);
+                block_values<XF>(a, kb, t, q[k][0], q[k][1], f);
+                encode_block<SWZ, SEARCH>(a, t, kb, f, key_value<F32>(block_max_key<F32>(q[k][0], q[k][1], f)), kc);
             }
         }
-        for (int g = wb + kRuns; g < we; g++) {
-            const uint8_t* src = w.xrow + w.cr * 1024 + lane * 32;
-            const bool valid = lane < w.nblk(a);
-            const uint4 v0 = ld_stream16_if(src, valid), v1 = ld_stream16_if(src + 16, valid);
-            float f[16];
-            block_values<XF>(a, w, t, lane, valid, v0, v1, f);
-            encode_block<SWZ, SEARCH>(w, lane, valid, f, key_value<F32>(block_max_key<F32>(v0, v1, f)), kc);
-            w.next(a);
+        for (int g = wb + kRuns; g < we; g += kBatch2) {
+            uint4 v[kBatch2][2];
+#pragma unroll
+            for (int u = 0; u < kBatch2; u++) {
+                const Blk kb(a, g + u, lane);
+                const bool ld = g + u < we && kb.valid;
+                const uint8_t* src = kb.src(a, t);
+                v[u][0] = ld_stream16_if(src, ld);
+                v[u][1] = ld_stream16_if(src + 16, ld);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch2; u++) {
+                if (g + u < we) {
+                    const Blk kb(a, g + u, lane);
+                    float f[16];
+                    block_values<XF>(a, kb, t, v[u][0], v[u][1], f);
+                    encode_block<SWZ, SEARCH>(a, t, kb, f, key_value<F32>(block_max_key<F32>(v[u][0], v[u][1], f)), kc);
+                }
+            }
         }
     }
 
     // zero the padding rows of the swizzled scale tiles (cols % 64 == 0, so
     // only the rows past `rows` up to the next multiple of 128 are padding)
     if (SWZ) {
-        const int64_t rows = a.runs_per_tensor / a.upr;
-        const int64_t tiles_c = a.tile_row / 512;
+        const int64_t rows = a.nblk / a.nb;
         const int64_t rows_pad = (rows + 127) / 128 * 128;
-        const int64_t sc_pad = tiles_c * 4;
+        const int64_t sc_pad = a.tiles_c * 4;
         const int64_t npad = (rows_pad - rows) * sc_pad;
         for (int tt = 0; tt < a.ntensors; tt++) {
             uint8_t* sb = a.scales[tt];
             for (int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x; i < npad; i += (int64_t)G * kQThreads) {
                 const int64_t r = rows + i / sc_pad, c = i % sc_pad;
-                sb[swz_offset(r, c, tiles_c)] = 0;
+                sb[swz_offset(r, c, a.tiles_c)] = 0;
             }
         }
     }
@@ -530,21 +529,31 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_fused_kernel(const __gr
 // LayerNorm + adaLN modulate + quantize in one cooperative launch, for inputs
 // whose rows fit in shared memory (one CTA of 512 threads per SM holds
 // ceil(rows / #SMs) rows):
-//   load     thread 0 bulk-copies the CTA's contiguous rows into shared
-//            memory (one cp.async.bulk per row) while the threads stage
-//            fl32(1 + scale[c]) and shift[c] as binary32;
-//   phase 1  a warp per row: the row statistics from shared memory in the
-//            fixed order of the two-launch path (lane j sums the 16-element
-//            blocks j, j+32, ... in order, the 32 partials meet in an xor
-//            butterfly; S2 over fl32(x - mean)^2), so both paths give the same
-//            bits; then the block maxima of the modulated values
+//   load     thread 0 bulk-copies the CTA's rows into shared memory, one copy
+//            per row, kLnGroups groups of rows each on its own mbarrier;
+//   stats    a warp per row, as its group lands: S1 = sum of x, lane j
+//            adding elements 256c + 8j .. 256c + 8j + 7 of c = 0, 1, ... in
+//            order (16 contiguous bytes a lane: conflict-free), the 32 partials
+//            met in an xor butterfly (16, 8, 4, 2, 1); mean = fl32(S1 / cols);
+//            S2 the same over fl32(x - mean)^2; rstd = 1 / sqrt(S2 / cols +
+//            eps) -- the order of the two-launch path's statistics kernel, so
+//            both paths give the same bits;
+//   max      the (512-column chunk, row) tasks in chunk-major order, split
+//            evenly over the warps, lane i holding block i of the chunk (its
+//            modulation columns stay in registers while the warp's chunk
+//            stays the same):
 //            m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift)
-//            and the CTA's maximum;
-//   barrier  the fused quantize's bounded grid barrier turns the CTAs' maxima
-//            into a32 = max |m| / 2688;
-//   phase 2  every block of m is recomputed from shared memory and encoded.
-// HBM: the input is read once and the codes and scales written once.
+//            (binary32 pairs) and the CTA's max |m|;
+//   barrier  the bounded grid barrier: a32 = max |m| / 2688;
+//   encode   the same tasks: m and its block max again, one scale and 8
+//            bytes of codes a lane.
+// A lane reads its 32-byte block as two 16-byte halves, lanes 4..7 of every
+// eight taking the second half first, so each warp-wide read covers all 32
+// banks four times (no conflicts).  HBM: the input is read once and the codes
+// and scales written once.
 // ---------------------------------------------------------------------------
+constexpr int kLnGroups = 8;  // groups of rows, each copied in on its own mbarrier
+
 struct LnArgs {
     const uint8_t* x;
     int64_t ld_bytes;
@@ -570,29 +579,59 @@ __device__ __forceinline__ float ln_butterfly(float s) {
     return s;
 }
 
-// the 16 bf16 of block b of a row staged in shared memory, as binary32
-__device__ __forceinline__ void ln_block(const uint8_t* row, int b, float* f) {
-    const uint4* p = reinterpret_cast<const uint4*>(row + b * 32);
-    bf16x8_to_f32(p[0], f);
-    bf16x8_to_f32(p[1], f + 8);
-}
-
-// the block's modulated values m (in place over x) and their |m| max
-__device__ __forceinline__ float ln_modulate16(float* f, float mean, float rstd, const float* sc1, const float* sh) {
-    float mx = 0.0f;
+// The lane's 16 modulation columns c0 .. c0+15: fl32(1 + scale) and shift
+// (1 and 0 where the vector is absent or the block is past the row).
+__device__ __forceinline__ void ln_columns(const LnArgs& a, int c0, bool valid, float* sc1, float* sh) {
 #pragma unroll
     for (int i = 0; i < 16; i++) {
-        const float h = __fmul_rn(__fsub_rn(f[i], mean), rstd);
-        f[i] = __fadd_rn(__fmul_rn(h, sc1[i]), sh[i]);
-        mx = fmaxf(mx, fabsf(f[i]));
+        sc1[i] = 1.0f;
+        sh[i] = 0.0f;
+    }
+    if (valid && a.mod_scale) {
+        const uint4* p = reinterpret_cast<const uint4*>(a.mod_scale + c0);
+        float v[16];
+        bf16x8_to_f32(__ldg(p), v);
+        bf16x8_to_f32(__ldg(p + 1), v + 8);
+#pragma unroll
+        for (int i = 0; i < 16; i++) sc1[i] = __fadd_rn(1.0f, v[i]);
+    }
+    if (valid && a.mod_shift) {
+        const uint4* p = reinterpret_cast<const uint4*>(a.mod_shift + c0);
+        bf16x8_to_f32(__ldg(p), sh);
+        bf16x8_to_f32(__ldg(p + 1), sh + 8);
+    }
+}
+
+// The lane's 16 bf16 of a row staged in shared memory (32 bytes at `p`) as
+// binary32, the halves read in the order that spreads a warp over all banks.
+__device__ __forceinline__ void ln_load16(const uint8_t* p, int lane, float* f) {
+    const int h = (lane >> 2) & 1;
+    const uint4 first = *reinterpret_cast<const uint4*>(p + 16 * h);
+    const uint4 second = *reinterpret_cast<const uint4*>(p + 16 * (h ^ 1));
+    bf16x8_to_f32(h ? second : first, f);
+    bf16x8_to_f32(h ? first : second, f + 8);
+}
+
+// m of 16 elements (in place over x) and their |m| max, binary32 pairs:
+// fl32(fl32(fl32(fl32(x - mean) * rstd) * sc1) + sh)
+__device__ __forceinline__ float ln_modulate16(float* f, float mean, float rstd, const float* sc1, const float* sh) {
+    const float2 nm = make_float2(-mean, -mean), rs = make_float2(rstd, rstd);
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float2 h = mul2(add2(make_float2(f[2 * i], f[2 * i + 1]), nm), rs);
+        const float2 m = add2(mul2(h, make_float2(sc1[2 * i], sc1[2 * i + 1])), make_float2(sh[2 * i], sh[2 * i + 1]));
+        f[2 * i] = m.x;
+        f[2 * i + 1] = m.y;
+        mx = fmaxf(mx, fmaxf(fabsf(m.x), fabsf(m.y)));
     }
     return mx;
 }
 
 template <bool SEARCH>
 __global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __grid_constant__ LnArgs a) {
-    extern __shared__ __align__(16) uint8_t ln_smem[];
-    __shared__ uint64_t bar;
+    extern __shared__ __align__(128) uint8_t ln_smem[];
+    __shared__ uint64_t bars[kLnGroups];
     __shared__ uint32_t s_red[kQWarps];
     __shared__ float s_inv[256];
     __shared__ float s_a32, s_d6, s_d4;
@@ -601,73 +640,102 @@ __global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
     const int r0 = (int)((int64_t)a.rows * blockIdx.x / G), r1 = (int)((int64_t)a.rows * (blockIdx.x + 1) / G);
-    const int nr = r1 - r0, cols = a.cols, nb = cols / 16;
+    const int nr = r1 - r0, cols = a.cols;
+    const int nch = (cols + 255) / 256;   // 256-element chunks per row (statistics)
+    const int nrun = (cols + 511) / 512;  // 512-element chunks per row (a block per lane)
     const int64_t row_bytes = (int64_t)cols * 2;
-    uint8_t* xs = ln_smem;                                              // [nr][cols] bf16
-    float* sc1 = reinterpret_cast<float*>(ln_smem + (int64_t)nr * row_bytes);  // [cols] fl32(1 + scale)
-    float* sh = sc1 + cols;                                             // [cols] shift
-    float2* st = reinterpret_cast<float2*>(sh + cols);                  // [nr] (mean, rstd)
+    uint8_t* xs = ln_smem;                                                      // [nr][cols] bf16
+    float2* st = reinterpret_cast<float2*>(ln_smem + (int64_t)nr * row_bytes);  // [nr] (mean, rstd)
     const uint32_t epoch = *(volatile uint32_t*)&a.ctl[kCtlEpoch] + 1u;  // same for every CTA of this launch
     const int par = (int)(epoch & 1u);
     if (threadIdx.x == 0) {
         s_ok = 1;
-        mbar_init(&bar, 1);
+        for (int g = 0; g < kLnGroups; g++) mbar_init(&bars[g], 1);
         fence_barrier_init();
-        fence_proxy_async_smem();
-        mbar_expect_tx(&bar, (uint32_t)(nr * row_bytes));
-        for (int r = 0; r < nr; r++) bulk_load(xs + r * row_bytes, a.x + (int64_t)(r0 + r) * a.ld_bytes, (uint32_t)row_bytes, &bar);
-    }
-    for (int c = threadIdx.x; c < cols; c += kQThreads) {
-        sc1[c] = a.mod_scale ? __fadd_rn(1.0f, __bfloat162float(a.mod_scale[c])) : 1.0f;
-        sh[c] = a.mod_shift ? __bfloat162float(a.mod_shift[c]) : 0.0f;
+        int r = 0;
+        for (int g = 0; g < kLnGroups; g++) {
+            const int re = (int)((int64_t)nr * (g + 1) / kLnGroups);
+            for (; r < re; r++) {
+                mbar_expect_tx_only(&bars[g], (uint32_t)row_bytes);
+                bulk_load(xs + r * row_bytes, a.x + (int64_t)(r0 + r) * a.ld_bytes, (uint32_t)row_bytes, &bars[g]);
+            }
+            mbar_arrive(&bars[g]);
+        }
     }
     __syncthreads();
+    // ---- statistics, a warp per row (as its group lands)
+    const float n = (float)cols;
+    bool landed = true;
     {
         volatile int never = 0;
-        const bool got = nr == 0 || mbar_wait_bounded(&bar, 0, &never, a.limit_ns);
-        if (!__syncthreads_and(got)) {
-            if (threadIdx.x == 0) record_error(a.err, NVFP4_ERR_TIMEOUT, 6);
-            return;
-        }
-    }
-    // ---- phase 1: statistics and the block maxima of m, a warp per row
-    const float n = (float)cols;
-    float lmax = 0.0f;
-    for (int r = warp; r < nr; r += kQWarps) {
-        const uint8_t* row = xs + r * row_bytes;
-        float s1 = 0.0f;
-        for (int b = lane; b < nb; b += 32) {
-            float f[16];
-            ln_block(row, b, f);
+        int g = 0;
+        for (int r = warp; r < nr && landed; r += kQWarps) {
+            while ((int64_t)(g + 1) * nr / kLnGroups <= r) g++;  // the group holding row r
+            landed = mbar_wait_bounded(&bars[g], 0, &never, a.limit_ns);
+            if (!landed) break;
+            const uint8_t* row = xs + r * row_bytes;
+            float s1 = 0.0f;
+            for (int c = 0; c < nch; c++) {
+                const int e0 = 256 * c + 8 * lane;
+                if (e0 < cols) {
+                    float f[8];
+                    bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + 2 * e0), f);
 #pragma unroll
-            for (int i = 0; i < 16; i++) s1 = __fadd_rn(s1, f[i]);
-        }
-        const float mean = __fdiv_rn(ln_butterfly(s1), n);
-        float s2 = 0.0f;
-        for (int b = lane; b < nb; b += 32) {
-            float f[16];
-            ln_block(row, b, f);
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const float d = __fsub_rn(f[i], mean);
-                s2 = __fadd_rn(s2, __fmul_rn(d, d));
+                    for (int i = 0; i < 8; i++) s1 = __fadd_rn(s1, f[i]);
+                }
             }
-        }
-        const float var = __fdiv_rn(ln_butterfly(s2), n);
-        const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
-        if (lane == 0) {
-            st[r] = make_float2(mean, rstd);
-            a.stats[r0 + r] = make_float2(mean, rstd);
-        }
-        if (!a.given) {
-            for (int b = lane; b < nb; b += 32) {
-                float f[16];
-                ln_block(row, b, f);
-                lmax = fmaxf(lmax, ln_modulate16(f, mean, rstd, sc1 + b * 16, sh + b * 16));
+            const float mean = __fdiv_rn(ln_butterfly(s1), n);
+            float s2 = 0.0f;
+            for (int c = 0; c < nch; c++) {
+                const int e0 = 256 * c + 8 * lane;
+                if (e0 < cols) {
+                    float f[8];
+                    bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + 2 * e0), f);
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        const float d = __fsub_rn(f[i], mean);
+                        s2 = __fadd_rn(s2, __fmul_rn(d, d));
+                    }
+                }
+            }
+            const float var = __fdiv_rn(ln_butterfly(s2), n);
+            const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
+            if (lane == 0) {
+                st[r] = make_float2(mean, rstd);
+                a.stats[r0 + r] = make_float2(mean, rstd);
             }
         }
     }
+    // every row's group has been waited on by the warp that took the row
+    if (!__syncthreads_and(landed)) {
+        if (threadIdx.x == 0) record_error(a.err, NVFP4_ERR_TIMEOUT, 6);
+        return;
+    }
+    // the warp's tasks: [tb, te) of the (512-column chunk, row) tasks in chunk-major order
+    const int ntask = nrun * nr;
+    const int tb = (int)((int64_t)ntask * warp / kQWarps), te = (int)((int64_t)ntask * (warp + 1) / kQWarps);
     if (!a.given) {
+        // ---- max |m| over the CTA's rows
+        float lmax = 0.0f;
+        int c = tb / max(nr, 1), r = tb - c * nr;  // task tb's chunk and row
+        float sc1[16], sh[16];
+        ln_columns(a, 512 * c + 16 * lane, 512 * c + 16 * lane < cols, sc1, sh);
+        for (int k = 0; tb + k < te; k++) {
+            const int e0 = 512 * c + 16 * lane;
+            float mx = 0.0f;
+            if (e0 < cols) {
+                float f[16];
+                ln_load16(xs + r * row_bytes + 2 * e0, lane, f);
+                const float2 rs = st[r];
+                mx = ln_modulate16(f, rs.x, rs.y, sc1, sh);
+            }
+            lmax = fmaxf(lmax, mx);
+            if (++r == nr && tb + k + 1 < te) {
+                r = 0;
+                ++c;
+                ln_columns(a, 512 * c + 16 * lane, 512 * c + 16 * lane < cols, sc1, sh);
+            }
+        }
         uint32_t m = __float_as_uint(lmax);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -677,25 +745,9 @@ __global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __
             uint32_t c0 = 0u;
 #pragma unroll
             for (int i = 0; i < kQWarps; i++) c0 = max(c0, s_red[i]);
-            uint32_t* cnt = a.ctl + kCtlCount + par;
-            uint32_t* mx = a.ctl + kCtlMax + 2 * par;
-            asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(mx), "r"(c0) : "memory");
-            uint32_t old;
-            asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
-            const uint64_t t_start = global_ns();
-            uint32_t cnt_now = old + 1u;
-            while (cnt_now < (uint32_t)G) {
-                __nanosleep(20);
-                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cnt_now) : "l"(cnt) : "memory");
-                if (cnt_now < (uint32_t)G && global_ns() - t_start > a.limit_ns) {
-                    record_error(a.err, NVFP4_ERR_TIMEOUT, 2);
-                    s_ok = 0;
-                    break;
-                }
-            }
-            uint32_t t0;
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(t0) : "l"(mx) : "memory");
-            s_total = t0;
+            uint32_t tot[2];
+            if (!grid_max_exchange(a.ctl, a.err, a.limit_ns, par, G, c0, 0u, tot)) s_ok = 0;
+            s_total = tot[0];
         }
         __syncthreads();
         if (!s_ok) return;
@@ -704,14 +756,7 @@ __global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __
             s_a32 = a32;
             if (blockIdx.x == 0) *a.gscale = a32;
         }
-        // every CTA has counted itself in: reset the other parity's words, then publish the epoch
-        if (blockIdx.x == 0 && threadIdx.x == 32) {
-            a.ctl[kCtlCount + (par ^ 1)] = 0u;
-            a.ctl[kCtlMax + 2 * (par ^ 1)] = 0u;
-            a.ctl[kCtlMax + 2 * (par ^ 1) + 1] = 0u;
-            __threadfence();
-            *(volatile uint32_t*)&a.ctl[kCtlEpoch] = epoch;
-        }
+        if (blockIdx.x == 0 && threadIdx.x == 32) grid_barrier_retire(a.ctl, par, epoch);
     } else if (threadIdx.x == 0) {
         s_a32 = *a.gscale;
     }
@@ -728,33 +773,44 @@ __global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __
         }
         __syncthreads();
     }
-    // ---- phase 2: encode every block of m
+    // ---- encode every block of m, the same tasks
     const EncodeConsts kc{s_a32, s_d6, s_d4, s_inv};
     const int64_t tiles_c = cols / 64;
-    for (int r = warp; r < nr; r += kQWarps) {
-        const uint8_t* row = xs + r * row_bytes;
-        const float2 rs = st[r];
-        const int64_t gr = r0 + r;
-        uint8_t* crow = a.codes + gr * (cols / 2);
-        for (int b = lane; b < nb; b += 32) {
-            float f[16];
-            ln_block(row, b, f);
-            const float amax_b = ln_modulate16(f, rs.x, rs.y, sc1 + b * 16, sh + b * 16);
-            uint32_t code = kc.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, kc.d6));
-            uint2 cw = encode16(f, kc.inv_tab[code]);
-            if (SEARCH) {
-                const uint32_t code4 = kc.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, kc.d4));
-                const uint2 c4 = encode16(f, kc.inv_tab[code4]);
-                if (block_sq_error(f, c4, e4m3_value(code4), kc.a32) < block_sq_error(f, cw, e4m3_value(code), kc.a32)) {
-                    code = code4;
-                    cw = c4;
+    {
+        int c = tb / max(nr, 1), r = tb - c * nr;
+        float sc1[16], sh[16];
+        ln_columns(a, 512 * c + 16 * lane, 512 * c + 16 * lane < cols, sc1, sh);
+        for (int k = 0; tb + k < te; k++) {
+            const int e0 = 512 * c + 16 * lane;
+            if (e0 < cols) {
+                float f[16];
+                ln_load16(xs + r * row_bytes + 2 * e0, lane, f);
+                const float2 rs = st[r];
+                const float mx = ln_modulate16(f, rs.x, rs.y, sc1, sh);
+                uint32_t code = kc.d6 == 0.0f ? 0u : e4m3_code(__fdiv_rn(mx, kc.d6));
+                uint2 cw = encode16(f, kc.inv_tab[code]);
+                if (SEARCH) {
+                    const uint32_t code4 = kc.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(mx, kc.d4));
+                    const uint2 c4 = encode16(f, kc.inv_tab[code4]);
+                    if (block_sq_error(f, c4, e4m3_value(code4), kc.a32) <
+                        block_sq_error(f, cw, e4m3_value(code), kc.a32)) {
+                        code = code4;
+                        cw = c4;
+                    }
                 }
+                const int64_t gr = r0 + r;
+                const int b = e0 >> 4;
+                *reinterpret_cast<uint2*>(a.codes + gr * (cols / 2) + (e0 >> 1)) = cw;
+                if (a.swizzled)
+                    a.scales[swz_offset(gr, b, tiles_c)] = (uint8_t)code;
+                else
+                    a.scales[gr * (cols / 16) + b] = (uint8_t)code;
             }
-            *reinterpret_cast<uint2*>(crow + b * 8) = cw;
-            if (a.swizzled)
-                a.scales[swz_offset(gr, b, tiles_c)] = (uint8_t)code;
-            else
-                a.scales[gr * nb + b] = (uint8_t)code;
+            if (++r == nr && tb + k + 1 < te) {
+                r = 0;
+                ++c;
+                ln_columns(a, 512 * c + 16 * lane, 512 * c + 16 * lane < cols, sc1, sh);
+            }
         }
     }
     // zero the padding rows of the swizzled scale tiles (rows past `rows` up to the next multiple of 128)
@@ -770,18 +826,37 @@ __global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __
 }
 
 // LayerNorm statistics of each row (one warp per row), in the fixed order of
-// the fused LayerNorm + modulate + quantize: lane j sums the 16-element
-// blocks j, j+32, ... of the row in order, the 32 partial sums meet in an
-// xor butterfly (16, 8, 4, 2, 1); mean = S1 / cols, var = S2 / cols with S2
-// over fl32(x - mean)^2, rstd = 1 / sqrt(var + eps), every step correctly
-// rounded binary32.
+// the one-launch LayerNorm + modulate + quantize: lane j adds elements
+// 256c + 8j .. 256c + 8j + 7 of chunks c = 0, 1, ... in order, the 32 partial
+// sums meet in an xor butterfly (16, 8, 4, 2, 1); mean = S1 / cols,
+// var = S2 / cols with S2 over fl32(x - mean)^2, rstd = 1 / sqrt(var + eps),
+// every step correctly rounded binary32.
 __device__ __forceinline__ float warp_butterfly_sum(float s) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xFFFFFFFFu, s, o));
     return s;
 }
 
-constexpr int kStatRegBlocks = 8;  // 16-element blocks a lane holds in registers (rows up to 4096 columns)
+constexpr int kStatRegChunks = 16;  // 256-element chunks a warp holds in registers (rows up to 4096 columns)
+
+__device__ __forceinline__ float stat_sum(const uint4& v, float s) {
+    float f[8];
+    bf16x8_to_f32(v, f);
+#pragma unroll
+    for (int i = 0; i < 8; i++) s = __fadd_rn(s, f[i]);
+    return s;
+}
+
+__device__ __forceinline__ float stat_sq_sum(const uint4& v, float mean, float s2) {
+    float f[8];
+    bf16x8_to_f32(v, f);
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float d = __fsub_rn(f[i], mean);
+        s2 = __fadd_rn(s2, __fmul_rn(d, d));
+    }
+    return s2;
+}
 
 __global__ void __launch_bounds__(256) ln_stats_kernel(const uint8_t* x, int64_t ld_bytes, int rows, int cols,
                                                        float eps, float2* out) {
@@ -789,59 +864,33 @@ __global__ void __launch_bounds__(256) ln_stats_kernel(const uint8_t* x, int64_t
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (row >= rows) return;
     const uint8_t* xr = x + (int64_t)row * ld_bytes;
-    const int nb = cols / 16;
+    const int nch = (cols + 255) / 256;
     const float n = (float)cols;
     float s = 0.0f, s2 = 0.0f, mean;
-    if (nb <= 32 * kStatRegBlocks) {
-        // the lane's blocks (lane, lane + 32, ...) loaded at once and kept for both sums
-        uint4 v[kStatRegBlocks][2];
+    if (nch <= kStatRegChunks) {
+        // the lane's 16 bytes of every chunk loaded at once and kept for both sums
+        uint4 v[kStatRegChunks];
 #pragma unroll
-        for (int k = 0; k < kStatRegBlocks; k++) {
-            const int b = lane + 32 * k;
-            const bool ok = b < nb;
-            v[k][0] = ok ? __ldg(reinterpret_cast<const uint4*>(xr + b * 32)) : make_uint4(0u, 0u, 0u, 0u);
-            v[k][1] = ok ? __ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)) : make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < kStatRegChunks; c++) {
+            const int e0 = 256 * c + 8 * lane;
+            v[c] = (c < nch && e0 < cols) ? __ldg(reinterpret_cast<const uint4*>(xr + 2 * e0)) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int k = 0; k < kStatRegBlocks; k++) {
-            if (lane + 32 * k >= nb) break;
-            float f[16];
-            bf16x8_to_f32(v[k][0], f);
-            bf16x8_to_f32(v[k][1], f + 8);
-#pragma unroll
-            for (int i = 0; i < 16; i++) s = __fadd_rn(s, f[i]);
-        }
+        for (int c = 0; c < kStatRegChunks; c++)
+            if (c < nch && 256 * c + 8 * lane < cols) s = stat_sum(v[c], s);
         mean = __fdiv_rn(warp_butterfly_sum(s), n);
 #pragma unroll
-        for (int k = 0; k < kStatRegBlocks; k++) {
-            if (lane + 32 * k >= nb) break;
-            float f[16];
-            bf16x8_to_f32(v[k][0], f);
-            bf16x8_to_f32(v[k][1], f + 8);
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const float d = __fsub_rn(f[i], mean);
-                s2 = __fadd_rn(s2, __fmul_rn(d, d));
-            }
-        }
+        for (int c = 0; c < kStatRegChunks; c++)
+            if (c < nch && 256 * c + 8 * lane < cols) s2 = stat_sq_sum(v[c], mean, s2);
     } else {
-        for (int b = lane; b < nb; b += 32) {
-            float f[16];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
-#pragma unroll
-            for (int i = 0; i < 16; i++) s = __fadd_rn(s, f[i]);
+        for (int c = 0; c < nch; c++) {
+            const int e0 = 256 * c + 8 * lane;
+            if (e0 < cols) s = stat_sum(__ldg(reinterpret_cast<const uint4*>(xr + 2 * e0)), s);
         }
         mean = __fdiv_rn(warp_butterfly_sum(s), n);
-        for (int b = lane; b < nb; b += 32) {
-            float f[16];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32)), f);
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + b * 32 + 16)), f + 8);
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const float d = __fsub_rn(f[i], mean);
-                s2 = __fadd_rn(s2, __fmul_rn(d, d));
-            }
+        for (int c = 0; c < nch; c++) {
+            const int e0 = 256 * c + 8 * lane;
+            if (e0 < cols) s2 = stat_sq_sum(__ldg(reinterpret_cast<const uint4*>(xr + 2 * e0)), mean, s2);
         }
     }
     const float var = __fdiv_rn(warp_butterfly_sum(s2), n);
@@ -1133,9 +1182,9 @@ static PerDevice<DequantResidency> g_dequant_resident;
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// dynamic shared memory of the one-launch LayerNorm quantize (rows, vectors,
+// dynamic shared memory of the one-launch LayerNorm quantize (rows and their
 // statistics); larger inputs take the two-launch path
-constexpr int64_t kLnSmemMax = 200 * 1024;
+constexpr int64_t kLnSmemMax = 224 * 1024;
 static PerDevice<bool> g_ln_attr;
 
 static int grid_for(int64_t work_items, int per_cta, int cap) {
@@ -1147,6 +1196,16 @@ static int grid_for(int64_t work_items, int per_cta, int cap) {
 
 static nvfp4_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// Magic number for b / d with b < 2^31 (division by an invariant integer,
+// Granlund and Montgomery): l = ceil(log2 d), m = floor(2^(31 + l) / d) + 1
+// (fits in 32 bits), b / d = umulhi(b, m) >> (l - 1).  d >= 2.
+static void div_magic(uint32_t d, uint32_t* m, int* shift) {
+    int l = 0;
+    while ((1ull << l) < d) l++;
+    *m = (uint32_t)(((uint64_t)1 << (31 + l)) / d + 1);
+    *shift = l - 1;
 }
 
 // one fused, cooperative launch over one or two tensors of the same shape
@@ -1164,18 +1223,14 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
         a.scales[t] = static_cast<uint8_t*>(scales[t]);
         a.gscale[t] = gscale[t];
     }
-    const int64_t upr = (cols + 511) / 512;
-    if (rows * upr > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
-    // the kernel's byte offsets inside a row are 32-bit: at most 2^30 elements
-    // per row (a KV chunk is one row of T*H*d elements)
-    if (cols > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
+    // the kernel indexes a tensor's 16-element blocks in 32 bits
+    if (cols > ((int64_t)1 << 30) || rows * (cols / 16) >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED;
     a.ld_bytes = ld * 2;
-    a.code_ld = cols / 2;
-    a.scale_ld = cols / 16;
-    a.tile_row = cols / 64 * 512;
-    a.upr = (int)upr;
-    a.last_nblk = (int)((cols - (upr - 1) * 512) / 16);
-    a.runs_per_tensor = (int)(rows * upr);
+    a.tiles_c = cols / 64;
+    a.nblk = (uint32_t)(rows * (cols / 16));
+    a.nb = (uint32_t)(cols / 16);
+    div_magic(a.nb, &a.nb_magic, &a.nb_shift);
+    a.runs_per_tensor = (int)((a.nblk + 31u) / 32u);
     a.ntensors = ntensors;
     a.given = given ? 1 : 0;
     a.ctl = static_cast<uint32_t*>(workspace);
@@ -1184,7 +1239,6 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
     a.ln_stats = ln_stats;
     a.mod_scale = static_cast<const __nv_bfloat16*>(mod_scale);
     a.mod_shift = static_cast<const __nv_bfloat16*>(mod_shift);
-    a.cols = (int)cols;
     if (smooth_mean) {
         a.smooth_mean[0] = smooth_mean[0];
         a.smooth_mean[1] = ntensors > 1 ? smooth_mean[1] : nullptr;
@@ -1196,7 +1250,8 @@ static nvfp4_status quantize_impl(int ntensors, const void* const* x, int64_t ro
         a.rope_d = rope_d;
         a.rope_hd = smooth_hd;
     }
-    const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), ((int64_t)a.runs_per_tensor * ntensors + kQWarps - 1) / kQWarps);
+    const int64_t total_runs = (int64_t)a.runs_per_tensor * ntensors;
+    const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), (total_runs + kQWarps - 1) / kQWarps);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kQThreads);
@@ -1235,7 +1290,9 @@ nvfp4_status quantize_check_args(const void* x_bf16, int64_t rows, int64_t cols,
     if (flags & ~(NVFP4_Q_GIVEN_GLOBAL | NVFP4_Q_ROWMAJOR_SCALES | NVFP4_Q_SCALE_SEARCH)) return NVFP4_ERR_INVALID_ARG;
     if (rows < 0 || cols <= 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
     if (cols % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
-    if (rows > ((int64_t)1 << 31) || cols > ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED;
+    // the kernel indexes a tensor's 16-element blocks in 32 bits
+    if (cols > ((int64_t)1 << 30) || rows >= ((int64_t)1 << 31) || rows * (cols / 16) >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED;
     if (!global_scale) return NVFP4_ERR_INVALID_ARG;
     if (rows == 0) return NVFP4_OK;
     if (!x_bf16 || !codes || !scales) return NVFP4_ERR_INVALID_ARG;
@@ -1255,8 +1312,6 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t
     if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE, rows, 0, cols)) return NVFP4_ERR_INVALID_ARG;
     if (rows == 0) return NVFP4_OK;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return NVFP4_ERR_MISALIGNED;
-    // the row and run counts the kernel indexes in 32 bits (also refused inside quantize_impl)
-    if (rows * ((cols + 511) / 512) > ((int64_t)1 << 30) || cols > ((int64_t)1 << 30)) return NVFP4_ERR_UNSUPPORTED;
     const void* xs[1] = {x_bf16};
     void* cs[1] = {codes};
     void* ss[1] = {scales};
@@ -1273,7 +1328,8 @@ extern "C" nvfp4_status nvfp4_ln_modulate_quantize(const void* x_bf16, int64_t r
     if (flags & ~(NVFP4_Q_GIVEN_GLOBAL | NVFP4_Q_ROWMAJOR_SCALES | NVFP4_Q_SCALE_SEARCH)) return NVFP4_ERR_INVALID_ARG;
     if (rows < 0 || cols <= 0 || ld < cols || !(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
     if (cols % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
-    if (rows > ((int64_t)1 << 30) || cols > ((int64_t)1 << 24)) return NVFP4_ERR_UNSUPPORTED;
+    if (rows > ((int64_t)1 << 30) || cols > ((int64_t)1 << 24) || rows * (cols / 16) >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED;
     if (!global_scale || !workspace) return NVFP4_ERR_INVALID_ARG;
     if (ws_bytes < nvfp4_workspace_bytes(NVFP4_OP_LN_QUANTIZE, rows, 0, cols)) return NVFP4_ERR_INVALID_ARG;
     if (rows == 0) return NVFP4_OK;
@@ -1287,7 +1343,7 @@ extern "C" nvfp4_status nvfp4_ln_modulate_quantize(const void* x_bf16, int64_t r
     // one launch when each CTA's rows fit in shared memory with the staged vectors
     const int G = (int)std::min<int64_t>(std::min(num_sms(), kMaxGrid), rows);
     const int64_t rows_per_cta = (rows + G - 1) / G;
-    const int64_t smem = rows_per_cta * cols * 2 + cols * 8 + rows_per_cta * 8;
+    const int64_t smem = rows_per_cta * cols * 2 + rows_per_cta * 8;
     if (smem <= kLnSmemMax) {
         LnArgs la{};
         la.x = static_cast<const uint8_t*>(x_bf16);

@@ -129,8 +129,8 @@ nvfp4_status nvfp4_read_device_error(void* workspace, nvfp4_stream_t stream, int
 #define NVFP4_Q_SCALE_SEARCH 4u
 
 /* x_bf16: bf16 [rows x cols], row stride ld elements (ld >= cols, ld % 8 == 0).
- * cols % 64 == 0, rows >= 0; cols <= 2^30 and rows * ceil(cols / 512) <= 2^30,
- * else NVFP4_ERR_UNSUPPORTED.
+ * cols % 64 == 0, rows >= 0; cols <= 2^30 and rows * cols / 16 < 2^31 (the
+ * tensor's 16-element blocks), else NVFP4_ERR_UNSUPPORTED.
  * codes: nvfp4_codes_bytes(rows, cols) bytes, rows of cols/2 bytes.
  * scales: nvfp4_scales_bytes(rows, cols, swizzled) bytes (padding zeroed).
  * global_scale: device binary32, written (COMPUTE) or read (GIVEN).
@@ -153,14 +153,15 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  *   mean = S1 / cols, var = S2 / cols, rstd = 1 / sqrt(var + eps),
  *   m = fl32(fl32(fl32(fl32(x - mean) * rstd) * fl32(1 + scale)) + shift),
  * where S1 = sum x and S2 = sum fl32(x - mean)^2 are summed as 32 partial
- * sums (partial j over the 16-element blocks j, j+32, ... in order) combined
- * by an xor butterfly over 16, 8, 4, 2, 1.  m is then quantized exactly as
+ * sums (partial j over elements 256c + 8j .. 256c + 8j + 7 of c = 0, 1, ...
+ * in order) combined by an xor butterfly over 16, 8, 4, 2, 1.  m is then quantized exactly as
  * nvfp4_quantize quantizes a tensor (flags as there), a32 from max |m|.
- * cols % 64 == 0, cols <= 2^24, rows <= 2^30; pointers 16-byte aligned.
+ * cols % 64 == 0, cols <= 2^24, rows <= 2^30, rows * cols / 16 < 2^31;
+ * pointers 16-byte aligned.
  * workspace: nvfp4_workspace_bytes(NVFP4_OP_LN_QUANTIZE, rows, 0, cols)
  * bytes (the control block, then the binary32 (mean, rstd) of every row,
  * which the call leaves there).  One cooperative launch when ceil(rows /
- * #SMs) rows fit in a CTA's shared memory (about 200 KB: 4096 x 3072 does,
+ * #SMs) rows fit in a CTA's shared memory (224 KB: 4096 x 3072 does,
  * 8192 x 3072 does not): the rows are bulk-copied in once, the statistics,
  * the tensor maximum and the encode all read them there.  Otherwise two
  * launches: the row statistics, then the fused quantize.  Both give the same

@@ -55,7 +55,7 @@ def strided_sum_depth(n: int, group: int = 1) -> int:
     """Most rounded additions any term passes through when n terms (taken in
     groups of `group` consecutive terms) are summed as 32 strided partial sums
     in order, then met in 5 pairwise levels: the order the kernels' headers
-    state for the LayerNorm row sums (group 16) and the channel means (group 1)."""
+    state for the LayerNorm row sums (group 8) and the channel means (group 1)."""
     groups = -(-n // group)
     return group * -(-groups // 32) + 5
 
@@ -84,7 +84,7 @@ def check_ln_stats(stats_dev, x_bits: np.ndarray, eps: float):
     ref = oracle.ln_stats(x_bits, eps=eps)
     x = syn.bf16_bits_to_f32(x_bits).astype(np.float64)
     rows, cols = x.shape
-    depth = strided_sum_depth(cols, 16)
+    depth = strided_sum_depth(cols, 8)
     assert_sum_within_bound(st[:, 0], ref[:, 0], np.abs(x).sum(1), depth, cols, "LayerNorm mean")
     # rstd: the variance's sum has relative error <= (depth + 2) u (a subtraction and a square per
     # term), plus delta^2 / var from the kernel's mean being off by delta; the root, the eps add and

@@ -121,6 +121,10 @@ def test_host_side_argument_checks(L):
     # rows longer than 2^30 elements (a KV chunk is one row of T*H*d) are refused before any launch
     st = L.nvfp4_quantize(fake, 1, (1 << 30) + 64, (1 << 30) + 64, fake, fake, fake, 0, fake, 1 << 16, None)
     assert st == nv.ERR_UNSUPPORTED
+    # so are tensors of 2^31 or more 16-element blocks (the kernel's block index is 32 bits)
+    st = L.nvfp4_quantize(fake, 1 << 21, 1 << 14, 1 << 14, fake, fake, fake, 0, fake, 1 << 16, None)
+    assert st == nv.ERR_UNSUPPORTED
+    assert L.nvfp4_quantize_noalloc(fake, 1 << 21, 1 << 14, 1 << 14, fake, fake, fake, 0, None) == nv.ERR_UNSUPPORTED
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 1, (1 << 23) + 1, 1, 128)  # (2^23 + 1) * 128 > 2^30
     assert L.nvfp4_kv_append(ctypes.byref(kv), 0, fake, fake, fake, 1 << 30, None) == nv.ERR_UNSUPPORTED
     # attention: the key tiles of the whole list are counted in 32 bits

@@ -65,6 +65,20 @@ def test_full_chunk_with_the_3d_table(smooth_k, smooth_v, search):
     assert np.array_equal(host_bits(ko)[0], kref) and np.array_equal(host_bits(vo)[0], vref)
 
 
+def test_two_chunk_append_takes_the_register_kernel():
+    """A 5280-token chunk (6 frames x 22 x 40; K + V = 32 M elements, past what the staged
+    kernel holds in shared memory): the fused kernel with RoPE and both smoothings."""
+    require_gpu()
+    T, H, d = 2 * syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+    f, hh, ww = syn.KV_GRID
+    cs, sn = syn.rope_table_3d(2 * f, hh, ww, d, frame0=3)
+    cache = nv.KVCache(1, T, H, d, smooth_k=True, smooth_v=True)
+    k, v = syn.kv_chunk_bf16(T, H, d, seed=501)
+    cache.append(0, dev_bf16(k), dev_bf16(v), rope=_dev_table(cs, sn))
+    torch.cuda.synchronize()
+    _check(cache, 0, k, v, cs, sn, smooth_k=True, smooth_v=True)
+
+
 @pytest.mark.parametrize("T,H,d", [(4, 3, 16), (12, 3, 16), (33, 2, 64), (64, 5, 32), (7, 1, 128)])
 @pytest.mark.parametrize("smooth_k", [False, True])
 def test_ragged_shapes_with_random_angles(T, H, d, smooth_k):

@@ -57,6 +57,14 @@ def test_ragged_shapes_and_strides(rows, cols, ld):
     _check(syn.activations_bf16(rows, cols, seed=rows + cols), ld=ld)
 
 
+@pytest.mark.parametrize("search,rowmajor", [(False, True), (True, False)])
+def test_inputs_beyond_shared_memory_take_the_register_kernel(search, rowmajor):
+    """8192 x 3072 (25 M elements) is past what the staged kernel holds in shared memory
+    (~17 M per launch): the fused kernel, which holds part of the runs in registers and
+    reads the rest again for the encode."""
+    _check(syn.activations_bf16(8192, 3072, seed=9), search=search, rowmajor=rowmajor)
+
+
 def test_all_zero_tensor():
     q = _check(np.zeros((64, 128), np.uint16))
     assert float(q.global_scale.item()) == 0.0
