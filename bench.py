@@ -402,9 +402,12 @@ def build_stack(nv, dev, layers: int, rank: int):
 
 def time_stack(st, x, steps: int, warmup: int, direct: bool):
     """Warm-up steps, then `steps` timed forwards of the stack (input quantize +
-    every GEMM), captured as one CUDA graph each unless `direct`, with an event
-    before every launch (event-record nodes inside the graph).  Returns the
-    total ms and the per-launch-class mean ms."""
+    every GEMM), captured as one CUDA graph each unless `direct`.  The timed
+    graph holds the launches only; a second graph of the same `steps`
+    forwards, with an event before every launch (event-record nodes), gives
+    the per-launch-class times (replayed apart from the timed region: each
+    event pair costs a few microseconds of its own).  Returns the timed and
+    the component runners, the component events and the graphs."""
     n = st.launches_per_forward()
     L = len(st.layers)
     evs = [[torch.cuda.Event(enable_timing=True, external=not direct) for _ in range(n + 1)] for _ in range(steps)]
@@ -425,22 +428,26 @@ def time_stack(st, x, steps: int, warmup: int, direct: bool):
 
     if direct:
         run_warm = lambda: [fwd() for _ in range(warmup)]
-        run_timed = lambda: [fwd(evs[i]) for i in range(steps)]
+        run_timed = lambda: [fwd() for _ in range(steps)]
+        run_comp = lambda: [fwd(evs[i]) for i in range(steps)]
         graphs = []
     else:
-        gw, gt = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        gw, gt, gc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(gw):
             for _ in range(warmup):
                 fwd()
         with torch.cuda.graph(gt):
             for i in range(steps):
+                fwd()
+        with torch.cuda.graph(gc):
+            for i in range(steps):
                 fwd(evs[i])
-        run_warm, run_timed = gw.replay, gt.replay
-        graphs = [gw, gt]
+        run_warm, run_timed, run_comp = gw.replay, gt.replay, gc.replay
+        graphs = [gw, gt, gc]
     torch.cuda.synchronize()
     run_warm()
     torch.cuda.synchronize()
-    return run_timed, evs, graphs
+    return run_timed, run_comp, evs, graphs
 
 
 def stack_components(evs, L: int) -> dict:
@@ -587,7 +594,7 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     code, _ = nv.read_device_error(st.ws_g)
     if code != nv.OK:
         raise RuntimeError(f"device error {code} during calibration")
-    run_timed, evs, graphs = time_stack(st, x, args.steps, args.warmup, args.direct)
+    run_timed, run_comp, evs, graphs = time_stack(st, x, args.steps, args.warmup, args.direct)
 
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
@@ -605,6 +612,8 @@ def run_ours(args, rank: int, world: int) -> dict | None:
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
+    run_comp()  # the per-launch times, apart from the timed region
+    torch.cuda.synchronize()
     del graphs
     code, _ = nv.read_device_error(st.ws_g)
     if code != nv.OK:
@@ -736,7 +745,12 @@ def sub_report(sub, lin, pk, fp4_peak) -> dict:
             "quantize_back_to_back": _rl("hbm", gbs(quant_bytes, sub["stream"]["quantize_ms"]), pk["hbm_gbs"],
                                          "GB/s", ms=round(sub["stream"]["quantize_ms"], 4),
                                          timing="32 launches back to back over 8 rotating 25 MB inputs (201 MB > "
-                                                "L2), one pair of events")},
+                                                "L2), one pair of events"),
+            "quantize_given_scale_back_to_back": _rl(
+                "hbm", gbs(quant_bytes, sub["stream"]["quantize_given_scale_ms"]), pk["hbm_gbs"], "GB/s",
+                ms=round(sub["stream"]["quantize_given_scale_ms"], 4),
+                timing="as quantize_back_to_back, the tensor scale given (NVFP4_Q_GIVEN_GLOBAL, delayed scaling: "
+                       "no grid-wide maximum, so the encode overlaps the loads)")},
         "kv": {
             "what": "NVFP4 KV cache of 21 slots x 2640 x 24 x 128: append of one K/V chunk (in place into ring "
                     "slot step mod 21), dequant-gather of all 21 slots to bf16",
@@ -867,7 +881,11 @@ def measure_codec_stream(nv, dev, rounds: int) -> dict:
     k0, v0 = (dev_bf16(x) for x in syn.kv_chunk_bf16(T, H, D, seed=50))
     chunks = [(k0.clone(), v0.clone()) for _ in range(nb)]
     cache = nv.KVCache(nb, T, H, D, dev)
+    given = torch.empty(1, dtype=torch.float32, device=dev)
+    nv.quantize(acts[0], out=outs[0], ws=ws_q)
+    given.copy_(outs[0].global_scale)
     calls = {"quantize_ms": lambda i: nv.quantize(acts[i], out=outs[i], ws=ws_q),
+             "quantize_given_scale_ms": lambda i: nv.quantize(acts[i], global_scale=given, out=outs[i], ws=ws_q),
              "kv_append_ms": lambda i: cache.append(i, *chunks[i]),
              "ln_quantize_ms": lambda i: nv.ln_modulate_quantize(acts[i], mod_scale=sc, mod_shift=sh, out=outs[i],
                                                                  ws=ws_ln)}
@@ -1045,6 +1063,7 @@ def main(argv=None) -> int:
         stream_res = measure_codec_stream(nv, dev, rounds=max(2, args.steps))
         pk = peaks()
         b = {"quantize_ms": syn.QKV.M * syn.QKV.K * 2.5625, "ln_quantize_ms": syn.QKV.M * syn.QKV.K * 2.5625,
+             "quantize_given_scale_ms": syn.QKV.M * syn.QKV.K * 2.5625,
              "kv_append_ms": 2 * syn.KV_TOKENS * syn.KV_HEADS * syn.KV_DIM * 2.5625,
              "kv_dequant_ms": 2 * syn.KV_SLOTS * syn.KV_TOKENS * syn.KV_HEADS * syn.KV_DIM * 2.5625}
         line = lambda r: {k: {"ms": round(v, 4), "GB/s": round(b[k] / (v * 1e-3) / 1e9, 1),
