@@ -971,6 +971,7 @@ def cpu_baseline(rows: int = 4) -> dict:
     td = _timed(lambda: [oracle.kv_dequant(*res["k"], T, H, Dh) for _ in range(syn.KV_SLOTS)] +
                 [oracle.kv_dequant(*res["v"], T, H, Dh) for _ in range(syn.KV_SLOTS)])
     kv_elems = T * H * Dh
+    gemms = oracle_gemm_configs(rows=8)
     return {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(), "kind": "oracle",
             "host_cores": os.cpu_count(),
             "sample": f"{rows} of {syn.STACK_M} token rows through one layer of the stack (input quantize, 4 fp64 "
@@ -980,7 +981,41 @@ def cpu_baseline(rows: int = 4) -> dict:
                 "quantize_4096x3072_GB/s": round(M * K * 2.5625 / tq / 1e9, 4),
                 "kv_append_GB/s": round(2 * kv_elems * 2.5625 / ta / 1e9, 4),
                 "kv_dequant_21_slots_GB/s": round(2 * syn.KV_SLOTS * kv_elems * 2.5625 / td / 1e9, 4),
-                "seconds": round(tq + ta + td, 2)}}
+                "seconds": round(tq + ta + td, 2)},
+            "gemm_configs": gemms}
+
+
+def oracle_gemm_configs(rows: int) -> dict:
+    """The oracle's fp64 GEMM (with its epilogue) per configuration: the tiny
+    64 x 128 x 256 case in full, the QKV projection and the FFN pair on `rows`
+    token rows (the weights quantized in full by the oracle first), with the
+    full-size time extrapolated from the rows' rate."""
+    import oracle
+
+    out = {}
+    a = syn.tiny_a_bf16(64, 256, seed=0)
+    w = syn.normal_bf16((128, 256), seed=1)
+    qa, qw = oracle.quantize(a), oracle.quantize(w)
+    t = _timed(lambda: oracle.gemm(qa, qw, want_bf16=True))
+    out["tiny_64x128x256_full"] = {"TFLOP/s": round(2.0 * 64 * 128 * 256 / t / 1e12, 6), "seconds": round(t, 4)}
+    shapes = {"qkv_4096x9216x3072": (syn.QKV, 0), "ffn_up_8192x14336x3072": (syn.FFN_UP, nv_act_gelu()),
+              "ffn_down_8192x3072x14336": (syn.FFN_DOWN, 0)}
+    for name, (sh, act) in shapes.items():
+        x = syn.activations_bf16(rows, sh.K, seed=2)
+        wq = oracle.quantize(syn.normal_bf16_blocks((sh.N, sh.K), seed=3, std=0.02))
+        bias = syn.normal_bf16((sh.N,), seed=4, std=0.02)
+        xq = oracle.quantize(x)
+        t = _timed(lambda: oracle.gemm(xq, wq, bias=bias, act=act, want_bf16=True))
+        rate = 2.0 * rows * sh.N * sh.K / t
+        out[name] = {"rows": rows, "TFLOP/s": round(rate / 1e12, 6),
+                     "extrapolated_full_s": round(2.0 * sh.M * sh.N * sh.K / rate, 1)}
+    return out
+
+
+def nv_act_gelu() -> int:
+    from bit_video_dit_b200 import nvfp4 as nv
+
+    return nv.ACT_GELU_TANH
 
 
 def run_reference(args) -> dict:

@@ -724,6 +724,10 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
                 const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ Params p) {
     using C = Cfg<PAIR>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // the next kernel on the stream (if launched with programmatic stream
+    // serialization) may be scheduled now; it waits for this grid to complete
+    // before it touches global memory
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_stage = ring + C::STAGES * C::STAGE_BYTES;  // 1024-aligned (STAGE_BYTES % 1024 == 0)
     float* vecs = reinterpret_cast<float*>(epi_stage + EPI_STAGE_BYTES);
@@ -765,6 +769,13 @@ __global__ void __launch_bounds__(threads_for(NC), 1)
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s->tmem_base;
+    // Launched with programmatic stream serialization, this grid may start
+    // while the previous kernel on the stream is still finishing (its CTAs
+    // free SMs one by one): everything above touches only this CTA's shared
+    // memory and TMEM; wait for that kernel to complete, with its memory
+    // visible, before any global access (its outputs are read here, and it may
+    // still read what this kernel writes).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 0) {
         if (lane == 0) producer<PAIR>(p, s, ring, &tma_a, &tma_b, &tma_sfa, &tma_sfb, rank);
@@ -1005,13 +1016,17 @@ extern "C" nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B,
         cfg.blockDim = dim3(gemm::threads_for(nc));
         cfg.dynamicSmemBytes = gemm::Cfg<true>::SMEM_BYTES;
         cfg.stream = (cudaStream_t)stream;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        // programmatic dependent launch: the grid's prologue (barriers, TMEM,
+        // cluster sync) overlaps the previous kernel's last tiles
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         if (cudaLaunchKernelEx(&cfg, nc == 2 ? gemm::gemm_kernel<true, 2> : gemm::gemm_kernel<true, 3>, ma, mb, msa, msb,
                                mc, p) != cudaSuccess) {
             cudaGetLastError();
