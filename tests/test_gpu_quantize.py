@@ -65,6 +65,27 @@ def test_inputs_beyond_shared_memory_take_the_register_kernel(search, rowmajor):
     _check(syn.activations_bf16(8192, 3072, seed=9), search=search, rowmajor=rowmajor)
 
 
+def test_back_to_back_launches_on_one_workspace():
+    """Twenty quantizes of different inputs queued on one stream with one workspace, no synchronisation between
+    them: the grid barrier's words alternate by launch parity and each launch resets the other parity's, so every
+    tensor scale and code comes out as the oracle's (a barrier word left over from a previous launch would merge
+    two launches' maxima)."""
+    require_gpu()
+    xs = [syn.activations_bf16(256 + 64 * (i % 3), 512, seed=300 + i) for i in range(20)]
+    # the third input is all zero: its tensor scale must not inherit a neighbour's maximum
+    xs[2] = np.zeros_like(xs[2])
+    ws = nv.workspace(nv.OP_QUANTIZE, 384, 0, 512)
+    xd = [dev_bf16(x) for x in xs]
+    torch.cuda.synchronize()
+    outs = [nv.quantize(d, ws=ws) for d in xd]
+    torch.cuda.synchronize()
+    for x, q in zip(xs, outs):
+        codes, scales, a32 = oracle.quantize(x)
+        assert f32_bits(q.global_scale.cpu().numpy()) == f32_bits(a32)
+        assert np.array_equal(host_u8(q.codes), codes)
+        assert np.array_equal(host_u8(q.scales), oracle.swizzle(scales))
+
+
 def test_all_zero_tensor():
     q = _check(np.zeros((64, 128), np.uint16))
     assert float(q.global_scale.item()) == 0.0
