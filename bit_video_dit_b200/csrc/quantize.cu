@@ -21,6 +21,10 @@
 //    by a per-token cos / sin table) and the K-smoothing mean subtraction, whose
 //    channel means come from a separate fixed-order kernel (of the turned keys
 //    when both apply).
+//  * LayerNorm + modulate + quantize in one cooperative launch when each CTA's
+//    rows fit in shared memory (ln_quantize_smem_kernel: the rows copied in
+//    once, statistics, tensor maximum and encode all read them there); larger
+//    inputs take the statistics kernel and the fused kernel's LN variant.
 #include <algorithm>
 
 #include "common.cuh"
