@@ -290,20 +290,18 @@ __device__ __forceinline__ float tile_max(uint32_t t_s, int valid) {
 // P row: 2^(c_s * s - m) for the tile's first `valid` keys (zero past them),
 // times w_s (RAW: a32_V / a32_ref) rounded to binary16, else bf16, written to
 // P at row `row`; returns the row's sum of the unrounded, unweighted values.
-// The next 32 columns load from TMEM while the current ones are processed.
+// 32 columns a TMEM load (the chunk loop is kept rolled: fewer live registers).
 template <bool RAW>
 __device__ __forceinline__ float write_p(uint32_t t_s, uint32_t p_s, int row, int valid, float c_s, float m,
                                          float w_s) {
     float2 sum[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
     const float2 cc = make_float2(c_s, c_s), mm = make_float2(-m, -m), ww = make_float2(w_s, w_s);
-    uint32_t r[2][32];
-    tmem_ld_32cols(t_s, r[0]);
-    tmem_ld_wait();
-    tmem_regs_ready(r[0]);
-#pragma unroll
+#pragma unroll 1
     for (int c = 0; c < 4; c++) {
-        if (c < 3) tmem_ld_32cols(t_s + 32 * (c + 1), r[(c + 1) & 1]);
-        const uint32_t* rc = r[c & 1];
+        uint32_t rc[32];
+        tmem_ld_32cols(t_s + 32 * c, rc);
+        tmem_ld_wait();
+        tmem_regs_ready(rc);
 #pragma unroll
         for (int q4 = 0; q4 < 4; q4++) {
             uint32_t w[4];
@@ -327,10 +325,6 @@ __device__ __forceinline__ float write_p(uint32_t t_s, uint32_t p_s, int row, in
                 }
             }
             st_shared16(p_s + (4 * c + q4) * 2048 + row * 16, make_uint4(w[0], w[1], w[2], w[3]));
-        }
-        if (c < 3) {
-            tmem_ld_wait();
-            tmem_regs_ready(r[(c + 1) & 1]);
         }
     }
     return (sum[0].x + sum[1].x) + (sum[0].y + sum[1].y);
