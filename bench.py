@@ -1062,6 +1062,9 @@ def main(argv=None) -> int:
                          "workloads and print their numbers (also the small case for profiling them)")
     ap.add_argument("--layers", type=int, default=syn.STACK_LAYERS,
                     help="layers of the stack (default 30, the workload; fewer only for profiling)")
+    ap.add_argument("--attention-only", action="store_true",
+                    help="time only the attention over the KV workload's 21-slot cache (about 1 GB on the device: "
+                         "the case for profiling the attention kernel) and print its numbers")
     ap.add_argument("--stack-only", action="store_true",
                     help="time the stack alone (skip the single-layer, KV and next-row measurements)")
     args = ap.parse_args(argv)
@@ -1088,6 +1091,23 @@ def main(argv=None) -> int:
         ffn = measure_ffn(nv, lambda: flush_buf.fill_(1), flush_buf.device, reps=max(1, args.steps))
         if rank == 0:
             print(json.dumps({"ffn_8192": {k: round(v, 4) for k, v in ffn.items()}}), flush=True)
+        return 0
+    if args.attention_only:
+        from bit_video_dit_b200 import build as nvbuild
+        from bit_video_dit_b200 import nvfp4 as nv
+        nvbuild.build()
+        dev = torch.device("cuda", local)
+        S, T, H, D = syn.KV_SLOTS, syn.KV_TOKENS, syn.KV_HEADS, syn.KV_DIM
+        cache = nv.KVCache(S, T, H, D, dev)
+        chunks = [tuple(dev_bf16(x) for x in syn.kv_chunk_bf16(T, H, D, seed=50 + i)) for i in range(4)]
+        for s_ in range(S):
+            cache.append(s_, *chunks[s_ % 4])
+        ring = torch.arange(S, dtype=torch.int32, device=dev)
+        k_out = torch.empty((S, T, H, D), dtype=torch.bfloat16, device=dev)
+        v_out = torch.empty_like(k_out)
+        res = measure_attention(nv, cache, ring, k_out, v_out, reps=max(3, args.steps))
+        if rank == 0:
+            print(json.dumps({"kv_attention": res, "bf16_peak_TFLOP/s": peaks()["bf16_tflops"]}), flush=True)
         return 0
     if args.codecs_only:
         from bit_video_dit_b200 import build as nvbuild

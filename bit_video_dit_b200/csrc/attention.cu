@@ -21,12 +21,13 @@
 // S = Q K^T and O += P V run as tcgen05.mma kind::f16 (binary32 accumulation)
 // in the order PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) per key tile j, so
 // while one query tile's softmax runs the tensor cores work on the other
-// tile's products.  The softmax is one pass with a lazy row maximum: P =
-// exp(scale * (s - m)) against a reference max m that moves only when a tile
-// exceeds it by more than 2^8 (then the row of O in TMEM and the running sum
-// are rescaled by the thread that owns the row), and O / sum is stored as
-// bf16.  Every wait is bounded; a timeout records NVFP4_ERR_TIMEOUT and every
-// role stops.
+// tile's products.  The softmax forms P = exp(scale * (s - m)) in one pass
+// against a reference row maximum m; only a row whose weights in the tile sum
+// above 2^15 (always the first tile) reads the tile's maximum, moves m to it
+// when it exceeds m by more than 2^8 (then the row of O in TMEM and the
+// running sum are rescaled by the thread that owns the row) and forms P
+// again.  O / sum is stored as bf16.  Every wait is bounded; a timeout
+// records NVFP4_ERR_TIMEOUT and every role stops.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>

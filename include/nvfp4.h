@@ -355,10 +355,13 @@ int32_t nvfp4_attention_chunks(int32_t t, int32_t sink_global, int32_t shot_star
  * are bf16 [tq][heads][head_dim] (token-major like the cache's chunks); scale
  * = 0 means 1 / sqrt(head_dim).  head_dim must be 128, and n * ceil(T / 128)
  * < 2^31 (else NVFP4_ERR_UNSUPPORTED).  Products on the tensor cores with
- * binary32 accumulation, a one-pass softmax in binary32 whose reference
- * maximum moves only when a tile exceeds it by more than 2^8 (O rescaled in
- * TMEM then), P rounded to the tiles' 16-bit type; one launch of
- * ceil(tq / 128) x heads CTAs.  An out-of-range slot records NVFP4_ERR_DEVICE
+ * binary32 accumulation, a one-pass softmax in binary32 against a reference
+ * maximum per query row: a row whose weights in a 128-key tile would sum
+ * above 2^15 (always the first tile) takes the tile's largest score, and the
+ * reference moves to it when it exceeds the reference by more than 2^8 (O
+ * rescaled in TMEM then); P rounded to the tiles' 16-bit type.  One launch of
+ * min(ceil(tq / 256) x heads, SMs) persistent CTAs, each taking one head and
+ * two 128-query tiles at a time.  An out-of-range slot records NVFP4_ERR_DEVICE
  * (info = list position) and is skipped.  workspace:
  * nvfp4_workspace_bytes(NVFP4_OP_KV_ATTENTION, 0, 0, 0) bytes; its bytes
  * 16..19 (a uint32 after the error record) count the rescales of O, one per
