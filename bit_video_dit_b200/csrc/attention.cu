@@ -117,21 +117,6 @@ __device__ __forceinline__ uint4 dq8(uint32_t q, uint32_t sc, float a32, const f
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// 8 E2M1 codes times their block scale, exactly, as binary16 (every product
-// e2m1 * s of an E2M1 value and an E4M3 scale is exact in binary16): the
-// operand values of the binary16 path, whose tensor scale a32 is applied to
-// the products instead.
-__device__ __forceinline__ uint4 raw8(uint32_t q, uint32_t sc) {
-    const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-        const __half2 v = __hmul2(e2m1x2_to_half2((q >> (8 * j)) & 0xFFu), s2);
-        o[j] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-    return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
 // One token row (token `tok` of slot s, head h) of K or V as stored: 64 code
 // bytes, 8 scale bytes and the slot's a32; zeros when the token is past the
 // slot's end.  Fetched a tile ahead so the loads overlap the tile in flight.
@@ -168,16 +153,33 @@ template <bool RAW>
 __device__ __forceinline__ void store_row(const AttnArgs& a, int t, int s, int h, const RowRaw& r, uint32_t base,
                                          int row) {
     const float* m = (a.mean[t] && r.valid) ? a.mean[t] + ((int64_t)s * a.heads + h) * kD : nullptr;
-    const uint32_t sw[2] = {r.sc.x, r.sc.y};
+    // the row's eight block scales, two per conversion
+    __half2 sp[4];
+#pragma unroll
+    for (int b2 = 0; b2 < 4; b2++)
+        sp[b2] = e4m3x2_to_half2((uint16_t)(((b2 < 2 ? r.sc.x : r.sc.y) >> (16 * (b2 & 1))) & 0xFFFFu));
 #pragma unroll
     for (int k = 0; k < 4; k++) {
         const uint32_t cw[4] = {r.c[k].x, r.c[k].y, r.c[k].z, r.c[k].w};
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             const int chunk = 4 * k + j;  // elements 8 * chunk .. + 7; block chunk / 2
-            const uint32_t sc = (sw[chunk / 8] >> (8 * ((chunk / 2) % 4))) & 0xFFu;
-            st_shared16(base + chunk * 2048 + row * 16,
-                        RAW ? raw8(cw[j], sc) : dq8(cw[j], sc, r.a32, m ? m + 8 * chunk : nullptr));
+            const int blk = chunk / 2;
+            const __half2 s2 = (blk & 1) ? __high2half2(sp[blk / 2]) : __low2half2(sp[blk / 2]);
+            if (RAW) {
+                // e2m1 * s exactly as binary16 (every product of an E2M1 value and an
+                // E4M3 scale is exact there); a32 is applied to the products instead
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const __half2 v = __hmul2(e2m1x2_to_half2((cw[j] >> (8 * e)) & 0xFFu), s2);
+                    o[e] = *reinterpret_cast<const uint32_t*>(&v);
+                }
+                st_shared16(base + chunk * 2048 + row * 16, make_uint4(o[0], o[1], o[2], o[3]));
+            } else {
+                const uint32_t sc = (((blk < 4 ? r.sc.x : r.sc.y) >> (8 * (blk % 4))) & 0xFFu);
+                st_shared16(base + chunk * 2048 + row * 16, dq8(cw[j], sc, r.a32, m ? m + 8 * chunk : nullptr));
+            }
         }
     }
 }
