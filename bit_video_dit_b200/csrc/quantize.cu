@@ -165,19 +165,25 @@ __device__ __forceinline__ uint2 encode16(const float* f, float inv) {
 
 // Squared error of an encoding of the block, binary32, in element order:
 // sum += (x - fl32(fl32(e2m1 * s) * a32))^2 (the dequant product, exact up to
-// the last multiply).
-__device__ __forceinline__ float block_sq_error(const float* f, uint2 c, float s, float a32) {
+// the last multiply).  e2m1 * s is exact in binary16 (at most 6 significant
+// bits, between 2^-10 and 2688), so it is formed there, two at a time; the
+// multiply by a32, the difference and the square run on binary32 pairs (each
+// lane rounded alone); only the sum is taken one element at a time.
+__device__ __forceinline__ float block_sq_error(const float* f, uint2 c, uint32_t code, float a32) {
     float sum = 0.0f;
+    const __half2 s2 = e4m3x2_to_half2((uint16_t)(code | (code << 8)));
+    const float2 aa = make_float2(a32, a32), m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
     for (int w = 0; w < 2; w++) {
         const uint32_t word = w ? c.y : c.x;
 #pragma unroll
         for (int j = 0; j < 4; j++) {
-            const float2 v = __half22float2(e2m1x2_to_half2((word >> (8 * j)) & 0xFFu));
-            const float d0 = __fmul_rn(__fmul_rn(v.x, s), a32), d1 = __fmul_rn(__fmul_rn(v.y, s), a32);
-            const float e0 = __fsub_rn(f[8 * w + 2 * j], d0), e1 = __fsub_rn(f[8 * w + 2 * j + 1], d1);
-            sum = __fadd_rn(sum, __fmul_rn(e0, e0));
-            sum = __fadd_rn(sum, __fmul_rn(e1, e1));
+            const float2 v = __half22float2(__hmul2(e2m1x2_to_half2((word >> (8 * j)) & 0xFFu), s2));
+            const float2 d = mul2(v, aa);
+            const float2 e = fma2(d, m1, make_float2(f[8 * w + 2 * j], f[8 * w + 2 * j + 1]));
+            const float2 e2 = mul2(e, e);
+            sum = __fadd_rn(sum, e2.x);
+            sum = __fadd_rn(sum, e2.y);
         }
     }
     return sum;
@@ -195,7 +201,7 @@ __device__ __forceinline__ void encode_block(const QuantArgs& a, int t, const Bl
     if (SEARCH) {
         const uint32_t code4 = kc.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(amax_b, kc.d4));
         const uint2 c4 = encode16(f, kc.inv_tab[code4]);
-        if (block_sq_error(f, c4, e4m3_value(code4), kc.a32) < block_sq_error(f, c, e4m3_value(code), kc.a32)) {
+        if (block_sq_error(f, c4, code4, kc.a32) < block_sq_error(f, c, code, kc.a32)) {
             code = code4;
             c = c4;
         }
@@ -796,8 +802,7 @@ __global__ void __launch_bounds__(kQThreads, 1) ln_quantize_smem_kernel(const __
                 if (SEARCH) {
                     const uint32_t code4 = kc.d4 == 0.0f ? 0u : e4m3_code(__fdiv_rn(mx, kc.d4));
                     const uint2 c4 = encode16(f, kc.inv_tab[code4]);
-                    if (block_sq_error(f, c4, e4m3_value(code4), kc.a32) <
-                        block_sq_error(f, cw, e4m3_value(code), kc.a32)) {
+                    if (block_sq_error(f, c4, code4, kc.a32) < block_sq_error(f, cw, code, kc.a32)) {
                         code = code4;
                         cw = c4;
                     }
