@@ -353,8 +353,8 @@ int32_t nvfp4_attention_chunks(int32_t t, int32_t sink_global, int32_t shot_star
  * the slot's a32 applied to the products); with K- or V-smoothing they are the
  * cache's bf16 dequant with the means added (bf16 tiles).  q_bf16 and o_bf16
  * are bf16 [tq][heads][head_dim] (token-major like the cache's chunks); scale
- * = 0 means 1 / sqrt(head_dim).  head_dim must be 128, and n * ceil(T / 128)
- * < 2^31 (else NVFP4_ERR_UNSUPPORTED).  Products on the tensor cores with
+ * = 0 means 1 / sqrt(head_dim).  head_dim must be 128, n * ceil(T / 128) < 2^31
+ * and ceil(tq / 256) * heads < 2^31 (else NVFP4_ERR_UNSUPPORTED).  Products on the tensor cores with
  * binary32 accumulation, a one-pass softmax in binary32 against a reference
  * maximum per query row: a row whose weights in a 128-key tile would sum
  * above 2^15 (always the first tile) takes the tile's largest score, and the
@@ -362,7 +362,8 @@ int32_t nvfp4_attention_chunks(int32_t t, int32_t sink_global, int32_t shot_star
  * rescaled in TMEM then); P rounded to the tiles' 16-bit type.  One launch of
  * min(ceil(tq / 256) x heads, SMs) persistent CTAs, each taking one head and
  * two 128-query tiles at a time.  An out-of-range slot records NVFP4_ERR_DEVICE
- * (info = list position) and is skipped.  workspace:
+ * (info = list position) and is skipped; a wait that runs out records
+ * NVFP4_ERR_TIMEOUT (info = which wait) and leaves O incomplete.  workspace:
  * nvfp4_workspace_bytes(NVFP4_OP_KV_ATTENTION, 0, 0, 0) bytes; its bytes
  * 16..19 (a uint32 after the error record) count the rescales of O, one per
  * warp and key tile in which a row's reference maximum moved after the first
