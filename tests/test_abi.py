@@ -131,6 +131,10 @@ def test_host_side_argument_checks(L):
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 1, 1 << 18, 1, 128)  # 2048 tiles per slot
     st = L.nvfp4_kv_attention(ctypes.byref(kv), fake, 1 << 20, fake, 128, ctypes.c_float(0.0), fake, fake, 256, None)
     assert st == nv.ERR_UNSUPPORTED
+    # and its work units (pairs of 128-query tiles x heads): 2^12 pairs x 2^20 heads = 2^32
+    kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 1, 128, 1 << 20, 128)
+    st = L.nvfp4_kv_attention(ctypes.byref(kv), fake, 1, fake, 1 << 20, ctypes.c_float(0.0), fake, fake, 256, None)
+    assert st == nv.ERR_UNSUPPORTED
     # the keys' RoPE tables: present, 16-byte aligned, and 32-bit flat indexes
     kv = nv.CKVCache(fake, fake, fake, fake, fake, fake, 4, 8, 2, 32)
     rope = L.nvfp4_kv_append_rope
